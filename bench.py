@@ -1,0 +1,372 @@
+"""Benchmark of the quantized MoE FFN hot path on B200.
+
+Default workload: 48-layer decode, one token per step (d=2560, 512 experts,
+top-10 + 1 shared, SwiGLU intermediate 512, Q4B32 weights, seeded synthetic
+inputs).  A step = one token through all 48 layers (router, top-k, dispatch,
+expert SwiGLU, down projection, combine, residual + rmsnorm), weights and
+inputs resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (under torchrun): independent replicas, one per GPU, each decoding its
+own tokens (the layer does not shard for one token stream); value = tokens
+of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "48-layer MoE decode tok/s & prefill tok/s; % of HBM / MMA roofline"
+DEFAULT_WORKLOAD = "decode_48l_q4_t1"
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def expert_bytes(cfg) -> int:
+    """Packed bytes of one expert (gate + up + down, codes + fp16 scales)."""
+    per_block = cfg.block_bytes + 2
+    return 3 * cfg.d * cfg.I // 32 * per_block
+
+
+def router_bytes(cfg) -> int:
+    return cfg.E * cfg.d * 4
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            p = [v.strip() for v in line.split(",")]
+            if len(p) >= 9:
+                try:
+                    rows.append((float(p[1]), float(p[2]), p[5:9]))
+                except ValueError:
+                    pass
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the baseline, and the --impl reference arm)
+# ---------------------------------------------------------------------------
+def oracle_decode_sample(cfg, n_layers: int, token_stream: int) -> float:
+    """Seconds the oracle takes to push one token through `n_layers` layers
+    (expert generation on the host is excluded from the timing)."""
+    import oracle
+    from tests.parity import ExpertSource
+    x = synth.tokens_bf16(cfg, 1, stream=token_stream)[0]
+    total = 0.0
+    for l in range(n_layers):
+        src = ExpertSource(cfg, l)
+        xf = oracle.bf16_to_f64(x)
+        ids, _, _ = oracle.route(oracle.router_logits(xf, src.router_w, src.router_b), cfg.k)
+        for e in ids:
+            src.expert(int(e))          # generate outside the timed region
+        src.shared(0)
+        t0 = time.perf_counter()
+        y, _, _, _ = oracle.moe_token(cfg.fmt, cfg.k, x, src.router_w, src.router_b, src.expert,
+                                      src.shared, cfg.n_shared)
+        r = oracle.rmsnorm(xf + y)
+        total += time.perf_counter() - t0
+        x = oracle.round_bf16(r)
+    return total
+
+
+def run_reference(args, cfg) -> dict:
+    layers = args.ref_layers
+    times = []
+    for s in range(args.warmup + args.steps):
+        dt = oracle_decode_sample(cfg, layers, token_stream=1000 + s)
+        if s >= args.warmup:
+            times.append(dt)
+    per_token = statistics.mean(times) * cfg.L / layers
+    value = cfg.T / per_token
+    sample = f"{cfg.T} token(s) through {layers} of {cfg.L} layers per step, time scaled x{cfg.L / layers:g}"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": cfg.name},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def timed_stack(sess, cfg, xs, r_out, steps, warmup, stream, dist_on):
+    from quantized_expert_ffn_token_b200 import capi
+    T = cfg.T
+    for s in range(warmup):
+        capi.moe_forward_stack(sess.ctx, 0, cfg.L, xs[s % len(xs)], T, r_out, None, stream)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    capi.moe_timing_read(sess.ctx)                     # reset counters
+    capi.moe_timing_enable(sess.ctx, True)
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(steps):
+        capi.moe_forward_stack(sess.ctx, 0, cfg.L, xs[(warmup + s) % len(xs)], T, r_out, None, stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    tim = capi.moe_timing_read(sess.ctx)
+    capi.moe_timing_enable(sess.ctx, False)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop), tim
+
+
+def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
+    from quantized_expert_ffn_token_b200 import capi, session
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(dev)
+    P = peaks()
+    sess = session.Session(cfg, device=local_rank, max_tokens=cfg.T)
+    with torch.cuda.stream(stream):
+        sess.load_synthetic(stream=stream)
+    torch.cuda.synchronize()
+    n_tok = args.warmup + args.steps
+    xs = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).to(dev)
+          for s in range(n_tok)]
+    r_out = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=dev)
+
+    with Clocks(local_rank) as clk:
+        ms, tim = timed_stack(sess, cfg, xs, r_out, args.steps, args.warmup, stream, dist_on)
+    clocks = clk.summary()
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist_on:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    ms_step = ms_max / args.steps
+    value = cfg.T * world / (ms_step / 1e3)
+
+    # roofline of the dominant (timed) kernel: expert weight bytes it streams
+    # per launch (one launch per layer; T=1 -> k routed + shared experts)
+    union = cfg.k if cfg.T == 1 else None
+    if union is None:
+        union = measured_union(sess, cfg, xs[0], dev)
+    alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)
+    avg_ms = tim["ms"] / max(1, tim["timed_launches"])
+    achieved = alg_bytes / (avg_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / P["hbm_gbs"], "traffic": None, "kernel": tim["kernel"],
+            "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_ms,
+            "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
+    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+
+    # end to end through the public host-buffer entry point
+    x_host = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).pin_memory()
+              for s in range(n_tok)]
+    r_host = torch.empty((cfg.T, cfg.d), dtype=torch.float32).pin_memory()
+    for s in range(args.warmup):
+        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[s], cfg.T, r_host, stream)
+    if dist_on:
+        torch.distributed.barrier()
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[args.warmup + s], cfg.T, r_host, stream)
+    e2e_s = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=dev)
+    if dist_on:
+        torch.distributed.all_reduce(e2e_s, op=torch.distributed.ReduceOp.MAX)
+    e2e = {"value": cfg.T * world * args.steps / float(e2e_s.item()), "unit": "tok/s",
+           "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
+           "timer": "host wall clock around synchronous calls"}
+    sess.close()
+    del xs
+    torch.cuda.empty_cache()
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32-accumulate over Q4B32/bf16" if cfg.fmt == "q4" else "fp32-accumulate over Q3B32/bf16",
+        "data": "synthetic (seeded counter-hash weights, N(0,1) bf16 tokens)",
+        "config": {"workload": f"{cfg.name}: d={cfg.d} E={cfg.E} top-{cfg.k}+{cfg.n_shared} shared "
+                               f"I={cfg.I} {cfg.fmt.upper()}B32 T={cfg.T} layers={cfg.L}",
+                   "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: each step streams {step_bytes / 1e9:.2f} GB of weights (> 126 MB L2) "
+                         "and routes a new token"},
+        "roofline": roof,
+        "step_roofline": {"alg_bytes_per_step": step_bytes,
+                          "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                          "frac": step_bytes / (ms_step / 1e3) / 1e9 / P["hbm_gbs"]},
+        "e2e": e2e,
+        "gpu_launches": tim["all_launches"],
+        "clocks": clocks,
+    }
+    return out
+
+
+def measured_union(sess, cfg, x, dev) -> int:
+    """Mean number of distinct routed experts per layer for one step (T > 1)."""
+    from quantized_expert_ffn_token_b200 import capi
+    L, T, k = cfg.L, cfg.T, cfg.k
+    idr = torch.empty((L, T, k), dtype=torch.int32, device=dev)
+    rec = capi.make_record(ids=idr)
+    r = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+    capi.moe_forward_stack(sess.ctx, 0, L, x, T, r, rec)
+    torch.cuda.synchronize()
+    ids = idr.cpu().numpy()
+    return int(round(np.mean([len(np.unique(ids[l])) for l in range(L)])))
+
+
+def secondary_prefill(args, local_rank) -> dict:
+    """Single-layer prefill (4096 tokens, Zipf-biased routing): tok/s and the
+    expert kernels' throughput against the dense tensor peak."""
+    from quantized_expert_ffn_token_b200 import capi, session
+    cfg = synth.CONFIGS["prefill_1l_q4_t4096_zipf"]
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(dev)
+    sess = session.Session(cfg, device=local_rank, max_tokens=cfg.T)
+    sess.load_synthetic(stream=stream)
+    x = torch.from_numpy(synth.tokens_bf16(cfg).view(np.int16)).to(dev)
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.int16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        capi.moe_forward(sess.ctx, 0, x, cfg.T, y, None, None, None, stream)
+    torch.cuda.synchronize()
+    times = []
+    capi.moe_timing_read(sess.ctx)
+    capi.moe_timing_enable(sess.ctx, True)
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        capi.moe_forward(sess.ctx, 0, x, cfg.T, y, None, None, None, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    tim = capi.moe_timing_read(sess.ctx)
+    sess.close()
+    ms = statistics.median(times)
+    flops_expert = 2 * cfg.T * (cfg.k + cfg.n_shared) * 3 * cfg.d * cfg.I
+    flops = flops_expert + 2 * cfg.T * cfg.E * cfg.d
+    P = peaks()
+    kms = tim["ms"] / max(1, tim["timed_launches"])
+    return {"workload": cfg.name, "tok_per_s": cfg.T / (ms / 1e3), "ms_per_layer": ms,
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": tim["kernel"],
+                         "achieved": flops_expert / (kms / 1e3) / 1e12,
+                         "peak": P["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": flops_expert / (kms / 1e3) / 1e12 / P["bf16_tflops_sustained"]},
+            "l2": "256 MB flush between timed calls"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-layers", type=int, default=12, help="oracle sample: layers per token")
+    ap.add_argument("--ref-layers", type=int, default=2, help="reference arm: layers per step")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    cfg = synth.CONFIGS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)))
+        return 0
+
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, cfg, rank, world, local_rank, dist_on)
+    if rank == 0:
+        if not args.no_secondary and world == 1:
+            out["secondary"] = {"prefill": secondary_prefill(args, local_rank)}
+        if world == 1:
+            sec = oracle_decode_sample(cfg, args.cpu_layers, token_stream=7)
+            v = cfg.T / (sec * cfg.L / args.cpu_layers)
+            out["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"{cfg.T} token(s) through {args.cpu_layers} of {cfg.L} "
+                                             f"layers, time scaled x{cfg.L / args.cpu_layers:g}"}
+        print(json.dumps(out))
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

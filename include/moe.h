@@ -1,0 +1,181 @@
+/*
+ * moe.h - quantized sparse Mixture-of-Experts feed-forward layer on one
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes, no C++ or torch
+ * types.  Every entry point returns a moe_status; nothing aborts or throws.
+ *
+ * The layer (per token t, per layer):
+ *   router   logit_e = x_t . W_r[e] (+ b_e)                 e = 0..E-1
+ *   route    p = softmax(logits); ids = the top_k experts by p (descending,
+ *            equal p -> lower id); w_j = p_ids[j] / sum_j p_ids[j]
+ *   experts  for each chosen expert and each shared expert:
+ *            g = W_g x_t, u = W_u x_t, h = silu(g) * u, y_e = W_d h
+ *   combine  y_t = bf16( sum_j w_j y_ids[j]  +  sum_s y_shared_s )
+ * Source passages: "Qwen3.8-Flash-Next at 45 Tokens/sec on a 12GB GPU?"
+ * (video transcript 1:37-2:16: 48 layers x 512 experts, a router per layer
+ * picks 10 of them plus one always-on shared expert; 3:36-3:47: the partial
+ * results of one token land on one output) and "Qwen3.8-Flash-Next on RTX
+ * 5090 + 64GB", section "The 30-Second Overview" (10 routed + 1 shared per
+ * token).  The pages do not define the expert network, the routing
+ * normalisation or the quantised layouts; this library fixes them: SwiGLU
+ * experts, softmax renormalised over the chosen k, and the two block formats
+ * below.
+ *
+ * Block formats (32 weights per block, blocks run along the reduction dim):
+ *   MOE_Q4B32  16 bytes of int4 codes, two per byte (byte b: code 2b in the
+ *              low nibble, code 2b+1 in the high nibble) + one fp16 scale s;
+ *              w = s * (q - 8).                                   4.5 bit/w
+ *   MOE_Q3B32  12 bytes: the 32 three-bit codes of one 96-bit little-endian
+ *              integer (code j in bits 3j..3j+2) + one fp16 scale s;
+ *              w = s * (q - 4).                                   3.5 bit/w
+ *
+ * Canonical tensor layouts accepted by moe_load_layer (row-major, SoA: codes
+ * and scales in separate arrays):
+ *   gate, up   codes  [E][d_ff][d_model/32][B]   scales [E][d_ff][d_model/32]
+ *   down       codes  [E][d_model][d_ff/32][B]   scales [E][d_model][d_ff/32]
+ *   B = 16 (Q4B32) or 12 (Q3B32); scales are IEEE fp16 bit patterns.
+ *   router_w   fp32 [E][d_model]; router_bias fp32 [E] or NULL.
+ *   Shared experts: the same with n_shared in place of E and d_ff_shared.
+ * The library copies them into its own device memory in a private tiled
+ * order (same byte count); the caller's buffers are not referenced after
+ * moe_load_layer returns.
+ */
+#ifndef QEFFN_MOE_H
+#define QEFFN_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,     /* NULL pointer, bad size, bad layer index */
+    MOE_ERR_OOM = -2,             /* device allocation failed or over the memory limit */
+    MOE_ERR_CUDA = -3,            /* a CUDA runtime call failed; see moe_last_error() */
+    MOE_ERR_NOT_LOADED = -4,      /* moe_forward on a layer never loaded */
+    MOE_ERR_TOO_MANY_TOKENS = -5, /* T > max_tokens */
+    MOE_ERR_DEVICE_TIMEOUT = -6,  /* a bounded device-side wait ran out */
+    MOE_ERR_UNSUPPORTED = -7      /* a shape this build does not implement */
+} moe_status;
+
+typedef enum { MOE_Q4B32 = 1, MOE_Q3B32 = 2 } moe_qformat;
+
+typedef struct {
+    int d_model;        /* hidden size d; multiple of 256 */
+    int n_experts;      /* routed experts E, 1..1024 */
+    int d_ff;           /* routed expert intermediate size I; multiple of 64 */
+    int top_k;          /* experts chosen per token, 1..min(E, 32) */
+    int n_shared;       /* always-on shared experts, 0..4 */
+    int d_ff_shared;    /* shared expert intermediate size; must equal d_ff */
+    int n_layers;       /* layers the context can hold */
+    int max_tokens;     /* largest T any call may pass */
+    int fmt;            /* moe_qformat */
+    long long device_mem_limit; /* bytes the context may allocate; 0 = no limit */
+} moe_config;
+
+typedef struct {
+    const float *router_w;          /* [E][d] */
+    const float *router_bias;       /* [E] or NULL (no bias) */
+    const uint8_t *codes[3];        /* gate, up, down (canonical layouts above) */
+    const uint16_t *scales[3];
+    const uint8_t *sh_codes[3];     /* shared experts; ignored when n_shared == 0 */
+    const uint16_t *sh_scales[3];
+    int on_device;                  /* 1: all pointers are device memory of the
+                                       context's device; 0: host memory */
+} moe_layer_weights;
+
+/* Per-layer records written by moe_forward_stack; any field may be NULL.
+ * Only the token rows listed in rows[0..n_rows) are recorded (rows == NULL:
+ * all T rows, in order).  Record r of layer l sits at [l][r][...]. */
+typedef struct {
+    uint16_t *x_bf16;   /* [n_layers][n_rec][d] bf16 input of each layer */
+    uint16_t *y_bf16;   /* [n_layers][n_rec][d] bf16 output of each layer */
+    float *y_f32;       /* [n_layers][n_rec][d] fp32 value that y_bf16 rounds */
+    int32_t *ids;       /* [n_layers][n_rec][k] */
+    float *w;           /* [n_layers][n_rec][k] */
+    const int32_t *rows;/* device array of token indices, or NULL */
+    int n_rows;         /* length of rows (ignored when rows == NULL) */
+} moe_stack_record;
+
+typedef struct moe_ctx moe_ctx;
+
+/* Create a context on CUDA device `device` and allocate its workspace (sized
+ * by max_tokens).  *out receives the handle.  Errors: INVALID_ARG (bad
+ * config), UNSUPPORTED (shape outside the limits above), OOM, CUDA. */
+MOE_API int moe_create(const moe_config *cfg, int device, moe_ctx **out);
+
+/* Copy one layer's weights into the context (repacking them on the device)
+ * and make the layer usable.  Reloading a layer replaces it.  Work is queued
+ * on `stream` (a cudaStream_t, NULL = default stream); the call returns after
+ * the copies from caller memory have completed.  Errors: INVALID_ARG, OOM,
+ * CUDA. */
+MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, void *stream);
+
+/* One layer on T tokens.  All pointers are device memory:
+ *   x_bf16 [T][d] input; y_bf16 [T][d] output; y_f32 [T][d] the fp32 value
+ *   before the bf16 rounding, or NULL; ids [T][k] chosen experts (descending
+ *   weight) and w [T][k] their weights, either may be NULL.
+ * Asynchronous on `stream`; no host synchronisation and no allocation.
+ * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA. */
+MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
+                uint16_t *y_bf16, float *y_f32, int32_t *ids, float *w,
+                void *stream);
+
+/* Layers [layer0, layer0 + n_layers) stacked with a residual stream:
+ *   r_0 = x (bf16 input, widened to fp32)
+ *   x_l = bf16(rmsnorm(r_l)),  rmsnorm(r) = r / sqrt(mean(r^2) + 1e-6)
+ *   r_{l+1} = r_l + float(moe_l(x_l))
+ * and resid_out [T][d] fp32 = r_{layer0+n_layers}.  The pages only say the
+ * layers are stacked; the normalisation without learned weight is this
+ * library's reading.  x_bf16 and resid_out are device pointers; rec may be
+ * NULL.  Asynchronous on `stream`, no allocation.  Errors as moe_forward. */
+MOE_API int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint16_t *x_bf16,
+                      int T, float *resid_out, const moe_stack_record *rec,
+                      void *stream);
+
+/* moe_forward_stack with HOST buffers: copies x_bf16 (host, pinned or
+ * pageable) to the device, runs the stack and copies resid_out back to the
+ * host; returns after the result is in host memory. */
+MOE_API int moe_forward_stack_host(moe_ctx *ctx, int layer0, int n_layers,
+                           const uint16_t *x_bf16_host, int T, float *resid_out_host,
+                           void *stream);
+
+/* Free every device allocation of the context.  NULL is accepted.  A handle
+ * must not be used after this call. */
+MOE_API int moe_destroy(moe_ctx *ctx);
+
+/* Read (and clear) the device error word that bounded device waits and
+ * in-kernel checks set.  *code receives 0 or a MOE_ERR_* value.  Synchronises
+ * the context's device. */
+MOE_API int moe_get_device_error(moe_ctx *ctx, int *code);
+
+/* Measurement hook.  While enabled, each forward records a CUDA event pair on
+ * the caller's stream around its dominant kernel (the kernel that streams the
+ * expert weights).  moe_timing_read synchronises the device and returns, since
+ * the previous read: the summed duration of the timed launches (ms), their
+ * number, every kernel launch the library issued (timed or not), and the
+ * name of the timed kernel (copied into name[0..name_len), NUL-terminated).
+ * At most 65536 launches are timed between reads; later ones are counted but
+ * not timed. */
+MOE_API int moe_timing_enable(moe_ctx *ctx, int on);
+MOE_API int moe_timing_read(moe_ctx *ctx, double *total_ms, long long *timed_launches,
+                            long long *all_launches, char *name, int name_len);
+
+/* Static text for a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* Text of the most recent MOE_ERR_CUDA / MOE_ERR_OOM on this host thread. */
+MOE_API const char *moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QEFFN_MOE_H */

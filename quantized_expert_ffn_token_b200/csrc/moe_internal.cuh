@@ -1,0 +1,215 @@
+// Internal declarations of the MoE FFN library: context, private weight
+// layout, launch helpers.  Nothing here is part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <utility>
+#include <vector>
+
+#include "moe.h"
+
+namespace qeffn {
+
+// ---------------------------------------------------------------------------
+// Private tiled weight layout ("row tiles").
+//
+// Every expert matrix is stored as tiles of 16 rows x K.  A gate/up tile t
+// holds gate rows 8t..8t+7 (tile rows 0..7) and up rows 8t..8t+7 (tile rows
+// 8..15), so one tile yields 8 SwiGLU outputs.  A down tile t holds output rows
+// 16t..16t+15.  Inside a tile the codes are grouped by 64-wide k groups; in a
+// k group, the 32 lanes of a warp each own one contiguous piece holding the
+// codes of the mma.m16n8k16 A fragments that lane needs for the group's four
+// 16-wide k slices:
+//   lane = 4*g + c  (g = row % 8, c = (k % 8) / 2)
+//   register a0: row g,   k = 16s + 2c + {0,1}     a1: row g+8, same k
+//   register a2: row g,   k = 16s + 2c + 8 + {0,1} a3: row g+8, same k
+// Q4B32: 16 bytes per lane and group = 4 words, word m = slice m, nibble n of
+//   the word (bits 4n..4n+3): n = reg + 4*hi  (hi = odd k of the pair).
+// Q3B32: 12 bytes per lane and group = 3 words.  Register q = 4*m + reg
+//   (0..15); for q < 15 its two codes are the 3-bit fields of word q/5 at bits
+//   3f (even k) and 16+3f (odd k), f = q%5; register 15's codes are spread
+//   over bit 15 (even k) and bit 31 (odd k) of words 0,1,2 (code bit b in
+//   word b).
+// After the codes: the tile's fp16 scales, [16 rows][K/32 blocks].
+// The byte count equals the canonical layout's.
+// ---------------------------------------------------------------------------
+struct MatLayout {
+    int K;           // reduction length (multiple of 64)
+    int n_tiles;     // 16-row tiles per expert
+    int kg_bytes;    // bytes per k group (all lanes): 512 (Q4) / 384 (Q3)
+    int code_bytes;  // (K/64) * kg_bytes
+    int tile_bytes;  // code_bytes + 16 * (K/32) * 2
+    size_t expert_bytes;
+};
+
+inline MatLayout make_layout(int fmt, int rows, int K) {
+    MatLayout L;
+    L.K = K;
+    L.n_tiles = rows / 16;
+    L.kg_bytes = (fmt == MOE_Q4B32) ? 512 : 384;
+    L.code_bytes = (K / 64) * L.kg_bytes;
+    L.tile_bytes = L.code_bytes + 16 * (K / 32) * 2;
+    L.expert_bytes = (size_t)L.n_tiles * L.tile_bytes;
+    return L;
+}
+
+// Byte offset (within a tile's code area) and bit offset of the code of
+// tile row r (0..15), column k, Q4B32.
+__host__ __device__ inline void q4_code_pos(int r, int k, int *byte, int *shift) {
+    int g = r & 7, half = r >> 3;
+    int s = k >> 4, kk = k & 15;
+    int kg = s >> 2, m = s & 3;
+    int c = (kk & 7) >> 1, hi = kk & 1, second = kk >> 3;
+    int reg = second * 2 + half;
+    int n = reg + 4 * hi;
+    *byte = kg * 512 + (g * 4 + c) * 16 + m * 4 + (n >> 1);
+    *shift = (n & 1) * 4;
+}
+
+// Q3B32: the three (byte, bit) positions of the code bits b = 0,1,2.
+__host__ __device__ inline void q3_code_pos(int r, int k, int byte[3], int bit[3]) {
+    int g = r & 7, half = r >> 3;
+    int s = k >> 4, kk = k & 15;
+    int kg = s >> 2, m = s & 3;
+    int c = (kk & 7) >> 1, hi = kk & 1, second = kk >> 3;
+    int reg = second * 2 + half;
+    int q = 4 * m + reg;
+    int base = kg * 384 + (g * 4 + c) * 12;
+    for (int b = 0; b < 3; ++b) {
+        int word, wbit;
+        if (q < 15) {
+            word = q / 5;
+            wbit = 3 * (q % 5) + 16 * hi + b;
+        } else {
+            word = b;
+            wbit = 15 + 16 * hi;
+        }
+        byte[b] = base + word * 4 + (wbit >> 3);
+        bit[b] = wbit & 7;
+    }
+}
+
+__device__ inline int tile_code(int fmt, const uint8_t *tile, int r, int k) {
+    if (fmt == MOE_Q4B32) {
+        int byte, sh;
+        q4_code_pos(r, k, &byte, &sh);
+        return (tile[byte] >> sh) & 15;
+    }
+    int byte[3], bit[3];
+    q3_code_pos(r, k, byte, bit);
+    int v = 0;
+    for (int b = 0; b < 3; ++b) v |= ((tile[byte[b]] >> bit[b]) & 1) << b;
+    return v;
+}
+
+__device__ inline float tile_scale(const uint8_t *tile, const MatLayout &L, int r, int blk) {
+    const __half *s = reinterpret_cast<const __half *>(tile + L.code_bytes);
+    return __half2float(s[r * (L.K / 32) + blk]);
+}
+
+// ---------------------------------------------------------------------------
+// Context
+// ---------------------------------------------------------------------------
+struct Layer {
+    bool loaded = false;
+    float *router_w = nullptr;   // [E][d]
+    float *router_b = nullptr;   // [E] (zeros when the layer has no bias)
+    uint8_t *gu = nullptr;       // [(E + n_shared)] x gu.expert_bytes
+    uint8_t *dn = nullptr;       // [(E + n_shared)] x dn.expert_bytes
+};
+
+struct Workspace {
+    float *logits = nullptr;     // [T][E]
+    int32_t *ids = nullptr;      // [T][k]
+    float *w = nullptr;          // [T][k]
+    int32_t *counts = nullptr;   // [E + n_sh]
+    int32_t *offsets = nullptr;  // [E + n_sh + 1]
+    int32_t *fill = nullptr;     // [E + n_sh]
+    int32_t *perm = nullptr;     // [S] slot at each grouped position
+    int32_t *inv = nullptr;      // [S] grouped position of each slot
+    int4 *chunks = nullptr;      // [max_chunks] (expert, start, n, 0)
+    int32_t *n_chunks = nullptr; // [1]
+    float *h = nullptr;          // [S][I] SwiGLU outputs by grouped position
+    float *yslot = nullptr;      // [S][d] expert outputs by grouped position
+    float *resid = nullptr;      // [T][d] residual stream of the stack
+    uint16_t *xs = nullptr;      // [T][d] bf16 layer input of the stack
+    uint16_t *ys = nullptr;      // [T][d] bf16 layer output of the stack
+    float *yf = nullptr;         // [T][d] fp32 layer output of the stack
+    uint16_t *x_io = nullptr;    // [T][d] staging for host I/O
+    float *r_io = nullptr;       // [T][d] staging for host I/O
+    int *dev_error = nullptr;    // [1]
+    int max_chunks = 0;
+};
+
+// Event pairs around the dominant kernel (moe_timing_enable).
+struct Timing {
+    bool on = false;
+    std::vector<cudaEvent_t> ev;   // 2 * capacity events
+    int used = 0;
+    long long dropped = 0;
+    long long launches_at_read = 0;
+    const char *name = "";
+};
+
+}  // namespace qeffn
+
+struct moe_ctx {
+    moe_config cfg;
+    int device;
+    int nx;                       // E + n_shared (experts stored per layer)
+    qeffn::MatLayout gu, dn;
+    std::vector<qeffn::Layer> layers;
+    qeffn::Workspace ws;
+    size_t allocated = 0;
+    std::vector<std::pair<void *, size_t>> allocs;
+    qeffn::Timing timing;
+};
+
+namespace qeffn {
+
+// Status plumbing (moe_api.cu)
+int set_cuda_error(cudaError_t e, const char *what);
+int set_oom(const char *what);
+int ctx_alloc(moe_ctx *ctx, void **p, size_t bytes, const char *what);
+void ctx_free(moe_ctx *ctx, void *p);
+
+#define QE_CHECK(call)                                                   \
+    do {                                                                 \
+        cudaError_t _e = (call);                                         \
+        if (_e != cudaSuccess) return qeffn::set_cuda_error(_e, #call);  \
+    } while (0)
+
+extern long long g_launches;   // every kernel launch the library issued
+
+#define QE_CHECK_LAUNCH(what)                                            \
+    do {                                                                 \
+        __atomic_add_fetch(&qeffn::g_launches, 1, __ATOMIC_RELAXED);     \
+        cudaError_t _e = cudaGetLastError();                             \
+        if (_e != cudaSuccess) return qeffn::set_cuda_error(_e, what);   \
+    } while (0)
+
+int timing_begin(moe_ctx *ctx, cudaStream_t st, const char *name);
+int timing_end(moe_ctx *ctx, cudaStream_t st);
+
+// Kernels' host launchers (each returns a moe_status)
+int launch_repack(moe_ctx *ctx, int fmt, const uint8_t *codes, const uint16_t *scales,
+                  const uint8_t *codes_up, const uint16_t *scales_up, int n_experts,
+                  int rows, int K, bool gate_up, uint8_t *dst, cudaStream_t st);
+int launch_router_simt(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
+                       float *logits, cudaStream_t st);
+int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, float *w,
+                cudaStream_t st);
+int launch_dispatch(moe_ctx *ctx, const int32_t *ids, int T, cudaStream_t st);
+int launch_experts_simt(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
+                        cudaStream_t st);
+int launch_combine(const moe_ctx *ctx, int T, const float *w, uint16_t *y, float *yf,
+                   cudaStream_t st);
+int launch_resid_norm(const moe_ctx *ctx, int T, float *resid, const uint16_t *y_add,
+                      const uint16_t *x_in, uint16_t *x_out, cudaStream_t st);
+int launch_record(const moe_ctx *ctx, int T, int layer_idx, const moe_stack_record *rec,
+                  const uint16_t *x, const uint16_t *y, const float *yf, const int32_t *ids,
+                  const float *w, cudaStream_t st);
+
+}  // namespace qeffn

@@ -1,0 +1,236 @@
+// Router logits, softmax top-k and the token -> expert dispatch
+// (count, exclusive scan, scatter).
+//
+// Routing rule: for every token a router picks top_k of the E experts and the
+// shared expert(s) always run ("Qwen3.8-Flash-Next at 45 Tokens/sec on a 12GB
+// GPU?", video transcript 1:50-2:16).  Weights are the softmax over all E
+// logits renormalised over the chosen k, which equals the softmax over the
+// chosen logits; the chosen ids are ordered by weight, equal logits -> lower id.
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace qeffn {
+
+namespace {
+
+constexpr int RT_TOK = 8;   // tokens per router block
+constexpr int RT_EXP = 8;   // experts per router block (one per warp)
+
+// logits[t][e] = sum_i x[t][i] * W[e][i] + b[e], fp32 FMA accumulation.
+__global__ void __launch_bounds__(256) k_router_simt(const uint16_t *__restrict__ x, int T, int d,
+                                                     int E, const float *__restrict__ W,
+                                                     const float *__restrict__ b,
+                                                     float *__restrict__ logits) {
+    extern __shared__ float xs[];   // [RT_TOK][d]
+    int t0 = blockIdx.y * RT_TOK;
+    int nt = min(RT_TOK, T - t0);
+    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
+        int tt = i / d, c = i % d;
+        uint32_t bits = (uint32_t)x[(size_t)(t0 + tt) * d + c] << 16;
+        xs[tt * d + c] = __uint_as_float(bits);
+    }
+    __syncthreads();
+    int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int e = blockIdx.x * RT_EXP + warp;
+    if (e >= E) return;
+    float acc[RT_TOK];
+#pragma unroll
+    for (int tt = 0; tt < RT_TOK; ++tt) acc[tt] = 0.f;
+    const float4 *Wr = reinterpret_cast<const float4 *>(W + (size_t)e * d);
+    for (int i4 = lane; i4 < d / 4; i4 += 32) {
+        float4 wv = Wr[i4];
+#pragma unroll
+        for (int tt = 0; tt < RT_TOK; ++tt) {
+            if (tt < nt) {
+                const float *xv = xs + tt * d + 4 * i4;
+                acc[tt] = fmaf(wv.x, xv[0], acc[tt]);
+                acc[tt] = fmaf(wv.y, xv[1], acc[tt]);
+                acc[tt] = fmaf(wv.z, xv[2], acc[tt]);
+                acc[tt] = fmaf(wv.w, xv[3], acc[tt]);
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < RT_TOK; ++tt) {
+        float v = acc[tt];
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && tt < nt) logits[(size_t)(t0 + tt) * E + e] = v + b[e];
+    }
+}
+
+// Larger (v, id) first: larger logit, equal logits -> lower id.
+__device__ inline bool better(float v, int id, float bv, int bid) {
+    return v > bv || (v == bv && id < bid);
+}
+
+// One warp per token: k rounds of warp arg-max over the token's E logits,
+// then the softmax over the chosen logits.
+__global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, int T, int E, int k,
+                                              int32_t *__restrict__ ids, float *__restrict__ w) {
+    extern __shared__ float lg[];   // [8][E]
+    int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    float *my = lg + warp * E;
+    for (int e = lane; e < E; e += 32) my[e] = logits[(size_t)t * E + e];
+    __syncwarp();
+    float chosen_v = -INFINITY;
+    int chosen_id = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bid = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            float v = my[e];
+            if (better(v, e, bv, bid)) {
+                bv = v;
+                bid = e;
+            }
+        }
+        for (int o = 16; o; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (lane == j) {
+            chosen_v = bv;
+            chosen_id = bid;
+        }
+        __syncwarp();
+        if (lane == 0) my[bid] = -INFINITY;
+        __syncwarp();
+    }
+    float top = __shfl_sync(0xffffffffu, chosen_v, 0);
+    float p = (lane < k) ? expf(chosen_v - top) : 0.f;
+    float z = p;
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < k) {
+        ids[(size_t)t * k + lane] = chosen_id;
+        w[(size_t)t * k + lane] = p / z;
+    }
+}
+
+__device__ inline int slot_expert(const int32_t *ids, int slot, int T, int k, int E) {
+    int routed = T * k;
+    return slot < routed ? ids[slot] : E + (slot - routed) / T;
+}
+
+__global__ void k_count(const int32_t *__restrict__ ids, int T, int k, int E, int S,
+                        int32_t *__restrict__ counts) {
+    for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < S; s += gridDim.x * blockDim.x)
+        atomicAdd(&counts[slot_expert(ids, s, T, k, E)], 1);
+}
+
+// Block-wide exclusive scan of up to 2*blockDim.x values held two per thread.
+__device__ int block_excl_scan(int v, int *warp_tot, int *total) {
+    int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int nw = blockDim.x >> 5;
+        int wv = lane < nw ? warp_tot[lane] : 0;
+        int wi = wv;
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        if (lane < nw) warp_tot[lane] = wi - wv;
+        if (lane == nw - 1) *total = wi;
+    }
+    __syncthreads();
+    int r = inc - v + warp_tot[warp];
+    __syncthreads();
+    return r;
+}
+
+// Single block: offsets = exclusive scan of counts; chunk list of <= CHUNK
+// consecutive grouped positions per expert; fill[] cleared for the scatter.
+__global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ counts, int nx, int chunk,
+                                               int32_t *__restrict__ offsets, int32_t *__restrict__ fill,
+                                               int4 *__restrict__ chunks, int32_t *__restrict__ n_chunks,
+                                               int max_chunks) {
+    __shared__ int warp_tot[32];
+    __shared__ int total;
+    int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+    int c0 = e0 < nx ? counts[e0] : 0, c1 = e1 < nx ? counts[e1] : 0;
+    int base = block_excl_scan(c0 + c1, warp_tot, &total);
+    if (e0 < nx) { offsets[e0] = base; fill[e0] = 0; }
+    if (e1 < nx) { offsets[e1] = base + c0; fill[e1] = 0; }
+    if (threadIdx.x == 0) offsets[nx] = total;
+    int k0 = (c0 + chunk - 1) / chunk, k1 = (c1 + chunk - 1) / chunk;
+    int cbase = block_excl_scan(k0 + k1, warp_tot, &total);
+    for (int i = 0; i < k0; ++i)
+        if (cbase + i < max_chunks)
+            chunks[cbase + i] = make_int4(e0, base + i * chunk, min(chunk, c0 - i * chunk), 0);
+    for (int i = 0; i < k1; ++i)
+        if (cbase + k0 + i < max_chunks)
+            chunks[cbase + k0 + i] = make_int4(e1, base + c0 + i * chunk, min(chunk, c1 - i * chunk), 0);
+    if (threadIdx.x == 0) *n_chunks = min(total, max_chunks);
+}
+
+__global__ void k_scatter(const int32_t *__restrict__ ids, int T, int k, int E, int S,
+                          const int32_t *__restrict__ offsets, int32_t *__restrict__ fill,
+                          int32_t *__restrict__ perm, int32_t *__restrict__ inv) {
+    for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < S; s += gridDim.x * blockDim.x) {
+        int e = slot_expert(ids, s, T, k, E);
+        int pos = offsets[e] + atomicAdd(&fill[e], 1);
+        perm[pos] = s;
+        inv[s] = pos;
+    }
+}
+
+}  // namespace
+
+int launch_router_simt(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
+                       float *logits, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    size_t smem = (size_t)RT_TOK * c.d_model * sizeof(float);
+    static bool attr_set = false;
+    if (!attr_set) {
+        QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      200 * 1024));
+        attr_set = true;
+    }
+    dim3 grid((c.n_experts + RT_EXP - 1) / RT_EXP, (T + RT_TOK - 1) / RT_TOK);
+    k_router_simt<<<grid, 256, smem, st>>>(x, T, c.d_model, c.n_experts, Ly.router_w, Ly.router_b,
+                                          logits);
+    QE_CHECK_LAUNCH("k_router_simt");
+    return MOE_OK;
+}
+
+int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, float *w,
+                cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    size_t smem = 8 * (size_t)c.n_experts * sizeof(float);
+    k_topk<<<(T + 7) / 8, 256, smem, st>>>(logits, T, c.n_experts, c.top_k, ids, w);
+    QE_CHECK_LAUNCH("k_topk");
+    return MOE_OK;
+}
+
+int launch_dispatch(moe_ctx *ctx, const int32_t *ids, int T, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    Workspace &ws = ctx->ws;
+    int S = T * (c.top_k + c.n_shared);
+    QE_CHECK(cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * ctx->nx, st));
+    int blocks = (S + 255) / 256;
+    if (blocks > 1184) blocks = 1184;
+    k_count<<<blocks, 256, 0, st>>>(ids, T, c.top_k, c.n_experts, S, ws.counts);
+    QE_CHECK_LAUNCH("k_count");
+    k_scan<<<1, 1024, 0, st>>>(ws.counts, ctx->nx, 8, ws.offsets, ws.fill, ws.chunks, ws.n_chunks,
+                              ws.max_chunks);
+    QE_CHECK_LAUNCH("k_scan");
+    k_scatter<<<blocks, 256, 0, st>>>(ids, T, c.top_k, c.n_experts, S, ws.offsets, ws.fill, ws.perm,
+                                     ws.inv);
+    QE_CHECK_LAUNCH("k_scatter");
+    return MOE_OK;
+}
+
+}  // namespace qeffn

@@ -113,17 +113,31 @@ def _key(cfg: LayerConfig, *parts: int) -> tuple[int, int]:
     return h, _mix_int(h ^ 0x85EBCA6B)
 
 
-def _words(k1: int, k2: int, start: int, n: int, device) -> torch.Tensor:
-    i = torch.arange(start, start + n, dtype=torch.int64, device=device)
-    return mix32((mix32(i ^ k1) + k2) & M32)
-
-
 def _rows(cfg: LayerConfig, tensor: int, shared: bool) -> tuple[int, int]:
     """(rows, K) of one expert's gate/up/down matrix."""
     inner = cfg.I_s if shared else cfg.I
     if tensor in (T_GATE, T_UP):
         return inner, cfg.d
     return cfg.d, inner
+
+
+def _expert_keys(cfg: LayerConfig, layer: int, tensor: int, kind: int, e0: int, e1: int,
+                 shared: bool, device) -> tuple[torch.Tensor, torch.Tensor]:
+    ks = [_key(cfg, layer, tensor, kind, (1 << 20) + e if shared else e) for e in range(e0, e1)]
+    k1 = torch.tensor([a for a, _ in ks], dtype=torch.int64, device=device)
+    k2 = torch.tensor([b for _, b in ks], dtype=torch.int64, device=device)
+    return k1, k2
+
+
+def _expert_words(cfg, layer, tensor, kind, e0, e1, n_words, shared, device, chunk_words=1 << 25):
+    """Yield (first expert, int64 [n, n_words] words) in bounded-size chunks."""
+    k1, k2 = _expert_keys(cfg, layer, tensor, kind, e0, e1, shared, device)
+    per = max(1, chunk_words // max(1, n_words))
+    i = torch.arange(n_words, dtype=torch.int64, device=device)
+    for a in range(0, e1 - e0, per):
+        b = min(e1 - e0, a + per)
+        w = mix32((mix32(i[None, :] ^ k1[a:b, None]) + k2[a:b, None]) & M32)
+        yield a, w
 
 
 def expert_codes(cfg: LayerConfig, layer: int, tensor: int, e0: int, e1: int,
@@ -135,14 +149,14 @@ def expert_codes(cfg: LayerConfig, layer: int, tensor: int, e0: int, e1: int,
     rows, K = _rows(cfg, tensor, shared)
     nb = K // 32
     B = cfg.block_bytes
-    per_expert_words = rows * nb * B // 4
-    out = torch.empty((e1 - e0, rows, nb, B), dtype=torch.uint8, device=device)
-    for e in range(e0, e1):
-        k1, k2 = _key(cfg, layer, tensor, _T_CODES, (1 << 20) + e if shared else e)
-        w = _words(k1, k2, 0, per_expert_words, device)
-        b = torch.stack([(w >> s) & 0xFF for s in (0, 8, 16, 24)], dim=1).to(torch.uint8)
-        out[e - e0] = b.reshape(rows, nb, B)
-    return out
+    n_words = rows * nb * B // 4
+    out = torch.empty((e1 - e0, rows * nb * B), dtype=torch.uint8, device=device)
+    for a, w in _expert_words(cfg, layer, tensor, _T_CODES, e0, e1, n_words, shared, device):
+        n = w.shape[0]
+        dst = out[a:a + n].view(n, n_words, 4)
+        for j, sh in enumerate((0, 8, 16, 24)):
+            dst[:, :, j] = ((w >> sh) & 0xFF).to(torch.uint8)
+    return out.view(e1 - e0, rows, nb, B)
 
 
 def expert_scales(cfg: LayerConfig, layer: int, tensor: int, e0: int, e1: int,
@@ -150,16 +164,14 @@ def expert_scales(cfg: LayerConfig, layer: int, tensor: int, e0: int, e1: int,
     """fp16 block scales of experts [e0, e1) as int16 bit patterns [e1-e0, rows, K/32]."""
     rows, K = _rows(cfg, tensor, shared)
     nb = K // 32
-    out = torch.empty((e1 - e0, rows, nb), dtype=torch.int16, device=device)
+    out = torch.empty((e1 - e0, rows * nb), dtype=torch.int16, device=device)
     lo = torch.tensor(cfg.scale_lo, dtype=torch.float32, device=device)
     span = torch.tensor(cfg.scale_hi, dtype=torch.float32, device=device) - lo
-    for e in range(e0, e1):
-        k1, k2 = _key(cfg, layer, tensor, _T_SCALES, (1 << 20) + e if shared else e)
-        w = _words(k1, k2, 0, rows * nb, device)
+    for a, w in _expert_words(cfg, layer, tensor, _T_SCALES, e0, e1, rows * nb, shared, device):
         u = (w >> 8).to(torch.float32) * (1.0 / (1 << 24))   # exact: 24-bit integer times 2^-24
         s = (u * span) + lo
-        out[e - e0] = s.to(torch.float16).view(torch.int16).reshape(rows, nb)
-    return out
+        out[a:a + w.shape[0]] = s.to(torch.float16).view(torch.int16)
+    return out.view(e1 - e0, rows, nb)
 
 
 def _np_rng(cfg: LayerConfig, *parts: int) -> np.random.Generator:

@@ -1,0 +1,208 @@
+"""GPU parity of one MoE layer through the C ABI against the oracle, plus the
+edge cases and error codes of the boundary."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import ExpertSource, check_rows, oracle_rows, rel_l2, to_np
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.CONFIGS["tiny_d256_e16_q4_t8"]
+
+
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_expert_ffn_token_b200 import capi, session
+    return capi, session
+
+
+def _tokens(cfg, T, stream=0):
+    return synth.tokens_bf16(cfg, T, stream)
+
+
+def _run(sess, layer, x_bits):
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    y, yf, ids, w = sess.forward(layer, x)
+    torch.cuda.synchronize()
+    return to_np(y), to_np(yf), to_np(ids), to_np(w)
+
+
+def test_generator_bits_identical_on_device():
+    _cuda()
+    c = synth.CONFIGS["verify_48l_q3_t4_zipf"]
+    for t in range(3):
+        a = synth.expert_codes(c, 3, t, 100, 102, device="cuda").cpu()
+        b = synth.expert_codes(c, 3, t, 100, 102)
+        assert torch.equal(a, b)
+        a = synth.expert_scales(c, 3, t, 7, 8, device="cuda").cpu()
+        assert torch.equal(a, synth.expert_scales(c, 3, t, 7, 8))
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q3"])
+def test_tiny_layer_all_tokens(fmt):
+    capi, session = _cuda()
+    import dataclasses
+    cfg = dataclasses.replace(TINY, fmt=fmt, name=TINY.name + fmt) if fmt != "q4" else TINY
+    sess = session.Session(cfg, max_tokens=256)
+    sess.load_synthetic()
+    x = _tokens(cfg, cfg.T)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    W = synth.layer_weights(cfg, 0)
+    oy, oids, ow, ogap = oracle.moe_layer(cfg.fmt, cfg.k, x, W)
+    src = ExpertSource(cfg, 0)
+    check_rows(cfg, src, x, list(range(cfg.T)), gy, gyf, gids, gw, o=(oy, oids, ow, ogap))
+    sess.close()
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 127, 128, 129])
+def test_tiny_ragged_token_counts(T):
+    capi, session = _cuda()
+    sess = session.Session(TINY, max_tokens=256)
+    sess.load_synthetic()
+    x = _tokens(TINY, T, stream=T)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    W = synth.layer_weights(TINY, 0)
+    o = oracle.moe_layer(TINY.fmt, TINY.k, x, W)
+    check_rows(TINY, ExpertSource(TINY, 0), x, list(range(T)), gy, gyf, gids, gw, o=o)
+    sess.close()
+
+
+def test_batch_equals_single_tokens():
+    capi, session = _cuda()
+    sess = session.Session(TINY, max_tokens=64)
+    sess.load_synthetic()
+    x = _tokens(TINY, 37, stream=5)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    for t in range(37):
+        y1, yf1, ids1, w1 = _run(sess, 0, x[t:t + 1])
+        assert np.array_equal(ids1[0], gids[t])
+        assert np.array_equal(y1[0], gy[t])
+        assert np.array_equal(yf1[0], gyf[t])
+    sess.close()
+
+
+def _tiny_weights_with(mutate):
+    W = synth.layer_weights(TINY, 0, device="cuda")
+    mutate(W)
+    return W
+
+
+def test_skew_every_token_to_the_same_experts():
+    capi, session = _cuda()
+    sess = session.Session(TINY, max_tokens=256)
+    bias = np.full(TINY.E, -30.0, dtype=np.float32)
+    bias[5], bias[11] = 30.0, 29.0
+
+    def mut(W):
+        W["router_b"] = bias
+    W = _tiny_weights_with(mut)
+    sess.load(0, W)
+    x = _tokens(TINY, 200, stream=9)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    assert np.all(gids[:, 0] == 5) and np.all(gids[:, 1] == 11)
+    Wh = synth.layer_weights(TINY, 0)
+    Wh["router_b"] = bias
+    o = oracle.moe_layer(TINY.fmt, TINY.k, x, Wh)
+    src = ExpertSource(TINY, 0)
+    src.router_b = bias
+    check_rows(TINY, src, x, list(range(200)), gy, gyf, gids, gw, o=o)
+    sess.close()
+
+
+def test_zero_scale_routed_experts_leave_only_shared():
+    capi, session = _cuda()
+    sess = session.Session(TINY, max_tokens=16)
+
+    def mut(W):
+        for t in range(3):
+            W["scales"][t].zero_()
+    sess.load(0, _tiny_weights_with(mut))
+    x = _tokens(TINY, 8)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    Wh = synth.layer_weights(TINY, 0)
+    xf = oracle.bf16_to_f64(x)
+    sh = tuple((Wh["sh_codes"][t][0].numpy(), Wh["sh_scales"][t][0].numpy()) for t in range(3))
+    want = np.array([oracle.expert("q4", *sh, xf[t]) for t in range(8)])
+    assert rel_l2(gyf, want) <= 1e-6
+    sess.close()
+
+
+def test_boundary_errors_and_noop():
+    capi, session = _cuda()
+    sess = session.Session(TINY, max_tokens=16, n_layers=2)
+    sess.load_synthetic(layers=[0])
+    x = torch.zeros((17, TINY.d), dtype=torch.int16, device="cuda")
+    y = torch.zeros((17, TINY.d), dtype=torch.int16, device="cuda")
+    with pytest.raises(capi.MoeError) as e:
+        capi.moe_forward(sess.ctx, 0, x, 17, y)
+    assert e.value.status == capi.MOE_ERR_TOO_MANY_TOKENS
+    with pytest.raises(capi.MoeError) as e:
+        capi.moe_forward(sess.ctx, 1, x, 4, y)
+    assert e.value.status == capi.MOE_ERR_NOT_LOADED
+    with pytest.raises(capi.MoeError) as e:
+        capi.moe_forward(sess.ctx, 2, x, 4, y)
+    assert e.value.status == capi.MOE_ERR_INVALID_ARG
+    with pytest.raises(capi.MoeError) as e:
+        capi.moe_forward(sess.ctx, 0, None, 4, y)
+    assert e.value.status == capi.MOE_ERR_INVALID_ARG
+    y.fill_(7)
+    capi.moe_forward(sess.ctx, 0, x, 0, y)          # T == 0: nothing written
+    torch.cuda.synchronize()
+    assert int(y.min()) == 7 and int(y.max()) == 7
+    assert capi.moe_get_device_error(sess.ctx) == 0
+    sess.close()
+
+
+def test_memory_limit_gives_oom():
+    capi, session = _cuda()
+    with pytest.raises(capi.MoeError) as e:
+        session.Session(TINY, max_tokens=16, mem_limit=4096)
+    assert e.value.status == capi.MOE_ERR_OOM
+    sess = session.Session(TINY, max_tokens=16, mem_limit=400_000)   # workspace fits, weights not
+    with pytest.raises(capi.MoeError) as e:
+        sess.load_synthetic(layers=[0])
+    assert e.value.status == capi.MOE_ERR_OOM
+    sess.close()
+
+
+def _full_layer(name, T, rows):
+    capi, session = _cuda()
+    cfg = synth.CONFIGS[name]
+    sess = session.Session(cfg, max_tokens=T, n_layers=1)
+    sess.load_synthetic(layers=[0])
+    x = _tokens(cfg, T)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    sess.close()
+    src = ExpertSource(cfg, 0)
+    rows = list(rows)
+    rep = {}
+    check_rows(cfg, src, x, rows, gy[rows], gyf[rows], gids[rows], gw[rows], report=rep)
+    return cfg, x, gids, gw, src, rep
+
+
+def test_decode_layer_full_size():
+    _full_layer("decode_48l_q4_t1", 1, [0])
+
+
+def test_verify_layer_full_size():
+    _full_layer("verify_48l_q3_t4_zipf", 4, range(4))
+
+
+def test_prefill_layer_full_size_sampled():
+    cfg, x, gids, gw, src, rep = _full_layer("prefill_1l_q4_t4096_zipf", 4096,
+                                             [0, 1, 2, 1000, 2047, 2048, 4094, 4095])
+    # routing of every token against the oracle (ids exact up to near ties)
+    flips = 0
+    for t in range(0, 4096, 8):
+        xf = oracle.bf16_to_f64(x[t])
+        ids, w, gap = oracle.route(oracle.router_logits(xf, src.router_w, src.router_b), cfg.k)
+        if not np.array_equal(ids, gids[t]):
+            assert gap < 1e-5
+            flips += 1
+        else:
+            assert np.max(np.abs(w - gw[t])) <= 1e-5
+    assert flips <= 2

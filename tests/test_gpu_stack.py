@@ -1,0 +1,74 @@
+"""GPU parity of the 48-layer stacks, teacher-forced: every layer's recorded
+bf16 input (the GPU's own) is fed to the oracle, whose output, ids and
+weights are compared with the GPU's record of that layer; the residual chain
+between layers is checked separately."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import ExpertSource, bits_to_f64, check_rows, oracle_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _stack(name, rows=None, check_layers=None):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_expert_ffn_token_b200 import capi, session
+    cfg = synth.CONFIGS[name]
+    L, T, d, k = cfg.L, cfg.T, cfg.d, cfg.k
+    sess = session.Session(cfg, max_tokens=T)
+    sess.load_synthetic()
+    x_bits = synth.tokens_bf16(cfg)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    n_rec = T if rows is None else len(rows)
+    dev = "cuda"
+    xr = torch.empty((L, n_rec, d), dtype=torch.int16, device=dev)
+    yr = torch.empty((L, n_rec, d), dtype=torch.int16, device=dev)
+    yfr = torch.empty((L, n_rec, d), dtype=torch.float32, device=dev)
+    idr = torch.empty((L, n_rec, k), dtype=torch.int32, device=dev)
+    wr = torch.empty((L, n_rec, k), dtype=torch.float32, device=dev)
+    rows_t = None if rows is None else torch.tensor(rows, dtype=torch.int32, device=dev)
+    rec = capi.make_record(xr, yr, yfr, idr, wr, rows_t)
+    r_out = torch.empty((T, d), dtype=torch.float32, device=dev)
+    capi.moe_forward_stack(sess.ctx, 0, L, x, T, r_out, rec)
+    torch.cuda.synchronize()
+    assert capi.moe_get_device_error(sess.ctx) == 0
+    sess.close()
+    xr, yr, yfr, idr, wr, r_out = map(to_np, (xr, yr, yfr, idr, wr, r_out))
+    rows = list(range(T)) if rows is None else list(rows)
+
+    # residual chain: r_0 = x, x_l = bf16(rmsnorm(r_l)), r_{l+1} = r_l + y_l
+    r = bits_to_f64(x_bits[rows])
+    for l in range(L):
+        want = np.array([oracle.rmsnorm(ri, 1e-6) for ri in r])
+        got = bits_to_f64(xr[l])
+        ulp = np.abs(bits_to_f64(oracle.round_bf16(want))) * 2.0 ** -7 + 1e-30
+        assert np.all(np.abs(got - want) <= ulp), f"layer {l}: stack input off by more than 1 ulp"
+        r = r + bits_to_f64(yr[l])
+    assert np.allclose(r_out[rows], r, rtol=1e-5, atol=1e-5 * np.abs(r).max())
+
+    worst = {}
+    for l in (range(L) if check_layers is None else check_layers):
+        src = ExpertSource(cfg, l)
+        rep = {}
+        idx = list(range(len(rows)))
+        check_rows(cfg, src, xr[l], idx, yr[l], yfr[l], idr[l], wr[l], report=rep)
+        worst[l] = rep
+    return worst
+
+
+def test_decode_stack_48_layers():
+    _stack("decode_48l_q4_t1")
+
+
+def test_verify_stack_48_layers():
+    _stack("verify_48l_q3_t4_zipf")
+
+
+@pytest.mark.slow
+def test_long_prefill_stack_48_layers_sampled():
+    _stack("prefill_48l_q3_t32768", rows=[0, 16383, 32767],
+           check_layers=[0, 1, 23, 46, 47])
