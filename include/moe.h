@@ -79,7 +79,17 @@ typedef struct {
     int max_tokens;     /* largest T any call may pass */
     int fmt;            /* moe_qformat */
     long long device_mem_limit; /* bytes the context may allocate; 0 = no limit */
+    int flags;          /* MOE_FLAG_* bits, 0 for normal use */
 } moe_config;
+
+/* moe_config.flags.  The first two pin a call to one implementation (tests
+ * compare the paths with each other); the last is a test hook for the
+ * bounded device waits: the decode kernel's CTA 0 withholds its router
+ * logits, every wait on them runs out after about one second, and the call
+ * reports MOE_ERR_DEVICE_TIMEOUT through moe_get_device_error. */
+#define MOE_FLAG_NO_DECODE_KERNEL 1   /* T == 1 runs the general path */
+#define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
+#define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
 
 typedef struct {
     const float *router_w;          /* [E][d] */

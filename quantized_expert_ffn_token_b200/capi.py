@@ -25,6 +25,9 @@ MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_ERR_UNSUPPORTED = -7
 MOE_Q4B32 = 1
 MOE_Q3B32 = 2
+MOE_FLAG_NO_DECODE_KERNEL = 1
+MOE_FLAG_NO_TENSOR_PREFILL = 2
+MOE_FLAG_TEST_WITHHOLD = 256
 FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32}
 
 EXPORTED = [
@@ -38,7 +41,7 @@ class moe_config(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int), ("n_experts", ctypes.c_int), ("d_ff", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_shared", ctypes.c_int), ("d_ff_shared", ctypes.c_int),
                 ("n_layers", ctypes.c_int), ("max_tokens", ctypes.c_int), ("fmt", ctypes.c_int),
-                ("device_mem_limit", ctypes.c_longlong)]
+                ("device_mem_limit", ctypes.c_longlong), ("flags", ctypes.c_int)]
 
 
 class moe_layer_weights(ctypes.Structure):

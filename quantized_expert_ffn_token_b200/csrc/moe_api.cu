@@ -127,6 +127,12 @@ int alloc_workspace(moe_ctx *ctx) {
     };
     for (auto &it : items) QE_TRY(ctx_alloc(ctx, it.p, it.bytes, it.name));
     QE_CHECK(cudaMemset(ws.dev_error, 0, 4));
+    QE_TRY(ctx_alloc(ctx, (void **)&ctx->d_layers, sizeof(LayerPtrs) * c.n_layers, "layer table"));
+    QE_CHECK(cudaMemset(ctx->d_layers, 0, sizeof(LayerPtrs) * c.n_layers));
+    QE_TRY(decode_setup(ctx));
+    size_t llb = decode_ll_bytes(c);
+    QE_TRY(ctx_alloc(ctx, (void **)&ctx->dec.ll, llb, "flag buffers"));
+    QE_CHECK(cudaMemset(ctx->dec.ll, 0, llb));
     return MOE_OK;
 }
 
@@ -199,6 +205,8 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
         temps.clear();
     }
     QE_CHECK(cudaStreamSynchronize(st));
+    LayerPtrs lp{Ly.router_w, Ly.router_b, Ly.gu, Ly.dn};
+    QE_CHECK(cudaMemcpy(ctx->d_layers + layer, &lp, sizeof(lp), cudaMemcpyHostToDevice));
     Ly.loaded = true;
     return MOE_OK;
 }
@@ -209,6 +217,12 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
     Workspace &ws = ctx->ws;
     int32_t *ids_ = ids ? ids : ws.ids;
     float *w_ = w ? w : ws.w;
+    if (decode_supported(ctx, T)) {
+        QE_TRY(timing_begin(ctx, st, "k_decode"));
+        QE_TRY(launch_decode(ctx, layer, 1, x, false, nullptr, y, yf, ids_, w_, nullptr, st));
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
     QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
     QE_TRY(launch_topk(ctx, ws.logits, T, ids_, w_, st));
     QE_TRY(launch_dispatch(ctx, ids_, T, st));
@@ -291,6 +305,14 @@ int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint16_t *x_
     QE_CHECK(cudaSetDevice(ctx->device));
     cudaStream_t st = (cudaStream_t)stream;
     Workspace &ws = ctx->ws;
+    if (decode_supported(ctx, T)) {
+        if (rec && rec->rows && rec->n_rows != 1) return MOE_ERR_INVALID_ARG;
+        QE_TRY(timing_begin(ctx, st, "k_decode"));
+        QE_TRY(launch_decode(ctx, layer0, n_layers, x_bf16, true, resid_out, nullptr, nullptr, nullptr,
+                             nullptr, rec, st));
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
     QE_TRY(launch_resid_norm(ctx, T, resid_out, nullptr, x_bf16, ws.xs, st));
     for (int l = 0; l < n_layers; ++l) {
         QE_TRY(forward_layer(ctx, layer0 + l, ws.xs, T, ws.ys, ws.yf, ws.ids, ws.w, st));

@@ -143,6 +143,25 @@ struct Workspace {
     int max_chunks = 0;
 };
 
+// Device-side table of one layer's weights (the persistent kernels walk it).
+struct LayerPtrs {
+    const float *rw;      // router [E][d]
+    const float *rb;      // router bias [E]
+    const uint8_t *gu;    // gate/up tiles of E + n_shared experts
+    const uint8_t *dn;    // down tiles of E + n_shared experts
+};
+
+// Launch plan of the single-token decode kernel (decode.cu).
+struct DecodeState {
+    int grid = 0;         // CTAs (one per SM)
+    int smem_bytes = 0;   // 0: the shape does not fit the kernel
+    int nslot = 0, slot_bytes = 0, rpc = 0;
+    int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
+        off_misc = 0;
+    uint2 *ll = nullptr;  // flagged-word exchange buffers
+    uint32_t epoch = 1;
+};
+
 // Event pairs around the dominant kernel (moe_timing_enable).
 struct Timing {
     bool on = false;
@@ -165,6 +184,8 @@ struct moe_ctx {
     size_t allocated = 0;
     std::vector<std::pair<void *, size_t>> allocs;
     qeffn::Timing timing;
+    qeffn::LayerPtrs *d_layers = nullptr;   // [n_layers] on the device
+    qeffn::DecodeState dec;
 };
 
 namespace qeffn {
@@ -208,6 +229,12 @@ int launch_combine(const moe_ctx *ctx, int T, const float *w, uint16_t *y, float
                    cudaStream_t st);
 int launch_resid_norm(const moe_ctx *ctx, int T, float *resid, const uint16_t *y_add,
                       const uint16_t *x_in, uint16_t *x_out, cudaStream_t st);
+bool decode_supported(const moe_ctx *ctx, int T);
+int decode_setup(moe_ctx *ctx);
+size_t decode_ll_bytes(const moe_config &c);
+int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
+                  uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
+                  cudaStream_t st);
 int launch_record(const moe_ctx *ctx, int T, int layer_idx, const moe_stack_record *rec,
                   const uint16_t *x, const uint16_t *y, const float *yf, const int32_t *ids,
                   const float *w, cudaStream_t st);

@@ -13,7 +13,7 @@ from . import capi
 
 
 def config_struct(cfg: "synth.LayerConfig", max_tokens: int | None = None,
-                  n_layers: int | None = None, mem_limit: int = 0) -> capi.moe_config:
+                  n_layers: int | None = None, mem_limit: int = 0, flags: int = 0) -> capi.moe_config:
     c = capi.moe_config()
     c.d_model, c.n_experts, c.d_ff, c.top_k = cfg.d, cfg.E, cfg.I, cfg.k
     c.n_shared, c.d_ff_shared = cfg.n_shared, cfg.I_s
@@ -21,6 +21,7 @@ def config_struct(cfg: "synth.LayerConfig", max_tokens: int | None = None,
     c.max_tokens = cfg.T if max_tokens is None else max_tokens
     c.fmt = capi.FORMATS[cfg.fmt]
     c.device_mem_limit = mem_limit
+    c.flags = flags
     return c
 
 
@@ -46,11 +47,11 @@ class Session:
     """One library context on one device."""
 
     def __init__(self, cfg: "synth.LayerConfig", device: int = 0, max_tokens: int | None = None,
-                 n_layers: int | None = None, mem_limit: int = 0):
+                 n_layers: int | None = None, mem_limit: int = 0, flags: int = 0):
         self.cfg = cfg
         self.device = torch.device("cuda", device)
         self.n_layers = cfg.L if n_layers is None else n_layers
-        self.ctx = capi.moe_create(config_struct(cfg, max_tokens, self.n_layers, mem_limit), device)
+        self.ctx = capi.moe_create(config_struct(cfg, max_tokens, self.n_layers, mem_limit, flags), device)
 
     def load_synthetic(self, layers=None, stream=None) -> None:
         for l in (range(self.n_layers) if layers is None else layers):

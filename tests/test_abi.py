@@ -40,11 +40,11 @@ def test_argument_checks_need_no_device():
     from quantized_expert_ffn_token_b200 import capi
     h = ctypes.c_void_p()
     assert capi.lib.moe_create(None, 0, ctypes.byref(h)) == capi.MOE_ERR_INVALID_ARG
-    c = capi.moe_config(256, 16, 128, 2, 1, 128, 1, 8, 9, 0)      # fmt 9 does not exist
+    c = capi.moe_config(256, 16, 128, 2, 1, 128, 1, 8, 9, 0, 0)      # fmt 9 does not exist
     assert capi.lib.moe_create(ctypes.byref(c), 0, ctypes.byref(h)) == capi.MOE_ERR_INVALID_ARG
-    c = capi.moe_config(250, 16, 128, 2, 1, 128, 1, 8, capi.MOE_Q4B32, 0)   # d not a multiple of 256
+    c = capi.moe_config(250, 16, 128, 2, 1, 128, 1, 8, capi.MOE_Q4B32, 0, 0)   # d not a multiple of 256
     assert capi.lib.moe_create(ctypes.byref(c), 0, ctypes.byref(h)) == capi.MOE_ERR_UNSUPPORTED
-    c = capi.moe_config(256, 16, 128, 17, 1, 128, 1, 8, capi.MOE_Q4B32, 0)  # k > E
+    c = capi.moe_config(256, 16, 128, 17, 1, 128, 1, 8, capi.MOE_Q4B32, 0, 0)  # k > E
     assert capi.lib.moe_create(ctypes.byref(c), 0, ctypes.byref(h)) == capi.MOE_ERR_INVALID_ARG
     assert capi.lib.moe_forward(None, 0, None, 1, None, None, None, None, None) == capi.MOE_ERR_INVALID_ARG
     assert capi.lib.moe_destroy(None) == capi.MOE_OK

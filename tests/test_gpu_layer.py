@@ -72,17 +72,43 @@ def test_tiny_ragged_token_counts(T):
 
 
 def test_batch_equals_single_tokens():
+    """Token independence of the grouped path: a token's output does not depend
+    on which other tokens share the call (bit for bit)."""
     capi, session = _cuda()
     sess = session.Session(TINY, max_tokens=64)
     sess.load_synthetic()
     x = _tokens(TINY, 37, stream=5)
     gy, gyf, gids, gw = _run(sess, 0, x)
     for t in range(37):
-        y1, yf1, ids1, w1 = _run(sess, 0, x[t:t + 1])
-        assert np.array_equal(ids1[0], gids[t])
-        assert np.array_equal(y1[0], gy[t])
-        assert np.array_equal(yf1[0], gyf[t])
+        pair = x[[t, (t + 11) % 37]]
+        y2, yf2, ids2, w2 = _run(sess, 0, pair)
+        assert np.array_equal(ids2[0], gids[t])
+        assert np.array_equal(y2[0], gy[t])
+        assert np.array_equal(yf2[0], gyf[t])
     sess.close()
+
+
+@pytest.mark.parametrize("name", ["tiny_d256_e16_q4_t8", "decode_48l_q4_t1"])
+def test_decode_kernel_matches_general_path(name):
+    """Single-token calls: the persistent decode kernel against the general
+    grouped path on the same inputs (same ids; fp32 outputs within 1e-5)."""
+    capi, session = _cuda()
+    cfg = synth.CONFIGS[name]
+    a = session.Session(cfg, max_tokens=4, n_layers=1)
+    b = session.Session(cfg, max_tokens=4, n_layers=1, flags=capi.MOE_FLAG_NO_DECODE_KERNEL)
+    W = synth.layer_weights(cfg, 0, device="cuda")
+    a.load(0, W)
+    b.load(0, W)
+    del W
+    for s in range(4):
+        x = _tokens(cfg, 1, stream=40 + s)
+        ya, yfa, ida, wa = _run(a, 0, x)
+        yb, yfb, idb, wb = _run(b, 0, x)
+        assert np.array_equal(ida, idb)
+        assert np.max(np.abs(wa - wb)) <= 1e-6
+        assert rel_l2(yfa, yfb) <= 1e-5
+    a.close()
+    b.close()
 
 
 def _tiny_weights_with(mutate):
