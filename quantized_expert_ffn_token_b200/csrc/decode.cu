@@ -776,20 +776,21 @@ int decode_setup(moe_ctx *ctx) {
     }
     int slot = ctx->gu.tile_bytes;
     if (slot < ctx->dn.tile_bytes) slot = ctx->dn.tile_bytes;
-    auto al = [](size_t v) { return (v + 127) & ~(size_t)127; };
+    // carve shared memory: each region 128-byte aligned, in this order, no overlap
     size_t fixed = 0;
-    ds.off_router = (int)fixed;
-    fixed = al(fixed + (size_t)rpc * c.d_model * 4);
-    ds.off_x16 = (int)fixed;
-    fixed = al(fixed + (size_t)c.d_model * 2);
-    ds.off_logits = (int)fixed;
-    fixed = al(fixed + (size_t)c.n_experts * 4);
-    ds.off_htab = (int)fixed;
-    fixed = al(fixed + (size_t)MAXU * 2 * c.d_ff * 2);
-    ds.off_red = (int)fixed;
-    fixed = al(fixed + (size_t)2 * NW * 16 * 4 > 8 * NW * 4 ? (size_t)2 * NW * 16 * 4 : (size_t)8 * NW * 4);
-    ds.off_misc = (int)fixed;
-    fixed = al(fixed + sizeof(Misc));
+    auto take = [&fixed](size_t bytes) {
+        int off = (int)fixed;
+        fixed = (fixed + bytes + 127) & ~(size_t)127;
+        return off;
+    };
+    size_t red_bytes = (size_t)2 * NW * 16 * 4;
+    if (red_bytes < (size_t)8 * NW * 4) red_bytes = (size_t)8 * NW * 4;
+    ds.off_router = take((size_t)rpc * c.d_model * 4);
+    ds.off_x16 = take((size_t)c.d_model * 2);
+    ds.off_logits = take((size_t)c.n_experts * 4);
+    ds.off_htab = take((size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2);   // fp16 hi + lo of h
+    ds.off_red = take(red_bytes);
+    ds.off_misc = take(sizeof(Misc));
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
