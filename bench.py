@@ -214,14 +214,17 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     union = cfg.k if cfg.T == 1 else None
     if union is None:
         union = measured_union(sess, cfg, xs[0], dev)
-    alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)
+    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+    if tim["kernel"] == "k_decode":
+        alg_bytes = step_bytes          # one launch runs the whole stack (router rows included)
+    else:
+        alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)   # one launch per layer, experts only
     avg_ms = tim["ms"] / max(1, tim["timed_launches"])
     achieved = alg_bytes / (avg_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / P["hbm_gbs"], "traffic": None, "kernel": tim["kernel"],
             "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_ms,
             "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
-    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
 
     # end to end through the public host-buffer entry point
     x_host = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).pin_memory()
@@ -331,9 +334,14 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=12, help="oracle sample: layers per token")
     ap.add_argument("--ref-layers", type=int, default=2, help="reference arm: layers per step")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="stack depth override (small cases for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     cfg = synth.CONFIGS[args.workload]
+    if args.layers is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, L=args.layers)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

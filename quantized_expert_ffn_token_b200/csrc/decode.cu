@@ -42,7 +42,6 @@ constexpr int MAX_SLOTS = 8;
 constexpr int MAXK = 32;
 constexpr int MAXU = MAXK + 4;
 constexpr int CAND_MAX = 256;
-constexpr int RMAX = 11;                         // residual floats per thread, d <= 4096
 constexpr long long SPIN_LIMIT = 2000000000LL;   // clock64 cycles, about one second
 
 struct Misc {
@@ -82,7 +81,7 @@ struct DecodeParams {
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
     int nslot, slot_bytes, rpc;
-    int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc;
+    int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid;
 };
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -194,22 +193,43 @@ __device__ __forceinline__ float bf16_bits_f(uint16_t b) { return __uint_as_floa
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
 
-// Poll one flagged word.  Returns false on timeout or when another CTA failed.
-__device__ __noinline__ bool ll_wait(const uint2 *p, uint32_t flag, float *out, int *err, long long t0) {
-    for (int it = 0;; ++it) {
-        uint2 v = ll_load(p);
-        if (v.y == flag) {
-            *out = __uint_as_float(v.x);
-            return true;
-        }
-        if ((it & 31) == 31) {
-            if (*(volatile int *)err != 0) return false;
-            if (clock64() - t0 > SPIN_LIMIT) {
-                atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
-                return false;
+// Poll the flagged words base[i], i = tid + NT*j < n, with up to B loads of
+// this thread in flight at a time; put(i, value) receives each value once.
+template <int B, typename F>
+__device__ __forceinline__ bool poll_words(const uint2 *base, int n, uint32_t flag, int *err, F &&put) {
+    long long t0 = clock64();
+    for (int j0 = threadIdx.x; j0 < n; j0 += NT * B) {
+        bool need[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) need[b] = j0 + b * NT < n;
+        for (int it = 0;; ++it) {
+            uint2 v[B];
+#pragma unroll
+            for (int b = 0; b < B; ++b)
+                if (need[b]) v[b] = ll_load(base + j0 + b * NT);
+            bool all = true;
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+                if (need[b]) {
+                    if (v[b].y == flag) {
+                        put(j0 + b * NT, __uint_as_float(v[b].x));
+                        need[b] = false;
+                    } else {
+                        all = false;
+                    }
+                }
+            }
+            if (all) break;
+            if ((it & 7) == 7) {
+                if (*(volatile int *)err != 0) return false;
+                if (clock64() - t0 > SPIN_LIMIT) {
+                    atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                    return false;
+                }
             }
         }
     }
+    return true;
 }
 
 __device__ __noinline__ bool mbar_wait(unsigned long long *b, uint32_t parity, int *err, bool honor_err) {
@@ -242,6 +262,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     __half *htab = reinterpret_cast<__half *>(smem + p.off_htab);
     float *red = reinterpret_cast<float *>(smem + p.off_red);   // [2][NW][16]
     Misc *ms = reinterpret_cast<Misc *>(smem + p.off_misc);
+    float *rs = reinterpret_cast<float *>(smem + p.off_resid);      // residual stream [d]
+    float *ybuf = reinterpret_cast<float *>(smem + p.off_htab);     // [d], free between layers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const int G = gridDim.x, cta = blockIdx.x;
@@ -275,7 +297,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     };
     if (tid == 0) issue_router(p.layer0);
 
-    float r[RMAX];                       // residual stream, elements i = tid + NT*j
     long long item = 0;                  // ring items planned so far (all layers)
     long long issued = 0;                // ring items whose copies were issued (thread 0)
     long long consumed = 0;              // ring items consumed so far
@@ -292,49 +313,34 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         // ---- 1. layer input -------------------------------------------------------
         if (p.stack) {
             if (l == 0) {
-#pragma unroll
-                for (int j = 0; j < RMAX; ++j) {
-                    int i = tid + NT * j;
-                    if (i < d) r[j] = bf16_bits_f(p.x_in[i]);
-                }
+                for (int i = tid; i < d; i += NT) rs[i] = bf16_bits_f(p.x_in[i]);
             } else {
-                long long t0 = clock64();
+                // previous layer's output = part 0 + part 1 of every row (same thread owns row i)
                 const uint2 *y0 = p.ll_y + (size_t)((l - 1) & 1) * 2 * d;
-#pragma unroll
-                for (int j = 0; j < RMAX; ++j) {
-                    int i = tid + NT * j;
-                    if (i < d && ok) {
-                        float a = 0.f, b = 0.f;
-                        ok = ll_wait(y0 + i, ep - 1, &a, err, t0) && ll_wait(y0 + d + i, ep - 1, &b, err, t0);
-                        float y = a + b;
-                        uint16_t yb = bf16_rn_bits(y);
-                        r[j] += bf16_bits_f(yb);
-                        if (cta == 0 && p.rec_on) {
-                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
-                            if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
-                        }
+                ok = poll_words<8>(y0, d, ep - 1, err, [&](int i, float v) { ybuf[i] = v; });
+                ok = ok && poll_words<8>(y0 + d, d, ep - 1, err, [&](int i, float v) {
+                    float y = ybuf[i] + v;
+                    uint16_t yb = bf16_rn_bits(y);
+                    rs[i] += bf16_bits_f(yb);
+                    if (cta == 0 && p.rec_on) {
+                        if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
+                        if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
                     }
-                }
+                });
                 if (cta_failed(ms, ok)) break;
             }
             float ss = 0.f;
-#pragma unroll
-            for (int j = 0; j < RMAX; ++j)
-                if (tid + NT * j < d) ss = fmaf(r[j], r[j], ss);
+            for (int i = tid; i < d; i += NT) ss = fmaf(rs[i], rs[i], ss);
             for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
             if (lane == 0) ms->red1[warp] = ss;
             __syncthreads();
             float tot = 0.f;
             for (int w = 0; w < NW; ++w) tot += ms->red1[w];
             float inv = 1.f / sqrtf(tot / (float)d + 1e-6f);
-#pragma unroll
-            for (int j = 0; j < RMAX; ++j) {
-                int i = tid + NT * j;
-                if (i < d) {
-                    uint16_t xb = bf16_rn_bits(r[j] * inv);
-                    x16[i] = __float2half_rn(bf16_bits_f(xb));
-                    if (cta == 0 && p.rec_on && p.rec.x_bf16) p.rec.x_bf16[(size_t)l * d + i] = xb;
-                }
+            for (int i = tid; i < d; i += NT) {
+                uint16_t xb = bf16_rn_bits(rs[i] * inv);
+                x16[i] = __float2half_rn(bf16_bits_f(xb));
+                if (cta == 0 && p.rec_on && p.rec.x_bf16) p.rec.x_bf16[(size_t)l * d + i] = xb;
             }
         } else {
             for (int i = tid; i < d; i += NT) x16[i] = __float2half_rn(bf16_bits_f(p.x_in[i]));
@@ -382,8 +388,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 
         // ---- 3. top-k on all logits (same result in every CTA) ------------------------
         {
-            long long t0 = clock64();
-            for (int e = tid; e < E && ok; e += NT) ok = ll_wait(p.ll_logits + (size_t)lpar * E + e, ep, &lg[e], err, t0);
+            ok = poll_words<3>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
             if (tid == 0) ms->ncand = 0;
             if (cta_failed(ms, ok)) break;
             // threshold: the k-th largest of the warps' maxima bounds the k-th largest logit from below
@@ -609,16 +614,13 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 
         // h of every expert in use -> fp16 hi + lo table
         {
-            long long t0 = clock64();
-            for (int i = tid; i < nU * I && ok; i += NT) {
-                float h = 0.f;
-                ok = ll_wait(p.ll_h + (size_t)lpar * MAXU * I + i, ep, &h, err, t0);
+            ok = poll_words<8>(p.ll_h + (size_t)lpar * MAXU * I, nU * I, ep, err, [&](int i, float h) {
                 __half hi = __float2half_rn(h);
                 __half lo = __float2half_rn(h - __half2float(hi));
                 int us = i / I, kk = i % I;
                 htab[(size_t)(2 * us) * I + kk] = hi;
                 htab[(size_t)(2 * us + 1) * I + kk] = lo;
-            }
+            });
             if (cta_failed(ms, ok)) break;
         }
 
@@ -711,33 +713,22 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         const int l = p.L - 1;
         const uint32_t ep = p.epoch0 + (uint32_t)l;
         const uint2 *y0 = p.ll_y + (size_t)(l & 1) * 2 * d;
-        long long t0 = clock64();
         if (cta == 0) {
-            if (p.stack) {
-#pragma unroll
-                for (int j = 0; j < RMAX; ++j) {
-                    int i = tid + NT * j;
-                    if (i < d && ok) {
-                        float a = 0.f, b = 0.f;
-                        ok = ll_wait(y0 + i, ep, &a, err, t0) && ll_wait(y0 + d + i, ep, &b, err, t0);
-                        float y = a + b;
-                        uint16_t yb = bf16_rn_bits(y);
-                        p.resid_out[i] = r[j] + bf16_bits_f(yb);
-                        if (p.rec_on) {
-                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)l * d + i] = yb;
-                            if (p.rec.y_f32) p.rec.y_f32[(size_t)l * d + i] = y;
-                        }
+            ok = poll_words<8>(y0, d, ep, err, [&](int i, float v) { ybuf[i] = v; });
+            ok = ok && poll_words<8>(y0 + d, d, ep, err, [&](int i, float v) {
+                float y = ybuf[i] + v;
+                uint16_t yb = bf16_rn_bits(y);
+                if (p.stack) {
+                    p.resid_out[i] = rs[i] + bf16_bits_f(yb);
+                    if (p.rec_on) {
+                        if (p.rec.y_bf16) p.rec.y_bf16[(size_t)l * d + i] = yb;
+                        if (p.rec.y_f32) p.rec.y_f32[(size_t)l * d + i] = y;
                     }
-                }
-            } else {
-                for (int i = tid; i < d && ok; i += NT) {
-                    float a = 0.f, b = 0.f;
-                    ok = ll_wait(y0 + i, ep, &a, err, t0) && ll_wait(y0 + d + i, ep, &b, err, t0);
-                    float y = a + b;
-                    p.y_out[i] = bf16_rn_bits(y);
+                } else {
+                    p.y_out[i] = yb;
                     if (p.yf_out) p.yf_out[i] = y;
                 }
-            }
+            });
         }
     }
     // drain copies still in flight (abort path) before the CTA's shared memory goes away
@@ -788,9 +779,12 @@ int decode_setup(moe_ctx *ctx) {
     ds.off_router = take((size_t)rpc * c.d_model * 4);
     ds.off_x16 = take((size_t)c.d_model * 2);
     ds.off_logits = take((size_t)c.n_experts * 4);
-    ds.off_htab = take((size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2);   // fp16 hi + lo of h
+    size_t htab = (size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2;   // fp16 hi + lo of h
+    if (htab < (size_t)c.d_model * 4) htab = (size_t)c.d_model * 4;    // doubles as the y buffer
+    ds.off_htab = take(htab);
     ds.off_red = take(red_bytes);
     ds.off_misc = take(sizeof(Misc));
+    ds.off_resid = take((size_t)c.d_model * 4);
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
@@ -861,6 +855,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_htab = ds.off_htab;
     p.off_red = ds.off_red;
     p.off_misc = ds.off_misc;
+    p.off_resid = ds.off_resid;
     void *args[] = {&p};
     QE_CHECK(cudaLaunchCooperativeKernel((void *)k_decode, dim3(ds.grid), dim3(NT), args,
                                          (size_t)ds.smem_bytes, st));

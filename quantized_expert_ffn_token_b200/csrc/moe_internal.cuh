@@ -157,7 +157,7 @@ struct DecodeState {
     int smem_bytes = 0;   // 0: the shape does not fit the kernel
     int nslot = 0, slot_bytes = 0, rpc = 0;
     int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
-        off_misc = 0;
+        off_misc = 0, off_resid = 0;
     uint2 *ll = nullptr;  // flagged-word exchange buffers
     uint32_t epoch = 1;
 };
