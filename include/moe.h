@@ -90,6 +90,7 @@ typedef struct {
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* T == 1 runs the general path */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
+#define MOE_FLAG_TRACE 4              /* record per-phase timestamps (moe_trace_read) */
 
 typedef struct {
     const float *router_w;          /* [E][d] */
@@ -178,6 +179,15 @@ MOE_API int moe_get_device_error(moe_ctx *ctx, int *code);
 MOE_API int moe_timing_enable(moe_ctx *ctx, int on);
 MOE_API int moe_timing_read(moe_ctx *ctx, double *total_ms, long long *timed_launches,
                             long long *all_launches, char *name, int name_len);
+
+/* Phase trace of the last persistent-kernel call (context created with
+ * MOE_FLAG_TRACE).  Copies up to n_max records into out (host memory) and
+ * returns their number in *n.  One record = 8 uint64: CTA index, layer, then
+ * the SM clock (clock64) at the end of each of the six phases of that layer
+ * in that CTA (input ready, router published, routing known, gate/up done,
+ * h ready, down done); the first timestamp is relative to the layer start.
+ * Synchronises the device. */
+MOE_API int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int *n);
 
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);

@@ -28,12 +28,14 @@ MOE_Q3B32 = 2
 MOE_FLAG_NO_DECODE_KERNEL = 1
 MOE_FLAG_NO_TENSOR_PREFILL = 2
 MOE_FLAG_TEST_WITHHOLD = 256
+MOE_FLAG_TRACE = 4
 FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32}
 
 EXPORTED = [
     "moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
     "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
     "moe_status_string", "moe_last_error", "moe_timing_enable", "moe_timing_read",
+    "moe_trace_read",
 ]
 
 
@@ -79,13 +81,14 @@ def _load() -> ctypes.CDLL:
     L.moe_timing_enable.argtypes = [vp, i]
     L.moe_timing_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
                                   ctypes.POINTER(ctypes.c_longlong), ctypes.c_char_p, i]
+    L.moe_trace_read.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong), i, ctypes.POINTER(i)]
     L.moe_status_string.argtypes = [i]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_error.argtypes = []
     L.moe_last_error.restype = ctypes.c_char_p
     for n in ("moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
               "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
-              "moe_timing_enable", "moe_timing_read"):
+              "moe_timing_enable", "moe_timing_read", "moe_trace_read"):
         getattr(L, n).restype = i
     return L
 
@@ -176,6 +179,14 @@ def moe_timing_read(ctx) -> dict:
            "moe_timing_read")
     return {"ms": ms.value, "timed_launches": timed.value, "all_launches": allk.value,
             "kernel": name.value.decode()}
+
+
+def moe_trace_read(ctx, n_max: int = 1 << 16):
+    """Phase trace records as a list of 8-tuples (see include/moe.h)."""
+    buf = (ctypes.c_ulonglong * (8 * n_max))()
+    n = ctypes.c_int(0)
+    _check(lib.moe_trace_read(ctx, buf, n_max, ctypes.byref(n)), "moe_trace_read")
+    return [tuple(buf[8 * i:8 * i + 8]) for i in range(n.value)]
 
 
 def make_record(x=None, y=None, y_f32=None, ids=None, w=None, rows=None) -> moe_stack_record:

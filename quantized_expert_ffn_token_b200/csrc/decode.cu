@@ -80,6 +80,7 @@ struct DecodeParams {
     uint32_t epoch0;
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
+    unsigned long long *trace; // [G][L][8] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid;
 };
@@ -253,6 +254,17 @@ __device__ __forceinline__ bool cta_failed(Misc *ms, bool mine_ok) {
     return ms->abort != 0;
 }
 
+__device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph, long long t) {
+    if (p.trace && threadIdx.x == 0) {
+        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * 8;
+        if (ph == 0) {
+            r[0] = blockIdx.x;
+            r[1] = l;
+        }
+        r[2 + ph] = (unsigned long long)t;
+    }
+}
+
 __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *ring = smem + p.off_ring;
@@ -309,6 +321,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         const LayerPtrs Lp = p.layers[layer];
         const uint32_t ep = p.epoch0 + (uint32_t)l;
         const int lpar = l & 1;
+        const long long tl0 = clock64();
 
         // ---- 1. layer input -------------------------------------------------------
         if (p.stack) {
@@ -347,6 +360,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         }
         __syncthreads();
 
+        trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
         {
             ok = mbar_wait(&ms->rbar, (uint32_t)(l & 1), err, true);
@@ -386,6 +400,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             }
         }
 
+        trace_mark(p, l, 1, clock64() - tl0);
         // ---- 3. top-k on all logits (same result in every CTA) ------------------------
         {
             ok = poll_words<3>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
@@ -487,6 +502,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             __syncthreads();
         }
 
+        trace_mark(p, l, 2, clock64() - tl0);
         // ---- 4./5. stream and compute ----------------------------------------------
         const int n_gu_all = nU * ntile_gu;
         const int n_gu = (cta < n_gu_all) ? (n_gu_all - cta + G - 1) / G : 0;   // units cta, cta+G, ...
@@ -612,6 +628,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         }
         if (ms->abort) break;
 
+        trace_mark(p, l, 3, clock64() - tl0);
         // h of every expert in use -> fp16 hi + lo table
         {
             ok = poll_words<8>(p.ll_h + (size_t)lpar * MAXU * I, nU * I, ep, err, [&](int i, float h) {
@@ -624,6 +641,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             if (cta_failed(ms, ok)) break;
         }
 
+        trace_mark(p, l, 4, clock64() - tl0);
         // down units: contiguous run [dn_lo, dn_hi) in (tile, expert) order
         float yacc = 0.f;   // warp 0, lane r < 16: running sum of output row r of the current tile
         for (int qi = 0; qi < n_dn_items; ++qi) {
@@ -706,6 +724,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             if (ms->abort) break;
         }
         if (ms->abort) break;
+        trace_mark(p, l, 5, clock64() - tl0);
     }
 
     // ---- outputs of the last layer ---------------------------------------------------
@@ -845,6 +864,20 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     if (ds.epoch < (uint32_t)L + 2) ds.epoch = 1;   // wrapped: never reuse 0 (initial contents)
     p.err = ctx->ws.dev_error;
     p.withhold = (c.flags & MOE_FLAG_TEST_WITHHOLD) ? 1 : 0;
+    if (c.flags & MOE_FLAG_TRACE) {
+        size_t need = (size_t)ds.grid * L * 8;
+        if (need > ds.trace_cap) {
+            if (ds.trace) ctx_free(ctx, ds.trace);
+            ds.trace = nullptr;
+            QE_CHECK(cudaSetDevice(ctx->device));
+            int s = ctx_alloc(ctx, (void **)&ds.trace, need * 8, "trace");
+            if (s != MOE_OK) return s;
+            ds.trace_cap = need;
+        }
+        QE_CHECK(cudaMemsetAsync(ds.trace, 0, need * 8, st));
+        ds.trace_n = (int)(ds.grid * L);
+        p.trace = ds.trace;
+    }
     p.nslot = ds.nslot;
     p.slot_bytes = ds.slot_bytes;
     p.rpc = ds.rpc;

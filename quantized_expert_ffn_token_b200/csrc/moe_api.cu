@@ -397,6 +397,18 @@ int moe_timing_read(moe_ctx *ctx, double *total_ms, long long *timed_launches,
     return MOE_OK;
 }
 
+int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int *n) {
+    if (!ctx || !n || (n_max > 0 && !out)) return MOE_ERR_INVALID_ARG;
+    QE_CHECK(cudaSetDevice(ctx->device));
+    QE_CHECK(cudaDeviceSynchronize());
+    int cnt = ctx->dec.trace ? ctx->dec.trace_n : 0;
+    if (cnt > n_max) cnt = n_max;
+    if (cnt > 0)
+        QE_CHECK(cudaMemcpy(out, ctx->dec.trace, (size_t)cnt * 8 * 8, cudaMemcpyDeviceToHost));
+    *n = cnt;
+    return MOE_OK;
+}
+
 const char *moe_status_string(int status) {
     switch (status) {
         case MOE_OK: return "ok";

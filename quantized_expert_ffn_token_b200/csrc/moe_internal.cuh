@@ -160,6 +160,9 @@ struct DecodeState {
         off_misc = 0, off_resid = 0;
     uint2 *ll = nullptr;  // flagged-word exchange buffers
     uint32_t epoch = 1;
+    unsigned long long *trace = nullptr;   // phase clocks (MOE_FLAG_TRACE)
+    size_t trace_cap = 0;                  // records allocated
+    int trace_n = 0;                       // records of the last call
 };
 
 // Event pairs around the dominant kernel (moe_timing_enable).
