@@ -80,8 +80,9 @@ struct DecodeParams {
     uint32_t epoch0;
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
-    unsigned long long *trace; // [G][L][8] phase clocks, or NULL
+    unsigned long long *trace; // [G][L][16] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
+    int dn_units_max;          // largest down-unit run of one CTA
     int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid;
 };
 
@@ -119,6 +120,9 @@ __device__ __forceinline__ void fence_proxy_async() {
 }
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void ll_store(uint2 *p, float v, uint32_t flag) {
     asm volatile("st.volatile.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(__float_as_uint(v)), "r"(flag)
@@ -256,7 +260,7 @@ __device__ __forceinline__ bool cta_failed(Misc *ms, bool mine_ok) {
 
 __device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph, long long t) {
     if (p.trace && threadIdx.x == 0) {
-        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * 8;
+        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * 16;
         if (ph == 0) {
             r[0] = blockIdx.x;
             r[1] = l;
@@ -558,17 +562,20 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 bx1[j] = act ? v1 : 0u;
             }
         }
+        long long tw_gu = 0, tw_dn = 0;   // cycles spent waiting for weights (trace)
 
-        // gate/up units
-        for (int q = 0; q < n_gu; ++q) {
-            long long it = item_base + q;
-            int s = (int)(it % p.nslot);
-            uint32_t parity = (uint32_t)((it / p.nslot) & 1);
-            ok = mbar_wait(&ms->full[s], parity, err, true);
-            if (cta_failed(ms, ok)) break;
-            const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
-            if (warp < GW) {
-                float D[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- gate/up: every warp with a k chunk walks all gate/up units of this CTA, waiting
+        // on each unit's barrier itself; partial sums go to red_gu[unit][warp][row]
+        if (warp < GW) {
+            for (int q = 0; q < n_gu && ok; ++q) {
+                long long it = item_base + q;
+                int s = (int)(it % p.nslot);
+                long long tw0 = clock64();
+                ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
+                tw_gu += clock64() - tw0;
+                if (!ok) break;
+                const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
+                float D0[4] = {0.f, 0.f, 0.f, 0.f}, D1[4] = {0.f, 0.f, 0.f, 0.f};
                 if (p.fmt == MOE_Q4B32) {
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq) {
@@ -578,7 +585,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                         for (int m = 0; m < 4; ++m) {
                             uint32_t a0, a1, a2, a3;
                             q4_frag(wv[m], a0, a1, a2, a3);
-                            mma16816(D, a0, a1, a2, a3, bx0[4 * kq + m], bx1[4 * kq + m]);
+                            mma16816((m & 1) ? D1 : D0, a0, a1, a2, a3, bx0[4 * kq + m], bx1[4 * kq + m]);
                         }
                     }
                 } else {
@@ -589,7 +596,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                         q3_frag(wp[0], wp[1], wp[2], rg);
 #pragma unroll
                         for (int m = 0; m < 4; ++m)
-                            mma16816(D, rg[4 * m], rg[4 * m + 1], rg[4 * m + 2], rg[4 * m + 3], bx0[4 * kq + m], bx1[4 * kq + m]);
+                            mma16816((m & 1) ? D1 : D0, rg[4 * m], rg[4 * m + 1], rg[4 * m + 2], rg[4 * m + 3],
+                                     bx0[4 * kq + m], bx1[4 * kq + m]);
                     }
                 }
                 // columns 2c, 2c+1 = blocks 8*warp + 2c, +1
@@ -597,38 +605,40 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 int b0 = 8 * warp + 2 * c;
                 float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + b0));
                 float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + b0));
-                float ag = fmaf(sg.x, D[0], sg.y * D[1]);
-                float a8 = fmaf(s8.x, D[2], s8.y * D[3]);
+                float ag = fmaf(sg.x, D0[0] + D1[0], sg.y * (D0[1] + D1[1]));
+                float a8 = fmaf(s8.x, D0[2] + D1[2], s8.y * (D0[3] + D1[3]));
                 ag += __shfl_xor_sync(0xffffffffu, ag, 1);
                 a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
                 ag += __shfl_xor_sync(0xffffffffu, ag, 2);
                 a8 += __shfl_xor_sync(0xffffffffu, a8, 2);
                 if (c == 0) {
-                    red[(par * NW + warp) * 16 + g] = ag;
-                    red[(par * NW + warp) * 16 + 8 + g] = a8;
+                    red[(q * NW + warp) * 16 + g] = ag;
+                    red[(q * NW + warp) * 16 + 8 + g] = a8;
                 }
             }
-            __syncthreads();
-            ++consumed;
-            if (tid == 0 && q + p.nslot < n_items) {
-                fence_proxy_async();
-                issue_item(q + p.nslot);
-            }
-            if (warp == 0 && lane < 8) {
-                float gs = 0.f, us_ = 0.f;
-                for (int w = 0; w < GW; ++w) {
-                    gs += red[(par * NW + w) * 16 + lane];
-                    us_ += red[(par * NW + w) * 16 + 8 + lane];
-                }
-                int u = cta + G * q;
-                int uslot = u / ntile_gu, t = u % ntile_gu;
-                ll_store(p.ll_h + ((size_t)lpar * MAXU + uslot) * I + 8 * t + lane, silu(gs) * us_, ep);
-            }
-            par ^= 1;
         }
-        if (ms->abort) break;
-
+        if (cta_failed(ms, ok)) break;
+        trace_mark(p, l, 6, clock64() - tl0);
+        consumed += n_gu;
+        // the gate/up slots are free: queue the down batches that did not fit the ring yet
+        if (tid == 0) {
+            fence_proxy_async();
+            for (int q = p.nslot; q < n_items && q < n_gu + p.nslot; ++q) issue_item(q);
+        }
+        // SwiGLU of every gate/up unit in parallel: thread (unit q, row i)
+        if (tid < n_gu * 8) {
+            int q = tid >> 3, i = tid & 7;
+            float gs = 0.f, us_ = 0.f;
+            for (int w = 0; w < GW; ++w) {
+                gs += red[(q * NW + w) * 16 + i];
+                us_ += red[(q * NW + w) * 16 + 8 + i];
+            }
+            int u = cta + G * q;
+            int uslot = u / ntile_gu, t = u % ntile_gu;
+            ll_store(p.ll_h + ((size_t)lpar * MAXU + uslot) * I + 8 * t + i, silu(gs) * us_, ep);
+        }
         trace_mark(p, l, 3, clock64() - tl0);
+
         // h of every expert in use -> fp16 hi + lo table
         {
             ok = poll_words<8>(p.ll_h + (size_t)lpar * MAXU * I, nU * I, ep, err, [&](int i, float h) {
@@ -640,24 +650,24 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             });
             if (cta_failed(ms, ok)) break;
         }
-
         trace_mark(p, l, 4, clock64() - tl0);
-        // down units: contiguous run [dn_lo, dn_hi) in (tile, expert) order
-        float yacc = 0.f;   // warp 0, lane r < 16: running sum of output row r of the current tile
-        for (int qi = 0; qi < n_dn_items; ++qi) {
-            int q = n_gu + qi;
-            long long it = item_base + q;
-            int s = (int)(it % p.nslot);
-            uint32_t parity = (uint32_t)((it / p.nslot) & 1);
-            ok = mbar_wait(&ms->full[s], parity, err, true);
-            if (cta_failed(ms, ok)) break;
-            int q0 = qi * dn_per_slot;
-            int cnt = min(dn_per_slot, n_dn - q0);
-            for (int ui = 0; ui < cnt; ++ui) {
-                int n = dn_lo + q0 + ui;
-                int j = n / nU, us = n % nU;
-                const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
-                if (warp < DW) {
+
+        // ---- down: every warp with a k group walks all down units of this CTA's contiguous
+        // run [dn_lo, dn_hi) ((tile, expert) order); partials to red[unit][warp][row]
+        if (warp < DW) {
+            for (int qi = 0; qi < n_dn_items && ok; ++qi) {
+                long long it = item_base + n_gu + qi;
+                int s = (int)(it % p.nslot);
+                long long tw0 = clock64();
+                ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
+                tw_dn += clock64() - tw0;
+                if (!ok) break;
+                int q0 = qi * dn_per_slot;
+                int cnt = min(dn_per_slot, n_dn - q0);
+                for (int ui = 0; ui < cnt; ++ui) {
+                    int nl = q0 + ui, n = dn_lo + nl;
+                    int us = n % nU;
+                    const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
                     float D[4] = {0.f, 0.f, 0.f, 0.f};
                     const __half *hp = htab + (size_t)(2 * us + (g & 1)) * I;
                     uint32_t a[16];
@@ -693,38 +703,42 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     ag += __shfl_xor_sync(0xffffffffu, ag, 2);
                     a8 += __shfl_xor_sync(0xffffffffu, a8, 2);
                     if (c == 0) {
-                        red[(par * NW + warp) * 16 + g] = ag;
-                        red[(par * NW + warp) * 16 + 8 + g] = a8;
+                        red[(nl * DW + warp) * 16 + g] = ag;
+                        red[(nl * DW + warp) * 16 + 8 + g] = a8;
                     }
                 }
-                __syncthreads();
-                if (ui == cnt - 1) {
-                    ++consumed;
-                    if (tid == 0 && q + p.nslot < n_items) {
-                        fence_proxy_async();
-                        issue_item(q + p.nslot);
-                    }
-                }
-                if (warp == 0 && lane < 16) {
-                    float v = 0.f;
-                    for (int w = 0; w < DW; ++w) v += red[(par * NW + w) * 16 + lane];
-                    yacc = fmaf(ms->uw[us], v, yacc);
-                    bool tile_end = (us == nU - 1) || (n == dn_hi - 1);
-                    if (tile_end) {
-                        int first = j * nU, last = j * nU + nU - 1;
-                        int part = (first >= dn_lo) ? 0 : 1;
-                        uint2 *yb = p.ll_y + (size_t)lpar * 2 * d;
-                        ll_store(yb + (size_t)part * d + 16 * j + lane, yacc, ep);
-                        if (part == 0 && last < dn_hi) ll_store(yb + d + 16 * j + lane, 0.f, ep);
-                        yacc = 0.f;
-                    }
-                }
-                par ^= 1;
             }
-            if (ms->abort) break;
         }
-        if (ms->abort) break;
+        if (cta_failed(ms, ok)) break;
+        consumed += n_dn_items;
+        trace_mark(p, l, 7, clock64() - tl0);
+        // unit sums (thread per (unit, row)), then per tile the fixed-order weighted sum
+        float *vsum = red + (size_t)p.dn_units_max * DW * 16;   // [unit][16]
+        for (int t = tid; t < n_dn * 16; t += NT) {
+            int nl = t >> 4, r = t & 15;
+            float v = 0.f;
+            for (int w = 0; w < DW; ++w) v += red[(nl * DW + w) * 16 + r];
+            vsum[t] = v;
+        }
+        __syncthreads();
+        {
+            int j_first = dn_lo / nU, j_last = (dn_hi - 1) / nU;
+            int n_tiles_mine = j_last - j_first + 1;
+            for (int t = tid; t < n_tiles_mine * 16; t += NT) {
+                int j = j_first + (t >> 4), r = t & 15;
+                int first = j * nU, last = j * nU + nU - 1;
+                int n0 = max(first, dn_lo), n1 = min(last, dn_hi - 1);
+                float y = 0.f;
+                for (int n = n0; n <= n1; ++n) y = fmaf(ms->uw[n % nU], vsum[(n - dn_lo) * 16 + r], y);
+                int part = (first >= dn_lo) ? 0 : 1;
+                uint2 *yb = p.ll_y + (size_t)lpar * 2 * d;
+                ll_store(yb + (size_t)part * d + 16 * j + r, y, ep);
+                if (part == 0 && last < dn_hi) ll_store(yb + d + 16 * j + r, 0.f, ep);
+            }
+        }
         trace_mark(p, l, 5, clock64() - tl0);
+        trace_mark(p, l, 10, tw_gu);
+        trace_mark(p, l, 12, tw_dn);
     }
 
     // ---- outputs of the last layer ---------------------------------------------------
@@ -793,8 +807,15 @@ int decode_setup(moe_ctx *ctx) {
         fixed = (fixed + bytes + 127) & ~(size_t)127;
         return off;
     };
-    size_t red_bytes = (size_t)2 * NW * 16 * 4;
-    if (red_bytes < (size_t)8 * NW * 4) red_bytes = (size_t)8 * NW * 4;
+    // per-CTA unit counts (gate/up round-robin, down contiguous runs)
+    int nU = c.top_k + c.n_shared;
+    int gu_max = (nU * (c.d_ff / 8) + G - 1) / G;
+    int dn_max = (nU * (c.d_model / 16) + G - 1) / G;
+    size_t red_bytes = (size_t)8 * NW * 4;                                   // router partials
+    if (red_bytes < (size_t)gu_max * NW * 16 * 4) red_bytes = (size_t)gu_max * NW * 16 * 4;
+    if (red_bytes < (size_t)dn_max * (NW + 1) * 16 * 4) red_bytes = (size_t)dn_max * (NW + 1) * 16 * 4;
+    ds.gu_units_max = gu_max;
+    ds.dn_units_max = dn_max;
     ds.off_router = take((size_t)rpc * c.d_model * 4);
     ds.off_x16 = take((size_t)c.d_model * 2);
     ds.off_logits = take((size_t)c.n_experts * 4);
@@ -807,7 +828,9 @@ int decode_setup(moe_ctx *ctx) {
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
-    if (nslot < 2) {
+    int dn_per_slot = slot / ctx->dn.tile_bytes;
+    // every gate/up tile of a layer and, after them, every down batch must fit the ring at once
+    if (nslot < 2 || gu_max > nslot || (dn_max + dn_per_slot - 1) / dn_per_slot > nslot) {
         ds.smem_bytes = 0;
         return MOE_OK;
     }
@@ -865,7 +888,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.err = ctx->ws.dev_error;
     p.withhold = (c.flags & MOE_FLAG_TEST_WITHHOLD) ? 1 : 0;
     if (c.flags & MOE_FLAG_TRACE) {
-        size_t need = (size_t)ds.grid * L * 8;
+        size_t need = (size_t)ds.grid * L * 16;
         if (need > ds.trace_cap) {
             if (ds.trace) ctx_free(ctx, ds.trace);
             ds.trace = nullptr;
@@ -881,6 +904,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.nslot = ds.nslot;
     p.slot_bytes = ds.slot_bytes;
     p.rpc = ds.rpc;
+    p.dn_units_max = ds.dn_units_max;
     p.off_ring = ds.off_ring;
     p.off_router = ds.off_router;
     p.off_x16 = ds.off_x16;

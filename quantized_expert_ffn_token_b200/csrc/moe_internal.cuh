@@ -156,6 +156,7 @@ struct DecodeState {
     int grid = 0;         // CTAs (one per SM)
     int smem_bytes = 0;   // 0: the shape does not fit the kernel
     int nslot = 0, slot_bytes = 0, rpc = 0;
+    int gu_units_max = 0, dn_units_max = 0;   // per-CTA unit counts the carve is sized for
     int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
         off_misc = 0, off_resid = 0;
     uint2 *ll = nullptr;  // flagged-word exchange buffers
