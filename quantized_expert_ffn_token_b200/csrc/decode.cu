@@ -38,6 +38,7 @@ namespace {
 
 constexpr int NT = 384;
 constexpr int NW = NT / 32;
+constexpr int PRODUCER = NT - 32;   // lane 0 of the last warp issues every bulk copy
 constexpr int MAX_SLOTS = 8;
 constexpr int MAXK = 32;
 constexpr int MAXU = MAXK + 4;
@@ -124,14 +125,18 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
+// A flagged word is one 64-bit value (low half: the float's bits, high half:
+// the epoch), stored and loaded as 64-bit elements so that a reader never sees
+// a new epoch with an old value.
 __device__ __forceinline__ void ll_store(uint2 *p, float v, uint32_t flag) {
-    asm volatile("st.volatile.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(__float_as_uint(v)), "r"(flag)
-                 : "memory");
+    unsigned long long w = ((unsigned long long)flag << 32) | __float_as_uint(v);
+    asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
-__device__ __forceinline__ uint2 ll_load(const uint2 *p) {
-    uint2 r;
-    asm volatile("ld.volatile.global.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p) : "memory");
-    return r;
+__device__ __forceinline__ void ll_load2(const uint2 *p, uint2 &a, uint2 &b) {
+    unsigned long long x, y;
+    asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "l"(p) : "memory");
+    a = make_uint2((uint32_t)x, (uint32_t)(x >> 32));
+    b = make_uint2((uint32_t)y, (uint32_t)(y >> 32));
 }
 __device__ __forceinline__ void mma16816(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -198,33 +203,33 @@ __device__ __forceinline__ float bf16_bits_f(uint16_t b) { return __uint_as_floa
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
 
-// Poll the flagged words base[i], i = tid + NT*j < n, with up to B loads of
-// this thread in flight at a time; put(i, value) receives each value once.
+// Poll the flagged words base[i], i < n (n even, base 16-byte aligned): this
+// thread owns the pairs (2q, 2q+1), q = tid + NT*j, and keeps up to B 16-byte
+// loads in flight; put(i, value) receives each value once.
 template <int B, typename F>
 __device__ __forceinline__ bool poll_words(const uint2 *base, int n, uint32_t flag, int *err, F &&put) {
     long long t0 = clock64();
-    for (int j0 = threadIdx.x; j0 < n; j0 += NT * B) {
-        bool need[B];
+    const int np = n >> 1;
+    for (int q0 = threadIdx.x; q0 < np; q0 += NT * B) {
+        uint32_t need = 0;   // bit 2b: word 2q of load b, bit 2b+1: word 2q+1
 #pragma unroll
-        for (int b = 0; b < B; ++b) need[b] = j0 + b * NT < n;
+        for (int b = 0; b < B; ++b)
+            if (q0 + b * NT < np) need |= 3u << (2 * b);
         for (int it = 0;; ++it) {
-            uint2 v[B];
+            uint2 v[2 * B];
 #pragma unroll
             for (int b = 0; b < B; ++b)
-                if (need[b]) v[b] = ll_load(base + j0 + b * NT);
-            bool all = true;
+                if (need & (3u << (2 * b))) ll_load2(base + 2 * (q0 + b * NT), v[2 * b], v[2 * b + 1]);
 #pragma unroll
-            for (int b = 0; b < B; ++b) {
-                if (need[b]) {
-                    if (v[b].y == flag) {
-                        put(j0 + b * NT, __uint_as_float(v[b].x));
-                        need[b] = false;
-                    } else {
-                        all = false;
+            for (int h = 0; h < 2 * B; ++h) {
+                if ((need >> h) & 1u) {
+                    if (v[h].y == flag) {
+                        put(2 * (q0 + (h >> 1) * NT) + (h & 1), __uint_as_float(v[h].x));
+                        need &= ~(1u << h);
                     }
                 }
             }
-            if (all) break;
+            if (!need) break;
             if ((it & 7) == 7) {
                 if (*(volatile int *)err != 0) return false;
                 if (clock64() - t0 > SPIN_LIMIT) {
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         for (int j = 0; j < nrows; ++j)
             bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
     };
-    if (tid == 0) issue_router(p.layer0);
+    if (tid == PRODUCER) issue_router(p.layer0);
 
     long long item = 0;                  // ring items planned so far (all layers)
     long long issued = 0;                // ring items whose copies were issued (thread 0)
@@ -334,8 +339,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             } else {
                 // previous layer's output = part 0 + part 1 of every row (same thread owns row i)
                 const uint2 *y0 = p.ll_y + (size_t)((l - 1) & 1) * 2 * d;
-                ok = poll_words<8>(y0, d, ep - 1, err, [&](int i, float v) { ybuf[i] = v; });
-                ok = ok && poll_words<8>(y0 + d, d, ep - 1, err, [&](int i, float v) {
+                ok = poll_words<4>(y0, d, ep - 1, err, [&](int i, float v) { ybuf[i] = v; });
+                ok = ok && poll_words<4>(y0 + d, d, ep - 1, err, [&](int i, float v) {
                     float y = ybuf[i] + v;
                     uint16_t yb = bf16_rn_bits(y);
                     rs[i] += bf16_bits_f(yb);
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 ll_store(p.ll_logits + (size_t)lpar * E + e, v + Lp.rb[e], ep);
             }
             __syncthreads();
-            if (tid == 0 && l + 1 < p.L) {
+            if (tid == PRODUCER && l + 1 < p.L) {
                 fence_proxy_async();
                 issue_router(layer + 1);
                 ++router_issued;
@@ -407,7 +412,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         trace_mark(p, l, 1, clock64() - tl0);
         // ---- 3. top-k on all logits (same result in every CTA) ------------------------
         {
-            ok = poll_words<3>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
+            ok = poll_words<2>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
             if (tid == 0) ms->ncand = 0;
             if (cta_failed(ms, ok)) break;
             // threshold: the k-th largest of the warps' maxima bounds the k-th largest logit from below
@@ -542,7 +547,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             }
             ++issued;
         };
-        if (tid == 0) {
+        if (tid == PRODUCER) {
             fence_proxy_async();
             int first = min(n_items, p.nslot);
             for (int q = 0; q < first; ++q) issue_item(q);
@@ -621,7 +626,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         trace_mark(p, l, 6, clock64() - tl0);
         consumed += n_gu;
         // the gate/up slots are free: queue the down batches that did not fit the ring yet
-        if (tid == 0) {
+        if (tid == PRODUCER) {
             fence_proxy_async();
             for (int q = p.nslot; q < n_items && q < n_gu + p.nslot; ++q) issue_item(q);
         }
@@ -747,8 +752,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         const uint32_t ep = p.epoch0 + (uint32_t)l;
         const uint2 *y0 = p.ll_y + (size_t)(l & 1) * 2 * d;
         if (cta == 0) {
-            ok = poll_words<8>(y0, d, ep, err, [&](int i, float v) { ybuf[i] = v; });
-            ok = ok && poll_words<8>(y0 + d, d, ep, err, [&](int i, float v) {
+            ok = poll_words<4>(y0, d, ep, err, [&](int i, float v) { ybuf[i] = v; });
+            ok = ok && poll_words<4>(y0 + d, d, ep, err, [&](int i, float v) {
                 float y = ybuf[i] + v;
                 uint16_t yb = bf16_rn_bits(y);
                 if (p.stack) {
@@ -765,7 +770,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         }
     }
     // drain copies still in flight (abort path) before the CTA's shared memory goes away
-    if (tid == 0) {
+    if (tid == PRODUCER) {
         for (long long it = consumed; it < issued; ++it)
             mbar_wait(&ms->full[(int)(it % p.nslot)], (uint32_t)((it / p.nslot) & 1), err, false);
         if (router_issued > router_waited)
@@ -779,6 +784,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 bool decode_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
     if (T != 1 || (c.flags & MOE_FLAG_NO_DECODE_KERNEL)) return false;
+    if (c.n_experts % 2) return false;   // flagged words are polled in 16-byte pairs
     if (c.d_model > 4096 || c.d_model / 256 > NW || c.d_ff / 64 > NW) return false;
     if (c.top_k > MAXK || c.top_k + c.n_shared > MAXU) return false;
     return ctx->dec.smem_bytes > 0;
