@@ -182,12 +182,11 @@ MOE_API int moe_timing_read(moe_ctx *ctx, double *total_ms, long long *timed_lau
 
 /* Phase trace of the last persistent-kernel call (context created with
  * MOE_FLAG_TRACE).  Copies up to n_max records into out (host memory) and
- * returns their number in *n.  One record = 16 uint64: CTA index, layer,
- * then SM clock cycles since the start of that layer in that CTA at: the end
- * of each of the six phases (input ready, router published, routing known,
- * gate/up done, h ready, down done), the arrival of the first and of the
- * last gate/up weight tile, and of the first and last down weight batch;
- * the rest is zero.  Synchronises the device. */
+ * returns their number in *n.  One record = 24 uint64: CTA index, layer,
+ * then 22 slots of SM clock cycles since the start of that layer in that CTA
+ * (phase ends and waits; the slot map is documented next to the kernel's
+ * trace marks).  The caller's buffer must hold 24 * n_max values.
+ * Synchronises the device. */
 MOE_API int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int *n);
 
 /* Static text for a status code. */

@@ -182,11 +182,11 @@ def moe_timing_read(ctx) -> dict:
 
 
 def moe_trace_read(ctx, n_max: int = 1 << 16):
-    """Phase trace records as a list of 16-tuples (see include/moe.h)."""
-    buf = (ctypes.c_ulonglong * (16 * n_max))()
+    """Phase trace records as a list of 24-tuples (see include/moe.h)."""
+    buf = (ctypes.c_ulonglong * (24 * n_max))()
     n = ctypes.c_int(0)
     _check(lib.moe_trace_read(ctx, buf, n_max, ctypes.byref(n)), "moe_trace_read")
-    return [tuple(buf[16 * i:16 * i + 16]) for i in range(n.value)]
+    return [tuple(buf[24 * i:24 * i + 24]) for i in range(n.value)]
 
 
 def make_record(x=None, y=None, y_f32=None, ids=None, w=None, rows=None) -> moe_stack_record:

@@ -81,7 +81,7 @@ struct DecodeParams {
     uint32_t epoch0;
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
-    unsigned long long *trace; // [G][L][16] phase clocks, or NULL
+    unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int dn_units_max;          // largest down-unit run of one CTA
     int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid;
@@ -263,9 +263,11 @@ __device__ __forceinline__ bool cta_failed(Misc *ms, bool mine_ok) {
     return ms->abort != 0;
 }
 
+constexpr int TRACE_WORDS = 24;   // per (CTA, layer) record: CTA, layer, 22 timestamps
+
 __device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph, long long t) {
-    if (p.trace && threadIdx.x == 0) {
-        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * 16;
+    if (p.trace && threadIdx.x == 0 && ph < TRACE_WORDS - 2) {
+        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * TRACE_WORDS;
         if (ph == 0) {
             r[0] = blockIdx.x;
             r[1] = l;
@@ -351,6 +353,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 });
                 if (cta_failed(ms, ok)) break;
             }
+            trace_mark(p, l, 13, clock64() - tl0);
             float ss = 0.f;
             for (int i = tid; i < d; i += NT) ss = fmaf(rs[i], rs[i], ss);
             for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -375,6 +378,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             ok = mbar_wait(&ms->rbar, (uint32_t)(l & 1), err, true);
             if (cta_failed(ms, ok)) break;
             ++router_waited;
+            trace_mark(p, l, 14, clock64() - tl0);
             int nrows = 0;
             for (int j = 0; j < p.rpc; ++j)
                 if (cta + G * j < E) ++nrows;
@@ -395,6 +399,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 if (lane == 0) red[j * NW + warp] = v;
             }
             __syncthreads();
+            trace_mark(p, l, 15, clock64() - tl0);
             if (tid < nrows && !(p.withhold && cta == 0)) {
                 float v = 0.f;
                 for (int w = 0; w < NW; ++w) v += red[tid * NW + w];
@@ -415,6 +420,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             ok = poll_words<2>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
             if (tid == 0) ms->ncand = 0;
             if (cta_failed(ms, ok)) break;
+            trace_mark(p, l, 8, clock64() - tl0);
             // threshold: the k-th largest of the warps' maxima bounds the k-th largest logit from below
             float m = -INFINITY;
             for (int e = tid; e < E; e += NT) m = fmaxf(m, lg[e]);
@@ -482,6 +488,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 }
             }
             __syncthreads();
+            trace_mark(p, l, 9, clock64() - tl0);
             if (warp == 0) {
                 float top = ms->vsel[0];
                 float pj = lane < k ? expf(ms->vsel[lane] - top) : 0.f;
@@ -894,7 +901,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.err = ctx->ws.dev_error;
     p.withhold = (c.flags & MOE_FLAG_TEST_WITHHOLD) ? 1 : 0;
     if (c.flags & MOE_FLAG_TRACE) {
-        size_t need = (size_t)ds.grid * L * 16;
+        size_t need = (size_t)ds.grid * L * TRACE_WORDS;
         if (need > ds.trace_cap) {
             if (ds.trace) ctx_free(ctx, ds.trace);
             ds.trace = nullptr;
@@ -905,6 +912,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
         }
         QE_CHECK(cudaMemsetAsync(ds.trace, 0, need * 8, st));
         ds.trace_n = (int)(ds.grid * L);
+        ds.trace_words = TRACE_WORDS;
         p.trace = ds.trace;
     }
     p.nslot = ds.nslot;

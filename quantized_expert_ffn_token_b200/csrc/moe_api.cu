@@ -404,7 +404,7 @@ int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int *n) {
     int cnt = ctx->dec.trace ? ctx->dec.trace_n : 0;
     if (cnt > n_max) cnt = n_max;
     if (cnt > 0)
-        QE_CHECK(cudaMemcpy(out, ctx->dec.trace, (size_t)cnt * 16 * 8, cudaMemcpyDeviceToHost));
+        QE_CHECK(cudaMemcpy(out, ctx->dec.trace, (size_t)cnt * ctx->dec.trace_words * 8, cudaMemcpyDeviceToHost));
     *n = cnt;
     return MOE_OK;
 }

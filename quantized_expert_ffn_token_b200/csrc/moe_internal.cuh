@@ -164,6 +164,7 @@ struct DecodeState {
     unsigned long long *trace = nullptr;   // phase clocks (MOE_FLAG_TRACE)
     size_t trace_cap = 0;                  // records allocated
     int trace_n = 0;                       // records of the last call
+    int trace_words = 24;                  // uint64 per record
 };
 
 // Event pairs around the dominant kernel (moe_timing_enable).
