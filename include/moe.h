@@ -189,6 +189,29 @@ MOE_API int moe_timing_read(moe_ctx *ctx, double *total_ms, long long *timed_lau
  * Synchronises the device. */
 MOE_API int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int *n);
 
+/* Routing without any device allocation.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory (code
+ * running inside another runtime's memory pool, services that forbid device
+ * allocation after start-up, plain C hosts that only receive device
+ * pointers).  It computes the router logits of T tokens and their softmax
+ * top-k exactly as moe_forward does, from caller-owned device buffers:
+ *   x_bf16 [T][d_model] bf16, router_w [n_experts][d_model] fp32,
+ *   router_bias [n_experts] fp32 or NULL; outputs ids [T][top_k] int32 and
+ *   w [T][top_k] fp32 (descending weight, equal logits -> lower id).
+ * The logits live in a fixed array in device memory that the library holds
+ * on every device that loads it, until the process exits:
+ * T * n_experts must not exceed MOE_ROUTE_STATIC_MAX_LOGITS
+ * (MOE_ERR_TOO_MANY_TOKENS otherwise, with a message in moe_last_error()).
+ * The first call on a device looks up that array's device address (make it
+ * before any stream capture on that device).  Calls share the array: calls
+ * that overlap on the GPU (other streams, other host threads) race; order
+ * them on one stream.  Asynchronous on `stream`; calls no allocating routine.
+ * Errors: INVALID_ARG, TOO_MANY_TOKENS, UNSUPPORTED (device index >= 64), CUDA. */
+#define MOE_ROUTE_STATIC_MAX_LOGITS 65536
+MOE_API int moe_route_static(const uint16_t *x_bf16, int T, int d_model, const float *router_w,
+                             const float *router_bias, int n_experts, int top_k, int32_t *ids,
+                             float *w, void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

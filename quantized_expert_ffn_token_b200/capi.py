@@ -29,13 +29,14 @@ MOE_FLAG_NO_DECODE_KERNEL = 1
 MOE_FLAG_NO_TENSOR_PREFILL = 2
 MOE_FLAG_TEST_WITHHOLD = 256
 MOE_FLAG_TRACE = 4
+MOE_ROUTE_STATIC_MAX_LOGITS = 65536
 FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32}
 
 EXPORTED = [
     "moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
     "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
     "moe_status_string", "moe_last_error", "moe_timing_enable", "moe_timing_read",
-    "moe_trace_read",
+    "moe_trace_read", "moe_route_static",
 ]
 
 
@@ -82,13 +83,14 @@ def _load() -> ctypes.CDLL:
     L.moe_timing_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
                                   ctypes.POINTER(ctypes.c_longlong), ctypes.c_char_p, i]
     L.moe_trace_read.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong), i, ctypes.POINTER(i)]
+    L.moe_route_static.argtypes = [vp, i, i, vp, vp, i, i, vp, vp, vp]
     L.moe_status_string.argtypes = [i]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_error.argtypes = []
     L.moe_last_error.restype = ctypes.c_char_p
     for n in ("moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
               "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
-              "moe_timing_enable", "moe_timing_read", "moe_trace_read"):
+              "moe_timing_enable", "moe_timing_read", "moe_trace_read", "moe_route_static"):
         getattr(L, n).restype = i
     return L
 
@@ -187,6 +189,13 @@ def moe_trace_read(ctx, n_max: int = 1 << 16):
     n = ctypes.c_int(0)
     _check(lib.moe_trace_read(ctx, buf, n_max, ctypes.byref(n)), "moe_trace_read")
     return [tuple(buf[24 * i:24 * i + 24]) for i in range(n.value)]
+
+
+def moe_route_static(x, T: int, d_model: int, router_w, router_bias, n_experts: int, top_k: int,
+                     ids, w, stream=None) -> None:
+    """Allocation-free routing (see include/moe.h): device buffers in, ids/w out."""
+    _check(lib.moe_route_static(_ptr(x), T, d_model, _ptr(router_w), _ptr(router_bias), n_experts,
+                                top_k, _ptr(ids), _ptr(w), _stream(stream)), "moe_route_static")
 
 
 def make_record(x=None, y=None, y_f32=None, ids=None, w=None, rows=None) -> moe_stack_record:

@@ -45,6 +45,11 @@ int set_oom(const char *what) {
     return MOE_ERR_OOM;
 }
 
+int set_too_many(const char *what) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+    return MOE_ERR_TOO_MANY_TOKENS;
+}
+
 int ctx_alloc(moe_ctx *ctx, void **p, size_t bytes, const char *what) {
     *p = nullptr;
     if (bytes == 0) bytes = 16;

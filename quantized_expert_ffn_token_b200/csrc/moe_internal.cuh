@@ -198,6 +198,7 @@ namespace qeffn {
 // Status plumbing (moe_api.cu)
 int set_cuda_error(cudaError_t e, const char *what);
 int set_oom(const char *what);
+int set_too_many(const char *what);
 int ctx_alloc(moe_ctx *ctx, void **p, size_t bytes, const char *what);
 void ctx_free(moe_ctx *ctx, void *p);
 
@@ -228,6 +229,8 @@ int launch_router_simt(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, i
 int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, float *w,
                 cudaStream_t st);
 int launch_dispatch(moe_ctx *ctx, const int32_t *ids, int T, cudaStream_t st);
+int launch_route_raw(const uint16_t *x, int T, int d, int E, int k, const float *W, const float *b,
+                     float *logits, int32_t *ids, float *w, cudaStream_t st);
 int launch_experts_simt(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
                         cudaStream_t st);
 int launch_combine(const moe_ctx *ctx, int T, const float *w, uint16_t *y, float *yf,

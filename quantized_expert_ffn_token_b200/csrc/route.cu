@@ -215,6 +215,20 @@ int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, fl
     return MOE_OK;
 }
 
+// Router + top-k on caller-provided pointers (no context): used by the
+// allocation-free routing entry point in route_static.cu.
+int launch_route_raw(const uint16_t *x, int T, int d, int E, int k, const float *W, const float *b,
+                     float *logits, int32_t *ids, float *w, cudaStream_t st) {
+    // same opt-in size as launch_router_simt, so neither caller shrinks it for the other
+    QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    dim3 grid((E + RT_EXP - 1) / RT_EXP, (T + RT_TOK - 1) / RT_TOK);
+    k_router_simt<<<grid, 256, (size_t)RT_TOK * d * sizeof(float), st>>>(x, T, d, E, W, b, logits);
+    QE_CHECK_LAUNCH("k_router_simt");
+    k_topk<<<(T + 7) / 8, 256, 8 * (size_t)E * sizeof(float), st>>>(logits, T, E, k, ids, w);
+    QE_CHECK_LAUNCH("k_topk");
+    return MOE_OK;
+}
+
 int launch_dispatch(moe_ctx *ctx, const int32_t *ids, int T, cudaStream_t st) {
     const moe_config &c = ctx->cfg;
     Workspace &ws = ctx->ws;
