@@ -84,7 +84,7 @@ struct DecodeParams {
     unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int dn_units_max;          // largest down-unit run of one CTA
-    int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid;
+    int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid, off_sums;
 };
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -122,9 +122,6 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
 // A flagged word is one 64-bit value (low half: the float's bits, high half:
 // the epoch), stored and loaded as 64-bit elements so that a reader never sees
 // a new epoch with an old value.
@@ -140,39 +137,26 @@ __device__ __forceinline__ void ll_load2(const uint2 *p, uint2 &a, uint2 &b) {
 }
 __device__ __forceinline__ void mma16816(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t r;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-
-// fp16x2 constants.  A code field OR-ed under the exponent of 1024.0
-// (0x6400) reads as 1024 + F*q for a field starting at bit log2(F); one fp16
-// FMA with 1/F and -(1024/F + zero) gives q - zero exactly.
-constexpr uint32_t H_MAGIC = 0x64006400u;
-constexpr uint32_t H_ONE = 0x3C003C00u;       // 1
-constexpr uint32_t H_SIXTEENTH = 0x2C002C00u; // 1/16
-constexpr uint32_t H_EIGHTH = 0x30003000u;    // 1/8
-constexpr uint32_t H_64TH = 0x24002400u;      // 1/64
-constexpr uint32_t H_M1032 = 0xE408E408u;     // -1032 = -(1024 + 8)
-constexpr uint32_t H_M72 = 0xD480D480u;       // -72   = -(64 + 8)
-constexpr uint32_t H_M1028 = 0xE404E404u;     // -1028 = -(1024 + 4)
-constexpr uint32_t H_M132 = 0xD820D820u;      // -132  = -(128 + 4)
-constexpr uint32_t H_M20 = 0xCD00CD00u;       // -20   = -(16 + 4)
+// Code -> bf16 without arithmetic: a field OR-ed into the low mantissa bits of
+// 128.0 (0x4300) reads as 128 + q, exactly.  The offset is removed in fp32
+// from each 32-block's partial sum: sum_k (128 + q_k) v_k - (128 + zero) *
+// sum_k v_k = sum_k (q_k - zero) v_k, with the block sums of the activations
+// precomputed once per layer (cancellation costs about 7 bits of the fp32
+// partial, far below the output tolerance).
+constexpr uint32_t BF_MAGIC = 0x43004300u;
 
 // Q4B32: one word = the 8 codes of one k16 slice (nibble n = reg + 4*hi).
 __device__ __forceinline__ void q4_frag(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2,
                                         uint32_t &a3) {
-    uint32_t w8 = w >> 8;
-    a0 = hfma2((w & 0x000F000Fu) | H_MAGIC, H_ONE, H_M1032);
-    a1 = hfma2((w & 0x00F000F0u) | H_MAGIC, H_SIXTEENTH, H_M72);
-    a2 = hfma2((w8 & 0x000F000Fu) | H_MAGIC, H_ONE, H_M1032);
-    a3 = hfma2((w8 & 0x00F000F0u) | H_MAGIC, H_SIXTEENTH, H_M72);
+    a0 = (w & 0x000F000Fu) | BF_MAGIC;
+    a1 = ((w >> 4) & 0x000F000Fu) | BF_MAGIC;
+    a2 = ((w >> 8) & 0x000F000Fu) | BF_MAGIC;
+    a3 = ((w >> 12) & 0x000F000Fu) | BF_MAGIC;
 }
 
 // Q3B32: three words = the 16 fragment registers of four k16 slices.
@@ -180,15 +164,11 @@ __device__ __forceinline__ void q3_frag(uint32_t w0, uint32_t w1, uint32_t w2, u
     uint32_t ws[3] = {w0, w1, w2};
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
-        uint32_t w = ws[j], w9 = ws[j] >> 9;
-        r[5 * j + 0] = hfma2((w & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
-        r[5 * j + 1] = hfma2((w & 0x00380038u) | H_MAGIC, H_EIGHTH, H_M132);
-        r[5 * j + 2] = hfma2((w & 0x01C001C0u) | H_MAGIC, H_64TH, H_M20);
-        r[5 * j + 3] = hfma2((w9 & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
-        r[5 * j + 4] = hfma2((w9 & 0x00380038u) | H_MAGIC, H_EIGHTH, H_M132);
+#pragma unroll
+        for (int f = 0; f < 5; ++f) r[5 * j + f] = ((ws[j] >> (3 * f)) & 0x00070007u) | BF_MAGIC;
     }
-    uint32_t s = ((w0 >> 15) & 0x00010001u) | ((w1 >> 14) & 0x00020002u) | ((w2 >> 13) & 0x00040004u);
-    r[15] = hfma2(s | H_MAGIC, H_ONE, H_M1028);
+    uint32_t t = ((w0 >> 15) & 0x00010001u) | ((w1 >> 14) & 0x00020002u) | ((w2 >> 13) & 0x00040004u);
+    r[15] = t | BF_MAGIC;
 }
 
 __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
@@ -280,9 +260,11 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *ring = smem + p.off_ring;
     float *rtr = reinterpret_cast<float *>(smem + p.off_router);
-    __half *x16 = reinterpret_cast<__half *>(smem + p.off_x16);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_x16);         // layer input, bf16 bits
+    float *xsum = reinterpret_cast<float *>(smem + p.off_sums);              // [d/32] block sums of x
+    float *hsum = xsum + p.d / 32;                                             // [nU][I/32] of h hi + lo
     float *lg = reinterpret_cast<float *>(smem + p.off_logits);
-    __half *htab = reinterpret_cast<__half *>(smem + p.off_htab);
+    uint16_t *htab = reinterpret_cast<uint16_t *>(smem + p.off_htab);   // bf16 hi / lo of h
     float *red = reinterpret_cast<float *>(smem + p.off_red);   // [2][NW][16]
     Misc *ms = reinterpret_cast<Misc *>(smem + p.off_misc);
     float *rs = reinterpret_cast<float *>(smem + p.off_resid);      // residual stream [d]
@@ -298,6 +280,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     const int GW = d / 256;              // warps with a gate/up K chunk (256 k each)
     const int DW = I / 64;               // warps with a down k group (64 k each)
     const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
+    const float off = (p.fmt == MOE_Q4B32) ? 136.f : 132.f;   // 128 + zero point
     int *err = p.err;
 
     if (tid == 0) {
@@ -324,7 +307,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     long long issued = 0;                // ring items whose copies were issued (thread 0)
     long long consumed = 0;              // ring items consumed so far
     int router_issued = 1, router_waited = 0;   // router prefetch fills (thread 0) / waits
-    int par = 0;
     bool ok = true;
 
     for (int l = 0; l < p.L; ++l) {
@@ -363,14 +345,20 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             for (int w = 0; w < NW; ++w) tot += ms->red1[w];
             float inv = 1.f / sqrtf(tot / (float)d + 1e-6f);
             for (int i = tid; i < d; i += NT) {
-                uint16_t xb = bf16_rn_bits(rs[i] * inv);
-                x16[i] = __float2half_rn(bf16_bits_f(xb));
-                if (cta == 0 && p.rec_on && p.rec.x_bf16) p.rec.x_bf16[(size_t)l * d + i] = xb;
+                uint16_t xv = bf16_rn_bits(rs[i] * inv);
+                xb[i] = xv;
+                if (cta == 0 && p.rec_on && p.rec.x_bf16) p.rec.x_bf16[(size_t)l * d + i] = xv;
             }
         } else {
-            for (int i = tid; i < d; i += NT) x16[i] = __float2half_rn(bf16_bits_f(p.x_in[i]));
+            for (int i = tid; i < d; i += NT) xb[i] = p.x_in[i];
         }
         __syncthreads();
+        // block sums of the input (offset removal in the gate/up flush)
+        for (int b = tid; b < nbd; b += NT) {
+            float sacc = 0.f;
+            for (int j = 0; j < 32; ++j) sacc += bf16_bits_f(xb[32 * b + j]);
+            xsum[b] = sacc;
+        }
 
         trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
@@ -387,7 +375,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) part[j] = 0.f;
             for (int i = tid; i < d; i += NT) {
-                float xv = __half2float(x16[i]);
+                float xv = bf16_bits_f(xb[i]);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     if (j < nrows) part[j] = fmaf(rtr[(size_t)j * d + i], xv, part[j]);
@@ -568,8 +556,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             for (int j = 0; j < 16; ++j) {
                 int s = 16 * warp + j;
                 bool act = (g == (j >> 1));
-                uint32_t v0 = *reinterpret_cast<const uint32_t *>(x16 + 16 * s + 2 * c);
-                uint32_t v1 = *reinterpret_cast<const uint32_t *>(x16 + 16 * s + 2 * c + 8);
+                uint32_t v0 = *reinterpret_cast<const uint32_t *>(xb + 16 * s + 2 * c);
+                uint32_t v1 = *reinterpret_cast<const uint32_t *>(xb + 16 * s + 2 * c + 8);
                 bx0[j] = act ? v0 : 0u;
                 bx1[j] = act ? v1 : 0u;
             }
@@ -617,8 +605,9 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 int b0 = 8 * warp + 2 * c;
                 float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + b0));
                 float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + b0));
-                float ag = fmaf(sg.x, D0[0] + D1[0], sg.y * (D0[1] + D1[1]));
-                float a8 = fmaf(s8.x, D0[2] + D1[2], s8.y * (D0[3] + D1[3]));
+                const float o0 = off * xsum[b0], o1 = off * xsum[b0 + 1];
+                float ag = fmaf(sg.x, D0[0] + D1[0] - o0, sg.y * (D0[1] + D1[1] - o1));
+                float a8 = fmaf(s8.x, D0[2] + D1[2] - o0, s8.y * (D0[3] + D1[3] - o1));
                 ag += __shfl_xor_sync(0xffffffffu, ag, 1);
                 a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
                 ag += __shfl_xor_sync(0xffffffffu, ag, 2);
@@ -654,13 +643,22 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         // h of every expert in use -> fp16 hi + lo table
         {
             ok = poll_words<8>(p.ll_h + (size_t)lpar * MAXU * I, nU * I, ep, err, [&](int i, float h) {
-                __half hi = __float2half_rn(h);
-                __half lo = __float2half_rn(h - __half2float(hi));
+                uint16_t hi = bf16_rn_bits(h);
+                uint16_t lo = bf16_rn_bits(h - bf16_bits_f(hi));
                 int us = i / I, kk = i % I;
                 htab[(size_t)(2 * us) * I + kk] = hi;
                 htab[(size_t)(2 * us + 1) * I + kk] = lo;
             });
             if (cta_failed(ms, ok)) break;
+            for (int t = tid; t < nU * nbi; t += NT) {
+                int us = t / nbi, b = t % nbi;
+                const uint16_t *hh = htab + (size_t)(2 * us) * I + 32 * b;
+                const uint16_t *hl = htab + (size_t)(2 * us + 1) * I + 32 * b;
+                float sacc = 0.f;
+                for (int j = 0; j < 32; ++j) sacc += bf16_bits_f(hh[j]) + bf16_bits_f(hl[j]);
+                hsum[t] = sacc;
+            }
+            __syncthreads();
         }
         trace_mark(p, l, 4, clock64() - tl0);
 
@@ -681,7 +679,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     int us = n % nU;
                     const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
                     float D[4] = {0.f, 0.f, 0.f, 0.f};
-                    const __half *hp = htab + (size_t)(2 * us + (g & 1)) * I;
+                    const uint16_t *hp = htab + (size_t)(2 * us + (g & 1)) * I;
                     uint32_t a[16];
                     if (p.fmt == MOE_Q4B32) {
                         uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)warp * 512 + lane * 16);
@@ -707,8 +705,9 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     float ag = 0.f, a8 = 0.f;
                     if (valid) {
                         const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
-                        ag = __half2float(sc[g * nbi + blk]) * (D[0] + D[1]);
-                        a8 = __half2float(sc[(g + 8) * nbi + blk]) * (D[2] + D[3]);
+                        const float o = off * hsum[us * nbi + blk];
+                        ag = __half2float(sc[g * nbi + blk]) * (D[0] + D[1] - o);
+                        a8 = __half2float(sc[(g + 8) * nbi + blk]) * (D[2] + D[3] - o);
                     }
                     ag += __shfl_xor_sync(0xffffffffu, ag, 1);
                     a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
@@ -838,6 +837,7 @@ int decode_setup(moe_ctx *ctx) {
     ds.off_red = take(red_bytes);
     ds.off_misc = take(sizeof(Misc));
     ds.off_resid = take((size_t)c.d_model * 4);
+    ds.off_sums = take((size_t)(c.d_model / 32 + nU * (c.d_ff / 32)) * 4);
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
@@ -927,6 +927,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_red = ds.off_red;
     p.off_misc = ds.off_misc;
     p.off_resid = ds.off_resid;
+    p.off_sums = ds.off_sums;
     void *args[] = {&p};
     QE_CHECK(cudaLaunchCooperativeKernel((void *)k_decode, dim3(ds.grid), dim3(NT), args,
                                          (size_t)ds.smem_bytes, st));

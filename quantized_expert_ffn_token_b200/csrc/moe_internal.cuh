@@ -158,7 +158,7 @@ struct DecodeState {
     int nslot = 0, slot_bytes = 0, rpc = 0;
     int gu_units_max = 0, dn_units_max = 0;   // per-CTA unit counts the carve is sized for
     int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
-        off_misc = 0, off_resid = 0;
+        off_misc = 0, off_resid = 0, off_sums = 0;
     uint2 *ll = nullptr;  // flagged-word exchange buffers
     uint32_t epoch = 1;
     unsigned long long *trace = nullptr;   // phase clocks (MOE_FLAG_TRACE)
