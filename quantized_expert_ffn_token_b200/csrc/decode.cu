@@ -183,6 +183,20 @@ __device__ __forceinline__ float bf16_bits_f(uint16_t b) { return __uint_as_floa
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
 
+// Sum of 32 consecutive bf16 values (16-byte aligned) with four 16-byte loads.
+__device__ __forceinline__ float sum32_bf16(const uint16_t *p) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 v = q[j];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) acc[h] += __uint_as_float(w[h] << 16) + __uint_as_float(w[h] & 0xFFFF0000u);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // Poll the flagged words base[i], i < n (n even, base 16-byte aligned): this
 // thread owns the pairs (2q, 2q+1), q = tid + NT*j, and keeps up to B 16-byte
 // loads in flight; put(i, value) receives each value once.
@@ -222,7 +236,7 @@ __device__ __forceinline__ bool poll_words(const uint2 *base, int n, uint32_t fl
     return true;
 }
 
-__device__ __noinline__ bool mbar_wait(unsigned long long *b, uint32_t parity, int *err, bool honor_err) {
+__device__ __forceinline__ bool mbar_wait(unsigned long long *b, uint32_t parity, int *err, bool honor_err) {
     long long t0 = clock64();
     for (int it = 0;; ++it) {
         if (mbar_try_wait(b, parity)) return true;
@@ -256,6 +270,7 @@ __device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph,
     }
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *ring = smem + p.off_ring;
@@ -280,7 +295,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     const int GW = d / 256;              // warps with a gate/up K chunk (256 k each)
     const int DW = I / 64;               // warps with a down k group (64 k each)
     const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
-    const float off = (p.fmt == MOE_Q4B32) ? 136.f : 132.f;   // 128 + zero point
+    constexpr float off = (FMT == MOE_Q4B32) ? 136.f : 132.f;   // 128 + zero point
     int *err = p.err;
 
     if (tid == 0) {
@@ -318,8 +333,13 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 
         // ---- 1. layer input -------------------------------------------------------
         if (p.stack) {
+            float ss = 0.f;   // this thread's share of sum(r^2)
             if (l == 0) {
-                for (int i = tid; i < d; i += NT) rs[i] = bf16_bits_f(p.x_in[i]);
+                for (int i = tid; i < d; i += NT) {
+                    float v = bf16_bits_f(p.x_in[i]);
+                    rs[i] = v;
+                    ss = fmaf(v, v, ss);
+                }
             } else {
                 // previous layer's output = part 0 + part 1 of every row (same thread owns row i)
                 const uint2 *y0 = p.ll_y + (size_t)((l - 1) & 1) * 2 * d;
@@ -327,7 +347,9 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 ok = ok && poll_words<4>(y0 + d, d, ep - 1, err, [&](int i, float v) {
                     float y = ybuf[i] + v;
                     uint16_t yb = bf16_rn_bits(y);
-                    rs[i] += bf16_bits_f(yb);
+                    float rn = rs[i] + bf16_bits_f(yb);
+                    rs[i] = rn;
+                    ss = fmaf(rn, rn, ss);
                     if (cta == 0 && p.rec_on) {
                         if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
                         if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
@@ -336,8 +358,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 if (cta_failed(ms, ok)) break;
             }
             trace_mark(p, l, 13, clock64() - tl0);
-            float ss = 0.f;
-            for (int i = tid; i < d; i += NT) ss = fmaf(rs[i], rs[i], ss);
             for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
             if (lane == 0) ms->red1[warp] = ss;
             __syncthreads();
@@ -354,11 +374,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         }
         __syncthreads();
         // block sums of the input (offset removal in the gate/up flush)
-        for (int b = tid; b < nbd; b += NT) {
-            float sacc = 0.f;
-            for (int j = 0; j < 32; ++j) sacc += bf16_bits_f(xb[32 * b + j]);
-            xsum[b] = sacc;
-        }
+        for (int b = tid; b < nbd; b += NT) xsum[b] = sum32_bf16(xb + 32 * b);
 
         trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
@@ -370,21 +386,29 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             int nrows = 0;
             for (int j = 0; j < p.rpc; ++j)
                 if (cta + G * j < E) ++nrows;
-            // warp w sums its strided share of k for every row
+            // thread sums its strided share of 4-wide k chunks for every live row
             float part[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) part[j] = 0.f;
-            for (int i = tid; i < d; i += NT) {
-                float xv = bf16_bits_f(xb[i]);
+            for (int i4 = tid; i4 < d / 4; i4 += NT) {
+                uint2 xv2 = *reinterpret_cast<const uint2 *>(xb + 4 * i4);
+                float x0 = __uint_as_float(xv2.x << 16), x1 = __uint_as_float(xv2.x & 0xFFFF0000u);
+                float x2 = __uint_as_float(xv2.y << 16), x3 = __uint_as_float(xv2.y & 0xFFFF0000u);
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (j < nrows) part[j] = fmaf(rtr[(size_t)j * d + i], xv, part[j]);
+                for (int j = 0; j < 8; ++j) {
+                    if (j < nrows) {
+                        float4 wv = *reinterpret_cast<const float4 *>(rtr + (size_t)j * d + 4 * i4);
+                        part[j] = fmaf(wv.x, x0, fmaf(wv.y, x1, fmaf(wv.z, x2, fmaf(wv.w, x3, part[j]))));
+                    }
+                }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                float v = part[j];
-                for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) red[j * NW + warp] = v;
+                if (j < nrows) {
+                    float v = part[j];
+                    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (lane == 0) red[j * NW + warp] = v;
+                }
             }
             __syncthreads();
             trace_mark(p, l, 15, clock64() - tl0);
@@ -415,14 +439,17 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) ms->wmax[warp] = m;
             __syncthreads();
+            // lane a ranks warp maximum a among the NW maxima; the k-th one is the threshold
             float tau = -INFINITY;
             if (k <= NW) {
-                for (int a = 0; a < NW; ++a) {
-                    int above = 0;
-                    for (int b = 0; b < NW; ++b)
-                        above += (ms->wmax[b] > ms->wmax[a]) || (ms->wmax[b] == ms->wmax[a] && b < a);
-                    if (above == k - 1) tau = ms->wmax[a];
+                float ma = lane < NW ? ms->wmax[lane] : -INFINITY;
+                int above = 0;
+                for (int b = 0; b < NW; ++b) {
+                    float mb = ms->wmax[b];
+                    above += (mb > ma) || (mb == ma && b < lane);
                 }
+                unsigned hit = __ballot_sync(0xffffffffu, lane < NW && above == k - 1);
+                tau = __shfl_sync(0xffffffffu, ma, __ffs(hit) - 1);
             }
             for (int e = tid; e < E; e += NT) {
                 float v = lg[e];
@@ -572,11 +599,12 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 int s = (int)(it % p.nslot);
                 long long tw0 = clock64();
                 ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
-                tw_gu += clock64() - tw0;
+                long long tw1 = clock64();
+                tw_gu += tw1 - tw0;
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
                 float D0[4] = {0.f, 0.f, 0.f, 0.f}, D1[4] = {0.f, 0.f, 0.f, 0.f};
-                if (p.fmt == MOE_Q4B32) {
+                if constexpr (FMT == MOE_Q4B32) {
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq) {
                         uint4 a = *reinterpret_cast<const uint4 *>(tile + (size_t)(4 * warp + kq) * 512 + lane * 16);
@@ -616,6 +644,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     red[(q * NW + warp) * 16 + g] = ag;
                     red[(q * NW + warp) * 16 + 8 + g] = a8;
                 }
+                if (q < 6) trace_mark(p, l, 16 + q, clock64() - tw1);
             }
         }
         if (cta_failed(ms, ok)) break;
@@ -652,11 +681,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             if (cta_failed(ms, ok)) break;
             for (int t = tid; t < nU * nbi; t += NT) {
                 int us = t / nbi, b = t % nbi;
-                const uint16_t *hh = htab + (size_t)(2 * us) * I + 32 * b;
-                const uint16_t *hl = htab + (size_t)(2 * us + 1) * I + 32 * b;
-                float sacc = 0.f;
-                for (int j = 0; j < 32; ++j) sacc += bf16_bits_f(hh[j]) + bf16_bits_f(hl[j]);
-                hsum[t] = sacc;
+                hsum[t] = sum32_bf16(htab + (size_t)(2 * us) * I + 32 * b) +
+                          sum32_bf16(htab + (size_t)(2 * us + 1) * I + 32 * b);
             }
             __syncthreads();
         }
@@ -681,7 +707,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     float D[4] = {0.f, 0.f, 0.f, 0.f};
                     const uint16_t *hp = htab + (size_t)(2 * us + (g & 1)) * I;
                     uint32_t a[16];
-                    if (p.fmt == MOE_Q4B32) {
+                    if constexpr (FMT == MOE_Q4B32) {
                         uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)warp * 512 + lane * 16);
                         q4_frag(av.x, a[0], a[1], a[2], a[3]);
                         q4_frag(av.y, a[4], a[5], a[6], a[7]);
@@ -852,9 +878,10 @@ int decode_setup(moe_ctx *ctx) {
     ds.slot_bytes = slot;
     ds.rpc = rpc;
     ds.smem_bytes = (int)(fixed + (size_t)nslot * slot);
-    QE_CHECK(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, ds.smem_bytes));
+    const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
+    QE_CHECK(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, ds.smem_bytes));
     int per_sm = 0;
-    QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode, NT, ds.smem_bytes));
+    QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NT, ds.smem_bytes));
     if (per_sm < 1) ds.smem_bytes = 0;
     return MOE_OK;
 }
@@ -929,7 +956,8 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_resid = ds.off_resid;
     p.off_sums = ds.off_sums;
     void *args[] = {&p};
-    QE_CHECK(cudaLaunchCooperativeKernel((void *)k_decode, dim3(ds.grid), dim3(NT), args,
+    const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
+    QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ds.grid), dim3(NT), args,
                                          (size_t)ds.smem_bytes, st));
     QE_CHECK_LAUNCH("k_decode");
     return MOE_OK;
