@@ -829,6 +829,7 @@ int decode_setup(moe_ctx *ctx) {
     cudaDeviceProp prop;
     QE_CHECK(cudaGetDeviceProperties(&prop, dev));
     int G = prop.multiProcessorCount;
+    ds.sms = G;
     if (G > c.d_model / 16) G = c.d_model / 16;   // a down tile then spans at most two CTAs
     ds.grid = G;
     int rpc = (c.n_experts + G - 1) / G;

@@ -84,12 +84,6 @@ using namespace qeffn;
 
 namespace {
 
-#define QE_TRY(call)                   \
-    do {                               \
-        int _s = (call);               \
-        if (_s != MOE_OK) return _s;   \
-    } while (0)
-
 int validate_config(const moe_config *c) {
     if (c->fmt != MOE_Q4B32 && c->fmt != MOE_Q3B32) return MOE_ERR_INVALID_ARG;
     if (c->d_model <= 0 || c->n_experts <= 0 || c->d_ff <= 0 || c->top_k <= 0 ||
@@ -129,8 +123,14 @@ int alloc_workspace(moe_ctx *ctx) {
         {(void **)&ws.x_io, MT * d * 2, "x_io"},
         {(void **)&ws.r_io, MT * d * 4, "r_io"},
         {(void **)&ws.dev_error, 4, "dev_error"},
+        {(void **)&ws.x16, MT * d * 2, "x16"},
+        {(void **)&ws.h16, S * I * 2, "h16"},
+        {(void **)&ws.y_acc, MT * d * 4, "y_acc"},
+        {(void **)&ws.tc_n_items, 4, "tc_n_items"},
     };
+    ws.tc_items_max = tc_items_max(c);
     for (auto &it : items) QE_TRY(ctx_alloc(ctx, it.p, it.bytes, it.name));
+    QE_TRY(ctx_alloc(ctx, (void **)&ws.tc_items, ws.tc_items_max * sizeof(int4), "tc_items"));
     QE_CHECK(cudaMemset(ws.dev_error, 0, 4));
     QE_TRY(ctx_alloc(ctx, (void **)&ctx->d_layers, sizeof(LayerPtrs) * c.n_layers, "layer table"));
     QE_CHECK(cudaMemset(ctx->d_layers, 0, sizeof(LayerPtrs) * c.n_layers));
@@ -231,6 +231,7 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
     QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
     QE_TRY(launch_topk(ctx, ws.logits, T, ids_, w_, st));
     QE_TRY(launch_dispatch(ctx, ids_, T, st));
+    if (tc_supported(ctx, T)) return launch_tc_experts(ctx, Ly, x, T, w_, y, yf, st);
     QE_TRY(timing_begin(ctx, st, "k_gateup_simt+k_down_simt"));
     QE_TRY(launch_experts_simt(ctx, Ly, x, T, st));
     QE_TRY(timing_end(ctx, st));

@@ -141,6 +141,13 @@ struct Workspace {
     float *r_io = nullptr;       // [T][d] staging for host I/O
     int *dev_error = nullptr;    // [1]
     int max_chunks = 0;
+    // tensor-core prefill path
+    uint16_t *x16 = nullptr;     // [T][d] fp16 copy of the layer input
+    uint16_t *h16 = nullptr;     // [S][I] fp16 SwiGLU outputs by grouped position
+    float *y_acc = nullptr;      // [T][d] fp32 output accumulator
+    int4 *tc_items = nullptr;    // work items of one grouped GEMM
+    int32_t *tc_n_items = nullptr;
+    size_t tc_items_max = 0;
 };
 
 // Device-side table of one layer's weights (the persistent kernels walk it).
@@ -159,6 +166,7 @@ struct DecodeState {
     int gu_units_max = 0, dn_units_max = 0;   // per-CTA unit counts the carve is sized for
     int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
         off_misc = 0, off_resid = 0, off_sums = 0;
+    int sms = 0;          // streaming multiprocessors of the device
     uint2 *ll = nullptr;  // flagged-word exchange buffers
     uint32_t epoch = 1;
     unsigned long long *trace = nullptr;   // phase clocks (MOE_FLAG_TRACE)
@@ -208,6 +216,12 @@ void ctx_free(moe_ctx *ctx, void *p);
         if (_e != cudaSuccess) return qeffn::set_cuda_error(_e, #call);  \
     } while (0)
 
+#define QE_TRY(call)                   \
+    do {                               \
+        int _s = (call);               \
+        if (_s != MOE_OK) return _s;   \
+    } while (0)
+
 extern long long g_launches;   // every kernel launch the library issued
 
 #define QE_CHECK_LAUNCH(what)                                            \
@@ -243,6 +257,10 @@ size_t decode_ll_bytes(const moe_config &c);
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
                   cudaStream_t st);
+bool tc_supported(const moe_ctx *ctx, int T);
+size_t tc_items_max(const moe_config &c);
+int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, const float *w_route,
+                      uint16_t *y, float *yf, cudaStream_t st);
 int launch_record(const moe_ctx *ctx, int T, int layer_idx, const moe_stack_record *rec,
                   const uint16_t *x, const uint16_t *y, const float *yf, const int32_t *ids,
                   const float *w, cudaStream_t st);

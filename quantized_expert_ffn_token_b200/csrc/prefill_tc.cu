@@ -1,0 +1,567 @@
+// Many-token (prefill) expert path on the 5th-generation tensor cores.
+//
+// After routing, the (token, expert) slots are grouped by expert; each expert
+// is then two GEMMs over its slots:
+//   gate/up  [cnt x d] . [d x 2I]  -> SwiGLU -> h [cnt x I]      (fp16)
+//   down     [cnt x I] . [I x d]   -> y[token] += w_slot * out   (fp32)
+// One persistent kernel per GEMM, one CTA per SM, warp-specialised:
+//   warp 0      : allocates TMEM, one lane issues tcgen05.mma (kind::f16,
+//                 fp16 x fp16 -> fp32 in TMEM) and tcgen05.commit;
+//   warps 1..8  : producers.  A rows (tokens or h rows) are gathered with
+//                 16-byte cp.async; the weights are decoded from the packed
+//                 row tiles to fp16 (w = s * (q - zero), one rounding) and
+//                 stored; both land in the 128-byte-swizzled K-major layout
+//                 the MMA descriptors describe;
+//   warps 12..15: epilogue, tcgen05.ld from TMEM.
+// A work item is (expert, 256 slots, 256 output columns): two M=128
+// accumulators share every decoded weight stage (TMEM: 2 x 256 fp32 columns),
+// so the weight decode is paid once per 256 slots.
+//
+// Expert network = SwiGLU; routing weights and block formats as in moe.h.
+// The weights are rounded to fp16 here (the tensor cores take one operand
+// type per MMA), which is the one place the layer is not exact in fp32; the
+// resulting error (about 4e-4 relative L2 before the bf16 output rounding) is
+// inside the layer's 1e-3 bound.
+#include <math.h>
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace qeffn {
+
+namespace {
+
+constexpr int TC_NT = 512;                 // 16 warps
+constexpr int TC_PROD_W0 = 1, TC_PROD_NW = 8;
+constexpr int TC_EPI_W0 = 12;              // warps 12..15: TMEM lane quarters 0..3
+constexpr int TC_BM = 256;                 // slots per work item (2 x M=128)
+constexpr int TC_BN = 256;                 // output columns per work item
+constexpr int TC_BK = 64;                  // k per pipeline stage (one 128-byte swizzle row)
+constexpr int TC_STAGES = 3;
+constexpr int A_STAGE_BYTES = TC_BM * TC_BK * 2;   // 32 KB
+constexpr int B_STAGE_BYTES = TC_BN * TC_BK * 2;   // 32 KB
+constexpr long long TC_SPIN = 4000000000LL;        // clock64 cycles, about two seconds
+
+struct TcParams {
+    int fmt, zero;
+    int K;                      // reduction length (d or I)
+    int N;                      // output columns (2I or d)
+    MatLayout L;                // weight row-tile layout of this GEMM
+    const uint8_t *W;           // [experts] packed tiles
+    const uint16_t *A;          // fp16 rows: x16 [T][d] (gate/up) or h16 [S][I] (down)
+    int a_by_token;             // 1: A row = token of the slot (gather), 0: A row = slot position
+    const int32_t *perm;        // grouped position -> slot
+    const int32_t *offsets;     // expert -> first grouped position
+    const int4 *items;          // (expert, first position, rows, n-tile)
+    const int32_t *n_items;
+    int T, k, E;
+    // gate/up epilogue
+    uint16_t *h16;              // [S][I] fp16
+    int I;
+    // down epilogue
+    float *y_acc;               // [T][d]
+    const float *w_route;       // [T][k]
+    int d;
+    int *err;
+};
+
+__device__ __forceinline__ uint32_t su32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, int count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; false on timeout or when another CTA reported an error.
+__device__ __forceinline__ bool mbar_wait_b(uint64_t *b, uint32_t parity, int *err) {
+    long long t0 = clock64();
+    for (int it = 0;; ++it) {
+        if (mbar_try(b, parity)) return true;
+        if ((it & 63) == 63) {
+            if (*(volatile int *)err != 0) return false;
+            if (clock64() - t0 > TC_SPIN) {
+                atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(su32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// --- tcgen05 -------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(dst)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] . B[smem]^T, M=128, N=256, K=16, fp16 in, fp32 accumulate.
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on *b once every MMA this thread issued before has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *b) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+                 : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), 16-byte leading offset (unused by this swizzle),
+// descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N=256, M=128.
+constexpr uint32_t IDESC = (1u << 4) | ((uint32_t)(TC_BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+// Byte offset of (row, k) in a K-major 128-byte-swizzled tile (64 fp16 per row).
+__device__ __forceinline__ uint32_t swz(int row, int k) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((k >> 3) ^ row) & 7) << 4) + ((k & 7) << 1));
+}
+
+// fp16x2 helpers
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// fp16 magic numbers: a field OR-ed under 1024.0 reads 1024 + F*q; one fp16
+// FMA with 1/F and -(1024/F + zero) gives q - zero exactly.
+constexpr uint32_t H_MAGIC = 0x64006400u, H_ONE = 0x3C003C00u, H_16TH = 0x2C002C00u;
+constexpr uint32_t H_8TH = 0x30003000u, H_64TH = 0x24002400u;
+constexpr uint32_t H_M1032 = 0xE408E408u, H_M72 = 0xD480D480u;              // Q4: -(1024+8), -(64+8)
+constexpr uint32_t H_M1028 = 0xE404E404u, H_M132 = 0xD820D820u, H_M20 = 0xCD00CD00u;  // Q3
+
+// The 16 (q - zero) fp16 pairs of one lane's piece of a k group, register
+// q = 4*slice + reg (reg a0..a3 as in the row-tile layout).
+template <int FMT>
+__device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16]) {
+    if constexpr (FMT == MOE_Q4B32) {
+        uint4 a = *reinterpret_cast<const uint4 *>(src);
+        uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint32_t w = wv[m], w8 = w >> 8;
+            r[4 * m + 0] = hfma2((w & 0x000F000Fu) | H_MAGIC, H_ONE, H_M1032);
+            r[4 * m + 1] = hfma2((w & 0x00F000F0u) | H_MAGIC, H_16TH, H_M72);
+            r[4 * m + 2] = hfma2((w8 & 0x000F000Fu) | H_MAGIC, H_ONE, H_M1032);
+            r[4 * m + 3] = hfma2((w8 & 0x00F000F0u) | H_MAGIC, H_16TH, H_M72);
+        }
+    } else {
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(src);
+        uint32_t ws[3] = {wp[0], wp[1], wp[2]};
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            uint32_t w = ws[j], w9 = ws[j] >> 9;
+            r[5 * j + 0] = hfma2((w & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
+            r[5 * j + 1] = hfma2((w & 0x00380038u) | H_MAGIC, H_8TH, H_M132);
+            r[5 * j + 2] = hfma2((w & 0x01C001C0u) | H_MAGIC, H_64TH, H_M20);
+            r[5 * j + 3] = hfma2((w9 & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
+            r[5 * j + 4] = hfma2((w9 & 0x00380038u) | H_MAGIC, H_8TH, H_M132);
+        }
+        uint32_t s = ((ws[0] >> 15) & 0x00010001u) | ((ws[1] >> 14) & 0x00020002u) | ((ws[2] >> 13) & 0x00040004u);
+        r[15] = hfma2(s | H_MAGIC, H_ONE, H_M1028);
+    }
+}
+
+__device__ __forceinline__ int slot_token(int slot, int T, int k) {
+    int routed = T * k;
+    return slot < routed ? slot / k : (slot - routed) % T;
+}
+
+struct TcSmem {
+    uint64_t full[TC_STAGES];
+    uint64_t empty[TC_STAGES];
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int FMT, bool GATEUP>
+__global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment of the swizzled tiles
+    uint8_t *smem = smem_raw + ((1024 - (su32(smem_raw) & 1023)) & 1023);
+    uint8_t *sA = smem;                                  // [stage][256 rows][128 B]
+    uint8_t *sB = smem + TC_STAGES * A_STAGE_BYTES;      // [stage][256 rows][128 B]
+    TcSmem *ss = reinterpret_cast<TcSmem *>(sB + TC_STAGES * B_STAGE_BYTES);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+    const int n_items = *p.n_items;
+    const int nk = p.K / TC_BK;
+
+    if (tid == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&ss->full[s], TC_PROD_NW * 32);
+            mbar_init(&ss->empty[s], 1);
+        }
+        mbar_init(&ss->acc_full, 1);
+        mbar_init(&ss->acc_empty, 128);
+        ss->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(&ss->tmem_base, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ss->tmem_base;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ---- MMA issuer ------------------------------------------------------------
+        int it = 0, ti = 0;
+        for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
+            int4 wi = p.items[item];
+            int rows = wi.z;
+            // accumulators free? (epilogue of the previous item has read them)
+            ok = mbar_wait_b(&ss->acc_empty, (uint32_t)((ti & 1) ^ 1), p.err);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+                int s = it % TC_STAGES;
+                ok = mbar_wait_b(&ss->full[s], (uint32_t)((it / TC_STAGES) & 1), p.err);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    uint32_t a0 = su32(sA + s * A_STAGE_BYTES), b0 = su32(sB + s * B_STAGE_BYTES);
+#pragma unroll
+                    for (int j = 0; j < TC_BK / 16; ++j) {
+                        uint64_t bd = sdesc(b0 + 32 * j);
+                        umma_f16(tmem, sdesc(a0 + 32 * j), bd, IDESC, (kb | j) != 0);
+                        if (rows > 128)
+                            umma_f16(tmem + 256, sdesc(a0 + 128 * 128 + 32 * j), bd, IDESC, (kb | j) != 0);
+                    }
+                    umma_commit(&ss->empty[s]);
+                }
+                __syncwarp();
+            }
+            if (ok && lane == 0) umma_commit(&ss->acc_full);
+            __syncwarp();
+        }
+    } else if (warp >= TC_PROD_W0 && warp < TC_PROD_W0 + TC_PROD_NW) {
+        // ---- producers ---------------------------------------------------------------
+        const int pt = tid - TC_PROD_W0 * 32;   // 0..255
+        const int pw = pt >> 5;                  // producer warp 0..7
+        const int g = lane >> 2, c = lane & 3;
+        int it = 0;
+        int pending = -1;                        // stage whose cp.async group is still in flight
+        for (int item = blockIdx.x; item < n_items && ok; item += G) {
+            int4 wi = p.items[item];
+            const int e = wi.x, pos0 = wi.y, rows = wi.z, nt = wi.w;
+            // the A rows this thread gathers: row r = pt (0..255), all 8 chunks of 16 bytes
+            int r = pt;
+            int rr = min(r, rows - 1);           // rows past the expert's end repeat its last row
+            int pos = pos0 + rr;
+            int arow = p.a_by_token ? slot_token(p.perm[pos], p.T, p.k) : pos;
+            const uint16_t *asrc = p.A + (size_t)arow * p.K;
+            // weights: this warp decodes row tiles 2*pw and 2*pw+1 of the 16 in the n-tile
+            const uint8_t *wexp = p.W + (size_t)e * p.L.expert_bytes;
+            const int nb = p.K / 32;
+            for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+                int s = it % TC_STAGES;
+                ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
+                if (!ok) break;
+                uint8_t *a_dst = sA + s * A_STAGE_BYTES;
+                uint8_t *b_dst = sB + s * B_STAGE_BYTES;
+                // A: 8 chunks of row r, k = 64*kb .. +63
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    cp_async16(a_dst + swz(r, ch * 8), asrc + 64 * kb + ch * 8);
+                cp_async_commit();
+                // B: two row tiles, k group kb
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    int tl = 2 * pw + tt;                       // tile within the n-tile
+                    const uint8_t *tile = wexp + (size_t)(nt * 16 + tl) * p.L.tile_bytes;
+                    uint32_t q[16];
+                    decode_piece<FMT>(tile + (size_t)kb * p.L.kg_bytes + lane * (FMT == MOE_Q4B32 ? 16 : 12), q);
+                    const __half *sc = reinterpret_cast<const __half *>(tile + p.L.code_bytes);
+                    // scales of rows g, g+8 for blocks 2kb, 2kb+1
+                    __half2 s0 = __halves2half2(sc[g * nb + 2 * kb], sc[g * nb + 2 * kb]);
+                    __half2 s1 = __halves2half2(sc[g * nb + 2 * kb + 1], sc[g * nb + 2 * kb + 1]);
+                    __half2 s8a = __halves2half2(sc[(g + 8) * nb + 2 * kb], sc[(g + 8) * nb + 2 * kb]);
+                    __half2 s8b = __halves2half2(sc[(g + 8) * nb + 2 * kb + 1], sc[(g + 8) * nb + 2 * kb + 1]);
+                    uint32_t us0 = *reinterpret_cast<uint32_t *>(&s0), us1 = *reinterpret_cast<uint32_t *>(&s1);
+                    uint32_t u80 = *reinterpret_cast<uint32_t *>(&s8a), u81 = *reinterpret_cast<uint32_t *>(&s8b);
+                    int n0 = 16 * tl + g;                       // rows g, g+8 of this tile
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        int kk = 16 * m + 2 * c;                // k of a0 / a1 within the stage
+                        uint32_t sg = m < 2 ? us0 : us1, s8 = m < 2 ? u80 : u81;
+                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk)) = hmul2(q[4 * m + 0], sg);
+                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk)) = hmul2(q[4 * m + 1], s8);
+                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk + 8)) = hmul2(q[4 * m + 2], sg);
+                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk + 8)) = hmul2(q[4 * m + 3], s8);
+                    }
+                }
+                // the previous stage's A gather is complete once at most this stage's group is pending
+                if (pending >= 0) {
+                    cp_async_wait<1>();
+                    fence_async_smem();
+                    mbar_arrive(&ss->full[pending]);
+                }
+                pending = s;
+                fence_async_smem();   // this stage's B stores (A follows with its group)
+            }
+            if (!ok) break;
+            // flush: the last stage of the item
+            cp_async_wait<0>();
+            fence_async_smem();
+            mbar_arrive(&ss->full[pending]);
+            pending = -1;
+        }
+        if (pending >= 0) cp_async_wait<0>();
+    } else if (warp >= TC_EPI_W0) {
+        // ---- epilogue ----------------------------------------------------------------
+        const int q4 = warp - TC_EPI_W0;        // TMEM lane quarter
+        const int row = 32 * q4 + lane;         // row within each M=128 accumulator
+        int ti = 0;
+        for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
+            int4 wi = p.items[item];
+            const int pos0 = wi.y, rows = wi.z, nt = wi.w;
+            ok = mbar_wait_b(&ss->acc_full, (uint32_t)(ti & 1), p.err);
+            if (!ok) break;
+            tc_fence_after();
+            for (int acc = 0; acc < 2; ++acc) {
+                int m = 128 * acc + row;
+                bool live = m < rows;
+                if (acc == 1 && rows <= 128) break;
+                int pos = pos0 + min(m, rows - 1);
+                uint32_t tbase = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(256 * acc);
+                if constexpr (GATEUP) {
+                    // columns: 16 per row tile, gate rows 0..7 then up rows 8..15
+                    uint16_t *hrow = p.h16 + (size_t)pos * p.I + (size_t)nt * (TC_BN / 2);
+                    for (int cb = 0; cb < TC_BN / 32; ++cb) {
+                        float v[32];
+                        tmem_ld32(tbase + 32 * cb, v);
+                        if (live) {
+                            uint32_t hw[8];
+#pragma unroll
+                            for (int t2 = 0; t2 < 2; ++t2) {
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2) {
+                                    float g0 = v[16 * t2 + i], g1 = v[16 * t2 + i + 1];
+                                    float u0 = v[16 * t2 + 8 + i], u1 = v[16 * t2 + 8 + i + 1];
+                                    float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+                                    __half2 hh = __floats2half2_rn(h0, h1);
+                                    hw[4 * t2 + i / 2] = *reinterpret_cast<uint32_t *>(&hh);
+                                }
+                            }
+                            // h index of this column block: 16 per 32 columns
+                            uint4 *dst = reinterpret_cast<uint4 *>(hrow + 16 * cb);
+                            dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                            dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+                        }
+                    }
+                } else {
+                    int slot = p.perm[pos];
+                    int tok = slot_token(slot, p.T, p.k);
+                    float wt = slot < p.T * p.k ? p.w_route[slot] : 1.f;
+                    float *yrow = p.y_acc + (size_t)tok * p.d + (size_t)nt * TC_BN;
+                    for (int cb = 0; cb < TC_BN / 32; ++cb) {
+                        float v[32];
+                        tmem_ld32(tbase + 32 * cb, v);
+                        if (live) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4) {
+                                float *dst = yrow + 32 * cb + i;
+                                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst),
+                                             "f"(wt * v[i]), "f"(wt * v[i + 1]), "f"(wt * v[i + 2]), "f"(wt * v[i + 3])
+                                             : "memory");
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&ss->acc_empty);
+        }
+    }
+    // every role done: release TMEM
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Work items of one GEMM: for every expert with slots, ceil(cnt/256) row
+// blocks x n_tiles column tiles.  Single block.
+__global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int nx,
+                           int n_tiles, int4 *__restrict__ items, int32_t *__restrict__ n_items, int max_items) {
+    __shared__ int total;
+    if (threadIdx.x == 0) total = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nx; e += blockDim.x) {
+        int cnt = counts[e];
+        int mb = (cnt + TC_BM - 1) / TC_BM;
+        if (mb == 0) continue;
+        int base = atomicAdd(&total, mb * n_tiles);
+        for (int b = 0; b < mb; ++b)
+            for (int t = 0; t < n_tiles; ++t) {
+                int idx = base + b * n_tiles + t;
+                if (idx < max_items)
+                    items[idx] = make_int4(e, offsets[e] + b * TC_BM, min(TC_BM, cnt - b * TC_BM), t);
+            }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) *n_items = min(total, max_items);
+}
+
+__global__ void k_bf16_to_f16(const uint16_t *__restrict__ x, __half *__restrict__ y, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        y[i] = __float2half_rn(__uint_as_float((uint32_t)x[i] << 16));
+}
+
+__global__ void k_finish(const float *__restrict__ yacc, size_t n, uint16_t *__restrict__ y, float *__restrict__ yf) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        float v = yacc[i];
+        __nv_bfloat16 b = __float2bfloat16_rn(v);
+        y[i] = *reinterpret_cast<uint16_t *>(&b);
+        if (yf) yf[i] = v;
+    }
+}
+
+template <int FMT, bool GATEUP>
+int launch_tc(const TcParams &p, int grid, cudaStream_t st) {
+    size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + sizeof(TcSmem) + 1024;
+    QE_CHECK(cudaFuncSetAttribute(k_tc_gemm<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_tc_gemm<FMT, GATEUP><<<grid, TC_NT, smem, st>>>(p);
+    QE_CHECK_LAUNCH(GATEUP ? "k_tc_gemm<gate/up>" : "k_tc_gemm<down>");
+    return MOE_OK;
+}
+
+}  // namespace
+
+bool tc_supported(const moe_ctx *ctx, int T) {
+    const moe_config &c = ctx->cfg;
+    if (c.flags & MOE_FLAG_NO_TENSOR_PREFILL) return false;
+    if (T < 64) return false;
+    // n-tiles of 256 output columns: 2I and d must be multiples of 256
+    return (2 * c.d_ff) % TC_BN == 0 && c.d_model % TC_BN == 0 && c.d_model % TC_BK == 0 && c.d_ff % TC_BK == 0;
+}
+
+size_t tc_items_max(const moe_config &c) {
+    size_t S = (size_t)c.max_tokens * (c.top_k + c.n_shared);
+    size_t nx = c.n_experts + c.n_shared;
+    size_t nt = (size_t)((2 * c.d_ff) / TC_BN > c.d_model / TC_BN ? (2 * c.d_ff) / TC_BN : c.d_model / TC_BN);
+    return (S / TC_BM + nx) * nt;
+}
+
+int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, const float *w_route,
+                      uint16_t *y, float *yf, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    Workspace &ws = ctx->ws;
+    int dev_sms = ctx->dec.sms;
+    size_t Td = (size_t)T * c.d_model;
+    k_bf16_to_f16<<<592, 256, 0, st>>>(x, reinterpret_cast<__half *>(ws.x16), Td);
+    QE_CHECK_LAUNCH("k_bf16_to_f16");
+    int max_items = (int)ws.tc_items_max;
+
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.fmt = c.fmt;
+    p.zero = c.fmt == MOE_Q4B32 ? 8 : 4;
+    p.perm = ws.perm;
+    p.offsets = ws.offsets;
+    p.items = ws.tc_items;
+    p.n_items = ws.tc_n_items;
+    p.T = T;
+    p.k = c.top_k;
+    p.E = c.n_experts;
+    p.I = c.d_ff;
+    p.d = c.d_model;
+    p.err = ws.dev_error;
+
+    // gate/up: A = x16 rows gathered by token, N = 2I, K = d
+    k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, (2 * c.d_ff) / TC_BN, ws.tc_items,
+                                   ws.tc_n_items, max_items);
+    QE_CHECK_LAUNCH("k_tc_items");
+    p.K = c.d_model;
+    p.N = 2 * c.d_ff;
+    p.L = ctx->gu;
+    p.W = Ly.gu;
+    p.A = ws.x16;
+    p.a_by_token = 1;
+    p.h16 = ws.h16;
+    int grid = dev_sms;
+    QE_TRY(timing_begin(ctx, st, "k_tc_gemm<gate/up>+k_tc_gemm<down>"));
+    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, true>(p, grid, st)));
+    else QE_TRY((launch_tc<MOE_Q3B32, true>(p, grid, st)));
+
+    // down: A = h16 rows by grouped position, N = d, K = I
+    QE_CHECK(cudaMemsetAsync(ws.y_acc, 0, Td * sizeof(float), st));
+    k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, c.d_model / TC_BN, ws.tc_items,
+                                   ws.tc_n_items, max_items);
+    QE_CHECK_LAUNCH("k_tc_items");
+    p.K = c.d_ff;
+    p.N = c.d_model;
+    p.L = ctx->dn;
+    p.W = Ly.dn;
+    p.A = ws.h16;
+    p.a_by_token = 0;
+    p.y_acc = ws.y_acc;
+    p.w_route = w_route;
+    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, false>(p, grid, st)));
+    else QE_TRY((launch_tc<MOE_Q3B32, false>(p, grid, st)));
+    QE_TRY(timing_end(ctx, st));
+    k_finish<<<592, 256, 0, st>>>(ws.y_acc, Td, y, yf);
+    QE_CHECK_LAUNCH("k_finish");
+    return MOE_OK;
+}
+
+}  // namespace qeffn

@@ -33,6 +33,16 @@ F32_TOL = 1e-3
 # a fraction ~e/ulp of elements, so the relative L2 of the difference is about
 # sqrt(e * ulp); e <= 1e-4 gives <= 8e-4.
 BF16_TOL = 1e-3
+# The tensor-core path (T >= 64) rounds the dequantised weights and the
+# SwiGLU outputs to fp16 (the MMA takes one operand type): about 4e-4
+# relative L2 before the bf16 rounding (inside F32_TOL), hence about
+# sqrt(4e-4 * 2^-7.5) = 1.5e-3 between the two bf16 roundings.
+TC_BF16_TOL = 2e-3
+TC_MIN_TOKENS = 64
+
+
+def bf16_tol(T: int) -> float:
+    return TC_BF16_TOL if T >= TC_MIN_TOKENS else BF16_TOL
 
 
 def rel_l2(a, b) -> float:
@@ -83,7 +93,7 @@ def oracle_rows(cfg, src: ExpertSource, x_bits: np.ndarray, rows):
             np.array([r[2] for r in res]), np.array([r[3] for r in res]))
 
 
-def check_rows(cfg, src, x_bits, rows, g_y_bits, g_yf, g_ids, g_w, o=None, report=None):
+def check_rows(cfg, src, x_bits, rows, g_y_bits, g_yf, g_ids, g_w, o=None, report=None, tol16=BF16_TOL):
     """Compare GPU outputs of `rows` (arrays indexed like rows) with the oracle."""
     oy, oids, ow, ogap = o if o is not None else oracle_rows(cfg, src, x_bits, rows)
     oy = oy.copy()
@@ -104,7 +114,7 @@ def check_rows(cfg, src, x_bits, rows, g_y_bits, g_yf, g_ids, g_w, o=None, repor
     own_round = oracle.round_bf16(np.asarray(g_yf, dtype=np.float64))
     assert np.array_equal(np.asarray(g_y_bits).view(np.uint16), own_round)
     e16 = rel_l2(bits_to_f64(g_y_bits), bits_to_f64(oracle.round_bf16(oy)))
-    assert e16 <= BF16_TOL, e16
+    assert e16 <= tol16, e16
     if report is not None:
         report.update(rel_l2_f32=e32, rel_l2_bf16=e16, near_tie_flips=flips)
     return e32, e16, flips

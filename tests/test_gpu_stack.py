@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity import ExpertSource, bits_to_f64, check_rows, oracle_rows, to_np
+from tests.parity import ExpertSource, bf16_tol, bits_to_f64, check_rows, oracle_rows, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def _stack(name, rows=None, check_layers=None):
         src = ExpertSource(cfg, l)
         rep = {}
         idx = list(range(len(rows)))
-        check_rows(cfg, src, xr[l], idx, yr[l], yfr[l], idr[l], wr[l], report=rep)
+        check_rows(cfg, src, xr[l], idx, yr[l], yfr[l], idr[l], wr[l], report=rep, tol16=bf16_tol(T))
         worst[l] = rep
     return worst
 
