@@ -174,6 +174,7 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
     if (!Ly.router_w) {
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.router_w, E * d * 4, "router_w"));
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.router_b, E * 4, "router_b"));
+        QE_TRY(ctx_alloc(ctx, (void **)&Ly.router_parts, 3 * E * d * 2, "router_parts"));
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.gu, ctx->nx * ctx->gu.expert_bytes, "gate/up"));
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.dn, ctx->nx * ctx->dn.expert_bytes, "down"));
     }
@@ -182,6 +183,7 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
     QE_CHECK(cudaMemcpyAsync(Ly.router_w, w->router_w, E * d * 4, kind, st));
     if (w->router_bias) QE_CHECK(cudaMemcpyAsync(Ly.router_b, w->router_bias, E * 4, kind, st));
     else QE_CHECK(cudaMemsetAsync(Ly.router_b, 0, E * 4, st));
+    QE_TRY(launch_split_router(Ly.router_w, E * d, Ly.router_parts, st));
 
     for (int part = 0; part < 2; ++part) {          // 0: routed experts, 1: shared experts
         size_t n = part == 0 ? E : nsh;
@@ -228,7 +230,8 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
         QE_TRY(timing_end(ctx, st));
         return MOE_OK;
     }
-    QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
+    if (tc_router_supported(ctx, T)) QE_TRY(launch_tc_router(ctx, Ly, x, T, ws.logits, st));
+    else QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
     QE_TRY(launch_topk(ctx, ws.logits, T, ids_, w_, st));
     QE_TRY(launch_dispatch(ctx, ids_, T, st));
     if (tc_supported(ctx, T)) return launch_tc_experts(ctx, Ly, x, T, w_, y, yf, st);

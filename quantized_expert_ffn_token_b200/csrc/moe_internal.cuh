@@ -116,6 +116,7 @@ struct Layer {
     bool loaded = false;
     float *router_w = nullptr;   // [E][d]
     float *router_b = nullptr;   // [E] (zeros when the layer has no bias)
+    uint16_t *router_parts = nullptr;  // [3][E][d] bf16 parts of router_w (tensor-core router)
     uint8_t *gu = nullptr;       // [(E + n_shared)] x gu.expert_bytes
     uint8_t *dn = nullptr;       // [(E + n_shared)] x dn.expert_bytes
 };
@@ -258,6 +259,9 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
                   cudaStream_t st);
 bool tc_supported(const moe_ctx *ctx, int T);
+bool tc_router_supported(const moe_ctx *ctx, int T);
+int launch_split_router(const float *w, size_t n, uint16_t *parts, cudaStream_t st);
+int launch_tc_router(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, float *logits, cudaStream_t st);
 size_t tc_items_max(const moe_config &c);
 int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, const float *w_route,
                       uint16_t *y, float *yf, cudaStream_t st);

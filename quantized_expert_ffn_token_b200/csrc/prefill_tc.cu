@@ -62,8 +62,15 @@ struct TcParams {
     float *y_acc;               // [T][d]
     const float *w_route;       // [T][k]
     int d;
+    // router mode
+    const uint16_t *rparts;     // [3][E][d] bf16 parts of the fp32 router rows
+    const float *rbias;         // [E]
+    float *logits;              // [T][E]
+    int n_items_direct;         // router: items computed from the index (no item list)
     int *err;
 };
+
+enum TcMode { TC_GATEUP = 0, TC_DOWN = 1, TC_ROUTER = 2 };
 
 __device__ __forceinline__ uint32_t su32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -159,8 +166,10 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
     d |= (uint64_t)2 << 61;
     return d;
 }
-// Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N=256, M=128.
+// Instruction descriptor: fp32 accumulator, fp16 (or bf16) A and B, both
+// K-major, N=256, M=128.
 constexpr uint32_t IDESC = (1u << 4) | ((uint32_t)(TC_BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t IDESC_BF16 = IDESC | (1u << 7) | (1u << 10);
 
 // Byte offset of (row, k) in a K-major 128-byte-swizzled tile (64 fp16 per row).
 __device__ __forceinline__ uint32_t swz(int row, int k) {
@@ -222,6 +231,19 @@ __device__ __forceinline__ int slot_token(int slot, int T, int k) {
     return slot < routed ? slot / k : (slot - routed) % T;
 }
 
+// Work item: (expert, first row, rows, n-tile).  The router's items are
+// (-, first token, tokens, n-tile) in token-block-major order.
+template <int MODE>
+__device__ __forceinline__ int4 item_of(const TcParams &p, int item) {
+    if constexpr (MODE == TC_ROUTER) {
+        int ntn = p.N / TC_BN;
+        int mb = item / ntn, nt = item % ntn;
+        return make_int4(0, mb * TC_BM, min(TC_BM, p.T - mb * TC_BM), nt);
+    } else {
+        return p.items[item];
+    }
+}
+
 struct TcSmem {
     uint64_t full[TC_STAGES];
     uint64_t empty[TC_STAGES];
@@ -231,8 +253,10 @@ struct TcSmem {
     int abort;
 };
 
-template <int FMT, bool GATEUP>
+template <int FMT, int MODE>
 __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
+    constexpr bool GATEUP = MODE == TC_GATEUP;
+    constexpr uint32_t ID = MODE == TC_ROUTER ? IDESC_BF16 : IDESC;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment of the swizzled tiles
     uint8_t *smem = smem_raw + ((1024 - (su32(smem_raw) & 1023)) & 1023);
@@ -242,8 +266,10 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
-    const int n_items = *p.n_items;
-    const int nk = p.K / TC_BK;
+    const int n_items = p.items ? *p.n_items : p.n_items_direct;
+    // router: three bf16 parts of the weights, each over the whole K
+    const int nkd = p.K / TC_BK;
+    const int nk = MODE == TC_ROUTER ? 3 * nkd : nkd;
 
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
@@ -266,7 +292,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         // ---- MMA issuer ------------------------------------------------------------
         int it = 0, ti = 0;
         for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
-            int4 wi = p.items[item];
+            int4 wi = item_of<MODE>(p, item);
             int rows = wi.z;
             // accumulators free? (epilogue of the previous item has read them)
             ok = mbar_wait_b(&ss->acc_empty, (uint32_t)((ti & 1) ^ 1), p.err);
@@ -282,9 +308,9 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 #pragma unroll
                     for (int j = 0; j < TC_BK / 16; ++j) {
                         uint64_t bd = sdesc(b0 + 32 * j);
-                        umma_f16(tmem, sdesc(a0 + 32 * j), bd, IDESC, (kb | j) != 0);
+                        umma_f16(tmem, sdesc(a0 + 32 * j), bd, ID, (kb | j) != 0);
                         if (rows > 128)
-                            umma_f16(tmem + 256, sdesc(a0 + 128 * 128 + 32 * j), bd, IDESC, (kb | j) != 0);
+                            umma_f16(tmem + 256, sdesc(a0 + 128 * 128 + 32 * j), bd, ID, (kb | j) != 0);
                     }
                     umma_commit(&ss->empty[s]);
                 }
@@ -301,13 +327,15 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         int it = 0;
         int pending = -1;                        // stage whose cp.async group is still in flight
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
-            int4 wi = p.items[item];
+            int4 wi = item_of<MODE>(p, item);
             const int e = wi.x, pos0 = wi.y, rows = wi.z, nt = wi.w;
             // the A rows this thread gathers: row r = pt (0..255), all 8 chunks of 16 bytes
             int r = pt;
             int rr = min(r, rows - 1);           // rows past the expert's end repeat its last row
             int pos = pos0 + rr;
-            int arow = p.a_by_token ? slot_token(p.perm[pos], p.T, p.k) : pos;
+            int arow;
+            if constexpr (MODE == TC_ROUTER) arow = pos;                      // token
+            else arow = p.a_by_token ? slot_token(p.perm[pos], p.T, p.k) : pos;
             const uint16_t *asrc = p.A + (size_t)arow * p.K;
             // weights: this warp decodes row tiles 2*pw and 2*pw+1 of the 16 in the n-tile
             const uint8_t *wexp = p.W + (size_t)e * p.L.expert_bytes;
@@ -318,11 +346,20 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 if (!ok) break;
                 uint8_t *a_dst = sA + s * A_STAGE_BYTES;
                 uint8_t *b_dst = sB + s * B_STAGE_BYTES;
-                // A: 8 chunks of row r, k = 64*kb .. +63
+                const int kx = MODE == TC_ROUTER ? kb % nkd : kb;   // k block of the activations
+                // A: 8 chunks of row r, k = 64*kx .. +63
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
-                    cp_async16(a_dst + swz(r, ch * 8), asrc + 64 * kb + ch * 8);
+                    cp_async16(a_dst + swz(r, ch * 8), asrc + 64 * kx + ch * 8);
+                if constexpr (MODE == TC_ROUTER) {
+                    // B: router row (expert) 256*nt + r of part kb / nkd
+                    const uint16_t *bsrc = p.rparts + ((size_t)(kb / nkd) * p.E + (size_t)nt * TC_BN + r) * p.K;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        cp_async16(b_dst + swz(r, ch * 8), bsrc + 64 * kx + ch * 8);
+                }
                 cp_async_commit();
+                if constexpr (MODE != TC_ROUTER) {
                 // B: two row tiles, k group kb
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt) {
@@ -349,6 +386,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk + 8)) = hmul2(q[4 * m + 3], s8);
                     }
                 }
+                }
                 // the previous stage's A gather is complete once at most this stage's group is pending
                 if (pending >= 0) {
                     cp_async_wait<1>();
@@ -372,7 +410,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         const int row = 32 * q4 + lane;         // row within each M=128 accumulator
         int ti = 0;
         for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
-            int4 wi = p.items[item];
+            int4 wi = item_of<MODE>(p, item);
             const int pos0 = wi.y, rows = wi.z, nt = wi.w;
             ok = mbar_wait_b(&ss->acc_full, (uint32_t)(ti & 1), p.err);
             if (!ok) break;
@@ -383,7 +421,22 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 if (acc == 1 && rows <= 128) break;
                 int pos = pos0 + min(m, rows - 1);
                 uint32_t tbase = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(256 * acc);
-                if constexpr (GATEUP) {
+                if constexpr (MODE == TC_ROUTER) {
+                    float *lrow = p.logits + (size_t)pos * p.E + (size_t)nt * TC_BN;
+                    const float *bb = p.rbias + (size_t)nt * TC_BN;
+                    for (int cb = 0; cb < TC_BN / 32; ++cb) {
+                        float v[32];
+                        tmem_ld32(tbase + 32 * cb, v);
+                        if (live) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4) {
+                                float4 o = make_float4(v[i] + bb[32 * cb + i], v[i + 1] + bb[32 * cb + i + 1],
+                                                       v[i + 2] + bb[32 * cb + i + 2], v[i + 3] + bb[32 * cb + i + 3]);
+                                *reinterpret_cast<float4 *>(lrow + 32 * cb + i) = o;
+                            }
+                        }
+                    }
+                } else if constexpr (GATEUP) {
                     // columns: 16 per row tile, gate rows 0..7 then up rows 8..15
                     uint16_t *hrow = p.h16 + (size_t)pos * p.I + (size_t)nt * (TC_BN / 2);
                     for (int cb = 0; cb < TC_BN / 32; ++cb) {
@@ -476,16 +529,59 @@ __global__ void k_finish(const float *__restrict__ yacc, size_t n, uint16_t *__r
     }
 }
 
-template <int FMT, bool GATEUP>
+template <int FMT, int MODE>
 int launch_tc(const TcParams &p, int grid, cudaStream_t st) {
     size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + sizeof(TcSmem) + 1024;
-    QE_CHECK(cudaFuncSetAttribute(k_tc_gemm<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_tc_gemm<FMT, GATEUP><<<grid, TC_NT, smem, st>>>(p);
-    QE_CHECK_LAUNCH(GATEUP ? "k_tc_gemm<gate/up>" : "k_tc_gemm<down>");
+    QE_CHECK(cudaFuncSetAttribute(k_tc_gemm<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_tc_gemm<FMT, MODE><<<grid, TC_NT, smem, st>>>(p);
+    QE_CHECK_LAUNCH(MODE == TC_GATEUP ? "k_tc_gemm<gate/up>" : MODE == TC_DOWN ? "k_tc_gemm<down>" : "k_tc_gemm<router>");
     return MOE_OK;
 }
 
+// fp32 router rows -> three bf16 parts: w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2).
+__global__ void k_split_router(const float *__restrict__ w, size_t n, uint16_t *__restrict__ parts) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        float v = w[i];
+        __nv_bfloat16 a = __float2bfloat16_rn(v);
+        float r1 = v - __bfloat162float(a);
+        __nv_bfloat16 b = __float2bfloat16_rn(r1);
+        float r2 = r1 - __bfloat162float(b);
+        __nv_bfloat16 c = __float2bfloat16_rn(r2);
+        parts[i] = *reinterpret_cast<uint16_t *>(&a);
+        parts[n + i] = *reinterpret_cast<uint16_t *>(&b);
+        parts[2 * n + i] = *reinterpret_cast<uint16_t *>(&c);
+    }
+}
+
 }  // namespace
+
+bool tc_router_supported(const moe_ctx *ctx, int T) {
+    const moe_config &c = ctx->cfg;
+    return tc_supported(ctx, T) && c.n_experts % TC_BN == 0;
+}
+
+int launch_split_router(const float *w, size_t n, uint16_t *parts, cudaStream_t st) {
+    k_split_router<<<592, 256, 0, st>>>(w, n, parts);
+    QE_CHECK_LAUNCH("k_split_router");
+    return MOE_OK;
+}
+
+int launch_tc_router(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, float *logits, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.K = c.d_model;
+    p.N = c.n_experts;
+    p.E = c.n_experts;
+    p.T = T;
+    p.A = x;
+    p.rparts = Ly.router_parts;
+    p.rbias = Ly.router_b;
+    p.logits = logits;
+    p.n_items_direct = ((T + TC_BM - 1) / TC_BM) * (c.n_experts / TC_BN);
+    p.err = ctx->ws.dev_error;
+    return launch_tc<MOE_Q4B32, TC_ROUTER>(p, ctx->dec.sms, st);
+}
 
 bool tc_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
@@ -540,8 +636,8 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.h16 = ws.h16;
     int grid = dev_sms;
     QE_TRY(timing_begin(ctx, st, "k_tc_gemm<gate/up>+k_tc_gemm<down>"));
-    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, true>(p, grid, st)));
-    else QE_TRY((launch_tc<MOE_Q3B32, true>(p, grid, st)));
+    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_GATEUP>(p, grid, st)));
+    else QE_TRY((launch_tc<MOE_Q3B32, TC_GATEUP>(p, grid, st)));
 
     // down: A = h16 rows by grouped position, N = d, K = I
     QE_CHECK(cudaMemsetAsync(ws.y_acc, 0, Td * sizeof(float), st));
@@ -556,8 +652,8 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.a_by_token = 0;
     p.y_acc = ws.y_acc;
     p.w_route = w_route;
-    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, false>(p, grid, st)));
-    else QE_TRY((launch_tc<MOE_Q3B32, false>(p, grid, st)));
+    if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_DOWN>(p, grid, st)));
+    else QE_TRY((launch_tc<MOE_Q3B32, TC_DOWN>(p, grid, st)));
     QE_TRY(timing_end(ctx, st));
     k_finish<<<592, 256, 0, st>>>(ws.y_acc, Td, y, yf);
     QE_CHECK_LAUNCH("k_finish");
