@@ -40,6 +40,8 @@ constexpr int TC_BK = 64;                  // k per pipeline stage (one 128-byte
 constexpr int TC_STAGES = 3;
 constexpr int A_STAGE_BYTES = TC_BM * TC_BK * 2;   // 32 KB
 constexpr int B_STAGE_BYTES = TC_BN * TC_BK * 2;   // 32 KB
+constexpr int RAW_THREAD_BYTES = 96;                 // 2 slots x (2 x 16 B codes + 4 x 4 B scales)
+constexpr int RAW_BYTES = TC_PROD_NW * 32 * RAW_THREAD_BYTES;
 constexpr long long TC_SPIN = 4000000000LL;        // clock64 cycles, about two seconds
 
 struct TcParams {
@@ -106,6 +108,9 @@ __device__ __forceinline__ bool mbar_wait_b(uint64_t *b, uint32_t parity, int *e
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(su32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(su32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -226,6 +231,32 @@ __device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16])
     }
 }
 
+// Decode this thread's two pieces (row tiles 2*pw, 2*pw+1 of the n-tile, lane
+// (g, c)) from its staging bytes into the stage's swizzled fp16 weight tile:
+// w = s * (q - zero), one fp16 rounding.
+template <int FMT>
+__device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *b_dst, int pw, int g, int c) {
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+        uint32_t q[16];
+        decode_piece<FMT>(raw + 16 * tt, q);
+        uint32_t sgp = *reinterpret_cast<const uint32_t *>(raw + 32 + 8 * tt);   // s[g][2kb], s[g][2kb+1]
+        uint32_t s8p = *reinterpret_cast<const uint32_t *>(raw + 36 + 8 * tt);   // rows g+8
+        uint32_t us0 = (sgp & 0xFFFFu) * 0x10001u, us1 = (sgp >> 16) * 0x10001u;
+        uint32_t u80 = (s8p & 0xFFFFu) * 0x10001u, u81 = (s8p >> 16) * 0x10001u;
+        int n0 = 16 * (2 * pw + tt) + g;                // rows g, g+8 of this tile
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            int kk = 16 * m + 2 * c;                    // k of a0 / a1 within the stage
+            uint32_t sg = m < 2 ? us0 : us1, s8 = m < 2 ? u80 : u81;
+            *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk)) = hmul2(q[4 * m + 0], sg);
+            *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk)) = hmul2(q[4 * m + 1], s8);
+            *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk + 8)) = hmul2(q[4 * m + 2], sg);
+            *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk + 8)) = hmul2(q[4 * m + 3], s8);
+        }
+    }
+}
+
 __device__ __forceinline__ int slot_token(int slot, int T, int k) {
     int routed = T * k;
     return slot < routed ? slot / k : (slot - routed) % T;
@@ -262,7 +293,8 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
     uint8_t *smem = smem_raw + ((1024 - (su32(smem_raw) & 1023)) & 1023);
     uint8_t *sA = smem;                                  // [stage][256 rows][128 B]
     uint8_t *sB = smem + TC_STAGES * A_STAGE_BYTES;      // [stage][256 rows][128 B]
-    TcSmem *ss = reinterpret_cast<TcSmem *>(sB + TC_STAGES * B_STAGE_BYTES);
+    uint8_t *sRaw = sB + TC_STAGES * B_STAGE_BYTES;      // producers' private weight staging
+    TcSmem *ss = reinterpret_cast<TcSmem *>(sRaw + RAW_BYTES);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
@@ -326,6 +358,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         const int g = lane >> 2, c = lane & 3;
         int it = 0;
         int pending = -1;                        // stage whose cp.async group is still in flight
+        uint8_t *myraw = sRaw + pt * RAW_THREAD_BYTES;
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             const int e = wi.x, pos0 = wi.y, rows = wi.z, nt = wi.w;
@@ -360,45 +393,39 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 }
                 cp_async_commit();
                 if constexpr (MODE != TC_ROUTER) {
-                // B: two row tiles, k group kb
+                    // this thread's weight bytes for k group kb (decoded one iteration later)
+                    uint8_t *raw = myraw + (it & 1) * 48;
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    int tl = 2 * pw + tt;                       // tile within the n-tile
-                    const uint8_t *tile = wexp + (size_t)(nt * 16 + tl) * p.L.tile_bytes;
-                    uint32_t q[16];
-                    decode_piece<FMT>(tile + (size_t)kb * p.L.kg_bytes + lane * (FMT == MOE_Q4B32 ? 16 : 12), q);
-                    const __half *sc = reinterpret_cast<const __half *>(tile + p.L.code_bytes);
-                    // scales of rows g, g+8 for blocks 2kb, 2kb+1
-                    __half2 s0 = __halves2half2(sc[g * nb + 2 * kb], sc[g * nb + 2 * kb]);
-                    __half2 s1 = __halves2half2(sc[g * nb + 2 * kb + 1], sc[g * nb + 2 * kb + 1]);
-                    __half2 s8a = __halves2half2(sc[(g + 8) * nb + 2 * kb], sc[(g + 8) * nb + 2 * kb]);
-                    __half2 s8b = __halves2half2(sc[(g + 8) * nb + 2 * kb + 1], sc[(g + 8) * nb + 2 * kb + 1]);
-                    uint32_t us0 = *reinterpret_cast<uint32_t *>(&s0), us1 = *reinterpret_cast<uint32_t *>(&s1);
-                    uint32_t u80 = *reinterpret_cast<uint32_t *>(&s8a), u81 = *reinterpret_cast<uint32_t *>(&s8b);
-                    int n0 = 16 * tl + g;                       // rows g, g+8 of this tile
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        int kk = 16 * m + 2 * c;                // k of a0 / a1 within the stage
-                        uint32_t sg = m < 2 ? us0 : us1, s8 = m < 2 ? u80 : u81;
-                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk)) = hmul2(q[4 * m + 0], sg);
-                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk)) = hmul2(q[4 * m + 1], s8);
-                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk + 8)) = hmul2(q[4 * m + 2], sg);
-                        *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk + 8)) = hmul2(q[4 * m + 3], s8);
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const uint8_t *tile = wexp + (size_t)(nt * 16 + 2 * pw + tt) * p.L.tile_bytes;
+                        const uint8_t *cs = tile + (size_t)kb * p.L.kg_bytes;
+                        if constexpr (FMT == MOE_Q4B32) {
+                            cp_async16(raw + 16 * tt, cs + lane * 16);
+                        } else {
+                            cp_async4(raw + 16 * tt, cs + lane * 12);
+                            cp_async4(raw + 16 * tt + 4, cs + lane * 12 + 4);
+                            cp_async4(raw + 16 * tt + 8, cs + lane * 12 + 8);
+                        }
+                        const uint8_t *sc = tile + p.L.code_bytes;
+                        cp_async4(raw + 32 + 8 * tt, sc + (size_t)(g * nb + 2 * kb) * 2);
+                        cp_async4(raw + 36 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
                     }
                 }
-                }
-                // the previous stage's A gather is complete once at most this stage's group is pending
+                cp_async_commit();
+                // the previous iteration's group (its A rows and weight bytes) is complete once
+                // at most this one is pending: decode its weights, publish the stage
                 if (pending >= 0) {
                     cp_async_wait<1>();
+                    if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, g, c);
                     fence_async_smem();
                     mbar_arrive(&ss->full[pending]);
                 }
                 pending = s;
-                fence_async_smem();   // this stage's B stores (A follows with its group)
             }
             if (!ok) break;
             // flush: the last stage of the item
             cp_async_wait<0>();
+            if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, g, c);
             fence_async_smem();
             mbar_arrive(&ss->full[pending]);
             pending = -1;
@@ -531,7 +558,7 @@ __global__ void k_finish(const float *__restrict__ yacc, size_t n, uint16_t *__r
 
 template <int FMT, int MODE>
 int launch_tc(const TcParams &p, int grid, cudaStream_t st) {
-    size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + sizeof(TcSmem) + 1024;
+    size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + RAW_BYTES + sizeof(TcSmem) + 1024;
     QE_CHECK(cudaFuncSetAttribute(k_tc_gemm<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     k_tc_gemm<FMT, MODE><<<grid, TC_NT, smem, st>>>(p);
     QE_CHECK_LAUNCH(MODE == TC_GATEUP ? "k_tc_gemm<gate/up>" : MODE == TC_DOWN ? "k_tc_gemm<down>" : "k_tc_gemm<router>");
