@@ -84,9 +84,10 @@ typedef struct {
 
 /* moe_config.flags.  The first two pin a call to one implementation (tests
  * compare the paths with each other); the last is a test hook for the
- * bounded device waits: the decode kernel's CTA 0 withholds its router
- * logits, every wait on them runs out after about one second, and the call
- * reports MOE_ERR_DEVICE_TIMEOUT through moe_get_device_error. */
+ * bounded device waits: in the context's first single-token call the decode
+ * kernel's CTA 0 withholds its router logits, every wait on them runs out
+ * after about one second, and the call reports MOE_ERR_DEVICE_TIMEOUT through
+ * moe_get_device_error; later calls run normally. */
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* T == 1 runs the general path */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
@@ -165,7 +166,10 @@ MOE_API int moe_destroy(moe_ctx *ctx);
 
 /* Read (and clear) the device error word that bounded device waits and
  * in-kernel checks set.  *code receives 0 or a MOE_ERR_* value.  Synchronises
- * the context's device. */
+ * the context's device.  When *code is nonzero the call also resets the
+ * single-token kernel's cross-CTA arrival counters, which a kernel that gave
+ * up part-way leaves mid-count: after a nonzero code, call this before the
+ * next forward on the context. */
 MOE_API int moe_get_device_error(moe_ctx *ctx, int *code);
 
 /* Measurement hook.  While enabled, each forward records a CUDA event pair on

@@ -3,26 +3,31 @@
 //
 // Per layer (one token):
 //   1. every CTA rebuilds the layer input from the previous layer's output
-//      (residual add + rmsnorm in the stack), bf16 -> fp16 in shared memory;
+//      (residual add + rmsnorm in the stack): bf16 x and, for Q4, fp16 x * 2^s
+//      (a power of two that keeps every value inside fp16) in shared memory;
 //   2. router: CTA c owns experts c, c+G, ...; their fp32 rows were bulk-copied
-//      into shared memory one layer ahead; logits are published with a flag;
+//      into shared memory during the previous layer; logits are exchanged;
 //   3. every CTA reads all E logits and selects the same top-k (threshold +
 //      candidate ranking), then streams its share of the chosen experts'
 //      packed weights (gate/up tiles, then down tiles) into a ring of shared
-//      memory slots with cp.async.bulk, all issued as soon as slots free up;
+//      memory slots with cp.async.bulk, refilling each slot as soon as its
+//      gate/up tile is consumed;
 //   4. gate/up: each 16-row tile (8 gate + 8 up rows) is one unit; the warps
-//      split K, decode int4/int3 codes to exact fp16 (q - zero) and run
+//      split K, turn int4/int3 codes into fp16/bf16 operands by OR-ing them
+//      into the mantissa of a constant (no arithmetic), and run
 //      mma.m16n8k16 with the token in the B operand, one 32-block per column,
-//      so each column collects one block's partial sum, which is scaled by the
-//      block's fp16 scale in fp32; the SwiGLU output h is published;
-//   5. down: units are (16 output rows, expert); h is split into fp16 hi + lo
-//      (exact to 2^-22) and a CTA's contiguous run of units, weighted by the
-//      routing weights, is summed per 16-row tile and published as one of at
-//      most two parts per tile; the next layer adds the two parts in order.
-// Cross-CTA data moves through "flagged words": a 64-bit store of (value,
-// epoch) that a reader polls until the epoch matches, so every sync costs one
-// L2 round trip and no separate barrier.  All waits are bounded (clock64); on
-// timeout the kernel sets the context's error word and every CTA returns.
+//      so each column collects one block's partial sum; the constant's share
+//      is removed with the block sums of x and the block's fp16 scale applied
+//      in fp32; the SwiGLU output h is exchanged;
+//   5. down: units are (16 output rows, expert), one warp per unit over the
+//      whole K; h enters as bf16 hi + lo (h to about 2^-16 relative), and a
+//      CTA's contiguous run of units, weighted by the routing weights, is
+//      summed per 16-row tile into one of at most two parts per tile; the next
+//      layer adds the two parts in order.
+// The three exchanges per layer (logits, h, output parts) go through plain
+// fp32 buffers and one arrival counter each (see "cross-CTA exchanges" below).
+// All waits are bounded (clock64); on timeout the kernel sets the context's
+// error word and every CTA returns.
 //
 // Routing/combine passages: "Qwen3.8-Flash-Next at 45 Tokens/sec on a 12GB
 // GPU?" (video transcript 1:50-2:16, 3:36-3:47); expert = SwiGLU and the block
@@ -47,18 +52,18 @@ constexpr long long SPIN_LIMIT = 2000000000LL;   // clock64 cycles, about one se
 
 struct Misc {
     unsigned long long full[MAX_SLOTS];
+    unsigned long long empty[MAX_SLOTS];   // gate/up item consumed by every gate/up warp
     unsigned long long rbar;
     int ids[MAXK];
-    float vsel[MAXK];
-    float wsel[MAXK];
+    float psel[MAXK];          // exp(logit - max logit) of the selected experts, in rank order
     int uexp[MAXU];
     float uw[MAXU];
     int ncand;
-    int abort;
+    float xinv;                // 2^-s: undoes the power-of-two scaling of the fp16 layer input
     float wmax[NW];
     float red1[NW];
-    float cand_v[CAND_MAX];
-    int cand_id[CAND_MAX];
+    float amax[NW];
+    __align__(16) float2 cand[CAND_MAX];     // (logit, id bits)
 };
 
 struct DecodeParams {
@@ -75,16 +80,16 @@ struct DecodeParams {
     float *w_out;              // single layer: [k] or NULL
     moe_stack_record rec;      // stack records (row 0 only)
     int rec_on;
-    uint2 *ll_logits;          // [2][E]
-    uint2 *ll_h;               // [2][MAXU][I]
-    uint2 *ll_y;               // [2][2][d]
-    uint32_t epoch0;
+    unsigned *cnt;             // exchange counters: logits, h, y (128 bytes apart)
+    float *x_logits;           // [E]
+    float *x_h;                // [MAXU][I]
+    float *x_y;                // [2][d]: the two parts of every output row
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
     unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int dn_units_max;          // largest down-unit run of one CTA
-    int off_ring, off_router, off_x16, off_logits, off_htab, off_red, off_misc, off_resid, off_sums;
+    int off_ring, off_router, off_x16, off_xh, off_logits, off_htab, off_red, off_misc, off_resid, off_sums;
 };
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -97,6 +102,9 @@ __device__ __forceinline__ void mbar_init(unsigned long long *b, int count) {
 __device__ __forceinline__ void mbar_expect_tx(unsigned long long *b, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
                  : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(unsigned long long *b, uint32_t parity) {
     uint32_t ok;
@@ -122,22 +130,16 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-// A flagged word is one 64-bit value (low half: the float's bits, high half:
-// the epoch), stored and loaded as 64-bit elements so that a reader never sees
-// a new epoch with an old value.
-__device__ __forceinline__ void ll_store(uint2 *p, float v, uint32_t flag) {
-    unsigned long long w = ((unsigned long long)flag << 32) | __float_as_uint(v);
-    asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
-}
-__device__ __forceinline__ void ll_load2(const uint2 *p, uint2 &a, uint2 &b) {
-    unsigned long long x, y;
-    asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "l"(p) : "memory");
-    a = make_uint2((uint32_t)x, (uint32_t)(x >> 32));
-    b = make_uint2((uint32_t)y, (uint32_t)(y >> 32));
-}
 __device__ __forceinline__ void mma16816(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_h(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -157,6 +159,22 @@ __device__ __forceinline__ void q4_frag(uint32_t w, uint32_t &a0, uint32_t &a1, 
     a1 = ((w >> 4) & 0x000F000Fu) | BF_MAGIC;
     a2 = ((w >> 8) & 0x000F000Fu) | BF_MAGIC;
     a3 = ((w >> 12) & 0x000F000Fu) | BF_MAGIC;
+}
+
+// Q4B32 into fp16 (gate/up): a nibble at bits 0-3 of a half under 1024.0
+// (0x6400) reads as 1024 + q, one at bits 4-7 as 1024 + 16 q, both exact.  In
+// the fragment order registers a0/a2 (row g) take the first kind and a1/a3
+// (row g+8) the second, so the row g+8 partial sums come out 16x larger and
+// are scaled back in fp32; the offsets are 1024 + zero (row g) and
+// 1024/16 + zero (row g+8).  Five integer operations per eight codes.
+constexpr uint32_t H_MAGIC = 0x64006400u;
+__device__ __forceinline__ void q4_frag_h(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2,
+                                          uint32_t &a3) {
+    const uint32_t w8 = w >> 8;
+    a0 = (w & 0x000F000Fu) | H_MAGIC;
+    a1 = (w & 0x00F000F0u) | H_MAGIC;
+    a2 = (w8 & 0x000F000Fu) | H_MAGIC;
+    a3 = (w8 & 0x00F000F0u) | H_MAGIC;
 }
 
 // Q3B32: three words = the 16 fragment registers of four k16 slices.
@@ -197,43 +215,81 @@ __device__ __forceinline__ float sum32_bf16(const uint16_t *p) {
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-// Poll the flagged words base[i], i < n (n even, base 16-byte aligned): this
-// thread owns the pairs (2q, 2q+1), q = tid + NT*j, and keeps up to B 16-byte
-// loads in flight; put(i, value) receives each value once.
-template <int B, typename F>
-__device__ __forceinline__ bool poll_words(const uint2 *base, int n, uint32_t flag, int *err, F &&put) {
+// Sum of 32 consecutive fp16 values (16-byte aligned).
+__device__ __forceinline__ float sum32_f16(const uint16_t *p) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 v = q[j];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
+            acc[h] += f.x + f.y;
+        }
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// 2^e as a float, |e| <= 126.
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+// ---- cross-CTA exchanges ------------------------------------------------------
+// Each exchange: every CTA stores its share of a plain fp32 buffer, one thread
+// adds 1 to the exchange's counter with release semantics, and the readers
+// wait (acquire) until all G CTAs have arrived, then load the buffer with
+// gpu-scope loads (never from a stale L1 line).  The three exchanges of a
+// layer (logits, h, y) have one counter each; CTA 0 zeroes the counter of the
+// next exchange before it arrives at the current one: that counter was last
+// waited on two exchanges earlier, which every CTA has left by the time it can
+// arrive at the current one, and the release orders the zeroing before any
+// CTA's next arrival there.
+constexpr int X_LOGITS = 0, X_H = 1, X_Y = 2;
+__device__ __forceinline__ unsigned *ctr(const DecodeParams &p, int kind) { return p.cnt + 32 * kind; }
+__device__ __forceinline__ void ctr_arrive(unsigned *c) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
+}
+__device__ __forceinline__ void ctr_zero(unsigned *c) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(c), "r"(0u) : "memory");
+}
+__device__ __forceinline__ unsigned ctr_load(const unsigned *c) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_gpu(const float *p) {
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_gpu4(const float *p) {
+    float4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+// One thread: wait until the counter reaches n; false on timeout (error word
+// set) or when another CTA reported an error.
+__device__ __forceinline__ bool ctr_wait(const unsigned *c, unsigned n, int *err) {
     long long t0 = clock64();
-    const int np = n >> 1;
-    for (int q0 = threadIdx.x; q0 < np; q0 += NT * B) {
-        uint32_t need = 0;   // bit 2b: word 2q of load b, bit 2b+1: word 2q+1
-#pragma unroll
-        for (int b = 0; b < B; ++b)
-            if (q0 + b * NT < np) need |= 3u << (2 * b);
-        for (int it = 0;; ++it) {
-            uint2 v[2 * B];
-#pragma unroll
-            for (int b = 0; b < B; ++b)
-                if (need & (3u << (2 * b))) ll_load2(base + 2 * (q0 + b * NT), v[2 * b], v[2 * b + 1]);
-#pragma unroll
-            for (int h = 0; h < 2 * B; ++h) {
-                if ((need >> h) & 1u) {
-                    if (v[h].y == flag) {
-                        put(2 * (q0 + (h >> 1) * NT) + (h & 1), __uint_as_float(v[h].x));
-                        need &= ~(1u << h);
-                    }
-                }
-            }
-            if (!need) break;
-            if ((it & 7) == 7) {
-                if (*(volatile int *)err != 0) return false;
-                if (clock64() - t0 > SPIN_LIMIT) {
-                    atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
-                    return false;
-                }
+    for (int it = 0;; ++it) {
+        if ((int)(ctr_load(c) - n) >= 0) return true;
+        if ((it & 7) == 7) {
+            if (*(volatile int *)err != 0) return false;
+            if (clock64() - t0 > SPIN_LIMIT) {
+                atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                return false;
             }
         }
     }
-    return true;
+}
+// Thread 0 of every CTA, after a barrier that follows the CTA's stores.
+__device__ __forceinline__ void xchg_arrive(const DecodeParams &p, int kind, bool arrive = true) {
+    if (blockIdx.x == 0) ctr_zero(ctr(p, (kind + 1) % 3));
+    if (arrive) ctr_arrive(ctr(p, kind));
 }
 
 __device__ __forceinline__ bool mbar_wait(unsigned long long *b, uint32_t parity, int *err, bool honor_err) {
@@ -250,14 +306,23 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *b, uint32_t parity
     }
 }
 
-// CTA-uniform abort decision after a phase.
-__device__ __forceinline__ bool cta_failed(Misc *ms, bool mine_ok) {
-    if (!mine_ok) ms->abort = 1;
-    __syncthreads();
-    return ms->abort != 0;
-}
+// CTA-uniform abort decision after a phase: one barrier that also ORs the
+// threads' failures, so every thread leaves at the same barrier.
+__device__ __forceinline__ bool cta_failed(bool mine_ok) { return __syncthreads_or(!mine_ok) != 0; }
 
-constexpr int TRACE_WORDS = 24;   // per (CTA, layer) record: CTA, layer, 22 timestamps
+// Trace record per (CTA, layer): word 0 = CTA, word 1 = layer, word 2 + slot =
+// SM clock cycles since the layer started in this CTA, except where noted:
+//   13 previous layer's output received   0 layer input ready
+//   14 router rows in shared memory       15 router dot products done
+//    1 logits published                    8 all logits received
+//    2 routing known                      11 this thread's gate/up units done
+//    6 every gate/up unit done             3 h published
+//    4 every expert's h received           9 this thread's down units done
+//    7 every down unit done                5 output tiles published
+//   10 cycles waiting for gate/up data    12 cycles waiting for down data
+//   16..20 compute cycles of gate/up units 0..4 (warp 0)
+//   21 global timer (ns) at the layer start
+constexpr int TRACE_WORDS = 24;
 
 __device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph, long long t) {
     if (p.trace && threadIdx.x == 0 && ph < TRACE_WORDS - 2) {
@@ -276,6 +341,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     uint8_t *ring = smem + p.off_ring;
     float *rtr = reinterpret_cast<float *>(smem + p.off_router);
     uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_x16);         // layer input, bf16 bits
+    uint16_t *xh = reinterpret_cast<uint16_t *>(smem + p.off_xh);          // layer input * 2^s, fp16 bits
     float *xsum = reinterpret_cast<float *>(smem + p.off_sums);              // [d/32] block sums of x
     float *hsum = xsum + p.d / 32;                                             // [nU][I/32] of h hi + lo
     float *lg = reinterpret_cast<float *>(smem + p.off_logits);
@@ -283,7 +349,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     float *red = reinterpret_cast<float *>(smem + p.off_red);   // [2][NW][16]
     Misc *ms = reinterpret_cast<Misc *>(smem + p.off_misc);
     float *rs = reinterpret_cast<float *>(smem + p.off_resid);      // residual stream [d]
-    float *ybuf = reinterpret_cast<float *>(smem + p.off_htab);     // [d], free between layers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const int G = gridDim.x, cta = blockIdx.x;
@@ -299,10 +364,16 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     int *err = p.err;
 
     if (tid == 0) {
-        for (int s = 0; s < p.nslot; ++s) mbar_init(&ms->full[s], 1);
+        for (int s = 0; s < p.nslot; ++s) {
+            mbar_init(&ms->full[s], 1);
+            mbar_init(&ms->empty[s], p.d / 256);   // one arrival per gate/up warp
+        }
         mbar_init(&ms->rbar, 1);
-        ms->abort = 0;
         fence_mbar_init();
+    }
+    if (tid < p.nsh) {   // shared experts follow the routed ones in the unit list, weight 1
+        ms->uexp[k + tid] = E + tid;
+        ms->uw[k + tid] = 1.f;
     }
     __syncthreads();
 
@@ -321,17 +392,26 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     long long item = 0;                  // ring items planned so far (all layers)
     long long issued = 0;                // ring items whose copies were issued (thread 0)
     long long consumed = 0;              // ring items consumed so far
-    int router_issued = 1, router_waited = 0;   // router prefetch fills (thread 0) / waits
+    int router_issued = 1, router_waited = 0;   // router prefetch fills (producer) / waits
+    uint32_t gu_par = 0;   // producer: bit s = parity of the gate/up items issued into slot s so far
     bool ok = true;
+    bool aborted = false;                // CTA-uniform: the layer loop was left on a failure
 
     for (int l = 0; l < p.L; ++l) {
         const int layer = p.layer0 + l;
         const LayerPtrs Lp = p.layers[layer];
-        const uint32_t ep = p.epoch0 + (uint32_t)l;
-        const int lpar = l & 1;
         const long long tl0 = clock64();
+        if (p.trace) {   // global time of the layer start (ns), to line up the CTAs' clocks
+            unsigned long long gt;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
+            trace_mark(p, l, 21, (long long)gt);
+        }
 
         // ---- 1. layer input -------------------------------------------------------
+        // xb = bf16 input; for Q4 also xh = fp16(x * 2^s) with the power of two chosen from
+        // max |x| so that every value fits fp16 (|x| * 2^s < 2^15), exact for bf16 inputs
+        float amx = 0.f;   // this thread's share of max |r| (stack) or max |x|
+        float inv = 1.f;
         if (p.stack) {
             float ss = 0.f;   // this thread's share of sum(r^2)
             if (l == 0) {
@@ -339,48 +419,116 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     float v = bf16_bits_f(p.x_in[i]);
                     rs[i] = v;
                     ss = fmaf(v, v, ss);
+                    amx = fmaxf(amx, fabsf(v));
                 }
             } else {
-                // previous layer's output = part 0 + part 1 of every row (same thread owns row i)
-                const uint2 *y0 = p.ll_y + (size_t)((l - 1) & 1) * 2 * d;
-                ok = poll_words<4>(y0, d, ep - 1, err, [&](int i, float v) { ybuf[i] = v; });
-                ok = ok && poll_words<4>(y0 + d, d, ep - 1, err, [&](int i, float v) {
-                    float y = ybuf[i] + v;
-                    uint16_t yb = bf16_rn_bits(y);
-                    float rn = rs[i] + bf16_bits_f(yb);
-                    rs[i] = rn;
-                    ss = fmaf(rn, rn, ss);
-                    if (cta == 0 && p.rec_on) {
-                        if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
-                        if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
+                // previous layer's output = part 0 + part 1 of every row, once every CTA published
+                if (tid == 0) ok = ctr_wait(ctr(p, X_Y), (unsigned)G, err);
+                if (cta_failed(ok)) {
+                    aborted = true;
+                    break;
+                }
+                for (int i4 = tid; i4 < d / 4; i4 += NT) {
+                    const float4 a = ld_gpu4(p.x_y + 4 * i4), b = ld_gpu4(p.x_y + d + 4 * i4);
+                    const float ya[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int i = 4 * i4 + j;
+                        const float y = ya[j];
+                        const uint16_t yb = bf16_rn_bits(y);
+                        const float rn = rs[i] + bf16_bits_f(yb);
+                        rs[i] = rn;
+                        ss = fmaf(rn, rn, ss);
+                        amx = fmaxf(amx, fabsf(rn));
+                        if (cta == 0 && p.rec_on) {
+                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
+                            if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
+                        }
                     }
-                });
-                if (cta_failed(ms, ok)) break;
+                }
             }
             trace_mark(p, l, 13, clock64() - tl0);
-            for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            if (lane == 0) ms->red1[warp] = ss;
-            __syncthreads();
-            float tot = 0.f;
-            for (int w = 0; w < NW; ++w) tot += ms->red1[w];
-            float inv = 1.f / sqrtf(tot / (float)d + 1e-6f);
-            for (int i = tid; i < d; i += NT) {
-                uint16_t xv = bf16_rn_bits(rs[i] * inv);
-                xb[i] = xv;
-                if (cta == 0 && p.rec_on && p.rec.x_bf16) p.rec.x_bf16[(size_t)l * d + i] = xv;
+            for (int o = 16; o; o >>= 1) {
+                ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
             }
+            if (lane == 0) {
+                ms->red1[warp] = ss;
+                ms->amax[warp] = amx;
+            }
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
+            float tot = lane < NW ? ms->red1[lane] : 0.f;
+            amx = lane < NW ? ms->amax[lane] : 0.f;
+            for (int o = 16; o; o >>= 1) {
+                tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
+            }
+            inv = 1.f / sqrtf(tot / (float)d + 1e-6f);
+            amx = bf16_bits_f(bf16_rn_bits(amx * inv));   // = max |bf16(r * inv)| (monotone rounding)
         } else {
-            for (int i = tid; i < d; i += NT) xb[i] = p.x_in[i];
+            for (int i = tid; i < d; i += NT) {
+                uint16_t v = p.x_in[i];
+                xb[i] = v;
+                amx = fmaxf(amx, fabsf(bf16_bits_f(v)));
+            }
+            for (int o = 16; o; o >>= 1) amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
+            if (lane == 0) ms->amax[warp] = amx;
+            __syncthreads();
+            amx = lane < NW ? ms->amax[lane] : 0.f;
+            for (int o = 16; o; o >>= 1) amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
+        }
+        int xe;
+        frexpf(amx, &xe);                    // amx < 2^xe
+        const int xs_exp = min(15 - xe, 100);
+        const float xscale = pow2i(xs_exp);
+        if (tid == 0) ms->xinv = (FMT == MOE_Q4B32) ? pow2i(-xs_exp) : 1.f;
+        // 8 consecutive elements per thread: bf16 (stack: rounded from r * inv), fp16 of x * 2^s
+        for (int i8 = tid; i8 < d / 8; i8 += NT) {
+            uint32_t xw[4], hw[4];
+            if (p.stack) {
+                const float4 r0 = reinterpret_cast<const float4 *>(rs)[2 * i8];
+                const float4 r1 = reinterpret_cast<const float4 *>(rs)[2 * i8 + 1];
+                const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    xw[j] = (uint32_t)bf16_rn_bits(rv[2 * j] * inv) |
+                            ((uint32_t)bf16_rn_bits(rv[2 * j + 1] * inv) << 16);
+                *reinterpret_cast<uint4 *>(xb + 8 * i8) = make_uint4(xw[0], xw[1], xw[2], xw[3]);
+                if (cta == 0 && p.rec_on && p.rec.x_bf16) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        p.rec.x_bf16[(size_t)l * d + 8 * i8 + j] = (uint16_t)(xw[j >> 1] >> (16 * (j & 1)));
+                }
+            } else {
+                const uint4 v = *reinterpret_cast<const uint4 *>(xb + 8 * i8);
+                xw[0] = v.x; xw[1] = v.y; xw[2] = v.z; xw[3] = v.w;
+            }
+            if constexpr (FMT == MOE_Q4B32) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    __half2 h2 = __floats2half2_rn(__uint_as_float(xw[j] << 16) * xscale,
+                                                   __uint_as_float(xw[j] & 0xFFFF0000u) * xscale);
+                    hw[j] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                *reinterpret_cast<uint4 *>(xh + 8 * i8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            }
         }
         __syncthreads();
-        // block sums of the input (offset removal in the gate/up flush)
-        for (int b = tid; b < nbd; b += NT) xsum[b] = sum32_bf16(xb + 32 * b);
+        // block sums of the operand the gate/up MMAs see (offset removal in their flush)
+        for (int b = tid; b < nbd; b += NT)
+            xsum[b] = (FMT == MOE_Q4B32) ? sum32_f16(xh + 32 * b) : sum32_bf16(xb + 32 * b);
 
         trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
         {
             ok = mbar_wait(&ms->rbar, (uint32_t)(l & 1), err, true);
-            if (cta_failed(ms, ok)) break;
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
             ++router_waited;
             trace_mark(p, l, 14, clock64() - tl0);
             int nrows = 0;
@@ -410,40 +558,48 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     if (lane == 0) red[j * NW + warp] = v;
                 }
             }
-            __syncthreads();
+            __syncthreads();   // partials written; every read of the router rows is done
             trace_mark(p, l, 15, clock64() - tl0);
-            if (tid < nrows && !(p.withhold && cta == 0)) {
-                float v = 0.f;
-                for (int w = 0; w < NW; ++w) v += red[tid * NW + w];
-                int e = cta + G * tid;
-                ll_store(p.ll_logits + (size_t)lpar * E + e, v + Lp.rb[e], ep);
-            }
-            __syncthreads();
-            if (tid == PRODUCER && l + 1 < p.L) {
-                fence_proxy_async();
-                issue_router(layer + 1);
-                ++router_issued;
+            if (warp < nrows) {   // warp j sums row j's NW partials
+                float v = lane < NW ? red[warp * NW + lane] : 0.f;
+                for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                const int e = cta + G * warp;
+                if (lane == 0) p.x_logits[e] = v + Lp.rb[e];
             }
         }
 
         trace_mark(p, l, 1, clock64() - tl0);
         // ---- 3. top-k on all logits (same result in every CTA) ------------------------
         {
-            ok = poll_words<2>(p.ll_logits + (size_t)lpar * E, E, ep, err, [&](int e, float v) { lg[e] = v; });
-            if (tid == 0) ms->ncand = 0;
-            if (cta_failed(ms, ok)) break;
-            trace_mark(p, l, 8, clock64() - tl0);
-            // threshold: the k-th largest of the warps' maxima bounds the k-th largest logit from below
-            float m = -INFINITY;
-            for (int e = tid; e < E; e += NT) m = fmaxf(m, lg[e]);
+            __syncthreads();   // this CTA's logits are stored
+            if (tid == 0) {
+                xchg_arrive(p, X_LOGITS, !(p.withhold && cta == 0));
+                ok = ctr_wait(ctr(p, X_LOGITS), (unsigned)G, err);
+                ms->ncand = 0;
+            }
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
+            float m = -INFINITY;   // max of the logits this thread read (every warp reads some)
+            for (int e = tid; e < E; e += NT) {
+                const float v = ld_gpu(p.x_logits + e);
+                lg[e] = v;
+                m = fmaxf(m, v);
+            }
             for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) ms->wmax[warp] = m;
             __syncthreads();
-            // lane a ranks warp maximum a among the NW maxima; the k-th one is the threshold
+            trace_mark(p, l, 8, clock64() - tl0);
+            // the k-th largest of the warps' maxima bounds the k-th largest logit from below:
+            // lane a ranks warp maximum a among the NW maxima
+            const float ma = lane < NW ? ms->wmax[lane] : -INFINITY;
+            float gmax = ma;
+            for (int o = 16; o; o >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
             float tau = -INFINITY;
             if (k <= NW) {
-                float ma = lane < NW ? ms->wmax[lane] : -INFINITY;
                 int above = 0;
+#pragma unroll
                 for (int b = 0; b < NW; ++b) {
                     float mb = ms->wmax[b];
                     above += (mb > ma) || (mb == ma && b < lane);
@@ -451,27 +607,45 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 unsigned hit = __ballot_sync(0xffffffffu, lane < NW && above == k - 1);
                 tau = __shfl_sync(0xffffffffu, ma, __ffs(hit) - 1);
             }
-            for (int e = tid; e < E; e += NT) {
-                float v = lg[e];
-                if (v >= tau) {
-                    int slot = atomicAdd(&ms->ncand, 1);
-                    if (slot < CAND_MAX) {
-                        ms->cand_v[slot] = v;
-                        ms->cand_id[slot] = e;
-                    }
+            // candidates (logit >= tau), appended with one shared atomic per warp and pass
+            for (int e0 = 0; e0 < E; e0 += NT) {
+                const int e = e0 + tid;
+                const float v = e < E ? lg[e] : -INFINITY;
+                const bool take = e < E && v >= tau;
+                const unsigned bal = __ballot_sync(0xffffffffu, take);
+                if (bal) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&ms->ncand, __popc(bal));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const int slot = base + __popc(bal & ((1u << lane) - 1u));
+                    if (take && slot < CAND_MAX) ms->cand[slot] = make_float2(v, __int_as_float(e));
                 }
             }
             __syncthreads();
-            int nc = ms->ncand;
+            const int nc = ms->ncand;
             if (nc <= CAND_MAX) {
+                // rank of candidate t = number of candidates ordered before it (value desc, id asc)
                 if (tid < nc) {
-                    float v = ms->cand_v[tid];
-                    int id = ms->cand_id[tid];
-                    int rank = 0;
-                    for (int j = 0; j < nc; ++j) rank += better(ms->cand_v[j], ms->cand_id[j], v, id);
+                    const float2 me = ms->cand[tid];
+                    const float v = me.x;
+                    const int id = __float_as_int(me.y);
+                    int rank = 0, j = 0;
+                    for (; j + 4 <= nc; j += 4) {
+                        const float4 c01 = *reinterpret_cast<const float4 *>(&ms->cand[j]);
+                        const float4 c23 = *reinterpret_cast<const float4 *>(&ms->cand[j + 2]);
+                        rank += better(c01.x, __float_as_int(c01.y), v, id) +
+                                better(c01.z, __float_as_int(c01.w), v, id) +
+                                better(c23.x, __float_as_int(c23.y), v, id) +
+                                better(c23.z, __float_as_int(c23.w), v, id);
+                    }
+                    for (; j < nc; ++j) {
+                        const float2 o = ms->cand[j];
+                        rank += better(o.x, __float_as_int(o.y), v, id);
+                    }
                     if (rank < k) {
                         ms->ids[rank] = id;
-                        ms->vsel[rank] = v;
+                        ms->uexp[rank] = id;
+                        ms->psel[rank] = expf(v - gmax);
                     }
                 }
             } else if (warp == 0) {
@@ -497,37 +671,10 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     }
                     if (lane == 0) {
                         ms->ids[j] = bid;
-                        ms->vsel[j] = bv;
+                        ms->uexp[j] = bid;
+                        ms->psel[j] = expf(bv - gmax);
                     }
                     __syncwarp();
-                }
-            }
-            __syncthreads();
-            trace_mark(p, l, 9, clock64() - tl0);
-            if (warp == 0) {
-                float top = ms->vsel[0];
-                float pj = lane < k ? expf(ms->vsel[lane] - top) : 0.f;
-                float z = pj;
-                for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-                if (lane < k) {
-                    float wj = pj / z;
-                    ms->wsel[lane] = wj;
-                    ms->uexp[lane] = ms->ids[lane];
-                    ms->uw[lane] = wj;
-                    if (cta == 0) {
-                        if (p.stack && p.rec_on) {
-                            if (p.rec.ids) p.rec.ids[(size_t)l * k + lane] = ms->ids[lane];
-                            if (p.rec.w) p.rec.w[(size_t)l * k + lane] = wj;
-                        }
-                        if (!p.stack) {
-                            if (p.ids_out) p.ids_out[lane] = ms->ids[lane];
-                            if (p.w_out) p.w_out[lane] = wj;
-                        }
-                    }
-                }
-                if (lane < p.nsh) {
-                    ms->uexp[k + lane] = E + lane;
-                    ms->uw[k + lane] = 1.f;
                 }
             }
             __syncthreads();
@@ -556,6 +703,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 const uint8_t *src = Lp.gu + (size_t)ms->uexp[us] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
                 mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
                 bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
+                gu_par ^= 1u << s;
             } else {
                 int q0 = (q - n_gu) * dn_per_slot;
                 int cnt = min(dn_per_slot, n_dn - q0);
@@ -575,16 +723,60 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             for (int q = 0; q < first; ++q) issue_item(q);
         }
         item += n_items;
+        // routing weights (needed from the down flush on): renormalised over the selected
+        // experts, in rank order
+        if (warp == NW - 1) {
+            const float pj = lane < k ? ms->psel[lane] : 0.f;
+            float z = pj;
+            for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            if (lane < k) {
+                const float wj = pj / z;
+                const int id = ms->ids[lane];
+                ms->uw[lane] = wj;
+                if (cta == 0) {
+                    if (p.stack && p.rec_on) {
+                        if (p.rec.ids) p.rec.ids[(size_t)l * k + lane] = id;
+                        if (p.rec.w) p.rec.w[(size_t)l * k + lane] = wj;
+                    }
+                    if (!p.stack) {
+                        if (p.ids_out) p.ids_out[lane] = id;
+                        if (p.w_out) p.w_out[lane] = wj;
+                    }
+                }
+            }
+        }
+
+        // producer, while the gate/up warps work: each down batch that did not fit the ring
+        // goes into a slot as soon as that slot's gate/up unit is consumed (its previous item
+        // is always a gate/up unit of this layer), then the next layer's router rows, so that
+        // no bulk copy is in flight during the exchanges that follow
+        if (tid == PRODUCER) {
+            bool pok = true;
+            for (int q = p.nslot; q < n_items && pok; ++q) {
+                const int s = (int)((item_base + q) % p.nslot);
+                pok = mbar_wait(&ms->empty[s], ((gu_par >> s) & 1u) ^ 1u, err, true);
+                if (pok) {
+                    fence_proxy_async();
+                    issue_item(q);
+                }
+            }
+            if (pok && l + 1 < p.L) {
+                issue_router(layer + 1);
+                ++router_issued;
+            }
+        }
 
         // gate/up B fragments of this warp's 256-wide k chunk (token in one column per block)
+        // (Q4: fp16 x * 2^s, Q3: bf16 x)
         uint32_t bx0[16], bx1[16];
         if (warp < GW) {
+            const uint16_t *xop = (FMT == MOE_Q4B32) ? xh : xb;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 int s = 16 * warp + j;
                 bool act = (g == (j >> 1));
-                uint32_t v0 = *reinterpret_cast<const uint32_t *>(xb + 16 * s + 2 * c);
-                uint32_t v1 = *reinterpret_cast<const uint32_t *>(xb + 16 * s + 2 * c + 8);
+                uint32_t v0 = *reinterpret_cast<const uint32_t *>(xop + 16 * s + 2 * c);
+                uint32_t v1 = *reinterpret_cast<const uint32_t *>(xop + 16 * s + 2 * c + 8);
                 bx0[j] = act ? v0 : 0u;
                 bx1[j] = act ? v1 : 0u;
             }
@@ -612,8 +804,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 #pragma unroll
                         for (int m = 0; m < 4; ++m) {
                             uint32_t a0, a1, a2, a3;
-                            q4_frag(wv[m], a0, a1, a2, a3);
-                            mma16816((m & 1) ? D1 : D0, a0, a1, a2, a3, bx0[4 * kq + m], bx1[4 * kq + m]);
+                            q4_frag_h(wv[m], a0, a1, a2, a3);
+                            mma16816_h((m & 1) ? D1 : D0, a0, a1, a2, a3, bx0[4 * kq + m], bx1[4 * kq + m]);
                         }
                     }
                 } else {
@@ -633,9 +825,18 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 int b0 = 8 * warp + 2 * c;
                 float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + b0));
                 float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + b0));
-                const float o0 = off * xsum[b0], o1 = off * xsum[b0 + 1];
-                float ag = fmaf(sg.x, D0[0] + D1[0] - o0, sg.y * (D0[1] + D1[1] - o1));
-                float a8 = fmaf(s8.x, D0[2] + D1[2] - o0, s8.y * (D0[3] + D1[3] - o1));
+                float ag, a8;
+                if constexpr (FMT == MOE_Q4B32) {
+                    // row g: codes read as 1024 + q; row g+8: as 1024 + 16 q (sums scaled by 1/16)
+                    const float x0 = xsum[b0], x1 = xsum[b0 + 1];
+                    ag = fmaf(sg.x, D0[0] + D1[0] - 1032.f * x0, sg.y * (D0[1] + D1[1] - 1032.f * x1));
+                    a8 = fmaf(s8.x, fmaf(D0[2] + D1[2], 0.0625f, -72.f * x0),
+                              s8.y * fmaf(D0[3] + D1[3], 0.0625f, -72.f * x1));
+                } else {
+                    const float o0 = off * xsum[b0], o1 = off * xsum[b0 + 1];
+                    ag = fmaf(sg.x, D0[0] + D1[0] - o0, sg.y * (D0[1] + D1[1] - o1));
+                    a8 = fmaf(s8.x, D0[2] + D1[2] - o0, s8.y * (D0[3] + D1[3] - o1));
+                }
                 ag += __shfl_xor_sync(0xffffffffu, ag, 1);
                 a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
                 ag += __shfl_xor_sync(0xffffffffu, ag, 2);
@@ -644,17 +845,18 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     red[(q * NW + warp) * 16 + g] = ag;
                     red[(q * NW + warp) * 16 + 8 + g] = a8;
                 }
-                if (q < 6) trace_mark(p, l, 16 + q, clock64() - tw1);
+                if (q < 5) trace_mark(p, l, 16 + q, clock64() - tw1);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ms->empty[s]);   // this warp is done with the slot
             }
         }
-        if (cta_failed(ms, ok)) break;
+        trace_mark(p, l, 11, clock64() - tl0);   // thread 0's own gate/up units done
+        if (cta_failed(ok)) {
+            aborted = true;
+            break;
+        }
         trace_mark(p, l, 6, clock64() - tl0);
         consumed += n_gu;
-        // the gate/up slots are free: queue the down batches that did not fit the ring yet
-        if (tid == PRODUCER) {
-            fence_proxy_async();
-            for (int q = p.nslot; q < n_items && q < n_gu + p.nslot; ++q) issue_item(q);
-        }
         // SwiGLU of every gate/up unit in parallel: thread (unit q, row i)
         if (tid < n_gu * 8) {
             int q = tid >> 3, i = tid & 7;
@@ -663,101 +865,129 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 gs += red[(q * NW + w) * 16 + i];
                 us_ += red[(q * NW + w) * 16 + 8 + i];
             }
+            const float xinv = ms->xinv;
+            gs *= xinv;
+            us_ *= xinv;
             int u = cta + G * q;
             int uslot = u / ntile_gu, t = u % ntile_gu;
-            ll_store(p.ll_h + ((size_t)lpar * MAXU + uslot) * I + 8 * t + i, silu(gs) * us_, ep);
+            p.x_h[(size_t)uslot * I + 8 * t + i] = silu(gs) * us_;
         }
         trace_mark(p, l, 3, clock64() - tl0);
 
-        // h of every expert in use -> fp16 hi + lo table
+        // h of every expert in use -> bf16 hi + lo table and per-block sums of hi + lo
         {
-            ok = poll_words<8>(p.ll_h + (size_t)lpar * MAXU * I, nU * I, ep, err, [&](int i, float h) {
-                uint16_t hi = bf16_rn_bits(h);
-                uint16_t lo = bf16_rn_bits(h - bf16_bits_f(hi));
-                int us = i / I, kk = i % I;
-                htab[(size_t)(2 * us) * I + kk] = hi;
-                htab[(size_t)(2 * us + 1) * I + kk] = lo;
-            });
-            if (cta_failed(ms, ok)) break;
-            for (int t = tid; t < nU * nbi; t += NT) {
-                int us = t / nbi, b = t % nbi;
-                hsum[t] = sum32_bf16(htab + (size_t)(2 * us) * I + 32 * b) +
-                          sum32_bf16(htab + (size_t)(2 * us + 1) * I + 32 * b);
+            __syncthreads();   // this CTA's h values are stored
+            if (tid == 0) {
+                xchg_arrive(p, X_H);
+                ok = ctr_wait(ctr(p, X_H), (unsigned)G, err);
+            }
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
+            // 4 values per thread; the 8 lanes of a 32-block are neighbours in the warp
+            const int n4 = nU * I / 4;   // a multiple of 8 (I % 64 == 0)
+            for (int b4 = 0; b4 < n4; b4 += NT) {
+                const int i4 = b4 + tid;
+                const bool valid = i4 < n4;
+                float part = 0.f;
+                if (valid) {
+                    const float4 h = ld_gpu4(p.x_h + 4 * i4);
+                    const float hv[4] = {h.x, h.y, h.z, h.w};
+                    uint32_t hi2[2], lo2[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint16_t h0 = bf16_rn_bits(hv[2 * j]), h1 = bf16_rn_bits(hv[2 * j + 1]);
+                        const uint16_t l0 = bf16_rn_bits(hv[2 * j] - bf16_bits_f(h0));
+                        const uint16_t l1 = bf16_rn_bits(hv[2 * j + 1] - bf16_bits_f(h1));
+                        hi2[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                        lo2[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                        part += (bf16_bits_f(h0) + bf16_bits_f(l0)) + (bf16_bits_f(h1) + bf16_bits_f(l1));
+                    }
+                    const int i = 4 * i4, us = i / I, kk = i - us * I;
+                    *reinterpret_cast<uint2 *>(htab + (size_t)(2 * us) * I + kk) = make_uint2(hi2[0], hi2[1]);
+                    *reinterpret_cast<uint2 *>(htab + (size_t)(2 * us + 1) * I + kk) = make_uint2(lo2[0], lo2[1]);
+                }
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                part += __shfl_xor_sync(0xffffffffu, part, 4);
+                if (valid && (lane & 7) == 0) hsum[i4 >> 3] = part;   // block (us, b) = us * nbi + b
             }
             __syncthreads();
         }
         trace_mark(p, l, 4, clock64() - tl0);
 
-        // ---- down: every warp with a k group walks all down units of this CTA's contiguous
-        // run [dn_lo, dn_hi) ((tile, expert) order); partials to red[unit][warp][row]
-        if (warp < DW) {
-            for (int qi = 0; qi < n_dn_items && ok; ++qi) {
-                long long it = item_base + n_gu + qi;
-                int s = (int)(it % p.nslot);
-                long long tw0 = clock64();
-                ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
-                tw_dn += clock64() - tw0;
-                if (!ok) break;
-                int q0 = qi * dn_per_slot;
-                int cnt = min(dn_per_slot, n_dn - q0);
-                for (int ui = 0; ui < cnt; ++ui) {
-                    int nl = q0 + ui, n = dn_lo + nl;
-                    int us = n % nU;
-                    const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
-                    float D[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint16_t *hp = htab + (size_t)(2 * us + (g & 1)) * I;
+        // ---- down: warp w takes this CTA's units w, w+NW, ... of the contiguous run
+        // [dn_lo, dn_hi) ((tile, expert) order) over the whole K = I, with one accumulator per
+        // group of four 32-blocks; the unit's 16 sums go to vsum[unit][row]
+        float *vsum = red;   // [unit][16]
+        for (int nl = warp; nl < n_dn && ok; nl += NW) {
+            const int qi = nl / dn_per_slot, ui = nl - qi * dn_per_slot;
+            const long long it = item_base + n_gu + qi;
+            const int s = (int)(it % p.nslot);
+            long long tw0 = clock64();
+            ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
+            tw_dn += clock64() - tw0;
+            if (!ok) break;
+            const int us = (dn_lo + nl) % nU;
+            const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
+            const uint16_t *hp = htab + (size_t)(2 * us + (g & 1)) * I;   // column g: hi (even) / lo (odd)
+            float D[6][4];   // up to 12 k groups (I <= 768)
+#pragma unroll
+            for (int j = 0; j < 6; ++j) D[j][0] = D[j][1] = D[j][2] = D[j][3] = 0.f;
+#pragma unroll
+            for (int kg = 0; kg < 12; ++kg) {
+                if (kg < DW) {
                     uint32_t a[16];
                     if constexpr (FMT == MOE_Q4B32) {
-                        uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)warp * 512 + lane * 16);
+                        uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)kg * 512 + lane * 16);
                         q4_frag(av.x, a[0], a[1], a[2], a[3]);
                         q4_frag(av.y, a[4], a[5], a[6], a[7]);
                         q4_frag(av.z, a[8], a[9], a[10], a[11]);
                         q4_frag(av.w, a[12], a[13], a[14], a[15]);
                     } else {
-                        const uint32_t *wp = reinterpret_cast<const uint32_t *>(tile + (size_t)warp * 384 + lane * 12);
+                        const uint32_t *wp = reinterpret_cast<const uint32_t *>(tile + (size_t)kg * 384 + lane * 12);
                         q3_frag(wp[0], wp[1], wp[2], a);
                     }
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        int sl = 4 * warp + m;           // k16 slice within K = I
-                        bool act = ((sl >> 1) & 3) == (g >> 1);
+                        const int sl = 4 * kg + m;           // k16 slice within K = I
+                        const bool act = ((sl >> 1) & 3) == (g >> 1);
                         uint32_t b0 = act ? *reinterpret_cast<const uint32_t *>(hp + 16 * sl + 2 * c) : 0u;
                         uint32_t b1 = act ? *reinterpret_cast<const uint32_t *>(hp + 16 * sl + 2 * c + 8) : 0u;
-                        mma16816(D, a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
-                    }
-                    // columns 2c (hi) and 2c+1 (lo) of block 4*(warp/2) + c
-                    int blk = 4 * (warp >> 1) + c;
-                    bool valid = (c >> 1) == (warp & 1);
-                    float ag = 0.f, a8 = 0.f;
-                    if (valid) {
-                        const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
-                        const float o = off * hsum[us * nbi + blk];
-                        ag = __half2float(sc[g * nbi + blk]) * (D[0] + D[1] - o);
-                        a8 = __half2float(sc[(g + 8) * nbi + blk]) * (D[2] + D[3] - o);
-                    }
-                    ag += __shfl_xor_sync(0xffffffffu, ag, 1);
-                    a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
-                    ag += __shfl_xor_sync(0xffffffffu, ag, 2);
-                    a8 += __shfl_xor_sync(0xffffffffu, a8, 2);
-                    if (c == 0) {
-                        red[(nl * DW + warp) * 16 + g] = ag;
-                        red[(nl * DW + warp) * 16 + 8 + g] = a8;
+                        mma16816(D[kg >> 1], a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
                     }
                 }
             }
+            // accumulator j, columns 2c (hi) and 2c+1 (lo): block 4j + c
+            const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
+            float ag = 0.f, a8 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 6; ++j) {
+                const int blk = 4 * j + c;
+                if (blk < nbi) {
+                    const float o = off * hsum[us * nbi + blk];
+                    ag = fmaf(__half2float(sc[g * nbi + blk]), D[j][0] + D[j][1] - o, ag);
+                    a8 = fmaf(__half2float(sc[(g + 8) * nbi + blk]), D[j][2] + D[j][3] - o, a8);
+                }
+            }
+            ag += __shfl_xor_sync(0xffffffffu, ag, 1);
+            a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
+            ag += __shfl_xor_sync(0xffffffffu, ag, 2);
+            a8 += __shfl_xor_sync(0xffffffffu, a8, 2);
+            if (c == 0) {
+                vsum[nl * 16 + g] = ag;
+                vsum[nl * 16 + 8 + g] = a8;
+            }
         }
-        if (cta_failed(ms, ok)) break;
+        trace_mark(p, l, 9, clock64() - tl0);   // thread 0's own down units done
+        if (cta_failed(ok)) {
+            aborted = true;
+            break;
+        }
         consumed += n_dn_items;
         trace_mark(p, l, 7, clock64() - tl0);
-        // unit sums (thread per (unit, row)), then per tile the fixed-order weighted sum
-        float *vsum = red + (size_t)p.dn_units_max * DW * 16;   // [unit][16]
-        for (int t = tid; t < n_dn * 16; t += NT) {
-            int nl = t >> 4, r = t & 15;
-            float v = 0.f;
-            for (int w = 0; w < DW; ++w) v += red[(nl * DW + w) * 16 + r];
-            vsum[t] = v;
-        }
-        __syncthreads();
+        // per tile the fixed-order weighted sum of its units
         {
             int j_first = dn_lo / nU, j_last = (dn_hi - 1) / nU;
             int n_tiles_mine = j_last - j_first + 1;
@@ -768,10 +998,11 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 float y = 0.f;
                 for (int n = n0; n <= n1; ++n) y = fmaf(ms->uw[n % nU], vsum[(n - dn_lo) * 16 + r], y);
                 int part = (first >= dn_lo) ? 0 : 1;
-                uint2 *yb = p.ll_y + (size_t)lpar * 2 * d;
-                ll_store(yb + (size_t)part * d + 16 * j + r, y, ep);
-                if (part == 0 && last < dn_hi) ll_store(yb + d + 16 * j + r, 0.f, ep);
+                p.x_y[(size_t)part * d + 16 * j + r] = y;
+                if (part == 0 && last < dn_hi) p.x_y[d + 16 * j + r] = 0.f;
             }
+            __syncthreads();   // this CTA's output parts are stored
+            if (tid == 0) xchg_arrive(p, X_Y);
         }
         trace_mark(p, l, 5, clock64() - tl0);
         trace_mark(p, l, 10, tw_gu);
@@ -779,26 +1010,30 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     }
 
     // ---- outputs of the last layer ---------------------------------------------------
-    if (!ms->abort && ok) {
+    if (!aborted && cta == 0) {
         const int l = p.L - 1;
-        const uint32_t ep = p.epoch0 + (uint32_t)l;
-        const uint2 *y0 = p.ll_y + (size_t)(l & 1) * 2 * d;
-        if (cta == 0) {
-            ok = poll_words<4>(y0, d, ep, err, [&](int i, float v) { ybuf[i] = v; });
-            ok = ok && poll_words<4>(y0 + d, d, ep, err, [&](int i, float v) {
-                float y = ybuf[i] + v;
-                uint16_t yb = bf16_rn_bits(y);
-                if (p.stack) {
-                    p.resid_out[i] = rs[i] + bf16_bits_f(yb);
-                    if (p.rec_on) {
-                        if (p.rec.y_bf16) p.rec.y_bf16[(size_t)l * d + i] = yb;
-                        if (p.rec.y_f32) p.rec.y_f32[(size_t)l * d + i] = y;
+        if (tid == 0) ok = ctr_wait(ctr(p, X_Y), (unsigned)G, err);
+        if (!cta_failed(ok)) {
+            for (int i4 = tid; i4 < d / 4; i4 += NT) {
+                const float4 a = ld_gpu4(p.x_y + 4 * i4), b = ld_gpu4(p.x_y + d + 4 * i4);
+                const float ya[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = 4 * i4 + j;
+                    const float y = ya[j];
+                    const uint16_t yb = bf16_rn_bits(y);
+                    if (p.stack) {
+                        p.resid_out[i] = rs[i] + bf16_bits_f(yb);
+                        if (p.rec_on) {
+                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)l * d + i] = yb;
+                            if (p.rec.y_f32) p.rec.y_f32[(size_t)l * d + i] = y;
+                        }
+                    } else {
+                        p.y_out[i] = yb;
+                        if (p.yf_out) p.yf_out[i] = y;
                     }
-                } else {
-                    p.y_out[i] = yb;
-                    if (p.yf_out) p.yf_out[i] = y;
                 }
-            });
+            }
         }
     }
     // drain copies still in flight (abort path) before the CTA's shared memory goes away
@@ -816,8 +1051,9 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 bool decode_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
     if (T != 1 || (c.flags & MOE_FLAG_NO_DECODE_KERNEL)) return false;
-    if (c.n_experts % 2) return false;   // flagged words are polled in 16-byte pairs
-    if (c.d_model > 4096 || c.d_model / 256 > NW || c.d_ff / 64 > NW) return false;
+    // gate/up k chunks go to warps 0..d/256-1; the last warp must stay free for the producer
+    if (c.d_model > 4096 || c.d_model / 256 > NW - 1 || c.d_ff / 64 > 12) return false;
+    if (c.n_experts % 4) return false;   // logits region of the exchange area stays 16-byte aligned
     if (c.top_k > MAXK || c.top_k + c.n_shared > MAXU) return false;
     return ctx->dec.smem_bytes > 0;
 }
@@ -852,14 +1088,14 @@ int decode_setup(moe_ctx *ctx) {
     int dn_max = (nU * (c.d_model / 16) + G - 1) / G;
     size_t red_bytes = (size_t)8 * NW * 4;                                   // router partials
     if (red_bytes < (size_t)gu_max * NW * 16 * 4) red_bytes = (size_t)gu_max * NW * 16 * 4;
-    if (red_bytes < (size_t)dn_max * (NW + 1) * 16 * 4) red_bytes = (size_t)dn_max * (NW + 1) * 16 * 4;
+    if (red_bytes < (size_t)dn_max * 16 * 4) red_bytes = (size_t)dn_max * 16 * 4;   // down unit sums
     ds.gu_units_max = gu_max;
     ds.dn_units_max = dn_max;
     ds.off_router = take((size_t)rpc * c.d_model * 4);
     ds.off_x16 = take((size_t)c.d_model * 2);
+    ds.off_xh = take((size_t)c.d_model * 2);
     ds.off_logits = take((size_t)c.n_experts * 4);
-    size_t htab = (size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2;   // fp16 hi + lo of h
-    if (htab < (size_t)c.d_model * 4) htab = (size_t)c.d_model * 4;    // doubles as the y buffer
+    size_t htab = (size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2;   // bf16 hi + lo of h
     ds.off_htab = take(htab);
     ds.off_red = take(red_bytes);
     ds.off_misc = take(sizeof(Misc));
@@ -887,9 +1123,12 @@ int decode_setup(moe_ctx *ctx) {
     return MOE_OK;
 }
 
-size_t decode_ll_bytes(const moe_config &c) {
-    return sizeof(uint2) * ((size_t)2 * c.n_experts + (size_t)2 * MAXU * c.d_ff + (size_t)4 * c.d_model);
-}
+// Exchange area: 3 counters (128 bytes apart), logits [E], h [MAXU][I], output parts [2][d].
+constexpr size_t XB_LOGITS = 384;
+static size_t xb_h_off(const moe_config &c) { return XB_LOGITS + (((size_t)c.n_experts * 4 + 127) & ~(size_t)127); }
+static size_t xb_y_off(const moe_config &c) { return xb_h_off(c) + (size_t)MAXU * c.d_ff * 4; }
+size_t decode_xchg_bytes(const moe_config &c) { return xb_y_off(c) + (size_t)2 * c.d_model * 4; }
+size_t decode_xchg_counter_bytes() { return XB_LOGITS; }
 
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
@@ -920,14 +1159,14 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
         p.rec = *rec;
         p.rec_on = 1;
     }
-    p.ll_logits = ds.ll;
-    p.ll_h = ds.ll + (size_t)2 * c.n_experts;
-    p.ll_y = p.ll_h + (size_t)2 * MAXU * c.d_ff;
-    p.epoch0 = ds.epoch;
-    ds.epoch += (uint32_t)L + 1;
-    if (ds.epoch < (uint32_t)L + 2) ds.epoch = 1;   // wrapped: never reuse 0 (initial contents)
+    p.cnt = reinterpret_cast<unsigned *>(ds.xbuf);
+    p.x_logits = reinterpret_cast<float *>(ds.xbuf + XB_LOGITS);
+    p.x_h = reinterpret_cast<float *>(ds.xbuf + xb_h_off(c));
+    p.x_y = reinterpret_cast<float *>(ds.xbuf + xb_y_off(c));
     p.err = ctx->ws.dev_error;
-    p.withhold = (c.flags & MOE_FLAG_TEST_WITHHOLD) ? 1 : 0;
+    // test hook: the context's first single-token call withholds CTA 0's logits
+    p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ds.withheld) ? 1 : 0;
+    if (p.withhold) ds.withheld = true;
     if (c.flags & MOE_FLAG_TRACE) {
         size_t need = (size_t)ds.grid * L * TRACE_WORDS;
         if (need > ds.trace_cap) {
@@ -950,6 +1189,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_ring = ds.off_ring;
     p.off_router = ds.off_router;
     p.off_x16 = ds.off_x16;
+    p.off_xh = ds.off_xh;
     p.off_logits = ds.off_logits;
     p.off_htab = ds.off_htab;
     p.off_red = ds.off_red;

@@ -135,9 +135,9 @@ int alloc_workspace(moe_ctx *ctx) {
     QE_TRY(ctx_alloc(ctx, (void **)&ctx->d_layers, sizeof(LayerPtrs) * c.n_layers, "layer table"));
     QE_CHECK(cudaMemset(ctx->d_layers, 0, sizeof(LayerPtrs) * c.n_layers));
     QE_TRY(decode_setup(ctx));
-    size_t llb = decode_ll_bytes(c);
-    QE_TRY(ctx_alloc(ctx, (void **)&ctx->dec.ll, llb, "flag buffers"));
-    QE_CHECK(cudaMemset(ctx->dec.ll, 0, llb));
+    size_t xb = decode_xchg_bytes(c);
+    QE_TRY(ctx_alloc(ctx, (void **)&ctx->dec.xbuf, xb, "exchange area"));
+    QE_CHECK(cudaMemset(ctx->dec.xbuf, 0, xb));
     return MOE_OK;
 }
 
@@ -362,6 +362,9 @@ int moe_get_device_error(moe_ctx *ctx, int *code) {
     QE_CHECK(cudaDeviceSynchronize());
     QE_CHECK(cudaMemcpy(code, ctx->ws.dev_error, 4, cudaMemcpyDeviceToHost));
     QE_CHECK(cudaMemset(ctx->ws.dev_error, 0, 4));
+    // a kernel that gave up part-way leaves the decode kernel's arrival counters
+    // mid-count: start them again from zero
+    if (*code != 0 && ctx->dec.xbuf) QE_CHECK(cudaMemset(ctx->dec.xbuf, 0, decode_xchg_counter_bytes()));
     return MOE_OK;
 }
 

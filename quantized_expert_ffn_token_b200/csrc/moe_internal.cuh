@@ -165,11 +165,11 @@ struct DecodeState {
     int smem_bytes = 0;   // 0: the shape does not fit the kernel
     int nslot = 0, slot_bytes = 0, rpc = 0;
     int gu_units_max = 0, dn_units_max = 0;   // per-CTA unit counts the carve is sized for
-    int off_ring = 0, off_router = 0, off_x16 = 0, off_logits = 0, off_htab = 0, off_red = 0,
+    int off_ring = 0, off_router = 0, off_x16 = 0, off_xh = 0, off_logits = 0, off_htab = 0, off_red = 0,
         off_misc = 0, off_resid = 0, off_sums = 0;
     int sms = 0;          // streaming multiprocessors of the device
-    uint2 *ll = nullptr;  // flagged-word exchange buffers
-    uint32_t epoch = 1;
+    uint8_t *xbuf = nullptr;   // cross-CTA exchange area (counters, logits, h, output parts)
+    bool withheld = false;     // the MOE_FLAG_TEST_WITHHOLD call has been made
     unsigned long long *trace = nullptr;   // phase clocks (MOE_FLAG_TRACE)
     size_t trace_cap = 0;                  // records allocated
     int trace_n = 0;                       // records of the last call
@@ -254,7 +254,8 @@ int launch_resid_norm(const moe_ctx *ctx, int T, float *resid, const uint16_t *y
                       const uint16_t *x_in, uint16_t *x_out, cudaStream_t st);
 bool decode_supported(const moe_ctx *ctx, int T);
 int decode_setup(moe_ctx *ctx);
-size_t decode_ll_bytes(const moe_config &c);
+size_t decode_xchg_bytes(const moe_config &c);
+size_t decode_xchg_counter_bytes();   // the counters at the start of the exchange area
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
                   cudaStream_t st);

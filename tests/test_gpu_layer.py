@@ -91,7 +91,13 @@ def test_batch_equals_single_tokens():
 @pytest.mark.parametrize("name", ["tiny_d256_e16_q4_t8", "decode_48l_q4_t1"])
 def test_decode_kernel_matches_general_path(name):
     """Single-token calls: the persistent decode kernel against the general
-    grouped path on the same inputs (same ids; fp32 outputs within 1e-5)."""
+    grouped path on the same inputs (same ids; fp32 outputs within 5e-5).
+
+    The decode kernel reads Q4 codes as fp16 1024 + q and removes 1032 x the
+    block sum of the input from each fp32 block partial afterwards; that
+    cancellation leaves about 2^-16 of relative error per partial (the offset
+    term is ~2^8 times the useful one), so the two paths agree to a few 1e-5,
+    not to fp32 rounding."""
     capi, session = _cuda()
     cfg = synth.CONFIGS[name]
     a = session.Session(cfg, max_tokens=4, n_layers=1)
@@ -106,9 +112,36 @@ def test_decode_kernel_matches_general_path(name):
         yb, yfb, idb, wb = _run(b, 0, x)
         assert np.array_equal(ida, idb)
         assert np.max(np.abs(wa - wb)) <= 1e-6
-        assert rel_l2(yfa, yfb) <= 1e-5
+        assert rel_l2(yfa, yfb) <= 5e-5
     a.close()
     b.close()
+
+
+def test_decode_wait_times_out_and_context_recovers():
+    """A bounded device wait that runs out, and recovery: with the test hook,
+    CTA 0 of the single-token kernel withholds its router logits in the
+    context's first call, every CTA's wait on them gives up after about a
+    second, moe_get_device_error reports MOE_ERR_DEVICE_TIMEOUT (and resets the
+    kernel's arrival counters), and the next call on the same context matches
+    the general path again."""
+    capi, session = _cuda()
+    s = session.Session(TINY, max_tokens=4, n_layers=1, flags=capi.MOE_FLAG_TEST_WITHHOLD)
+    ref = session.Session(TINY, max_tokens=4, n_layers=1, flags=capi.MOE_FLAG_NO_DECODE_KERNEL)
+    W = synth.layer_weights(TINY, 0, device="cuda")
+    s.load(0, W)
+    ref.load(0, W)
+    del W
+    x = _tokens(TINY, 1, stream=77)
+    _run(s, 0, x)
+    assert capi.moe_get_device_error(s.ctx) == capi.MOE_ERR_DEVICE_TIMEOUT
+    for rep in range(3):
+        y, yf, ids, w = _run(s, 0, x)
+        assert capi.moe_get_device_error(s.ctx) == 0
+        yb, yfb, idb, wb = _run(ref, 0, x)
+        assert np.array_equal(ids, idb)
+        assert rel_l2(yf, yfb) <= 5e-5
+    s.close()
+    ref.close()
 
 
 def _tiny_weights_with(mutate):
