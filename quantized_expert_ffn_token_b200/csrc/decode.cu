@@ -1,5 +1,8 @@
 // Single-token decode: one persistent kernel runs whole layers (and the whole
-// 48-layer stack) with one CTA per SM.
+// 48-layer stack) with one CTA per SM: 12 compute warps, which synchronise on
+// a named barrier, and one producer warp that issues every bulk copy and is
+// paced by mbarriers only (a thread that issues copies can stall while the
+// copy engine's queue drains; the compute warps must not wait for it).
 //
 // Per layer (one token):
 //   1. every CTA rebuilds the layer input from the previous layer's output
@@ -20,7 +23,8 @@
 //      is removed with the block sums of x and the block's fp16 scale applied
 //      in fp32; the SwiGLU output h is exchanged;
 //   5. down: units are (16 output rows, expert), one warp per unit over the
-//      whole K; h enters as bf16 hi + lo (h to about 2^-16 relative), and a
+//      whole K; h enters as hi + lo parts (Q4: fp16 of h * 2^s with s per
+//      32-block, about 2^-22 relative; Q3: bf16, about 2^-16), and a
 //      CTA's contiguous run of units, weighted by the routing weights, is
 //      summed per 16-row tile into one of at most two parts per tile; the next
 //      layer adds the two parts in order.
@@ -41,19 +45,23 @@ namespace qeffn {
 
 namespace {
 
-constexpr int NT = 384;
+constexpr int NT = 384;             // compute threads (12 warps)
 constexpr int NW = NT / 32;
-constexpr int PRODUCER = NT - 32;   // lane 0 of the last warp issues every bulk copy
+constexpr int NTT = NT + 32;        // plus one producer warp: its lane 0 issues every bulk copy
 constexpr int MAX_SLOTS = 8;
 constexpr int MAXK = 32;
 constexpr int MAXU = MAXK + 4;
 constexpr int CAND_MAX = 256;
+constexpr int YMAX = 3;    // float4 groups of the output per thread (d <= 4096)
+constexpr int EMAX = 3;    // logits per thread (E <= 1024)
+constexpr int HB = 4;      // float4 loads of h in flight per thread
 constexpr long long SPIN_LIMIT = 2000000000LL;   // clock64 cycles, about one second
 
 struct Misc {
     unsigned long long full[MAX_SLOTS];
     unsigned long long empty[MAX_SLOTS];   // gate/up item consumed by every gate/up warp
     unsigned long long rbar;
+    unsigned long long route;              // one arrival per layer: routing known (ids in uexp)
     int ids[MAXK];
     float psel[MAXK];          // exp(logit - max logit) of the selected experts, in rank order
     int uexp[MAXU];
@@ -144,33 +152,25 @@ __device__ __forceinline__ void mma16816_h(float *d, uint32_t a0, uint32_t a1, u
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// Code -> bf16 without arithmetic: a field OR-ed into the low mantissa bits of
-// 128.0 (0x4300) reads as 128 + q, exactly.  The offset is removed in fp32
-// from each 32-block's partial sum: sum_k (128 + q_k) v_k - (128 + zero) *
+// Q3B32 codes -> bf16 without arithmetic: a field OR-ed into the low mantissa
+// bits of 128.0 (0x4300) reads as 128 + q, exactly.  The offset is removed in
+// fp32 from each 32-block's partial sum: sum_k (128 + q_k) v_k - (128 + zero) *
 // sum_k v_k = sum_k (q_k - zero) v_k, with the block sums of the activations
-// precomputed once per layer (cancellation costs about 7 bits of the fp32
+// precomputed once per layer (cancellation costs about 5 bits of the fp32
 // partial, far below the output tolerance).
 constexpr uint32_t BF_MAGIC = 0x43004300u;
 
-// Q4B32: one word = the 8 codes of one k16 slice (nibble n = reg + 4*hi).
-__device__ __forceinline__ void q4_frag(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2,
-                                        uint32_t &a3) {
-    a0 = (w & 0x000F000Fu) | BF_MAGIC;
-    a1 = ((w >> 4) & 0x000F000Fu) | BF_MAGIC;
-    a2 = ((w >> 8) & 0x000F000Fu) | BF_MAGIC;
-    a3 = ((w >> 12) & 0x000F000Fu) | BF_MAGIC;
-}
-
-// Q4B32 into fp16 (gate/up): a nibble at bits 0-3 of a half under 1024.0
+// Q4B32 into fp16: a nibble at bits 0-3 of a half under 1024.0
 // (0x6400) reads as 1024 + q, one at bits 4-7 as 1024 + 16 q, both exact.  In
 // the fragment order registers a0/a2 (row g) take the first kind and a1/a3
 // (row g+8) the second, so the row g+8 partial sums come out 16x larger and
 // are scaled back in fp32; the offsets are 1024 + zero (row g) and
-// 1024/16 + zero (row g+8).  Five integer operations per eight codes.
+// 1024/16 + zero (row g+8).  Four ALU operations and one high multiply per
+// eight codes.
 constexpr uint32_t H_MAGIC = 0x64006400u;
 __device__ __forceinline__ void q4_frag_h(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2,
                                           uint32_t &a3) {
-    const uint32_t w8 = w >> 8;
+    const uint32_t w8 = __umulhi(w, 1u << 24);   // w >> 8 on the multiply pipe, off the integer ALU
     a0 = (w & 0x000F000Fu) | H_MAGIC;
     a1 = (w & 0x00F000F0u) | H_MAGIC;
     a2 = (w8 & 0x000F000Fu) | H_MAGIC;
@@ -213,6 +213,26 @@ __device__ __forceinline__ float sum32_bf16(const uint16_t *p) {
         for (int h = 0; h < 4; ++h) acc[h] += __uint_as_float(w[h] << 16) + __uint_as_float(w[h] & 0xFFFF0000u);
     }
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// B-fragment order of the h table (per expert, 256 * JN halves, JN = ceil(I/128)):
+// lane (g, c) of the down MMAs reads, for k-group pair j, the 8 halves
+// [sp][which][e] of slices 8j + 2 (g >> 1) + sp from row r = g & 1 (hi / lo),
+// register which (b0: k 2c, 2c+1; b1: k 2c+8, 2c+9), element e; one 16-byte load.
+// Index of the first half of (slice sl, lane column c, row r, register which).
+__device__ __forceinline__ int hfrag_index(int sl, int c, int r, int which, int JN) {
+    const int b4 = (sl >> 1) & 3, j = sl >> 3, sp = sl & 1;
+    return ((((b4 * 4 + c) * 2 + r) * JN + j) * 2 + sp) * 4 + which * 2;
+}
+// x * mask for a packed pair of fp16 (Q4) or bf16 (Q3) values, mask 1.0 or 0 in both
+// halves: zeroes the inactive block columns on the multiply pipe.
+__device__ __forceinline__ uint32_t hmul2_mask(int fmt, uint32_t x, uint32_t mask) {
+    uint32_t r;
+    if (fmt == MOE_Q4B32)
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(mask));
+    else
+        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(mask));
+    return r;
 }
 
 // Sum of 32 consecutive fp16 values (16-byte aligned).
@@ -306,9 +326,21 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *b, uint32_t parity
     }
 }
 
+// Barriers of the compute warps (named barrier 1, NT threads); the producer
+// warp never joins them and synchronises through mbarriers only.
+__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 // CTA-uniform abort decision after a phase: one barrier that also ORs the
-// threads' failures, so every thread leaves at the same barrier.
-__device__ __forceinline__ bool cta_failed(bool mine_ok) { return __syncthreads_or(!mine_ok) != 0; }
+// compute threads' failures, so every one of them leaves at the same barrier.
+__device__ __forceinline__ bool cta_failed(bool mine_ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"(mine_ok ? 0u : 1u), "n"(NT)
+        : "memory");
+    return r != 0;
+}
 
 // Trace record per (CTA, layer): word 0 = CTA, word 1 = layer, word 2 + slot =
 // SM clock cycles since the layer started in this CTA, except where noted:
@@ -320,23 +352,60 @@ __device__ __forceinline__ bool cta_failed(bool mine_ok) { return __syncthreads_
 //    4 every expert's h received           9 this thread's down units done
 //    7 every down unit done                5 output tiles published
 //   10 cycles waiting for gate/up data    12 cycles waiting for down data
-//   16..20 compute cycles of gate/up units 0..4 (warp 0)
+//   16 / 17 / 18 warp 0's first down unit: accumulation done / reduced /
+//      first k-group pair done (cycles since its data was ready)
+//   19, 20 compute cycles of gate/up units 0, 1 (warp 0)
 //   21 global timer (ns) at the layer start
 constexpr int TRACE_WORDS = 24;
 
+// Out of line: the record store is rare, and the kernel's code footprint per
+// layer is what the instruction cache sees.
+__device__ __noinline__ void trace_store(unsigned long long *trace, int L, int l, int ph, long long t) {
+    unsigned long long *r = trace + ((size_t)blockIdx.x * L + l) * TRACE_WORDS;
+    if (ph == 0) {
+        r[0] = blockIdx.x;
+        r[1] = l;
+    }
+    r[2 + ph] = (unsigned long long)t;
+}
 __device__ __forceinline__ void trace_mark(const DecodeParams &p, int l, int ph, long long t) {
-    if (p.trace && threadIdx.x == 0 && ph < TRACE_WORDS - 2) {
-        unsigned long long *r = p.trace + ((size_t)blockIdx.x * p.L + l) * TRACE_WORDS;
-        if (ph == 0) {
-            r[0] = blockIdx.x;
-            r[1] = l;
+    if (p.trace && threadIdx.x == 0 && ph < TRACE_WORDS - 2) trace_store(p.trace, p.L, l, ph, t);
+}
+
+// Top-k by k rounds of warp arg-max (warp 0), for the rare case of more
+// candidates than the ranking buffer holds (many equal logits).
+__device__ __noinline__ void topk_argmax_rounds(Misc *ms, const float *lg, int E, int k, float gmax) {
+    const int lane = threadIdx.x & 31;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bid = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            bool taken = false;
+            for (int q = 0; q < j; ++q) taken |= (ms->ids[q] == e);
+            if (!taken && better(lg[e], e, bv, bid)) {
+                bv = lg[e];
+                bid = e;
+            }
         }
-        r[2 + ph] = (unsigned long long)t;
+        for (int o = 16; o; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (lane == 0) {
+            ms->ids[j] = bid;
+            ms->uexp[j] = bid;
+            ms->psel[j] = expf(bv - gmax);
+        }
+        __syncwarp();
     }
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
+__global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *ring = smem + p.off_ring;
     float *rtr = reinterpret_cast<float *>(smem + p.off_router);
@@ -344,8 +413,10 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     uint16_t *xh = reinterpret_cast<uint16_t *>(smem + p.off_xh);          // layer input * 2^s, fp16 bits
     float *xsum = reinterpret_cast<float *>(smem + p.off_sums);              // [d/32] block sums of x
     float *hsum = xsum + p.d / 32;                                             // [nU][I/32] of h hi + lo
+    float *hinv = hsum + (p.k + p.nsh) * (p.I / 32);                           // [nU][I/32] Q4: 2^-s of the block
     float *lg = reinterpret_cast<float *>(smem + p.off_logits);
-    uint16_t *htab = reinterpret_cast<uint16_t *>(smem + p.off_htab);   // bf16 hi / lo of h
+    // h of every expert in use, hi and lo parts, in B-fragment order (see the down phase)
+    uint16_t *htab = reinterpret_cast<uint16_t *>(smem + p.off_htab);
     float *red = reinterpret_cast<float *>(smem + p.off_red);   // [2][NW][16]
     Misc *ms = reinterpret_cast<Misc *>(smem + p.off_misc);
     float *rs = reinterpret_cast<float *>(smem + p.off_resid);      // residual stream [d]
@@ -360,6 +431,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     const int GW = d / 256;              // warps with a gate/up K chunk (256 k each)
     const int DW = I / 64;               // warps with a down k group (64 k each)
     const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
+    const int JN = (I + 127) / 128;      // k-group pairs of the down K (h table blocks)
+    const uint32_t ONE2 = (FMT == MOE_Q4B32) ? 0x3C003C00u : 0x3F803F80u;   // 1.0 in both halves
     constexpr float off = (FMT == MOE_Q4B32) ? 136.f : 132.f;   // 128 + zero point
     int *err = p.err;
 
@@ -369,6 +442,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             mbar_init(&ms->empty[s], p.d / 256);   // one arrival per gate/up warp
         }
         mbar_init(&ms->rbar, 1);
+        mbar_init(&ms->route, 1);
         fence_mbar_init();
     }
     if (tid < p.nsh) {   // shared experts follow the routed ones in the unit list, weight 1
@@ -377,23 +451,108 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
     }
     __syncthreads();
 
-    // router rows of this CTA: experts cta + G*j
-    auto issue_router = [&](int layer) {
-        const float *rw = p.layers[layer].rw;
-        int nrows = 0;
-        for (int j = 0; j < p.rpc; ++j)
-            if (cta + G * j < E) ++nrows;
-        mbar_expect_tx(&ms->rbar, (uint32_t)(nrows * d * 4));
-        for (int j = 0; j < nrows; ++j)
-            bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
+    // per-layer unit split of this CTA (same in the producer and the compute warps)
+    struct Split {
+        int n_gu, n_dn, dn_lo, dn_hi, n_dn_items, n_items;
     };
-    if (tid == PRODUCER) issue_router(p.layer0);
+    auto split = [&]() {
+        Split sp;
+        const int n_gu_all = nU * ntile_gu;
+        sp.n_gu = (cta < n_gu_all) ? (n_gu_all - cta + G - 1) / G : 0;   // units cta, cta+G, ...
+        const int n_dn_all = nU * ntile_dn;
+        sp.dn_lo = cta * n_dn_all / G;   // n_dn_all * G < 2^31
+        sp.dn_hi = (cta + 1) * n_dn_all / G;
+        sp.n_dn = sp.dn_hi - sp.dn_lo;
+        sp.n_dn_items = (sp.n_dn + dn_per_slot - 1) / dn_per_slot;
+        sp.n_items = sp.n_gu + sp.n_dn_items;
+        return sp;
+    };
+    // ring slot of item q of a layer whose first item sits in slot s0 (fill parity p0)
+    auto ring_slot = [&](int s0, uint32_t p0, int q, uint32_t &par) {
+        int sq = s0 + q;
+        par = p0;
+        while (sq >= p.nslot) {
+            sq -= p.nslot;
+            par ^= 1u;
+        }
+        return sq;
+    };
 
-    long long item = 0;                  // ring items planned so far (all layers)
-    long long issued = 0;                // ring items whose copies were issued (thread 0)
-    long long consumed = 0;              // ring items consumed so far
-    int router_issued = 1, router_waited = 0;   // router prefetch fills (producer) / waits
-    uint32_t gu_par = 0;   // producer: bit s = parity of the gate/up items issued into slot s so far
+    // ---- producer warp (lane 0): every bulk copy, paced by mbarriers only ----------------
+    if (warp == NW) {
+        if (lane != 0) return;
+        uint32_t gu_par = 0;     // bit s: parity of the gate/up items issued into slot s so far
+        uint32_t fill_par = 0;   // bit s: parity of all fills of slot s so far
+        uint32_t filled = 0;     // bit s: slot s was filled at least once
+        int router_fills = 0;
+        // router rows of this CTA: experts cta + G*j
+        auto issue_router = [&](int layer) {
+            const float *rw = p.layers[layer].rw;
+            int nrows = 0;
+            for (int j = 0; j < p.rpc; ++j)
+                if (cta + G * j < E) ++nrows;
+            fence_proxy_async();
+            mbar_expect_tx(&ms->rbar, (uint32_t)(nrows * d * 4));
+            for (int j = 0; j < nrows; ++j)
+                bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
+            ++router_fills;
+        };
+        issue_router(p.layer0);
+        int s0 = 0;
+        uint32_t p0 = 0;
+        for (int l = 0; l < p.L; ++l) {
+            const int layer = p.layer0 + l;
+            const LayerPtrs Lp = p.layers[layer];
+            // the compute warps have chosen the experts (uexp) and are done with the previous
+            // layer's slots and with the router rows
+            if (!mbar_wait(&ms->route, (uint32_t)(l & 1), err, true)) break;
+            const Split sp = split();
+            bool pok = true;
+            for (int q = 0; q < sp.n_items && pok; ++q) {
+                uint32_t par;
+                const int s = ring_slot(s0, p0, q, par);
+                // items past the ring reuse a slot whose gate/up unit of this layer is consumed
+                if (q >= p.nslot) pok = mbar_wait(&ms->empty[s], ((gu_par >> s) & 1u) ^ 1u, err, true);
+                if (!pok) break;
+                fence_proxy_async();
+                uint8_t *dst = ring + (size_t)s * p.slot_bytes;
+                if (q < sp.n_gu) {
+                    const int u = cta + G * q;
+                    const int us = u / ntile_gu, t = u % ntile_gu;
+                    const uint8_t *src = Lp.gu + (size_t)ms->uexp[us] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
+                    mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
+                    bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
+                    gu_par ^= 1u << s;
+                } else {
+                    const int q0 = (q - sp.n_gu) * dn_per_slot;
+                    const int cnt = min(dn_per_slot, sp.n_dn - q0);
+                    mbar_expect_tx(&ms->full[s], (uint32_t)(cnt * p.dn.tile_bytes));
+                    for (int i = 0; i < cnt; ++i) {
+                        const int n = sp.dn_lo + q0 + i;
+                        const int j = n / nU, us = n % nU;
+                        const uint8_t *src = Lp.dn + (size_t)ms->uexp[us] * p.dn.expert_bytes + (size_t)j * p.dn.tile_bytes;
+                        bulk_g2s(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s]);
+                    }
+                }
+                fill_par ^= 1u << s;
+                filled |= 1u << s;
+            }
+            if (!pok) break;
+            if (l + 1 < p.L) issue_router(layer + 1);
+            uint32_t par;
+            s0 = ring_slot(s0, p0, sp.n_items, par);
+            p0 = par;
+        }
+        // every copy has landed before the CTA's shared memory goes away (the last fill of each
+        // slot and the last router fill; earlier fills of a slot completed before its reuse)
+        for (int s = 0; s < p.nslot; ++s)
+            if ((filled >> s) & 1u) mbar_wait(&ms->full[s], ((fill_par >> s) & 1u) ^ 1u, err, false);
+        if (router_fills > 0) mbar_wait(&ms->rbar, (uint32_t)((router_fills - 1) & 1), err, false);
+        return;
+    }
+
+    int ring_s0 = 0;                     // ring slot of this layer's first item
+    uint32_t ring_p0 = 0;                // and the parity of that slot's fill
     bool ok = true;
     bool aborted = false;                // CTA-uniform: the layer loop was left on a failure
 
@@ -428,8 +587,21 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     aborted = true;
                     break;
                 }
-                for (int i4 = tid; i4 < d / 4; i4 += NT) {
-                    const float4 a = ld_gpu4(p.x_y + 4 * i4), b = ld_gpu4(p.x_y + d + 4 * i4);
+                // every load first (one L2 round trip), then the arithmetic
+                float4 pa[YMAX], pb[YMAX];
+#pragma unroll
+                for (int t = 0; t < YMAX; ++t) {
+                    const int i4 = tid + t * NT;
+                    if (i4 < d / 4) {
+                        pa[t] = ld_gpu4(p.x_y + 4 * i4);
+                        pb[t] = ld_gpu4(p.x_y + d + 4 * i4);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < YMAX; ++t) {
+                    const int i4 = tid + t * NT;
+                    if (i4 >= d / 4) break;
+                    const float4 a = pa[t], b = pb[t];
                     const float ya[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -476,7 +648,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             }
             for (int o = 16; o; o >>= 1) amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
             if (lane == 0) ms->amax[warp] = amx;
-            __syncthreads();
+            csync();
             amx = lane < NW ? ms->amax[lane] : 0.f;
             for (int o = 16; o; o >>= 1) amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
         }
@@ -516,7 +688,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 *reinterpret_cast<uint4 *>(xh + 8 * i8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             }
         }
-        __syncthreads();
+        csync();
         // block sums of the operand the gate/up MMAs see (offset removal in their flush)
         for (int b = tid; b < nbd; b += NT)
             xsum[b] = (FMT == MOE_Q4B32) ? sum32_f16(xh + 32 * b) : sum32_bf16(xb + 32 * b);
@@ -529,7 +701,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 aborted = true;
                 break;
             }
-            ++router_waited;
             trace_mark(p, l, 14, clock64() - tl0);
             int nrows = 0;
             for (int j = 0; j < p.rpc; ++j)
@@ -558,7 +729,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     if (lane == 0) red[j * NW + warp] = v;
                 }
             }
-            __syncthreads();   // partials written; every read of the router rows is done
+            csync();   // partials written; every read of the router rows is done
             trace_mark(p, l, 15, clock64() - tl0);
             if (warp < nrows) {   // warp j sums row j's NW partials
                 float v = lane < NW ? red[warp * NW + lane] : 0.f;
@@ -571,7 +742,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         trace_mark(p, l, 1, clock64() - tl0);
         // ---- 3. top-k on all logits (same result in every CTA) ------------------------
         {
-            __syncthreads();   // this CTA's logits are stored
+            csync();   // this CTA's logits are stored
             if (tid == 0) {
                 xchg_arrive(p, X_LOGITS, !(p.withhold && cta == 0));
                 ok = ctr_wait(ctr(p, X_LOGITS), (unsigned)G, err);
@@ -582,14 +753,22 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 break;
             }
             float m = -INFINITY;   // max of the logits this thread read (every warp reads some)
-            for (int e = tid; e < E; e += NT) {
-                const float v = ld_gpu(p.x_logits + e);
-                lg[e] = v;
-                m = fmaxf(m, v);
+            {
+                float lv[EMAX];
+#pragma unroll
+                for (int t = 0; t < EMAX; ++t)
+                    if (tid + t * NT < E) lv[t] = ld_gpu(p.x_logits + tid + t * NT);
+#pragma unroll
+                for (int t = 0; t < EMAX; ++t) {
+                    if (tid + t * NT < E) {
+                        lg[tid + t * NT] = lv[t];
+                        m = fmaxf(m, lv[t]);
+                    }
+                }
             }
             for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) ms->wmax[warp] = m;
-            __syncthreads();
+            csync();
             trace_mark(p, l, 8, clock64() - tl0);
             // the k-th largest of the warps' maxima bounds the k-th largest logit from below:
             // lane a ranks warp maximum a among the NW maxima
@@ -621,7 +800,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     if (take && slot < CAND_MAX) ms->cand[slot] = make_float2(v, __int_as_float(e));
                 }
             }
-            __syncthreads();
+            csync();
             const int nc = ms->ncand;
             if (nc <= CAND_MAX) {
                 // rank of candidate t = number of candidates ordered before it (value desc, id asc)
@@ -649,80 +828,20 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     }
                 }
             } else if (warp == 0) {
-                // many candidates (ties or a flat distribution): k rounds of warp arg-max
-                for (int j = 0; j < k; ++j) {
-                    float bv = -INFINITY;
-                    int bid = 0x7fffffff;
-                    for (int e = lane; e < E; e += 32) {
-                        bool taken = false;
-                        for (int q = 0; q < j; ++q) taken |= (ms->ids[q] == e);
-                        if (!taken && better(lg[e], e, bv, bid)) {
-                            bv = lg[e];
-                            bid = e;
-                        }
-                    }
-                    for (int o = 16; o; o >>= 1) {
-                        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                        int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-                        if (better(ov, oid, bv, bid)) {
-                            bv = ov;
-                            bid = oid;
-                        }
-                    }
-                    if (lane == 0) {
-                        ms->ids[j] = bid;
-                        ms->uexp[j] = bid;
-                        ms->psel[j] = expf(bv - gmax);
-                    }
-                    __syncwarp();
-                }
+                topk_argmax_rounds(ms, lg, E, k, gmax);   // many candidates (ties or a flat distribution)
             }
-            __syncthreads();
+            csync();
         }
 
+        if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
         trace_mark(p, l, 2, clock64() - tl0);
         // ---- 4./5. stream and compute ----------------------------------------------
-        const int n_gu_all = nU * ntile_gu;
-        const int n_gu = (cta < n_gu_all) ? (n_gu_all - cta + G - 1) / G : 0;   // units cta, cta+G, ...
-        const int n_dn_all = nU * ntile_dn;
-        const int dn_lo = (int)((long long)cta * n_dn_all / G);
-        const int dn_hi = (int)((long long)(cta + 1) * n_dn_all / G);
-        const int n_dn = dn_hi - dn_lo;
-        const int n_dn_items = (n_dn + dn_per_slot - 1) / dn_per_slot;
-        const int n_items = n_gu + n_dn_items;
-        const long long item_base = item;   // first ring item of this layer
-
-        // item q of this layer -> ring slot; issue the copies of item q
-        auto issue_item = [&](int q) {
-            long long it = item_base + q;
-            int s = (int)(it % p.nslot);
-            uint8_t *dst = ring + (size_t)s * p.slot_bytes;
-            if (q < n_gu) {
-                int u = cta + G * q;
-                int us = u / ntile_gu, t = u % ntile_gu;
-                const uint8_t *src = Lp.gu + (size_t)ms->uexp[us] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
-                mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
-                bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
-                gu_par ^= 1u << s;
-            } else {
-                int q0 = (q - n_gu) * dn_per_slot;
-                int cnt = min(dn_per_slot, n_dn - q0);
-                mbar_expect_tx(&ms->full[s], (uint32_t)(cnt * p.dn.tile_bytes));
-                for (int i = 0; i < cnt; ++i) {
-                    int n = dn_lo + q0 + i;
-                    int j = n / nU, us = n % nU;
-                    const uint8_t *src = Lp.dn + (size_t)ms->uexp[us] * p.dn.expert_bytes + (size_t)j * p.dn.tile_bytes;
-                    bulk_g2s(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s]);
-                }
-            }
-            ++issued;
-        };
-        if (tid == PRODUCER) {
-            fence_proxy_async();
-            int first = min(n_items, p.nslot);
-            for (int q = 0; q < first; ++q) issue_item(q);
-        }
-        item += n_items;
+        // the producer warp streams the gate/up tiles, then the down batches (each into a slot
+        // as soon as that slot's gate/up unit is consumed), then the next layer's router rows
+        const Split sp = split();
+        const int n_gu = sp.n_gu, n_dn = sp.n_dn, dn_lo = sp.dn_lo, dn_hi = sp.dn_hi;
+        const int n_items = sp.n_items;
+        auto slot_of = [&](int q, uint32_t &par) { return ring_slot(ring_s0, ring_p0, q, par); };
         // routing weights (needed from the down flush on): renormalised over the selected
         // experts, in rank order
         if (warp == NW - 1) {
@@ -743,26 +862,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                         if (p.w_out) p.w_out[lane] = wj;
                     }
                 }
-            }
-        }
-
-        // producer, while the gate/up warps work: each down batch that did not fit the ring
-        // goes into a slot as soon as that slot's gate/up unit is consumed (its previous item
-        // is always a gate/up unit of this layer), then the next layer's router rows, so that
-        // no bulk copy is in flight during the exchanges that follow
-        if (tid == PRODUCER) {
-            bool pok = true;
-            for (int q = p.nslot; q < n_items && pok; ++q) {
-                const int s = (int)((item_base + q) % p.nslot);
-                pok = mbar_wait(&ms->empty[s], ((gu_par >> s) & 1u) ^ 1u, err, true);
-                if (pok) {
-                    fence_proxy_async();
-                    issue_item(q);
-                }
-            }
-            if (pok && l + 1 < p.L) {
-                issue_router(layer + 1);
-                ++router_issued;
             }
         }
 
@@ -787,10 +886,10 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         // on each unit's barrier itself; partial sums go to red_gu[unit][warp][row]
         if (warp < GW) {
             for (int q = 0; q < n_gu && ok; ++q) {
-                long long it = item_base + q;
-                int s = (int)(it % p.nslot);
+                uint32_t par;
+                const int s = slot_of(q, par);
                 long long tw0 = clock64();
-                ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
+                ok = mbar_wait(&ms->full[s], par, err, true);
                 long long tw1 = clock64();
                 tw_gu += tw1 - tw0;
                 if (!ok) break;
@@ -845,7 +944,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                     red[(q * NW + warp) * 16 + g] = ag;
                     red[(q * NW + warp) * 16 + 8 + g] = a8;
                 }
-                if (q < 5) trace_mark(p, l, 16 + q, clock64() - tw1);
+                if (q < 2) trace_mark(p, l, 19 + q, clock64() - tw1);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ms->empty[s]);   // this warp is done with the slot
             }
@@ -856,7 +955,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             break;
         }
         trace_mark(p, l, 6, clock64() - tl0);
-        consumed += n_gu;
         // SwiGLU of every gate/up unit in parallel: thread (unit q, row i)
         if (tid < n_gu * 8) {
             int q = tid >> 3, i = tid & 7;
@@ -876,7 +974,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 
         // h of every expert in use -> bf16 hi + lo table and per-block sums of hi + lo
         {
-            __syncthreads();   // this CTA's h values are stored
+            csync();   // this CTA's h values are stored
             if (tid == 0) {
                 xchg_arrive(p, X_H);
                 ok = ctr_wait(ctr(p, X_H), (unsigned)G, err);
@@ -885,35 +983,78 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 aborted = true;
                 break;
             }
-            // 4 values per thread; the 8 lanes of a 32-block are neighbours in the warp
+            // 4 values per thread; the 8 lanes of a 32-block are neighbours in the warp.
+            // Q4: fp16 hi + lo of h * 2^s, s per 32-block from the block's max |h| (so the
+            //     values fit fp16; the down flush multiplies by 2^-s);
+            // Q3: bf16 hi + lo of h.
             const int n4 = nU * I / 4;   // a multiple of 8 (I % 64 == 0)
-            for (int b4 = 0; b4 < n4; b4 += NT) {
-                const int i4 = b4 + tid;
-                const bool valid = i4 < n4;
-                float part = 0.f;
-                if (valid) {
-                    const float4 h = ld_gpu4(p.x_h + 4 * i4);
-                    const float hv[4] = {h.x, h.y, h.z, h.w};
-                    uint32_t hi2[2], lo2[2];
+            for (int b4 = 0; b4 < n4; b4 += HB * NT) {
+                float4 hb[HB];   // a batch of loads in flight together, then the arithmetic
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const uint16_t h0 = bf16_rn_bits(hv[2 * j]), h1 = bf16_rn_bits(hv[2 * j + 1]);
-                        const uint16_t l0 = bf16_rn_bits(hv[2 * j] - bf16_bits_f(h0));
-                        const uint16_t l1 = bf16_rn_bits(hv[2 * j + 1] - bf16_bits_f(h1));
-                        hi2[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                        lo2[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-                        part += (bf16_bits_f(h0) + bf16_bits_f(l0)) + (bf16_bits_f(h1) + bf16_bits_f(l1));
-                    }
-                    const int i = 4 * i4, us = i / I, kk = i - us * I;
-                    *reinterpret_cast<uint2 *>(htab + (size_t)(2 * us) * I + kk) = make_uint2(hi2[0], hi2[1]);
-                    *reinterpret_cast<uint2 *>(htab + (size_t)(2 * us + 1) * I + kk) = make_uint2(lo2[0], lo2[1]);
+                for (int t = 0; t < HB; ++t) {
+                    hb[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (b4 + t * NT + tid < n4) hb[t] = ld_gpu4(p.x_h + 4 * (b4 + t * NT + tid));
                 }
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                if (valid && (lane & 7) == 0) hsum[i4 >> 3] = part;   // block (us, b) = us * nbi + b
+#pragma unroll
+                for (int t = 0; t < HB; ++t) {
+                    const int i4 = b4 + t * NT + tid;
+                    const bool valid = i4 < n4;
+                    const float hv[4] = {hb[t].x, hb[t].y, hb[t].z, hb[t].w};
+                    float scale = 1.f;
+                    if constexpr (FMT == MOE_Q4B32) {
+                        float mx = fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3])));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        int he;
+                        frexpf(mx, &he);   // mx < 2^he
+                        const int sh = min(15 - he, 100);
+                        scale = pow2i(sh);
+                        if (valid && (lane & 7) == 0) hinv[i4 >> 3] = pow2i(-sh);
+                    }
+                    float part = 0.f;
+                    if (valid) {
+                        uint32_t hi2[2], lo2[2];
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            if constexpr (FMT == MOE_Q4B32) {
+                                const float v0 = hv[2 * j] * scale, v1 = hv[2 * j + 1] * scale;
+                                const __half2 hh = __floats2half2_rn(v0, v1);
+                                const float2 hf = __half22float2(hh);
+                                const __half2 ll = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
+                                const float2 lf = __half22float2(ll);
+                                hi2[j] = *reinterpret_cast<const uint32_t *>(&hh);
+                                lo2[j] = *reinterpret_cast<const uint32_t *>(&ll);
+                                part += (hf.x + lf.x) + (hf.y + lf.y);
+                            } else {
+                                const uint16_t h0 = bf16_rn_bits(hv[2 * j]), h1 = bf16_rn_bits(hv[2 * j + 1]);
+                                const uint16_t l0 = bf16_rn_bits(hv[2 * j] - bf16_bits_f(h0));
+                                const uint16_t l1 = bf16_rn_bits(hv[2 * j + 1] - bf16_bits_f(h1));
+                                hi2[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                                lo2[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                                part += (bf16_bits_f(h0) + bf16_bits_f(l0)) + (bf16_bits_f(h1) + bf16_bits_f(l1));
+                            }
+                        }
+                        // values kk..kk+3 of expert us: one slice, one register of the pair, the
+                        // element pairs of lanes c0 and c0+1
+                        const int i = 4 * i4, us = i / I, kk = i - us * I;
+                        const int sl = kk >> 4, which = (kk >> 3) & 1, c0 = (kk & 7) >> 1;
+                        uint16_t *hx = htab + (size_t)us * 256 * JN;
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int off_hi = hfrag_index(sl, c0 + q, 0, which, JN);
+                            const int off_lo = hfrag_index(sl, c0 + q, 1, which, JN);
+                            *reinterpret_cast<uint32_t *>(hx + off_hi) = hi2[q];
+                            *reinterpret_cast<uint32_t *>(hx + off_lo) = lo2[q];
+                        }
+                    }
+                    part += __shfl_xor_sync(0xffffffffu, part, 1);
+                    part += __shfl_xor_sync(0xffffffffu, part, 2);
+                    part += __shfl_xor_sync(0xffffffffu, part, 4);
+                    if (valid && (lane & 7) == 0) hsum[i4 >> 3] = part;   // block (us, b) = us * nbi + b
+                }
             }
-            __syncthreads();
+            csync();
         }
         trace_mark(p, l, 4, clock64() - tl0);
 
@@ -923,58 +1064,85 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         float *vsum = red;   // [unit][16]
         for (int nl = warp; nl < n_dn && ok; nl += NW) {
             const int qi = nl / dn_per_slot, ui = nl - qi * dn_per_slot;
-            const long long it = item_base + n_gu + qi;
-            const int s = (int)(it % p.nslot);
+            uint32_t par;
+            const int s = slot_of(n_gu + qi, par);
             long long tw0 = clock64();
-            ok = mbar_wait(&ms->full[s], (uint32_t)((it / p.nslot) & 1), err, true);
+            ok = mbar_wait(&ms->full[s], par, err, true);
             tw_dn += clock64() - tw0;
             if (!ok) break;
+            const long long td0 = clock64();
             const int us = (dn_lo + nl) % nU;
             const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
-            const uint16_t *hp = htab + (size_t)(2 * us + (g & 1)) * I;   // column g: hi (even) / lo (odd)
-            float D[6][4];   // up to 12 k groups (I <= 768)
+            // this lane's B values: column g holds h hi (g even) or lo (g odd) of the blocks
+            // 4j + (g >> 1); one 16-byte load per k-group pair j
+            const uint16_t *hq = htab + (size_t)us * 256 * JN + hfrag_index(2 * (g >> 1), c, g & 1, 0, JN);
+            // 1.0 where this lane's column is the block of MMA (h, m >> 1), else 0 (per half)
+            uint32_t hmask[2][2];
 #pragma unroll
-            for (int j = 0; j < 6; ++j) D[j][0] = D[j][1] = D[j][2] = D[j][3] = 0.f;
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int kg = 0; kg < 12; ++kg) {
-                if (kg < DW) {
-                    uint32_t a[16];
-                    if constexpr (FMT == MOE_Q4B32) {
-                        uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)kg * 512 + lane * 16);
-                        q4_frag(av.x, a[0], a[1], a[2], a[3]);
-                        q4_frag(av.y, a[4], a[5], a[6], a[7]);
-                        q4_frag(av.z, a[8], a[9], a[10], a[11]);
-                        q4_frag(av.w, a[12], a[13], a[14], a[15]);
-                    } else {
-                        const uint32_t *wp = reinterpret_cast<const uint32_t *>(tile + (size_t)kg * 384 + lane * 12);
-                        q3_frag(wp[0], wp[1], wp[2], a);
-                    }
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const int sl = 4 * kg + m;           // k16 slice within K = I
-                        const bool act = ((sl >> 1) & 3) == (g >> 1);
-                        uint32_t b0 = act ? *reinterpret_cast<const uint32_t *>(hp + 16 * sl + 2 * c) : 0u;
-                        uint32_t b1 = act ? *reinterpret_cast<const uint32_t *>(hp + 16 * sl + 2 * c + 8) : 0u;
-                        mma16816(D[kg >> 1], a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
-                    }
-                }
-            }
-            // accumulator j, columns 2c (hi) and 2c+1 (lo): block 4j + c
+                for (int mh = 0; mh < 2; ++mh)
+                    hmask[hh][mh] = (2 * hh + mh == (g >> 1)) ? ONE2 : 0u;
+            // k groups in pairs (kept rolled: this code runs once per unit and layer): the pair
+            // (2j, 2j+1) covers blocks 4j..4j+3, one per column pair (2c hi, 2c+1 lo)
             const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
             float ag = 0.f, a8 = 0.f;
+#pragma unroll 1
+            for (int j = 0; 2 * j < DW; ++j) {
+                if (nl == 0 && j == 1) trace_mark(p, l, 18, clock64() - td0);
+                float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint4 bj = *reinterpret_cast<const uint4 *>(hq + 8 * j);   // (b0, b1) of slices sp = 0, 1
 #pragma unroll
-            for (int j = 0; j < 6; ++j) {
+                for (int h = 0; h < 2; ++h) {
+                    const int kg = 2 * j + h;
+                    if (kg < DW) {
+                        uint32_t a[16];
+                        if constexpr (FMT == MOE_Q4B32) {
+                            uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)kg * 512 + lane * 16);
+                            q4_frag_h(av.x, a[0], a[1], a[2], a[3]);
+                            q4_frag_h(av.y, a[4], a[5], a[6], a[7]);
+                            q4_frag_h(av.z, a[8], a[9], a[10], a[11]);
+                            q4_frag_h(av.w, a[12], a[13], a[14], a[15]);
+                        } else {
+                            const uint32_t *wp = reinterpret_cast<const uint32_t *>(tile + (size_t)kg * 384 + lane * 12);
+                            q3_frag(wp[0], wp[1], wp[2], a);
+                        }
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            // slice 4 kg + m belongs to block 4j + 2h + (m >> 1): live in this lane's
+                            // column only when that is its block
+                            const uint32_t mk = hmask[h][m >> 1];
+                            const uint32_t b0 = hmul2_mask(FMT, (m & 1) ? bj.z : bj.x, mk);
+                            const uint32_t b1 = hmul2_mask(FMT, (m & 1) ? bj.w : bj.y, mk);
+                            if constexpr (FMT == MOE_Q4B32)
+                                mma16816_h(h ? Db : Da, a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
+                            else
+                                mma16816(h ? Db : Da, a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
+                        }
+                    }
+                }
                 const int blk = 4 * j + c;
                 if (blk < nbi) {
-                    const float o = off * hsum[us * nbi + blk];
-                    ag = fmaf(__half2float(sc[g * nbi + blk]), D[j][0] + D[j][1] - o, ag);
-                    a8 = fmaf(__half2float(sc[(g + 8) * nbi + blk]), D[j][2] + D[j][3] - o, a8);
+                    const float hs = hsum[us * nbi + blk];
+                    const float sg = __half2float(sc[g * nbi + blk]), s8 = __half2float(sc[(g + 8) * nbi + blk]);
+                    if constexpr (FMT == MOE_Q4B32) {
+                        // row g: 1024 + q; row g+8: 1024 + 16 q (sums / 16); h entered as h * 2^s
+                        const float hi = hinv[us * nbi + blk];
+                        ag = fmaf(sg * hi, (Da[0] + Da[1]) + (Db[0] + Db[1]) - 1032.f * hs, ag);
+                        a8 = fmaf(s8 * hi, fmaf((Da[2] + Da[3]) + (Db[2] + Db[3]), 0.0625f, -72.f * hs), a8);
+                    } else {
+                        const float o = off * hs;
+                        ag = fmaf(sg, (Da[0] + Da[1]) + (Db[0] + Db[1]) - o, ag);
+                        a8 = fmaf(s8, (Da[2] + Da[3]) + (Db[2] + Db[3]) - o, a8);
+                    }
                 }
             }
+            if (nl == 0) trace_mark(p, l, 16, clock64() - td0);
             ag += __shfl_xor_sync(0xffffffffu, ag, 1);
             a8 += __shfl_xor_sync(0xffffffffu, a8, 1);
             ag += __shfl_xor_sync(0xffffffffu, ag, 2);
             a8 += __shfl_xor_sync(0xffffffffu, a8, 2);
+            if (nl == 0) trace_mark(p, l, 17, clock64() - td0);
             if (c == 0) {
                 vsum[nl * 16 + g] = ag;
                 vsum[nl * 16 + 8 + g] = a8;
@@ -985,7 +1153,12 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             aborted = true;
             break;
         }
-        consumed += n_dn_items;
+        {
+            uint32_t par;
+            const int s_next = slot_of(n_items, par);   // next layer's first item
+            ring_s0 = s_next;
+            ring_p0 = par;
+        }
         trace_mark(p, l, 7, clock64() - tl0);
         // per tile the fixed-order weighted sum of its units
         {
@@ -1001,7 +1174,7 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
                 p.x_y[(size_t)part * d + 16 * j + r] = y;
                 if (part == 0 && last < dn_hi) p.x_y[d + 16 * j + r] = 0.f;
             }
-            __syncthreads();   // this CTA's output parts are stored
+            csync();   // this CTA's output parts are stored
             if (tid == 0) xchg_arrive(p, X_Y);
         }
         trace_mark(p, l, 5, clock64() - tl0);
@@ -1014,8 +1187,20 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
         const int l = p.L - 1;
         if (tid == 0) ok = ctr_wait(ctr(p, X_Y), (unsigned)G, err);
         if (!cta_failed(ok)) {
-            for (int i4 = tid; i4 < d / 4; i4 += NT) {
-                const float4 a = ld_gpu4(p.x_y + 4 * i4), b = ld_gpu4(p.x_y + d + 4 * i4);
+            float4 pa[YMAX], pb[YMAX];
+#pragma unroll
+            for (int t = 0; t < YMAX; ++t) {
+                const int i4 = tid + t * NT;
+                if (i4 < d / 4) {
+                    pa[t] = ld_gpu4(p.x_y + 4 * i4);
+                    pb[t] = ld_gpu4(p.x_y + d + 4 * i4);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < YMAX; ++t) {
+                const int i4 = tid + t * NT;
+                if (i4 >= d / 4) break;
+                const float4 a = pa[t], b = pb[t];
                 const float ya[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -1036,14 +1221,6 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
             }
         }
     }
-    // drain copies still in flight (abort path) before the CTA's shared memory goes away
-    if (tid == PRODUCER) {
-        for (long long it = consumed; it < issued; ++it)
-            mbar_wait(&ms->full[(int)(it % p.nslot)], (uint32_t)((it / p.nslot) & 1), err, false);
-        if (router_issued > router_waited)
-            mbar_wait(&ms->rbar, (uint32_t)(router_waited & 1), err, false);
-    }
-    __syncthreads();
 }
 
 }  // namespace
@@ -1051,8 +1228,8 @@ __global__ void __launch_bounds__(NT, 1) k_decode(DecodeParams p) {
 bool decode_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
     if (T != 1 || (c.flags & MOE_FLAG_NO_DECODE_KERNEL)) return false;
-    // gate/up k chunks go to warps 0..d/256-1; the last warp must stay free for the producer
-    if (c.d_model > 4096 || c.d_model / 256 > NW - 1 || c.d_ff / 64 > 12) return false;
+    // gate/up k chunks go to compute warps 0..d/256-1
+    if (c.d_model > 4096 || c.d_model / 256 > NW || c.d_ff / 64 > 12) return false;
     if (c.n_experts % 4) return false;   // logits region of the exchange area stays 16-byte aligned
     if (c.top_k > MAXK || c.top_k + c.n_shared > MAXU) return false;
     return ctx->dec.smem_bytes > 0;
@@ -1095,12 +1272,12 @@ int decode_setup(moe_ctx *ctx) {
     ds.off_x16 = take((size_t)c.d_model * 2);
     ds.off_xh = take((size_t)c.d_model * 2);
     ds.off_logits = take((size_t)c.n_experts * 4);
-    size_t htab = (size_t)(c.top_k + c.n_shared) * 2 * c.d_ff * 2;   // bf16 hi + lo of h
+    size_t htab = (size_t)(c.top_k + c.n_shared) * 256 * ((c.d_ff + 127) / 128) * 2;   // hi + lo of h
     ds.off_htab = take(htab);
     ds.off_red = take(red_bytes);
     ds.off_misc = take(sizeof(Misc));
     ds.off_resid = take((size_t)c.d_model * 4);
-    ds.off_sums = take((size_t)(c.d_model / 32 + nU * (c.d_ff / 32)) * 4);
+    ds.off_sums = take((size_t)(c.d_model / 32 + 2 * nU * (c.d_ff / 32)) * 4);
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
@@ -1118,7 +1295,7 @@ int decode_setup(moe_ctx *ctx) {
     const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
     QE_CHECK(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, ds.smem_bytes));
     int per_sm = 0;
-    QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NT, ds.smem_bytes));
+    QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NTT, ds.smem_bytes));
     if (per_sm < 1) ds.smem_bytes = 0;
     return MOE_OK;
 }
@@ -1198,7 +1375,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_sums = ds.off_sums;
     void *args[] = {&p};
     const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
-    QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ds.grid), dim3(NT), args,
+    QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ds.grid), dim3(NTT), args,
                                          (size_t)ds.smem_bytes, st));
     QE_CHECK_LAUNCH("k_decode");
     return MOE_OK;
