@@ -7,12 +7,14 @@
 // One persistent kernel per GEMM, one CTA per SM, warp-specialised:
 //   warp 0      : allocates TMEM, one lane issues tcgen05.mma (kind::f16,
 //                 fp16 x fp16 -> fp32 in TMEM) and tcgen05.commit;
-//   warps 1..8  : producers.  A rows (tokens or h rows) are gathered with
-//                 16-byte cp.async; the weights are decoded from the packed
-//                 row tiles to fp16 (w = s * (q - zero), one rounding) and
-//                 stored; both land in the 128-byte-swizzled K-major layout
-//                 the MMA descriptors describe;
-//   warps 12..15: epilogue, tcgen05.ld from TMEM.
+//   warps 1..8  : weight producers, two 16-row tiles of the B stage each: the
+//                 weights are decoded from the packed row tiles to fp16
+//                 (w = s * (q - zero), one rounding) and stored with stmatrix
+//                 in the 128-byte-swizzled K-major layout the MMA descriptors
+//                 describe;
+//   warps 9..11 : A-row loaders: A rows (tokens or h rows) are gathered with
+//                 16-byte cp.async into the same layout;
+//   warps 12..15: epilogue, tcgen05.ld from TMEM (lane quarter = warp % 4).
 // A work item is (expert, 256 slots, 256 output columns): two M=128
 // accumulators share every decoded weight stage (TMEM: 2 x 256 fp32 columns),
 // so the weight decode is paid once per 256 slots.
@@ -32,9 +34,12 @@ namespace qeffn {
 namespace {
 
 constexpr int TC_NT = 512;                 // 16 warps
-constexpr int TC_PROD_W0 = 1, TC_PROD_NW = 8;
-constexpr int TC_EPI_W0 = 12;              // warps 12..15: TMEM lane quarters 0..3
+constexpr int TC_PROD_W0 = 1, TC_PROD_NW = 8;   // weight producers: two row tiles of the B stage each
+constexpr int TC_ALD_W0 = 9, TC_ALD_NW = 3;     // A-row loaders
+constexpr int TC_ALD_NT = TC_ALD_NW * 32;
+constexpr int TC_EPI_W0 = 12;              // warps 12..15: TMEM lane quarters 0..3 (warp % 4)
 constexpr int TC_BM = 256;                 // slots per work item (2 x M=128)
+constexpr int TC_ALD_MAXJ = (TC_BM * 8 + TC_ALD_NT - 1) / TC_ALD_NT;   // 16-byte A chunks per loader and stage
 constexpr int TC_BN = 256;                 // output columns per work item
 constexpr int TC_BK = 64;                  // k per pipeline stage (one 128-byte swizzle row)
 constexpr int TC_STAGES = 3;
@@ -231,11 +236,25 @@ __device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16])
     }
 }
 
-// Decode this thread's two pieces (row tiles 2*pw, 2*pw+1 of the n-tile, lane
-// (g, c)) from its staging bytes into the stage's swizzled fp16 weight tile:
-// w = s * (q - zero), one fp16 rounding.
+// Four 8x8 fp16 matrices from mma-fragment registers to shared memory: lane i
+// gives the address of row i % 8 of matrix i / 8 (16 bytes).
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// Decode this warp's two row tiles (2*pw, 2*pw+1 of the n-tile; this lane's
+// pieces, lane (g, c)) from the staging bytes into the stage's swizzled fp16
+// weight tile: w = s * (q - zero), one fp16 rounding.  The registers are in
+// mma fragment order, so each 16x16 block (k16 slice m of a tile) goes out as
+// one stmatrix: matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7,
+// k 8-15), (rows 8-15, k 8-15) = registers a0, a1, a2, a3.
 template <int FMT>
-__device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *b_dst, int pw, int g, int c) {
+__device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *b_dst, int pw, int lane) {
+    const uint32_t bd = su32(b_dst);
+    const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);   // row within the tile this lane addresses
+    const int mk = 8 * (lane >> 4);                         // k offset of its matrix
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
         uint32_t q[16];
@@ -244,15 +263,12 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *b_dst,
         uint32_t s8p = *reinterpret_cast<const uint32_t *>(raw + 36 + 8 * tt);   // rows g+8
         uint32_t us0 = (sgp & 0xFFFFu) * 0x10001u, us1 = (sgp >> 16) * 0x10001u;
         uint32_t u80 = (s8p & 0xFFFFu) * 0x10001u, u81 = (s8p >> 16) * 0x10001u;
-        int n0 = 16 * (2 * pw + tt) + g;                // rows g, g+8 of this tile
+        const int row = 16 * (2 * pw + tt) + mrow;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            int kk = 16 * m + 2 * c;                    // k of a0 / a1 within the stage
             uint32_t sg = m < 2 ? us0 : us1, s8 = m < 2 ? u80 : u81;
-            *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk)) = hmul2(q[4 * m + 0], sg);
-            *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk)) = hmul2(q[4 * m + 1], s8);
-            *reinterpret_cast<uint32_t *>(b_dst + swz(n0, kk + 8)) = hmul2(q[4 * m + 2], sg);
-            *reinterpret_cast<uint32_t *>(b_dst + swz(n0 + 8, kk + 8)) = hmul2(q[4 * m + 3], s8);
+            stmatrix_x4(bd + swz(row, 16 * m + mk), hmul2(q[4 * m + 0], sg), hmul2(q[4 * m + 1], s8),
+                        hmul2(q[4 * m + 2], sg), hmul2(q[4 * m + 3], s8));
         }
     }
 }
@@ -278,8 +294,8 @@ __device__ __forceinline__ int4 item_of(const TcParams &p, int item) {
 struct TcSmem {
     uint64_t full[TC_STAGES];
     uint64_t empty[TC_STAGES];
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint64_t acc_full[2];       // TMEM slot (256 columns) written by the MMAs
+    uint64_t acc_empty[2];      // TMEM slot read out by the epilogue
     uint32_t tmem_base;
     int abort;
 };
@@ -305,11 +321,13 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(&ss->full[s], TC_PROD_NW * 32);
+            mbar_init(&ss->full[s], TC_PROD_NW * 32 + TC_ALD_NT);
             mbar_init(&ss->empty[s], 1);
         }
-        mbar_init(&ss->acc_full, 1);
-        mbar_init(&ss->acc_empty, 128);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&ss->acc_full[t], 1);
+            mbar_init(&ss->acc_empty[t], 128);
+        }
         ss->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -322,14 +340,20 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 
     if (warp == 0) {
         // ---- MMA issuer ------------------------------------------------------------
-        int it = 0, ti = 0;
-        for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
+        // TMEM is a ring of two 256-column slots; an item takes one slot per M=128
+        // accumulator, so an item of at most 128 rows runs while the epilogue still
+        // reads the previous item's slot
+        int it = 0;
+        uint32_t u = 0;                          // slot uses so far (slot u & 1, phase u >> 1)
+        for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             int rows = wi.z;
-            // accumulators free? (epilogue of the previous item has read them)
-            ok = mbar_wait_b(&ss->acc_empty, (uint32_t)((ti & 1) ^ 1), p.err);
+            const int na = rows > 128 ? 2 : 1;
+            for (int a = 0; a < na && ok; ++a)
+                ok = mbar_wait_b(&ss->acc_empty[(u + a) & 1], (((u + a) >> 1) & 1) ^ 1, p.err);
             if (!ok) break;
             tc_fence_after();
+            const uint32_t t0 = tmem + 256 * (u & 1), t1 = tmem + 256 * ((u + 1) & 1);
             for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                 int s = it % TC_STAGES;
                 ok = mbar_wait_b(&ss->full[s], (uint32_t)((it / TC_STAGES) & 1), p.err);
@@ -340,36 +364,31 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 #pragma unroll
                     for (int j = 0; j < TC_BK / 16; ++j) {
                         uint64_t bd = sdesc(b0 + 32 * j);
-                        umma_f16(tmem, sdesc(a0 + 32 * j), bd, ID, (kb | j) != 0);
-                        if (rows > 128)
-                            umma_f16(tmem + 256, sdesc(a0 + 128 * 128 + 32 * j), bd, ID, (kb | j) != 0);
+                        umma_f16(t0, sdesc(a0 + 32 * j), bd, ID, (kb | j) != 0);
+                        if (na == 2) umma_f16(t1, sdesc(a0 + 128 * 128 + 32 * j), bd, ID, (kb | j) != 0);
                     }
                     umma_commit(&ss->empty[s]);
                 }
                 __syncwarp();
             }
-            if (ok && lane == 0) umma_commit(&ss->acc_full);
+            if (ok && lane == 0)
+                for (int a = 0; a < na; ++a) umma_commit(&ss->acc_full[(u + a) & 1]);
             __syncwarp();
+            u += na;
         }
     } else if (warp >= TC_PROD_W0 && warp < TC_PROD_W0 + TC_PROD_NW) {
         // ---- producers ---------------------------------------------------------------
         const int pt = tid - TC_PROD_W0 * 32;   // 0..255
-        const int pw = pt >> 5;                  // producer warp 0..7
-        const int g = lane >> 2, c = lane & 3;
+        const int pw = pt >> 5;                  // producer warp 0..7: row tiles 2 pw, 2 pw + 1
+        const int g = lane >> 2;                 // scale rows g, g+8 of this lane's pieces
         int it = 0;
         int pending = -1;                        // stage whose cp.async group is still in flight
         uint8_t *myraw = sRaw + pt * RAW_THREAD_BYTES;
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
-            const int e = wi.x, pos0 = wi.y, rows = wi.z, nt = wi.w;
-            // the A rows this thread gathers: row r = pt (0..255), all 8 chunks of 16 bytes
-            int r = pt;
-            int rr = min(r, rows - 1);           // rows past the expert's end repeat its last row
-            int pos = pos0 + rr;
-            int arow;
-            if constexpr (MODE == TC_ROUTER) arow = pos;                      // token
-            else arow = p.a_by_token ? slot_token(p.perm[pos], p.T, p.k) : pos;
-            const uint16_t *asrc = p.A + (size_t)arow * p.K;
+            const int e = wi.x, nt = wi.w;
+            const int ch = pt & 7;                   // router B: chunk of rows 32j + pt / 8
+            const uint32_t a_off = swz(pt >> 3, ch * 8);
             // weights: this warp decodes row tiles 2*pw and 2*pw+1 of the 16 in the n-tile
             const uint8_t *wexp = p.W + (size_t)e * p.L.expert_bytes;
             const int nb = p.K / 32;
@@ -377,21 +396,16 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 int s = it % TC_STAGES;
                 ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
                 if (!ok) break;
-                uint8_t *a_dst = sA + s * A_STAGE_BYTES;
                 uint8_t *b_dst = sB + s * B_STAGE_BYTES;
                 const int kx = MODE == TC_ROUTER ? kb % nkd : kb;   // k block of the activations
-                // A: 8 chunks of row r, k = 64*kx .. +63
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    cp_async16(a_dst + swz(r, ch * 8), asrc + 64 * kx + ch * 8);
                 if constexpr (MODE == TC_ROUTER) {
-                    // B: router row (expert) 256*nt + r of part kb / nkd
-                    const uint16_t *bsrc = p.rparts + ((size_t)(kb / nkd) * p.E + (size_t)nt * TC_BN + r) * p.K;
+                    // B: router rows (experts) 256*nt + 32j + pt/8 of part kb / nkd: one warp
+                    // instruction reads four whole 128-byte row segments
+                    const uint16_t *bsrc = p.rparts + ((size_t)(kb / nkd) * p.E + (size_t)nt * TC_BN) * p.K + ch * 8;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        cp_async16(b_dst + swz(r, ch * 8), bsrc + 64 * kx + ch * 8);
+                    for (int j = 0; j < 8; ++j)
+                        cp_async16(b_dst + 4096 * j + a_off, bsrc + (size_t)(32 * j + (pt >> 3)) * p.K + 64 * kx);
                 }
-                cp_async_commit();
                 if constexpr (MODE != TC_ROUTER) {
                     // this thread's weight bytes for k group kb (decoded one iteration later)
                     uint8_t *raw = myraw + (it & 1) * 48;
@@ -411,12 +425,12 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         cp_async4(raw + 36 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
                     }
                 }
-                cp_async_commit();
-                // the previous iteration's group (its A rows and weight bytes) is complete once
-                // at most this one is pending: decode its weights, publish the stage
+                cp_async_commit();   // one group per stage: its weight bytes
+                // the previous stage's group is complete once at most this one is pending: decode
+                // its weights, publish it (this stage's loads stay in flight meanwhile)
                 if (pending >= 0) {
                     cp_async_wait<1>();
-                    if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, g, c);
+                    if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, lane);
                     fence_async_smem();
                     mbar_arrive(&ss->full[pending]);
                 }
@@ -425,7 +439,57 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             if (!ok) break;
             // flush: the last stage of the item
             cp_async_wait<0>();
-            if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, g, c);
+            if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, lane);
+            fence_async_smem();
+            mbar_arrive(&ss->full[pending]);
+            pending = -1;
+        }
+        if (pending >= 0) cp_async_wait<0>();
+    } else if (warp >= TC_ALD_W0 && warp < TC_ALD_W0 + TC_ALD_NW) {
+        // ---- A-row loaders -------------------------------------------------------------
+        // 16-byte chunk q = at + TC_ALD_NT * j of the stage: row q / 8, chunk q % 8 (the same
+        // for every j), so one warp instruction reads four whole 128-byte row segments
+        const int at = tid - TC_ALD_W0 * 32;
+        const int ch = at & 7;
+        int it = 0;
+        int pending = -1;
+        for (int item = blockIdx.x; item < n_items && ok; item += G) {
+            int4 wi = item_of<MODE>(p, item);
+            const int pos0 = wi.y, rows = wi.z;
+            int aoff[TC_ALD_MAXJ];                   // element offset of each chunk's row in A
+#pragma unroll
+            for (int j = 0; j < TC_ALD_MAXJ; ++j) {
+                const int q = at + TC_ALD_NT * j;
+                aoff[j] = 0;
+                if (q < TC_BM * 8) {
+                    const int pos = pos0 + min(q >> 3, rows - 1);   // rows past the end repeat the last
+                    int arow;
+                    if constexpr (MODE == TC_ROUTER) arow = pos;    // token
+                    else arow = p.a_by_token ? slot_token(p.perm[pos], p.T, p.k) : pos;
+                    aoff[j] = arow * p.K + ch * 8;
+                }
+            }
+            for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+                int s = it % TC_STAGES;
+                ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
+                if (!ok) break;
+                uint8_t *a_dst = sA + s * A_STAGE_BYTES;
+                const int kx = MODE == TC_ROUTER ? kb % nkd : kb;   // k block of the activations
+#pragma unroll
+                for (int j = 0; j < TC_ALD_MAXJ; ++j) {
+                    const int q = at + TC_ALD_NT * j;
+                    if (q < TC_BM * 8) cp_async16(a_dst + swz(q >> 3, ch * 8), p.A + aoff[j] + 64 * kx);
+                }
+                cp_async_commit();
+                if (pending >= 0) {   // the previous stage's rows have landed: publish them
+                    cp_async_wait<1>();
+                    fence_async_smem();
+                    mbar_arrive(&ss->full[pending]);
+                }
+                pending = s;
+            }
+            if (!ok) break;
+            cp_async_wait<0>();
             fence_async_smem();
             mbar_arrive(&ss->full[pending]);
             pending = -1;
@@ -435,19 +499,19 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         // ---- epilogue ----------------------------------------------------------------
         const int q4 = warp - TC_EPI_W0;        // TMEM lane quarter
         const int row = 32 * q4 + lane;         // row within each M=128 accumulator
-        int ti = 0;
-        for (int item = blockIdx.x; item < n_items && ok; item += G, ++ti) {
+        uint32_t u = 0;                          // TMEM slot uses, in the MMA issuer's order
+        for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             const int pos0 = wi.y, rows = wi.z, nt = wi.w;
-            ok = mbar_wait_b(&ss->acc_full, (uint32_t)(ti & 1), p.err);
-            if (!ok) break;
-            tc_fence_after();
-            for (int acc = 0; acc < 2; ++acc) {
+            const int na = rows > 128 ? 2 : 1;
+            for (int acc = 0; acc < na && ok; ++acc, ++u) {
+                ok = mbar_wait_b(&ss->acc_full[u & 1], (u >> 1) & 1, p.err);
+                if (!ok) break;
+                tc_fence_after();
                 int m = 128 * acc + row;
                 bool live = m < rows;
-                if (acc == 1 && rows <= 128) break;
                 int pos = pos0 + min(m, rows - 1);
-                uint32_t tbase = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(256 * acc);
+                uint32_t tbase = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(256 * (u & 1));
                 if constexpr (MODE == TC_ROUTER) {
                     float *lrow = p.logits + (size_t)pos * p.E + (size_t)nt * TC_BN;
                     const float *bb = p.rbias + (size_t)nt * TC_BN;
@@ -507,9 +571,9 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(&ss->acc_empty[u & 1]);   // this slot may be overwritten
             }
-            tc_fence_before();
-            mbar_arrive(&ss->acc_empty);
         }
     }
     // every role done: release TMEM
@@ -615,7 +679,10 @@ bool tc_supported(const moe_ctx *ctx, int T) {
     if (c.flags & MOE_FLAG_NO_TENSOR_PREFILL) return false;
     if (T < 64) return false;
     // n-tiles of 256 output columns: 2I and d must be multiples of 256
-    return (2 * c.d_ff) % TC_BN == 0 && c.d_model % TC_BN == 0 && c.d_model % TC_BK == 0 && c.d_ff % TC_BK == 0;
+    if ((2 * c.d_ff) % TC_BN || c.d_model % TC_BN || c.d_model % TC_BK || c.d_ff % TC_BK) return false;
+    // A-row offsets are 32-bit element indices: rows (tokens or slots) x K below 2^31
+    const long long slots = (long long)c.max_tokens * (c.top_k + c.n_shared);
+    return slots * (c.d_model > c.d_ff ? c.d_model : c.d_ff) < (1LL << 31);
 }
 
 size_t tc_items_max(const moe_config &c) {
