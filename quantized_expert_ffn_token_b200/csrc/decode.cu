@@ -352,9 +352,8 @@ __device__ __forceinline__ bool cta_failed(bool mine_ok) {
 //    4 every expert's h received           9 this thread's down units done
 //    7 every down unit done                5 output tiles published
 //   10 cycles waiting for gate/up data    12 cycles waiting for down data
-//   16 / 17 / 18 warp 0's first down unit: accumulation done / reduced /
-//      first k-group pair done (cycles since its data was ready)
-//   19, 20 compute cycles of gate/up units 0, 1 (warp 0)
+//   16 / 17 warp 0's first down unit: accumulation done / reduced (cycles
+//      since its data was ready)
 //   21 global timer (ns) at the layer start
 constexpr int TRACE_WORDS = 24;
 
@@ -944,7 +943,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                     red[(q * NW + warp) * 16 + g] = ag;
                     red[(q * NW + warp) * 16 + 8 + g] = a8;
                 }
-                if (q < 2) trace_mark(p, l, 19 + q, clock64() - tw1);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ms->empty[s]);   // this warp is done with the slot
             }
@@ -1083,13 +1081,13 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
 #pragma unroll
                 for (int mh = 0; mh < 2; ++mh)
                     hmask[hh][mh] = (2 * hh + mh == (g >> 1)) ? ONE2 : 0u;
-            // k groups in pairs (kept rolled: this code runs once per unit and layer): the pair
-            // (2j, 2j+1) covers blocks 4j..4j+3, one per column pair (2c hi, 2c+1 lo)
+            // k groups in pairs: the pair (2j, 2j+1) covers blocks 4j..4j+3, one per column
+            // pair (2c hi, 2c+1 lo)
             const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
             float ag = 0.f, a8 = 0.f;
-#pragma unroll 1
-            for (int j = 0; 2 * j < DW; ++j) {
-                if (nl == 0 && j == 1) trace_mark(p, l, 18, clock64() - td0);
+#pragma unroll
+            for (int j = 0; j < 6; ++j) {   // I <= 768
+                if (2 * j >= DW) break;
                 float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint4 bj = *reinterpret_cast<const uint4 *>(hq + 8 * j);   // (b0, b1) of slices sp = 0, 1
 #pragma unroll
