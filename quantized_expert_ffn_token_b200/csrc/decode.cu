@@ -219,10 +219,11 @@ __device__ __forceinline__ float sum32_bf16(const uint16_t *p) {
 // lane (g, c) of the down MMAs reads, for k-group pair j, the 8 halves
 // [sp][which][e] of slices 8j + 2 (g >> 1) + sp from row r = g & 1 (hi / lo),
 // register which (b0: k 2c, 2c+1; b1: k 2c+8, 2c+9), element e; one 16-byte load.
+// Pair-major: the 32 lanes' entries of one pair are contiguous (512 bytes).
 // Index of the first half of (slice sl, lane column c, row r, register which).
-__device__ __forceinline__ int hfrag_index(int sl, int c, int r, int which, int JN) {
+__device__ __forceinline__ int hfrag_index(int sl, int c, int r, int which) {
     const int b4 = (sl >> 1) & 3, j = sl >> 3, sp = sl & 1;
-    return ((((b4 * 4 + c) * 2 + r) * JN + j) * 2 + sp) * 4 + which * 2;
+    return ((j * 32 + (b4 * 4 + c) * 2 + r) * 2 + sp) * 4 + which * 2;
 }
 // x * mask for a packed pair of fp16 (Q4) or bf16 (Q3) values, mask 1.0 or 0 in both
 // halves: zeroes the inactive block columns on the multiply pipe.
@@ -1040,8 +1041,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                         uint16_t *hx = htab + (size_t)us * 256 * JN;
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
-                            const int off_hi = hfrag_index(sl, c0 + q, 0, which, JN);
-                            const int off_lo = hfrag_index(sl, c0 + q, 1, which, JN);
+                            const int off_hi = hfrag_index(sl, c0 + q, 0, which);
+                            const int off_lo = hfrag_index(sl, c0 + q, 1, which);
                             *reinterpret_cast<uint32_t *>(hx + off_hi) = hi2[q];
                             *reinterpret_cast<uint32_t *>(hx + off_lo) = lo2[q];
                         }
@@ -1073,7 +1074,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
             const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
             // this lane's B values: column g holds h hi (g even) or lo (g odd) of the blocks
             // 4j + (g >> 1); one 16-byte load per k-group pair j
-            const uint16_t *hq = htab + (size_t)us * 256 * JN + hfrag_index(2 * (g >> 1), c, g & 1, 0, JN);
+            const uint16_t *hq = htab + (size_t)us * 256 * JN + hfrag_index(2 * (g >> 1), c, g & 1, 0);
             // 1.0 where this lane's column is the block of MMA (h, m >> 1), else 0 (per half)
             uint32_t hmask[2][2];
 #pragma unroll
@@ -1089,7 +1090,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
             for (int j = 0; j < 6; ++j) {   // I <= 768
                 if (2 * j >= DW) break;
                 float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint4 bj = *reinterpret_cast<const uint4 *>(hq + 8 * j);   // (b0, b1) of slices sp = 0, 1
+                const uint4 bj = *reinterpret_cast<const uint4 *>(hq + 256 * j);   // (b0, b1) of slices sp = 0, 1
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int kg = 2 * j + h;

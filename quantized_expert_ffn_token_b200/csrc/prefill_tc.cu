@@ -45,8 +45,11 @@ constexpr int TC_BK = 64;                  // k per pipeline stage (one 128-byte
 constexpr int TC_STAGES = 3;
 constexpr int A_STAGE_BYTES = TC_BM * TC_BK * 2;   // 32 KB
 constexpr int B_STAGE_BYTES = TC_BN * TC_BK * 2;   // 32 KB
-constexpr int RAW_THREAD_BYTES = 96;                 // 2 slots x (2 x 16 B codes + 4 x 4 B scales)
-constexpr int RAW_BYTES = TC_PROD_NW * 32 * RAW_THREAD_BYTES;
+// Producers' weight staging: 2 slots x 3 fields (codes of tile 0, codes of
+// tile 1, the four scales) x one 16-byte entry per producer thread, field-major
+// so that a warp's accesses to one field are contiguous (no bank conflicts).
+constexpr int RAW_FIELD = TC_PROD_NW * 32 * 16;
+constexpr int RAW_BYTES = 2 * 3 * RAW_FIELD;
 constexpr long long TC_SPIN = 4000000000LL;        // clock64 cycles, about two seconds
 
 struct TcParams {
@@ -258,9 +261,9 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *b_dst,
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
         uint32_t q[16];
-        decode_piece<FMT>(raw + 16 * tt, q);
-        uint32_t sgp = *reinterpret_cast<const uint32_t *>(raw + 32 + 8 * tt);   // s[g][2kb], s[g][2kb+1]
-        uint32_t s8p = *reinterpret_cast<const uint32_t *>(raw + 36 + 8 * tt);   // rows g+8
+        decode_piece<FMT>(raw + tt * RAW_FIELD, q);
+        uint32_t sgp = *reinterpret_cast<const uint32_t *>(raw + 2 * RAW_FIELD + 8 * tt);   // s[g][2kb], s[g][2kb+1]
+        uint32_t s8p = *reinterpret_cast<const uint32_t *>(raw + 2 * RAW_FIELD + 4 + 8 * tt);   // rows g+8
         uint32_t us0 = (sgp & 0xFFFFu) * 0x10001u, us1 = (sgp >> 16) * 0x10001u;
         uint32_t u80 = (s8p & 0xFFFFu) * 0x10001u, u81 = (s8p >> 16) * 0x10001u;
         const int row = 16 * (2 * pw + tt) + mrow;
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         const int g = lane >> 2;                 // scale rows g, g+8 of this lane's pieces
         int it = 0;
         int pending = -1;                        // stage whose cp.async group is still in flight
-        uint8_t *myraw = sRaw + pt * RAW_THREAD_BYTES;
+        uint8_t *myraw = sRaw + pt * 16;         // + (slot * 3 + field) * RAW_FIELD
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             const int e = wi.x, nt = wi.w;
@@ -408,21 +411,21 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 }
                 if constexpr (MODE != TC_ROUTER) {
                     // this thread's weight bytes for k group kb (decoded one iteration later)
-                    uint8_t *raw = myraw + (it & 1) * 48;
+                    uint8_t *raw = myraw + (it & 1) * 3 * RAW_FIELD;
 #pragma unroll
                     for (int tt = 0; tt < 2; ++tt) {
                         const uint8_t *tile = wexp + (size_t)(nt * 16 + 2 * pw + tt) * p.L.tile_bytes;
                         const uint8_t *cs = tile + (size_t)kb * p.L.kg_bytes;
                         if constexpr (FMT == MOE_Q4B32) {
-                            cp_async16(raw + 16 * tt, cs + lane * 16);
+                            cp_async16(raw + tt * RAW_FIELD, cs + lane * 16);
                         } else {
-                            cp_async4(raw + 16 * tt, cs + lane * 12);
-                            cp_async4(raw + 16 * tt + 4, cs + lane * 12 + 4);
-                            cp_async4(raw + 16 * tt + 8, cs + lane * 12 + 8);
+                            cp_async4(raw + tt * RAW_FIELD, cs + lane * 12);
+                            cp_async4(raw + tt * RAW_FIELD + 4, cs + lane * 12 + 4);
+                            cp_async4(raw + tt * RAW_FIELD + 8, cs + lane * 12 + 8);
                         }
                         const uint8_t *sc = tile + p.L.code_bytes;
-                        cp_async4(raw + 32 + 8 * tt, sc + (size_t)(g * nb + 2 * kb) * 2);
-                        cp_async4(raw + 36 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
+                        cp_async4(raw + 2 * RAW_FIELD + 8 * tt, sc + (size_t)(g * nb + 2 * kb) * 2);
+                        cp_async4(raw + 2 * RAW_FIELD + 4 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
                     }
                 }
                 cp_async_commit();   // one group per stage: its weight bytes
@@ -430,7 +433,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 // its weights, publish it (this stage's loads stay in flight meanwhile)
                 if (pending >= 0) {
                     cp_async_wait<1>();
-                    if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, lane);
+                    if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 3 * RAW_FIELD, sB + pending * B_STAGE_BYTES, pw, lane);
                     fence_async_smem();
                     mbar_arrive(&ss->full[pending]);
                 }
@@ -439,7 +442,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             if (!ok) break;
             // flush: the last stage of the item
             cp_async_wait<0>();
-            if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 48, sB + pending * B_STAGE_BYTES, pw, lane);
+            if constexpr (MODE != TC_ROUTER) decode_stage<FMT>(myraw + ((it - 1) & 1) * 3 * RAW_FIELD, sB + pending * B_STAGE_BYTES, pw, lane);
             fence_async_smem();
             mbar_arrive(&ss->full[pending]);
             pending = -1;
