@@ -97,7 +97,8 @@ struct DecodeParams {
     unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int dn_units_max;          // largest down-unit run of one CTA
-    int off_ring, off_router, off_x16, off_xh, off_logits, off_htab, off_red, off_misc, off_resid, off_sums;
+    int off_ring, off_router, off_x16, off_xh, off_logits, off_htab, off_red, off_misc, off_resid, off_sums,
+        off_ltab;
 };
 
 // ---- PTX helpers -------------------------------------------------------------
@@ -420,6 +421,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
     float *red = reinterpret_cast<float *>(smem + p.off_red);   // [2][NW][16]
     Misc *ms = reinterpret_cast<Misc *>(smem + p.off_misc);
     float *rs = reinterpret_cast<float *>(smem + p.off_resid);      // residual stream [d]
+    LayerPtrs *ltab = reinterpret_cast<LayerPtrs *>(smem + p.off_ltab);   // [L] weight pointers
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const int G = gridDim.x, cta = blockIdx.x;
@@ -449,6 +451,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         ms->uexp[k + tid] = E + tid;
         ms->uw[k + tid] = 1.f;
     }
+    for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];   // this call's layers
     __syncthreads();
 
     // per-layer unit split of this CTA (same in the producer and the compute warps)
@@ -487,7 +490,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         int router_fills = 0;
         // router rows of this CTA: experts cta + G*j
         auto issue_router = [&](int layer) {
-            const float *rw = p.layers[layer].rw;
+            const float *rw = ltab[layer - p.layer0].rw;
             int nrows = 0;
             for (int j = 0; j < p.rpc; ++j)
                 if (cta + G * j < E) ++nrows;
@@ -502,7 +505,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         uint32_t p0 = 0;
         for (int l = 0; l < p.L; ++l) {
             const int layer = p.layer0 + l;
-            const LayerPtrs Lp = p.layers[layer];
+            const LayerPtrs Lp = ltab[l];
             // the compute warps have chosen the experts (uexp) and are done with the previous
             // layer's slots and with the router rows
             if (!mbar_wait(&ms->route, (uint32_t)(l & 1), err, true)) break;
@@ -557,8 +560,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
     bool aborted = false;                // CTA-uniform: the layer loop was left on a failure
 
     for (int l = 0; l < p.L; ++l) {
-        const int layer = p.layer0 + l;
-        const LayerPtrs Lp = p.layers[layer];
+        const LayerPtrs Lp = ltab[l];
         const long long tl0 = clock64();
         if (p.trace) {   // global time of the layer start (ns), to line up the CTAs' clocks
             unsigned long long gt;
@@ -696,15 +698,17 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
         {
+            int nrows = 0;
+            for (int j = 0; j < p.rpc; ++j)
+                if (cta + G * j < E) ++nrows;
+            // this warp's bias (row warp), loaded now so that its latency hides behind the dot products
+            const float bias = (warp < nrows && lane == 0) ? __ldg(Lp.rb + cta + G * warp) : 0.f;
             ok = mbar_wait(&ms->rbar, (uint32_t)(l & 1), err, true);
             if (cta_failed(ok)) {
                 aborted = true;
                 break;
             }
             trace_mark(p, l, 14, clock64() - tl0);
-            int nrows = 0;
-            for (int j = 0; j < p.rpc; ++j)
-                if (cta + G * j < E) ++nrows;
             // thread sums its strided share of 4-wide k chunks for every live row
             float part[8];
 #pragma unroll
@@ -735,7 +739,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 float v = lane < NW ? red[warp * NW + lane] : 0.f;
                 for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                 const int e = cta + G * warp;
-                if (lane == 0) p.x_logits[e] = v + Lp.rb[e];
+                if (lane == 0) p.x_logits[e] = v + bias;
             }
         }
 
@@ -1168,7 +1172,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 int first = j * nU, last = j * nU + nU - 1;
                 int n0 = max(first, dn_lo), n1 = min(last, dn_hi - 1);
                 float y = 0.f;
-                for (int n = n0; n <= n1; ++n) y = fmaf(ms->uw[n % nU], vsum[(n - dn_lo) * 16 + r], y);
+                for (int n = n0, us = n0 - first; n <= n1; ++n, ++us)   // us = n % nU
+                    y = fmaf(ms->uw[us], vsum[(n - dn_lo) * 16 + r], y);
                 int part = (first >= dn_lo) ? 0 : 1;
                 p.x_y[(size_t)part * d + 16 * j + r] = y;
                 if (part == 0 && last < dn_hi) p.x_y[d + 16 * j + r] = 0.f;
@@ -1277,6 +1282,7 @@ int decode_setup(moe_ctx *ctx) {
     ds.off_misc = take(sizeof(Misc));
     ds.off_resid = take((size_t)c.d_model * 4);
     ds.off_sums = take((size_t)(c.d_model / 32 + 2 * nU * (c.d_ff / 32)) * 4);
+    ds.off_ltab = take((size_t)c.n_layers * sizeof(LayerPtrs));   // a call runs at most n_layers layers
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
     while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
@@ -1372,6 +1378,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_misc = ds.off_misc;
     p.off_resid = ds.off_resid;
     p.off_sums = ds.off_sums;
+    p.off_ltab = ds.off_ltab;
     void *args[] = {&p};
     const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
     QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ds.grid), dim3(NTT), args,

@@ -166,7 +166,7 @@ struct DecodeState {
     int nslot = 0, slot_bytes = 0, rpc = 0;
     int gu_units_max = 0, dn_units_max = 0;   // per-CTA unit counts the carve is sized for
     int off_ring = 0, off_router = 0, off_x16 = 0, off_xh = 0, off_logits = 0, off_htab = 0, off_red = 0,
-        off_misc = 0, off_resid = 0, off_sums = 0;
+        off_misc = 0, off_resid = 0, off_sums = 0, off_ltab = 0;
     int sms = 0;          // streaming multiprocessors of the device
     uint8_t *xbuf = nullptr;   // cross-CTA exchange area (counters, logits, h, output parts)
     bool withheld = false;     // the MOE_FLAG_TEST_WITHHOLD call has been made
