@@ -86,8 +86,8 @@ struct DecodeParams {
     float *yf_out;             // single layer: fp32 [d] or NULL
     int32_t *ids_out;          // single layer: [k] or NULL
     float *w_out;              // single layer: [k] or NULL
-    moe_stack_record rec;      // stack records (row 0 only)
-    int rec_on;
+    moe_stack_record rec;      // stack records: this token is record row rec_r of rec_n
+    int rec_on, rec_n, rec_r;
     unsigned *cnt;             // exchange counters: logits, h, y (128 bytes apart)
     float *x_logits;           // [E]
     float *x_h;                // [MAXU][I]
@@ -615,8 +615,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                         ss = fmaf(rn, rn, ss);
                         amx = fmaxf(amx, fabsf(rn));
                         if (cta == 0 && p.rec_on) {
-                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)(l - 1) * d + i] = yb;
-                            if (p.rec.y_f32) p.rec.y_f32[(size_t)(l - 1) * d + i] = y;
+                            const size_t ro = ((size_t)(l - 1) * p.rec_n + p.rec_r) * d + i;
+                            if (p.rec.y_bf16) p.rec.y_bf16[ro] = yb;
+                            if (p.rec.y_f32) p.rec.y_f32[ro] = y;
                         }
                     }
                 }
@@ -674,7 +675,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 if (cta == 0 && p.rec_on && p.rec.x_bf16) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        p.rec.x_bf16[(size_t)l * d + 8 * i8 + j] = (uint16_t)(xw[j >> 1] >> (16 * (j & 1)));
+                        p.rec.x_bf16[((size_t)l * p.rec_n + p.rec_r) * d + 8 * i8 + j] =
+                            (uint16_t)(xw[j >> 1] >> (16 * (j & 1)));
                 }
             } else {
                 const uint4 v = *reinterpret_cast<const uint4 *>(xb + 8 * i8);
@@ -858,8 +860,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 ms->uw[lane] = wj;
                 if (cta == 0) {
                     if (p.stack && p.rec_on) {
-                        if (p.rec.ids) p.rec.ids[(size_t)l * k + lane] = id;
-                        if (p.rec.w) p.rec.w[(size_t)l * k + lane] = wj;
+                        const size_t ro = ((size_t)l * p.rec_n + p.rec_r) * k + lane;
+                        if (p.rec.ids) p.rec.ids[ro] = id;
+                        if (p.rec.w) p.rec.w[ro] = wj;
                     }
                     if (!p.stack) {
                         if (p.ids_out) p.ids_out[lane] = id;
@@ -1214,8 +1217,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                     if (p.stack) {
                         p.resid_out[i] = rs[i] + bf16_bits_f(yb);
                         if (p.rec_on) {
-                            if (p.rec.y_bf16) p.rec.y_bf16[(size_t)l * d + i] = yb;
-                            if (p.rec.y_f32) p.rec.y_f32[(size_t)l * d + i] = y;
+                            const size_t ro = ((size_t)l * p.rec_n + p.rec_r) * d + i;
+                            if (p.rec.y_bf16) p.rec.y_bf16[ro] = yb;
+                            if (p.rec.y_f32) p.rec.y_f32[ro] = y;
                         }
                     } else {
                         p.y_out[i] = yb;
@@ -1229,9 +1233,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
 
 }  // namespace
 
-bool decode_supported(const moe_ctx *ctx, int T) {
+bool decode_supported(const moe_ctx *ctx) {
     const moe_config &c = ctx->cfg;
-    if (T != 1 || (c.flags & MOE_FLAG_NO_DECODE_KERNEL)) return false;
+    if (c.flags & MOE_FLAG_NO_DECODE_KERNEL) return false;
     // gate/up k chunks go to compute warps 0..d/256-1
     if (c.d_model > 4096 || c.d_model / 256 > NW || c.d_ff / 64 > 12) return false;
     if (c.n_experts % 4) return false;   // logits region of the exchange area stays 16-byte aligned
@@ -1314,7 +1318,7 @@ size_t decode_xchg_counter_bytes() { return XB_LOGITS; }
 
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
-                  cudaStream_t st) {
+                  int rec_n, int rec_r, cudaStream_t st) {
     const moe_config &c = ctx->cfg;
     DecodeState &ds = ctx->dec;
     DecodeParams p;
@@ -1340,6 +1344,8 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     if (rec) {
         p.rec = *rec;
         p.rec_on = 1;
+        p.rec_n = rec_n;
+        p.rec_r = rec_r;
     }
     p.cnt = reinterpret_cast<unsigned *>(ds.xbuf);
     p.x_logits = reinterpret_cast<float *>(ds.xbuf + XB_LOGITS);

@@ -224,9 +224,13 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
     Workspace &ws = ctx->ws;
     int32_t *ids_ = ids ? ids : ws.ids;
     float *w_ = w ? w : ws.w;
-    if (decode_supported(ctx, T)) {
+    if (T <= DECODE_TOKENS_MAX && decode_supported(ctx)) {
+        const moe_config &c = ctx->cfg;
         QE_TRY(timing_begin(ctx, st, "k_decode"));
-        QE_TRY(launch_decode(ctx, layer, 1, x, false, nullptr, y, yf, ids_, w_, nullptr, st));
+        for (int t = 0; t < T; ++t)
+            QE_TRY(launch_decode(ctx, layer, 1, x + (size_t)t * c.d_model, false, nullptr, y + (size_t)t * c.d_model,
+                                 yf ? yf + (size_t)t * c.d_model : nullptr, ids_ + (size_t)t * c.top_k,
+                                 w_ + (size_t)t * c.top_k, nullptr, 1, 0, st));
         QE_TRY(timing_end(ctx, st));
         return MOE_OK;
     }
@@ -314,11 +318,17 @@ int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint16_t *x_
     QE_CHECK(cudaSetDevice(ctx->device));
     cudaStream_t st = (cudaStream_t)stream;
     Workspace &ws = ctx->ws;
-    if (decode_supported(ctx, T)) {
+    // few tokens: the single-token kernel runs each token through the whole stack (records of
+    // every row, or of the one row of a single token; a device row list with more tokens takes
+    // the general path)
+    if (T <= DECODE_TOKENS_MAX && decode_supported(ctx) && (!rec || !rec->rows || T == 1)) {
         if (rec && rec->rows && rec->n_rows != 1) return MOE_ERR_INVALID_ARG;
+        const moe_config &c = ctx->cfg;
         QE_TRY(timing_begin(ctx, st, "k_decode"));
-        QE_TRY(launch_decode(ctx, layer0, n_layers, x_bf16, true, resid_out, nullptr, nullptr, nullptr,
-                             nullptr, rec, st));
+        for (int t = 0; t < T; ++t)
+            QE_TRY(launch_decode(ctx, layer0, n_layers, x_bf16 + (size_t)t * c.d_model, true,
+                                 resid_out + (size_t)t * c.d_model, nullptr, nullptr, nullptr, nullptr, rec,
+                                 rec && !rec->rows ? T : 1, rec && !rec->rows ? t : 0, st));
         QE_TRY(timing_end(ctx, st));
         return MOE_OK;
     }

@@ -252,12 +252,15 @@ int launch_combine(const moe_ctx *ctx, int T, const float *w, uint16_t *y, float
                    cudaStream_t st);
 int launch_resid_norm(const moe_ctx *ctx, int T, float *resid, const uint16_t *y_add,
                       const uint16_t *x_in, uint16_t *x_out, cudaStream_t st);
-bool decode_supported(const moe_ctx *ctx, int T);
+bool decode_supported(const moe_ctx *ctx);   // the shape fits the single-token kernel
+// Token counts up to this run the single-token kernel once per token (the tokens
+// of a layer, and of a stack, are independent).
+constexpr int DECODE_TOKENS_MAX = 16;
 int decode_setup(moe_ctx *ctx);
 size_t decode_xchg_bytes(const moe_config &c);
 size_t decode_xchg_counter_bytes();   // the counters at the start of the exchange area
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
-                  uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
+                  uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n, int rec_r,
                   cudaStream_t st);
 bool tc_supported(const moe_ctx *ctx, int T);
 bool tc_router_supported(const moe_ctx *ctx, int T);

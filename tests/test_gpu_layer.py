@@ -1,5 +1,7 @@
 """GPU parity of one MoE layer through the C ABI against the oracle, plus the
 edge cases and error codes of the boundary."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -11,6 +13,7 @@ from tests.parity import ExpertSource, bf16_tol, check_rows, oracle_rows, rel_l2
 pytestmark = pytest.mark.gpu
 
 TINY = synth.CONFIGS["tiny_d256_e16_q4_t8"]
+TINY_Q3 = dataclasses.replace(TINY, name="tiny_d256_e16_q3_t8", fmt="q3")
 
 
 def _cuda():
@@ -73,9 +76,10 @@ def test_tiny_ragged_token_counts(T):
 
 def test_batch_equals_single_tokens():
     """Token independence of the grouped path: a token's output does not depend
-    on which other tokens share the call (bit for bit)."""
+    on which other tokens share the call (bit for bit).  Pinned to the grouped
+    path: small calls would otherwise run the single-token kernel per token."""
     capi, session = _cuda()
-    sess = session.Session(TINY, max_tokens=64)
+    sess = session.Session(TINY, max_tokens=64, flags=capi.MOE_FLAG_NO_DECODE_KERNEL)
     sess.load_synthetic()
     x = _tokens(TINY, 37, stream=5)
     gy, gyf, gids, gw = _run(sess, 0, x)
@@ -88,7 +92,7 @@ def test_batch_equals_single_tokens():
     sess.close()
 
 
-@pytest.mark.parametrize("name", ["tiny_d256_e16_q4_t8", "decode_48l_q4_t1"])
+@pytest.mark.parametrize("name", ["tiny_d256_e16_q4_t8", "tiny_q3", "decode_48l_q4_t1", "verify_48l_q3_t4_zipf"])
 def test_decode_kernel_matches_general_path(name):
     """Single-token calls: the persistent decode kernel against the general
     grouped path on the same inputs (same ids; fp32 outputs within 5e-5).
@@ -99,7 +103,7 @@ def test_decode_kernel_matches_general_path(name):
     term is ~2^8 times the useful one), so the two paths agree to a few 1e-5,
     not to fp32 rounding."""
     capi, session = _cuda()
-    cfg = synth.CONFIGS[name]
+    cfg = TINY_Q3 if name == "tiny_q3" else synth.CONFIGS[name]
     a = session.Session(cfg, max_tokens=4, n_layers=1)
     b = session.Session(cfg, max_tokens=4, n_layers=1, flags=capi.MOE_FLAG_NO_DECODE_KERNEL)
     W = synth.layer_weights(cfg, 0, device="cuda")
@@ -173,6 +177,10 @@ def test_skew_every_token_to_the_same_experts():
 
 
 def test_zero_scale_routed_experts_leave_only_shared():
+    """With every routed expert's scales zeroed the layer is the shared expert
+    alone.  A routed expert that still contributed would move the output by
+    O(1) relative; the bound 5e-5 covers the single-token kernel's arithmetic
+    (the per-block offset removal leaves ~2^-16 relative per block partial)."""
     capi, session = _cuda()
     sess = session.Session(TINY, max_tokens=16)
 
@@ -186,7 +194,7 @@ def test_zero_scale_routed_experts_leave_only_shared():
     xf = oracle.bf16_to_f64(x)
     sh = tuple((Wh["sh_codes"][t][0].numpy(), Wh["sh_scales"][t][0].numpy()) for t in range(3))
     want = np.array([oracle.expert("q4", *sh, xf[t]) for t in range(8)])
-    assert rel_l2(gyf, want) <= 1e-6
+    assert rel_l2(gyf, want) <= 5e-5
     sess.close()
 
 
