@@ -77,7 +77,7 @@ struct Misc {
 struct DecodeParams {
     const LayerPtrs *layers;
     int layer0, L;
-    int fmt, d, E, I, k, nsh;
+    int d, E, I, k, nsh;
     MatLayout gu, dn;
     int stack;                 // 1: residual stream + rmsnorm between layers
     const uint16_t *x_in;      // bf16 [d]
@@ -96,7 +96,6 @@ struct DecodeParams {
     int withhold;              // test hook: CTA 0 does not publish its logits
     unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
-    int dn_units_max;          // largest down-unit run of one CTA
     int off_ring, off_router, off_x16, off_xh, off_logits, off_htab, off_red, off_misc, off_resid, off_sums,
         off_ltab;
 };
@@ -1326,7 +1325,6 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.layers = ctx->d_layers;
     p.layer0 = layer0;
     p.L = L;
-    p.fmt = c.fmt;
     p.d = c.d_model;
     p.E = c.n_experts;
     p.I = c.d_ff;
@@ -1373,7 +1371,6 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.nslot = ds.nslot;
     p.slot_bytes = ds.slot_bytes;
     p.rpc = ds.rpc;
-    p.dn_units_max = ds.dn_units_max;
     p.off_ring = ds.off_ring;
     p.off_router = ds.off_router;
     p.off_x16 = ds.off_x16;
