@@ -459,6 +459,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             const int pos0 = wi.y, rows = wi.z;
+            const int arows = rows > 128 ? TC_BM : 128;   // rows the MMAs read (one or two accumulators)
             int aoff[TC_ALD_MAXJ];                   // element offset of each chunk's row in A
 #pragma unroll
             for (int j = 0; j < TC_ALD_MAXJ; ++j) {
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
 #pragma unroll
                 for (int j = 0; j < TC_ALD_MAXJ; ++j) {
                     const int q = at + TC_ALD_NT * j;
-                    if (q < TC_BM * 8) cp_async16(a_dst + swz(q >> 3, ch * 8), p.A + aoff[j] + 64 * kx);
+                    if (q < arows * 8) cp_async16(a_dst + swz(q >> 3, ch * 8), p.A + aoff[j] + 64 * kx);
                 }
                 cp_async_commit();
                 if (pending >= 0) {   // the previous stage's rows have landed: publish them
