@@ -55,6 +55,27 @@ def router_bytes(cfg) -> int:
     return cfg.E * cfg.d * 4
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from one ncu capture of
+# the current kernels on one B200:
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \
+#       --clock-control none -k regex:k_decode -s 3 -c 1 \
+#       python bench.py --steps 3 --warmup 3 --no-secondary --cpu-layers 1 --layers 4
+# (a 4-layer stack: 118,442,240 B read + 2,858,752 B written; traffic grows with the layers a launch
+# runs, so a 48-layer launch is scaled by 48/4), and
+#   ncu ... -k regex:k_tc_gemm -s 9 -c 3 python bench.py --workload prefill_1l_q4_t4096_zipf \
+#       --steps 2 --warmup 3 --no-secondary --cpu-layers 1
+# (gate/up 375,051,776 + 34,839,808 B; down 259,929,856 + 23,429,120 B).
+DECODE_Q4_TRAFFIC_PER_LAYER = (118_442_240 + 2_858_752) / 4
+PREFILL_Q4_T4096_TRAFFIC = 375_051_776 + 34_839_808 + 259_929_856 + 23_429_120
+
+
+def decode_traffic(cfg, kernel: str):
+    """Measured DRAM bytes per launch of the single-token kernel for the Q4 decode shape."""
+    if kernel != "k_decode" or cfg.fmt != "q4" or cfg.T != 1 or (cfg.d, cfg.E, cfg.I, cfg.k) != (2560, 512, 512, 10):
+        return None
+    return DECODE_Q4_TRAFFIC_PER_LAYER * cfg.L
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -223,7 +244,7 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     avg_ms = tim["ms"] / max(1, tim["timed_launches"])
     achieved = alg_bytes / (avg_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / P["hbm_gbs"], "traffic": None, "kernel": tim["kernel"],
+            "frac": achieved / P["hbm_gbs"], "traffic": decode_traffic(cfg, tim["kernel"]), "kernel": tim["kernel"],
             "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_ms,
             "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
 
@@ -321,7 +342,8 @@ def secondary_prefill(args, local_rank) -> dict:
             "roofline": {"bound": "tensor", "kernel": tim["kernel"],
                          "achieved": flops_expert / (kms / 1e3) / 1e12,
                          "peak": P["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": flops_expert / (kms / 1e3) / 1e12 / P["bf16_tflops_sustained"]},
+                         "frac": flops_expert / (kms / 1e3) / 1e12 / P["bf16_tflops_sustained"],
+                         "traffic": PREFILL_Q4_T4096_TRAFFIC if cfg.name == "prefill_1l_q4_t4096_zipf" else None},
             "l2": "256 MB flush between timed calls"}
 
 
