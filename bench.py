@@ -69,6 +69,19 @@ DECODE_Q4_TRAFFIC_PER_LAYER = (118_442_240 + 2_858_752) / 4
 PREFILL_Q4_T4096_TRAFFIC = 375_051_776 + 34_839_808 + 259_929_856 + 23_429_120
 
 
+def max_over_ranks(v: float, dist_on: bool, device) -> float:
+    """The largest of every rank's value (a time): the job takes as long as its slowest rank."""
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """Units processed by all ranks together per second (weak scaling: fixed units per rank)."""
+    return units_per_rank * world / seconds
+
+
 def decode_traffic(cfg, kernel: str):
     """Measured DRAM bytes per launch of the single-token kernel for the Q4 decode shape."""
     if kernel != "k_decode" or cfg.fmt != "q4" or cfg.T != 1 or (cfg.d, cfg.E, cfg.I, cfg.k) != (2560, 512, 512, 10):
@@ -224,12 +237,9 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     with Clocks(local_rank) as clk:
         ms, tim = timed_stack(sess, cfg, xs, r_out, args.steps, args.warmup, stream, dist_on)
     clocks = clk.summary()
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist_on:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dist_on, dev)
     ms_step = ms_max / args.steps
-    value = cfg.T * world / (ms_step / 1e3)
+    value = whole_job_rate(cfg.T, world, ms_step / 1e3)
 
     # roofline of the dominant (timed) kernel: expert weight bytes it streams
     # per launch (one launch per layer; T=1 -> k routed + shared experts)
@@ -259,10 +269,8 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     t0 = time.perf_counter()
     for s in range(args.steps):
         capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[args.warmup + s], cfg.T, r_host, stream)
-    e2e_s = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=dev)
-    if dist_on:
-        torch.distributed.all_reduce(e2e_s, op=torch.distributed.ReduceOp.MAX)
-    e2e = {"value": cfg.T * world * args.steps / float(e2e_s.item()), "unit": "tok/s",
+    e2e_s = max_over_ranks(time.perf_counter() - t0, dist_on, dev)
+    e2e = {"value": whole_job_rate(cfg.T * args.steps, world, e2e_s), "unit": "tok/s",
            "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
            "timer": "host wall clock around synchronous calls"}
     sess.close()
