@@ -88,7 +88,7 @@ typedef struct {
  * kernel's CTA 0 withholds its router logits, every wait on them runs out
  * after about one second, and the call reports MOE_ERR_DEVICE_TIMEOUT through
  * moe_get_device_error; later calls run normally. */
-#define MOE_FLAG_NO_DECODE_KERNEL 1   /* T == 1 runs the general path */
+#define MOE_FLAG_NO_DECODE_KERNEL 1   /* small T runs the general path, not the single-token kernel */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
 #define MOE_FLAG_TRACE 4              /* record per-phase timestamps (moe_trace_read) */
@@ -136,7 +136,11 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  *   before the bf16 rounding, or NULL; ids [T][k] chosen experts (descending
  *   weight) and w [T][k] their weights, either may be NULL.
  * Asynchronous on `stream`; no host synchronisation and no allocation.
- * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA. */
+ * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA.
+ * Implementation (not part of the contract): up to 16 tokens run the
+ * persistent single-token kernel once per token, fewer than 64 the CUDA-core
+ * grouped path, 64 and more the tensor-core grouped GEMMs; each path meets the
+ * same accuracy bound. */
 MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
                 uint16_t *y_bf16, float *y_f32, int32_t *ids, float *w,
                 void *stream);
