@@ -241,16 +241,18 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     ms_step = ms_max / args.steps
     value = whole_job_rate(cfg.T, world, ms_step / 1e3)
 
-    # roofline of the dominant (timed) kernel: expert weight bytes it streams
-    # per launch (one launch per layer; T=1 -> k routed + shared experts)
-    union = cfg.k if cfg.T == 1 else None
-    if union is None:
-        union = measured_union(sess, cfg, xs[0], dev)
-    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+    # roofline of the dominant (timed) kernel: the bytes it must stream per launch.  The
+    # single-token kernel runs one token through the whole stack per launch: k routed + the
+    # shared experts and the router rows of every layer; the grouped paths launch once per
+    # layer and stream the union of the batch's experts
+    union = cfg.k if cfg.T == 1 else measured_union(sess, cfg, xs[0], dev)
     if tim["kernel"] == "k_decode":
-        alg_bytes = step_bytes          # one launch runs the whole stack (router rows included)
+        alg_bytes = cfg.L * ((cfg.k + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
     else:
-        alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)   # one launch per layer, experts only
+        alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)   # experts only
+    # the step's algorithmic bytes: every layer's router rows and the union of the experts the
+    # batch's tokens chose (a path that streams some of them more than once moves more)
+    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
     avg_ms = tim["ms"] / max(1, tim["timed_launches"])
     achieved = alg_bytes / (avg_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",

@@ -977,7 +977,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         }
         trace_mark(p, l, 3, clock64() - tl0);
 
-        // h of every expert in use -> bf16 hi + lo table and per-block sums of hi + lo
+        // h of every expert in use -> hi + lo table (B-fragment order) and per-block sums of hi + lo
         {
             csync();   // this CTA's h values are stored
             if (tid == 0) {
