@@ -119,6 +119,12 @@ typedef struct {
 
 typedef struct moe_ctx moe_ctx;
 
+/* A context owns one workspace (intermediates, the single-token kernel's
+ * exchange buffers and counters).  Its forward calls must therefore run one
+ * after another on the device: issue them on one stream, or order them with
+ * events; calls that overlap on the GPU corrupt each other's results.  Use
+ * one context per concurrent stream. */
+
 /* Create a context on CUDA device `device` and allocate its workspace (sized
  * by max_tokens).  *out receives the handle.  Errors: INVALID_ARG (bad
  * config), UNSUPPORTED (shape outside the limits above), OOM, CUDA. */

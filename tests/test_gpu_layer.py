@@ -61,7 +61,7 @@ def test_tiny_layer_all_tokens(fmt):
     sess.close()
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 5, 127, 128, 129])
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 16, 17, 63, 64, 127, 128, 129])
 def test_tiny_ragged_token_counts(T):
     capi, session = _cuda()
     sess = session.Session(TINY, max_tokens=256)
