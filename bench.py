@@ -62,11 +62,11 @@ def router_bytes(cfg) -> int:
 #       python bench.py --steps 3 --warmup 3 --no-secondary --cpu-layers 1 --layers 4
 # (a 4-layer stack: 118,442,240 B read + 2,858,752 B written; traffic grows with the layers a launch
 # runs, so a 48-layer launch is scaled by 48/4), and
-#   ncu ... -k regex:k_tc_gemm -s 9 -c 3 python bench.py --workload prefill_1l_q4_t4096_zipf \
-#       --steps 2 --warmup 3 --no-secondary --cpu-layers 1
-# (gate/up 375,051,776 + 34,839,808 B; down 259,929,856 + 23,429,120 B).
+#   ncu ... -k regex:"k_tc_gemm|k_cache_fill" -s 12 -c 4 python bench.py \
+#       --workload prefill_1l_q4_t4096_zipf --steps 2 --warmup 3 --no-secondary --cpu-layers 1
+# (the cache fill and the two expert GEMMs of one layer; router excluded).
 DECODE_Q4_TRAFFIC_PER_LAYER = (118_442_240 + 2_858_752) / 4
-PREFILL_Q4_T4096_TRAFFIC = 375_051_776 + 34_839_808 + 259_929_856 + 23_429_120
+PREFILL_Q4_T4096_TRAFFIC = None   # set from the capture of the current kernels
 
 
 def max_over_ranks(v: float, dist_on: bool, device) -> float:
@@ -353,7 +353,8 @@ def secondary_prefill(args, local_rank) -> dict:
                          "achieved": flops_expert / (kms / 1e3) / 1e12,
                          "peak": P["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": flops_expert / (kms / 1e3) / 1e12 / P["bf16_tflops_sustained"],
-                         "traffic": PREFILL_Q4_T4096_TRAFFIC if cfg.name == "prefill_1l_q4_t4096_zipf" else None},
+                         "traffic": PREFILL_Q4_T4096_TRAFFIC if cfg.name == "prefill_1l_q4_t4096_zipf" else None,
+                         "traffic_kernels": "k_cache_fill + k_tc_gemm<gate/up> + k_tc_gemm<down>"},
             "l2": "256 MB flush between timed calls"}
 
 

@@ -127,7 +127,11 @@ typedef struct moe_ctx moe_ctx;
 
 /* Create a context on CUDA device `device` and allocate its workspace (sized
  * by max_tokens).  *out receives the handle.  Errors: INVALID_ARG (bad
- * config), UNSUPPORTED (shape outside the limits above), OOM, CUDA. */
+ * config), UNSUPPORTED (shape outside the limits above), OOM, CUDA.
+ * When the tensor-core path can run, the workspace also holds a decoded-weight
+ * cache of min(experts, max_tokens * (top_k + n_shared) / 256) experts
+ * (6 * d_model * d_ff bytes each) if it fits device_mem_limit; without it the
+ * results are the same, only slower. */
 MOE_API int moe_create(const moe_config *cfg, int device, moe_ctx **out);
 
 /* Copy one layer's weights into the context (repacking them on the device)

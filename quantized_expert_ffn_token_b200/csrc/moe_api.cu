@@ -131,6 +131,25 @@ int alloc_workspace(moe_ctx *ctx) {
     ws.tc_items_max = tc_items_max(c);
     for (auto &it : items) QE_TRY(ctx_alloc(ctx, it.p, it.bytes, it.name));
     QE_TRY(ctx_alloc(ctx, (void **)&ws.tc_items, ws.tc_items_max * sizeof(int4), "tc_items"));
+    QE_TRY(ctx_alloc(ctx, (void **)&ws.cache_slot, (size_t)ctx->nx * 4, "cache_slot"));
+    QE_TRY(ctx_alloc(ctx, (void **)&ws.cache_n, 4, "cache_n"));
+    {
+        // decoded-weight cache: at most one slot per 256 grouped rows beyond the first block of
+        // an expert; optional: left out when it does not fit the memory limit or the device
+        size_t per = (size_t)6 * c.d_model * c.d_ff;   // bytes of one expert's fp16 B stages
+        size_t cap = (size_t)c.max_tokens * (c.top_k + c.n_shared) / 256;
+        if (cap > (size_t)ctx->nx) cap = ctx->nx;
+        if (!tc_supported(ctx, 64)) cap = 0;   // only the tensor-core path reads it
+        long long lim = c.device_mem_limit;
+        if (cap > 0 && lim > 0 && (long long)(ctx->allocated + cap * per + cap * 4) > lim) cap = 0;
+        if (cap > 0 && ctx_alloc(ctx, (void **)&ws.wcache, cap * per, "weight cache") != MOE_OK) cap = 0;
+        if (cap > 0 && ctx_alloc(ctx, (void **)&ws.cache_expert, cap * 4, "cache_expert") != MOE_OK) {
+            ctx_free(ctx, ws.wcache);
+            ws.wcache = nullptr;
+            cap = 0;
+        }
+        ws.cache_cap = (int)cap;
+    }
     QE_CHECK(cudaMemset(ws.dev_error, 0, 4));
     QE_TRY(ctx_alloc(ctx, (void **)&ctx->d_layers, sizeof(LayerPtrs) * c.n_layers, "layer table"));
     QE_CHECK(cudaMemset(ctx->d_layers, 0, sizeof(LayerPtrs) * c.n_layers));

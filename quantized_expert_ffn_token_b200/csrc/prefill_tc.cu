@@ -77,6 +77,11 @@ struct TcParams {
     const float *rbias;         // [E]
     float *logits;              // [T][E]
     int n_items_direct;         // router: items computed from the index (no item list)
+    // decoded-weight cache: stage images of experts with more than one 256-row block
+    const uint16_t *wcache;     // [slot][gate/up stages, down stages][256 x 64 fp16, swizzled]
+    const int32_t *cache_slot;  // [expert] slot or -1 (NULL: no cache)
+    size_t cache_off;           // fp16 offset of this GEMM's stages within a slot
+    size_t cache_stride;        // fp16 per slot (3 d I)
     int *err;
 };
 
@@ -114,6 +119,17 @@ __device__ __forceinline__ bool mbar_wait_b(uint64_t *b, uint32_t parity, int *e
     }
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// This thread's arrival on *b, adding `bytes` of expected transfer to the phase.
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+// Bulk copy global -> shared (16-byte aligned, size a multiple of 16), completing on *b.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *b) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     su32(dst)),
+                 "l"(src), "r"(bytes), "r"(su32(b))
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(su32(dst)), "l"(src) : "memory");
 }
@@ -395,6 +411,29 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             // weights: this warp decodes row tiles 2*pw and 2*pw+1 of the 16 in the n-tile
             const uint8_t *wexp = p.W + (size_t)e * p.L.expert_bytes;
             const int nb = p.K / 32;
+            if constexpr (MODE != TC_ROUTER) {
+                const int cslot = p.cache_slot ? p.cache_slot[e] : -1;
+                if (cslot >= 0) {
+                    // the expert's stage images were decoded once already: one bulk copy per stage
+                    // (its bytes complete the stage's barrier together with every producer's arrival)
+                    const uint16_t *cs = p.wcache + (size_t)cslot * p.cache_stride + p.cache_off +
+                                         (size_t)nt * nk * (B_STAGE_BYTES / 2);
+                    for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+                        int s = it % TC_STAGES;
+                        ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
+                        if (!ok) break;
+                        if (pt == 0) {
+                            fence_async_smem();
+                            mbar_arrive_tx(&ss->full[s], B_STAGE_BYTES);
+                            bulk_copy_g2s(sB + s * B_STAGE_BYTES, cs + (size_t)kb * (B_STAGE_BYTES / 2),
+                                          B_STAGE_BYTES, &ss->full[s]);
+                        } else {
+                            mbar_arrive(&ss->full[s]);
+                        }
+                    }
+                    continue;
+                }
+            }
             for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                 int s = it % TC_STAGES;
                 ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
@@ -587,6 +626,78 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// Cache slots for the experts with more than one 256-row block (slot order is
+// arbitrary; slots past the capacity fall back to decoding in the GEMM).
+__global__ void k_cache_assign(const int32_t *__restrict__ counts, int nx, int cap, int32_t *__restrict__ slot,
+                               int32_t *__restrict__ expert, int32_t *__restrict__ n_used) {
+    for (int e = threadIdx.x; e < nx; e += blockDim.x) {
+        int sl = -1;
+        if (counts[e] > TC_BM) {
+            sl = atomicAdd(n_used, 1);
+            if (sl >= cap) sl = -1;
+            else expert[sl] = e;
+        }
+        slot[e] = sl;
+    }
+}
+
+// Decode the stage images of every cached expert: unit = (slot, GEMM, n-tile,
+// k group); 8 warps decode the 16 row tiles of the n-tile exactly as the GEMM's
+// producers do (same function, same bytes, same fp16 values) into shared
+// memory, then the 32 KB image is written out.
+template <int FMT>
+__global__ void __launch_bounds__(256) k_cache_fill(const uint8_t *__restrict__ gu, MatLayout Lg,
+                                                    const uint8_t *__restrict__ dn, MatLayout Ld,
+                                                    const int32_t *__restrict__ expert,
+                                                    const int32_t *__restrict__ n_used, int cap,
+                                                    uint16_t *__restrict__ wcache, int d, int I) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *stage = smem_raw + ((1024 - (su32(smem_raw) & 1023)) & 1023);   // 32 KB, 1024-aligned
+    uint8_t *raw = stage + B_STAGE_BYTES;                                     // 3 x RAW_FIELD
+    const int pt = threadIdx.x, pw = pt >> 5, lane = pt & 31, g = lane >> 2;
+    const int nslot = min(*n_used, cap);
+    const int ntg = 2 * I / TC_BN, nkg = d / TC_BK;      // gate/up stages per n-tile row
+    const int ntd = d / TC_BN, nkd = I / TC_BK;          // down
+    const int per_slot = ntg * nkg + ntd * nkd;
+    const size_t stride = (size_t)3 * d * I;
+    for (int u = blockIdx.x; u < nslot * per_slot; u += gridDim.x) {
+        const int sl = u / per_slot;
+        int r = u - sl * per_slot;
+        const bool gate = r < ntg * nkg;
+        if (!gate) r -= ntg * nkg;
+        const int nk = gate ? nkg : nkd;
+        const int nt = r / nk, kb = r - nt * nk;
+        const MatLayout &L = gate ? Lg : Ld;
+        const uint8_t *wexp = (gate ? gu : dn) + (size_t)expert[sl] * L.expert_bytes;
+        const int nb = L.K / 32;
+        uint8_t *myraw = raw + pt * 16;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const uint8_t *tile = wexp + (size_t)(nt * 16 + 2 * pw + tt) * L.tile_bytes;
+            const uint8_t *cs = tile + (size_t)kb * L.kg_bytes;
+            if constexpr (FMT == MOE_Q4B32) {
+                cp_async16(myraw + tt * RAW_FIELD, cs + lane * 16);
+            } else {
+                cp_async4(myraw + tt * RAW_FIELD, cs + lane * 12);
+                cp_async4(myraw + tt * RAW_FIELD + 4, cs + lane * 12 + 4);
+                cp_async4(myraw + tt * RAW_FIELD + 8, cs + lane * 12 + 8);
+            }
+            const uint8_t *sc = tile + L.code_bytes;
+            cp_async4(myraw + 2 * RAW_FIELD + 8 * tt, sc + (size_t)(g * nb + 2 * kb) * 2);
+            cp_async4(myraw + 2 * RAW_FIELD + 4 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        decode_stage<FMT>(myraw, stage, pw, lane);
+        __syncthreads();
+        uint16_t *dst = wcache + (size_t)sl * stride + (gate ? 0 : (size_t)2 * I * d) +
+                        ((size_t)nt * nk + kb) * (B_STAGE_BYTES / 2);
+        for (int i = pt; i < B_STAGE_BYTES / 16; i += 256)
+            reinterpret_cast<uint4 *>(dst)[i] = reinterpret_cast<const uint4 *>(stage)[i];
+        __syncthreads();
+    }
+}
+
 // Work items of one GEMM: for every expert with slots, ceil(cnt/256) row
 // blocks x n_tiles column tiles.  Single block.
 __global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int nx,
@@ -721,10 +832,37 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.d = c.d_model;
     p.err = ws.dev_error;
 
+    // decoded-weight cache for the experts with more than one 256-row block (part of the timed
+    // expert work: it takes over decoding from the GEMMs)
+    QE_TRY(timing_begin(ctx, st, "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>"));
+    if (ws.cache_cap > 0) {
+        QE_CHECK(cudaMemsetAsync(ws.cache_n, 0, 4, st));
+        k_cache_assign<<<1, 1024, 0, st>>>(ws.counts, ctx->nx, ws.cache_cap, ws.cache_slot, ws.cache_expert,
+                                           ws.cache_n);
+        QE_CHECK_LAUNCH("k_cache_assign");
+        const size_t fsm = B_STAGE_BYTES + 3 * RAW_FIELD + 1024;
+        if (c.fmt == MOE_Q4B32) {
+            QE_CHECK(cudaFuncSetAttribute(k_cache_fill<MOE_Q4B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm));
+            k_cache_fill<MOE_Q4B32><<<4 * dev_sms, 256, fsm, st>>>(Ly.gu, ctx->gu, Ly.dn, ctx->dn, ws.cache_expert,
+                                                                   ws.cache_n, ws.cache_cap, ws.wcache, c.d_model,
+                                                                   c.d_ff);
+        } else {
+            QE_CHECK(cudaFuncSetAttribute(k_cache_fill<MOE_Q3B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm));
+            k_cache_fill<MOE_Q3B32><<<4 * dev_sms, 256, fsm, st>>>(Ly.gu, ctx->gu, Ly.dn, ctx->dn, ws.cache_expert,
+                                                                   ws.cache_n, ws.cache_cap, ws.wcache, c.d_model,
+                                                                   c.d_ff);
+        }
+        QE_CHECK_LAUNCH("k_cache_fill");
+        p.wcache = ws.wcache;
+        p.cache_slot = ws.cache_slot;
+        p.cache_stride = (size_t)3 * c.d_model * c.d_ff;
+    }
+
     // gate/up: A = x16 rows gathered by token, N = 2I, K = d
     k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, (2 * c.d_ff) / TC_BN, ws.tc_items,
                                    ws.tc_n_items, max_items);
     QE_CHECK_LAUNCH("k_tc_items");
+    p.cache_off = 0;
     p.K = c.d_model;
     p.N = 2 * c.d_ff;
     p.L = ctx->gu;
@@ -733,7 +871,6 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.a_by_token = 1;
     p.h16 = ws.h16;
     int grid = dev_sms;
-    QE_TRY(timing_begin(ctx, st, "k_tc_gemm<gate/up>+k_tc_gemm<down>"));
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_GATEUP>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_GATEUP>(p, grid, st)));
 
@@ -750,6 +887,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.a_by_token = 0;
     p.y_acc = ws.y_acc;
     p.w_route = w_route;
+    p.cache_off = (size_t)2 * c.d_ff * c.d_model;   // the down GEMM's stages follow the gate/up ones
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_DOWN>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_DOWN>(p, grid, st)));
     QE_TRY(timing_end(ctx, st));
