@@ -66,7 +66,9 @@ def router_bytes(cfg) -> int:
 #       --workload prefill_1l_q4_t4096_zipf --steps 2 --warmup 3 --no-secondary --cpu-layers 1
 # (the cache fill and the two expert GEMMs of one layer; router excluded).
 DECODE_Q4_TRAFFIC_PER_LAYER = (118_442_240 + 2_858_752) / 4
-PREFILL_Q4_T4096_TRAFFIC = None   # set from the capture of the current kernels
+PREFILL_Q4_T4096_TRAFFIC = (61_968_640 + 157_297_920          # k_cache_fill
+                            + 500_800_256 + 41_342_720        # k_tc_gemm<gate/up>
+                            + 341_344_768 + 61_933_312)       # k_tc_gemm<down>
 
 
 def max_over_ranks(v: float, dist_on: bool, device) -> float:
