@@ -11,6 +11,12 @@ inputs resident in HBM.  Prints one JSON line (rank 0).
 N > 1 (under torchrun): independent replicas, one per GPU, each decoding its
 own tokens (the layer does not shard for one token stream); value = tokens
 of all ranks / max-over-ranks time.
+
+  python bench.py --sweep [--sweep-workload W] [--sweep-t 1,2,...]
+
+times one layer at each token count on every path that accepts it (single-token
+kernel, CUDA-core path, tensor-core path) and ends with the fastest path per
+token count next to the one the library's dispatch picks.
 """
 from __future__ import annotations
 
@@ -360,6 +366,100 @@ def secondary_prefill(args, local_rank) -> dict:
             "l2": "256 MB flush between timed calls"}
 
 
+# ---- token-count sweep (python bench.py --sweep): one layer, every path that accepts T ------------
+
+# The library's path selection by T (include/moe.h, moe_forward): the single-token kernel once per
+# token up to DISPATCH_DECODE_MAX tokens, the tensor-core path from DISPATCH_TC_MIN tokens, the
+# CUDA-core path in between.  The flags below pin a context to one path.
+DISPATCH_DECODE_MAX = 16
+DISPATCH_TC_MIN = 64
+SWEEP_T = (1, 2, 4, 8, 16, 17, 32, 48, 63, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
+SWEEP_PATHS = ("single-token kernel", "cuda-core", "tensor-core")
+
+
+def sweep_flags(path: str) -> int:
+    no_decode, no_tensor = 1, 2   # MOE_FLAG_NO_DECODE_KERNEL, MOE_FLAG_NO_TENSOR_PREFILL
+    return {"single-token kernel": 0, "cuda-core": no_decode | no_tensor, "tensor-core": no_decode}[path]
+
+
+def sweep_eligible(path: str, T: int) -> bool:
+    """Whether a context pinned to `path` runs T tokens on that path."""
+    if path == "single-token kernel":
+        return T <= DISPATCH_DECODE_MAX
+    if path == "tensor-core":
+        return T >= DISPATCH_TC_MIN
+    return True
+
+
+def default_path(T: int) -> str:
+    if T <= DISPATCH_DECODE_MAX:
+        return "single-token kernel"
+    return "tensor-core" if T >= DISPATCH_TC_MIN else "cuda-core"
+
+
+def sweep_summary(rows: list[dict]) -> list[dict]:
+    """Per T: the fastest measured path and whether the default dispatch picks it."""
+    out = []
+    for T in sorted({r["T"] for r in rows}):
+        at = [r for r in rows if r["T"] == T]
+        best = min(at, key=lambda r: r["ms"])
+        dflt = next((r for r in at if r["path"] == default_path(T)), None)
+        out.append({"T": T, "fastest": best["path"], "fastest_ms": best["ms"],
+                    "default": default_path(T), "default_ms": dflt["ms"] if dflt else None,
+                    "default_is_fastest": dflt is not None and dflt["path"] == best["path"]})
+    return out
+
+
+def sweep(args, local_rank) -> list[dict]:
+    """Time one layer of `args.sweep_workload` at every T of the sweep on every path that accepts
+    it: a 256 MB L2 flush before each timed call, CUDA events on the call's stream, median of
+    args.steps calls after args.warmup untimed ones.  Prints one JSON line per (T, path)."""
+    from quantized_expert_ffn_token_b200 import capi, session
+    cfg = synth.CONFIGS[args.sweep_workload]
+    Ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else list(SWEEP_T)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    x_all = torch.from_numpy(synth.tokens_bf16(cfg, T=max(Ts)).view(np.int16)).to(dev)
+    rows = []
+    for path in SWEEP_PATHS:
+        ts = [T for T in Ts if sweep_eligible(path, T)]
+        if not ts:
+            continue
+        sess = session.Session(cfg, device=local_rank, max_tokens=max(ts), n_layers=1, flags=sweep_flags(path))
+        sess.load_synthetic(stream=stream)
+        torch.cuda.synchronize()
+        for T in ts:
+            x = x_all[:T]
+            y = torch.empty((T, cfg.d), dtype=torch.int16, device=dev)
+            ids = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+            for _ in range(args.warmup):
+                capi.moe_forward(sess.ctx, 0, x, T, y, None, ids, None, stream)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(args.steps):
+                with torch.cuda.stream(stream):
+                    flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                capi.moe_forward(sess.ctx, 0, x, T, y, None, ids, None, stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            ms = statistics.median(times)
+            union = int(torch.unique(ids).numel())
+            nbytes = (union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg)
+            flops = 2 * T * (cfg.k + cfg.n_shared) * 3 * cfg.d * cfg.I + 2 * T * cfg.E * cfg.d
+            row = {"sweep": cfg.name, "T": T, "path": path, "ms": ms, "tok_per_s": T / (ms / 1e3),
+                   "experts_touched": union + cfg.n_shared,
+                   "alg_gbs": nbytes / (ms / 1e3) / 1e9, "tflops": flops / (ms / 1e3) / 1e12}
+            print(json.dumps(row), flush=True)
+            rows.append(row)
+        sess.close()
+        torch.cuda.synchronize()
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,6 +472,11 @@ def main():
     ap.add_argument("--ref-layers", type=int, default=2, help="reference arm: layers per step")
     ap.add_argument("--layers", type=int, default=None,
                     help="stack depth override (small cases for profiler captures)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="token-count sweep of one layer over every path (one JSON line per T and path)")
+    ap.add_argument("--sweep-workload", default="prefill_1l_q4_t4096_zipf", choices=sorted(synth.CONFIGS),
+                    help="layer shape and routing of the sweep (layer 0 of this workload)")
+    ap.add_argument("--sweep-t", default=None, help="comma-separated token counts (default: 1 ... 8192)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     cfg = synth.CONFIGS[args.workload]
@@ -383,6 +488,14 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     dist_on = world > 1
+
+    if args.sweep:
+        if rank != 0:
+            return 0
+        rows = sweep(args, local_rank)
+        print(json.dumps({"sweep_summary": sweep_summary(rows), "l2": "256 MB flush between timed calls",
+                          "steps": args.steps, "warmup": args.warmup}))
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
