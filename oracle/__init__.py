@@ -24,10 +24,10 @@ _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-Q4B32, Q3B32 = 1, 2
-FMT = {"q4": Q4B32, "q3": Q3B32}
-ZERO = {Q4B32: 8, Q3B32: 4}
-BLOCK_BYTES = {Q4B32: 16, Q3B32: 12}
+Q4B32, Q3B32, Q2B32 = 1, 2, 3
+FMT = {"q4": Q4B32, "q3": Q3B32, "q2": Q2B32}
+ZERO = {Q4B32: 8, Q3B32: 4, Q2B32: 2}
+BLOCK_BYTES = {Q4B32: 16, Q3B32: 12, Q2B32: 8}
 
 _dp = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _fp = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
@@ -136,15 +136,15 @@ def round_bf16(v) -> np.ndarray:
 
 
 def block_codes(fmt, blk) -> np.ndarray:
-    """The 32 codes of one packed block (Q4B32: nibbles, low first; Q3B32: 3-bit
-    fields of a little-endian 96-bit integer)."""
+    """The 32 codes of one packed block (Q4B32: nibbles, low first; Q3B32 / Q2B32:
+    3-bit / 2-bit fields of a little-endian 96-bit / 64-bit integer)."""
     f = _fmt(fmt)
     blk = _u8a(blk)
     return np.array([lib().oracle_code(f, blk, j) for j in range(32)], dtype=np.int64)
 
 
 def block_weights(fmt, blk, scale_bits) -> np.ndarray:
-    """w_j = s * (q_j - 8) (Q4B32) or s * (q_j - 4) (Q3B32)."""
+    """w_j = s * (q_j - 8) (Q4B32), s * (q_j - 4) (Q3B32) or s * (q_j - 2) (Q2B32)."""
     f = _fmt(fmt)
     blk = _u8a(blk)
     return np.array([lib().oracle_weight(f, blk, int(scale_bits) & 0xFFFF, j) for j in range(32)])

@@ -23,7 +23,11 @@
  *     chosen k; shared expert weight 1;
  *   - block formats Q4B32 and Q3B32 (the pages name IQ3_S, IQ2_XS, Q2_0 ...
  *     but never define a layout; "Running Qwen3.8-Flash-Next on a 4090 24GB",
- *     section "The engine rejects Unsloth's embedding format").
+ *     section "The engine rejects Unsloth's embedding format"), and the
+ *     2-bit Q2B32 for the pages' fastest size, Q2_0 ("Strata: Qwen3.8-Flash-
+ *     Next (125B Moe) on a 8GB+ Nvidia GPU", tables "How fast?" and "The
+ *     size"; video transcript 6:18-6:32), defined the same way: 32 codes and
+ *     one fp16 scale, the zero point at half the code range.
  *
  * Every function below computes in fp64.  Parity of each is pinned by the
  * CPU tests against hand-built blocks, closed forms, brute force and the
@@ -36,6 +40,7 @@
 
 #define ORACLE_Q4B32 1
 #define ORACLE_Q3B32 2
+#define ORACLE_Q2B32 3
 
 /* IEEE 754 binary16 -> double, written from the format's definition:
  * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
@@ -65,13 +70,17 @@ double oracle_bf16_to_double(uint16_t b)
  * Q4B32: 16 bytes, two 4-bit codes per byte; byte b holds code 2b in its low
  *        nibble and code 2b+1 in its high nibble.
  * Q3B32: 12 bytes read as one 96-bit little-endian integer; code j is bits
- *        3j..3j+2 (bit 0 of byte 0 is the least significant bit). */
+ *        3j..3j+2 (bit 0 of byte 0 is the least significant bit).
+ * Q2B32: 8 bytes read as one 64-bit little-endian integer; code j is bits
+ *        2j..2j+1, i.e. byte j/4, starting at bit 2*(j mod 4). */
 int oracle_code(int fmt, const uint8_t *blk, int j)
 {
     if (fmt == ORACLE_Q4B32) {
         uint8_t byte = blk[j >> 1];
         return (j & 1) ? (byte >> 4) : (byte & 15);
     }
+    if (fmt == ORACLE_Q2B32)
+        return (blk[j >> 2] >> (2 * (j & 3))) & 3;
     int v = 0;
     for (int t = 0; t < 3; ++t) {
         int bit = 3 * j + t;
@@ -81,14 +90,14 @@ int oracle_code(int fmt, const uint8_t *blk, int j)
 }
 
 /* Weight j of a block: w = s * (q - 8) for Q4B32, w = s * (q - 4) for Q3B32,
- * s the block's fp16 scale. */
+ * w = s * (q - 2) for Q2B32, s the block's fp16 scale. */
 double oracle_weight(int fmt, const uint8_t *blk, uint16_t scale, int j)
 {
-    int zero = (fmt == ORACLE_Q4B32) ? 8 : 4;
+    int zero = (fmt == ORACLE_Q4B32) ? 8 : (fmt == ORACLE_Q2B32) ? 2 : 4;
     return oracle_half_to_double(scale) * (double)(oracle_code(fmt, blk, j) - zero);
 }
 
-static int block_bytes(int fmt) { return fmt == ORACLE_Q4B32 ? 16 : 12; }
+static int block_bytes(int fmt) { return fmt == ORACLE_Q4B32 ? 16 : (fmt == ORACLE_Q2B32) ? 8 : 12; }
 
 /* y[r] = sum_k W[r][k] x[k] for a packed matrix of `rows` rows and K columns,
  * blocks of 32 running along k: codes [rows][K/32][B], scales [rows][K/32]. */

@@ -57,7 +57,7 @@ class LayerConfig:
     I_s: int            # shared expert intermediate size
     L: int              # layers in the stack
     T: int              # tokens per call
-    fmt: str            # "q4" (Q4B32) or "q3" (Q3B32)
+    fmt: str            # "q4" (Q4B32), "q3" (Q3B32) or "q2" (Q2B32)
     scale_lo: float
     scale_hi: float
     zipf_s: float | None  # Zipf exponent of the router bias, None = no bias
@@ -70,7 +70,7 @@ class LayerConfig:
 
 def block_bytes(fmt: str) -> int:
     """Bytes of packed codes in one 32-weight block."""
-    return {"q4": 16, "q3": 12}[fmt]
+    return {"q4": 16, "q3": 12, "q2": 8}[fmt]
 
 
 CONFIGS = {

@@ -76,7 +76,7 @@ def _golden():
     return rows
 
 
-@pytest.mark.parametrize("case", range(7))
+@pytest.mark.parametrize("case", range(len(_golden())))
 def test_golden_blocks(case):
     fmt, blk, sbits, want = _golden()[case]
     got = oracle.block_weights(fmt, np.frombuffer(blk, np.uint8), sbits)
@@ -84,16 +84,16 @@ def test_golden_blocks(case):
     assert np.array_equal(got, want)
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q3"])
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
 def test_block_codes_roundtrip_through_independent_packer(fmt):
     rng = np.random.default_rng(2)
-    q = rng.integers(0, 16 if fmt == "q4" else 8, size=(50, 32))
+    q = rng.integers(0, {"q4": 16, "q3": 8, "q2": 4}[fmt], size=(50, 32))
     packed = pack(fmt, q)
     for r in range(50):
         assert np.array_equal(oracle.block_codes(fmt, packed[r, 0]), q[r])
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q3"])
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
 def test_qmatvec_matches_dense_definition(fmt):
     rng = np.random.default_rng(3)
     q, s, packed, W = random_matrix(rng, fmt, 40, 96)
@@ -112,6 +112,20 @@ def test_qmatvec_constant_codes_closed_form():
         want = (c - 8) * (s.astype(np.float64) @ xb)
         got = oracle.qmatvec("q4", pack("q4", q), s.view(np.uint16), x)
         assert np.allclose(got, want, rtol=1e-13, atol=1e-15)
+
+
+def test_qmatvec_q2_constant_codes_closed_form():
+    # Q2B32, every code c: W[r, k] = s[r, b] (c - 2); code 2 gives an all-zero matrix
+    rng = np.random.default_rng(5)
+    for c in range(4):
+        q = np.full((5, 96), c)
+        s = rng.uniform(0.01, 0.04, size=(5, 3)).astype(np.float16)
+        x = rng.standard_normal(96)
+        want = (c - 2) * (s.astype(np.float64) @ x.reshape(3, 32).sum(axis=1))
+        got = oracle.qmatvec("q2", pack("q2", q), s.view(np.uint16), x)
+        assert np.allclose(got, want, rtol=1e-13, atol=1e-15)
+        if c == 2:
+            assert np.all(got == 0.0)
 
 
 # --- activation -----------------------------------------------------------------
@@ -186,7 +200,7 @@ def _dense_swiglu(Wg, Wu, Wd, x):
     return Wd @ (g * scipy.special.expit(g) * u)
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q3"])
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
 def test_expert_matches_dense_swiglu(fmt):
     rng = np.random.default_rng(7)
     d, I = 128, 64
@@ -223,7 +237,7 @@ def _tokens(rng, T, d):
     return oracle.round_bf16(rng.standard_normal((T, d)))
 
 
-@pytest.mark.parametrize("fmt,bias", [("q4", False), ("q3", True)])
+@pytest.mark.parametrize("fmt,bias", [("q4", False), ("q3", True), ("q2", True)])
 def test_layer_brute_force(fmt, bias):
     rng = np.random.default_rng(8)
     d, E, I, k, T = 64, 6, 32, 2, 5
