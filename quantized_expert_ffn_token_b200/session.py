@@ -80,6 +80,12 @@ class Session:
             capi.moe_destroy(self.ctx)
             self.ctx = None
 
+    def __enter__(self) -> "Session":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.close()
+
     def __del__(self):
         try:
             self.close()
