@@ -49,3 +49,40 @@ def test_argument_checks_need_no_device():
     assert capi.lib.moe_forward(None, 0, None, 1, None, None, None, None, None) == capi.MOE_ERR_INVALID_ARG
     assert capi.lib.moe_destroy(None) == capi.MOE_OK
     assert capi.status_string(capi.MOE_ERR_NOT_LOADED) == "layer not loaded"
+
+
+def test_plain_c_program_compiles_links_and_calls_the_abi(tmp_path):
+    """The public header is plain C: a C99 program includes it, links against
+    the library and calls the entry points that need no device (argument
+    checks, status strings)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "quantized_expert_ffn_token_b200")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+    moe_ctx *ctx = 0;
+    moe_config c;
+    memset(&c, 0, sizeof c);
+    if (moe_create(0, 0, &ctx) != MOE_ERR_INVALID_ARG) return 1;
+    c.fmt = (moe_qformat)9;
+    if (moe_create(&c, 0, &ctx) != MOE_ERR_INVALID_ARG || ctx != 0) return 2;
+    if (moe_forward(0, 0, 0, 1, 0, 0, 0, 0, 0) != MOE_ERR_INVALID_ARG) return 3;
+    if (moe_destroy(0) != MOE_OK) return 4;
+    printf("%s\n", moe_status_string(MOE_ERR_NOT_LOADED));
+    return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(root, "include"),
+                           "-o", str(exe), str(src), "-L", pkg, "-lqeffn", "-Wl,-rpath," + pkg])
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip() == "layer not loaded"
