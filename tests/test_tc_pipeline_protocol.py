@@ -4,7 +4,10 @@ Agents, as in the kernel:
   * B producers and A loaders each fill the stage ring (S stages) for every
     k block of every item.  Before writing a stage they wait on its "empty"
     barrier, and they publish a stage on its "full" barrier one k block late.
-    They flush the last stage at the end of each item.
+    They flush the last stage at the end of each item.  For an item of a
+    cached expert the B producers instead issue one bulk copy of the stage
+    image, completing on the stage's "cbar" barrier, and arrive on "full" at
+    once; the MMA issuer waits on both.
   * The MMA issuer.  For an item with one or two M=128 accumulators (na) it
     waits until the epilogue has released the TMEM slots it will use: a ring
     of two slots, u counting slot uses, slot u & 1, phase u >> 1.  For each k
@@ -24,9 +27,11 @@ epilogue reads a finished accumulator of the right item; nothing deadlocks.
 import random
 
 
-def run(items, nk, S, rng, mistake=None):
+def run(items, nk, S, rng, mistake=None, cached=None):
+    cached = cached or [False] * len(items)
     full = [0] * S             # completed phases
     empty = [0] * S
+    cbar = [0] * S
     acc_full = [0, 0]
     acc_empty = [0, 0]
     full_arrivals = [0] * S    # arrivals in the current phase (2 producer agents)
@@ -38,10 +43,19 @@ def run(items, nk, S, rng, mistake=None):
     slot_done = [None, None]   # (item, accumulator) whose MMAs have all completed
     slot_reading = [False, False]
     pipe = []                  # tensor pipe queue: ("mma", stage, slots) or ("commit", barrier)
+    copies = []                # bulk copies in flight: (stage, k block)
 
     def producer(part):
         it, pending = 0, None
         for i, na in enumerate(items):
+            if part == "B" and cached[i]:
+                for kb in range(nk):
+                    s = it % S
+                    yield ("wait", ("empty", s), ((it // S) & 1) ^ 1)
+                    yield ("bulk", s, (i, kb))
+                    yield ("publish_now", s)
+                    it += 1
+                continue
             for kb in range(nk):
                 s = it % S
                 yield ("wait", ("empty", s), ((it // S) & 1) ^ (0 if mistake == "producer_parity" else 1))
@@ -55,6 +69,7 @@ def run(items, nk, S, rng, mistake=None):
 
     def mma():
         it, u = 0, 0
+        cpar = [0] * S
         for i, na in enumerate(items):
             for a in range(na):
                 par = (((u + a) >> 1) & 1) ^ (0 if mistake == "acc_empty_parity" else 1)
@@ -64,6 +79,10 @@ def run(items, nk, S, rng, mistake=None):
             for kb in range(nk):
                 s = it % S
                 yield ("wait", ("full", s), (it // S) & 1)
+                if cached[i] and mistake != "skip_cbar":
+                    yield ("wait", ("cbar", s), cpar[s])
+                if cached[i]:
+                    cpar[s] ^= 1
                 yield ("issue", s, (i, kb), slots)
                 yield ("commit", ("empty", s))
                 it += 1
@@ -85,7 +104,7 @@ def run(items, nk, S, rng, mistake=None):
                     yield ("release", sl)
                 u += 1
 
-    bars = {"full": full, "empty": empty, "acc_full": acc_full, "acc_empty": acc_empty}
+    bars = {"full": full, "empty": empty, "acc_full": acc_full, "acc_empty": acc_empty, "cbar": cbar}
     agents = [producer("B"), producer("A"), mma(), epilogue()]
     pending_step = [next(a, None) for a in agents]
     done_reading = set()
@@ -108,8 +127,14 @@ def run(items, nk, S, rng, mistake=None):
             if name == "acc_full":
                 slot_done[idx] = slot_item[idx]
 
-    while any(p is not None for p in pending_step) or pipe:
+    while any(p is not None for p in pending_step) or pipe or copies:
         ready = [j for j, p in enumerate(pending_step) if p is not None and can_run(p)]
+        if copies and (not ready or rng.random() < 0.3):
+            s, blk = copies.pop(rng.randrange(len(copies)))   # a stage image lands
+            writing[s].discard("B")
+            stage[s]["B"] = blk
+            cbar[s] += 1
+            continue
         if pipe and (not ready or rng.random() < 0.35):
             complete(pipe.pop(0))
             continue
@@ -122,6 +147,19 @@ def run(items, nk, S, rng, mistake=None):
             assert reading[s] == 0, f"stage {s} rewritten for {blk} while an MMA reads it"
             writing[s].add(part)
             stage[s][part] = None
+        elif kind == "bulk":
+            _, s, blk = st
+            assert reading[s] == 0, f"stage {s} rewritten for {blk} while an MMA reads it"
+            assert all(cs != s for cs, _ in copies), f"stage {s} copied into twice at once"
+            writing[s].add("B")
+            stage[s]["B"] = None
+            copies.append((s, blk))
+        elif kind == "publish_now":
+            s = st[1]
+            full_arrivals[s] += 1
+            if full_arrivals[s] == 2:
+                full_arrivals[s] = 0
+                full[s] += 1
         elif kind == "publish":
             _, part, (s, blk) = st
             writing[s].discard(part)
@@ -174,6 +212,25 @@ def test_pipeline_never_overwrites_and_never_deadlocks():
     for _ in range(500):
         items, nk, S = random_case(rng)
         run(items, nk, S, rng)
+
+
+def test_pipeline_with_cached_stage_images():
+    rng = random.Random(37)
+    for _ in range(500):
+        items, nk, S = random_case(rng)
+        run(items, nk, S, rng, cached=[rng.random() < 0.5 for _ in items])
+
+
+def test_mma_that_skips_the_image_barrier_would_be_caught():
+    rng = random.Random(41)
+    caught = 0
+    for _ in range(300):
+        items, nk, S = random_case(rng)
+        try:
+            run(items, nk, S, rng, mistake="skip_cbar", cached=[True] * len(items))
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 def _caught(mistake, seed):
