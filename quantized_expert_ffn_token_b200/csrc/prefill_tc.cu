@@ -118,6 +118,18 @@ __device__ __forceinline__ bool mbar_wait_b(uint64_t *b, uint32_t parity, int *e
         }
     }
 }
+// Bounded wait that does not stop early on an error elsewhere: for draining work that is in
+// flight before the CTA exits (a copy or an MMA always completes).
+__device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity, int *err) {
+    long long t0 = clock64();
+    for (int it = 0;; ++it) {
+        if (mbar_try(b, parity)) return;
+        if ((it & 63) == 63 && clock64() - t0 > TC_SPIN) {
+            atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+            return;
+        }
+    }
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // This thread's arrival on *b, adding `bytes` of expected transfer to the phase.
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes) {
@@ -313,6 +325,8 @@ __device__ __forceinline__ int4 item_of(const TcParams &p, int item) {
 struct TcSmem {
     uint64_t full[TC_STAGES];
     uint64_t empty[TC_STAGES];
+    uint64_t cbar[TC_STAGES];   // bytes of a cached stage image landed (one phase per cached fill)
+    uint64_t mma_done;          // every MMA this CTA issued has completed (exit only)
     uint64_t acc_full[2];       // TMEM slot (256 columns) written by the MMAs
     uint64_t acc_empty[2];      // TMEM slot read out by the epilogue
     uint32_t tmem_base;
@@ -342,7 +356,9 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         for (int s = 0; s < TC_STAGES; ++s) {
             mbar_init(&ss->full[s], TC_PROD_NW * 32 + TC_ALD_NT);
             mbar_init(&ss->empty[s], 1);
+            mbar_init(&ss->cbar[s], 1);
         }
+        mbar_init(&ss->mma_done, 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(&ss->acc_full[t], 1);
             mbar_init(&ss->acc_empty[t], 128);
@@ -364,10 +380,13 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         // reads the previous item's slot
         int it = 0;
         uint32_t u = 0;                          // slot uses so far (slot u & 1, phase u >> 1)
+        uint32_t cpar = 0;                       // bit s: parity of the cached fills of stage s so far
+        bool issued = false;                     // this thread issued MMAs
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
             int rows = wi.z;
             const int na = rows > 128 ? 2 : 1;
+            const bool cached = MODE != TC_ROUTER && p.cache_slot && p.cache_slot[wi.x] >= 0;
             for (int a = 0; a < na && ok; ++a)
                 ok = mbar_wait_b(&ss->acc_empty[(u + a) & 1], (((u + a) >> 1) & 1) ^ 1, p.err);
             if (!ok) break;
@@ -376,9 +395,14 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                 int s = it % TC_STAGES;
                 ok = mbar_wait_b(&ss->full[s], (uint32_t)((it / TC_STAGES) & 1), p.err);
+                if (ok && cached) {   // the stage's weights came as one bulk copy of a cached image
+                    ok = mbar_wait_b(&ss->cbar[s], (cpar >> s) & 1u, p.err);
+                    cpar ^= 1u << s;
+                }
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
+                    issued = true;
                     uint32_t a0 = su32(sA + s * A_STAGE_BYTES), b0 = su32(sB + s * B_STAGE_BYTES);
 #pragma unroll
                     for (int j = 0; j < TC_BK / 16; ++j) {
@@ -395,6 +419,13 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             __syncwarp();
             u += na;
         }
+        // no MMA may still read shared memory or write TMEM when the CTA frees them (after a
+        // failed wait nobody else waited for the last commits)
+        if (lane == 0 && issued) {
+            umma_commit(&ss->mma_done);
+            mbar_drain(&ss->mma_done, 0, p.err);
+        }
+        __syncwarp();
     } else if (warp >= TC_PROD_W0 && warp < TC_PROD_W0 + TC_PROD_NW) {
         // ---- producers ---------------------------------------------------------------
         const int pt = tid - TC_PROD_W0 * 32;   // 0..255
@@ -402,6 +433,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
         const int g = lane >> 2;                 // scale rows g, g+8 of this lane's pieces
         int it = 0;
         int pending = -1;                        // stage whose cp.async group is still in flight
+        uint32_t cpar = 0, cfilled = 0;          // thread 0: cached-fill parity / issued, per stage
         uint8_t *myraw = sRaw + pt * 16;         // + (slot * 3 + field) * RAW_FIELD
         for (int item = blockIdx.x; item < n_items && ok; item += G) {
             int4 wi = item_of<MODE>(p, item);
@@ -414,8 +446,8 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             if constexpr (MODE != TC_ROUTER) {
                 const int cslot = p.cache_slot ? p.cache_slot[e] : -1;
                 if (cslot >= 0) {
-                    // the expert's stage images were decoded once already: one bulk copy per stage
-                    // (its bytes complete the stage's barrier together with every producer's arrival)
+                    // the expert's stage images were decoded once already: one bulk copy per stage,
+                    // completing on the stage's cached-image barrier (the MMA warp waits on both)
                     const uint16_t *cs = p.wcache + (size_t)cslot * p.cache_stride + p.cache_off +
                                          (size_t)nt * nk * (B_STAGE_BYTES / 2);
                     for (int kb = 0; kb < nk && ok; ++kb, ++it) {
@@ -424,12 +456,13 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         if (!ok) break;
                         if (pt == 0) {
                             fence_async_smem();
-                            mbar_arrive_tx(&ss->full[s], B_STAGE_BYTES);
+                            mbar_arrive_tx(&ss->cbar[s], B_STAGE_BYTES);
                             bulk_copy_g2s(sB + s * B_STAGE_BYTES, cs + (size_t)kb * (B_STAGE_BYTES / 2),
-                                          B_STAGE_BYTES, &ss->full[s]);
-                        } else {
-                            mbar_arrive(&ss->full[s]);
+                                          B_STAGE_BYTES, &ss->cbar[s]);
+                            cpar ^= 1u << s;
+                            cfilled |= 1u << s;
                         }
+                        mbar_arrive(&ss->full[s]);
                     }
                     continue;
                 }
@@ -487,6 +520,11 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             pending = -1;
         }
         if (pending >= 0) cp_async_wait<0>();
+        // every bulk copy has landed before the CTA's shared memory goes away: the last cached
+        // fill of each stage (earlier ones were waited for by the MMA warp before the reuse)
+        if (pt == 0)
+            for (int s = 0; s < TC_STAGES; ++s)
+                if ((cfilled >> s) & 1u) mbar_drain(&ss->cbar[s], ((cpar >> s) & 1u) ^ 1u, p.err);
     } else if (warp >= TC_ALD_W0 && warp < TC_ALD_W0 + TC_ALD_NW) {
         // ---- A-row loaders -------------------------------------------------------------
         // 16-byte chunk q = at + TC_ALD_NT * j of the stage: row q / 8, chunk q % 8 (the same

@@ -6,9 +6,8 @@ Agents, as in the kernel:
     barrier, and they publish a stage on its "full" barrier one k block late.
     They flush the last stage at the end of each item.  For an item of a
     cached expert the B producers instead issue one bulk copy of the stage
-    image: one thread's arrival on "full" adds the image's bytes to the phase
-    (expect-tx), every B producer arrives at once, and the phase completes only
-    when the arrivals are in and the bytes have landed.
+    image, completing on the stage's "cbar" barrier, and arrive on "full" at
+    once; the MMA issuer waits on both.
   * The MMA issuer.  For an item with one or two M=128 accumulators (na) it
     waits until the epilogue has released the TMEM slots it will use: a ring
     of two slots, u counting slot uses, slot u & 1, phase u >> 1.  For each k
@@ -32,10 +31,10 @@ def run(items, nk, S, rng, mistake=None, cached=None):
     cached = cached or [False] * len(items)
     full = [0] * S             # completed phases
     empty = [0] * S
+    cbar = [0] * S
     acc_full = [0, 0]
     acc_empty = [0, 0]
     full_arrivals = [0] * S    # arrivals in the current phase (2 producer agents)
-    tx_pending = [0] * S       # bulk copies the current phase still waits for
     stage = [dict(B=None, A=None) for _ in range(S)]   # published content per part
     writing = [set() for _ in range(S)]                 # parts being written now
     reading = [0] * S          # MMAs in flight that read the stage
@@ -54,6 +53,7 @@ def run(items, nk, S, rng, mistake=None, cached=None):
                     s = it % S
                     yield ("wait", ("empty", s), ((it // S) & 1) ^ 1)
                     yield ("bulk", s, (i, kb))
+                    yield ("publish_now", s)
                     it += 1
                 continue
             for kb in range(nk):
@@ -69,6 +69,7 @@ def run(items, nk, S, rng, mistake=None, cached=None):
 
     def mma():
         it, u = 0, 0
+        cpar = [0] * S
         for i, na in enumerate(items):
             for a in range(na):
                 par = (((u + a) >> 1) & 1) ^ (0 if mistake == "acc_empty_parity" else 1)
@@ -78,6 +79,10 @@ def run(items, nk, S, rng, mistake=None, cached=None):
             for kb in range(nk):
                 s = it % S
                 yield ("wait", ("full", s), (it // S) & 1)
+                if cached[i] and mistake != "skip_cbar":
+                    yield ("wait", ("cbar", s), cpar[s])
+                if cached[i]:
+                    cpar[s] ^= 1
                 yield ("issue", s, (i, kb), slots)
                 yield ("commit", ("empty", s))
                 it += 1
@@ -99,7 +104,7 @@ def run(items, nk, S, rng, mistake=None, cached=None):
                     yield ("release", sl)
                 u += 1
 
-    bars = {"full": full, "empty": empty, "acc_full": acc_full, "acc_empty": acc_empty}
+    bars = {"full": full, "empty": empty, "acc_full": acc_full, "acc_empty": acc_empty, "cbar": cbar}
     agents = [producer("B"), producer("A"), mma(), epilogue()]
     pending_step = [next(a, None) for a in agents]
     done_reading = set()
@@ -122,23 +127,13 @@ def run(items, nk, S, rng, mistake=None, cached=None):
             if name == "acc_full":
                 slot_done[idx] = slot_item[idx]
 
-    def full_arrive(s):
-        full_arrivals[s] += 1
-        maybe_complete_full(s)
-
-    def maybe_complete_full(s):
-        if full_arrivals[s] == 2 and tx_pending[s] == 0:
-            full_arrivals[s] = 0
-            full[s] += 1
-
     while any(p is not None for p in pending_step) or pipe or copies:
         ready = [j for j, p in enumerate(pending_step) if p is not None and can_run(p)]
         if copies and (not ready or rng.random() < 0.3):
             s, blk = copies.pop(rng.randrange(len(copies)))   # a stage image lands
             writing[s].discard("B")
             stage[s]["B"] = blk
-            tx_pending[s] -= 1
-            maybe_complete_full(s)
+            cbar[s] += 1
             continue
         if pipe and (not ready or rng.random() < 0.35):
             complete(pipe.pop(0))
@@ -155,17 +150,24 @@ def run(items, nk, S, rng, mistake=None, cached=None):
         elif kind == "bulk":
             _, s, blk = st
             assert reading[s] == 0, f"stage {s} rewritten for {blk} while an MMA reads it"
+            assert all(cs != s for cs, _ in copies), f"stage {s} copied into twice at once"
             writing[s].add("B")
             stage[s]["B"] = None
-            if mistake != "no_expect_tx":
-                tx_pending[s] += 1      # the expect-tx arrival: the phase now also waits for the bytes
             copies.append((s, blk))
-            full_arrive(s)              # every B producer's arrival on the stage
+        elif kind == "publish_now":
+            s = st[1]
+            full_arrivals[s] += 1
+            if full_arrivals[s] == 2:
+                full_arrivals[s] = 0
+                full[s] += 1
         elif kind == "publish":
             _, part, (s, blk) = st
             writing[s].discard(part)
             stage[s][part] = blk
-            full_arrive(s)
+            full_arrivals[s] += 1
+            if full_arrivals[s] == 2:
+                full_arrivals[s] = 0
+                full[s] += 1
         elif kind == "claim":
             _, slots, i = st
             for a, sl in enumerate(slots):
@@ -212,6 +214,25 @@ def test_pipeline_never_overwrites_and_never_deadlocks():
         run(items, nk, S, rng)
 
 
+def test_pipeline_with_cached_stage_images():
+    rng = random.Random(37)
+    for _ in range(500):
+        items, nk, S = random_case(rng)
+        run(items, nk, S, rng, cached=[rng.random() < 0.5 for _ in items])
+
+
+def test_mma_that_skips_the_image_barrier_would_be_caught():
+    rng = random.Random(41)
+    caught = 0
+    for _ in range(300):
+        items, nk, S = random_case(rng)
+        try:
+            run(items, nk, S, rng, mistake="skip_cbar", cached=[True] * len(items))
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
 def _caught(mistake, seed):
     rng = random.Random(seed)
     caught = 0
@@ -222,27 +243,6 @@ def _caught(mistake, seed):
         except AssertionError:
             caught += 1
     return caught
-
-
-def test_pipeline_with_cached_stage_images():
-    rng = random.Random(37)
-    for _ in range(500):
-        items, nk, S = random_case(rng)
-        run(items, nk, S, rng, cached=[rng.random() < 0.5 for _ in items])
-
-
-def test_image_copy_without_expect_tx_would_be_caught():
-    """Without the expect-tx arrival the stage's phase can complete before the
-    image has landed, and the MMA reads a half-written stage."""
-    rng = random.Random(41)
-    caught = 0
-    for _ in range(300):
-        items, nk, S = random_case(rng)
-        try:
-            run(items, nk, S, rng, mistake="no_expect_tx", cached=[True] * len(items))
-        except AssertionError:
-            caught += 1
-    assert caught > 0
 
 
 def test_wrong_slot_release_parity_would_be_caught():
