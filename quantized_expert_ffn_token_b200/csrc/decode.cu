@@ -1235,6 +1235,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
 bool decode_supported(const moe_ctx *ctx) {
     const moe_config &c = ctx->cfg;
     if (c.flags & MOE_FLAG_NO_DECODE_KERNEL) return false;
+    if (c.fmt != MOE_Q4B32 && c.fmt != MOE_Q3B32) return false;   // operand decoders exist for these
     // gate/up k chunks go to compute warps 0..d/256-1
     if (c.d_model > 4096 || c.d_model / 256 > NW || c.d_ff / 64 > 12) return false;
     if (c.n_experts % 4) return false;   // logits region of the exchange area stays 16-byte aligned
@@ -1252,6 +1253,10 @@ int decode_setup(moe_ctx *ctx) {
     ds.sms = G;
     if (G > c.d_model / 16) G = c.d_model / 16;   // a down tile then spans at most two CTAs
     ds.grid = G;
+    if (c.fmt != MOE_Q4B32 && c.fmt != MOE_Q3B32) {   // no operand decoder: the kernel is not used
+        ds.smem_bytes = 0;
+        return MOE_OK;
+    }
     int rpc = (c.n_experts + G - 1) / G;
     if (rpc > 8) {
         ds.smem_bytes = 0;

@@ -792,6 +792,7 @@ int launch_tc_router(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, fl
 bool tc_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
     if (c.flags & MOE_FLAG_NO_TENSOR_PREFILL) return false;
+    if (c.fmt != MOE_Q4B32 && c.fmt != MOE_Q3B32) return false;   // stage decoders exist for these
     if (T < 64) return false;
     // n-tiles of 256 output columns: 2I and d must be multiples of 256
     if ((2 * c.d_ff) % TC_BN || c.d_model % TC_BN || c.d_model % TC_BK || c.d_ff % TC_BK) return false;

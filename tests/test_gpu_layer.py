@@ -14,6 +14,9 @@ pytestmark = pytest.mark.gpu
 
 TINY = synth.CONFIGS["tiny_d256_e16_q4_t8"]
 TINY_Q3 = dataclasses.replace(TINY, name="tiny_d256_e16_q3_t8", fmt="q3")
+# the decode shape in the 2-bit format (every token count runs on the CUDA-core path)
+DECODE_Q2 = dataclasses.replace(synth.CONFIGS["decode_48l_q4_t1"], name="decode_48l_q2_t1", fmt="q2",
+                                scale_lo=0.02, scale_hi=0.08)
 
 
 def _cuda():
@@ -45,7 +48,7 @@ def test_generator_bits_identical_on_device():
         assert torch.equal(a, synth.expert_scales(c, 3, t, 7, 8))
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q3"])
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
 def test_tiny_layer_all_tokens(fmt):
     capi, session = _cuda()
     import dataclasses
@@ -238,7 +241,7 @@ def test_memory_limit_gives_oom():
 
 def _full_layer(name, T, rows):
     capi, session = _cuda()
-    cfg = synth.CONFIGS[name]
+    cfg = synth.CONFIGS[name] if isinstance(name, str) else name
     sess = session.Session(cfg, max_tokens=T, n_layers=1)
     sess.load_synthetic(layers=[0])
     x = _tokens(cfg, T)
@@ -257,6 +260,14 @@ def test_decode_layer_full_size():
 
 def test_verify_layer_full_size():
     _full_layer("verify_48l_q3_t4_zipf", 4, range(4))
+
+
+def test_q2_layer_full_size_one_token():
+    _full_layer(DECODE_Q2, 1, [0])
+
+
+def test_q2_layer_full_size_sampled():
+    _full_layer(DECODE_Q2, 96, [0, 1, 31, 63, 64, 95])
 
 
 def test_prefill_layer_full_size_sampled():
