@@ -70,7 +70,7 @@ class MoeError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m quantized_expert_ffn_token_b200.build`")
+                          "`python quantized_expert_ffn_token_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i = ctypes.c_void_p, ctypes.c_int
     L.moe_create.argtypes = [ctypes.POINTER(moe_config), i, ctypes.POINTER(vp)]
