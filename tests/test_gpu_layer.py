@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 TINY = synth.CONFIGS["tiny_d256_e16_q4_t8"]
 TINY_Q3 = dataclasses.replace(TINY, name="tiny_d256_e16_q3_t8", fmt="q3")
-# the decode shape in the 2-bit format (every token count runs on the CUDA-core path)
+# the decode shape in the 2-bit format (CUDA-core path below 64 tokens, tensor cores from 64)
 DECODE_Q2 = dataclasses.replace(synth.CONFIGS["decode_48l_q4_t1"], name="decode_48l_q2_t1", fmt="q2",
                                 scale_lo=0.02, scale_hi=0.08)
 
@@ -266,7 +266,11 @@ def test_q2_layer_full_size_one_token():
     _full_layer(DECODE_Q2, 1, [0])
 
 
-def test_q2_layer_full_size_sampled():
+def test_q2_layer_full_size_cuda_core_path():
+    _full_layer(DECODE_Q2, 40, [0, 1, 17, 39])
+
+
+def test_q2_layer_full_size_tensor_core_path():
     _full_layer(DECODE_Q2, 96, [0, 1, 31, 63, 64, 95])
 
 
@@ -287,13 +291,13 @@ def test_prefill_layer_full_size_sampled():
 
 
 @pytest.mark.parametrize("name,T", [("tiny_d256_e16_q4_t8", 300), ("prefill_1l_q4_t4096_zipf", 512),
-                                    ("verify_48l_q3_t4_zipf", 256)])
+                                    ("verify_48l_q3_t4_zipf", 256), (DECODE_Q2, 256)])
 def test_tensor_core_path_matches_cuda_core_path(name, T):
     """Many-token calls: the tcgen05 grouped GEMM path against the CUDA-core
     path (exact fp32 weights) on the same inputs: same ids and weights, fp32
     outputs within the fp16 weight rounding (relative L2 <= 1e-3)."""
     capi, session = _cuda()
-    cfg = synth.CONFIGS[name]
+    cfg = synth.CONFIGS[name] if isinstance(name, str) else name
     a = session.Session(cfg, max_tokens=T, n_layers=1)
     b = session.Session(cfg, max_tokens=T, n_layers=1, flags=capi.MOE_FLAG_NO_TENSOR_PREFILL)
     W = synth.layer_weights(cfg, 0, device="cuda")
