@@ -14,7 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_fresh_checkout_builds_and_imports(tmp_path):
     if not (shutil.which("nvcc") or os.path.exists("/usr/local/cuda/bin/nvcc")):
         pytest.skip("nvcc not available")
-    if shutil.which("git") is None or not os.path.isdir(os.path.join(ROOT, ".git")):
+    if shutil.which("git") is None or subprocess.run(
+            ["git", "rev-parse", "--is-inside-work-tree"], cwd=ROOT, capture_output=True).returncode != 0:
         pytest.skip("not a git checkout")
     files = subprocess.check_output(["git", "ls-files"], cwd=ROOT, text=True).split("\n")
     for f in files:
