@@ -32,9 +32,7 @@
  *              w = s * (q - 2).                                   2.5 bit/w
  *              For the pages' fastest size Q2_0 ("Strata: Qwen3.8-Flash-Next
  *              (125B Moe) on a 8GB+ Nvidia GPU", tables "How fast?" and "The
- *              size").  Up to 63 tokens run on the CUDA-core path (the
- *              single-token kernel does not take this format yet), 64 and
- *              more on the tensor-core path.
+ *              size").
  *
  * Canonical tensor layouts accepted by moe_load_layer (row-major, SoA: codes
  * and scales in separate arrays):
