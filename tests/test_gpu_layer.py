@@ -15,9 +15,7 @@ pytestmark = pytest.mark.gpu
 TINY = synth.CONFIGS["tiny_d256_e16_q4_t8"]
 TINY_Q3 = dataclasses.replace(TINY, name="tiny_d256_e16_q3_t8", fmt="q3")
 TINY_Q2 = dataclasses.replace(TINY, name="tiny_d256_e16_q2_t8", fmt="q2", scale_lo=0.02, scale_hi=0.08)
-# the decode shape in the 2-bit format
-DECODE_Q2 = dataclasses.replace(synth.CONFIGS["decode_48l_q4_t1"], name="decode_48l_q2_t1", fmt="q2",
-                                scale_lo=0.02, scale_hi=0.08)
+DECODE_Q2 = synth.CONFIGS["decode_48l_q2_t1"]
 
 
 def _cuda():
