@@ -17,7 +17,7 @@
  * 5090 + 64GB", section "The 30-Second Overview" (10 routed + 1 shared per
  * token).  The pages do not define the expert network, the routing
  * normalisation or the quantised layouts; this library fixes them: SwiGLU
- * experts, softmax renormalised over the chosen k, and the two block formats
+ * experts, softmax renormalised over the chosen k, and the block formats
  * below.
  *
  * Block formats (32 weights per block, blocks run along the reduction dim):
@@ -27,12 +27,18 @@
  *   MOE_Q3B32  12 bytes: the 32 three-bit codes of one 96-bit little-endian
  *              integer (code j in bits 3j..3j+2) + one fp16 scale s;
  *              w = s * (q - 4).                                   3.5 bit/w
+ *   MOE_Q2B32  8 bytes: the 32 two-bit codes of one 64-bit little-endian
+ *              integer (code j in bits 2j..2j+1) + one fp16 scale s;
+ *              w = s * (q - 2).                                   2.5 bit/w
+ *              For the pages' fastest size Q2_0 ("Strata: Qwen3.8-Flash-Next
+ *              (125B Moe) on a 8GB+ Nvidia GPU", tables "How fast?" and "The
+ *              size").
  *
  * Canonical tensor layouts accepted by moe_load_layer (row-major, SoA: codes
  * and scales in separate arrays):
  *   gate, up   codes  [E][d_ff][d_model/32][B]   scales [E][d_ff][d_model/32]
  *   down       codes  [E][d_model][d_ff/32][B]   scales [E][d_model][d_ff/32]
- *   B = 16 (Q4B32) or 12 (Q3B32); scales are IEEE fp16 bit patterns.
+ *   B = 16 (Q4B32), 12 (Q3B32) or 8 (Q2B32); scales are IEEE fp16 bit patterns.
  *   router_w   fp32 [E][d_model]; router_bias fp32 [E] or NULL.
  *   Shared experts: the same with n_shared in place of E and d_ff_shared.
  * The library copies them into its own device memory in a private tiled
@@ -66,7 +72,7 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = -7      /* a shape this build does not implement */
 } moe_status;
 
-typedef enum { MOE_Q4B32 = 1, MOE_Q3B32 = 2 } moe_qformat;
+typedef enum { MOE_Q4B32 = 1, MOE_Q3B32 = 2, MOE_Q2B32 = 3 } moe_qformat;
 
 typedef struct {
     int d_model;        /* hidden size d; multiple of 256 */

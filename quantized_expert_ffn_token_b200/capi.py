@@ -25,12 +25,13 @@ MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_ERR_UNSUPPORTED = -7
 MOE_Q4B32 = 1
 MOE_Q3B32 = 2
+MOE_Q2B32 = 3
 MOE_FLAG_NO_DECODE_KERNEL = 1
 MOE_FLAG_NO_TENSOR_PREFILL = 2
 MOE_FLAG_TEST_WITHHOLD = 256
 MOE_FLAG_TRACE = 4
 MOE_ROUTE_STATIC_MAX_LOGITS = 65536
-FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32}
+FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32, "q2": MOE_Q2B32}
 
 EXPORTED = [
     "moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",

@@ -177,6 +177,25 @@ __device__ __forceinline__ void q4_frag_h(uint32_t w, uint32_t &a0, uint32_t &a1
     a3 = (w8 & 0x00F000F0u) | H_MAGIC;
 }
 
+// Q2B32: one lane's 8-byte piece = the 16 fragment registers of four k16 slices, each code
+// OR-ed under fp16 1024 at its place: word w gives registers a0..a3 of slice w as 1024 + q
+// (rows g) and 1024 + 4q (rows g+8), and those of slice w + 2 as 1024 + 16q and 1024 + 64q.
+__device__ __forceinline__ void q2_frag_h(uint2 piece, uint32_t r[16]) {
+    const uint32_t wv[2] = {piece.x, piece.y};
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const uint32_t x = wv[w], x8 = __umulhi(wv[w], 1u << 24);   // x >> 8 on the multiply pipe
+        r[4 * w + 0] = (x & 0x00030003u) | H_MAGIC;
+        r[4 * w + 1] = (x & 0x000C000Cu) | H_MAGIC;
+        r[4 * w + 2] = (x8 & 0x00030003u) | H_MAGIC;
+        r[4 * w + 3] = (x8 & 0x000C000Cu) | H_MAGIC;
+        r[4 * w + 8] = (x & 0x00300030u) | H_MAGIC;
+        r[4 * w + 9] = (x & 0x00C000C0u) | H_MAGIC;
+        r[4 * w + 10] = (x8 & 0x00300030u) | H_MAGIC;
+        r[4 * w + 11] = (x8 & 0x00C000C0u) | H_MAGIC;
+    }
+}
+
 // Q3B32: three words = the 16 fragment registers of four k16 slices.
 __device__ __forceinline__ void q3_frag(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t r[16]) {
     uint32_t ws[3] = {w0, w1, w2};
@@ -225,11 +244,11 @@ __device__ __forceinline__ int hfrag_index(int sl, int c, int r, int which) {
     const int b4 = (sl >> 1) & 3, j = sl >> 3, sp = sl & 1;
     return ((j * 32 + (b4 * 4 + c) * 2 + r) * 2 + sp) * 4 + which * 2;
 }
-// x * mask for a packed pair of fp16 (Q4) or bf16 (Q3) values, mask 1.0 or 0 in both
+// x * mask for a packed pair of fp16 (Q4, Q2) or bf16 (Q3) values, mask 1.0 or 0 in both
 // halves: zeroes the inactive block columns on the multiply pipe.
 __device__ __forceinline__ uint32_t hmul2_mask(int fmt, uint32_t x, uint32_t mask) {
     uint32_t r;
-    if (fmt == MOE_Q4B32)
+    if (fmt != MOE_Q3B32)
         asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(mask));
     else
         asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(mask));
@@ -433,7 +452,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
     const int DW = I / 64;               // warps with a down k group (64 k each)
     const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
     const int JN = (I + 127) / 128;      // k-group pairs of the down K (h table blocks)
-    const uint32_t ONE2 = (FMT == MOE_Q4B32) ? 0x3C003C00u : 0x3F803F80u;   // 1.0 in both halves
+    constexpr bool F16OP = (FMT != MOE_Q3B32);   // fp16 operands (Q4B32, Q2B32), else bf16 (Q3B32)
+    const uint32_t ONE2 = F16OP ? 0x3C003C00u : 0x3F803F80u;   // 1.0 in both halves
     constexpr float off = (FMT == MOE_Q4B32) ? 136.f : 132.f;   // 128 + zero point
     int *err = p.err;
 
@@ -658,7 +678,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         frexpf(amx, &xe);                    // amx < 2^xe
         const int xs_exp = min(15 - xe, 100);
         const float xscale = pow2i(xs_exp);
-        if (tid == 0) ms->xinv = (FMT == MOE_Q4B32) ? pow2i(-xs_exp) : 1.f;
+        if (tid == 0) ms->xinv = F16OP ? pow2i(-xs_exp) : 1.f;
         // 8 consecutive elements per thread: bf16 (stack: rounded from r * inv), fp16 of x * 2^s
         for (int i8 = tid; i8 < d / 8; i8 += NT) {
             uint32_t xw[4], hw[4];
@@ -681,7 +701,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(xb + 8 * i8);
                 xw[0] = v.x; xw[1] = v.y; xw[2] = v.z; xw[3] = v.w;
             }
-            if constexpr (FMT == MOE_Q4B32) {
+            if constexpr (F16OP) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     __half2 h2 = __floats2half2_rn(__uint_as_float(xw[j] << 16) * xscale,
@@ -694,7 +714,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         csync();
         // block sums of the operand the gate/up MMAs see (offset removal in their flush)
         for (int b = tid; b < nbd; b += NT)
-            xsum[b] = (FMT == MOE_Q4B32) ? sum32_f16(xh + 32 * b) : sum32_bf16(xb + 32 * b);
+            xsum[b] = F16OP ? sum32_f16(xh + 32 * b) : sum32_bf16(xb + 32 * b);
 
         trace_mark(p, l, 0, clock64() - tl0);
         // ---- 2. router ----------------------------------------------------------
@@ -875,7 +895,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
         // (Q4: fp16 x * 2^s, Q3: bf16 x)
         uint32_t bx0[16], bx1[16];
         if (warp < GW) {
-            const uint16_t *xop = (FMT == MOE_Q4B32) ? xh : xb;
+            const uint16_t *xop = F16OP ? xh : xb;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 int s = 16 * warp + j;
@@ -901,7 +921,17 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
                 float D0[4] = {0.f, 0.f, 0.f, 0.f}, D1[4] = {0.f, 0.f, 0.f, 0.f};
-                if constexpr (FMT == MOE_Q4B32) {
+                if constexpr (FMT == MOE_Q2B32) {
+#pragma unroll
+                    for (int kq = 0; kq < 4; ++kq) {
+                        uint32_t rg[16];
+                        q2_frag_h(*reinterpret_cast<const uint2 *>(tile + (size_t)(4 * warp + kq) * 256 + lane * 8), rg);
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            mma16816_h((m & 1) ? D1 : D0, rg[4 * m], rg[4 * m + 1], rg[4 * m + 2], rg[4 * m + 3],
+                                       bx0[4 * kq + m], bx1[4 * kq + m]);
+                    }
+                } else if constexpr (FMT == MOE_Q4B32) {
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq) {
                         uint4 a = *reinterpret_cast<const uint4 *>(tile + (size_t)(4 * warp + kq) * 512 + lane * 16);
@@ -931,7 +961,14 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + b0));
                 float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + b0));
                 float ag, a8;
-                if constexpr (FMT == MOE_Q4B32) {
+                if constexpr (FMT == MOE_Q2B32) {
+                    // column 2c = the k group's first block: rows g read 1024 + q, rows g+8 1024 + 4q;
+                    // column 2c+1 = its second block: 1024 + 16q and 1024 + 64q
+                    const float x0 = xsum[b0], x1 = xsum[b0 + 1];
+                    ag = fmaf(sg.x, D0[0] + D1[0] - 1026.f * x0, sg.y * fmaf(D0[1] + D1[1], 0.0625f, -66.f * x1));
+                    a8 = fmaf(s8.x, fmaf(D0[2] + D1[2], 0.25f, -258.f * x0),
+                              s8.y * fmaf(D0[3] + D1[3], 0.015625f, -18.f * x1));
+                } else if constexpr (FMT == MOE_Q4B32) {
                     // row g: codes read as 1024 + q; row g+8: as 1024 + 16 q (sums scaled by 1/16)
                     const float x0 = xsum[b0], x1 = xsum[b0 + 1];
                     ag = fmaf(sg.x, D0[0] + D1[0] - 1032.f * x0, sg.y * (D0[1] + D1[1] - 1032.f * x1));
@@ -1006,7 +1043,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                     const bool valid = i4 < n4;
                     const float hv[4] = {hb[t].x, hb[t].y, hb[t].z, hb[t].w};
                     float scale = 1.f;
-                    if constexpr (FMT == MOE_Q4B32) {
+                    if constexpr (F16OP) {
                         float mx = fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3])));
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -1022,7 +1059,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                         uint32_t hi2[2], lo2[2];
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            if constexpr (FMT == MOE_Q4B32) {
+                            if constexpr (F16OP) {
                                 const float v0 = hv[2 * j] * scale, v1 = hv[2 * j + 1] * scale;
                                 const __half2 hh = __floats2half2_rn(v0, v1);
                                 const float2 hf = __half22float2(hh);
@@ -1102,7 +1139,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                     const int kg = 2 * j + h;
                     if (kg < DW) {
                         uint32_t a[16];
-                        if constexpr (FMT == MOE_Q4B32) {
+                        if constexpr (FMT == MOE_Q2B32) {
+                            q2_frag_h(*reinterpret_cast<const uint2 *>(tile + (size_t)kg * 256 + lane * 8), a);
+                        } else if constexpr (FMT == MOE_Q4B32) {
                             uint4 av = *reinterpret_cast<const uint4 *>(tile + (size_t)kg * 512 + lane * 16);
                             q4_frag_h(av.x, a[0], a[1], a[2], a[3]);
                             q4_frag_h(av.y, a[4], a[5], a[6], a[7]);
@@ -1119,7 +1158,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                             const uint32_t mk = hmask[h][m >> 1];
                             const uint32_t b0 = hmul2_mask(FMT, (m & 1) ? bj.z : bj.x, mk);
                             const uint32_t b1 = hmul2_mask(FMT, (m & 1) ? bj.w : bj.y, mk);
-                            if constexpr (FMT == MOE_Q4B32)
+                            if constexpr (F16OP)
                                 mma16816_h(h ? Db : Da, a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
                             else
                                 mma16816(h ? Db : Da, a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3], b0, b1);
@@ -1130,7 +1169,16 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 if (blk < nbi) {
                     const float hs = hsum[us * nbi + blk];
                     const float sg = __half2float(sc[g * nbi + blk]), s8 = __half2float(sc[(g + 8) * nbi + blk]);
-                    if constexpr (FMT == MOE_Q4B32) {
+                    if constexpr (FMT == MOE_Q2B32) {
+                        // block 4j + c is the first block of its k group for even c (rows g: 1024 + q,
+                        // rows g+8: 1024 + 4q), the second for odd c (1024 + 16q, 1024 + 64q)
+                        const float hi = hinv[us * nbi + blk];
+                        const bool second = c & 1;
+                        const float mg = second ? 0.0625f : 1.f, og = second ? 66.f : 1026.f;
+                        const float m8 = second ? 0.015625f : 0.25f, o8 = second ? 18.f : 258.f;
+                        ag = fmaf(sg * hi, fmaf((Da[0] + Da[1]) + (Db[0] + Db[1]), mg, -og * hs), ag);
+                        a8 = fmaf(s8 * hi, fmaf((Da[2] + Da[3]) + (Db[2] + Db[3]), m8, -o8 * hs), a8);
+                    } else if constexpr (FMT == MOE_Q4B32) {
                         // row g: 1024 + q; row g+8: 1024 + 16 q (sums / 16); h entered as h * 2^s
                         const float hi = hinv[us * nbi + blk];
                         ag = fmaf(sg * hi, (Da[0] + Da[1]) + (Db[0] + Db[1]) - 1032.f * hs, ag);
@@ -1300,7 +1348,9 @@ int decode_setup(moe_ctx *ctx) {
     ds.slot_bytes = slot;
     ds.rpc = rpc;
     ds.smem_bytes = (int)(fixed + (size_t)nslot * slot);
-    const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
+    const void *kfn = (c.fmt == MOE_Q4B32)   ? (const void *)k_decode<MOE_Q4B32>
+                          : (c.fmt == MOE_Q2B32) ? (const void *)k_decode<MOE_Q2B32>
+                                                 : (const void *)k_decode<MOE_Q3B32>;
     QE_CHECK(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, ds.smem_bytes));
     int per_sm = 0;
     QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NTT, ds.smem_bytes));
@@ -1383,7 +1433,9 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     p.off_sums = ds.off_sums;
     p.off_ltab = ds.off_ltab;
     void *args[] = {&p};
-    const void *kfn = (c.fmt == MOE_Q4B32) ? (const void *)k_decode<MOE_Q4B32> : (const void *)k_decode<MOE_Q3B32>;
+    const void *kfn = (c.fmt == MOE_Q4B32)   ? (const void *)k_decode<MOE_Q4B32>
+                          : (c.fmt == MOE_Q2B32) ? (const void *)k_decode<MOE_Q2B32>
+                                                 : (const void *)k_decode<MOE_Q3B32>;
     QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ds.grid), dim3(NTT), args,
                                          (size_t)ds.smem_bytes, st));
     QE_CHECK_LAUNCH("k_decode");

@@ -151,7 +151,7 @@ int launch_experts_simt(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
     a.E = c.n_experts;
     a.d = c.d_model;
     a.I = c.d_ff;
-    a.zero = c.fmt == MOE_Q4B32 ? 8 : 4;
+    a.zero = c.fmt == MOE_Q4B32 ? 8 : (c.fmt == MOE_Q2B32) ? 2 : 4;
     a.gu = ctx->gu;
     a.dn = ctx->dn;
     a.gu_w = Ly.gu;

@@ -85,7 +85,7 @@ using namespace qeffn;
 namespace {
 
 int validate_config(const moe_config *c) {
-    if (c->fmt != MOE_Q4B32 && c->fmt != MOE_Q3B32) return MOE_ERR_INVALID_ARG;
+    if (c->fmt != MOE_Q4B32 && c->fmt != MOE_Q3B32 && c->fmt != MOE_Q2B32) return MOE_ERR_INVALID_ARG;
     if (c->d_model <= 0 || c->n_experts <= 0 || c->d_ff <= 0 || c->top_k <= 0 ||
         c->n_shared < 0 || c->n_layers <= 0 || c->max_tokens <= 0 || c->device_mem_limit < 0)
         return MOE_ERR_INVALID_ARG;
@@ -189,7 +189,7 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
     const moe_config &c = ctx->cfg;
     Layer &Ly = ctx->layers[layer];
     size_t E = c.n_experts, d = c.d_model, I = c.d_ff, nsh = c.n_shared;
-    size_t B = c.fmt == MOE_Q4B32 ? 16 : 12;
+    size_t B = c.fmt == MOE_Q4B32 ? 16 : (c.fmt == MOE_Q2B32) ? 8 : 12;
     if (!Ly.router_w) {
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.router_w, E * d * 4, "router_w"));
         QE_TRY(ctx_alloc(ctx, (void **)&Ly.router_b, E * 4, "router_b"));

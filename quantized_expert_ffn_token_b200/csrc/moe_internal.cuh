@@ -32,13 +32,20 @@ namespace qeffn {
 //   3f (even k) and 16+3f (odd k), f = q%5; register 15's codes are spread
 //   over bit 15 (even k) and bit 31 (odd k) of words 0,1,2 (code bit b in
 //   word b).
+// Q2B32: 8 bytes per lane and group = 2 words.  Bits 16*hi + 2f (f = 0..7) of
+//   word w hold the code of slice m = w + 2*((f >> 1) & 1), register
+//   reg = (f & 1) + 2*(f >> 2): a word's fields 0,1,4,5 are the four
+//   registers of slice w (first 32-block of the group) and fields 2,3,6,7
+//   those of slice w + 2 (second block), so that an fp16 decode can OR each
+//   field into the mantissa of 1024 at its place (x1, x4, x16, x64) with the
+//   same multiplier for every row of a block.
 // After the codes: the tile's fp16 scales, [16 rows][K/32 blocks].
 // The byte count equals the canonical layout's.
 // ---------------------------------------------------------------------------
 struct MatLayout {
     int K;           // reduction length (multiple of 64)
     int n_tiles;     // 16-row tiles per expert
-    int kg_bytes;    // bytes per k group (all lanes): 512 (Q4) / 384 (Q3)
+    int kg_bytes;    // bytes per k group (all lanes): 512 (Q4) / 384 (Q3) / 256 (Q2)
     int code_bytes;  // (K/64) * kg_bytes
     int tile_bytes;  // code_bytes + 16 * (K/32) * 2
     size_t expert_bytes;
@@ -48,7 +55,7 @@ inline MatLayout make_layout(int fmt, int rows, int K) {
     MatLayout L;
     L.K = K;
     L.n_tiles = rows / 16;
-    L.kg_bytes = (fmt == MOE_Q4B32) ? 512 : 384;
+    L.kg_bytes = (fmt == MOE_Q4B32) ? 512 : (fmt == MOE_Q2B32) ? 256 : 384;
     L.code_bytes = (K / 64) * L.kg_bytes;
     L.tile_bytes = L.code_bytes + 16 * (K / 32) * 2;
     L.expert_bytes = (size_t)L.n_tiles * L.tile_bytes;
@@ -91,11 +98,30 @@ __host__ __device__ inline void q3_code_pos(int r, int k, int byte[3], int bit[3
     }
 }
 
+// Q2B32: byte offset and bit offset of the 2-bit code of tile row r, column k.
+__host__ __device__ inline void q2_code_pos(int r, int k, int *byte, int *shift) {
+    int g = r & 7, half = r >> 3;
+    int s = k >> 4, kk = k & 15;
+    int kg = s >> 2, m = s & 3;
+    int c = (kk & 7) >> 1, hi = kk & 1, second = kk >> 3;
+    int reg = second * 2 + half;
+    int w = m & 1;
+    int f = (reg & 1) + 2 * (m >> 1) + 4 * (reg >> 1);
+    int bit = 16 * hi + 2 * f;
+    *byte = kg * 256 + (g * 4 + c) * 8 + w * 4 + (bit >> 3);
+    *shift = bit & 7;
+}
+
 __device__ inline int tile_code(int fmt, const uint8_t *tile, int r, int k) {
     if (fmt == MOE_Q4B32) {
         int byte, sh;
         q4_code_pos(r, k, &byte, &sh);
         return (tile[byte] >> sh) & 15;
+    }
+    if (fmt == MOE_Q2B32) {
+        int byte, sh;
+        q2_code_pos(r, k, &byte, &sh);
+        return (tile[byte] >> sh) & 3;
     }
     int byte[3], bit[3];
     q3_code_pos(r, k, byte, bit);

@@ -148,6 +148,9 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(su32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(su32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -234,12 +237,33 @@ constexpr uint32_t H_MAGIC = 0x64006400u, H_ONE = 0x3C003C00u, H_16TH = 0x2C002C
 constexpr uint32_t H_8TH = 0x30003000u, H_64TH = 0x24002400u;
 constexpr uint32_t H_M1032 = 0xE408E408u, H_M72 = 0xD480D480u;              // Q4: -(1024+8), -(64+8)
 constexpr uint32_t H_M1028 = 0xE404E404u, H_M132 = 0xD820D820u, H_M20 = 0xCD00CD00u;  // Q3
+constexpr uint32_t H_4TH = 0x34003400u;
+constexpr uint32_t H_M1026 = 0xE402E402u, H_M258 = 0xDC08DC08u, H_M66 = 0xD420D420u,   // Q2: -(1024+2),
+                   H_M18 = 0xCC80CC80u;                                                 // -(256+2), -(64+2), -(16+2)
 
 // The 16 (q - zero) fp16 pairs of one lane's piece of a k group, register
 // q = 4*slice + reg (reg a0..a3 as in the row-tile layout).
 template <int FMT>
 __device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16]) {
-    if constexpr (FMT == MOE_Q4B32) {
+    if constexpr (FMT == MOE_Q2B32) {
+        // word w: the 2-bit fields at bits 0, 2, 4, 6 of each half (of w, then of w >> 8) read
+        // 1024 + {1, 4, 16, 64} q; fields 0,1,4,5 are registers a0..a3 of slice w, fields
+        // 2,3,6,7 those of slice w + 2
+        uint2 a = *reinterpret_cast<const uint2 *>(src);
+        uint32_t wv[2] = {a.x, a.y};
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t x = wv[w], x8 = wv[w] >> 8;
+            r[4 * w + 0] = hfma2((x & 0x00030003u) | H_MAGIC, H_ONE, H_M1026);
+            r[4 * w + 1] = hfma2((x & 0x000C000Cu) | H_MAGIC, H_4TH, H_M258);
+            r[4 * w + 2] = hfma2((x8 & 0x00030003u) | H_MAGIC, H_ONE, H_M1026);
+            r[4 * w + 3] = hfma2((x8 & 0x000C000Cu) | H_MAGIC, H_4TH, H_M258);
+            r[4 * w + 8] = hfma2((x & 0x00300030u) | H_MAGIC, H_16TH, H_M66);
+            r[4 * w + 9] = hfma2((x & 0x00C000C0u) | H_MAGIC, H_64TH, H_M18);
+            r[4 * w + 10] = hfma2((x8 & 0x00300030u) | H_MAGIC, H_16TH, H_M66);
+            r[4 * w + 11] = hfma2((x8 & 0x00C000C0u) | H_MAGIC, H_64TH, H_M18);
+        }
+    } else if constexpr (FMT == MOE_Q4B32) {
         uint4 a = *reinterpret_cast<const uint4 *>(src);
         uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
@@ -490,6 +514,8 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         const uint8_t *cs = tile + (size_t)kb * p.L.kg_bytes;
                         if constexpr (FMT == MOE_Q4B32) {
                             cp_async16(raw + tt * RAW_FIELD, cs + lane * 16);
+                        } else if constexpr (FMT == MOE_Q2B32) {
+                            cp_async8(raw + tt * RAW_FIELD, cs + lane * 8);
                         } else {
                             cp_async4(raw + tt * RAW_FIELD, cs + lane * 12);
                             cp_async4(raw + tt * RAW_FIELD + 4, cs + lane * 12 + 4);
@@ -715,6 +741,8 @@ __global__ void __launch_bounds__(256) k_cache_fill(const uint8_t *__restrict__ 
             const uint8_t *cs = tile + (size_t)kb * L.kg_bytes;
             if constexpr (FMT == MOE_Q4B32) {
                 cp_async16(myraw + tt * RAW_FIELD, cs + lane * 16);
+            } else if constexpr (FMT == MOE_Q2B32) {
+                cp_async8(myraw + tt * RAW_FIELD, cs + lane * 8);
             } else {
                 cp_async4(myraw + tt * RAW_FIELD, cs + lane * 12);
                 cp_async4(myraw + tt * RAW_FIELD + 4, cs + lane * 12 + 4);
@@ -858,7 +886,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     TcParams p;
     memset(&p, 0, sizeof(p));
     p.fmt = c.fmt;
-    p.zero = c.fmt == MOE_Q4B32 ? 8 : 4;
+    p.zero = c.fmt == MOE_Q4B32 ? 8 : (c.fmt == MOE_Q2B32) ? 2 : 4;
     p.perm = ws.perm;
     p.offsets = ws.offsets;
     p.items = ws.tc_items;
@@ -882,6 +910,11 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
         if (c.fmt == MOE_Q4B32) {
             QE_CHECK(cudaFuncSetAttribute(k_cache_fill<MOE_Q4B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm));
             k_cache_fill<MOE_Q4B32><<<4 * dev_sms, 256, fsm, st>>>(Ly.gu, ctx->gu, Ly.dn, ctx->dn, ws.cache_expert,
+                                                                   ws.cache_n, ws.cache_cap, ws.wcache, c.d_model,
+                                                                   c.d_ff);
+        } else if (c.fmt == MOE_Q2B32) {
+            QE_CHECK(cudaFuncSetAttribute(k_cache_fill<MOE_Q2B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm));
+            k_cache_fill<MOE_Q2B32><<<4 * dev_sms, 256, fsm, st>>>(Ly.gu, ctx->gu, Ly.dn, ctx->dn, ws.cache_expert,
                                                                    ws.cache_n, ws.cache_cap, ws.wcache, c.d_model,
                                                                    c.d_ff);
         } else {
@@ -910,6 +943,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.h16 = ws.h16;
     int grid = dev_sms;
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_GATEUP>(p, grid, st)));
+    else if (c.fmt == MOE_Q2B32) QE_TRY((launch_tc<MOE_Q2B32, TC_GATEUP>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_GATEUP>(p, grid, st)));
 
     // down: A = h16 rows by grouped position, N = d, K = I
@@ -927,6 +961,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.w_route = w_route;
     p.cache_off = (size_t)2 * c.d_ff * c.d_model;   // the down GEMM's stages follow the gate/up ones
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_DOWN>(p, grid, st)));
+    else if (c.fmt == MOE_Q2B32) QE_TRY((launch_tc<MOE_Q2B32, TC_DOWN>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_DOWN>(p, grid, st)));
     QE_TRY(timing_end(ctx, st));
     k_finish<<<592, 256, 0, st>>>(ws.y_acc, Td, y, yf);

@@ -7,9 +7,11 @@ namespace qeffn {
 namespace {
 
 // Canonical code j of block `blk` (Q4B32: nibble j%2 of byte j/2, low first;
-// Q3B32: bits 3j..3j+2 of the 96-bit little-endian block).
+// Q3B32: bits 3j..3j+2 of the 96-bit little-endian block; Q2B32: bits 2j..2j+1
+// of the 64-bit little-endian block).
 __device__ inline int canon_code(int fmt, const uint8_t *blk, int j) {
     if (fmt == MOE_Q4B32) return (blk[j >> 1] >> ((j & 1) * 4)) & 15;
+    if (fmt == MOE_Q2B32) return (blk[j >> 2] >> (2 * (j & 3))) & 3;
     int v = 0;
     for (int t = 0; t < 3; ++t) {
         int bit = 3 * j + t;
@@ -39,7 +41,7 @@ __device__ inline int src_row(const RepackArgs &a, int t, int r, int *up) {
 __device__ inline int fetch_code(const RepackArgs &a, int e, int t, int r, int k) {
     int up;
     int row = src_row(a, t, r, &up);
-    int B = a.fmt == MOE_Q4B32 ? 16 : 12;
+    int B = a.fmt == MOE_Q4B32 ? 16 : (a.fmt == MOE_Q2B32) ? 8 : 12;
     size_t nb = a.K / 32;
     const uint8_t *base = up ? a.codes_up : a.codes;
     const uint8_t *blk = base + (((size_t)e * a.rows + row) * nb + (k >> 5)) * B;
@@ -74,6 +76,19 @@ __global__ void k_repack_codes(RepackArgs a) {
             }
             uint4 v = make_uint4(words[0], words[1], words[2], words[3]);
             *reinterpret_cast<uint4 *>(tile + kg * 512 + lane * 16) = v;
+        } else if (a.fmt == MOE_Q2B32) {
+            // word w, field f, half hi: slice w + 2*((f >> 1) & 1), register (f & 1) + 2*(f >> 2)
+            uint32_t words[2] = {0, 0};
+            for (int w = 0; w < 2; ++w)
+                for (int f = 0; f < 8; ++f) {
+                    int m = w + 2 * ((f >> 1) & 1), reg = (f & 1) + 2 * (f >> 2);
+                    int r = g + 8 * (reg & 1);
+                    for (int hi = 0; hi < 2; ++hi) {
+                        int k = 64 * kg + 16 * m + 8 * (reg >> 1) + 2 * c + hi;
+                        words[w] |= (uint32_t)fetch_code(a, e, t, r, k) << (16 * hi + 2 * f);
+                    }
+                }
+            *reinterpret_cast<uint2 *>(tile + kg * 256 + lane * 8) = make_uint2(words[0], words[1]);
         } else {
             uint32_t w3[3] = {0, 0, 0};
             for (int q = 0; q < 16; ++q) {

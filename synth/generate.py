@@ -81,6 +81,8 @@ CONFIGS = {
         LayerConfig("verify_48l_q3_t4_zipf", 2560, 512, 512, 10, 1, 512, 48, 4, "q3", 0.01, 0.04, 1.1),
         LayerConfig("prefill_1l_q4_t4096_zipf", 2560, 512, 512, 10, 1, 512, 1, 4096, "q4", 0.005, 0.02, 1.1),
         LayerConfig("prefill_48l_q3_t32768", 2560, 512, 512, 10, 1, 512, 48, 32768, "q3", 0.01, 0.04, None),
+        # the decode shape in the 2-bit format (the pages' fastest size, Q2_0)
+        LayerConfig("decode_48l_q2_t1", 2560, 512, 512, 10, 1, 512, 48, 1, "q2", 0.02, 0.08, None),
     ]
 }
 

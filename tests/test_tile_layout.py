@@ -41,8 +41,17 @@ int main() {
             q3_code_pos(r, k, byte, bit);
             printf("q3 %%d %%d %%d %%d %%d\n", r, k, byte[0] * 8 + bit[0], byte[1] * 8 + bit[1], byte[2] * 8 + bit[2]);
         }
+    // Q2B32: one 2-bit field per position
+    for (int r = 0; r < 16; ++r)
+        for (int k = 0; k < K; ++k) {
+            int byte, sh;
+            q2_code_pos(r, k, &byte, &sh);
+            printf("q2 %%d %%d %%d\n", r, k, byte * 8 + sh);
+        }
     MatLayout l4 = make_layout(MOE_Q4B32, 16, K), l3 = make_layout(MOE_Q3B32, 16, K);
-    printf("bytes %%d %%d %%d %%d\n", l4.code_bytes, l4.kg_bytes, l3.code_bytes, l3.kg_bytes);
+    MatLayout l2 = make_layout(MOE_Q2B32, 16, K);
+    printf("bytes %%d %%d %%d %%d %%d %%d\n", l4.code_bytes, l4.kg_bytes, l3.code_bytes, l3.kg_bytes,
+           l2.code_bytes, l2.kg_bytes);
     return 0;
 }
 """ % K
@@ -58,7 +67,7 @@ def positions(tmp_path_factory):
     src.write_text(PROGRAM)
     subprocess.check_call([nvcc, "-std=c++17", "-I", INCLUDE, "-I", CSRC, "-o", str(exe), str(src)])
     out = subprocess.check_output([str(exe)], text=True).split("\n")
-    rows = {"q4": {}, "q3": {}}
+    rows = {"q4": {}, "q3": {}, "q2": {}}
     sizes = None
     for line in out:
         p = line.split()
@@ -75,13 +84,16 @@ def _bits(fmt, pos):
     """All code bits (absolute bit index in the code area) of one position."""
     if fmt == "q4":
         return [pos[0] + b for b in range(4)]
+    if fmt == "q2":
+        return [pos[0], pos[0] + 1]
     return pos
 
 
-@pytest.mark.parametrize("fmt, width, kg_bytes", [("q4", 4, 512), ("q3", 3, 384)])
+@pytest.mark.parametrize("fmt, width, kg_bytes", [("q4", 4, 512), ("q3", 3, 384), ("q2", 2, 256)])
 def test_codes_fill_the_code_area_exactly_once(positions, fmt, width, kg_bytes):
     rows, sizes = positions
-    code_bytes = {"q4": sizes[0], "q3": sizes[2]}[fmt]
+    code_bytes = {"q4": sizes[0], "q3": sizes[2], "q2": sizes[4]}[fmt]
+    assert {"q4": sizes[1], "q3": sizes[3], "q2": sizes[5]}[fmt] == kg_bytes
     assert code_bytes == (K // 64) * kg_bytes == 16 * K * width // 8
     seen = set()
     for (r, k), pos in rows[fmt].items():
@@ -92,7 +104,7 @@ def test_codes_fill_the_code_area_exactly_once(positions, fmt, width, kg_bytes):
     assert len(seen) == 8 * code_bytes
 
 
-@pytest.mark.parametrize("fmt, piece", [("q4", 16), ("q3", 12)])
+@pytest.mark.parametrize("fmt, piece", [("q4", 16), ("q3", 12), ("q2", 8)])
 def test_each_lane_piece_holds_its_fragment_codes(positions, fmt, piece):
     rows, _ = positions
     kg_bytes = 32 * piece
@@ -102,3 +114,18 @@ def test_each_lane_piece_holds_its_fragment_codes(positions, fmt, piece):
         start = 8 * ((k // 64) * kg_bytes + lane * piece)
         for b in _bits(fmt, pos):
             assert start <= b < start + 8 * piece, f"{fmt}: row {r}, k {k} outside lane {lane}'s piece"
+
+
+def test_q2_fields_of_a_block_share_one_multiplier(positions):
+    """Q2B32: within a lane's word, the fields of the first 32-block of a k group
+    sit at bit offsets 0, 2, 8, 10 of a half (multipliers 1 and 4 once OR-ed into
+    an fp16 mantissa, taking the word and the word shifted right by 8) and those
+    of the second block at 4, 6, 12, 14 (multipliers 16 and 64); rows g use the
+    lower multiplier of each pair and rows g + 8 the higher one."""
+    rows, _ = positions
+    for (r, k), pos in rows["q2"].items():
+        off = pos[0] % 16                       # bit offset inside the 16-bit half
+        first_block = (k % 64) < 32
+        assert off in ((0, 2, 8, 10) if first_block else (4, 6, 12, 14))
+        low_multiplier = (off % 8) in (0, 4)    # fields 0, 4 of a byte-half: x1 or x16
+        assert low_multiplier == (r < 8)
