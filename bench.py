@@ -371,9 +371,9 @@ def secondary_prefill(args, local_rank) -> dict:
 # The library's path selection by T (include/moe.h, moe_forward): the single-token kernel once per
 # token up to DISPATCH_DECODE_MAX tokens, the tensor-core path from DISPATCH_TC_MIN tokens, the
 # CUDA-core path in between.  The flags below pin a context to one path.
-DISPATCH_DECODE_MAX = 16
-DISPATCH_TC_MIN = 64
-SWEEP_T = (1, 2, 4, 8, 16, 17, 32, 48, 63, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
+DISPATCH_DECODE_MAX = 8
+DISPATCH_TC_MIN = 9
+SWEEP_T = (1, 2, 4, 6, 8, 9, 10, 12, 16, 24, 32, 48, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
 SWEEP_PATHS = ("single-token kernel", "cuda-core", "tensor-core")
 
 

@@ -153,10 +153,11 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  *   weight) and w [T][k] their weights, either may be NULL.
  * Asynchronous on `stream`; no host synchronisation and no allocation.
  * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA.
- * Implementation (not part of the contract): up to 16 tokens run the
- * persistent single-token kernel once per token, fewer than 64 the CUDA-core
- * grouped path, 64 and more the tensor-core grouped GEMMs; each path meets the
- * same accuracy bound. */
+ * Implementation (not part of the contract): up to 8 tokens run the
+ * persistent single-token kernel once per token, 9 and more the tensor-core
+ * grouped GEMMs; the CUDA-core grouped path runs where neither fits the shape
+ * (or under MOE_FLAG_NO_DECODE_KERNEL / MOE_FLAG_NO_TENSOR_PREFILL); each path
+ * meets the same accuracy bound. */
 MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
                 uint16_t *y_bf16, float *y_f32, int32_t *ids, float *w,
                 void *stream);

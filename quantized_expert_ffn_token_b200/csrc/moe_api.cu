@@ -139,7 +139,7 @@ int alloc_workspace(moe_ctx *ctx) {
         size_t per = (size_t)6 * c.d_model * c.d_ff;   // bytes of one expert's fp16 B stages
         size_t cap = (size_t)c.max_tokens * (c.top_k + c.n_shared) / 256;
         if (cap > (size_t)ctx->nx) cap = ctx->nx;
-        if (!tc_supported(ctx, 64)) cap = 0;   // only the tensor-core path reads it
+        if (!tc_supported(ctx, TC_MIN_TOKENS)) cap = 0;   // only the tensor-core path reads it
         long long lim = c.device_mem_limit;
         if (cap > 0 && lim > 0 && (long long)(ctx->allocated + cap * per + cap * 4) > lim) cap = 0;
         if (cap > 0 && ctx_alloc(ctx, (void **)&ws.wcache, cap * per, "weight cache") != MOE_OK) cap = 0;

@@ -287,8 +287,13 @@ int launch_resid_norm(const moe_ctx *ctx, int T, float *resid, const uint16_t *y
                       const uint16_t *x_in, uint16_t *x_out, cudaStream_t st);
 bool decode_supported(const moe_ctx *ctx);   // the shape fits the single-token kernel
 // Token counts up to this run the single-token kernel once per token (the tokens
-// of a layer, and of a stack, are independent).
-constexpr int DECODE_TOKENS_MAX = 16;
+// of a layer, and of a stack, are independent); from TC_MIN_TOKENS on the
+// tensor-core grouped GEMMs take over.  Measured on a B200 (one layer of the
+// 2560 x 512-expert shape, Q4B32): the single-token kernel costs ~25 us per token,
+// the tensor-core path ~280 us at 64 tokens and less with fewer experts touched,
+// the CUDA-core path 0.8 ms at 16 tokens; so the tensor cores take over early.
+constexpr int DECODE_TOKENS_MAX = 8;
+constexpr int TC_MIN_TOKENS = DECODE_TOKENS_MAX + 1;
 int decode_setup(moe_ctx *ctx);
 size_t decode_xchg_bytes(const moe_config &c);
 size_t decode_xchg_counter_bytes();   // the counters at the start of the exchange area

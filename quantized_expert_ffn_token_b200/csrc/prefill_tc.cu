@@ -858,7 +858,7 @@ int launch_tc_router(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, fl
 bool tc_supported(const moe_ctx *ctx, int T) {
     const moe_config &c = ctx->cfg;
     if (c.flags & MOE_FLAG_NO_TENSOR_PREFILL) return false;
-    if (T < 64) return false;
+    if (T < TC_MIN_TOKENS) return false;
     // n-tiles of 256 output columns: 2I and d must be multiples of 256
     if ((2 * c.d_ff) % TC_BN || c.d_model % TC_BN || c.d_model % TC_BK || c.d_ff % TC_BK) return false;
     // A-row offsets are 32-bit element indices: rows (tokens or slots) x K below 2^31

@@ -38,7 +38,7 @@ BF16_TOL = 1e-3
 # relative L2 before the bf16 rounding (inside F32_TOL), hence about
 # sqrt(4e-4 * 2^-7.5) = 1.5e-3 between the two bf16 roundings.
 TC_BF16_TOL = 2e-3
-TC_MIN_TOKENS = 64
+TC_MIN_TOKENS = 9   # the library's first token count on the tensor-core path
 
 
 def bf16_tol(T: int) -> float:

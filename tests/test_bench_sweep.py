@@ -21,9 +21,8 @@ def test_flags_match_the_binding():
 
 @pytest.mark.parametrize("T, paths, default", [
     (1, {"single-token kernel", "cuda-core"}, "single-token kernel"),
-    (16, {"single-token kernel", "cuda-core"}, "single-token kernel"),
-    (17, {"cuda-core"}, "cuda-core"),
-    (63, {"cuda-core"}, "cuda-core"),
+    (8, {"single-token kernel", "cuda-core"}, "single-token kernel"),
+    (9, {"cuda-core", "tensor-core"}, "tensor-core"),
     (64, {"cuda-core", "tensor-core"}, "tensor-core"),
     (8192, {"cuda-core", "tensor-core"}, "tensor-core"),
 ])
@@ -38,11 +37,11 @@ def test_summary_names_the_fastest_path_and_checks_the_default():
             {"T": 8, "path": "cuda-core", "ms": 0.15},
             {"T": 128, "path": "cuda-core", "ms": 1.0},
             {"T": 128, "path": "tensor-core", "ms": 0.4},
-            {"T": 32, "path": "cuda-core", "ms": 0.3}]
+            {"T": 32, "path": "tensor-core", "ms": 0.3}]
     s = {r["T"]: r for r in bench.sweep_summary(rows)}
     assert [r["T"] for r in bench.sweep_summary(rows)] == [8, 32, 128]
     assert s[8]["fastest"] == "cuda-core" and not s[8]["default_is_fastest"] and s[8]["default_ms"] == 0.20
-    assert s[32]["fastest"] == "cuda-core" and s[32]["default_is_fastest"]
+    assert s[32]["fastest"] == "tensor-core" and s[32]["default_is_fastest"]
     assert s[128]["fastest"] == "tensor-core" and s[128]["default_is_fastest"] and s[128]["fastest_ms"] == 0.4
 
 
@@ -60,7 +59,7 @@ def test_thresholds_match_the_library_sources():
     internal = open(os.path.join(csrc, "moe_internal.cuh")).read()
     m = re.search(r"constexpr int DECODE_TOKENS_MAX = (\d+);", internal)
     assert m and int(m.group(1)) == bench.DISPATCH_DECODE_MAX
+    m = re.search(r"constexpr int TC_MIN_TOKENS = DECODE_TOKENS_MAX \+ (\d+);", internal)
+    assert m and bench.DISPATCH_DECODE_MAX + int(m.group(1)) == bench.DISPATCH_TC_MIN
     tc = open(os.path.join(csrc, "prefill_tc.cu")).read()
-    body = tc[tc.index("bool tc_supported("):]
-    m = re.search(r"if \(T < (\d+)\) return false;", body)
-    assert m and int(m.group(1)) == bench.DISPATCH_TC_MIN
+    assert "if (T < TC_MIN_TOKENS) return false;" in tc[tc.index("bool tc_supported("):]

@@ -63,7 +63,7 @@ def test_tiny_layer_all_tokens(fmt):
     sess.close()
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 5, 16, 17, 63, 64, 127, 128, 129])
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8, 9, 16, 17, 63, 64, 127, 128, 129])
 def test_tiny_ragged_token_counts(T):
     capi, session = _cuda()
     sess = session.Session(TINY, max_tokens=256)
@@ -77,11 +77,13 @@ def test_tiny_ragged_token_counts(T):
 
 
 def test_batch_equals_single_tokens():
-    """Token independence of the grouped path: a token's output does not depend
-    on which other tokens share the call (bit for bit).  Pinned to the grouped
-    path: small calls would otherwise run the single-token kernel per token."""
+    """Token independence of the CUDA-core grouped path: a token's output does not
+    depend on which other tokens share the call (bit for bit).  Pinned to that
+    path: small calls would otherwise run the single-token kernel and larger ones
+    the tensor cores, whose fp32 atomics sum in no fixed order."""
     capi, session = _cuda()
-    sess = session.Session(TINY, max_tokens=64, flags=capi.MOE_FLAG_NO_DECODE_KERNEL)
+    sess = session.Session(TINY, max_tokens=64,
+                           flags=capi.MOE_FLAG_NO_DECODE_KERNEL | capi.MOE_FLAG_NO_TENSOR_PREFILL)
     sess.load_synthetic()
     x = _tokens(TINY, 37, stream=5)
     gy, gyf, gids, gw = _run(sess, 0, x)
