@@ -220,15 +220,19 @@ MOE_API int moe_trace_read(moe_ctx *ctx, unsigned long long *out, int n_max, int
  * allocation after start-up, plain C hosts that only receive device
  * pointers).  It computes the router logits of T tokens and their softmax
  * top-k exactly as moe_forward does, from caller-owned device buffers:
- *   x_bf16 [T][d_model] bf16, router_w [n_experts][d_model] fp32,
- *   router_bias [n_experts] fp32 or NULL; outputs ids [T][top_k] int32 and
- *   w [T][top_k] fp32 (descending weight, equal logits -> lower id).
+ *   x_bf16 [T][d_model] bf16, router_w [n_experts][d_model] fp32 (16-byte
+ *   aligned), router_bias [n_experts] fp32 or NULL; outputs ids [T][top_k]
+ *   int32 and w [T][top_k] fp32 (descending weight, equal logits -> lower id;
+ *   a NaN logit ranks as -inf).  Limits: d_model a multiple of 4 and at most
+ *   16384, n_experts <= 1024, top_k <= min(n_experts, 32); anything else, or
+ *   a misaligned router_w, returns MOE_ERR_INVALID_ARG before any work.
  * The logits live in a fixed array in device memory that the library holds
  * on every device that loads it, until the process exits:
  * T * n_experts must not exceed MOE_ROUTE_STATIC_MAX_LOGITS
  * (MOE_ERR_TOO_MANY_TOKENS otherwise, with a message in moe_last_error()).
  * The first call on a device looks up that array's device address (make it
- * before any stream capture on that device).  Calls share the array: calls
+ * before any stream capture on that device); the address is kept for the
+ * process, so do not call this on a device after cudaDeviceReset on it.  Calls share the array: calls
  * that overlap on the GPU (other streams, other host threads) race; order
  * them on one stream.  Asynchronous on `stream`; calls no allocating routine.
  * Errors: INVALID_ARG, TOO_MANY_TOKENS, UNSUPPORTED (device index >= 64), CUDA. */

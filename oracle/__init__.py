@@ -61,6 +61,8 @@ def lib():
             L.oracle_weight.argtypes = [ctypes.c_int, _u8, ctypes.c_uint16, ctypes.c_int]
             L.oracle_silu.restype = ctypes.c_double
             L.oracle_silu.argtypes = [ctypes.c_double]
+            L.oracle_dequant.restype = None
+            L.oracle_dequant.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8, _u16, _dp]
             L.oracle_qmatvec.restype = None
             L.oracle_qmatvec.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8, _u16, _dp, _dp]
             L.oracle_expert.restype = None
@@ -150,19 +152,14 @@ def block_weights(fmt, blk, scale_bits) -> np.ndarray:
     return np.array([lib().oracle_weight(f, blk, int(scale_bits) & 0xFFFF, j) for j in range(32)])
 
 
-def dequant_matrix(fmt, codes, scales) -> np.ndarray:
+def dequant(fmt, codes, scales) -> np.ndarray:
     """Dense fp64 [rows, K] of a packed matrix (codes [rows, K/32, B], scales
-    [rows, K/32]), built with ``qmatvec`` on unit vectors so that it goes
-    through the same decode as every other oracle call."""
+    [rows, K/32]): w = s * (q - zero) element by element, in C."""
     codes = _u8a(_np(codes))
+    scales = _u16a(_np(scales))
     rows, nb = codes.shape[0], codes.shape[1]
-    K = nb * 32
-    out = np.empty((rows, K))
-    e = np.zeros(K)
-    for k in range(K):
-        e[:] = 0.0
-        e[k] = 1.0
-        out[:, k] = qmatvec(fmt, codes, scales, e)
+    out = np.empty((rows, nb * 32))
+    lib().oracle_dequant(_fmt(fmt), rows, nb * 32, codes, scales, out)
     return out
 
 
@@ -300,3 +297,67 @@ def moe_token_with_ids(fmt, x_bf16_row, ids, router_w, router_b, get_expert, get
         g, u, dn = get_shared(s)
         y += expert(fmt, g, u, dn, x)
     return y, w
+
+
+def moe_rows_dense(fmt, k, x_bf16, router_w, router_b, get_expert, get_shared, n_shared=1,
+                   ids_for=None, threads: int | None = None):
+    """The layer for many tokens, each on its own, with the experts' matrix
+    products done per expert over all of its tokens at once.
+
+    Same steps and the same fp64 arithmetic as ``moe_token`` (router logits,
+    softmax top-k, SwiGLU per chosen expert, weighted sum + shared), with two
+    library primitives in place of the per-token loops: the router logits are
+    one fp64 matrix product, and every expert is dequantised once (``dequant``)
+    and applied to the stacked rows of its tokens with fp64 matrix products.
+    Only the order of the fp64 sums differs from ``moe_token``.
+
+    x_bf16: bf16 bits [n, d].  ids_for: optional {row: ids} for rows whose
+    experts are given (the GPU's choice at a near tie); their weights are the
+    softmax of the oracle's logits renormalised over the given ids, as in
+    ``moe_token_with_ids``.  Returns (y fp64 [n, d], ids [n, k], w [n, k],
+    gap [n])."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    x = bf16_to_f64(np.asarray(x_bf16))
+    n, d = x.shape
+    lg = x @ np.asarray(router_w, dtype=np.float64).T
+    if router_b is not None:
+        lg = lg + np.asarray(router_b, dtype=np.float64)
+    ids = np.empty((n, k), dtype=np.int32)
+    w = np.empty((n, k))
+    gap = np.empty(n)
+    for t in range(n):
+        ids[t], w[t], gap[t] = route(lg[t], k)
+    for t, g_ids in (ids_for or {}).items():
+        p = np.exp(lg[t] - lg[t].max())
+        p /= p.sum()
+        g_ids = np.asarray(g_ids, dtype=np.int64)
+        ids[t] = g_ids
+        w[t] = p[g_ids] / p[g_ids].sum()
+    y = np.zeros((n, d))
+    experts = sorted(set(int(e) for e in ids.ravel()))
+
+    def apply(mats, xs):
+        (gc, gs), (uc, us), (dc, ds) = mats
+        g = xs @ dequant(fmt, gc, gs).T
+        u = xs @ dequant(fmt, uc, us).T
+        h = g / (1.0 + np.exp(-g)) * u
+        return h @ dequant(fmt, dc, ds).T
+
+    def routed(e):
+        rows, slots = np.nonzero(ids == e)
+        return e, rows, slots, apply(get_expert(e), x[rows])
+
+    with ThreadPoolExecutor(max_workers=threads or min(16, os.cpu_count() or 1)) as ex:
+        res = list(ex.map(routed, experts))
+        shared = list(ex.map(lambda s: apply(get_shared(s), x), range(n_shared)))
+    contrib = [[] for _ in range(n)]   # (slot j, y_e row) per token
+    for e, rows, slots, ye in res:
+        for i, (t, j) in enumerate(zip(rows, slots)):
+            contrib[t].append((int(j), ye[i]))
+    for t in range(n):
+        for j, ye in sorted(contrib[t], key=lambda c: c[0]):   # j = 0..k-1, as moe_token
+            y[t] += w[t, j] * ye
+    for ys in shared:
+        y += ys
+    return y, ids, w, gap

@@ -117,6 +117,24 @@ void oracle_qmatvec(int fmt, int rows, int K, const uint8_t *codes,
     }
 }
 
+/* Dense fp64 copy of a packed matrix: out[r][k] = W[r][k] = s_rb * (q - zero)
+ * for k in block b, straight from the block definition (one scale decode per
+ * block).  codes [rows][K/32][B], scales [rows][K/32], out [rows][K]. */
+void oracle_dequant(int fmt, int rows, int K, const uint8_t *codes,
+                    const uint16_t *scales, double *out)
+{
+    int nb = K / 32, B = block_bytes(fmt);
+    int zero = (fmt == ORACLE_Q4B32) ? 8 : (fmt == ORACLE_Q2B32) ? 2 : 4;
+    for (int r = 0; r < rows; ++r)
+        for (int b = 0; b < nb; ++b) {
+            const uint8_t *blk = codes + ((size_t)r * nb + b) * B;
+            double s = oracle_half_to_double(scales[(size_t)r * nb + b]);
+            double *o = out + (size_t)r * K + (size_t)b * 32;
+            for (int j = 0; j < 32; ++j)
+                o[j] = s * (double)(oracle_code(fmt, blk, j) - zero);
+        }
+}
+
 /* silu(z) = z / (1 + e^-z). */
 double oracle_silu(double z) { return z / (1.0 + exp(-z)); }
 

@@ -782,7 +782,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                 float lv[EMAX];
 #pragma unroll
                 for (int t = 0; t < EMAX; ++t)
-                    if (tid + t * NT < E) lv[t] = ld_gpu(p.x_logits + tid + t * NT);
+                    lv[t] = (tid + t * NT < E) ? ld_gpu(p.x_logits + tid + t * NT) : -INFINITY;
+                // a NaN logit ranks as -inf (last, by id): the selection below then always
+                // finds k distinct experts below E
+#pragma unroll
+                for (int t = 0; t < EMAX; ++t) lv[t] = isnan(lv[t]) ? -INFINITY : lv[t];
 #pragma unroll
                 for (int t = 0; t < EMAX; ++t) {
                     if (tid + t * NT < E) {

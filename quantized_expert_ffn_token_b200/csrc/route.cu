@@ -17,40 +17,50 @@ namespace {
 constexpr int RT_TOK = 8;   // tokens per router block
 constexpr int RT_EXP = 8;   // experts per router block (one per warp)
 
-// logits[t][e] = sum_i x[t][i] * W[e][i] + b[e], fp32 FMA accumulation.
+// logits[t][e] = sum_i x[t][i] * W[e][i] + b[e], fp32 FMA accumulation.  The
+// tokens' inputs pass through shared memory RT_CHUNK columns at a time, so any
+// d fits; each lane's FMAs run in the same order whatever the chunking.
+constexpr int RT_CHUNK = 4096;
 __global__ void __launch_bounds__(256) k_router_simt(const uint16_t *__restrict__ x, int T, int d,
                                                      int E, const float *__restrict__ W,
                                                      const float *__restrict__ b,
                                                      float *__restrict__ logits) {
-    extern __shared__ float xs[];   // [RT_TOK][d]
-    int t0 = blockIdx.y * RT_TOK;
-    int nt = min(RT_TOK, T - t0);
-    for (int i = threadIdx.x; i < nt * d; i += blockDim.x) {
-        int tt = i / d, c = i % d;
-        uint32_t bits = (uint32_t)x[(size_t)(t0 + tt) * d + c] << 16;
-        xs[tt * d + c] = __uint_as_float(bits);
-    }
-    __syncthreads();
-    int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int e = blockIdx.x * RT_EXP + warp;
-    if (e >= E) return;
+    extern __shared__ float xs[];   // [RT_TOK][min(d, RT_CHUNK)]
+    const int t0 = blockIdx.y * RT_TOK;
+    const int nt = min(RT_TOK, T - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * RT_EXP + warp;
+    const int cw = min(d, RT_CHUNK);
     float acc[RT_TOK];
 #pragma unroll
     for (int tt = 0; tt < RT_TOK; ++tt) acc[tt] = 0.f;
-    const float4 *Wr = reinterpret_cast<const float4 *>(W + (size_t)e * d);
-    for (int i4 = lane; i4 < d / 4; i4 += 32) {
-        float4 wv = Wr[i4];
+    for (int c0 = 0; c0 < d; c0 += cw) {
+        const int n = min(cw, d - c0);
+        __syncthreads();   // the previous chunk is no longer read
+        for (int i = threadIdx.x; i < nt * n; i += blockDim.x) {
+            int tt = i / n, c = i % n;
+            uint32_t bits = (uint32_t)x[(size_t)(t0 + tt) * d + c0 + c] << 16;
+            xs[tt * cw + c] = __uint_as_float(bits);
+        }
+        __syncthreads();
+        if (e < E) {
+            const float4 *Wr = reinterpret_cast<const float4 *>(W + (size_t)e * d + c0);
+            for (int i4 = lane; i4 < n / 4; i4 += 32) {
+                float4 wv = Wr[i4];
 #pragma unroll
-        for (int tt = 0; tt < RT_TOK; ++tt) {
-            if (tt < nt) {
-                const float *xv = xs + tt * d + 4 * i4;
-                acc[tt] = fmaf(wv.x, xv[0], acc[tt]);
-                acc[tt] = fmaf(wv.y, xv[1], acc[tt]);
-                acc[tt] = fmaf(wv.z, xv[2], acc[tt]);
-                acc[tt] = fmaf(wv.w, xv[3], acc[tt]);
+                for (int tt = 0; tt < RT_TOK; ++tt) {
+                    if (tt < nt) {
+                        const float *xv = xs + tt * cw + 4 * i4;
+                        acc[tt] = fmaf(wv.x, xv[0], acc[tt]);
+                        acc[tt] = fmaf(wv.y, xv[1], acc[tt]);
+                        acc[tt] = fmaf(wv.z, xv[2], acc[tt]);
+                        acc[tt] = fmaf(wv.w, xv[3], acc[tt]);
+                    }
+                }
             }
         }
     }
+    if (e >= E) return;
 #pragma unroll
     for (int tt = 0; tt < RT_TOK; ++tt) {
         float v = acc[tt];
@@ -65,7 +75,9 @@ __device__ inline bool better(float v, int id, float bv, int bid) {
 }
 
 // One warp per token: k rounds of warp arg-max over the token's E logits,
-// then the softmax over the chosen logits.
+// then the softmax over the chosen logits.  A NaN logit is read as -inf (it
+// ranks last, by id); a chosen expert is marked NaN, which better() never
+// accepts, so every round picks a distinct id below E (k <= E).
 __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, int T, int E, int k,
                                               int32_t *__restrict__ ids, float *__restrict__ w) {
     extern __shared__ float lg[];   // [8][E]
@@ -73,7 +85,10 @@ __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, 
     int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
     float *my = lg + warp * E;
-    for (int e = lane; e < E; e += 32) my[e] = logits[(size_t)t * E + e];
+    for (int e = lane; e < E; e += 32) {
+        const float v = logits[(size_t)t * E + e];
+        my[e] = isnan(v) ? -INFINITY : v;
+    }
     __syncwarp();
     float chosen_v = -INFINITY;
     int chosen_id = -1;
@@ -95,12 +110,13 @@ __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, 
                 bid = oid;
             }
         }
+        if (bid >= E) bid = 0;   // unreachable while k <= E; keeps every index in range
         if (lane == j) {
             chosen_v = bv;
             chosen_id = bid;
         }
         __syncwarp();
-        if (lane == 0) my[bid] = -INFINITY;
+        if (lane == 0) my[bid] = __int_as_float(0x7fc00000);   // NaN: taken
         __syncwarp();
     }
     float top = __shfl_sync(0xffffffffu, chosen_v, 0);
@@ -187,18 +203,17 @@ __global__ void k_scatter(const int32_t *__restrict__ ids, int T, int k, int E, 
     }
 }
 
+// Dynamic shared memory of k_router_simt for hidden size d.
+size_t router_simt_smem(int d) { return (size_t)RT_TOK * (d < RT_CHUNK ? d : RT_CHUNK) * sizeof(float); }
+
 }  // namespace
 
 int launch_router_simt(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T,
                        float *logits, cudaStream_t st) {
     const moe_config &c = ctx->cfg;
-    size_t smem = (size_t)RT_TOK * c.d_model * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      200 * 1024));
-        attr_set = true;
-    }
+    const size_t smem = router_simt_smem(c.d_model);
+    QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)router_simt_smem(RT_CHUNK)));
     dim3 grid((c.n_experts + RT_EXP - 1) / RT_EXP, (T + RT_TOK - 1) / RT_TOK);
     k_router_simt<<<grid, 256, smem, st>>>(x, T, c.d_model, c.n_experts, Ly.router_w, Ly.router_b,
                                           logits);
@@ -220,9 +235,10 @@ int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, fl
 int launch_route_raw(const uint16_t *x, int T, int d, int E, int k, const float *W, const float *b,
                      float *logits, int32_t *ids, float *w, cudaStream_t st) {
     // same opt-in size as launch_router_simt, so neither caller shrinks it for the other
-    QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    QE_CHECK(cudaFuncSetAttribute(k_router_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)router_simt_smem(RT_CHUNK)));
     dim3 grid((E + RT_EXP - 1) / RT_EXP, (T + RT_TOK - 1) / RT_TOK);
-    k_router_simt<<<grid, 256, (size_t)RT_TOK * d * sizeof(float), st>>>(x, T, d, E, W, b, logits);
+    k_router_simt<<<grid, 256, router_simt_smem(d), st>>>(x, T, d, E, W, b, logits);
     QE_CHECK_LAUNCH("k_router_simt");
     k_topk<<<(T + 7) / 8, 256, 8 * (size_t)E * sizeof(float), st>>>(logits, T, E, k, ids, w);
     QE_CHECK_LAUNCH("k_topk");

@@ -25,7 +25,9 @@ std::mutex g_mu;
 float *g_scratch_ptr[kMaxDevices] = {};   // device address of g_route_scratch, per device
 
 // Host code cannot take the device address of a __device__ array directly;
-// ask the runtime for it once per device, with that device current.
+// ask the runtime for it once per device, with that device current.  The
+// address belongs to the device's primary context: after cudaDeviceReset on a
+// device this library must not be used on that device again in the process.
 int scratch_for_current_device(float **out) {
     int dev = 0;
     QE_CHECK(cudaGetDevice(&dev));
@@ -47,8 +49,10 @@ extern "C" int moe_route_static(const uint16_t *x_bf16, int T, int d_model, cons
                                 const float *router_bias, int n_experts, int top_k, int32_t *ids,
                                 float *w, void *stream) {
     if (!x_bf16 || !router_w || !ids || !w || T < 0 || d_model <= 0 || n_experts <= 0 || top_k <= 0 ||
-        top_k > n_experts || top_k > 32 || n_experts > 1024 || d_model % 4 != 0 || d_model > 12288)
+        top_k > n_experts || top_k > 32 || n_experts > 1024 || d_model % 4 != 0 || d_model > 16384)
         return MOE_ERR_INVALID_ARG;
+    // the router reads its weight rows with 16-byte loads
+    if (reinterpret_cast<uintptr_t>(router_w) % 16 != 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if ((long long)T * n_experts > MOE_ROUTE_STATIC_MAX_LOGITS) {
         return qeffn::set_too_many(

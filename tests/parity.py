@@ -56,6 +56,74 @@ def bits_to_f64(bits) -> np.ndarray:
     return oracle.bf16_to_f64(np.asarray(bits).view(np.uint16))
 
 
+class HostLayer:
+    """One whole layer of the seeded generator in host memory, generated on the
+    device (fast) and copied over once; the same interface as ExpertSource."""
+
+    def __init__(self, cfg: synth.LayerConfig, layer: int, device="cuda"):
+        self.cfg, self.layer = cfg, layer
+        W = synth.layer_weights(cfg, layer, device=device)
+        self.router_w = np.asarray(W["router_w"], dtype=np.float32)
+        self.router_b = W["router_b"]
+        self.codes = [to_np(t) for t in W["codes"]]
+        self.scales = [to_np(t).view(np.uint16) for t in W["scales"]]
+        self.sh_codes = [to_np(t) for t in W["sh_codes"]]
+        self.sh_scales = [to_np(t).view(np.uint16) for t in W["sh_scales"]]
+        del W
+
+    def expert(self, e: int):
+        return tuple((self.codes[t][e], self.scales[t][e]) for t in range(3))
+
+    def shared(self, s: int):
+        return tuple((self.sh_codes[t][s], self.sh_scales[t][s]) for t in range(3))
+
+
+def oracle_rows_dense(cfg, src, x_bits: np.ndarray, rows):
+    """Oracle outputs of many token rows at once (experts applied per expert
+    with fp64 matrix products): (y [n, d], ids, w, gap)."""
+    rows = list(rows)
+    return oracle.moe_rows_dense(cfg.fmt, cfg.k, x_bits[rows], src.router_w, src.router_b,
+                                 src.expert, src.shared, cfg.n_shared)
+
+
+def oracle_routing(cfg, src, x_bits: np.ndarray):
+    """Oracle routing of every row (router logits as one fp64 matrix product,
+    then the oracle's softmax top-k per token): ids [n, k], w [n, k], gap [n]."""
+    x = oracle.bf16_to_f64(np.asarray(x_bits).view(np.uint16))
+    lg = x @ np.asarray(src.router_w, dtype=np.float64).T
+    if src.router_b is not None:
+        lg = lg + np.asarray(src.router_b, dtype=np.float64)
+    n = lg.shape[0]
+    ids = np.empty((n, cfg.k), dtype=np.int32)
+    w = np.empty((n, cfg.k))
+    gap = np.empty(n)
+    for t in range(n):
+        ids[t], w[t], gap[t] = oracle.route(lg[t], cfg.k)
+    return ids, w, gap, lg
+
+
+def ids_agree(g_ids, o_ids, o_gap: float, logits) -> str:
+    """How the GPU's ids of one token relate to the oracle's.
+
+    'same': identical, in order.  'order': the same experts, and wherever the
+    order differs the oracle's logits of the two experts at that position are
+    within NEAR_TIE of each other (a near tie inside the chosen set).  'tie':
+    a different set, allowed because the oracle's k-th and (k+1)-th logits are
+    within NEAR_TIE.  Anything else fails the assertion."""
+    g_ids, o_ids = np.asarray(g_ids), np.asarray(o_ids)
+    if np.array_equal(g_ids, o_ids):
+        return "same"
+    if sorted(g_ids.tolist()) == sorted(o_ids.tolist()):
+        lg = logits()
+        diff = np.nonzero(g_ids != o_ids)[0]
+        worst = max(abs(lg[g_ids[j]] - lg[o_ids[j]]) for j in diff)
+        assert worst < NEAR_TIE, f"ids {g_ids.tolist()} != oracle {o_ids.tolist()} (order, gap {worst:.3g})"
+        return "order"
+    assert o_gap < NEAR_TIE, (f"ids {g_ids.tolist()} != oracle {o_ids.tolist()} "
+                              f"(k-th to (k+1)-th gap {o_gap:.3g})")
+    return "tie"
+
+
 class ExpertSource:
     """Generates (on the host) exactly the experts the oracle asks for."""
 
@@ -94,20 +162,28 @@ def oracle_rows(cfg, src: ExpertSource, x_bits: np.ndarray, rows):
 
 
 def check_rows(cfg, src, x_bits, rows, g_y_bits, g_yf, g_ids, g_w, o=None, report=None, tol16=BF16_TOL):
-    """Compare GPU outputs of `rows` (arrays indexed like rows) with the oracle."""
+    """Compare GPU outputs of `rows` (arrays indexed like rows) with the oracle.
+
+    Ids follow the near-tie rule (ids_agree); a token whose set differs at a
+    near tie is re-evaluated by the oracle with the GPU's ids; a token whose
+    chosen experts come in another order at a near tie is compared weight by
+    weight in the GPU's order."""
     oy, oids, ow, ogap = o if o is not None else oracle_rows(cfg, src, x_bits, rows)
     oy = oy.copy()
     ow = ow.copy()
-    flips = 0
+    flips = reorders = 0
     for i, t in enumerate(rows):
-        if not np.array_equal(g_ids[i], oids[i]):
-            assert ogap[i] < NEAR_TIE, (
-                f"token {t}: ids {g_ids[i].tolist()} != oracle {oids[i].tolist()} "
-                f"(10th-11th gap {ogap[i]:.3g})")
+        xf = lambda: oracle.router_logits(oracle.bf16_to_f64(x_bits[t]), src.router_w, src.router_b)
+        kind = ids_agree(g_ids[i], oids[i], ogap[i], xf)
+        if kind == "tie":
             flips += 1
             oy[i], ow[i] = oracle.moe_token_with_ids(cfg.fmt, x_bits[t], g_ids[i], src.router_w,
                                                      src.router_b, src.expert, src.shared,
                                                      cfg.n_shared)
+        elif kind == "order":
+            reorders += 1
+            pos = {int(e): j for j, e in enumerate(oids[i])}
+            ow[i] = ow[i][[pos[int(e)] for e in g_ids[i]]]
     assert np.max(np.abs(g_w - ow)) <= W_TOL, np.max(np.abs(g_w - ow))
     e32 = rel_l2(g_yf, oy)
     assert e32 <= F32_TOL, e32
@@ -116,7 +192,7 @@ def check_rows(cfg, src, x_bits, rows, g_y_bits, g_yf, g_ids, g_w, o=None, repor
     e16 = rel_l2(bits_to_f64(g_y_bits), bits_to_f64(oracle.round_bf16(oy)))
     assert e16 <= tol16, e16
     if report is not None:
-        report.update(rel_l2_f32=e32, rel_l2_bf16=e16, near_tie_flips=flips)
+        report.update(rel_l2_f32=e32, rel_l2_bf16=e16, near_tie_flips=flips, near_tie_reorders=reorders)
     return e32, e16, flips
 
 

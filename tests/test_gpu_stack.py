@@ -8,12 +8,19 @@ import torch
 
 import oracle
 import synth
-from tests.parity import ExpertSource, bf16_tol, bits_to_f64, check_rows, oracle_rows, to_np
+from tests.parity import (W_TOL, ExpertSource, HostLayer, bf16_tol, bits_to_f64, check_rows, ids_agree,
+                          oracle_routing, oracle_rows_dense, to_np)
 
 pytestmark = pytest.mark.gpu
 
 
-def _stack(name, rows=None, check_layers=None):
+def _stack(name, rows=None, check_layers=None, dense=False, layer0_all=False):
+    """The whole stack through the C ABI with per-layer records of `rows` (all
+    when None), checked layer by layer against the oracle (teacher-forced).
+    dense: the oracle evaluates each layer's rows with per-expert fp64 matrix
+    products over a host copy of that layer.  layer0_all: also route every
+    token of layer 0 (its recorded input) and check every token's ids and
+    weights against the oracle."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from quantized_expert_ffn_token_b200 import capi, session
@@ -36,6 +43,16 @@ def _stack(name, rows=None, check_layers=None):
     capi.moe_forward_stack(sess.ctx, 0, L, x, T, r_out, rec)
     torch.cuda.synchronize()
     assert capi.moe_get_device_error(sess.ctx) == 0
+    all0 = None
+    if layer0_all:
+        x0 = torch.empty((1, T, d), dtype=torch.int16, device=dev)
+        id0 = torch.empty((1, T, k), dtype=torch.int32, device=dev)
+        w0 = torch.empty((1, T, k), dtype=torch.float32, device=dev)
+        r1 = torch.empty((T, d), dtype=torch.float32, device=dev)
+        capi.moe_forward_stack(sess.ctx, 0, 1, x, T, r1, capi.make_record(x=x0, ids=id0, w=w0))
+        torch.cuda.synchronize()
+        all0 = (to_np(x0[0]), to_np(id0[0]), to_np(w0[0]))
+        del x0, id0, w0, r1
     sess.close()
     xr, yr, yfr, idr, wr, r_out = map(to_np, (xr, yr, yfr, idr, wr, r_out))
     rows = list(range(T)) if rows is None else list(rows)
@@ -52,11 +69,26 @@ def _stack(name, rows=None, check_layers=None):
 
     worst = {}
     for l in (range(L) if check_layers is None else check_layers):
-        src = ExpertSource(cfg, l)
+        src = HostLayer(cfg, l) if dense else ExpertSource(cfg, l)
         rep = {}
         idx = list(range(len(rows)))
-        check_rows(cfg, src, xr[l], idx, yr[l], yfr[l], idr[l], wr[l], report=rep, tol16=bf16_tol(T))
+        o = oracle_rows_dense(cfg, src, xr[l], idx) if dense else None
+        check_rows(cfg, src, xr[l], idx, yr[l], yfr[l], idr[l], wr[l], o=o, report=rep, tol16=bf16_tol(T))
         worst[l] = rep
+        if l == 0 and all0 is not None:
+            # every token of layer 0: the recorded input of a sampled row is the same row of the
+            # all-token record, and every token's routing matches the oracle
+            xa, ida, wa = all0
+            assert np.array_equal(xa[rows], xr[0])
+            oids, ow, ogap, olg = oracle_routing(cfg, src, xa)
+            flips = 0
+            for t in range(T):
+                kind = ids_agree(ida[t], oids[t], ogap[t], lambda: olg[t])
+                if kind == "same":
+                    assert np.max(np.abs(wa[t] - ow[t])) <= W_TOL
+                flips += kind != "same"
+            worst["layer0_all_tokens_not_identical"] = flips
+        del src
     return worst
 
 
@@ -70,5 +102,9 @@ def test_verify_stack_48_layers():
 
 @pytest.mark.slow
 def test_long_prefill_stack_48_layers_sampled():
-    _stack("prefill_48l_q3_t32768", rows=[0, 16383, 32767],
-           check_layers=[0, 1, 23, 46, 47])
+    """The long-prefill stack (32768 tokens, 48 layers, Q3B32): a seeded sample
+    of 256 tokens checked in every one of the 48 layers, plus the routing of
+    every token in layer 0."""
+    T = synth.CONFIGS["prefill_48l_q3_t32768"].T
+    rows = sorted(np.random.default_rng(2026).choice(T, size=256, replace=False).tolist())
+    _stack("prefill_48l_q3_t32768", rows=rows, dense=True, layer0_all=True)

@@ -84,6 +84,20 @@ def test_golden_blocks(case):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("case", range(len(_golden())))
+def test_golden_blocks_dense(case):
+    fmt, blk, sbits, want = _golden()[case]
+    got = oracle.dequant(fmt, np.frombuffer(blk, np.uint8).reshape(1, 1, -1), np.array([[sbits]], np.uint16))
+    assert np.array_equal(got[0], want)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
+def test_dequant_matches_independent_packer_dense(fmt):
+    rng = np.random.default_rng(21)
+    q, s, packed, W = random_matrix(rng, fmt, 24, 160)
+    assert np.array_equal(oracle.dequant(fmt, packed, s), W)
+
+
 @pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
 def test_block_codes_roundtrip_through_independent_packer(fmt):
     rng = np.random.default_rng(2)
@@ -237,13 +251,21 @@ def _tokens(rng, T, d):
     return oracle.round_bf16(rng.standard_normal((T, d)))
 
 
-@pytest.mark.parametrize("fmt,bias", [("q4", False), ("q3", True), ("q2", True)])
-def test_layer_brute_force(fmt, bias):
+def _rows_dense(fmt, k, x, W, ids_for=None):
+    ge = lambda e: tuple((W["codes"][t][e], W["scales"][t][e]) for t in range(3))
+    gs = lambda s: tuple((W["sh_codes"][t][s], W["sh_scales"][t][s]) for t in range(3))
+    return oracle.moe_rows_dense(fmt, k, x, W["router_w"], W["router_b"], ge, gs,
+                                 n_shared=W["sh_codes"][0].shape[0], ids_for=ids_for)
+
+
+@pytest.mark.parametrize("fmt,bias,batched", [("q4", False, False), ("q3", True, False), ("q2", True, False),
+                                              ("q4", True, True), ("q3", False, True), ("q2", True, True)])
+def test_layer_brute_force(fmt, bias, batched):
     rng = np.random.default_rng(8)
     d, E, I, k, T = 64, 6, 32, 2, 5
     W = _layer(rng, fmt, d, E, I, 1, 32, bias=bias)
     x = _tokens(rng, T, d)
-    y, ids, w, gap = oracle.moe_layer(fmt, k, x, W)
+    y, ids, w, gap = (_rows_dense if batched else oracle.moe_layer)(fmt, k, x, W)
     xf = x.view(np.uint16).astype(np.uint32) << 16
     xf = xf.view(np.float32).astype(np.float64)
     for t in range(T):
@@ -355,3 +377,28 @@ def test_rmsnorm_closed_forms():
     out = oracle.rmsnorm(r, 0.0)
     assert math.isclose(np.mean(out ** 2), 1.0, rel_tol=1e-13)
     assert np.allclose(oracle.rmsnorm(r * 1024.0, 0.0), out, rtol=1e-14)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
+def test_rows_dense_matches_moe_layer_and_given_ids(fmt):
+    """The batched evaluation is the per-token layer with its fp64 sums reordered;
+    with ids given it matches moe_token_with_ids."""
+    rng = np.random.default_rng(22)
+    d, E, I, k, T = 96, 8, 64, 3, 17
+    W = _layer(rng, fmt, d, E, I, 1, 64, bias=True)
+    x = _tokens(rng, T, d)
+    y, ids, w, gap = oracle.moe_layer(fmt, k, x, W)
+    yd, idd, wd, gd = _rows_dense(fmt, k, x, W)
+    assert np.array_equal(ids, idd)
+    assert np.allclose(wd, w, rtol=1e-13)
+    assert np.allclose(gd, gap, rtol=1e-9, atol=1e-12)
+    assert np.allclose(yd, y, rtol=1e-12, atol=1e-13)
+    alt = {4: ids[4][::-1].copy(), 9: np.array([0, 1, 2], np.int32)}
+    ya, ida, wa, _ = _rows_dense(fmt, k, x, W, ids_for=alt)
+    ge = lambda e: tuple((W["codes"][t][e], W["scales"][t][e]) for t in range(3))
+    gs = lambda s: tuple((W["sh_codes"][t][s], W["sh_scales"][t][s]) for t in range(3))
+    for t, g_ids in alt.items():
+        yw, ww = oracle.moe_token_with_ids(fmt, x[t], g_ids, W["router_w"], W["router_b"], ge, gs)
+        assert np.array_equal(ida[t], g_ids)
+        assert np.allclose(wa[t], ww, rtol=1e-13)
+        assert np.allclose(ya[t], yw, rtol=1e-12, atol=1e-13)
