@@ -1,26 +1,32 @@
 """Benchmark of the quantized MoE FFN hot path on B200.
 
-Default workload: 48-layer decode, one token per step (d=2560, 512 experts,
-top-10 + 1 shared, SwiGLU intermediate 512, Q4B32 weights, seeded synthetic
-inputs).  A step = one token through all 48 layers (router, top-k, dispatch,
-expert SwiGLU, down projection, combine, residual + rmsnorm), weights and
-inputs resident in HBM.  Prints one JSON line (rank 0).
+A step is one pass of the whole path over one batch of seeded synthetic input,
+weights and inputs resident in HBM: router, top-k, dispatch, expert SwiGLU,
+down projection, shared expert, combine and, in the 48-layer stacks, residual
+add and rmsnorm between layers.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 (under torchrun): independent replicas, one per GPU, each decoding its
-own tokens (the layer does not shard for one token stream); value = tokens
+The headline is 48-layer single-token decode (d=2560, 512 experts, top-10 + 1
+shared, intermediate 512, Q4B32): one token through all 48 layers per step.
+The same line carries, under "secondary", the other measured workloads, each
+with its own roofline, CPU baseline and end-to-end figure: 48-layer verify
+(4 tokens, Q3B32, Zipf-biased routing), single-layer prefill (4096 tokens,
+Q4B32, Zipf-biased) and 48-layer long prefill (32768 tokens, Q3B32).
+
+N > 1 (under torchrun): independent replicas of the headline, one per GPU,
+each decoding its own tokens (one token stream does not shard); value = tokens
 of all ranks / max-over-ranks time.
 
   python bench.py --sweep [--sweep-workload W] [--sweep-t 1,2,...]
 
-times one layer at each token count on every path that accepts it (single-token
-kernel, CUDA-core path, tensor-core path) and ends with the fastest path per
-token count next to the one the library's dispatch picks.
+times one layer at each token count on every path that accepts it and ends
+with the fastest path per token count next to the one the dispatch picks.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -39,6 +45,8 @@ import synth  # noqa: E402
 
 METRIC = "48-layer MoE decode tok/s & prefill tok/s; % of HBM / MMA roofline"
 DEFAULT_WORKLOAD = "decode_48l_q4_t1"
+SECONDARY = ("verify_48l_q3_t4_zipf", "prefill_1l_q4_t4096_zipf", "prefill_48l_q3_t32768")
+FLUSH_BYTES = 256 << 20   # L2 flush between timed steps of workloads whose step streams less than ~1 GB
 
 
 def peaks() -> dict:
@@ -61,20 +69,36 @@ def router_bytes(cfg) -> int:
     return cfg.E * cfg.d * 4
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from one ncu capture of
-# the current kernels on one B200:
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \
-#       --clock-control none -k regex:k_decode -s 3 -c 1 \
-#       python bench.py --steps 3 --warmup 3 --no-secondary --cpu-layers 1 --layers 4
-# (a 4-layer stack: 118,442,240 B read + 2,858,752 B written; traffic grows with the layers a launch
-# runs, so a 48-layer launch is scaled by 48/4), and
-#   ncu ... -k regex:"k_tc_gemm|k_cache_fill" -s 12 -c 4 python bench.py \
-#       --workload prefill_1l_q4_t4096_zipf --steps 2 --warmup 3 --no-secondary --cpu-layers 1
-# (the cache fill and the two expert GEMMs of one layer; router excluded).
-DECODE_Q4_TRAFFIC_PER_LAYER = (118_442_240 + 2_858_752) / 4
-PREFILL_Q4_T4096_TRAFFIC = (61_968_640 + 157_297_920          # k_cache_fill
-                            + 500_800_256 + 41_342_720        # k_tc_gemm<gate/up>
-                            + 341_344_768 + 61_933_312)       # k_tc_gemm<down>
+def expert_flops(cfg, T: int) -> int:
+    """Multiply-adds x 2 of the experts of one layer on T tokens (k routed + shared per token)."""
+    return 2 * T * (cfg.k + cfg.n_shared) * 3 * cfg.d * cfg.I
+
+
+def router_flops(cfg, T: int) -> int:
+    return 2 * T * cfg.E * cfg.d
+
+
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, per unit
+# of work, each with the SHA-256 of the kernel source it was measured on: a figure is reported only
+# while that source is unchanged (a changed kernel reports null until it is measured again).  The
+# commands that produced them are in the profiles/ summaries named beside each entry.
+MEASURED_TRAFFIC = [
+    # {"kernel": ..., "workload": ..., "src": "<file>", "sha256": "...", "bytes_per_layer": ...,
+    #  "profile": "profiles/<name>.md"}
+]
+
+
+def _src_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, "quantized_expert_ffn_token_b200", "csrc", rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def measured_traffic(kernel: str, workload: str, layers: int):
+    """DRAM bytes per launch of `kernel` on `workload` from a capture of the current source, else None."""
+    for m in MEASURED_TRAFFIC:
+        if m["kernel"] == kernel and m["workload"] == workload and _src_sha(m["src"]) == m["sha256"]:
+            return m["bytes_per_layer"] * layers
+    return None
 
 
 def max_over_ranks(v: float, dist_on: bool, device) -> float:
@@ -90,11 +114,11 @@ def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
     return units_per_rank * world / seconds
 
 
-def decode_traffic(cfg, kernel: str):
-    """Measured DRAM bytes per launch of the single-token kernel for the Q4 decode shape."""
-    if kernel != "k_decode" or cfg.fmt != "q4" or cfg.T != 1 or (cfg.d, cfg.E, cfg.I, cfg.k) != (2560, 512, 512, 10):
-        return None
-    return DECODE_Q4_TRAFFIC_PER_LAYER * cfg.L
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 # ---------------------------------------------------------------------------
@@ -152,48 +176,78 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
-# CPU oracle timing (the baseline, and the --impl reference arm)
+# CPU oracle timing (each entry's cpu_baseline, and the --impl reference arm)
 # ---------------------------------------------------------------------------
-def oracle_decode_sample(cfg, n_layers: int, token_stream: int, n_tokens: int = 1) -> float:
-    """Seconds the oracle (one host core) takes to push `n_tokens` tokens through
-    `n_layers` layers; expert generation on the host is excluded from the timing."""
+def oracle_sample(cfg, n_tokens: int, threads: int, token_stream: int) -> dict:
+    """Time the oracle (plain C, fp64) on `n_tokens` independent tokens through one layer (layer 0),
+    `threads` tokens at a time on the host cores (its C calls release the GIL).  The experts the
+    tokens need are generated before the timed region.  The oracle's cost is the same for every
+    token and layer of a workload, so the rate of the whole workload follows by scaling."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     from tests.parity import ExpertSource
-    total = 0.0
-    for tk in range(n_tokens):
-        x = synth.tokens_bf16(cfg, 1, stream=token_stream + 7919 * tk)[0]
-        for l in range(n_layers):
-            src = ExpertSource(cfg, l)
-            xf = oracle.bf16_to_f64(x)
-            ids, _, _ = oracle.route(oracle.router_logits(xf, src.router_w, src.router_b), cfg.k)
-            for e in ids:
-                src.expert(int(e))          # generate outside the timed region
-            src.shared(0)
-            t0 = time.perf_counter()
-            y, _, _, _ = oracle.moe_token(cfg.fmt, cfg.k, x, src.router_w, src.router_b, src.expert,
-                                          src.shared, cfg.n_shared)
-            r = oracle.rmsnorm(xf + y)
-            total += time.perf_counter() - t0
-            x = oracle.round_bf16(r)
-    return total
+
+    src = ExpertSource(cfg, 0)
+    x = synth.tokens_bf16(cfg, n_tokens, stream=token_stream)
+    xf = oracle.bf16_to_f64(x)
+    need = set()
+    for t in range(n_tokens):
+        ids, _, _ = oracle.route(oracle.router_logits(xf[t], src.router_w, src.router_b), cfg.k)
+        need.update(int(e) for e in ids)
+    cache = {e: src.expert(e) for e in sorted(need)}       # generated outside the timed region
+    shared = {s: src.shared(s) for s in range(cfg.n_shared)}
+
+    def one(t):
+        oracle.moe_token(cfg.fmt, cfg.k, x[t], src.router_w, src.router_b, cache.__getitem__,
+                         shared.__getitem__, cfg.n_shared)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, range(min(threads, n_tokens))))    # warm the threads and the code
+        t0 = time.perf_counter()
+        list(ex.map(one, range(n_tokens)))
+        dt = time.perf_counter() - t0
+    return {"seconds": dt, "token_layers": n_tokens, "threads": threads}
+
+
+def cpu_baseline(cfg, budget_s: float = 12.0) -> dict:
+    """The oracle's rate on this workload (tok/s over all of its layers), on all host cores, from
+    a bounded sample of about `budget_s` seconds."""
+    cores = host_cores()
+    threads = max(1, min(cores, 64))
+    probe = oracle_sample(cfg, threads, threads, token_stream=7)
+    per_tl = probe["seconds"] / probe["token_layers"]          # seconds per token-layer, all threads busy
+    n = max(threads, min(4096, int(budget_s / max(per_tl, 1e-6)) // threads * threads))
+    s = oracle_sample(cfg, n, threads, token_stream=11)
+    rate_tl = s["token_layers"] / s["seconds"]
+    return {"value": rate_tl / cfg.L, "unit": "tok/s", "cores": threads, "host_cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} tokens through one layer of {cfg.name} ({threads} at a time, one per host "
+                      f"thread), {s['seconds']:.1f} s; tok/s over the workload's {cfg.L} layer(s) = "
+                      f"token-layers per second / {cfg.L} (the oracle's cost is the same for every "
+                      "token and layer)"}
 
 
 def run_reference(args, cfg) -> dict:
-    layers = args.ref_layers
+    """The reference arm: the oracle as it stands, on the host cores; each step is a bounded sample
+    (one token per host thread through one layer), timed as a whole."""
+    cores = host_cores()
+    threads = max(1, min(cores, 64))
     times = []
     for s in range(args.warmup + args.steps):
-        dt = oracle_decode_sample(cfg, layers, token_stream=1000 + s)
+        r = oracle_sample(cfg, threads, threads, token_stream=1000 + 97 * s)
         if s >= args.warmup:
-            times.append(dt)
-    per_token = statistics.mean(times) * cfg.L / layers
-    value = 1.0 / per_token
-    sample = f"1 token through {layers} of {cfg.L} layers per step, time scaled x{cfg.L / layers:g}"
+            times.append(r["seconds"])
+    step_s = statistics.mean(times)
+    value = threads / (step_s * cfg.L)
+    sample = (f"each step: {threads} tokens through one layer of {cfg.name}, one per host thread; "
+              f"tok/s = tokens / (step time x {cfg.L} layers)")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": {"workload": cfg.name},
-        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": threads, "host_cores": cores,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -201,35 +255,65 @@ def run_reference(args, cfg) -> dict:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def timed_stack(sess, cfg, xs, r_out, steps, warmup, stream, dist_on):
-    from quantized_expert_ffn_token_b200 import capi
-    T = cfg.T
+def _step(capi, sess, cfg, x, out, stream):
+    if cfg.L > 1:
+        capi.moe_forward_stack(sess.ctx, 0, cfg.L, x, cfg.T, out, None, stream)
+    else:
+        capi.moe_forward(sess.ctx, 0, x, cfg.T, out, None, None, None, stream)
+
+
+def timed_steps(capi, sess, cfg, xs, out, steps, warmup, stream, dist_on, flush=None):
+    """W untimed steps, then K timed ones between a barrier and a device sync on both sides; CUDA
+    events on the launching stream around each step (an L2 flush, when given, runs before each
+    step outside its events).  Returns (ms of the K steps, the library's timing record)."""
     for s in range(warmup):
-        capi.moe_forward_stack(sess.ctx, 0, cfg.L, xs[s % len(xs)], T, r_out, None, stream)
+        _step(capi, sess, cfg, xs[s % len(xs)], out, stream)
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     capi.moe_timing_read(sess.ctx)                     # reset counters
     capi.moe_timing_enable(sess.ctx, True)
-    start = torch.cuda.Event(enable_timing=True)
-    stop = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
+    evs = []
     for s in range(steps):
-        capi.moe_forward_stack(sess.ctx, 0, cfg.L, xs[(warmup + s) % len(xs)], T, r_out, None, stream)
-    stop.record(stream)
+        if flush is not None:
+            with torch.cuda.stream(stream):
+                flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        _step(capi, sess, cfg, xs[(warmup + s) % len(xs)], out, stream)
+        b.record(stream)
+        evs.append((a, b))
     torch.cuda.synchronize()
     tim = capi.moe_timing_read(sess.ctx)
     capi.moe_timing_enable(sess.ctx, False)
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    return start.elapsed_time(stop), tim
+    return sum(a.elapsed_time(b) for a, b in evs), tim
 
 
-def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
+def layer_unions(capi, sess, cfg, x, dev) -> list[int]:
+    """Distinct routed experts per layer of one step (the bytes a pass must stream)."""
+    L, T, k = cfg.L, cfg.T, cfg.k
+    if T == 1:
+        return [k] * L
+    idr = torch.empty((L, T, k), dtype=torch.int32, device=dev)
+    if L > 1:
+        r = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+        capi.moe_forward_stack(sess.ctx, 0, L, x, T, r, capi.make_record(ids=idr))
+    else:
+        y = torch.empty((T, cfg.d), dtype=torch.int16, device=dev)
+        capi.moe_forward(sess.ctx, 0, x, T, y, None, idr[0], None)
+    torch.cuda.synchronize()
+    ids = idr.cpu().numpy()
+    return [len(np.unique(ids[l])) for l in range(L)]
+
+
+def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict:
+    """One workload: value (tok/s, device-timed), roofline of the dominant kernel, end-to-end rate
+    through the host-buffer entry point, clocks, launches, and (rank 0) the oracle's rate."""
     from quantized_expert_ffn_token_b200 import capi, session
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.Stream(dev)
     P = peaks()
@@ -237,133 +321,91 @@ def run_ours(args, cfg, rank, world, local_rank, dist_on) -> dict | None:
     with torch.cuda.stream(stream):
         sess.load_synthetic(stream=stream)
     torch.cuda.synchronize()
-    n_tok = args.warmup + args.steps
+    n_in = min(args.warmup + args.steps, 8)
     xs = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).to(dev)
-          for s in range(n_tok)]
-    r_out = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=dev)
+          for s in range(n_in)]
+    if cfg.L > 1:
+        out = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=dev)
+    else:
+        out = torch.empty((cfg.T, cfg.d), dtype=torch.int16, device=dev)
+    unions = layer_unions(capi, sess, cfg, xs[0], dev)
+    step_bytes = sum((u + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg) for u in unions)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if step_bytes < (1 << 30) else None
 
     with Clocks(local_rank) as clk:
-        ms, tim = timed_stack(sess, cfg, xs, r_out, args.steps, args.warmup, stream, dist_on)
+        ms, tim = timed_steps(capi, sess, cfg, xs, out, args.steps, args.warmup, stream, dist_on, flush)
     clocks = clk.summary()
-    ms_max = max_over_ranks(ms, dist_on, dev)
-    ms_step = ms_max / args.steps
+    ms_step = max_over_ranks(ms, dist_on, dev) / args.steps
     value = whole_job_rate(cfg.T, world, ms_step / 1e3)
-
-    # roofline of the dominant (timed) kernel: the bytes it must stream per launch.  The
-    # single-token kernel runs one token through the whole stack per launch: k routed + the
-    # shared experts and the router rows of every layer; the grouped paths launch once per
-    # layer and stream the union of the batch's experts
-    union = cfg.k if cfg.T == 1 else measured_union(sess, cfg, xs[0], dev)
-    if tim["kernel"] == "k_decode":
-        alg_bytes = cfg.L * ((cfg.k + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+    kernel = tim["kernel"]
+    launches = max(1, tim["timed_launches"])
+    avg_ms = tim["ms"] / launches
+    tensor_bound = cfg.T >= 9 and kernel.startswith("k_cache_fill")
+    if tensor_bound:
+        # the expert GEMMs (decoded-weight cache fill + gate/up + down) of one layer per timed region
+        flops = expert_flops(cfg, cfg.T)
+        burst = cfg.L == 1            # one ~1 ms call timed alone: burst peak; a long step: sustained
+        peak = P["bf16_tflops"] if burst else P["bf16_tflops_sustained"]
+        achieved = flops / (avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": measured_traffic(kernel, cfg.name, 1),
+                "kernel": kernel, "alg_flops_per_launch": flops, "avg_launch_ms": avg_ms,
+                "peak_source": f"{P['source']} ({'bf16_tflops, burst' if burst else 'bf16_tflops_sustained'}); "
+                               "fp16 dense MMA rate = bf16's"}
+        step_flops = cfg.L * (expert_flops(cfg, cfg.T) + router_flops(cfg, cfg.T))
+        step_roof = {"alg_flops_per_step": step_flops,
+                     "achieved_tflops": step_flops / (ms_step / 1e3) / 1e12,
+                     "frac": step_flops / (ms_step / 1e3) / 1e12 / peak}
     else:
-        alg_bytes = (union + cfg.n_shared) * expert_bytes(cfg)   # experts only
-    # the step's algorithmic bytes: every layer's router rows and the union of the experts the
-    # batch's tokens chose (a path that streams some of them more than once moves more)
-    step_bytes = cfg.L * ((union + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
-    avg_ms = tim["ms"] / max(1, tim["timed_launches"])
-    achieved = alg_bytes / (avg_ms / 1e3) / 1e9
-    roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / P["hbm_gbs"], "traffic": decode_traffic(cfg, tim["kernel"]), "kernel": tim["kernel"],
-            "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": avg_ms,
-            "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
+        # the single-token kernel: one launch = one token through every layer of the call
+        layers_per_launch = cfg.L
+        alg = layers_per_launch * ((cfg.k + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+        achieved = alg / (avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / P["hbm_gbs"], "traffic": measured_traffic(kernel, cfg.name, layers_per_launch),
+                "kernel": kernel, "alg_bytes_per_launch": alg, "avg_launch_ms": avg_ms,
+                "launches_per_step": launches / args.steps,
+                "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
+        step_roof = {"alg_bytes_per_step": step_bytes, "experts_streamed_per_layer": statistics.mean(unions),
+                     "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                     "frac": step_bytes / (ms_step / 1e3) / 1e9 / P["hbm_gbs"]}
 
-    # end to end through the public host-buffer entry point
+    # end to end through the public host-buffer entry point (copies inside the timed region)
     x_host = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).pin_memory()
-              for s in range(n_tok)]
+              for s in range(min(n_in, 4))]
     r_host = torch.empty((cfg.T, cfg.d), dtype=torch.float32).pin_memory()
-    for s in range(args.warmup):
-        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[s], cfg.T, r_host, stream)
+    for s in range(max(1, args.warmup)):
+        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[s % len(x_host)], cfg.T, r_host, stream)
     if dist_on:
         torch.distributed.barrier()
     t0 = time.perf_counter()
     for s in range(args.steps):
-        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[args.warmup + s], cfg.T, r_host, stream)
+        capi.moe_forward_stack_host(sess.ctx, 0, cfg.L, x_host[s % len(x_host)], cfg.T, r_host, stream)
     e2e_s = max_over_ranks(time.perf_counter() - t0, dist_on, dev)
     e2e = {"value": whole_job_rate(cfg.T * args.steps, world, e2e_s), "unit": "tok/s",
            "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
+           "entry_point": "moe_forward_stack_host" + (" (one layer: rmsnorm + layer + residual)" if cfg.L == 1 else ""),
            "timer": "host wall clock around synchronous calls"}
     sess.close()
-    del xs
+    del xs, out, flush
     torch.cuda.empty_cache()
 
-    out = {
-        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp32-accumulate over Q4B32/bf16" if cfg.fmt == "q4" else "fp32-accumulate over Q3B32/bf16",
-        "data": "synthetic (seeded counter-hash weights, N(0,1) bf16 tokens)",
+    fmt = cfg.fmt.upper() + "B32"
+    entry = {
+        "workload": cfg.name, "value": value, "unit": "tok/s", "ms_per_step": ms_step,
         "config": {"workload": f"{cfg.name}: d={cfg.d} E={cfg.E} top-{cfg.k}+{cfg.n_shared} shared "
-                               f"I={cfg.I} {cfg.fmt.upper()}B32 T={cfg.T} layers={cfg.L}",
+                               f"I={cfg.I} {fmt} T={cfg.T} layers={cfg.L}",
                    "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: each step streams {step_bytes / 1e9:.2f} GB of weights (> 126 MB L2) "
-                         "and routes a new token"},
-        "roofline": roof,
-        "step_roofline": {"alg_bytes_per_step": step_bytes,
-                          "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-                          "frac": step_bytes / (ms_step / 1e3) / 1e9 / P["hbm_gbs"]},
-        "e2e": e2e,
-        "gpu_launches": tim["all_launches"],
-        "clocks": clocks,
+                   "l2": (f"{FLUSH_BYTES >> 20} MB flush before each timed step" if flush is not None else
+                          f"no flush: each step streams {step_bytes / 1e9:.2f} GB (> 126 MB L2)")},
+        "dtype": ("fp16 tensor-core MMA, fp32 accumulate, over " if tensor_bound else
+                  "exact code operands, fp32 accumulate, over ") + fmt + " weights / bf16 activations",
+        "roofline": roof, "step_roofline": step_roof, "e2e": e2e,
+        "gpu_launches": tim["all_launches"], "clocks": clocks,
     }
-    return out
-
-
-def measured_union(sess, cfg, x, dev) -> int:
-    """Mean number of distinct routed experts per layer for one step (T > 1)."""
-    from quantized_expert_ffn_token_b200 import capi
-    L, T, k = cfg.L, cfg.T, cfg.k
-    idr = torch.empty((L, T, k), dtype=torch.int32, device=dev)
-    rec = capi.make_record(ids=idr)
-    r = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
-    capi.moe_forward_stack(sess.ctx, 0, L, x, T, r, rec)
-    torch.cuda.synchronize()
-    ids = idr.cpu().numpy()
-    return int(round(np.mean([len(np.unique(ids[l])) for l in range(L)])))
-
-
-def secondary_prefill(args, local_rank) -> dict:
-    """Single-layer prefill (4096 tokens, Zipf-biased routing): tok/s and the
-    expert kernels' throughput against the dense tensor peak."""
-    from quantized_expert_ffn_token_b200 import capi, session
-    cfg = synth.CONFIGS["prefill_1l_q4_t4096_zipf"]
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(dev)
-    sess = session.Session(cfg, device=local_rank, max_tokens=cfg.T)
-    sess.load_synthetic(stream=stream)
-    x = torch.from_numpy(synth.tokens_bf16(cfg).view(np.int16)).to(dev)
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.int16, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for _ in range(2):
-        capi.moe_forward(sess.ctx, 0, x, cfg.T, y, None, None, None, stream)
-    torch.cuda.synchronize()
-    times = []
-    capi.moe_timing_read(sess.ctx)
-    capi.moe_timing_enable(sess.ctx, True)
-    for _ in range(3):
-        with torch.cuda.stream(stream):
-            flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        capi.moe_forward(sess.ctx, 0, x, cfg.T, y, None, None, None, stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        times.append(a.elapsed_time(b))
-    tim = capi.moe_timing_read(sess.ctx)
-    sess.close()
-    ms = statistics.median(times)
-    flops_expert = 2 * cfg.T * (cfg.k + cfg.n_shared) * 3 * cfg.d * cfg.I
-    flops = flops_expert + 2 * cfg.T * cfg.E * cfg.d
-    P = peaks()
-    kms = tim["ms"] / max(1, tim["timed_launches"])
-    return {"workload": cfg.name, "tok_per_s": cfg.T / (ms / 1e3), "ms_per_layer": ms,
-            "tflops": flops / (ms / 1e3) / 1e12,
-            "roofline": {"bound": "tensor", "kernel": tim["kernel"],
-                         "achieved": flops_expert / (kms / 1e3) / 1e12,
-                         "peak": P["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": flops_expert / (kms / 1e3) / 1e12 / P["bf16_tflops_sustained"],
-                         "traffic": PREFILL_Q4_T4096_TRAFFIC if cfg.name == "prefill_1l_q4_t4096_zipf" else None,
-                         "traffic_kernels": "k_cache_fill + k_tc_gemm<gate/up> + k_tc_gemm<down>"},
-            "l2": "256 MB flush between timed calls"}
+    if with_cpu:
+        entry["cpu_baseline"] = cpu_baseline(cfg)
+    return entry
 
 
 # ---- token-count sweep (python bench.py --sweep): one layer, every path that accepts T ------------
@@ -467,9 +509,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
-    ap.add_argument("--no-secondary", action="store_true")
-    ap.add_argument("--cpu-layers", type=int, default=12, help="oracle sample: layers per token")
-    ap.add_argument("--ref-layers", type=int, default=2, help="reference arm: layers per step")
+    ap.add_argument("--no-secondary", action="store_true", help="time the headline workload only")
+    ap.add_argument("--no-cpu", action="store_true", help="leave out the oracle's CPU baselines")
     ap.add_argument("--layers", type=int, default=None,
                     help="stack depth override (small cases for profiler captures)")
     ap.add_argument("--sweep", action="store_true",
@@ -508,19 +549,27 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                              device_id=torch.device("cuda", local_rank))
-    out = run_ours(args, cfg, rank, world, local_rank, dist_on)
+    torch.cuda.set_device(local_rank)
+    head = measure(args, cfg, rank, world, local_rank, dist_on, with_cpu=(rank == 0 and world == 1
+                                                                        and not args.no_cpu))
     if rank == 0:
-        if not args.no_secondary and world == 1:
-            out["secondary"] = {"prefill": secondary_prefill(args, local_rank)}
-        if world == 1:
-            nt = min(cfg.T, 4)
-            layers = min(args.cpu_layers, cfg.L)
-            sec = oracle_decode_sample(cfg, layers, token_stream=7, n_tokens=nt)
-            v = nt / (sec * cfg.L / layers)
-            out["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": 1, "kind": "oracle",
-                                   "sample": f"{nt} token(s) through {layers} of {cfg.L} layers, "
-                                             f"time scaled x{cfg.L / layers:g}; the oracle's cost is "
-                                             "per token, so tokens/s does not depend on the batch"}
+        out = {
+            "metric": METRIC, "value": head["value"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+            "data": "synthetic (seeded counter-hash weights, N(0,1) bf16 tokens)",
+            "config": head["config"], "roofline": head["roofline"], "step_roofline": head["step_roofline"],
+            "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        }
+        if "cpu_baseline" in head:
+            out["cpu_baseline"] = head["cpu_baseline"]
+        if world == 1 and not args.no_secondary and args.layers is None:
+            out["secondary"] = {}
+            for name in SECONDARY:
+                if name == cfg.name:
+                    continue
+                out["secondary"][name] = measure(args, synth.CONFIGS[name], rank, world, local_rank, dist_on,
+                                                 with_cpu=not args.no_cpu)
         print(json.dumps(out))
     if dist_on:
         torch.distributed.barrier()

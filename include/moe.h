@@ -88,14 +88,17 @@ typedef struct {
     int flags;          /* MOE_FLAG_* bits, 0 for normal use */
 } moe_config;
 
-/* moe_config.flags.  The first two pin a call to one implementation (tests
- * compare the paths with each other); the last is a test hook for the
+/* moe_config.flags: test and diagnostic hooks, 0 in normal use (no page has a
+ * counterpart).  The first two pin a call to one implementation (tests
+ * compare the paths with each other); MOE_FLAG_TRACE records the decode
+ * kernel's phase clocks; MOE_FLAG_TEST_WITHHOLD is a test hook for the
  * bounded device waits: in the context's first single-token call the decode
  * kernel's CTA 0 withholds its router logits, every wait on them runs out
  * after about one second, and the call reports MOE_ERR_DEVICE_TIMEOUT through
  * moe_get_device_error; later calls run normally. */
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* small T runs the general path, not the single-token kernel */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
+#define MOE_FLAG_NO_MULTI_DECODE 8    /* 2..16 tokens run the single-token kernel per token, not the few-token kernel */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
 #define MOE_FLAG_TRACE 4              /* record per-phase timestamps (moe_trace_read) */
 
@@ -132,7 +135,10 @@ typedef struct moe_ctx moe_ctx;
  * one context per concurrent stream. */
 
 /* Create a context on CUDA device `device` and allocate its workspace (sized
- * by max_tokens).  *out receives the handle.  Errors: INVALID_ARG (bad
+ * by max_tokens).  The context holds one stack of MoE layers of one shape (the
+ * pages' model: 48 layers of 512 experts, 10 routed + 1 shared per token;
+ * "Qwen3.8-Flash-Next at 45 Tokens/sec on a 12GB GPU?", video transcript
+ * 1:37-2:16).  *out receives the handle.  Errors: INVALID_ARG (bad
  * config), UNSUPPORTED (shape outside the limits above), OOM, CUDA.
  * When the tensor-core path can run, the workspace also holds a decoded-weight
  * cache of min(experts, max_tokens * (top_k + n_shared) / 256) experts
@@ -141,13 +147,20 @@ typedef struct moe_ctx moe_ctx;
 MOE_API int moe_create(const moe_config *cfg, int device, moe_ctx **out);
 
 /* Copy one layer's weights into the context (repacking them on the device)
- * and make the layer usable.  Reloading a layer replaces it.  Work is queued
+ * and make the layer usable.  The weights are the block formats above (the
+ * pages name their quantised types, e.g. IQ3_S or Q2_0, but give no layout:
+ * "Running Qwen3.8-Flash-Next on a 4090 24GB", section "The engine rejects
+ * Unsloth's embedding format"; this library's formats fix one).  Reloading a layer replaces it.  Work is queued
  * on `stream` (a cudaStream_t, NULL = default stream); the call returns after
  * the copies from caller memory have completed.  Errors: INVALID_ARG, OOM,
  * CUDA. */
 MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, void *stream);
 
-/* One layer on T tokens.  All pointers are device memory:
+/* One layer on T tokens: router, softmax top-k, the chosen experts and the
+ * shared expert, weighted combine ("Qwen3.8-Flash-Next at 45 Tokens/sec on a
+ * 12GB GPU?", video transcript 1:50-2:16 and 3:36-3:47; "Qwen3.8-Flash-Next on
+ * RTX 5090 + 64GB", section "The 30-Second Overview").  All pointers are
+ * device memory:
  *   x_bf16 [T][d] input; y_bf16 [T][d] output; y_f32 [T][d] the fp32 value
  *   before the bf16 rounding, or NULL; ids [T][k] chosen experts (descending
  *   weight) and w [T][k] their weights, either may be NULL.
@@ -162,7 +175,10 @@ MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
                 uint16_t *y_bf16, float *y_f32, int32_t *ids, float *w,
                 void *stream);
 
-/* Layers [layer0, layer0 + n_layers) stacked with a residual stream:
+/* Layers [layer0, layer0 + n_layers) stacked with a residual stream (the
+ * pages' 48 stacked layers, video transcript 1:37-1:50 of "Qwen3.8-Flash-Next
+ * at 45 Tokens/sec on a 12GB GPU?"; the normalisation between them is this
+ * library's reading, below):
  *   r_0 = x (bf16 input, widened to fp32)
  *   x_l = bf16(rmsnorm(r_l)),  rmsnorm(r) = r / sqrt(mean(r^2) + 1e-6)
  *   r_{l+1} = r_l + float(moe_l(x_l))
@@ -176,12 +192,17 @@ MOE_API int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint
 
 /* moe_forward_stack with HOST buffers: copies x_bf16 (host, pinned or
  * pageable) to the device, runs the stack and copies resid_out back to the
- * host; returns after the result is in host memory. */
+ * host; returns after the result is in host memory.  (The pages' engine takes
+ * tokens from a host program; this is the same layer stack behind a call that
+ * owns the copies.)  Errors as moe_forward_stack. */
 MOE_API int moe_forward_stack_host(moe_ctx *ctx, int layer0, int n_layers,
                            const uint16_t *x_bf16_host, int T, float *resid_out_host,
                            void *stream);
 
-/* Free every device allocation of the context.  NULL is accepted.  A handle
+/* Library plumbing without a counterpart in the pages: teardown, error
+ * reporting, measurement and tracing.
+ *
+ * Free every device allocation of the context.  NULL is accepted.  A handle
  * must not be used after this call. */
 MOE_API int moe_destroy(moe_ctx *ctx);
 

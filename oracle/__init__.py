@@ -348,7 +348,13 @@ def moe_rows_dense(fmt, k, x_bf16, router_w, router_b, get_expert, get_shared, n
         rows, slots = np.nonzero(ids == e)
         return e, rows, slots, apply(get_expert(e), x[rows])
 
-    with ThreadPoolExecutor(max_workers=threads or min(16, os.cpu_count() or 1)) as ex:
+    try:   # one BLAS thread per worker: the workers already use every core
+        from threadpoolctl import threadpool_limits
+        blas = threadpool_limits(1)
+    except ImportError:
+        import contextlib
+        blas = contextlib.nullcontext()
+    with blas, ThreadPoolExecutor(max_workers=threads or min(32, os.cpu_count() or 1)) as ex:
         res = list(ex.map(routed, experts))
         shared = list(ex.map(lambda s: apply(get_shared(s), x), range(n_shared)))
     contrib = [[] for _ in range(n)]   # (slot j, y_e row) per token

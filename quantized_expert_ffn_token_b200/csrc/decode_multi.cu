@@ -1,0 +1,1068 @@
+// Few-token decode (2..8 tokens per launch): one persistent kernel runs whole
+// layers (and the whole 48-layer stack) for a small batch of tokens, reading
+// the union of the batch's experts once per layer.  This is the step that
+// checks several guessed tokens at once ("Strata: Qwen3.8-Flash-Next (125B
+// Moe) on a 8GB+ Nvidia GPU", README section "How does it work": guess, then
+// check all the guesses in one go; "Running Qwen3.8-Flash-Next on a 4090
+// 24GB", the --spec 4 setting).  Routing and combine follow "Qwen3.8-Flash-
+// Next at 45 Tokens/sec on a 12GB GPU?" (video transcript 1:50-2:16,
+// 3:36-3:47); the expert network and block formats are include/moe.h's.
+//
+// One CTA per SM (cooperative launch), 12 compute warps and one producer warp
+// that issues every bulk copy into a ring of shared-memory slots.  Per layer:
+//   1. input: every CTA rebuilds all T token rows (stack: residual + rmsnorm,
+//      the residual stream living in global memory, each CTA owning a slice);
+//   2. router: CTA c owns experts c, c+G, ...; a warp computes whole
+//      (expert, token) dot products from router rows prefetched into shared
+//      memory during the previous layer; logits are exchanged (counter 0);
+//   3. every CTA selects each token's top-k (a warp per token), forms the
+//      sorted union U of the chosen experts (+ the shared expert) and the
+//      weight table w[u][t];
+//   4. gate/up: units (u, 16-row tile) round-robin over the CTAs in u-major
+//      order; the tokens sit in the MMA's B columns (column t = token t), the
+//      codes become exact fp16/bf16 operands (as in the single-token kernel)
+//      and each 32-block's partial is flushed with its scale and the offset
+//      term in fp32; the warps' k chunks meet in shared-memory sums, and the
+//      last warp of a unit applies SwiGLU, stores h and adds one arrival to
+//      that expert's h counter;
+//   5. down: units (u, 16-row output tile) in u-major order, a contiguous run
+//      per CTA (so a CTA touches two or three experts); once those experts' h
+//      counters are complete, h enters as hi + lo parts in B-fragment order;
+//      each unit's weighted 16 x T output is added to the layer's fp32 output
+//      buffer with vector atomics; a y counter closes the layer.
+// Every wait is bounded (clock64); on timeout the kernel sets the context's
+// error word and every CTA leaves.  The host zeroes the counters and the
+// output buffers before each launch.
+#include <string.h>
+
+#include "decode_common.cuh"
+
+namespace qeffn {
+
+namespace {
+
+using namespace dec;
+
+constexpr int TMAX = 8;         // tokens per launch: the eight B columns of mma.m16n8k16
+constexpr int KMAX = 32;        // top_k limit
+constexpr int EPL = 32;         // logits per lane in the top-k (E <= 1024)
+constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
+
+struct MiscM {
+    unsigned long long full[MAX_SLOTS];
+    unsigned long long empty[MAX_SLOTS];   // one arrival per consumed item
+    unsigned long long rbar;
+    unsigned long long route;              // one arrival per layer: routing known
+    int gcnt[MAX_SLOTS];                   // gate/up warps done with the unit in slot s
+    int nU;                                // experts in use this layer (routed union + shared)
+    int nR;                                // routed part of the union
+    int ids[TMAX][KMAX];
+    float w[TMAX][KMAX];
+    unsigned bits[32];                     // union bitmap over E <= 1024
+    float xinv[TMAX];                      // 2^-s of a token's fp16 operand (1 for bf16 operands)
+    float xscale[TMAX];                    // 2^s
+    float ss[NW][TMAX];                    // per-warp sums of squares / maxima of the input phase
+    float mx[NW][TMAX];
+};
+
+struct MultiParams {
+    const LayerPtrs *layers;
+    int layer0, L;
+    int d, E, I, k, nsh, T, TM;    // T tokens of this launch, TM the carve's token capacity
+    MatLayout gu, dn;
+    int stack;
+    const uint16_t *x_in;          // bf16 [T][d]
+    float *resid_out;              // stack: [T][d]
+    uint16_t *y_out;               // single layer: bf16 [T][d]
+    float *yf_out;                 // single layer: fp32 [T][d] or NULL
+    int32_t *ids_out;              // single layer: [T][k] or NULL
+    float *w_out;                  // single layer: [T][k] or NULL
+    moe_stack_record rec;          // records: token t is record row rec_r0 + t of rec_n
+    int rec_on, rec_n, rec_r0;
+    unsigned *cnt;                 // [0] logits arrivals, [32] y arrivals, [64 + 8u] h arrivals of union slot u
+    float *x_logits;               // [TM][E]
+    float *x_h;                    // [UM][TM][I]
+    float *y_acc;                  // [2][TM][d] layer outputs, accumulated with atomics
+    float *r_buf;                  // [2][TM][d] residual stream (stack)
+    int *err;
+    int withhold;
+    int nslot, slot_bytes, rpc, span, UM;
+    int off_ring, off_router, off_xb, off_red, off_xsum, off_hsum, off_uexp, off_hcum, off_wtab,
+        off_misc, off_ltab;
+};
+
+constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;
+__device__ __forceinline__ unsigned *hctr(const MultiParams &p, int u) { return p.cnt + C_H + 8 * u; }
+
+__device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+__device__ __forceinline__ uint16_t f2h_bits(float v) {
+    __half h = __float2half_rn(v);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+__device__ __forceinline__ float h_bits_f(uint16_t b) {
+    return __half2float(*reinterpret_cast<const __half *>(&b));
+}
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// The 16 A-fragment registers of one lane's piece of a k group (four k16 slices).
+template <int FMT>
+__device__ __forceinline__ void frag16(const uint8_t *piece, uint32_t r[16]) {
+    if constexpr (FMT == MOE_Q2B32) {
+        q2_frag_h(*reinterpret_cast<const uint2 *>(piece), r);
+    } else if constexpr (FMT == MOE_Q4B32) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(piece);
+        const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) q4_frag_h(wv[m], r[4 * m], r[4 * m + 1], r[4 * m + 2], r[4 * m + 3]);
+    } else {
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(piece);
+        q3_frag(wp[0], wp[1], wp[2], r);
+    }
+}
+template <int FMT>
+__device__ __forceinline__ void mma_fmt(float *d, const uint32_t *a, uint32_t b0, uint32_t b1) {
+    if constexpr (FMT == MOE_Q3B32) mma16816(d, a[0], a[1], a[2], a[3], b0, b1);
+    else mma16816_h(d, a[0], a[1], a[2], a[3], b0, b1);
+}
+template <int FMT>
+constexpr int piece_bytes() { return FMT == MOE_Q4B32 ? 16 : FMT == MOE_Q2B32 ? 8 : 12; }
+
+// Flush one 32-block's MMA partial D (rows g, g+8 x columns 2c, 2c+1) into acc:
+// acc += s_row * (D * mult_row - off_row * vsum_col), where the codes were read
+// as 1024 + F q (fp16) or 128 + q (bf16) and vsum is the block sum of the
+// column's B operand.  `second` = the k group's second block (Q2B32 only).
+template <int FMT>
+__device__ __forceinline__ void flush_block(float *acc, const float *D, float sg, float s8, float v0, float v1,
+                                            bool second) {
+    float mg, m8, og, o8;
+    if constexpr (FMT == MOE_Q4B32) {
+        mg = 1.f; og = 1032.f; m8 = 0.0625f; o8 = 72.f;
+    } else if constexpr (FMT == MOE_Q2B32) {
+        if (!second) { mg = 1.f; og = 1026.f; m8 = 0.25f; o8 = 258.f; }
+        else { mg = 0.0625f; og = 66.f; m8 = 0.015625f; o8 = 18.f; }
+    } else {
+        mg = 1.f; og = 132.f; m8 = 1.f; o8 = 132.f;
+    }
+    acc[0] = fmaf(sg, fmaf(D[0], mg, -og * v0), acc[0]);
+    acc[1] = fmaf(sg, fmaf(D[1], mg, -og * v1), acc[1]);
+    acc[2] = fmaf(s8, fmaf(D[2], m8, -o8 * v0), acc[2]);
+    acc[3] = fmaf(s8, fmaf(D[3], m8, -o8 * v1), acc[3]);
+}
+
+// Position of the 16-byte B fragment of (expert-in-span su, k group kg, slice m,
+// lane) in the down phase's h table: [su][kg][m][lane] x 16 bytes, so that one
+// warp instruction reads 512 contiguous bytes.
+__device__ __forceinline__ int hfrag_off(int su, int nkg, int kg, int m, int lane) {
+    return (((su * nkg + kg) * 4 + m) * 32 + lane) * 16;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *ring = smem + p.off_ring;
+    float *rtr = reinterpret_cast<float *>(smem + p.off_router);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_xb);     // [TM][d] bf16 input; then the h table
+    uint8_t *htab = smem + p.off_xb;
+    float *red = reinterpret_cast<float *>(smem + p.off_red);         // [nslot][16][TM]
+    float *xsum = reinterpret_cast<float *>(smem + p.off_xsum);       // [TM][d/32]
+    float *hsum = reinterpret_cast<float *>(smem + p.off_hsum);       // [span][TM][I/32], then hinv
+    int *uexp = reinterpret_cast<int *>(smem + p.off_uexp);           // [UM]
+    unsigned *hcum = reinterpret_cast<unsigned *>(smem + p.off_hcum); // [UM]
+    float *wtab = reinterpret_cast<float *>(smem + p.off_wtab);       // [UM][TM]
+    MiscM *ms = reinterpret_cast<MiscM *>(smem + p.off_misc);
+    LayerPtrs *ltab = reinterpret_cast<LayerPtrs *>(smem + p.off_ltab);
+
+    constexpr bool F16OP = (FMT != MOE_Q3B32);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const int d = p.d, E = p.E, I = p.I, k = p.k, T = p.T, TM = p.TM;
+    const int nbd = d / 32, nbi = I / 32, nkgi = I / 64;
+    const int ntile_gu = I / 8, ntile_dn = d / 16;
+    const int GW = d / 256;                          // warps with a gate/up k chunk
+    const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
+    const int d4 = d / 4;
+    const int own_lo = cta * d4 / G, own_hi = (cta + 1) * d4 / G;   // float4 columns this CTA owns
+    float *hinv = hsum + p.span * TM * nbi;
+    int *err = p.err;
+
+    if (tid == 0) {
+        for (int s = 0; s < p.nslot; ++s) {
+            mbar_init(&ms->full[s], 1);
+            mbar_init(&ms->empty[s], 1);
+            ms->gcnt[s] = 0;
+        }
+        mbar_init(&ms->rbar, 1);
+        mbar_init(&ms->route, 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < p.nslot * 16 * TM; i += NTT) red[i] = 0.f;
+    for (int i = tid; i < 32; i += NTT) ms->bits[i] = 0u;
+    for (int i = tid; i < p.UM; i += NTT) hcum[i] = 0u;
+    for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];
+    __syncthreads();
+
+    // this CTA's work in a layer with nU experts in use
+    struct Split {
+        int n_gu, dn_lo, dn_hi, n_dn, n_dn_items, n_items;
+    };
+    auto split = [&](int nU) {
+        Split sp;
+        const int n_gu_all = nU * ntile_gu;
+        sp.n_gu = (cta < n_gu_all) ? (n_gu_all - cta + G - 1) / G : 0;   // units cta, cta + G, ...
+        const int n_dn_all = nU * ntile_dn;
+        sp.dn_lo = (int)((long long)cta * n_dn_all / G);
+        sp.dn_hi = (int)((long long)(cta + 1) * n_dn_all / G);
+        sp.n_dn = sp.dn_hi - sp.dn_lo;
+        sp.n_dn_items = (sp.n_dn + dn_per_slot - 1) / dn_per_slot;
+        sp.n_items = sp.n_gu + sp.n_dn_items;
+        return sp;
+    };
+    auto ring_slot = [&](int s0, uint32_t p0, int q, uint32_t &par) {
+        int sq = s0 + q;
+        par = p0;
+        while (sq >= p.nslot) {
+            sq -= p.nslot;
+            par ^= 1u;
+        }
+        return sq;
+    };
+
+    // ---- producer warp (lane 0) -----------------------------------------------------------
+    if (warp == NW) {
+        if (lane != 0) return;
+        uint32_t fpar = 0;       // bit s: parity of the fills of slot s so far
+        uint32_t filled = 0;     // bit s: slot s was filled at least once
+        int router_fills = 0;
+        auto issue_router = [&](int li) {
+            const float *rw = ltab[li].rw;
+            int nrows = 0;
+            for (int j = 0; j < p.rpc; ++j)
+                if (cta + G * j < E) ++nrows;
+            fence_proxy_async();
+            mbar_expect_tx(&ms->rbar, (uint32_t)(nrows * d * 4));
+            for (int j = 0; j < nrows; ++j)
+                bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
+            ++router_fills;
+        };
+        issue_router(0);
+        int s_next = 0;
+        for (int l = 0; l < p.L; ++l) {
+            const LayerPtrs Lp = ltab[l];
+            if (!mbar_wait(&ms->route, (uint32_t)(l & 1), err, true)) break;
+            const Split sp = split(ms->nU);
+            bool pok = true;
+            for (int q = 0; q < sp.n_items && pok; ++q) {
+                const int s = s_next;
+                s_next = (s_next + 1 == p.nslot) ? 0 : s_next + 1;
+                if ((filled >> s) & 1u) pok = mbar_wait(&ms->empty[s], ((fpar >> s) & 1u) ^ 1u, err, true);
+                if (!pok) break;
+                fence_proxy_async();
+                uint8_t *dst = ring + (size_t)s * p.slot_bytes;
+                if (q < sp.n_gu) {
+                    const int n = cta + G * q;
+                    const int u = n / ntile_gu, t = n - u * ntile_gu;
+                    const uint8_t *src = Lp.gu + (size_t)uexp[u] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
+                    mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
+                    bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
+                } else {
+                    const int q0 = (q - sp.n_gu) * dn_per_slot;
+                    const int cnt = min(dn_per_slot, sp.n_dn - q0);
+                    mbar_expect_tx(&ms->full[s], (uint32_t)(cnt * p.dn.tile_bytes));
+                    for (int i = 0; i < cnt; ++i) {
+                        const int n = sp.dn_lo + q0 + i;
+                        const int u = n / ntile_dn, j = n - u * ntile_dn;
+                        const uint8_t *src = Lp.dn + (size_t)uexp[u] * p.dn.expert_bytes + (size_t)j * p.dn.tile_bytes;
+                        bulk_g2s(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s]);
+                    }
+                }
+                fpar ^= 1u << s;
+                filled |= 1u << s;
+            }
+            if (!pok) break;
+            if (l + 1 < p.L) issue_router(l + 1);
+        }
+        // every copy has landed before the CTA's shared memory goes away
+        for (int s = 0; s < p.nslot; ++s)
+            if ((filled >> s) & 1u) mbar_wait(&ms->full[s], ((fpar >> s) & 1u) ^ 1u, err, false);
+        if (router_fills > 0) mbar_wait(&ms->rbar, (uint32_t)((router_fills - 1) & 1), err, false);
+        return;
+    }
+
+    int ring_s0 = 0;
+    uint32_t ring_p0 = 0;
+    bool ok = true;
+    bool aborted = false;
+
+    for (int l = 0; l < p.L; ++l) {
+        const LayerPtrs Lp = ltab[l];
+        const int yb = l & 1;                      // output buffer of this layer
+        float *yacc = p.y_acc + (size_t)yb * TM * d;
+
+        // ---- 1. layer input: xb[t] (bf16) for every token; per-token max |x| -------------------
+        float amx[TMAX];
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) amx[t] = 0.f;
+        if (p.stack) {
+            float ssq[TMAX];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) ssq[t] = 0.f;
+            if (l > 0) {
+                if (tid == 0) ok = ctr_wait(p.cnt + C_Y, (unsigned)(G * l), err);
+                if (cta_failed(ok)) {
+                    aborted = true;
+                    break;
+                }
+            }
+            const float *rprev = p.r_buf + (size_t)((l + 1) & 1) * TM * d;
+            const float *yprev = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
+            float *rcur = p.r_buf + (size_t)yb * TM * d;
+            // pass 1: r = r_prev + bf16(y_prev) (layer 0: r = x), sums of squares and max |r|; the
+            // owned columns of r are stored for the next layer
+            for (int i4 = tid; i4 < d4; i4 += NT) {
+                const bool own = i4 >= own_lo && i4 < own_hi;
+#pragma unroll
+                for (int t = 0; t < TMAX; ++t) {
+                    if (t >= T) break;
+                    float4 r;
+                    if (l == 0) {
+                        const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
+                        r = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16), bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
+                    } else {
+                        const float4 a = ld_gpu4(rprev + (size_t)t * d + 4 * i4);
+                        const float4 y = ld_gpu4(yprev + (size_t)t * d + 4 * i4);
+                        const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
+                                       b3 = bf16_rn_bits(y.w);
+                        r = make_float4(a.x + bf16_bits_f(b0), a.y + bf16_bits_f(b1), a.z + bf16_bits_f(b2),
+                                        a.w + bf16_bits_f(b3));
+                        if (own && p.rec_on) {
+                            const size_t ro = ((size_t)(l - 1) * p.rec_n + p.rec_r0 + t) * d + 4 * i4;
+                            if (p.rec.y_bf16)
+                                *reinterpret_cast<uint2 *>(p.rec.y_bf16 + ro) =
+                                    make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+                            if (p.rec.y_f32) *reinterpret_cast<float4 *>(p.rec.y_f32 + ro) = y;
+                        }
+                    }
+                    if (own) *reinterpret_cast<float4 *>(rcur + (size_t)t * d + 4 * i4) = r;
+                    ssq[t] = fmaf(r.x, r.x, fmaf(r.y, r.y, fmaf(r.z, r.z, fmaf(r.w, r.w, ssq[t]))));
+                    amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(r.x), fabsf(r.y)), fmaxf(fabsf(r.z), fabsf(r.w))));
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                float a = ssq[t], m = amx[t];
+                for (int o = 16; o; o >>= 1) {
+                    a += __shfl_xor_sync(0xffffffffu, a, o);
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                }
+                if (lane == 0) {
+                    ms->ss[warp][t] = a;
+                    ms->mx[warp][t] = m;
+                }
+            }
+            csync();
+            float inv[TMAX];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                float a = 0.f, m = 0.f;
+                for (int w = 0; w < NW; ++w) {
+                    a += ms->ss[w][t];
+                    m = fmaxf(m, ms->mx[w][t]);
+                }
+                inv[t] = 1.f / sqrtf(a / (float)d + 1e-6f);
+                amx[t] = bf16_bits_f(bf16_rn_bits(m * inv[t]));   // = max |bf16(r * inv)|
+            }
+            // pass 2: x = bf16(r * inv) (r recomputed from the same loads)
+            for (int i4 = tid; i4 < d4; i4 += NT) {
+                const bool own = i4 >= own_lo && i4 < own_hi;
+#pragma unroll
+                for (int t = 0; t < TMAX; ++t) {
+                    if (t >= T) break;
+                    float4 r;
+                    if (l == 0) {
+                        const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
+                        r = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16), bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
+                    } else {
+                        const float4 a = ld_gpu4(rprev + (size_t)t * d + 4 * i4);
+                        const float4 y = ld_gpu4(yprev + (size_t)t * d + 4 * i4);
+                        r = make_float4(a.x + bf16_bits_f(bf16_rn_bits(y.x)), a.y + bf16_bits_f(bf16_rn_bits(y.y)),
+                                        a.z + bf16_bits_f(bf16_rn_bits(y.z)), a.w + bf16_bits_f(bf16_rn_bits(y.w)));
+                    }
+                    const uint2 xv = make_uint2(
+                        (uint32_t)bf16_rn_bits(r.x * inv[t]) | ((uint32_t)bf16_rn_bits(r.y * inv[t]) << 16),
+                        (uint32_t)bf16_rn_bits(r.z * inv[t]) | ((uint32_t)bf16_rn_bits(r.w * inv[t]) << 16));
+                    *reinterpret_cast<uint2 *>(xb + (size_t)t * d + 4 * i4) = xv;
+                    if (own && p.rec_on && p.rec.x_bf16)
+                        *reinterpret_cast<uint2 *>(p.rec.x_bf16 + ((size_t)l * p.rec_n + p.rec_r0 + t) * d + 4 * i4) = xv;
+                }
+            }
+        } else {
+            for (int i4 = tid; i4 < d4; i4 += NT) {
+#pragma unroll
+                for (int t = 0; t < TMAX; ++t) {
+                    if (t >= T) break;
+                    const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
+                    *reinterpret_cast<uint2 *>(xb + (size_t)t * d + 4 * i4) = xv;
+                    amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(bf16f(xv.x & 0xFFFFu)), fabsf(bf16f(xv.x >> 16))),
+                                                 fmaxf(fabsf(bf16f(xv.y & 0xFFFFu)), fabsf(bf16f(xv.y >> 16)))));
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                float m = amx[t];
+                for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) ms->mx[warp][t] = m;
+            }
+            csync();
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                float m = 0.f;
+                for (int w = 0; w < NW; ++w) m = fmaxf(m, ms->mx[w][t]);
+                amx[t] = m;
+            }
+        }
+        // fp16 operand scale of every token: 2^s with max |x| * 2^s < 2^15 (exact for bf16 inputs)
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+            if (t == tid) {
+                int xe;
+                frexpf(amx[t], &xe);
+                const int s = min(15 - xe, 100);
+                ms->xscale[t] = F16OP ? pow2i(s) : 1.f;
+                ms->xinv[t] = F16OP ? pow2i(-s) : 1.f;
+            }
+        }
+        csync();   // xb complete, operand scales known
+        // block sums of the B operand the gate/up MMAs see (fp16 of x * 2^s, or bf16 x)
+        for (int i = tid; i < T * nbd; i += NT) {
+            const int t = i / nbd, b = i - t * nbd;
+            const uint16_t *src = xb + (size_t)t * d + 32 * b;
+            float acc = 0.f;
+            if constexpr (F16OP) {
+                const float sc = ms->xscale[t];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc += h_bits_f(f2h_bits(bf16_bits_f(src[j]) * sc));
+            } else {
+                acc = sum32_bf16(src);
+            }
+            xsum[t * nbd + b] = acc;
+        }
+
+        // ---- 2. router: warp w computes the (row, token) pairs w, w + NW, ... ----------------------
+        {
+            int nrows = 0;
+            for (int j = 0; j < p.rpc; ++j)
+                if (cta + G * j < E) ++nrows;
+            ok = mbar_wait(&ms->rbar, (uint32_t)(l & 1), err, true);
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
+            for (int pr = warp; pr < nrows * T; pr += NW) {
+                const int j = pr / T, t = pr - j * T;
+                const float *wr = rtr + (size_t)j * d;
+                const uint16_t *xr = xb + (size_t)t * d;
+                float acc = 0.f;
+                for (int i4 = lane; i4 < d4; i4 += 32) {
+                    const float4 wv = *reinterpret_cast<const float4 *>(wr + 4 * i4);
+                    const uint2 xv = *reinterpret_cast<const uint2 *>(xr + 4 * i4);
+                    acc = fmaf(wv.x, bf16f(xv.x & 0xFFFFu), acc);
+                    acc = fmaf(wv.y, bf16f(xv.x >> 16), acc);
+                    acc = fmaf(wv.z, bf16f(xv.y & 0xFFFFu), acc);
+                    acc = fmaf(wv.w, bf16f(xv.y >> 16), acc);
+                }
+                for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                const int e = cta + G * j;
+                if (lane == 0) p.x_logits[(size_t)t * E + e] = acc + __ldg(Lp.rb + e);
+            }
+        }
+        csync();   // this CTA's logits are stored; the router rows are no longer read
+        if (tid == 0) {
+            if (!(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
+            ok = ctr_wait(p.cnt + C_LOGITS, (unsigned)(G * (l + 1)), err);
+        }
+        if (cta_failed(ok)) {
+            aborted = true;
+            break;
+        }
+        // every CTA has read the previous layer's output: clear the owned columns of its buffer,
+        // which accumulates the next layer's output
+        if (l >= 1 && l + 1 < p.L) {
+            float *ynext = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
+            for (int i = tid; i < T * (own_hi - own_lo); i += NT) {
+                const int t = i / (own_hi - own_lo), i4 = own_lo + i - t * (own_hi - own_lo);
+                *reinterpret_cast<float4 *>(ynext + (size_t)t * d + 4 * i4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+
+        // ---- 3. top-k per token (warp t), union, weights --------------------------------------------
+        if (warp < T) {
+            const int t = warp;
+            float v[EPL];
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = lane + 32 * i;
+                float x = (e < E) ? ld_gpu(p.x_logits + (size_t)t * E + e) : __int_as_float(0x7fc00000);
+                if (e < E && isnan(x)) x = -INFINITY;   // a NaN logit ranks as -inf (last, by id)
+                v[i] = x;                               // past E: NaN, never chosen
+            }
+            float top = -INFINITY, z = 0.f, pj = 0.f;
+            int myid = -1;
+            for (int j = 0; j < k; ++j) {
+                float bv = -INFINITY;
+                int bid = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) {
+                    const int e = lane + 32 * i;
+                    if (better(v[i], e, bv, bid)) {
+                        bv = v[i];
+                        bid = e;
+                    }
+                }
+                for (int o = 16; o; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+                    if (better(ov, oid, bv, bid)) {
+                        bv = ov;
+                        bid = oid;
+                    }
+                }
+                if (bid >= E) bid = 0;   // unreachable while k <= E
+                if (j == 0) top = bv;
+                if ((bid & 31) == lane) {
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i)
+                        if (lane + 32 * i == bid) v[i] = __int_as_float(0x7fc00000);   // taken
+                }
+                const float pe = expf(bv - top);
+                if (lane == j) {
+                    myid = bid;
+                    pj = pe;
+                }
+                z += pe;
+            }
+            if (lane < k) {
+                ms->ids[t][lane] = myid;
+                ms->w[t][lane] = pj / z;
+                atomicOr(&ms->bits[myid >> 5], 1u << (myid & 31));
+            }
+        }
+        csync();
+        if (warp == 0) {
+            // union in ascending expert order, then the shared experts
+            const int nwords = (E + 31) / 32;
+            const unsigned word = lane < nwords ? ms->bits[lane] : 0u;
+            int pre = __popc(word);
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, pre, o);
+                if (lane >= o) pre += n;
+            }
+            const int total = __shfl_sync(0xffffffffu, pre, 31);
+            pre -= __popc(word);   // exclusive
+            unsigned wv = word;
+            int pos = pre;
+            while (wv) {
+                const int b = __ffs(wv) - 1;
+                wv &= wv - 1;
+                uexp[pos++] = 32 * lane + b;
+            }
+            if (lane < p.nsh) uexp[total + lane] = E + lane;
+            const int nU = total + p.nsh;
+            for (int i = lane; i < nU * TM; i += 32) wtab[i] = 0.f;
+            if (lane < nU) hcum[lane] += (unsigned)ntile_gu;
+            for (int u = 32 + lane; u < nU; u += 32) hcum[u] += (unsigned)ntile_gu;
+            __syncwarp();
+            // weight table: token t's j-th expert sits at union slot (ones below it in the bitmap)
+            for (int i = lane; i < T * k; i += 32) {
+                const int t = i / k, j = i - t * k;
+                const int e = ms->ids[t][j];
+                const int wi = e >> 5;
+                int slot = __popc(ms->bits[wi] & ((1u << (e & 31)) - 1u));
+                for (int q = 0; q < wi; ++q) slot += __popc(ms->bits[q]);
+                wtab[slot * TM + t] = ms->w[t][j];
+            }
+            for (int i = lane; i < p.nsh * T; i += 32) wtab[(total + i / T) * TM + i % T] = 1.f;
+            __syncwarp();
+            if (lane < nwords) ms->bits[lane] = 0u;
+            if (lane == 0) {
+                ms->nU = nU;
+                ms->nR = total;
+            }
+            // routing outputs
+            if (cta == 0) {
+                for (int i = lane; i < T * k; i += 32) {
+                    const int t = i / k, j = i - t * k;
+                    if (p.stack && p.rec_on) {
+                        const size_t ro = ((size_t)l * p.rec_n + p.rec_r0 + t) * k + j;
+                        if (p.rec.ids) p.rec.ids[ro] = ms->ids[t][j];
+                        if (p.rec.w) p.rec.w[ro] = ms->w[t][j];
+                    }
+                    if (!p.stack) {
+                        if (p.ids_out) p.ids_out[(size_t)t * k + j] = ms->ids[t][j];
+                        if (p.w_out) p.w_out[(size_t)t * k + j] = ms->w[t][j];
+                    }
+                }
+            }
+        }
+        csync();
+        if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
+        const int nU = ms->nU;
+        const Split sp = split(nU);
+        auto slot_of = [&](int q, uint32_t &par) { return ring_slot(ring_s0, ring_p0, q, par); };
+
+        // ---- 4. gate/up ------------------------------------------------------------------------------
+        if (warp < GW) {
+            // B fragments of this warp's 256-wide k chunk: column g = token g (zero past T)
+            uint32_t bx0[16], bx1[16];
+            {
+                const bool live = g < T;
+                const uint16_t *xr = xb + (size_t)(live ? g : 0) * d + 256 * warp + 2 * c;
+                const float sc = live ? ms->xscale[g] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t v0 = live ? *reinterpret_cast<const uint32_t *>(xr + 16 * j) : 0u;
+                    const uint32_t v1 = live ? *reinterpret_cast<const uint32_t *>(xr + 16 * j + 8) : 0u;
+                    if constexpr (F16OP) {
+                        const __half2 h0 = __floats2half2_rn(bf16f(v0 & 0xFFFFu) * sc, bf16f(v0 >> 16) * sc);
+                        const __half2 h1 = __floats2half2_rn(bf16f(v1 & 0xFFFFu) * sc, bf16f(v1 >> 16) * sc);
+                        bx0[j] = *reinterpret_cast<const uint32_t *>(&h0);
+                        bx1[j] = *reinterpret_cast<const uint32_t *>(&h1);
+                    } else {
+                        bx0[j] = v0;
+                        bx1[j] = v1;
+                    }
+                }
+            }
+            // block sums of the operand for this lane's columns (tokens 2c, 2c+1), this chunk's 8 blocks
+            float xs0[8], xs1[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                xs0[b] = (2 * c < T) ? xsum[(2 * c) * nbd + 8 * warp + b] : 0.f;
+                xs1[b] = (2 * c + 1 < T) ? xsum[(2 * c + 1) * nbd + 8 * warp + b] : 0.f;
+            }
+            for (int q = 0; q < sp.n_gu && ok; ++q) {
+                uint32_t par;
+                const int s = slot_of(q, par);
+                ok = mbar_wait(&ms->full[s], par, err, true);
+                if (!ok) break;
+                const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
+                // this lane's scales: rows g and g+8, the chunk's 8 blocks
+                const uint4 sgv = *reinterpret_cast<const uint4 *>(tile + p.gu.code_bytes + ((size_t)g * nbd + 8 * warp) * 2);
+                const uint4 s8v = *reinterpret_cast<const uint4 *>(tile + p.gu.code_bytes + ((size_t)(g + 8) * nbd + 8 * warp) * 2);
+                const uint32_t sgw[4] = {sgv.x, sgv.y, sgv.z, sgv.w}, s8w[4] = {s8v.x, s8v.y, s8v.z, s8v.w};
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq) {
+                    uint32_t a[16];
+                    frag16<FMT>(tile + (size_t)(4 * warp + kq) * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
+                    float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_fmt<FMT>(Da, a + 0, bx0[4 * kq + 0], bx1[4 * kq + 0]);
+                    mma_fmt<FMT>(Da, a + 4, bx0[4 * kq + 1], bx1[4 * kq + 1]);
+                    mma_fmt<FMT>(Db, a + 8, bx0[4 * kq + 2], bx1[4 * kq + 2]);
+                    mma_fmt<FMT>(Db, a + 12, bx0[4 * kq + 3], bx1[4 * kq + 3]);
+                    const float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(&sgw[kq]));
+                    const float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(&s8w[kq]));
+                    flush_block<FMT>(acc, Da, sg.x, s8.x, xs0[2 * kq], xs1[2 * kq], false);
+                    flush_block<FMT>(acc, Db, sg.y, s8.y, xs0[2 * kq + 1], xs1[2 * kq + 1], true);
+                }
+                // the chunk's partial of rows g, g+8 for tokens 2c, 2c+1 into the unit's sums
+                float *rs = red + (size_t)s * 16 * TM;
+                if (2 * c < T) {
+                    atomicAdd(rs + g * TM + 2 * c, acc[0]);
+                    atomicAdd(rs + (g + 8) * TM + 2 * c, acc[2]);
+                }
+                if (2 * c + 1 < T) {
+                    atomicAdd(rs + g * TM + 2 * c + 1, acc[1]);
+                    atomicAdd(rs + (g + 8) * TM + 2 * c + 1, acc[3]);
+                }
+                __threadfence_block();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&ms->gcnt[s], 1) == GW - 1;
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    // every warp's share is in: SwiGLU of the unit's 8 rows for every token
+                    __threadfence_block();
+                    const int n = cta + G * q;
+                    const int u = n / ntile_gu, t8 = n - u * ntile_gu;
+                    for (int i = lane; i < 8 * T; i += 32) {
+                        const int r = i & 7, t = i >> 3;
+                        const float xi = ms->xinv[t];
+                        const float gs = rs[r * TM + t] * xi, us_ = rs[(8 + r) * TM + t] * xi;
+                        p.x_h[((size_t)u * TM + t) * I + 8 * t8 + r] = silu(gs) * us_;
+                    }
+                    for (int i = lane; i < 16 * TM; i += 32) rs[i] = 0.f;
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ms->gcnt[s] = 0;
+                        ctr_arrive(hctr(p, u));          // one more tile of expert slot u is done
+                        mbar_arrive(&ms->empty[s]);      // the slot may be refilled
+                    }
+                }
+            }
+        }
+        if (cta_failed(ok)) {
+            aborted = true;
+            break;
+        }
+
+        // ---- 5. down ---------------------------------------------------------------------------------
+        const int u_first = sp.n_dn > 0 ? sp.dn_lo / ntile_dn : 0;
+        const int n_span = sp.n_dn > 0 ? (sp.dn_hi - 1) / ntile_dn - u_first + 1 : 0;
+        if (n_span > 0) {
+            if (tid == 0) {
+                for (int su = 0; su < n_span && ok; ++su) ok = ctr_wait(hctr(p, u_first + su), hcum[u_first + su], err);
+            }
+            if (cta_failed(ok)) {
+                aborted = true;
+                break;
+            }
+            // h of the run's experts -> hi + lo B fragments (8 columns, zero past T) and, per
+            // (expert, token, 32-block), the sum of hi + lo and (fp16) the block's 2^-s
+            const int nq = n_span * TMAX * (I / 4);   // 4 values per thread and step; 8 lanes per block
+            for (int i = tid; i < nq; i += NT) {
+                const int su = i / (TMAX * (I / 4));
+                const int rem = i - su * (TMAX * (I / 4));
+                const int t = rem / (I / 4), k4 = rem - t * (I / 4);
+                const bool live = t < T;
+                float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (live) hv = ld_gpu4(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4);
+                const float h4[4] = {hv.x, hv.y, hv.z, hv.w};
+                float scale = 1.f;
+                if constexpr (F16OP) {
+                    float mx = fmaxf(fmaxf(fabsf(h4[0]), fabsf(h4[1])), fmaxf(fabsf(h4[2]), fabsf(h4[3])));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    int he;
+                    frexpf(mx, &he);
+                    const int sh = min(15 - he, 100);
+                    scale = pow2i(sh);
+                    if (live && (lane & 7) == 0) hinv[(su * TM + t) * nbi + (k4 >> 3)] = pow2i(-sh);
+                }
+                uint32_t hi2[2], lo2[2];
+                float part = 0.f;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    if constexpr (F16OP) {
+                        const float v0 = h4[2 * j] * scale, v1 = h4[2 * j + 1] * scale;
+                        const __half2 hh = __floats2half2_rn(v0, v1);
+                        const float2 hf = __half22float2(hh);
+                        const __half2 ll = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
+                        const float2 lf = __half22float2(ll);
+                        hi2[j] = *reinterpret_cast<const uint32_t *>(&hh);
+                        lo2[j] = *reinterpret_cast<const uint32_t *>(&ll);
+                        part += (hf.x + lf.x) + (hf.y + lf.y);
+                    } else {
+                        const uint16_t h0 = bf16_rn_bits(h4[2 * j]), h1 = bf16_rn_bits(h4[2 * j + 1]);
+                        const uint16_t l0 = bf16_rn_bits(h4[2 * j] - bf16_bits_f(h0));
+                        const uint16_t l1 = bf16_rn_bits(h4[2 * j + 1] - bf16_bits_f(h1));
+                        hi2[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                        lo2[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                        part += (bf16_bits_f(h0) + bf16_bits_f(l0)) + (bf16_bits_f(h1) + bf16_bits_f(l1));
+                    }
+                }
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                part += __shfl_xor_sync(0xffffffffu, part, 4);
+                if (live && (lane & 7) == 0) hsum[(su * TM + t) * nbi + (k4 >> 3)] = part;
+                // values k = 4 k4 .. 4 k4 + 3 of token t: slice sl, register b0 (kk < 8) or b1, the
+                // lanes (t, c0) and (t, c0 + 1)
+                const int kk = 4 * k4;
+                const int sl = kk >> 4, w16 = kk & 15, which = w16 >> 3, c0 = (w16 & 7) >> 1;
+                const int kg = sl >> 2, m = sl & 3;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(htab + hfrag_off(su, nkgi, kg, m, 4 * t + c0 + q));
+                    dst[which] = hi2[q];
+                    dst[2 + which] = lo2[q];
+                }
+            }
+            csync();
+        }
+        // units of this CTA's run, in batches of dn_per_slot (one ring item each); item i -> warp i % NW
+        for (int it = warp; it < sp.n_dn_items && ok; it += NW) {
+            uint32_t par;
+            const int s = slot_of(sp.n_gu + it, par);
+            ok = mbar_wait(&ms->full[s], par, err, true);
+            if (!ok) break;
+            const int q0 = it * dn_per_slot;
+            const int cnt = min(dn_per_slot, sp.n_dn - q0);
+            for (int ui = 0; ui < cnt; ++ui) {
+                const int n = sp.dn_lo + q0 + ui;
+                const int u = n / ntile_dn, j = n - u * ntile_dn;
+                const int su = u - u_first;
+                const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
+                const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const int t0 = 2 * c, t1 = 2 * c + 1;
+                const float *hs0 = hsum + (su * TM + min(t0, TM - 1)) * nbi;
+                const float *hs1 = hsum + (su * TM + min(t1, TM - 1)) * nbi;
+                const float *hi0 = hinv + (su * TM + min(t0, TM - 1)) * nbi;
+                const float *hi1 = hinv + (su * TM + min(t1, TM - 1)) * nbi;
+                const bool l0 = t0 < T, l1 = t1 < T;
+                for (int kg = 0; kg < nkgi; ++kg) {
+                    uint32_t a[16];
+                    frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
+                    float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint4 bq = *reinterpret_cast<const uint4 *>(htab + hfrag_off(su, nkgi, kg, m, lane));
+                        float *D = (m < 2) ? Da : Db;
+                        mma_fmt<FMT>(D, a + 4 * m, bq.x, bq.y);   // hi
+                        mma_fmt<FMT>(D, a + 4 * m, bq.z, bq.w);   // lo
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int b = 2 * kg + h;
+                        const float v0 = l0 ? hs0[b] : 0.f, v1 = l1 ? hs1[b] : 0.f;
+                        float sg = __half2float(sc[g * nbi + b]), s8 = __half2float(sc[(g + 8) * nbi + b]);
+                        float Dv[4] = {h ? Db[0] : Da[0], h ? Db[1] : Da[1], h ? Db[2] : Da[2], h ? Db[3] : Da[3]};
+                        if constexpr (F16OP) {
+                            // h entered as h * 2^s per (token, block): scale back per column
+                            const float i0 = l0 ? hi0[b] : 0.f, i1 = l1 ? hi1[b] : 0.f;
+                            float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+                            flush_block<FMT>(tmp, Dv, sg, s8, v0, v1, h == 1);
+                            acc[0] = fmaf(tmp[0], i0, acc[0]);
+                            acc[1] = fmaf(tmp[1], i1, acc[1]);
+                            acc[2] = fmaf(tmp[2], i0, acc[2]);
+                            acc[3] = fmaf(tmp[3], i1, acc[3]);
+                        } else {
+                            flush_block<FMT>(acc, Dv, sg, s8, v0, v1, h == 1);
+                        }
+                    }
+                }
+                // weighted by each token's routing weight for this expert, then 4 consecutive rows of
+                // one token per lane (a 4 x 4 transpose among the lanes g = 4m' .. 4m' + 3 of a column
+                // pair) for one vector atomic each
+                const float w0 = l0 ? wtab[u * TM + t0] : 0.f, w1 = l1 ? wtab[u * TM + t1] : 0.f;
+                const float val[4] = {acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1};
+                const int gi = g & 3, gbase = lane - 4 * gi;   // lane of (g - gi, c)
+                float vec[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int sidx = (gi + r) & 3, didx = (gi - r) & 3;
+                    const float send = sidx == 0 ? val[0] : sidx == 1 ? val[1] : sidx == 2 ? val[2] : val[3];
+                    const float got = __shfl_sync(0xffffffffu, send, gbase + 4 * didx);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) vec[q] = (q == didx) ? got : vec[q];
+                }
+                // lane (g, c) now holds rows 4 (g >> 2) + 8 (gi >> 1) + 0..3 of token 2c + (gi & 1)
+                const int tok = 2 * c + (gi & 1);
+                const int row0 = 16 * j + 4 * (g >> 2) + 8 * (gi >> 1);
+                if (tok < T && wtab[u * TM + tok] != 0.f)
+                    red_add_v4(yacc + (size_t)tok * d + row0, vec[0], vec[1], vec[2], vec[3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ms->empty[s]);
+        }
+        {
+            uint32_t par;
+            ring_s0 = slot_of(sp.n_items, par);
+            ring_p0 = par;
+        }
+        __threadfence();
+        if (cta_failed(ok)) {
+            aborted = true;
+            break;
+        }
+        if (tid == 0) ctr_arrive(p.cnt + C_Y);
+    }
+
+    // ---- outputs of the last layer: each CTA its owned columns -------------------------------------
+    if (!aborted) {
+        if (tid == 0) ok = ctr_wait(p.cnt + C_Y, (unsigned)(G * p.L), err);
+        if (!cta_failed(ok)) {
+            const int lb = (p.L - 1) & 1;
+            const float *yl = p.y_acc + (size_t)lb * TM * d;
+            const float *rl = p.r_buf + (size_t)lb * TM * d;
+            for (int i = tid; i < T * (own_hi - own_lo); i += NT) {
+                const int t = i / (own_hi - own_lo), i4 = own_lo + i - t * (own_hi - own_lo);
+                const float4 y = ld_gpu4(yl + (size_t)t * d + 4 * i4);
+                const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
+                               b3 = bf16_rn_bits(y.w);
+                const uint2 yb2 = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+                if (p.stack) {
+                    const float4 r = ld_gpu4(rl + (size_t)t * d + 4 * i4);
+                    *reinterpret_cast<float4 *>(p.resid_out + (size_t)t * d + 4 * i4) =
+                        make_float4(r.x + bf16_bits_f(b0), r.y + bf16_bits_f(b1), r.z + bf16_bits_f(b2),
+                                    r.w + bf16_bits_f(b3));
+                    if (p.rec_on) {
+                        const size_t ro = ((size_t)(p.L - 1) * p.rec_n + p.rec_r0 + t) * d + 4 * i4;
+                        if (p.rec.y_bf16) *reinterpret_cast<uint2 *>(p.rec.y_bf16 + ro) = yb2;
+                        if (p.rec.y_f32) *reinterpret_cast<float4 *>(p.rec.y_f32 + ro) = y;
+                    }
+                } else {
+                    *reinterpret_cast<uint2 *>(p.y_out + (size_t)t * d + 4 * i4) = yb2;
+                    if (p.yf_out) *reinterpret_cast<float4 *>(p.yf_out + (size_t)t * d + 4 * i4) = y;
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+
+// ---- host side -----------------------------------------------------------------------------------
+
+static int multi_tm(const moe_config &c) { return c.max_tokens < TMAX ? c.max_tokens : TMAX; }
+static int multi_um(const moe_config &c) { return multi_tm(c) * c.top_k + c.n_shared; }
+
+size_t decode_multi_counter_bytes(const moe_config &c) {
+    return (((size_t)(C_H + 8 * multi_um(c)) * 4) + 255) & ~(size_t)255;
+}
+static size_t xm_logits_off(const moe_config &c) { return decode_multi_counter_bytes(c); }
+static size_t xm_h_off(const moe_config &c) {
+    return xm_logits_off(c) + (((size_t)multi_tm(c) * c.n_experts * 4 + 255) & ~(size_t)255);
+}
+static size_t xm_y_off(const moe_config &c) {
+    return xm_h_off(c) + (size_t)multi_um(c) * multi_tm(c) * c.d_ff * 4;
+}
+static size_t xm_r_off(const moe_config &c) { return xm_y_off(c) + (size_t)2 * multi_tm(c) * c.d_model * 4; }
+size_t decode_multi_xchg_bytes(const moe_config &c) {
+    return xm_r_off(c) + (size_t)2 * multi_tm(c) * c.d_model * 4;
+}
+
+bool decode_multi_supported(const moe_ctx *ctx) {
+    const moe_config &c = ctx->cfg;
+    if (c.flags & MOE_FLAG_NO_DECODE_KERNEL) return false;
+    if (c.max_tokens < 2) return false;
+    if (c.d_model > 4096 || c.d_model / 256 > NW || c.n_experts > 32 * EPL || c.n_experts % 4) return false;
+    if (c.top_k > KMAX) return false;
+    return ctx->mdec.smem_bytes > 0;
+}
+
+int decode_multi_setup(moe_ctx *ctx) {
+    const moe_config &c = ctx->cfg;
+    MultiState &ms = ctx->mdec;
+    ms.smem_bytes = 0;
+    if (c.max_tokens < 2) return MOE_OK;
+    cudaDeviceProp prop;
+    QE_CHECK(cudaGetDeviceProperties(&prop, ctx->device));
+    int G = prop.multiProcessorCount;
+    if (G > c.d_model / 16) G = c.d_model / 16;
+    const int TM = multi_tm(c), UM = multi_um(c);
+    const int rpc = (c.n_experts + G - 1) / G;
+    if (rpc > 8) return MOE_OK;
+    // experts a CTA's down run may touch
+    const long long n_dn_max = ((long long)UM * (c.d_model / 16) + G - 1) / G;
+    const int ntile_dn = c.d_model / 16;
+    const int span = (int)((n_dn_max + ntile_dn - 2) / ntile_dn) + 1;
+    if (span > MAX_SPAN) return MOE_OK;
+    int slot = ctx->gu.tile_bytes > ctx->dn.tile_bytes ? ctx->gu.tile_bytes : ctx->dn.tile_bytes;
+    size_t fixed = 0;
+    auto take = [&fixed](size_t bytes) {
+        int off = (int)fixed;
+        fixed = (fixed + bytes + 127) & ~(size_t)127;
+        return off;
+    };
+    const size_t xb_bytes = (size_t)TM * c.d_model * 2;
+    const size_t htab_bytes = (size_t)span * (c.d_ff / 64) * 4 * 32 * 16;
+    ms.off_router = take((size_t)rpc * c.d_model * 4);
+    ms.off_xb = take(xb_bytes > htab_bytes ? xb_bytes : htab_bytes);
+    ms.off_xsum = take((size_t)TM * (c.d_model / 32) * 4);
+    ms.off_hsum = take((size_t)2 * span * TM * (c.d_ff / 32) * 4);
+    ms.off_uexp = take((size_t)UM * 4);
+    ms.off_hcum = take((size_t)UM * 4);
+    ms.off_wtab = take((size_t)UM * TM * 4);
+    ms.off_misc = take(sizeof(MiscM));
+    ms.off_ltab = take((size_t)c.n_layers * sizeof(LayerPtrs));
+    const size_t red_per_slot = (size_t)16 * TM * 4;
+    size_t limit = (size_t)prop.sharedMemPerBlockOptin;
+    int nslot = MAX_SLOTS;
+    while (nslot >= 2 && ((fixed + nslot * red_per_slot + 127) & ~(size_t)127) + (size_t)nslot * slot > limit) --nslot;
+    if (nslot < 2) return MOE_OK;
+    ms.off_red = take((size_t)nslot * red_per_slot);
+    ms.off_ring = (int)fixed;
+    ms.nslot = nslot;
+    ms.slot_bytes = slot;
+    ms.rpc = rpc;
+    ms.span = span;
+    ms.grid = G;
+    ms.tm = TM;
+    ms.um = UM;
+    ms.smem_bytes = (int)(fixed + (size_t)nslot * slot);
+    const void *kfn = c.fmt == MOE_Q4B32   ? (const void *)k_decode_multi<MOE_Q4B32>
+                      : c.fmt == MOE_Q2B32 ? (const void *)k_decode_multi<MOE_Q2B32>
+                                           : (const void *)k_decode_multi<MOE_Q3B32>;
+    QE_CHECK(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, ms.smem_bytes));
+    int per_sm = 0;
+    QE_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, NTT, ms.smem_bytes));
+    if (per_sm < 1) ms.smem_bytes = 0;
+    return MOE_OK;
+}
+
+int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int T, bool stack, float *resid_out,
+                        uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n,
+                        int rec_r0, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    MultiState &ms = ctx->mdec;
+    if (T < 1 || T > ms.tm) return MOE_ERR_INVALID_ARG;
+    MultiParams p;
+    memset(&p, 0, sizeof(p));
+    p.layers = ctx->d_layers;
+    p.layer0 = layer0;
+    p.L = L;
+    p.d = c.d_model;
+    p.E = c.n_experts;
+    p.I = c.d_ff;
+    p.k = c.top_k;
+    p.nsh = c.n_shared;
+    p.T = T;
+    p.TM = ms.tm;
+    p.gu = ctx->gu;
+    p.dn = ctx->dn;
+    p.stack = stack ? 1 : 0;
+    p.x_in = x;
+    p.resid_out = resid_out;
+    p.y_out = y;
+    p.yf_out = yf;
+    p.ids_out = ids;
+    p.w_out = w;
+    if (rec) {
+        p.rec = *rec;
+        p.rec_on = 1;
+        p.rec_n = rec_n;
+        p.rec_r0 = rec_r0;
+    }
+    uint8_t *xb = ms.xbuf;
+    p.cnt = reinterpret_cast<unsigned *>(xb);
+    p.x_logits = reinterpret_cast<float *>(xb + xm_logits_off(c));
+    p.x_h = reinterpret_cast<float *>(xb + xm_h_off(c));
+    p.y_acc = reinterpret_cast<float *>(xb + xm_y_off(c));
+    p.r_buf = reinterpret_cast<float *>(xb + xm_r_off(c));
+    p.err = ctx->ws.dev_error;
+    p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ctx->dec.withheld) ? 1 : 0;
+    if (p.withhold) ctx->dec.withheld = true;
+    p.nslot = ms.nslot;
+    p.slot_bytes = ms.slot_bytes;
+    p.rpc = ms.rpc;
+    p.span = ms.span;
+    p.UM = ms.um;
+    p.off_ring = ms.off_ring;
+    p.off_router = ms.off_router;
+    p.off_xb = ms.off_xb;
+    p.off_red = ms.off_red;
+    p.off_xsum = ms.off_xsum;
+    p.off_hsum = ms.off_hsum;
+    p.off_uexp = ms.off_uexp;
+    p.off_hcum = ms.off_hcum;
+    p.off_wtab = ms.off_wtab;
+    p.off_misc = ms.off_misc;
+    p.off_ltab = ms.off_ltab;
+    // counters start from zero, and so do both output buffers
+    QE_CHECK(cudaMemsetAsync(xb, 0, decode_multi_counter_bytes(c), st));
+    QE_CHECK(cudaMemsetAsync(p.y_acc, 0, (size_t)2 * ms.tm * c.d_model * 4, st));
+    void *args[] = {&p};
+    const void *kfn = c.fmt == MOE_Q4B32   ? (const void *)k_decode_multi<MOE_Q4B32>
+                      : c.fmt == MOE_Q2B32 ? (const void *)k_decode_multi<MOE_Q2B32>
+                                           : (const void *)k_decode_multi<MOE_Q3B32>;
+    QE_CHECK(cudaLaunchCooperativeKernel(kfn, dim3(ms.grid), dim3(NTT), args, (size_t)ms.smem_bytes, st));
+    QE_CHECK_LAUNCH("k_decode_multi");
+    return MOE_OK;
+}
+
+}  // namespace qeffn

@@ -157,6 +157,12 @@ int alloc_workspace(moe_ctx *ctx) {
     size_t xb = decode_xchg_bytes(c);
     QE_TRY(ctx_alloc(ctx, (void **)&ctx->dec.xbuf, xb, "exchange area"));
     QE_CHECK(cudaMemset(ctx->dec.xbuf, 0, xb));
+    QE_TRY(decode_multi_setup(ctx));
+    if (ctx->mdec.smem_bytes > 0) {
+        size_t xm = decode_multi_xchg_bytes(c);
+        QE_TRY(ctx_alloc(ctx, (void **)&ctx->mdec.xbuf, xm, "few-token exchange area"));
+        QE_CHECK(cudaMemset(ctx->mdec.xbuf, 0, xm));
+    }
     return MOE_OK;
 }
 
@@ -237,12 +243,31 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
     return MOE_OK;
 }
 
+bool multi_ok(const moe_ctx *ctx) {
+    return !(ctx->cfg.flags & MOE_FLAG_NO_MULTI_DECODE) && decode_multi_supported(ctx);
+}
+
 int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y, float *yf,
                   int32_t *ids, float *w, cudaStream_t st) {
     const Layer &Ly = ctx->layers[layer];
     Workspace &ws = ctx->ws;
     int32_t *ids_ = ids ? ids : ws.ids;
     float *w_ = w ? w : ws.w;
+    if (T >= 2 && T <= DECODE_MULTI_MAX && multi_ok(ctx)) {
+        // the few-token kernel, at most eight tokens per launch, in near-equal chunks
+        const moe_config &c = ctx->cfg;
+        const int n = (T + ctx->mdec.tm - 1) / ctx->mdec.tm;
+        QE_TRY(timing_begin(ctx, st, "k_decode_multi"));
+        for (int i = 0, t0 = 0; i < n; ++i) {
+            const int tn = (T - t0) / (n - i);
+            QE_TRY(launch_decode_multi(ctx, layer, 1, x + (size_t)t0 * c.d_model, tn, false, nullptr,
+                                       y + (size_t)t0 * c.d_model, yf ? yf + (size_t)t0 * c.d_model : nullptr,
+                                       ids_ + (size_t)t0 * c.top_k, w_ + (size_t)t0 * c.top_k, nullptr, 0, 0, st));
+            t0 += tn;
+        }
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
     if (T <= DECODE_TOKENS_MAX && decode_supported(ctx)) {
         const moe_config &c = ctx->cfg;
         QE_TRY(timing_begin(ctx, st, "k_decode"));
@@ -253,9 +278,14 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
         QE_TRY(timing_end(ctx, st));
         return MOE_OK;
     }
-    if (tc_router_supported(ctx, T)) QE_TRY(launch_tc_router(ctx, Ly, x, T, ws.logits, st));
-    else QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
-    QE_TRY(launch_topk(ctx, ws.logits, T, ids_, w_, st));
+    if (tc_router_supported(ctx, T)) {
+        // tensor-core logits pick the candidates; their logits are recomputed in fp32 for the choice
+        QE_TRY(launch_tc_router(ctx, Ly, x, T, ws.logits, st));
+        QE_TRY(launch_topk_refine(ctx, Ly, x, ws.logits, T, ids_, w_, st));
+    } else {
+        QE_TRY(launch_router_simt(ctx, Ly, x, T, ws.logits, st));
+        QE_TRY(launch_topk(ctx, ws.logits, T, ids_, w_, st));
+    }
     QE_TRY(launch_dispatch(ctx, ids_, T, st));
     if (tc_supported(ctx, T)) return launch_tc_experts(ctx, Ly, x, T, w_, y, yf, st);
     QE_TRY(timing_begin(ctx, st, "k_gateup_simt+k_down_simt"));
@@ -337,9 +367,24 @@ int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint16_t *x_
     QE_CHECK(cudaSetDevice(ctx->device));
     cudaStream_t st = (cudaStream_t)stream;
     Workspace &ws = ctx->ws;
-    // few tokens: the single-token kernel runs each token through the whole stack (records of
-    // every row, or of the one row of a single token; a device row list with more tokens takes
-    // the general path)
+    // few tokens: the few-token kernel runs up to eight tokens per launch through the whole stack
+    // (records of every row; a device row list with more than one token takes the general path)
+    if (T >= 2 && T <= DECODE_MULTI_MAX && multi_ok(ctx) && (!rec || !rec->rows)) {
+        const moe_config &c = ctx->cfg;
+        const int n = (T + ctx->mdec.tm - 1) / ctx->mdec.tm;
+        QE_TRY(timing_begin(ctx, st, "k_decode_multi"));
+        for (int i = 0, t0 = 0; i < n; ++i) {
+            const int tn = (T - t0) / (n - i);
+            QE_TRY(launch_decode_multi(ctx, layer0, n_layers, x_bf16 + (size_t)t0 * c.d_model, tn, true,
+                                       resid_out + (size_t)t0 * c.d_model, nullptr, nullptr, nullptr, nullptr, rec,
+                                       T, t0, st));
+            t0 += tn;
+        }
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
+    // the single-token kernel runs each token through the whole stack (records of every row, or
+    // of the one row of a single token; a device row list with more tokens takes the general path)
     if (T <= DECODE_TOKENS_MAX && decode_supported(ctx) && (!rec || !rec->rows || T == 1)) {
         if (rec && rec->rows && rec->n_rows != 1) return MOE_ERR_INVALID_ARG;
         const moe_config &c = ctx->cfg;

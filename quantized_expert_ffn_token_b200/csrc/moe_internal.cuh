@@ -209,6 +209,18 @@ struct DecodeState {
     int trace_words = 24;                  // uint64 per record
 };
 
+// Launch plan of the few-token decode kernel (decode_multi.cu).
+struct MultiState {
+    int grid = 0;
+    int smem_bytes = 0;   // 0: the shape does not fit the kernel
+    int tm = 0;           // tokens per launch the carve holds (<= 8)
+    int um = 0;           // union slots: tm * top_k + n_shared
+    int nslot = 0, slot_bytes = 0, rpc = 0, span = 0;
+    int off_ring = 0, off_router = 0, off_xb = 0, off_red = 0, off_xsum = 0, off_hsum = 0, off_uexp = 0,
+        off_hcum = 0, off_wtab = 0, off_misc = 0, off_ltab = 0;
+    uint8_t *xbuf = nullptr;   // counters, logits, h, output and residual buffers
+};
+
 // Event pairs around the dominant kernel (moe_timing_enable).
 struct Timing {
     bool on = false;
@@ -233,6 +245,7 @@ struct moe_ctx {
     qeffn::Timing timing;
     qeffn::LayerPtrs *d_layers = nullptr;   // [n_layers] on the device
     qeffn::DecodeState dec;
+    qeffn::MultiState mdec;
 };
 
 namespace qeffn {
@@ -276,6 +289,8 @@ int launch_router_simt(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, i
                        float *logits, cudaStream_t st);
 int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, float *w,
                 cudaStream_t st);
+int launch_topk_refine(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, const float *logits, int T,
+                       int32_t *ids, float *w, cudaStream_t st);
 int launch_dispatch(moe_ctx *ctx, const int32_t *ids, int T, cudaStream_t st);
 int launch_route_raw(const uint16_t *x, int T, int d, int E, int k, const float *W, const float *b,
                      float *logits, int32_t *ids, float *w, cudaStream_t st);
@@ -297,6 +312,16 @@ constexpr int TC_MIN_TOKENS = DECODE_TOKENS_MAX + 1;
 int decode_setup(moe_ctx *ctx);
 size_t decode_xchg_bytes(const moe_config &c);
 size_t decode_xchg_counter_bytes();   // the counters at the start of the exchange area
+// Few-token decode: 2..DECODE_MULTI_MAX tokens run the few-token kernel, up to
+// eight tokens per launch (one read of the batch's experts per layer).
+constexpr int DECODE_MULTI_MAX = 16;
+bool decode_multi_supported(const moe_ctx *ctx);
+int decode_multi_setup(moe_ctx *ctx);
+size_t decode_multi_xchg_bytes(const moe_config &c);
+size_t decode_multi_counter_bytes(const moe_config &c);
+int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int T, bool stack, float *resid_out,
+                        uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n,
+                        int rec_r0, cudaStream_t st);
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n, int rec_r,
                   cudaStream_t st);

@@ -129,6 +129,121 @@ __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, 
     }
 }
 
+// Top-k from approximate logits (the tensor-core router sums its products in
+// the MMA units' own order and precision): one warp per token takes the
+// k + REFINE_EXTRA best experts by the approximate logits, recomputes those
+// experts' logits with fp32 FMAs (lane-strided over d, then a warp sum, as the
+// CUDA-core router does), and selects the top k among them by the recomputed
+// values; the weights are the softmax over the chosen recomputed logits.  An
+// expert outside the candidates could only be chosen if the approximate
+// logits erred by more than the gap across REFINE_EXTRA ranks.
+constexpr int REFINE_EXTRA = 6;
+__global__ void __launch_bounds__(256) k_topk_refine(const float *__restrict__ logits, int T, int E, int k,
+                                                     const uint16_t *__restrict__ x, int d,
+                                                     const float *__restrict__ W, const float *__restrict__ b,
+                                                     int32_t *__restrict__ ids, float *__restrict__ w) {
+    extern __shared__ float lg[];   // [8][E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    float *my = lg + warp * E;
+    for (int e = lane; e < E; e += 32) {
+        const float v = logits[(size_t)t * E + e];
+        my[e] = isnan(v) ? -INFINITY : v;
+    }
+    __syncwarp();
+    const int R = min(E, k + REFINE_EXTRA);   // <= 38: two candidates per lane at most
+    int cid0 = 0, cid1 = 0;
+    for (int j = 0; j < R; ++j) {
+        float bv = -INFINITY;
+        int bid = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            const float v = my[e];
+            if (better(v, e, bv, bid)) {
+                bv = v;
+                bid = e;
+            }
+        }
+        for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (bid >= E) bid = 0;
+        if (lane == (j & 31)) {
+            if (j < 32) cid0 = bid;
+            else cid1 = bid;
+        }
+        __syncwarp();
+        if (lane == 0) my[bid] = __int_as_float(0x7fc00000);   // taken
+        __syncwarp();
+    }
+    // recompute the candidates' logits: candidate j's dot product over the whole warp
+    const uint16_t *xr = x + (size_t)t * d;
+    float ex0 = __int_as_float(0x7fc00000), ex1 = __int_as_float(0x7fc00000);   // NaN: no candidate
+    for (int j = 0; j < R; ++j) {
+        const int e = __shfl_sync(0xffffffffu, j < 32 ? cid0 : cid1, j & 31);
+        const float4 *Wr = reinterpret_cast<const float4 *>(W + (size_t)e * d);
+        float acc = 0.f;
+        for (int i4 = lane; i4 < d / 4; i4 += 32) {
+            const float4 wv = Wr[i4];
+            const uint2 xv = *reinterpret_cast<const uint2 *>(xr + 4 * i4);
+            acc = fmaf(wv.x, __uint_as_float(xv.x << 16), acc);
+            acc = fmaf(wv.y, __uint_as_float(xv.x & 0xFFFF0000u), acc);
+            acc = fmaf(wv.z, __uint_as_float(xv.y << 16), acc);
+            acc = fmaf(wv.w, __uint_as_float(xv.y & 0xFFFF0000u), acc);
+        }
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        float v = acc + b[e];
+        if (isnan(v)) v = -INFINITY;
+        if (lane == (j & 31)) {
+            if (j < 32) ex0 = v;
+            else ex1 = v;
+        }
+    }
+    // top k among the candidates by the recomputed logits (taken ones become NaN)
+    float chosen_v = -INFINITY, top = -INFINITY;
+    int chosen_id = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bid = 0x7fffffff;
+        if (better(ex0, cid0, bv, bid)) {
+            bv = ex0;
+            bid = cid0;
+        }
+        if (lane + 32 < R && better(ex1, cid1, bv, bid)) {
+            bv = ex1;
+            bid = cid1;
+        }
+        for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (bid >= E) bid = 0;
+        if (j == 0) top = bv;
+        if (lane == j) {
+            chosen_v = bv;
+            chosen_id = bid;
+        }
+        if (cid0 == bid && lane < R) ex0 = __int_as_float(0x7fc00000);
+        if (cid1 == bid && lane + 32 < R) ex1 = __int_as_float(0x7fc00000);
+    }
+    const float p = (lane < k) ? expf(chosen_v - top) : 0.f;
+    float z = p;
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < k) {
+        ids[(size_t)t * k + lane] = chosen_id;
+        w[(size_t)t * k + lane] = p / z;
+    }
+}
+
 __device__ inline int slot_expert(const int32_t *ids, int slot, int T, int k, int E) {
     int routed = T * k;
     return slot < routed ? ids[slot] : E + (slot - routed) / T;
@@ -227,6 +342,16 @@ int launch_topk(const moe_ctx *ctx, const float *logits, int T, int32_t *ids, fl
     size_t smem = 8 * (size_t)c.n_experts * sizeof(float);
     k_topk<<<(T + 7) / 8, 256, smem, st>>>(logits, T, c.n_experts, c.top_k, ids, w);
     QE_CHECK_LAUNCH("k_topk");
+    return MOE_OK;
+}
+
+int launch_topk_refine(const moe_ctx *ctx, const Layer &Ly, const uint16_t *x, const float *logits, int T,
+                       int32_t *ids, float *w, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    size_t smem = 8 * (size_t)c.n_experts * sizeof(float);
+    k_topk_refine<<<(T + 7) / 8, 256, smem, st>>>(logits, T, c.n_experts, c.top_k, x, c.d_model, Ly.router_w,
+                                                  Ly.router_b, ids, w);
+    QE_CHECK_LAUNCH("k_topk_refine");
     return MOE_OK;
 }
 

@@ -9,8 +9,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_reference_arm_prints_one_complete_json_line():
-    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
-                        "--ref-layers", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -23,6 +22,9 @@ def test_reference_arm_prints_one_complete_json_line():
     assert d["config"]["workload"] == "decode_48l_q4_t1"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert cb["host_cores"] >= cb["cores"]
+    # the step time is the measured time of one bounded sample, and the run fits its own steps
+    assert 0 < d["ms_per_step"] < 60_000
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
@@ -35,8 +37,7 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
         port = s.getsockname()[1]
     r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
                         "--master-addr", "127.0.0.1", "--master-port", str(port),
-                        "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
-                        "--ref-layers", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+                        "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
     assert len(lines) == 1

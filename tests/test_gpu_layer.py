@@ -64,7 +64,7 @@ def test_tiny_layer_all_tokens(fmt):
     sess.close()
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 5, 8, 9, 16, 17, 63, 64, 127, 128, 129])
+@pytest.mark.parametrize("T", list(range(1, 18)) + [63, 64, 127, 128, 129])
 def test_tiny_ragged_token_counts(T):
     capi, session = _cuda()
     sess = session.Session(TINY, max_tokens=256)
@@ -75,6 +75,82 @@ def test_tiny_ragged_token_counts(T):
     o = oracle.moe_layer(TINY.fmt, TINY.k, x, W)
     check_rows(TINY, ExpertSource(TINY, 0), x, list(range(T)), gy, gyf, gids, gw, o=o, tol16=bf16_tol(T))
     sess.close()
+
+
+@pytest.mark.parametrize("fmt,T", [("q3", 2), ("q3", 7), ("q3", 12), ("q2", 3), ("q2", 8), ("q2", 16)])
+def test_few_token_kernel_other_formats(fmt, T):
+    """The few-token kernel (2..16 tokens, up to eight per launch) on Q3B32 and
+    Q2B32 against the oracle, every token."""
+    capi, session = _cuda()
+    cfg = TINY_Q3 if fmt == "q3" else TINY_Q2
+    sess = session.Session(cfg, max_tokens=16)
+    sess.load_synthetic()
+    x = _tokens(cfg, T, stream=100 + T)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    o = oracle.moe_layer(cfg.fmt, cfg.k, x, synth.layer_weights(cfg, 0))
+    check_rows(cfg, ExpertSource(cfg, 0), x, list(range(T)), gy, gyf, gids, gw, o=o)
+    sess.close()
+
+
+@pytest.mark.parametrize("name,T", [("tiny_d256_e16_q4_t8", 6), ("verify_48l_q3_t4_zipf", 4),
+                                    ("decode_48l_q4_t1", 8), ("decode_q2", 5)])
+def test_few_token_kernel_matches_single_token_kernel(name, T):
+    """A batch through the few-token kernel against the same tokens one at a
+    time through the single-token kernel (both exact-operand paths whose
+    per-block offset removal leaves about 2^-16 relative per partial): same
+    ids, weights within 1e-6, fp32 outputs within 1e-4 relative L2."""
+    capi, session = _cuda()
+    cfg = {"decode_q2": DECODE_Q2}.get(name) or synth.CONFIGS[name]
+    a = session.Session(cfg, max_tokens=16, n_layers=1)
+    b = session.Session(cfg, max_tokens=16, n_layers=1, flags=capi.MOE_FLAG_NO_MULTI_DECODE)
+    W = synth.layer_weights(cfg, 0, device="cuda")
+    a.load(0, W)
+    b.load(0, W)
+    del W
+    x = _tokens(cfg, T, stream=55)
+    ya, yfa, ida, wa = _run(a, 0, x)
+    yb, yfb, idb, wb = _run(b, 0, x)
+    assert capi.moe_get_device_error(a.ctx) == 0
+    assert np.array_equal(ida, idb)
+    assert np.max(np.abs(wa - wb)) <= 1e-6
+    assert rel_l2(yfa, yfb) <= 1e-4
+    a.close()
+    b.close()
+
+
+@pytest.mark.parametrize("name,T", [("decode_48l_q4_t1", 8), ("decode_48l_q4_t1", 13), ("verify_48l_q3_t4_zipf", 16)])
+def test_few_token_full_size(name, T):
+    """Full-size layers through the few-token kernel (one launch of eight, two
+    launches for 13 and 16 tokens), every token against the oracle."""
+    capi, session = _cuda()
+    cfg = synth.CONFIGS[name]
+    sess = session.Session(cfg, max_tokens=T, n_layers=1)
+    sess.load_synthetic(layers=[0])
+    x = _tokens(cfg, T, stream=900 + T)
+    gy, gyf, gids, gw = _run(sess, 0, x)
+    assert capi.moe_get_device_error(sess.ctx) == 0
+    sess.close()
+    src = HostLayer(cfg, 0)
+    rows = list(range(T))
+    check_rows(cfg, src, x, rows, gy, gyf, gids, gw, o=oracle_rows_dense(cfg, src, x, rows))
+
+
+def test_few_token_wait_times_out_and_context_recovers():
+    """The bounded waits of the few-token kernel: with the test hook its CTA 0
+    withholds its logits in the context's first call, every wait gives up,
+    MOE_ERR_DEVICE_TIMEOUT is reported, and the next calls are correct."""
+    capi, session = _cuda()
+    s = session.Session(TINY, max_tokens=8, n_layers=1, flags=capi.MOE_FLAG_TEST_WITHHOLD)
+    s.load_synthetic()
+    x = _tokens(TINY, 5, stream=78)
+    _run(s, 0, x)
+    assert capi.moe_get_device_error(s.ctx) == capi.MOE_ERR_DEVICE_TIMEOUT
+    o = oracle.moe_layer(TINY.fmt, TINY.k, x, synth.layer_weights(TINY, 0))
+    for rep in range(2):
+        gy, gyf, gids, gw = _run(s, 0, x)
+        assert capi.moe_get_device_error(s.ctx) == 0
+        check_rows(TINY, ExpertSource(TINY, 0), x, list(range(5)), gy, gyf, gids, gw, o=o)
+    s.close()
 
 
 def test_batch_equals_single_tokens():

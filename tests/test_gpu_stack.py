@@ -24,7 +24,7 @@ def _stack(name, rows=None, check_layers=None, dense=False, layer0_all=False):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from quantized_expert_ffn_token_b200 import capi, session
-    cfg = synth.CONFIGS[name]
+    cfg = synth.CONFIGS[name] if isinstance(name, str) else name
     L, T, d, k = cfg.L, cfg.T, cfg.d, cfg.k
     sess = session.Session(cfg, max_tokens=T)
     sess.load_synthetic()
@@ -98,6 +98,14 @@ def test_decode_stack_48_layers():
 
 def test_verify_stack_48_layers():
     _stack("verify_48l_q3_t4_zipf")
+
+
+def test_few_token_stack_48_layers_13_tokens():
+    """Thirteen tokens through the 48-layer Q4 stack: two launches of the
+    few-token kernel (7 + 6 tokens), every token's record of every layer
+    against the oracle."""
+    import dataclasses
+    _stack(dataclasses.replace(synth.CONFIGS["decode_48l_q4_t1"], T=13))
 
 
 @pytest.mark.slow
