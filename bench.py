@@ -387,6 +387,8 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
            "entry_point": "moe_forward_stack_host" + (" (one layer: rmsnorm + layer + residual)" if cfg.L == 1 else ""),
            "timer": "host wall clock around synchronous calls"}
     sess.close()
+    l2 = (f"{FLUSH_BYTES >> 20} MB flush before each timed step" if flush is not None else
+          f"no flush: each step streams {step_bytes / 1e9:.2f} GB (> 126 MB L2)")
     del xs, out, flush
     torch.cuda.empty_cache()
 
@@ -396,8 +398,7 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
         "config": {"workload": f"{cfg.name}: d={cfg.d} E={cfg.E} top-{cfg.k}+{cfg.n_shared} shared "
                                f"I={cfg.I} {fmt} T={cfg.T} layers={cfg.L}",
                    "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
-                   "l2": (f"{FLUSH_BYTES >> 20} MB flush before each timed step" if flush is not None else
-                          f"no flush: each step streams {step_bytes / 1e9:.2f} GB (> 126 MB L2)")},
+                   "l2": l2},
         "dtype": ("fp16 tensor-core MMA, fp32 accumulate, over " if tensor_bound else
                   "exact code operands, fp32 accumulate, over ") + fmt + " weights / bf16 activations",
         "roofline": roof, "step_roofline": step_roof, "e2e": e2e,

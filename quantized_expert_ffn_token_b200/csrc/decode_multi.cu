@@ -54,6 +54,7 @@ struct MiscM {
     unsigned long long rbar;
     unsigned long long route;              // one arrival per layer: routing known
     int gcnt[MAX_SLOTS];                   // gate/up warps done with the unit in slot s
+    int ccnt[MAX_SLOTS];                   // items of slot s consumed so far in this launch
     int nU;                                // experts in use this layer (routed union + shared)
     int nR;                                // routed part of the union
     int ids[TMAX][KMAX];
@@ -152,6 +153,22 @@ __device__ __forceinline__ void flush_block(float *acc, const float *D, float sg
     acc[3] = fmaf(s8, fmaf(D[3], m8, -o8 * v1), acc[3]);
 }
 
+// Bounded wait of a warp (all lanes poll) until a shared-memory counter reaches n; false on timeout
+// (error word set) or when another CTA reported an error.
+__device__ __forceinline__ bool smem_count_wait(const int *c, int n, int *err) {
+    long long t0 = clock64();
+    for (int it = 0;; ++it) {
+        if (*(volatile const int *)c >= n) return true;
+        if ((it & 15) == 15) {
+            if (*(volatile int *)err != 0) return false;
+            if (clock64() - t0 > SPIN_LIMIT) {
+                atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 // Position of the 16-byte B fragment of (expert-in-span su, k group kg, slice m,
 // lane) in the down phase's h table: [su][kg][m][lane] x 16 bytes, so that one
 // warp instruction reads 512 contiguous bytes.
@@ -193,6 +210,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             mbar_init(&ms->full[s], 1);
             mbar_init(&ms->empty[s], 1);
             ms->gcnt[s] = 0;
+            ms->ccnt[s] = 0;
         }
         mbar_init(&ms->rbar, 1);
         mbar_init(&ms->route, 1);
@@ -220,15 +238,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         sp.n_items = sp.n_gu + sp.n_dn_items;
         return sp;
     };
-    auto ring_slot = [&](int s0, uint32_t p0, int q, uint32_t &par) {
-        int sq = s0 + q;
-        par = p0;
-        while (sq >= p.nslot) {
-            sq -= p.nslot;
-            par ^= 1u;
-        }
-        return sq;
-    };
+    // items fill the ring cyclically from the launch's first item: the item with absolute index a
+    // sits in slot a % nslot as that slot's (a / nslot)-th fill
 
     // ---- producer warp (lane 0) -----------------------------------------------------------
     if (warp == NW) {
@@ -291,8 +302,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         return;
     }
 
-    int ring_s0 = 0;
-    uint32_t ring_p0 = 0;
+    int ring_base = 0;                  // absolute index of this layer's first item
     bool ok = true;
     bool aborted = false;
 
@@ -610,7 +620,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
         const int nU = ms->nU;
         const Split sp = split(nU);
-        auto slot_of = [&](int q, uint32_t &par) { return ring_slot(ring_s0, ring_p0, q, par); };
+        auto slot_of = [&](int q, uint32_t &par, int &fill) {
+            const int a = ring_base + q;
+            fill = a / p.nslot;
+            par = (uint32_t)(fill & 1);
+            return a - fill * p.nslot;
+        };
 
         // ---- 4. gate/up ------------------------------------------------------------------------------
         if (warp < GW) {
@@ -643,8 +658,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 xs1[b] = (2 * c + 1 < T) ? xsum[(2 * c + 1) * nbd + 8 * warp + b] : 0.f;
             }
             for (int q = 0; q < sp.n_gu && ok; ++q) {
+                // every gate/up warp consumes every unit in order, so the slot's previous item is one
+                // this warp has finished: the parity below cannot refer to an older fill
                 uint32_t par;
-                const int s = slot_of(q, par);
+                int fill;
+                const int s = slot_of(q, par, fill);
                 ok = mbar_wait(&ms->full[s], par, err, true);
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
@@ -699,6 +717,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     if (lane == 0) {
                         ms->gcnt[s] = 0;
                         ctr_arrive(hctr(p, u));          // one more tile of expert slot u is done
+                        atomicAdd(&ms->ccnt[s], 1);
                         mbar_arrive(&ms->empty[s]);      // the slot may be refilled
                     }
                 }
@@ -785,9 +804,14 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         }
         // units of this CTA's run, in batches of dn_per_slot (one ring item each); item i -> warp i % NW
         for (int it = warp; it < sp.n_dn_items && ok; it += NW) {
+            // items go round-robin to the warps, so this warp may reach an item while its slot still
+            // holds an older one (consumed by another warp): first wait until every earlier item of
+            // the slot is consumed, then the fill parity names this item's fill unambiguously
             uint32_t par;
-            const int s = slot_of(sp.n_gu + it, par);
-            ok = mbar_wait(&ms->full[s], par, err, true);
+            int fill;
+            const int s = slot_of(sp.n_gu + it, par, fill);
+            ok = smem_count_wait(&ms->ccnt[s], fill, err);
+            if (ok) ok = mbar_wait(&ms->full[s], par, err, true);
             if (!ok) break;
             const int q0 = it * dn_per_slot;
             const int cnt = min(dn_per_slot, sp.n_dn - q0);
@@ -857,13 +881,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     red_add_v4(yacc + (size_t)tok * d + row0, vec[0], vec[1], vec[2], vec[3]);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ms->empty[s]);
+            if (lane == 0) {
+                atomicAdd(&ms->ccnt[s], 1);
+                mbar_arrive(&ms->empty[s]);
+            }
         }
-        {
-            uint32_t par;
-            ring_s0 = slot_of(sp.n_items, par);
-            ring_p0 = par;
-        }
+        ring_base += sp.n_items;
         __threadfence();
         if (cta_failed(ok)) {
             aborted = true;
