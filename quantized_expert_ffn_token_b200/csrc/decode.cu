@@ -1122,6 +1122,24 @@ static size_t xb_y_off(const moe_config &c) { return xb_h_off(c) + (size_t)MAXU 
 size_t decode_xchg_bytes(const moe_config &c) { return xb_y_off(c) + (size_t)2 * c.d_model * 4; }
 size_t decode_xchg_counter_bytes() { return XB_LOGITS; }
 
+int decode_trace_buffer(moe_ctx *ctx, int grid, int L, int words, cudaStream_t st, unsigned long long **out) {
+    DecodeState &ds = ctx->dec;
+    size_t need = (size_t)grid * L * words;
+    if (need > ds.trace_cap) {
+        if (ds.trace) ctx_free(ctx, ds.trace);
+        ds.trace = nullptr;
+        ds.trace_cap = 0;
+        QE_CHECK(cudaSetDevice(ctx->device));
+        QE_TRY(ctx_alloc(ctx, (void **)&ds.trace, need * 8, "trace"));
+        ds.trace_cap = need;
+    }
+    QE_CHECK(cudaMemsetAsync(ds.trace, 0, need * 8, st));
+    ds.trace_n = grid * L;
+    ds.trace_words = words;
+    *out = ds.trace;
+    return MOE_OK;
+}
+
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec,
                   int rec_n, int rec_r, cudaStream_t st) {
@@ -1160,21 +1178,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     // test hook: the context's first single-token call withholds CTA 0's logits
     p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ds.withheld) ? 1 : 0;
     if (p.withhold) ds.withheld = true;
-    if (c.flags & MOE_FLAG_TRACE) {
-        size_t need = (size_t)ds.grid * L * TRACE_WORDS;
-        if (need > ds.trace_cap) {
-            if (ds.trace) ctx_free(ctx, ds.trace);
-            ds.trace = nullptr;
-            QE_CHECK(cudaSetDevice(ctx->device));
-            int s = ctx_alloc(ctx, (void **)&ds.trace, need * 8, "trace");
-            if (s != MOE_OK) return s;
-            ds.trace_cap = need;
-        }
-        QE_CHECK(cudaMemsetAsync(ds.trace, 0, need * 8, st));
-        ds.trace_n = (int)(ds.grid * L);
-        ds.trace_words = TRACE_WORDS;
-        p.trace = ds.trace;
-    }
+    if (c.flags & MOE_FLAG_TRACE) QE_TRY(decode_trace_buffer(ctx, ds.grid, L, TRACE_WORDS, st, &p.trace));
     p.nslot = ds.nslot;
     p.slot_bytes = ds.slot_bytes;
     p.rpc = ds.rpc;

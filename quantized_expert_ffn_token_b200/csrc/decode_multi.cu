@@ -55,6 +55,7 @@ struct MiscM {
     unsigned long long route;              // one arrival per layer: routing known
     int gcnt[MAX_SLOTS];                   // gate/up warps done with the unit in slot s
     int ccnt[MAX_SLOTS];                   // items of slot s consumed so far in this launch
+    int icnt[MAX_SLOTS];                   // down units of the item in slot s finished so far
     int nU;                                // experts in use this layer (routed union + shared)
     int nR;                                // routed part of the union
     int ids[TMAX][KMAX];
@@ -87,6 +88,7 @@ struct MultiParams {
     float *r_buf;                  // [2][TM][d] residual stream (stack)
     int *err;
     int withhold;
+    unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
     int off_ring, off_router, off_xb, off_red, off_xsum, off_hsum, off_uexp, off_hcum, off_wtab,
         off_misc, off_ltab;
@@ -94,6 +96,23 @@ struct MultiParams {
 
 constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;
 __device__ __forceinline__ unsigned *hctr(const MultiParams &p, int u) { return p.cnt + C_H + 8 * u; }
+
+// Phase trace (MOE_FLAG_TRACE): per (CTA, layer) record of 24 words: CTA, layer, then SM clock
+// cycles since the layer started in this CTA:
+//   0 input ready          1 logits stored        2 all logits received  3 routing known
+//   4 gate/up done         5 h of the down run's experts complete       6 h table built
+//   7 down done            8 output contributions released            9 warp 0: cycles waiting
+//  10 warp 0: cycles waiting for down data        11 previous layer's output received
+//  21 global timer (ns) at the layer start
+constexpr int TRACE_WORDS_M = 24;
+__device__ __noinline__ void mtrace_store(unsigned long long *trace, int L, int l, int ph, long long t) {
+    unsigned long long *r = trace + ((size_t)blockIdx.x * L + l) * TRACE_WORDS_M;
+    if (ph == 0) {
+        r[0] = blockIdx.x;
+        r[1] = l;
+    }
+    r[2 + ph] = (unsigned long long)t;
+}
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 __device__ __forceinline__ uint16_t f2h_bits(float v) {
@@ -211,6 +230,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             mbar_init(&ms->empty[s], 1);
             ms->gcnt[s] = 0;
             ms->ccnt[s] = 0;
+            ms->icnt[s] = 0;
         }
         mbar_init(&ms->rbar, 1);
         mbar_init(&ms->route, 1);
@@ -310,6 +330,16 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         const LayerPtrs Lp = ltab[l];
         const int yb = l & 1;                      // output buffer of this layer
         float *yacc = p.y_acc + (size_t)yb * TM * d;
+        const long long tl0 = clock64();
+        auto mark = [&](int ph, long long v) {
+            if (p.trace && tid == 0) mtrace_store(p.trace, p.L, l, ph, v);
+        };
+        if (p.trace && tid == 0) {
+            unsigned long long gt;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
+            mtrace_store(p.trace, p.L, l, 21, (long long)gt);
+        }
+        long long tw_gu = 0, tw_dn = 0;
 
         // ---- 1. layer input: xb[t] (bf16) for every token; per-token max |x| -------------------
         float amx[TMAX];
@@ -325,6 +355,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     aborted = true;
                     break;
                 }
+                mark(11, clock64() - tl0);
             }
             const float *rprev = p.r_buf + (size_t)((l + 1) & 1) * TM * d;
             const float *yprev = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
@@ -445,6 +476,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
         }
         csync();   // xb complete, operand scales known
+        mark(0, clock64() - tl0);
         // block sums of the B operand the gate/up MMAs see (fp16 of x * 2^s, or bf16 x)
         for (int i = tid; i < T * nbd; i += NT) {
             const int t = i / nbd, b = i - t * nbd;
@@ -489,6 +521,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
         }
         csync();   // this CTA's logits are stored; the router rows are no longer read
+        mark(1, clock64() - tl0);
         if (tid == 0) {
             if (!(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
             ok = ctr_wait(p.cnt + C_LOGITS, (unsigned)(G * (l + 1)), err);
@@ -497,6 +530,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             aborted = true;
             break;
         }
+        mark(2, clock64() - tl0);
         // every CTA has read the previous layer's output: clear the owned columns of its buffer,
         // which accumulates the next layer's output
         if (l >= 1 && l + 1 < p.L) {
@@ -526,7 +560,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
 #pragma unroll
                 for (int i = 0; i < EPL; ++i) {
                     const int e = lane + 32 * i;
-                    if (better(v[i], e, bv, bid)) {
+                    if (32 * i < E && better(v[i], e, bv, bid)) {
                         bv = v[i];
                         bid = e;
                     }
@@ -618,6 +652,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         }
         csync();
         if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
+        mark(3, clock64() - tl0);
         const int nU = ms->nU;
         const Split sp = split(nU);
         auto slot_of = [&](int q, uint32_t &par, int &fill) {
@@ -663,7 +698,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 uint32_t par;
                 int fill;
                 const int s = slot_of(q, par, fill);
+                const long long tw0 = clock64();
                 ok = mbar_wait(&ms->full[s], par, err, true);
+                tw_gu += clock64() - tw0;
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
                 // this lane's scales: rows g and g+8, the chunk's 8 blocks
@@ -727,6 +764,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             aborted = true;
             break;
         }
+        mark(4, clock64() - tl0);
 
         // ---- 5. down ---------------------------------------------------------------------------------
         const int u_first = sp.n_dn > 0 ? sp.dn_lo / ntile_dn : 0;
@@ -739,6 +777,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 aborted = true;
                 break;
             }
+            mark(5, clock64() - tl0);
             // h of the run's experts -> hi + lo B fragments (8 columns, zero past T) and, per
             // (expert, token, 32-block), the sum of hi + lo and (fp16) the block's 2^-s
             const int nq = n_span * TMAX * (I / 4);   // 4 values per thread and step; 8 lanes per block
@@ -802,21 +841,25 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
             csync();
         }
-        // units of this CTA's run, in batches of dn_per_slot (one ring item each); item i -> warp i % NW
-        for (int it = warp; it < sp.n_dn_items && ok; it += NW) {
-            // items go round-robin to the warps, so this warp may reach an item while its slot still
-            // holds an older one (consumed by another warp): first wait until every earlier item of
-            // the slot is consumed, then the fill parity names this item's fill unambiguously
+        mark(6, clock64() - tl0);
+        // units of this CTA's run, in batches of dn_per_slot (one ring item each); units go round-robin
+        // to the warps, and the warp that finishes an item's last unit releases its slot
+        for (int ui_all = warp; ui_all < sp.n_dn && ok; ui_all += NW) {
+            const int it = ui_all / dn_per_slot, ui = ui_all - it * dn_per_slot;
+            const int cnt = min(dn_per_slot, sp.n_dn - it * dn_per_slot);
+            // this warp may reach an item while its slot still holds an older one (consumed by other
+            // warps): first wait until every earlier item of the slot is consumed, then the fill
+            // parity names this item's fill unambiguously
             uint32_t par;
             int fill;
             const int s = slot_of(sp.n_gu + it, par, fill);
+            const long long tw0 = clock64();
             ok = smem_count_wait(&ms->ccnt[s], fill, err);
             if (ok) ok = mbar_wait(&ms->full[s], par, err, true);
+            tw_dn += clock64() - tw0;
             if (!ok) break;
-            const int q0 = it * dn_per_slot;
-            const int cnt = min(dn_per_slot, sp.n_dn - q0);
-            for (int ui = 0; ui < cnt; ++ui) {
-                const int n = sp.dn_lo + q0 + ui;
+            {
+                const int n = sp.dn_lo + ui_all;
                 const int u = n / ntile_dn, j = n - u * ntile_dn;
                 const int su = u - u_first;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
@@ -882,8 +925,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
             __syncwarp();
             if (lane == 0) {
-                atomicAdd(&ms->ccnt[s], 1);
-                mbar_arrive(&ms->empty[s]);
+                // the last unit of the item frees its slot
+                if (atomicAdd(&ms->icnt[s], 1) == cnt - 1) {
+                    ms->icnt[s] = 0;
+                    atomicAdd(&ms->ccnt[s], 1);
+                    mbar_arrive(&ms->empty[s]);
+                }
             }
         }
         ring_base += sp.n_items;
@@ -892,7 +939,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             aborted = true;
             break;
         }
+        mark(7, clock64() - tl0);
         if (tid == 0) ctr_arrive(p.cnt + C_Y);
+        mark(8, clock64() - tl0);
+        mark(9, tw_gu);
+        mark(10, tw_dn);
     }
 
     // ---- outputs of the last layer: each CTA its owned columns -------------------------------------
@@ -1060,6 +1111,7 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.err = ctx->ws.dev_error;
     p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ctx->dec.withheld) ? 1 : 0;
     if (p.withhold) ctx->dec.withheld = true;
+    if (c.flags & MOE_FLAG_TRACE) QE_TRY(decode_trace_buffer(ctx, ms.grid, L, TRACE_WORDS_M, st, &p.trace));
     p.nslot = ms.nslot;
     p.slot_bytes = ms.slot_bytes;
     p.rpc = ms.rpc;

@@ -322,6 +322,8 @@ size_t decode_multi_counter_bytes(const moe_config &c);
 int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int T, bool stack, float *resid_out,
                         uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n,
                         int rec_r0, cudaStream_t st);
+// Phase-trace buffer of the persistent decode kernels (grid x L records of `words` uint64), cleared on st.
+int decode_trace_buffer(moe_ctx *ctx, int grid, int L, int words, cudaStream_t st, unsigned long long **out);
 int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out,
                   uint16_t *y, float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n, int rec_r,
                   cudaStream_t st);
