@@ -357,14 +357,15 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
                      "achieved_tflops": step_flops / (ms_step / 1e3) / 1e12,
                      "frac": step_flops / (ms_step / 1e3) / 1e12 / peak}
     else:
-        # the single-token kernel: one launch = one token through every layer of the call
-        layers_per_launch = cfg.L
-        alg = layers_per_launch * ((cfg.k + cfg.n_shared) * expert_bytes(cfg) + router_bytes(cfg))
+        # the decode kernels run every layer of the stack in one launch (the few-token kernel: one
+        # launch per eight tokens); the timed region is one call, streaming each layer's router rows
+        # and the union of the experts its tokens chose: the step's algorithmic bytes
+        alg = step_bytes
         achieved = alg / (avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / P["hbm_gbs"], "traffic": measured_traffic(kernel, cfg.name, layers_per_launch),
+                "frac": achieved / P["hbm_gbs"], "traffic": measured_traffic(kernel, cfg.name, cfg.L),
                 "kernel": kernel, "alg_bytes_per_launch": alg, "avg_launch_ms": avg_ms,
-                "launches_per_step": launches / args.steps,
+                "timed_regions_per_step": launches / args.steps,
                 "peak_source": P["source"] + " (hbm_gbs, STREAM-style copy)"}
         step_roof = {"alg_bytes_per_step": step_bytes, "experts_streamed_per_layer": statistics.mean(unions),
                      "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,

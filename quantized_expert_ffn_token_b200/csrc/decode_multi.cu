@@ -11,7 +11,9 @@
 // One CTA per SM (cooperative launch), 12 compute warps and one producer warp
 // that issues every bulk copy into a ring of shared-memory slots.  Per layer:
 //   1. input: every CTA rebuilds all T token rows (stack: residual + rmsnorm,
-//      the residual stream living in global memory, each CTA owning a slice);
+//      the residual stream living in global memory, each CTA owning a slice;
+//      the ring, idle until the layer's routing is known, holds the rows in
+//      fp32 between the two passes);
 //   2. router: CTA c owns experts c, c+G, ...; a warp computes whole
 //      (expert, token) dot products from router rows prefetched into shared
 //      memory during the previous layer; logits are exchanged (counter 0);
@@ -23,11 +25,11 @@
 //      codes become exact fp16/bf16 operands (as in the single-token kernel)
 //      and each 32-block's partial is flushed with its scale and the offset
 //      term in fp32; the warps' k chunks meet in shared-memory sums, and the
-//      last warp of a unit applies SwiGLU, stores h and adds one arrival to
-//      that expert's h counter;
+//      last warp of a unit applies SwiGLU and stores h; one release per CTA
+//      publishes its h values (counter 2);
 //   5. down: units (u, 16-row output tile) in u-major order, a contiguous run
-//      per CTA (so a CTA touches two or three experts); once those experts' h
-//      counters are complete, h enters as hi + lo parts in B-fragment order;
+//      per CTA (so a CTA touches two or three experts); once every CTA's h is
+//      published, h enters as hi + lo parts in B-fragment order;
 //      each unit's weighted 16 x T output is added to the layer's fp32 output
 //      buffer with vector atomics; a y counter closes the layer.
 // Every wait is bounded (clock64); on timeout the kernel sets the context's
@@ -47,6 +49,8 @@ constexpr int TMAX = 8;         // tokens per launch: the eight B columns of mma
 constexpr int KMAX = 32;        // top_k limit
 constexpr int EPL = 32;         // logits per lane in the top-k (E <= 1024)
 constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
+constexpr int IN_IT = 3;
+constexpr int HB_M = 4;         // float4 loads of h in flight per thread        // float4 columns of a token row per thread in the input phase (d <= 4608)
 
 struct MiscM {
     unsigned long long full[MAX_SLOTS];
@@ -81,7 +85,7 @@ struct MultiParams {
     float *w_out;                  // single layer: [T][k] or NULL
     moe_stack_record rec;          // records: token t is record row rec_r0 + t of rec_n
     int rec_on, rec_n, rec_r0;
-    unsigned *cnt;                 // [0] logits arrivals, [32] y arrivals, [64 + 8u] h arrivals of union slot u
+    unsigned *cnt;                 // [0] logits, [32] y and [64] h arrivals (one per CTA and layer each)
     float *x_logits;               // [TM][E]
     float *x_h;                    // [UM][TM][I]
     float *y_acc;                  // [2][TM][d] layer outputs, accumulated with atomics
@@ -90,12 +94,11 @@ struct MultiParams {
     int withhold;
     unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
-    int off_ring, off_router, off_xb, off_red, off_xsum, off_hsum, off_uexp, off_hcum, off_wtab,
+    int off_ring, off_router, off_xb, off_red, off_xsum, off_hsum, off_uexp, off_wtab,
         off_misc, off_ltab;
 };
 
-constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;
-__device__ __forceinline__ unsigned *hctr(const MultiParams &p, int u) { return p.cnt + C_H + 8 * u; }
+constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;   // counters, 128 bytes apart
 
 // Phase trace (MOE_FLAG_TRACE): per (CTA, layer) record of 24 words: CTA, layer, then SM clock
 // cycles since the layer started in this CTA:
@@ -206,7 +209,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     float *xsum = reinterpret_cast<float *>(smem + p.off_xsum);       // [TM][d/32]
     float *hsum = reinterpret_cast<float *>(smem + p.off_hsum);       // [span][TM][I/32], then hinv
     int *uexp = reinterpret_cast<int *>(smem + p.off_uexp);           // [UM]
-    unsigned *hcum = reinterpret_cast<unsigned *>(smem + p.off_hcum); // [UM]
     float *wtab = reinterpret_cast<float *>(smem + p.off_wtab);       // [UM][TM]
     MiscM *ms = reinterpret_cast<MiscM *>(smem + p.off_misc);
     LayerPtrs *ltab = reinterpret_cast<LayerPtrs *>(smem + p.off_ltab);
@@ -238,7 +240,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     }
     for (int i = tid; i < p.nslot * 16 * TM; i += NTT) red[i] = 0.f;
     for (int i = tid; i < 32; i += NTT) ms->bits[i] = 0u;
-    for (int i = tid; i < p.UM; i += NTT) hcum[i] = 0u;
     for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];
     __syncthreads();
 
@@ -360,35 +361,62 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const float *rprev = p.r_buf + (size_t)((l + 1) & 1) * TM * d;
             const float *yprev = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
             float *rcur = p.r_buf + (size_t)yb * TM * d;
+            // the ring is idle until this layer's routing is known: it holds r [T][d] fp32 between
+            // the two passes (the producer's proxy fence orders these writes before its next fills)
+            float *rsm = reinterpret_cast<float *>(ring);
             // pass 1: r = r_prev + bf16(y_prev) (layer 0: r = x), sums of squares and max |r|; the
-            // owned columns of r are stored for the next layer
-            for (int i4 = tid; i4 < d4; i4 += NT) {
-                const bool own = i4 >= own_lo && i4 < own_hi;
+            // owned columns of r are stored for the next layer.  Two tokens' loads are issued
+            // before any of them is used (L2 round trips overlap; 13 warps leave 128 registers).
 #pragma unroll
-                for (int t = 0; t < TMAX; ++t) {
-                    if (t >= T) break;
-                    float4 r;
-                    if (l == 0) {
-                        const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
-                        r = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16), bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
-                    } else {
-                        const float4 a = ld_gpu4(rprev + (size_t)t * d + 4 * i4);
-                        const float4 y = ld_gpu4(yprev + (size_t)t * d + 4 * i4);
-                        const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
-                                       b3 = bf16_rn_bits(y.w);
-                        r = make_float4(a.x + bf16_bits_f(b0), a.y + bf16_bits_f(b1), a.z + bf16_bits_f(b2),
-                                        a.w + bf16_bits_f(b3));
-                        if (own && p.rec_on) {
-                            const size_t ro = ((size_t)(l - 1) * p.rec_n + p.rec_r0 + t) * d + 4 * i4;
-                            if (p.rec.y_bf16)
-                                *reinterpret_cast<uint2 *>(p.rec.y_bf16 + ro) =
-                                    make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
-                            if (p.rec.y_f32) *reinterpret_cast<float4 *>(p.rec.y_f32 + ro) = y;
+            for (int t0 = 0; t0 < TMAX; t0 += 2) {
+                if (t0 >= T) break;
+                float4 av[2][IN_IT], yv[2][IN_IT];
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+                    for (int it = 0; it < IN_IT; ++it) {
+                        const int t = t0 + tt, i4 = tid + it * NT;
+                        av[tt][it] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        yv[tt][it] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (t < T && i4 < d4) {
+                            if (l == 0) {
+                                const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
+                                av[tt][it] = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16),
+                                                         bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
+                            } else {
+                                av[tt][it] = __ldcg(reinterpret_cast<const float4 *>(rprev + (size_t)t * d + 4 * i4));
+                                yv[tt][it] = __ldcg(reinterpret_cast<const float4 *>(yprev + (size_t)t * d + 4 * i4));
+                            }
                         }
                     }
-                    if (own) *reinterpret_cast<float4 *>(rcur + (size_t)t * d + 4 * i4) = r;
-                    ssq[t] = fmaf(r.x, r.x, fmaf(r.y, r.y, fmaf(r.z, r.z, fmaf(r.w, r.w, ssq[t]))));
-                    amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(r.x), fabsf(r.y)), fmaxf(fabsf(r.z), fabsf(r.w))));
+                }
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+                    for (int it = 0; it < IN_IT; ++it) {
+                        const int t = t0 + tt, i4 = tid + it * NT;
+                        if (t >= T || i4 >= d4) continue;
+                        const bool own = i4 >= own_lo && i4 < own_hi;
+                        float4 r = av[tt][it];
+                        if (l > 0) {
+                            const float4 y = yv[tt][it];
+                            const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
+                                           b3 = bf16_rn_bits(y.w);
+                            r = make_float4(r.x + bf16_bits_f(b0), r.y + bf16_bits_f(b1), r.z + bf16_bits_f(b2),
+                                            r.w + bf16_bits_f(b3));
+                            if (own && p.rec_on) {
+                                const size_t ro = ((size_t)(l - 1) * p.rec_n + p.rec_r0 + t) * d + 4 * i4;
+                                if (p.rec.y_bf16)
+                                    *reinterpret_cast<uint2 *>(p.rec.y_bf16 + ro) =
+                                        make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+                                if (p.rec.y_f32) *reinterpret_cast<float4 *>(p.rec.y_f32 + ro) = y;
+                            }
+                        }
+                        if (own) *reinterpret_cast<float4 *>(rcur + (size_t)t * d + 4 * i4) = r;
+                        *reinterpret_cast<float4 *>(rsm + (size_t)t * d + 4 * i4) = r;
+                        ssq[t] = fmaf(r.x, r.x, fmaf(r.y, r.y, fmaf(r.z, r.z, fmaf(r.w, r.w, ssq[t]))));
+                        amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(r.x), fabsf(r.y)), fmaxf(fabsf(r.z), fabsf(r.w))));
+                    }
                 }
             }
 #pragma unroll
@@ -415,27 +443,17 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 inv[t] = 1.f / sqrtf(a / (float)d + 1e-6f);
                 amx[t] = bf16_bits_f(bf16_rn_bits(m * inv[t]));   // = max |bf16(r * inv)|
             }
-            // pass 2: x = bf16(r * inv) (r recomputed from the same loads)
-            for (int i4 = tid; i4 < d4; i4 += NT) {
-                const bool own = i4 >= own_lo && i4 < own_hi;
+            // pass 2: x = bf16(r * inv), r from shared memory
 #pragma unroll
-                for (int t = 0; t < TMAX; ++t) {
-                    if (t >= T) break;
-                    float4 r;
-                    if (l == 0) {
-                        const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
-                        r = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16), bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
-                    } else {
-                        const float4 a = ld_gpu4(rprev + (size_t)t * d + 4 * i4);
-                        const float4 y = ld_gpu4(yprev + (size_t)t * d + 4 * i4);
-                        r = make_float4(a.x + bf16_bits_f(bf16_rn_bits(y.x)), a.y + bf16_bits_f(bf16_rn_bits(y.y)),
-                                        a.z + bf16_bits_f(bf16_rn_bits(y.z)), a.w + bf16_bits_f(bf16_rn_bits(y.w)));
-                    }
+            for (int t = 0; t < TMAX; ++t) {
+                if (t >= T) break;
+                for (int i4 = tid; i4 < d4; i4 += NT) {
+                    const float4 r = *reinterpret_cast<const float4 *>(rsm + (size_t)t * d + 4 * i4);
                     const uint2 xv = make_uint2(
                         (uint32_t)bf16_rn_bits(r.x * inv[t]) | ((uint32_t)bf16_rn_bits(r.y * inv[t]) << 16),
                         (uint32_t)bf16_rn_bits(r.z * inv[t]) | ((uint32_t)bf16_rn_bits(r.w * inv[t]) << 16));
                     *reinterpret_cast<uint2 *>(xb + (size_t)t * d + 4 * i4) = xv;
-                    if (own && p.rec_on && p.rec.x_bf16)
+                    if (i4 >= own_lo && i4 < own_hi && p.rec_on && p.rec.x_bf16)
                         *reinterpret_cast<uint2 *>(p.rec.x_bf16 + ((size_t)l * p.rec_n + p.rec_r0 + t) * d + 4 * i4) = xv;
                 }
             }
@@ -548,7 +566,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = lane + 32 * i;
-                float x = (e < E) ? ld_gpu(p.x_logits + (size_t)t * E + e) : __int_as_float(0x7fc00000);
+                float x = (e < E) ? __ldcg(p.x_logits + (size_t)t * E + e) : __int_as_float(0x7fc00000);
                 if (e < E && isnan(x)) x = -INFINITY;   // a NaN logit ranks as -inf (last, by id)
                 v[i] = x;                               // past E: NaN, never chosen
             }
@@ -615,8 +633,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             if (lane < p.nsh) uexp[total + lane] = E + lane;
             const int nU = total + p.nsh;
             for (int i = lane; i < nU * TM; i += 32) wtab[i] = 0.f;
-            if (lane < nU) hcum[lane] += (unsigned)ntile_gu;
-            for (int u = 32 + lane; u < nU; u += 32) hcum[u] += (unsigned)ntile_gu;
             __syncwarp();
             // weight table: token t's j-th expert sits at union slot (ones below it in the bitmap)
             for (int i = lane; i < T * k; i += 32) {
@@ -749,11 +765,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                         p.x_h[((size_t)u * TM + t) * I + 8 * t8 + r] = silu(gs) * us_;
                     }
                     for (int i = lane; i < 16 * TM; i += 32) rs[i] = 0.f;
-                    __threadfence();
                     __syncwarp();
                     if (lane == 0) {
                         ms->gcnt[s] = 0;
-                        ctr_arrive(hctr(p, u));          // one more tile of expert slot u is done
                         atomicAdd(&ms->ccnt[s], 1);
                         mbar_arrive(&ms->empty[s]);      // the slot may be refilled
                     }
@@ -764,15 +778,15 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             aborted = true;
             break;
         }
+        // this CTA's h values are stored: one release for all of them
+        if (tid == 0) ctr_arrive(p.cnt + C_H);
         mark(4, clock64() - tl0);
 
         // ---- 5. down ---------------------------------------------------------------------------------
         const int u_first = sp.n_dn > 0 ? sp.dn_lo / ntile_dn : 0;
         const int n_span = sp.n_dn > 0 ? (sp.dn_hi - 1) / ntile_dn - u_first + 1 : 0;
         if (n_span > 0) {
-            if (tid == 0) {
-                for (int su = 0; su < n_span && ok; ++su) ok = ctr_wait(hctr(p, u_first + su), hcum[u_first + su], err);
-            }
+            if (tid == 0) ok = ctr_wait(p.cnt + C_H, (unsigned)(G * (l + 1)), err);
             if (cta_failed(ok)) {
                 aborted = true;
                 break;
@@ -781,13 +795,28 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             // h of the run's experts -> hi + lo B fragments (8 columns, zero past T) and, per
             // (expert, token, 32-block), the sum of hi + lo and (fp16) the block's 2^-s
             const int nq = n_span * TMAX * (I / 4);   // 4 values per thread and step; 8 lanes per block
-            for (int i = tid; i < nq; i += NT) {
+            for (int i0 = 0; i0 < nq; i0 += HB_M * NT) {
+              float4 hb[HB_M];   // a batch of loads in flight together, then the arithmetic
+#pragma unroll
+              for (int bq = 0; bq < HB_M; ++bq) {
+                const int i = i0 + bq * NT + tid;
+                hb[bq] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < nq) {
+                    const int su = i / (TMAX * (I / 4));
+                    const int rem = i - su * (TMAX * (I / 4));
+                    const int t = rem / (I / 4), k4 = rem - t * (I / 4);
+                    if (t < T) hb[bq] = __ldcg(reinterpret_cast<const float4 *>(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4));
+                }
+              }
+#pragma unroll
+              for (int bq = 0; bq < HB_M; ++bq) {
+                const int i = i0 + bq * NT + tid;
+                if (i >= nq) break;   // uniform across the warp (nq is a multiple of 32)
                 const int su = i / (TMAX * (I / 4));
                 const int rem = i - su * (TMAX * (I / 4));
                 const int t = rem / (I / 4), k4 = rem - t * (I / 4);
                 const bool live = t < T;
-                float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (live) hv = ld_gpu4(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4);
+                const float4 hv = hb[bq];
                 const float h4[4] = {hv.x, hv.y, hv.z, hv.w};
                 float scale = 1.f;
                 if constexpr (F16OP) {
@@ -838,6 +867,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     dst[which] = hi2[q];
                     dst[2 + which] = lo2[q];
                 }
+              }
             }
             csync();
         }
@@ -955,12 +985,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const float *rl = p.r_buf + (size_t)lb * TM * d;
             for (int i = tid; i < T * (own_hi - own_lo); i += NT) {
                 const int t = i / (own_hi - own_lo), i4 = own_lo + i - t * (own_hi - own_lo);
-                const float4 y = ld_gpu4(yl + (size_t)t * d + 4 * i4);
+                const float4 y = __ldcg(reinterpret_cast<const float4 *>(yl + (size_t)t * d + 4 * i4));
                 const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
                                b3 = bf16_rn_bits(y.w);
                 const uint2 yb2 = make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
                 if (p.stack) {
-                    const float4 r = ld_gpu4(rl + (size_t)t * d + 4 * i4);
+                    const float4 r = __ldcg(reinterpret_cast<const float4 *>(rl + (size_t)t * d + 4 * i4));
                     *reinterpret_cast<float4 *>(p.resid_out + (size_t)t * d + 4 * i4) =
                         make_float4(r.x + bf16_bits_f(b0), r.y + bf16_bits_f(b1), r.z + bf16_bits_f(b2),
                                     r.w + bf16_bits_f(b3));
@@ -985,9 +1015,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
 static int multi_tm(const moe_config &c) { return c.max_tokens < TMAX ? c.max_tokens : TMAX; }
 static int multi_um(const moe_config &c) { return multi_tm(c) * c.top_k + c.n_shared; }
 
-size_t decode_multi_counter_bytes(const moe_config &c) {
-    return (((size_t)(C_H + 8 * multi_um(c)) * 4) + 255) & ~(size_t)255;
-}
+size_t decode_multi_counter_bytes(const moe_config &) { return 512; }
 static size_t xm_logits_off(const moe_config &c) { return decode_multi_counter_bytes(c); }
 static size_t xm_h_off(const moe_config &c) {
     return xm_logits_off(c) + (((size_t)multi_tm(c) * c.n_experts * 4 + 255) & ~(size_t)255);
@@ -1040,7 +1068,6 @@ int decode_multi_setup(moe_ctx *ctx) {
     ms.off_xsum = take((size_t)TM * (c.d_model / 32) * 4);
     ms.off_hsum = take((size_t)2 * span * TM * (c.d_ff / 32) * 4);
     ms.off_uexp = take((size_t)UM * 4);
-    ms.off_hcum = take((size_t)UM * 4);
     ms.off_wtab = take((size_t)UM * TM * 4);
     ms.off_misc = take(sizeof(MiscM));
     ms.off_ltab = take((size_t)c.n_layers * sizeof(LayerPtrs));
@@ -1050,6 +1077,8 @@ int decode_multi_setup(moe_ctx *ctx) {
     while (nslot >= 2 && ((fixed + nslot * red_per_slot + 127) & ~(size_t)127) + (size_t)nslot * slot > limit) --nslot;
     if (nslot < 2) return MOE_OK;
     ms.off_red = take((size_t)nslot * red_per_slot);
+    // the input phase keeps the token rows (fp32) in the ring between its two passes
+    if ((size_t)nslot * slot < (size_t)TM * c.d_model * 4) return MOE_OK;
     ms.off_ring = (int)fixed;
     ms.nslot = nslot;
     ms.slot_bytes = slot;
@@ -1124,7 +1153,6 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.off_xsum = ms.off_xsum;
     p.off_hsum = ms.off_hsum;
     p.off_uexp = ms.off_uexp;
-    p.off_hcum = ms.off_hcum;
     p.off_wtab = ms.off_wtab;
     p.off_misc = ms.off_misc;
     p.off_ltab = ms.off_ltab;
