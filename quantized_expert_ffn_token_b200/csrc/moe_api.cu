@@ -157,6 +157,13 @@ int alloc_workspace(moe_ctx *ctx) {
     size_t xb = decode_xchg_bytes(c);
     QE_TRY(ctx_alloc(ctx, (void **)&ctx->dec.xbuf, xb, "exchange area"));
     QE_CHECK(cudaMemset(ctx->dec.xbuf, 0, xb));
+    QE_TRY(decode_split_setup(ctx));
+    if (ctx->split_layout && ctx->sdec.smem_bytes == 0) ctx->split_layout = false;   // no layer loaded yet
+    if (ctx->split_layout) {
+        size_t xs = decode_split_xchg_bytes(c);
+        QE_TRY(ctx_alloc(ctx, (void **)&ctx->sdec.xbuf, xs, "split exchange area"));
+        QE_CHECK(cudaMemset(ctx->sdec.xbuf, 0, xs));
+    }
     QE_TRY(decode_multi_setup(ctx));
     if (ctx->mdec.smem_bytes > 0) {
         size_t xm = decode_multi_xchg_bytes(c);
@@ -228,9 +235,13 @@ int load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, cudaStream_t
                              (int)d, true, Ly.gu + off * ctx->gu.expert_bytes, st));
         QE_TRY(stage(ctx, codes[2], dn_codes, w->on_device, st, &p[4], temps));
         QE_TRY(stage(ctx, scales[2], dn_sc, w->on_device, st, &p[5], temps));
-        QE_TRY(launch_repack(ctx, c.fmt, (const uint8_t *)p[4], (const uint16_t *)p[5], nullptr,
-                             nullptr, (int)n, (int)d, (int)I, false,
-                             Ly.dn + off * ctx->dn.expert_bytes, st));
+        if (ctx->split_layout)
+            QE_TRY(launch_repack_chunks(ctx, c.fmt, (const uint8_t *)p[4], (const uint16_t *)p[5], (int)n,
+                                        Ly.dn + off * ctx->chunk.expert_bytes, st));
+        else
+            QE_TRY(launch_repack(ctx, c.fmt, (const uint8_t *)p[4], (const uint16_t *)p[5], nullptr,
+                                 nullptr, (int)n, (int)d, (int)I, false,
+                                 Ly.dn + off * ctx->dn.expert_bytes, st));
         // Free staging of this part before the next to bound peak memory.
         QE_CHECK(cudaStreamSynchronize(st));
         for (void *t : temps) ctx_free(ctx, t);
@@ -253,6 +264,12 @@ int forward_layer(moe_ctx *ctx, int layer, const uint16_t *x, int T, uint16_t *y
     Workspace &ws = ctx->ws;
     int32_t *ids_ = ids ? ids : ws.ids;
     float *w_ = w ? w : ws.w;
+    if (ctx->split_layout) {   // one-token context: the split kernel (T == 1 here)
+        QE_TRY(timing_begin(ctx, st, "k_decode_split"));
+        QE_TRY(launch_decode_split(ctx, layer, 1, x, false, nullptr, y, yf, ids_, w_, nullptr, 1, 0, st));
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
     if (T >= 2 && T <= DECODE_MULTI_MAX && multi_ok(ctx)) {
         // the few-token kernel, at most eight tokens per launch, in near-equal chunks
         const moe_config &c = ctx->cfg;
@@ -323,6 +340,11 @@ int moe_create(const moe_config *cfg, int device, moe_ctx **out) {
     ctx->nx = cfg->n_experts + cfg->n_shared;
     ctx->gu = make_layout(cfg->fmt, 2 * cfg->d_ff, cfg->d_model);
     ctx->dn = make_layout(cfg->fmt, cfg->d_model, cfg->d_ff);
+    ctx->chunk = make_chunk_layout(cfg->fmt, cfg->d_model, cfg->d_ff);
+    // one token per call: the down matrices in chunk order for the split kernel (decided before any
+    // layer is loaded; the set-up turns it off when the shape does not fit that kernel)
+    ctx->split_layout = cfg->max_tokens == 1 && !(cfg->flags & MOE_FLAG_NO_DECODE_KERNEL) &&
+                        cfg->d_model % 64 == 0 && cfg->d_ff % 32 == 0;
     ctx->layers.resize(cfg->n_layers);
     int s = alloc_workspace(ctx);
     if (s != MOE_OK) {
@@ -367,6 +389,14 @@ int moe_forward_stack(moe_ctx *ctx, int layer0, int n_layers, const uint16_t *x_
     QE_CHECK(cudaSetDevice(ctx->device));
     cudaStream_t st = (cudaStream_t)stream;
     Workspace &ws = ctx->ws;
+    if (ctx->split_layout) {   // one-token context: the split kernel runs the whole stack
+        if (rec && rec->rows && rec->n_rows != 1) return MOE_ERR_INVALID_ARG;
+        QE_TRY(timing_begin(ctx, st, "k_decode_split"));
+        QE_TRY(launch_decode_split(ctx, layer0, n_layers, x_bf16, true, resid_out, nullptr, nullptr, nullptr, nullptr,
+                                   rec, 1, 0, st));
+        QE_TRY(timing_end(ctx, st));
+        return MOE_OK;
+    }
     // few tokens: the few-token kernel runs up to eight tokens per launch through the whole stack
     // (records of every row; a device row list with more than one token takes the general path)
     if (T >= 2 && T <= DECODE_MULTI_MAX && multi_ok(ctx) && (!rec || !rec->rows)) {

@@ -62,6 +62,29 @@ inline MatLayout make_layout(int fmt, int rows, int K) {
     return L;
 }
 
+// Down matrix in chunk order (the single-token split kernel, decode_split.cu; used by
+// contexts whose calls carry one token).  Per expert: for each 16-wide k chunk c16 (= one k16
+// slice of the down projection's reduction dimension, i.e. 16 SwiGLU rows), the codes of all d
+// output rows as d/64 row groups of 32 lane pieces; a piece holds the mma A fragments of the
+// group's four 16-row tiles for that slice, in the row-tile layout's bit order with "slice m of
+// the k group" read as "row tile m of the group" (so the same code-to-operand conversions apply).
+// After every chunk's codes: the scales by 32-block, [I/32][d] fp16.  Same byte count as the
+// row-tile layout.
+struct ChunkLayout {
+    int chunk_bytes = 0;       // (d / 64) * kg_bytes
+    int code_bytes = 0;        // (I / 16) * chunk_bytes
+    size_t expert_bytes = 0;   // code_bytes + (I / 32) * d * 2
+};
+
+inline ChunkLayout make_chunk_layout(int fmt, int d, int I) {
+    ChunkLayout C;
+    const int kg_bytes = (fmt == MOE_Q4B32) ? 512 : (fmt == MOE_Q2B32) ? 256 : 384;
+    C.chunk_bytes = (d / 64) * kg_bytes;
+    C.code_bytes = (I / 16) * C.chunk_bytes;
+    C.expert_bytes = (size_t)C.code_bytes + (size_t)(I / 32) * d * 2;
+    return C;
+}
+
 // Byte offset (within a tile's code area) and bit offset of the code of
 // tile row r (0..15), column k, Q4B32.
 __host__ __device__ inline void q4_code_pos(int r, int k, int *byte, int *shift) {
@@ -221,6 +244,16 @@ struct MultiState {
     uint8_t *xbuf = nullptr;   // counters, logits, h, output and residual buffers
 };
 
+// Launch plan of the single-token split kernel (decode_split.cu).
+struct SplitState {
+    int grid = 0;
+    int smem_bytes = 0;   // 0: the shape does not fit the kernel
+    int nslot = 0, slot_bytes = 0, rpc = 0;
+    int off_ring = 0, off_router = 0, off_xb = 0, off_xh = 0, off_logits = 0, off_gp = 0, off_ysm = 0,
+        off_red = 0, off_misc = 0, off_resid = 0, off_sums = 0, off_ltab = 0;
+    uint8_t *xbuf = nullptr;   // counters, logits, the two output buffers
+};
+
 // Event pairs around the dominant kernel (moe_timing_enable).
 struct Timing {
     bool on = false;
@@ -246,6 +279,11 @@ struct moe_ctx {
     qeffn::LayerPtrs *d_layers = nullptr;   // [n_layers] on the device
     qeffn::DecodeState dec;
     qeffn::MultiState mdec;
+    // one-token contexts (max_tokens == 1) keep the down matrices in chunk order for the split
+    // kernel; every other context keeps the row-tile order
+    bool split_layout = false;
+    qeffn::ChunkLayout chunk;
+    qeffn::SplitState sdec;
 };
 
 namespace qeffn {
@@ -312,6 +350,15 @@ constexpr int TC_MIN_TOKENS = DECODE_TOKENS_MAX + 1;
 int decode_setup(moe_ctx *ctx);
 size_t decode_xchg_bytes(const moe_config &c);
 size_t decode_xchg_counter_bytes();   // the counters at the start of the exchange area
+// Single-token split kernel (contexts with max_tokens == 1; down matrices in chunk order).
+bool decode_split_supported(const moe_ctx *ctx);
+int decode_split_setup(moe_ctx *ctx);
+size_t decode_split_xchg_bytes(const moe_config &c);
+int launch_decode_split(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack, float *resid_out, uint16_t *y,
+                        float *yf, int32_t *ids, float *w, const moe_stack_record *rec, int rec_n, int rec_r,
+                        cudaStream_t st);
+int launch_repack_chunks(moe_ctx *ctx, int fmt, const uint8_t *codes, const uint16_t *scales, int n_experts,
+                         uint8_t *dst, cudaStream_t st);
 // Few-token decode: 2..DECODE_MULTI_MAX tokens run the few-token kernel, up to
 // eight tokens per launch (one read of the batch's experts per layer).
 constexpr int DECODE_MULTI_MAX = 16;

@@ -1,5 +1,7 @@
 // Canonical packed tensors -> the library's private row-tile layout
 // (moe_internal.cuh).  Pure byte moves: no code or scale is changed.
+#include <string.h>
+
 #include "moe_internal.cuh"
 
 namespace qeffn {
@@ -22,6 +24,8 @@ __device__ inline int canon_code(int fmt, const uint8_t *blk, int j) {
 
 struct RepackArgs {
     int fmt, n_experts, rows, K, gate_up;
+    int chunk;                  // down matrix in chunk order (ChunkLayout) instead of row tiles
+    ChunkLayout C;
     const uint8_t *codes, *codes_up;
     const uint16_t *scales, *scales_up;
     uint8_t *dst;
@@ -40,7 +44,17 @@ __device__ inline int src_row(const RepackArgs &a, int t, int r, int *up) {
 
 __device__ inline int fetch_code(const RepackArgs &a, int e, int t, int r, int k) {
     int up;
-    int row = src_row(a, t, r, &up);
+    int row;
+    if (a.chunk) {
+        // t = k chunk, and the "k group" index of the caller (k >> 6) = group of 64 rows; the
+        // caller's k - 64 kg = 16 m + j names row tile m of the group and position j in the chunk
+        const int kg = k >> 6, k64 = k & 63;
+        row = 64 * kg + 16 * (k64 >> 4) + r;
+        k = 16 * t + (k64 & 15);
+        up = 0;
+    } else {
+        row = src_row(a, t, r, &up);
+    }
     int B = a.fmt == MOE_Q4B32 ? 16 : (a.fmt == MOE_Q2B32) ? 8 : 12;
     size_t nb = a.K / 32;
     const uint8_t *base = up ? a.codes_up : a.codes;
@@ -48,20 +62,23 @@ __device__ inline int fetch_code(const RepackArgs &a, int e, int t, int r, int k
     return canon_code(a.fmt, blk, k & 31);
 }
 
-// One thread per (expert, tile, k group, lane): writes that lane's piece.
+// One thread per (expert, tile, k group, lane): writes that lane's piece.  In chunk order the
+// "tile" is the k chunk and the "k group" the group of 64 output rows.
 __global__ void k_repack_codes(RepackArgs a) {
-    size_t n_kg = a.K / 64;
-    size_t total = (size_t)a.n_experts * a.L.n_tiles * n_kg * 32;
+    const size_t n_kg = a.chunk ? a.rows / 64 : a.K / 64;
+    const int n_tiles = a.chunk ? a.K / 16 : a.L.n_tiles;
+    size_t total = (size_t)a.n_experts * n_tiles * n_kg * 32;
     for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
          id += (size_t)gridDim.x * blockDim.x) {
         int lane = id & 31;
         size_t rest = id >> 5;
         int kg = rest % n_kg;
         rest /= n_kg;
-        int t = rest % a.L.n_tiles;
-        int e = rest / a.L.n_tiles;
+        int t = rest % n_tiles;
+        int e = rest / n_tiles;
         int g = lane >> 2, c = lane & 3;
-        uint8_t *tile = a.dst + (size_t)e * a.L.expert_bytes + (size_t)t * a.L.tile_bytes;
+        uint8_t *tile = a.chunk ? a.dst + (size_t)e * a.C.expert_bytes + (size_t)t * a.C.chunk_bytes
+                                : a.dst + (size_t)e * a.L.expert_bytes + (size_t)t * a.L.tile_bytes;
         if (a.fmt == MOE_Q4B32) {
             uint32_t words[4];
             for (int m = 0; m < 4; ++m) {
@@ -112,6 +129,22 @@ __global__ void k_repack_codes(RepackArgs a) {
     }
 }
 
+// Scales of the down matrix in chunk order: [I/32 blocks][d rows] after the expert's codes.
+__global__ void k_repack_scales_chunks(RepackArgs a) {
+    const int nb = a.K / 32;
+    const size_t total = (size_t)a.n_experts * a.rows * nb;
+    for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
+         id += (size_t)gridDim.x * blockDim.x) {
+        const int row = id % a.rows;
+        const size_t rest = id / a.rows;
+        const int blk = rest % nb;
+        const int e = rest / nb;
+        const uint16_t v = a.scales[((size_t)e * a.rows + row) * nb + blk];
+        uint8_t *ex = a.dst + (size_t)e * a.C.expert_bytes + a.C.code_bytes;
+        reinterpret_cast<uint16_t *>(ex)[(size_t)blk * a.rows + row] = v;
+    }
+}
+
 __global__ void k_repack_scales(RepackArgs a) {
     int nb = a.K / 32;
     size_t total = (size_t)a.n_experts * a.L.n_tiles * 16 * nb;
@@ -149,10 +182,34 @@ int launch_repack(moe_ctx *ctx, int fmt, const uint8_t *codes, const uint16_t *s
     a.scales_up = scales_up;
     a.dst = dst;
     a.L = gate_up ? ctx->gu : ctx->dn;
+    a.chunk = 0;
     k_repack_codes<<<1184, 256, 0, st>>>(a);
     QE_CHECK_LAUNCH("k_repack_codes");
     k_repack_scales<<<1184, 256, 0, st>>>(a);
     QE_CHECK_LAUNCH("k_repack_scales");
+    return MOE_OK;
+}
+
+int launch_repack_chunks(moe_ctx *ctx, int fmt, const uint8_t *codes, const uint16_t *scales, int n_experts,
+                         uint8_t *dst, cudaStream_t st) {
+    const moe_config &c = ctx->cfg;
+    RepackArgs a;
+    memset(&a, 0, sizeof(a));
+    a.fmt = fmt;
+    a.n_experts = n_experts;
+    a.rows = c.d_model;
+    a.K = c.d_ff;
+    a.gate_up = 0;
+    a.codes = codes;
+    a.scales = scales;
+    a.dst = dst;
+    a.L = ctx->dn;
+    a.chunk = 1;
+    a.C = ctx->chunk;
+    k_repack_codes<<<1184, 256, 0, st>>>(a);
+    QE_CHECK_LAUNCH("k_repack_codes");
+    k_repack_scales_chunks<<<1184, 256, 0, st>>>(a);
+    QE_CHECK_LAUNCH("k_repack_scales_chunks");
     return MOE_OK;
 }
 

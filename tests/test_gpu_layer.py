@@ -153,6 +153,67 @@ def test_few_token_wait_times_out_and_context_recovers():
     s.close()
 
 
+@pytest.mark.parametrize("fmt", ["q4", "q3", "q2"])
+def test_split_kernel_tiny_against_oracle(fmt):
+    """One-token contexts (max_tokens = 1) run the split kernel (gate/up and the matching slice of
+    the down projection per 16-row unit, the shared expert during the logits exchange): several
+    single tokens against the oracle."""
+    capi, session = _cuda()
+    cfg = {"q4": TINY, "q3": TINY_Q3, "q2": TINY_Q2}[fmt]
+    sess = session.Session(cfg, max_tokens=1)
+    sess.load_synthetic()
+    W = synth.layer_weights(cfg, 0)
+    for s in range(6):
+        x = _tokens(cfg, 1, stream=300 + s)
+        gy, gyf, gids, gw = _run(sess, 0, x)
+        assert capi.moe_get_device_error(sess.ctx) == 0
+        o = oracle.moe_layer(cfg.fmt, cfg.k, x, W)
+        check_rows(cfg, ExpertSource(cfg, 0), x, [0], gy, gyf, gids, gw, o=o)
+    sess.close()
+
+
+@pytest.mark.parametrize("name", ["decode_48l_q4_t1", "verify_48l_q3_t4_zipf", "decode_q2"])
+def test_split_kernel_matches_single_token_kernel(name):
+    """The split kernel (one-token context) against the single-token kernel (a context that allows
+    two tokens, called with one): same ids, weights within 1e-6, fp32 outputs within 1e-4 relative
+    L2 (both remove the code offset per block in fp32)."""
+    capi, session = _cuda()
+    cfg = {"decode_q2": DECODE_Q2}.get(name) or synth.CONFIGS[name]
+    a = session.Session(cfg, max_tokens=1, n_layers=1)
+    b = session.Session(cfg, max_tokens=2, n_layers=1, flags=capi.MOE_FLAG_NO_MULTI_DECODE)
+    W = synth.layer_weights(cfg, 0, device="cuda")
+    a.load(0, W)
+    b.load(0, W)
+    del W
+    for s in range(4):
+        x = _tokens(cfg, 1, stream=600 + s)
+        ya, yfa, ida, wa = _run(a, 0, x)
+        yb, yfb, idb, wb = _run(b, 0, x)
+        assert capi.moe_get_device_error(a.ctx) == 0
+        assert np.array_equal(ida, idb)
+        assert np.max(np.abs(wa - wb)) <= 1e-6
+        assert rel_l2(yfa, yfb) <= (1e-4 if cfg.fmt == "q2" else 5e-5)
+    a.close()
+    b.close()
+
+
+def test_split_wait_times_out_and_context_recovers():
+    """The split kernel's bounded waits: CTA 0 withholds its logits in the context's first call,
+    the waits give up, MOE_ERR_DEVICE_TIMEOUT is reported, and later calls are correct."""
+    capi, session = _cuda()
+    s = session.Session(TINY, max_tokens=1, n_layers=1, flags=capi.MOE_FLAG_TEST_WITHHOLD)
+    s.load_synthetic()
+    x = _tokens(TINY, 1, stream=79)
+    _run(s, 0, x)
+    assert capi.moe_get_device_error(s.ctx) == capi.MOE_ERR_DEVICE_TIMEOUT
+    o = oracle.moe_layer(TINY.fmt, TINY.k, x, synth.layer_weights(TINY, 0))
+    for rep in range(2):
+        gy, gyf, gids, gw = _run(s, 0, x)
+        assert capi.moe_get_device_error(s.ctx) == 0
+        check_rows(TINY, ExpertSource(TINY, 0), x, [0], gy, gyf, gids, gw, o=o)
+    s.close()
+
+
 def test_batch_equals_single_tokens():
     """Token independence of the CUDA-core grouped path: a token's output does not
     depend on which other tokens share the call (bit for bit).  Pinned to that
