@@ -48,16 +48,16 @@ using namespace dec;
 constexpr int TMAX = 8;         // tokens per launch: the eight B columns of mma.m16n8k16
 constexpr int KMAX = 32;        // top_k limit
 constexpr int EPL = 32;         // logits per lane in the top-k (E <= 1024)
+constexpr int CANDM = 64;       // top-k candidates per token held for ranking
 constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
-constexpr int IN_IT = 3;
-constexpr int HB_M = 4;         // float4 loads of h in flight per thread        // float4 columns of a token row per thread in the input phase (d <= 4608)
+constexpr int IN_IT = 2;        // float4 columns of a token row per thread in the input phase (d <= 3072)
+constexpr int HB_M = 4;         // float4 loads of h in flight per thread
 
 struct MiscM {
     unsigned long long full[MAX_SLOTS];
     unsigned long long empty[MAX_SLOTS];   // one arrival per consumed item
     unsigned long long rbar;
     unsigned long long route;              // one arrival per layer: routing known
-    int gcnt[MAX_SLOTS];                   // gate/up warps done with the unit in slot s
     int ccnt[MAX_SLOTS];                   // items of slot s consumed so far in this launch
     int icnt[MAX_SLOTS];                   // down units of the item in slot s finished so far
     int nU;                                // experts in use this layer (routed union + shared)
@@ -67,6 +67,7 @@ struct MiscM {
     unsigned bits[32];                     // union bitmap over E <= 1024
     float xinv[TMAX];                      // 2^-s of a token's fp16 operand (1 for bf16 operands)
     float xscale[TMAX];                    // 2^s
+    float2 cand[TMAX][CANDM];              // top-k candidates of each token: (logit, id bits)
     float ss[NW][TMAX];                    // per-warp sums of squares / maxima of the input phase
     float mx[NW][TMAX];
 };
@@ -94,7 +95,7 @@ struct MultiParams {
     int withhold;
     unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
-    int off_ring, off_router, off_xb, off_red, off_xsum, off_hsum, off_uexp, off_wtab,
+    int off_ring, off_router, off_xb, off_xsum, off_hsum, off_uexp, off_wtab,
         off_misc, off_ltab;
 };
 
@@ -118,13 +119,6 @@ __device__ __noinline__ void mtrace_store(unsigned long long *trace, int L, int 
 }
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
-__device__ __forceinline__ uint16_t f2h_bits(float v) {
-    __half h = __float2half_rn(v);
-    return *reinterpret_cast<uint16_t *>(&h);
-}
-__device__ __forceinline__ float h_bits_f(uint16_t b) {
-    return __half2float(*reinterpret_cast<const __half *>(&b));
-}
 __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -205,7 +199,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     float *rtr = reinterpret_cast<float *>(smem + p.off_router);
     uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_xb);     // [TM][d] bf16 input; then the h table
     uint8_t *htab = smem + p.off_xb;
-    float *red = reinterpret_cast<float *>(smem + p.off_red);         // [nslot][16][TM]
     float *xsum = reinterpret_cast<float *>(smem + p.off_xsum);       // [TM][d/32]
     float *hsum = reinterpret_cast<float *>(smem + p.off_hsum);       // [span][TM][I/32], then hinv
     int *uexp = reinterpret_cast<int *>(smem + p.off_uexp);           // [UM]
@@ -219,9 +212,10 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     const int d = p.d, E = p.E, I = p.I, k = p.k, T = p.T, TM = p.TM;
     const int nbd = d / 32, nbi = I / 32, nkgi = I / 64;
     const int ntile_gu = I / 8, ntile_dn = d / 16;
-    const int GW = d / 256;                          // warps with a gate/up k chunk
     const int dn_per_slot = p.slot_bytes / p.dn.tile_bytes;
     const int d4 = d / 4;
+    const int XS = d + 8;   // row stride of the token rows in shared memory (halves): rows 16 bytes apart
+                            // in bank order, so the 8 rows' B fragments load without conflicts
     const int own_lo = cta * d4 / G, own_hi = (cta + 1) * d4 / G;   // float4 columns this CTA owns
     float *hinv = hsum + p.span * TM * nbi;
     int *err = p.err;
@@ -230,7 +224,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         for (int s = 0; s < p.nslot; ++s) {
             mbar_init(&ms->full[s], 1);
             mbar_init(&ms->empty[s], 1);
-            ms->gcnt[s] = 0;
             ms->ccnt[s] = 0;
             ms->icnt[s] = 0;
         }
@@ -238,7 +231,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         mbar_init(&ms->route, 1);
         fence_mbar_init();
     }
-    for (int i = tid; i < p.nslot * 16 * TM; i += NTT) red[i] = 0.f;
     for (int i = tid; i < 32; i += NTT) ms->bits[i] = 0u;
     for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];
     __syncthreads();
@@ -365,14 +357,14 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             // the two passes (the producer's proxy fence orders these writes before its next fills)
             float *rsm = reinterpret_cast<float *>(ring);
             // pass 1: r = r_prev + bf16(y_prev) (layer 0: r = x), sums of squares and max |r|; the
-            // owned columns of r are stored for the next layer.  Two tokens' loads are issued
+            // owned columns of r are stored for the next layer.  Four tokens' loads are issued
             // before any of them is used (L2 round trips overlap; 13 warps leave 128 registers).
 #pragma unroll
-            for (int t0 = 0; t0 < TMAX; t0 += 2) {
+            for (int t0 = 0; t0 < TMAX; t0 += 4) {
                 if (t0 >= T) break;
-                float4 av[2][IN_IT], yv[2][IN_IT];
+                float4 av[4][IN_IT], yv[4][IN_IT];
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
+                for (int tt = 0; tt < 4; ++tt) {
 #pragma unroll
                     for (int it = 0; it < IN_IT; ++it) {
                         const int t = t0 + tt, i4 = tid + it * NT;
@@ -391,7 +383,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     }
                 }
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
+                for (int tt = 0; tt < 4; ++tt) {
 #pragma unroll
                     for (int it = 0; it < IN_IT; ++it) {
                         const int t = t0 + tt, i4 = tid + it * NT;
@@ -452,7 +444,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     const uint2 xv = make_uint2(
                         (uint32_t)bf16_rn_bits(r.x * inv[t]) | ((uint32_t)bf16_rn_bits(r.y * inv[t]) << 16),
                         (uint32_t)bf16_rn_bits(r.z * inv[t]) | ((uint32_t)bf16_rn_bits(r.w * inv[t]) << 16));
-                    *reinterpret_cast<uint2 *>(xb + (size_t)t * d + 4 * i4) = xv;
+                    *reinterpret_cast<uint2 *>(xb + (size_t)t * XS + 4 * i4) = xv;
                     if (i4 >= own_lo && i4 < own_hi && p.rec_on && p.rec.x_bf16)
                         *reinterpret_cast<uint2 *>(p.rec.x_bf16 + ((size_t)l * p.rec_n + p.rec_r0 + t) * d + 4 * i4) = xv;
                 }
@@ -463,7 +455,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 for (int t = 0; t < TMAX; ++t) {
                     if (t >= T) break;
                     const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
-                    *reinterpret_cast<uint2 *>(xb + (size_t)t * d + 4 * i4) = xv;
+                    *reinterpret_cast<uint2 *>(xb + (size_t)t * XS + 4 * i4) = xv;
                     amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(bf16f(xv.x & 0xFFFFu)), fabsf(bf16f(xv.x >> 16))),
                                                  fmaxf(fabsf(bf16f(xv.y & 0xFFFFu)), fabsf(bf16f(xv.y >> 16)))));
                 }
@@ -495,21 +487,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         }
         csync();   // xb complete, operand scales known
         mark(0, clock64() - tl0);
-        // block sums of the B operand the gate/up MMAs see (fp16 of x * 2^s, or bf16 x)
-        for (int i = tid; i < T * nbd; i += NT) {
-            const int t = i / nbd, b = i - t * nbd;
-            const uint16_t *src = xb + (size_t)t * d + 32 * b;
-            float acc = 0.f;
-            if constexpr (F16OP) {
-                const float sc = ms->xscale[t];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) acc += h_bits_f(f2h_bits(bf16_bits_f(src[j]) * sc));
-            } else {
-                acc = sum32_bf16(src);
-            }
-            xsum[t * nbd + b] = acc;
-        }
-
         // ---- 2. router: warp w computes the (row, token) pairs w, w + NW, ... ----------------------
         {
             int nrows = 0;
@@ -523,7 +500,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             for (int pr = warp; pr < nrows * T; pr += NW) {
                 const int j = pr / T, t = pr - j * T;
                 const float *wr = rtr + (size_t)j * d;
-                const uint16_t *xr = xb + (size_t)t * d;
+                const uint16_t *xr = xb + (size_t)t * XS;
                 float acc = 0.f;
                 for (int i4 = lane; i4 < d4; i4 += 32) {
                     const float4 wv = *reinterpret_cast<const float4 *>(wr + 4 * i4);
@@ -538,10 +515,34 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 if (lane == 0) p.x_logits[(size_t)t * E + e] = acc + __ldg(Lp.rb + e);
             }
         }
-        csync();   // this CTA's logits are stored; the router rows are no longer read
+        csync();   // this CTA's logits are stored; the router rows and the bf16 rows are no longer read
+        if (tid == 0 && !(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
         mark(1, clock64() - tl0);
+        // the gate/up B operand in place of the bf16 rows (fp16 of x * 2^s for fp16 code operands),
+        // and its 32-block sums (the offset removal in the gate/up flush)
+        if constexpr (F16OP) {
+            for (int i = tid; i < T * (d / 8); i += NT) {
+                const int t = i / (d / 8), i8 = i - t * (d / 8);
+                uint4 *pv = reinterpret_cast<uint4 *>(xb + (size_t)t * XS + 8 * i8);
+                const uint4 v = *pv;
+                const float sc = ms->xscale[t];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __half2 h2 = __floats2half2_rn(bf16f(w[j] & 0xFFFFu) * sc, bf16f(w[j] >> 16) * sc);
+                    o[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                *pv = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            csync();
+        }
+        for (int i = tid; i < T * nbd; i += NT) {
+            const int t = i / nbd, b = i - t * nbd;
+            const uint16_t *src = xb + (size_t)t * XS + 32 * b;
+            xsum[t * nbd + b] = F16OP ? sum32_f16(src) : sum32_bf16(src);
+        }
         if (tid == 0) {
-            if (!(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
             ok = ctr_wait(p.cnt + C_LOGITS, (unsigned)(G * (l + 1)), err);
         }
         if (cta_failed(ok)) {
@@ -560,55 +561,107 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         }
 
         // ---- 3. top-k per token (warp t), union, weights --------------------------------------------
+        // Threshold and rank: the k-th largest of the 32 lanes' maxima is a lower bound of the k-th
+        // largest logit, so every expert of the top k is among the values at or above it; those
+        // candidates are ranked by counting the candidates ordered before each (larger logit, equal
+        // logits: lower id).  Too many candidates (flat or equal logits): k rounds of warp arg-max.
         if (warp < T) {
             const int t = warp;
             float v[EPL];
+            float lmax = -INFINITY;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = lane + 32 * i;
                 float x = (e < E) ? __ldcg(p.x_logits + (size_t)t * E + e) : __int_as_float(0x7fc00000);
                 if (e < E && isnan(x)) x = -INFINITY;   // a NaN logit ranks as -inf (last, by id)
-                v[i] = x;                               // past E: NaN, never chosen
+                v[i] = x;                               // past E: NaN, never a candidate
+                if (e < E) lmax = fmaxf(lmax, x);
             }
-            float top = -INFINITY, z = 0.f, pj = 0.f;
-            int myid = -1;
-            for (int j = 0; j < k; ++j) {
-                float bv = -INFINITY;
-                int bid = 0x7fffffff;
+            int rk = 0;
+            for (int j = 0; j < 32; ++j) {
+                const float mj = __shfl_sync(0xffffffffu, lmax, j);
+                rk += (mj > lmax) || (mj == lmax && j < lane);
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, rk == k - 1);
+            const float tau = __shfl_sync(0xffffffffu, lmax, __ffs(hit) - 1);
+            int mine = 0;
 #pragma unroll
-                for (int i = 0; i < EPL; ++i) {
-                    const int e = lane + 32 * i;
-                    if (32 * i < E && better(v[i], e, bv, bid)) {
-                        bv = v[i];
-                        bid = e;
+            for (int i = 0; i < EPL; ++i) mine += (32 * i < E) && (v[i] >= tau);
+            int incl = mine;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nb;
+            }
+            const int ncand = __shfl_sync(0xffffffffu, incl, 31);
+            float2 *cand = ms->cand[t];
+            int pv_id = -1;
+            float pv = -INFINITY;
+            if (ncand <= CANDM) {
+                int pos = incl - mine;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if ((32 * i < E) && v[i] >= tau) cand[pos++] = make_float2(v[i], __int_as_float(lane + 32 * i));
+                __syncwarp();
+                for (int ci = lane; ci < ncand; ci += 32) {
+                    const float2 me = cand[ci];
+                    const int id = __float_as_int(me.y);
+                    int r = 0;
+                    for (int j = 0; j < ncand; ++j) {
+                        const float2 o = cand[j];
+                        r += better(o.x, __float_as_int(o.y), me.x, id);
+                    }
+                    if (r < k) {
+                        ms->ids[t][r] = id;
+                        ms->w[t][r] = me.x;   // the logit for now; the weight below
                     }
                 }
-                for (int o = 16; o; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-                    if (better(ov, oid, bv, bid)) {
-                        bv = ov;
-                        bid = oid;
+                __syncwarp();
+                if (lane < k) {
+                    pv_id = ms->ids[t][lane];
+                    pv = ms->w[t][lane];
+                }
+            } else {
+                for (int j = 0; j < k; ++j) {
+                    float bv = -INFINITY;
+                    int bid = 0x7fffffff;
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) {
+                        const int e = lane + 32 * i;
+                        if (32 * i < E && better(v[i], e, bv, bid)) {
+                            bv = v[i];
+                            bid = e;
+                        }
+                    }
+                    for (int o = 16; o; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                        const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+                        if (better(ov, oid, bv, bid)) {
+                            bv = ov;
+                            bid = oid;
+                        }
+                    }
+                    if (bid >= E) bid = 0;   // unreachable while k <= E
+                    if ((bid & 31) == lane) {
+#pragma unroll
+                        for (int i = 0; i < EPL; ++i)
+                            if (lane + 32 * i == bid) v[i] = __int_as_float(0x7fc00000);   // taken
+                    }
+                    if (lane == j) {
+                        pv_id = bid;
+                        pv = bv;
                     }
                 }
-                if (bid >= E) bid = 0;   // unreachable while k <= E
-                if (j == 0) top = bv;
-                if ((bid & 31) == lane) {
-#pragma unroll
-                    for (int i = 0; i < EPL; ++i)
-                        if (lane + 32 * i == bid) v[i] = __int_as_float(0x7fc00000);   // taken
-                }
-                const float pe = expf(bv - top);
-                if (lane == j) {
-                    myid = bid;
-                    pj = pe;
-                }
-                z += pe;
             }
+            // softmax over the chosen logits, in rank order
+            const float top = __shfl_sync(0xffffffffu, pv, 0);
+            const float pe = lane < k ? expf(pv - top) : 0.f;
+            float z = pe;
+            for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            __syncwarp();
             if (lane < k) {
-                ms->ids[t][lane] = myid;
-                ms->w[t][lane] = pj / z;
-                atomicOr(&ms->bits[myid >> 5], 1u << (myid & 31));
+                ms->ids[t][lane] = pv_id;
+                ms->w[t][lane] = pe / z;
+                atomicOr(&ms->bits[pv_id >> 5], 1u << (pv_id & 31));
             }
         }
         csync();
@@ -678,99 +731,68 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             return a - fill * p.nslot;
         };
 
-        // ---- 4. gate/up ------------------------------------------------------------------------------
-        if (warp < GW) {
-            // B fragments of this warp's 256-wide k chunk: column g = token g (zero past T)
-            uint32_t bx0[16], bx1[16];
-            {
-                const bool live = g < T;
-                const uint16_t *xr = xb + (size_t)(live ? g : 0) * d + 256 * warp + 2 * c;
-                const float sc = live ? ms->xscale[g] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const uint32_t v0 = live ? *reinterpret_cast<const uint32_t *>(xr + 16 * j) : 0u;
-                    const uint32_t v1 = live ? *reinterpret_cast<const uint32_t *>(xr + 16 * j + 8) : 0u;
-                    if constexpr (F16OP) {
-                        const __half2 h0 = __floats2half2_rn(bf16f(v0 & 0xFFFFu) * sc, bf16f(v0 >> 16) * sc);
-                        const __half2 h1 = __floats2half2_rn(bf16f(v1 & 0xFFFFu) * sc, bf16f(v1 >> 16) * sc);
-                        bx0[j] = *reinterpret_cast<const uint32_t *>(&h0);
-                        bx1[j] = *reinterpret_cast<const uint32_t *>(&h1);
-                    } else {
-                        bx0[j] = v0;
-                        bx1[j] = v1;
-                    }
-                }
-            }
-            // block sums of the operand for this lane's columns (tokens 2c, 2c+1), this chunk's 8 blocks
-            float xs0[8], xs1[8];
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                xs0[b] = (2 * c < T) ? xsum[(2 * c) * nbd + 8 * warp + b] : 0.f;
-                xs1[b] = (2 * c + 1 < T) ? xsum[(2 * c + 1) * nbd + 8 * warp + b] : 0.f;
-            }
-            for (int q = 0; q < sp.n_gu && ok; ++q) {
-                // every gate/up warp consumes every unit in order, so the slot's previous item is one
-                // this warp has finished: the parity below cannot refer to an older fill
+        // ---- 4. gate/up: a warp takes whole units (both matrices' 8 rows over all of K) ----------------
+        // Units go round-robin to the warps; a unit's warp may reach its item while the slot still
+        // holds an older item consumed by another warp, so it first waits until every earlier item of
+        // the slot is consumed.  B operand: column g = token g (zero past T), from the token rows.
+        {
+            const bool live = g < T;
+            const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 2 * c;
+            const int t0 = 2 * c, t1 = 2 * c + 1;
+            const bool l0 = t0 < T, l1 = t1 < T;
+            const float *xs0 = xsum + (size_t)min(t0, TM - 1) * nbd;
+            const float *xs1 = xsum + (size_t)min(t1, TM - 1) * nbd;
+            const int nkg = d / 64;
+            for (int q = warp; q < sp.n_gu && ok; q += NW) {
                 uint32_t par;
                 int fill;
                 const int s = slot_of(q, par, fill);
                 const long long tw0 = clock64();
-                ok = mbar_wait(&ms->full[s], par, err, true);
+                ok = smem_count_wait(&ms->ccnt[s], fill, err);
+                if (ok) ok = mbar_wait(&ms->full[s], par, err, true);
                 tw_gu += clock64() - tw0;
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
-                // this lane's scales: rows g and g+8, the chunk's 8 blocks
-                const uint4 sgv = *reinterpret_cast<const uint4 *>(tile + p.gu.code_bytes + ((size_t)g * nbd + 8 * warp) * 2);
-                const uint4 s8v = *reinterpret_cast<const uint4 *>(tile + p.gu.code_bytes + ((size_t)(g + 8) * nbd + 8 * warp) * 2);
-                const uint32_t sgw[4] = {sgv.x, sgv.y, sgv.z, sgv.w}, s8w[4] = {s8v.x, s8v.y, s8v.z, s8v.w};
+                const __half *sc = reinterpret_cast<const __half *>(tile + p.gu.code_bytes);
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq) {
+#pragma unroll 2
+                for (int kg = 0; kg < nkg; ++kg) {
                     uint32_t a[16];
-                    frag16<FMT>(tile + (size_t)(4 * warp + kq) * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
+                    frag16<FMT>(tile + (size_t)kg * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
+                    uint32_t b0[4], b1[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        b0[m] = live ? *reinterpret_cast<const uint32_t *>(xr + 64 * kg + 16 * m) : 0u;
+                        b1[m] = live ? *reinterpret_cast<const uint32_t *>(xr + 64 * kg + 16 * m + 8) : 0u;
+                    }
                     float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_fmt<FMT>(Da, a + 0, bx0[4 * kq + 0], bx1[4 * kq + 0]);
-                    mma_fmt<FMT>(Da, a + 4, bx0[4 * kq + 1], bx1[4 * kq + 1]);
-                    mma_fmt<FMT>(Db, a + 8, bx0[4 * kq + 2], bx1[4 * kq + 2]);
-                    mma_fmt<FMT>(Db, a + 12, bx0[4 * kq + 3], bx1[4 * kq + 3]);
-                    const float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(&sgw[kq]));
-                    const float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(&s8w[kq]));
-                    flush_block<FMT>(acc, Da, sg.x, s8.x, xs0[2 * kq], xs1[2 * kq], false);
-                    flush_block<FMT>(acc, Db, sg.y, s8.y, xs0[2 * kq + 1], xs1[2 * kq + 1], true);
+                    mma_fmt<FMT>(Da, a + 0, b0[0], b1[0]);
+                    mma_fmt<FMT>(Da, a + 4, b0[1], b1[1]);
+                    mma_fmt<FMT>(Db, a + 8, b0[2], b1[2]);
+                    mma_fmt<FMT>(Db, a + 12, b0[3], b1[3]);
+                    const int bl = 2 * kg;
+                    const float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + bl));
+                    const float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + bl));
+                    const float v00 = l0 ? xs0[bl] : 0.f, v10 = l1 ? xs1[bl] : 0.f;
+                    const float v01 = l0 ? xs0[bl + 1] : 0.f, v11 = l1 ? xs1[bl + 1] : 0.f;
+                    flush_block<FMT>(acc, Da, sg.x, s8.x, v00, v10, false);
+                    flush_block<FMT>(acc, Db, sg.y, s8.y, v01, v11, true);
                 }
-                // the chunk's partial of rows g, g+8 for tokens 2c, 2c+1 into the unit's sums
-                float *rs = red + (size_t)s * 16 * TM;
-                if (2 * c < T) {
-                    atomicAdd(rs + g * TM + 2 * c, acc[0]);
-                    atomicAdd(rs + (g + 8) * TM + 2 * c, acc[2]);
+                // rows g (gate) and g + 8 (up) of the unit for tokens 2c, 2c + 1: SwiGLU in place
+                const int n = cta + G * q;
+                const int u = n / ntile_gu, t8 = n - u * ntile_gu;
+                if (l0) {
+                    const float xi = ms->xinv[t0];
+                    p.x_h[((size_t)u * TM + t0) * I + 8 * t8 + g] = silu(acc[0] * xi) * (acc[2] * xi);
                 }
-                if (2 * c + 1 < T) {
-                    atomicAdd(rs + g * TM + 2 * c + 1, acc[1]);
-                    atomicAdd(rs + (g + 8) * TM + 2 * c + 1, acc[3]);
+                if (l1) {
+                    const float xi = ms->xinv[t1];
+                    p.x_h[((size_t)u * TM + t1) * I + 8 * t8 + g] = silu(acc[1] * xi) * (acc[3] * xi);
                 }
-                __threadfence_block();
                 __syncwarp();
-                int last = 0;
-                if (lane == 0) last = atomicAdd(&ms->gcnt[s], 1) == GW - 1;
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    // every warp's share is in: SwiGLU of the unit's 8 rows for every token
-                    __threadfence_block();
-                    const int n = cta + G * q;
-                    const int u = n / ntile_gu, t8 = n - u * ntile_gu;
-                    for (int i = lane; i < 8 * T; i += 32) {
-                        const int r = i & 7, t = i >> 3;
-                        const float xi = ms->xinv[t];
-                        const float gs = rs[r * TM + t] * xi, us_ = rs[(8 + r) * TM + t] * xi;
-                        p.x_h[((size_t)u * TM + t) * I + 8 * t8 + r] = silu(gs) * us_;
-                    }
-                    for (int i = lane; i < 16 * TM; i += 32) rs[i] = 0.f;
-                    __syncwarp();
-                    if (lane == 0) {
-                        ms->gcnt[s] = 0;
-                        atomicAdd(&ms->ccnt[s], 1);
-                        mbar_arrive(&ms->empty[s]);      // the slot may be refilled
-                    }
+                if (lane == 0) {
+                    atomicAdd(&ms->ccnt[s], 1);
+                    mbar_arrive(&ms->empty[s]);      // the slot may be refilled
                 }
             }
         }
@@ -1032,7 +1054,7 @@ bool decode_multi_supported(const moe_ctx *ctx) {
     const moe_config &c = ctx->cfg;
     if (c.flags & MOE_FLAG_NO_DECODE_KERNEL) return false;
     if (c.max_tokens < 2) return false;
-    if (c.d_model > 4096 || c.d_model / 256 > NW || c.n_experts > 32 * EPL || c.n_experts % 4) return false;
+    if (c.d_model > 2 * 4 * NT || c.d_model / 256 > NW || c.n_experts > 32 * EPL || c.n_experts % 4) return false;
     if (c.top_k > KMAX) return false;
     return ctx->mdec.smem_bytes > 0;
 }
@@ -1061,7 +1083,7 @@ int decode_multi_setup(moe_ctx *ctx) {
         fixed = (fixed + bytes + 127) & ~(size_t)127;
         return off;
     };
-    const size_t xb_bytes = (size_t)TM * c.d_model * 2;
+    const size_t xb_bytes = (size_t)TM * (c.d_model + 8) * 2;
     const size_t htab_bytes = (size_t)span * (c.d_ff / 64) * 4 * 32 * 16;
     ms.off_router = take((size_t)rpc * c.d_model * 4);
     ms.off_xb = take(xb_bytes > htab_bytes ? xb_bytes : htab_bytes);
@@ -1071,12 +1093,10 @@ int decode_multi_setup(moe_ctx *ctx) {
     ms.off_wtab = take((size_t)UM * TM * 4);
     ms.off_misc = take(sizeof(MiscM));
     ms.off_ltab = take((size_t)c.n_layers * sizeof(LayerPtrs));
-    const size_t red_per_slot = (size_t)16 * TM * 4;
     size_t limit = (size_t)prop.sharedMemPerBlockOptin;
     int nslot = MAX_SLOTS;
-    while (nslot >= 2 && ((fixed + nslot * red_per_slot + 127) & ~(size_t)127) + (size_t)nslot * slot > limit) --nslot;
+    while (nslot >= 2 && fixed + (size_t)nslot * slot > limit) --nslot;
     if (nslot < 2) return MOE_OK;
-    ms.off_red = take((size_t)nslot * red_per_slot);
     // the input phase keeps the token rows (fp32) in the ring between its two passes
     if ((size_t)nslot * slot < (size_t)TM * c.d_model * 4) return MOE_OK;
     ms.off_ring = (int)fixed;
@@ -1149,7 +1169,6 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.off_ring = ms.off_ring;
     p.off_router = ms.off_router;
     p.off_xb = ms.off_xb;
-    p.off_red = ms.off_red;
     p.off_xsum = ms.off_xsum;
     p.off_hsum = ms.off_hsum;
     p.off_uexp = ms.off_uexp;

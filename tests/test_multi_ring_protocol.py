@@ -4,12 +4,14 @@ One CTA, one layer, random interleavings of the producer (fills items in
 order, refilling a slot once its previous item is consumed) and the compute
 warps:
 
-* gate/up items: every gate/up warp reads every unit in order; the warp that
-  finishes a unit last frees its slot (counter per slot);
+* gate/up items: one unit each; units go round-robin to all warps, and the
+  unit's warp frees the slot;
 * down items: batches of units; units go round-robin to all warps, the warp
-  that finishes an item's last unit frees the slot; before waiting on a slot
-  a unit's warp waits until every earlier item of that slot is consumed, so
-  the fill parity it waits on names its own item.
+  that finishes an item's last unit frees the slot;
+* before waiting on a slot, a unit's warp waits until every earlier item of
+  that slot is consumed, so the fill parity it waits on names its own item;
+* every warp finishes its gate/up units before any down unit starts (the
+  kernel's barrier and its grid-wide h exchange).
 
 mbarriers are modelled with their phase-parity semantics (a wait on parity P
 passes once the phase with parity P has completed, i.e. while the current
@@ -43,11 +45,11 @@ class Stale(AssertionError):
     pass
 
 
-def run(nslot, n_gu, n_dn, dps, GW=10, NW=12, seed=0, gate_on_earlier=True, free_on_last=True):
+def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_last=True):
     rnd = random.Random(seed)
     full = [MBar(1) for _ in range(nslot)]
     empty = [MBar(1) for _ in range(nslot)]
-    gcnt, ccnt, icnt = [0] * nslot, [0] * nslot, [0] * nslot
+    ccnt, icnt = [0] * nslot, [0] * nslot
     n_dn_items = (n_dn + dps - 1) // dps
     n_items = n_gu + n_dn_items
     content = [None] * nslot           # item in the slot
@@ -57,7 +59,7 @@ def run(nslot, n_gu, n_dn, dps, GW=10, NW=12, seed=0, gate_on_earlier=True, free
     def slot(a):
         return a % nslot, (a // nslot) & 1, a // nslot
 
-    warps = [{"ph": "gu" if w < GW else "wait", "q": 0, "u": w, "busy": None} for w in range(NW)]
+    warps = [{"ph": "gu", "q": w, "u": w, "busy": None} for w in range(NW)]
     for _ in range(400000):
         actors = (["p"] if prod["q"] < n_items else []) + [w for w in range(NW) if warps[w]["ph"] != "done"]
         if not actors:
@@ -86,17 +88,16 @@ def run(nslot, n_gu, n_dn, dps, GW=10, NW=12, seed=0, gate_on_earlier=True, free
                     ws["ph"] = "wait"
                     moved = True
                     break
-                s, par, _ = slot(q)
+                s, par, fill = slot(q)
+                if gate_on_earlier and ccnt[s] < fill:
+                    continue
                 if not full[s].try_wait(par):
                     continue
                 if content[s] != q:
                     raise Stale(f"gate/up unit {q} read slot {s} holding item {content[s]}")
-                gcnt[s] += 1
-                if gcnt[s] == GW:
-                    gcnt[s] = 0
-                    ccnt[s] += 1
-                    empty[s].arrive()
-                ws["q"] += 1
+                ccnt[s] += 1
+                empty[s].arrive()
+                ws["q"] += NW
                 moved = True
                 break
             if ws["ph"] == "wait":
