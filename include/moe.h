@@ -89,8 +89,10 @@ typedef struct {
 } moe_config;
 
 /* moe_config.flags: test and diagnostic hooks, 0 in normal use (no page has a
- * counterpart).  The first two pin a call to one implementation (tests
- * compare the paths with each other); MOE_FLAG_TRACE records the decode
+ * counterpart).  The NO_* flags pin a call to one implementation (tests
+ * compare the paths with each other); MOE_FLAG_SPLIT_DECODE selects an
+ * alternative single-token kernel (measured slower on this shape, kept for
+ * comparison); MOE_FLAG_TRACE records the decode
  * kernel's phase clocks; MOE_FLAG_TEST_WITHHOLD is a test hook for the
  * bounded device waits: in the context's first single-token call the decode
  * kernel's CTA 0 withholds its router logits, every wait on them runs out
@@ -99,6 +101,7 @@ typedef struct {
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* small T runs the general path, not the single-token kernel */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
 #define MOE_FLAG_NO_MULTI_DECODE 8    /* 2..16 tokens run the single-token kernel per token, not the few-token kernel */
+#define MOE_FLAG_SPLIT_DECODE 16      /* with max_tokens == 1: the split single-token kernel (down projection by k chunk) */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
 #define MOE_FLAG_TRACE 4              /* record per-phase timestamps (moe_trace_read) */
 

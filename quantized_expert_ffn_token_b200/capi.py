@@ -29,6 +29,7 @@ MOE_Q2B32 = 3
 MOE_FLAG_NO_DECODE_KERNEL = 1
 MOE_FLAG_NO_TENSOR_PREFILL = 2
 MOE_FLAG_NO_MULTI_DECODE = 8
+MOE_FLAG_SPLIT_DECODE = 16
 MOE_FLAG_TEST_WITHHOLD = 256
 MOE_FLAG_TRACE = 4
 MOE_ROUTE_STATIC_MAX_LOGITS = 65536

@@ -754,9 +754,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
                 const __half *sc = reinterpret_cast<const __half *>(tile + p.gu.code_bytes);
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                // two accumulator chains (even and odd k groups), summed at the end: the flushes of
+                // consecutive k groups do not wait on each other
+                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 2
                 for (int kg = 0; kg < nkg; ++kg) {
+                    float *acc = acc2[kg & 1];
                     uint32_t a[16];
                     frag16<FMT>(tile + (size_t)kg * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
                     uint32_t b0[4], b1[4];
@@ -778,6 +781,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     flush_block<FMT>(acc, Da, sg.x, s8.x, v00, v10, false);
                     flush_block<FMT>(acc, Db, sg.y, s8.y, v01, v11, true);
                 }
+                const float acc[4] = {acc2[0][0] + acc2[1][0], acc2[0][1] + acc2[1][1], acc2[0][2] + acc2[1][2],
+                                      acc2[0][3] + acc2[1][3]};
                 // rows g (gate) and g + 8 (up) of the unit for tokens 2c, 2c + 1: SwiGLU in place
                 const int n = cta + G * q;
                 const int u = n / ntile_gu, t8 = n - u * ntile_gu;
@@ -916,14 +921,16 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const int su = u - u_first;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
                 const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 const int t0 = 2 * c, t1 = 2 * c + 1;
                 const float *hs0 = hsum + (su * TM + min(t0, TM - 1)) * nbi;
                 const float *hs1 = hsum + (su * TM + min(t1, TM - 1)) * nbi;
                 const float *hi0 = hinv + (su * TM + min(t0, TM - 1)) * nbi;
                 const float *hi1 = hinv + (su * TM + min(t1, TM - 1)) * nbi;
                 const bool l0 = t0 < T, l1 = t1 < T;
+#pragma unroll 2
                 for (int kg = 0; kg < nkgi; ++kg) {
+                    float *acc = acc2[kg & 1];   // two accumulator chains (even and odd k groups)
                     uint32_t a[16];
                     frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
                     float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
@@ -954,6 +961,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                         }
                     }
                 }
+                const float acc[4] = {acc2[0][0] + acc2[1][0], acc2[0][1] + acc2[1][1], acc2[0][2] + acc2[1][2],
+                                      acc2[0][3] + acc2[1][3]};
                 // weighted by each token's routing weight for this expert, then 4 consecutive rows of
                 // one token per lane (a 4 x 4 transpose among the lanes g = 4m' .. 4m' + 3 of a column
                 // pair) for one vector atomic each

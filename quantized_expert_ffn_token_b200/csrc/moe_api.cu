@@ -341,10 +341,10 @@ int moe_create(const moe_config *cfg, int device, moe_ctx **out) {
     ctx->gu = make_layout(cfg->fmt, 2 * cfg->d_ff, cfg->d_model);
     ctx->dn = make_layout(cfg->fmt, cfg->d_model, cfg->d_ff);
     ctx->chunk = make_chunk_layout(cfg->fmt, cfg->d_model, cfg->d_ff);
-    // one token per call: the down matrices in chunk order for the split kernel (decided before any
-    // layer is loaded; the set-up turns it off when the shape does not fit that kernel)
-    ctx->split_layout = cfg->max_tokens == 1 && !(cfg->flags & MOE_FLAG_NO_DECODE_KERNEL) &&
-                        cfg->d_model % 64 == 0 && cfg->d_ff % 32 == 0;
+    // one token per call and MOE_FLAG_SPLIT_DECODE: the down matrices in chunk order for the split
+    // kernel (decided before any layer is loaded; the set-up turns it off when the shape does not fit)
+    ctx->split_layout = (cfg->flags & MOE_FLAG_SPLIT_DECODE) && cfg->max_tokens == 1 &&
+                        !(cfg->flags & MOE_FLAG_NO_DECODE_KERNEL) && cfg->d_model % 64 == 0 && cfg->d_ff % 32 == 0;
     ctx->layers.resize(cfg->n_layers);
     int s = alloc_workspace(ctx);
     if (s != MOE_OK) {

@@ -14,7 +14,7 @@ from tests.parity import (W_TOL, ExpertSource, HostLayer, bf16_tol, bits_to_f64,
 pytestmark = pytest.mark.gpu
 
 
-def _stack(name, rows=None, check_layers=None, dense=False, layer0_all=False):
+def _stack(name, rows=None, check_layers=None, dense=False, layer0_all=False, flags=0):
     """The whole stack through the C ABI with per-layer records of `rows` (all
     when None), checked layer by layer against the oracle (teacher-forced).
     dense: the oracle evaluates each layer's rows with per-expert fp64 matrix
@@ -26,7 +26,7 @@ def _stack(name, rows=None, check_layers=None, dense=False, layer0_all=False):
     from quantized_expert_ffn_token_b200 import capi, session
     cfg = synth.CONFIGS[name] if isinstance(name, str) else name
     L, T, d, k = cfg.L, cfg.T, cfg.d, cfg.k
-    sess = session.Session(cfg, max_tokens=T)
+    sess = session.Session(cfg, max_tokens=T, flags=flags)
     sess.load_synthetic()
     x_bits = synth.tokens_bf16(cfg)
     x = torch.from_numpy(x_bits.view(np.int16)).cuda()
@@ -98,6 +98,12 @@ def test_decode_stack_48_layers():
 
 def test_verify_stack_48_layers():
     _stack("verify_48l_q3_t4_zipf")
+
+
+def test_split_kernel_stack_48_layers():
+    """The 48-layer Q4 decode stack through the split single-token kernel (MOE_FLAG_SPLIT_DECODE)."""
+    from quantized_expert_ffn_token_b200 import capi
+    _stack("decode_48l_q4_t1", flags=capi.MOE_FLAG_SPLIT_DECODE)
 
 
 def test_few_token_stack_48_layers_13_tokens():
