@@ -1,5 +1,6 @@
-// Few-token decode (2..8 tokens per launch): one persistent kernel runs whole
-// layers (and the whole 48-layer stack) for a small batch of tokens, reading
+// Few-token decode (2..8 tokens per launch; the host runs 9..16 tokens as two
+// launches): one persistent kernel runs whole layers (and the whole 48-layer
+// stack) for a small batch of tokens, reading
 // the union of the batch's experts once per layer.  This is the step that
 // checks several guessed tokens at once ("Strata: Qwen3.8-Flash-Next (125B
 // Moe) on a 8GB+ Nvidia GPU", README section "How does it work": guess, then
@@ -10,10 +11,11 @@
 //
 // One CTA per SM (cooperative launch), 12 compute warps and one producer warp
 // that issues every bulk copy into a ring of shared-memory slots.  Per layer:
-//   1. input: every CTA rebuilds all T token rows (stack: residual + rmsnorm,
-//      the residual stream living in global memory, each CTA owning a slice;
-//      the ring, idle until the layer's routing is known, holds the rows in
-//      fp32 between the two passes);
+//   1. input: every CTA rebuilds all T token rows (stack: r = r_prev + bf16(y),
+//      rmsnorm, bf16 x).  The residual stream lives in global memory, each CTA
+//      storing the slice of columns it owns; r_prev is loaded into the idle
+//      ring at the end of the previous layer, so only the layer output is read
+//      after the output exchange;
 //   2. router: CTA c owns experts c, c+G, ...; a warp computes whole
 //      (expert, token) dot products from router rows prefetched into shared
 //      memory during the previous layer; logits are exchanged (counter 0);
@@ -24,14 +26,16 @@
 //      order; the tokens sit in the MMA's B columns (column t = token t), the
 //      codes become exact fp16/bf16 operands (as in the single-token kernel)
 //      and each 32-block's partial is flushed with its scale and the offset
-//      term in fp32; the warps' k chunks meet in shared-memory sums, and the
-//      last warp of a unit applies SwiGLU and stores h; one release per CTA
-//      publishes its h values (counter 2);
+//      term in fp32.  Inside a CTA the units' k-group steps are cut into 12
+//      near-equal ranges, one per warp; a unit cut by a range boundary meets
+//      in shared-memory sums and its last part applies SwiGLU and stores h;
+//      one release per CTA publishes its h values (counter 2);
 //   5. down: units (u, 16-row output tile) in u-major order, a contiguous run
-//      per CTA (so a CTA touches two or three experts); once every CTA's h is
-//      published, h enters as hi + lo parts in B-fragment order;
-//      each unit's weighted 16 x T output is added to the layer's fp32 output
-//      buffer with vector atomics; a y counter closes the layer.
+//      per CTA (so a CTA touches two or three experts), round-robin over its
+//      warps; once every CTA's h is published, h enters as hi + lo parts in
+//      B-fragment order; each unit's weighted 16 x T output is added to the
+//      layer's fp32 output buffer with vector atomics; a y counter closes the
+//      layer.
 // Every wait is bounded (clock64); on timeout the kernel sets the context's
 // error word and every CTA leaves.  The host zeroes the counters and the
 // output buffers before each launch.
@@ -47,7 +51,7 @@ using namespace dec;
 
 constexpr int TMAX = 8;         // tokens per launch: the eight B columns of mma.m16n8k16
 constexpr int KMAX = 32;        // top_k limit
-constexpr int EPL = 32;         // logits per lane in the top-k (E <= 1024)
+constexpr int EPL = 16;         // logits per lane in the top-k (E <= 512)
 constexpr int CANDM = 64;       // top-k candidates per token held for ranking
 constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
 constexpr int IN_IT = 2;        // float4 columns of a token row per thread in the input phase (d <= 3072)
@@ -65,11 +69,19 @@ struct MiscM {
     int ids[TMAX][KMAX];
     float w[TMAX][KMAX];
     unsigned bits[32];                     // union bitmap over E <= 1024
+    int wpre[32];                          // union slots below each bitmap word
     float xinv[TMAX];                      // 2^-s of a token's fp16 operand (1 for bf16 operands)
     float xscale[TMAX];                    // 2^s
-    float2 cand[TMAX][CANDM];              // top-k candidates of each token: (logit, id bits)
+    union {
+        float2 cand[TMAX][CANDM];          // top-k: candidates of each token (logit, id bits)
+        float pacc[NW - 1][32][4];         // gate/up: sums of a unit cut by warp boundaries, by its first warp
+    };
+    int pcnt[NW - 1];                      // gate/up: parts of that unit finished
     float ss[NW][TMAX];                    // per-warp sums of squares / maxima of the input phase
     float mx[NW][TMAX];
+    float tinv[TMAX];                      // 1 / rms of each token's residual row
+    float tmax[TMAX];                      // max |x| of each token's input row
+    float rbias[8];                        // router bias of this CTA's expert rows
 };
 
 struct MultiParams {
@@ -107,6 +119,11 @@ constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;   // counters, 128 bytes apart
 //   4 gate/up done         5 h of the down run's experts complete       6 h table built
 //   7 down done            8 output contributions released            9 warp 0: cycles waiting
 //  10 warp 0: cycles waiting for down data        11 previous layer's output received
+//  12 input pass 1 done (thread 0)                13 input sums of squares combined
+//  14 input pass 2 done (thread 0)                15 router rows landed
+//  16 operand conversion and block sums done      17 top-k: logits loaded (warp 0)
+//  18 top-k: candidates ranked (warp 0)           19 all tokens' top-k done
+//  20 union and weight table built
 //  21 global timer (ns) at the layer start
 constexpr int TRACE_WORDS_M = 24;
 __device__ __noinline__ void mtrace_store(unsigned long long *trace, int L, int l, int ph, long long t) {
@@ -232,6 +249,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         fence_mbar_init();
     }
     for (int i = tid; i < 32; i += NTT) ms->bits[i] = 0u;
+    for (int i = tid; i < NW - 1; i += NTT) ms->pcnt[i] = 0;
     for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];
     __syncthreads();
 
@@ -333,15 +351,17 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             mtrace_store(p.trace, p.L, l, 21, (long long)gt);
         }
         long long tw_gu = 0, tw_dn = 0;
+        if (tid < p.rpc && cta + G * tid < E) ms->rbias[tid] = __ldg(Lp.rb + cta + G * tid);
 
         // ---- 1. layer input: xb[t] (bf16) for every token; per-token max |x| -------------------
-        float amx[TMAX];
-#pragma unroll
-        for (int t = 0; t < TMAX; ++t) amx[t] = 0.f;
+        // The ring is idle until this layer's routing is known: it holds the token rows r [T][d] in
+        // fp32 (rsm) from the end of the previous layer through both passes (the producer's proxy
+        // fence orders these writes before its next fills).
+        float *rsm = reinterpret_cast<float *>(ring);
         if (p.stack) {
-            float ssq[TMAX];
+            float ssq[TMAX], amx[TMAX];
 #pragma unroll
-            for (int t = 0; t < TMAX; ++t) ssq[t] = 0.f;
+            for (int t = 0; t < TMAX; ++t) ssq[t] = amx[t] = 0.f;
             if (l > 0) {
                 if (tid == 0) ok = ctr_wait(p.cnt + C_Y, (unsigned)(G * l), err);
                 if (cta_failed(ok)) {
@@ -350,34 +370,28 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
                 mark(11, clock64() - tl0);
             }
-            const float *rprev = p.r_buf + (size_t)((l + 1) & 1) * TM * d;
             const float *yprev = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
             float *rcur = p.r_buf + (size_t)yb * TM * d;
-            // the ring is idle until this layer's routing is known: it holds r [T][d] fp32 between
-            // the two passes (the producer's proxy fence orders these writes before its next fills)
-            float *rsm = reinterpret_cast<float *>(ring);
-            // pass 1: r = r_prev + bf16(y_prev) (layer 0: r = x), sums of squares and max |r|; the
-            // owned columns of r are stored for the next layer.  Four tokens' loads are issued
-            // before any of them is used (L2 round trips overlap; 13 warps leave 128 registers).
+            // pass 1: r = r_prev + bf16(y_prev) (layer 0: r = x), with r_prev already in rsm; sums
+            // of squares and max |r|; the owned columns of r are stored for the next layer.  Four
+            // tokens' loads are issued before any of them is used.
 #pragma unroll
             for (int t0 = 0; t0 < TMAX; t0 += 4) {
                 if (t0 >= T) break;
-                float4 av[4][IN_IT], yv[4][IN_IT];
+                float4 av[4][IN_IT];
 #pragma unroll
                 for (int tt = 0; tt < 4; ++tt) {
 #pragma unroll
                     for (int it = 0; it < IN_IT; ++it) {
                         const int t = t0 + tt, i4 = tid + it * NT;
                         av[tt][it] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        yv[tt][it] = make_float4(0.f, 0.f, 0.f, 0.f);
                         if (t < T && i4 < d4) {
                             if (l == 0) {
                                 const uint2 xv = *reinterpret_cast<const uint2 *>(p.x_in + (size_t)t * d + 4 * i4);
                                 av[tt][it] = make_float4(bf16f(xv.x & 0xFFFFu), bf16f(xv.x >> 16),
                                                          bf16f(xv.y & 0xFFFFu), bf16f(xv.y >> 16));
                             } else {
-                                av[tt][it] = __ldcg(reinterpret_cast<const float4 *>(rprev + (size_t)t * d + 4 * i4));
-                                yv[tt][it] = __ldcg(reinterpret_cast<const float4 *>(yprev + (size_t)t * d + 4 * i4));
+                                av[tt][it] = __ldcg(reinterpret_cast<const float4 *>(yprev + (size_t)t * d + 4 * i4));
                             }
                         }
                     }
@@ -389,13 +403,14 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                         const int t = t0 + tt, i4 = tid + it * NT;
                         if (t >= T || i4 >= d4) continue;
                         const bool own = i4 >= own_lo && i4 < own_hi;
+                        float4 *rp = reinterpret_cast<float4 *>(rsm + (size_t)t * d + 4 * i4);
                         float4 r = av[tt][it];
                         if (l > 0) {
-                            const float4 y = yv[tt][it];
+                            const float4 y = r, rv = *rp;
                             const uint16_t b0 = bf16_rn_bits(y.x), b1 = bf16_rn_bits(y.y), b2 = bf16_rn_bits(y.z),
                                            b3 = bf16_rn_bits(y.w);
-                            r = make_float4(r.x + bf16_bits_f(b0), r.y + bf16_bits_f(b1), r.z + bf16_bits_f(b2),
-                                            r.w + bf16_bits_f(b3));
+                            r = make_float4(rv.x + bf16_bits_f(b0), rv.y + bf16_bits_f(b1), rv.z + bf16_bits_f(b2),
+                                            rv.w + bf16_bits_f(b3));
                             if (own && p.rec_on) {
                                 const size_t ro = ((size_t)(l - 1) * p.rec_n + p.rec_r0 + t) * d + 4 * i4;
                                 if (p.rec.y_bf16)
@@ -405,14 +420,16 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                             }
                         }
                         if (own) *reinterpret_cast<float4 *>(rcur + (size_t)t * d + 4 * i4) = r;
-                        *reinterpret_cast<float4 *>(rsm + (size_t)t * d + 4 * i4) = r;
+                        *rp = r;
                         ssq[t] = fmaf(r.x, r.x, fmaf(r.y, r.y, fmaf(r.z, r.z, fmaf(r.w, r.w, ssq[t]))));
                         amx[t] = fmaxf(amx[t], fmaxf(fmaxf(fabsf(r.x), fabsf(r.y)), fmaxf(fabsf(r.z), fabsf(r.w))));
                     }
                 }
             }
+            mark(12, clock64() - tl0);
 #pragma unroll
             for (int t = 0; t < TMAX; ++t) {
+                if (t >= T) break;
                 float a = ssq[t], m = amx[t];
                 for (int o = 16; o; o >>= 1) {
                     a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -424,32 +441,38 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
             }
             csync();
-            float inv[TMAX];
-#pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
+            // token t's statistics, once (lane 0 of warp t, the warps' sums in warp order)
+            if (warp < T && lane == 0) {
+                const int t = warp;
                 float a = 0.f, m = 0.f;
                 for (int w = 0; w < NW; ++w) {
                     a += ms->ss[w][t];
                     m = fmaxf(m, ms->mx[w][t]);
                 }
-                inv[t] = 1.f / sqrtf(a / (float)d + 1e-6f);
-                amx[t] = bf16_bits_f(bf16_rn_bits(m * inv[t]));   // = max |bf16(r * inv)|
+                const float inv = 1.f / sqrtf(a / (float)d + 1e-6f);
+                ms->tinv[t] = inv;
+                ms->tmax[t] = bf16_bits_f(bf16_rn_bits(m * inv));   // = max |bf16(r * inv)|
             }
+            csync();
+            mark(13, clock64() - tl0);
             // pass 2: x = bf16(r * inv), r from shared memory
-#pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
-                if (t >= T) break;
-                for (int i4 = tid; i4 < d4; i4 += NT) {
-                    const float4 r = *reinterpret_cast<const float4 *>(rsm + (size_t)t * d + 4 * i4);
-                    const uint2 xv = make_uint2(
-                        (uint32_t)bf16_rn_bits(r.x * inv[t]) | ((uint32_t)bf16_rn_bits(r.y * inv[t]) << 16),
-                        (uint32_t)bf16_rn_bits(r.z * inv[t]) | ((uint32_t)bf16_rn_bits(r.w * inv[t]) << 16));
-                    *reinterpret_cast<uint2 *>(xb + (size_t)t * XS + 4 * i4) = xv;
-                    if (i4 >= own_lo && i4 < own_hi && p.rec_on && p.rec.x_bf16)
-                        *reinterpret_cast<uint2 *>(p.rec.x_bf16 + ((size_t)l * p.rec_n + p.rec_r0 + t) * d + 4 * i4) = xv;
-                }
+            for (int i = tid; i < T * d4; i += NT) {
+                const int t = i / d4, i4 = i - t * d4;
+                const float inv = ms->tinv[t];
+                const float4 r = *reinterpret_cast<const float4 *>(rsm + (size_t)t * d + 4 * i4);
+                const uint2 xv = make_uint2(
+                    (uint32_t)bf16_rn_bits(r.x * inv) | ((uint32_t)bf16_rn_bits(r.y * inv) << 16),
+                    (uint32_t)bf16_rn_bits(r.z * inv) | ((uint32_t)bf16_rn_bits(r.w * inv) << 16));
+                *reinterpret_cast<uint2 *>(xb + (size_t)t * XS + 4 * i4) = xv;
+                if (i4 >= own_lo && i4 < own_hi && p.rec_on && p.rec.x_bf16)
+                    *reinterpret_cast<uint2 *>(p.rec.x_bf16 + ((size_t)l * p.rec_n + p.rec_r0 + t) * d + 4 * i4) = xv;
             }
+            fence_proxy_async();   // these generic writes to the ring before the producer's next fills
+            mark(14, clock64() - tl0);
         } else {
+            float amx[TMAX];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) amx[t] = 0.f;
             for (int i4 = tid; i4 < d4; i4 += NT) {
 #pragma unroll
                 for (int t = 0; t < TMAX; ++t) {
@@ -462,30 +485,28 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
 #pragma unroll
             for (int t = 0; t < TMAX; ++t) {
+                if (t >= T) break;
                 float m = amx[t];
                 for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
                 if (lane == 0) ms->mx[warp][t] = m;
             }
             csync();
-#pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
+            if (warp < T && lane == 0) {
                 float m = 0.f;
-                for (int w = 0; w < NW; ++w) m = fmaxf(m, ms->mx[w][t]);
-                amx[t] = m;
+                for (int w = 0; w < NW; ++w) m = fmaxf(m, ms->mx[w][warp]);
+                ms->tmax[warp] = m;
             }
         }
+        csync();   // xb and the token maxima complete
         // fp16 operand scale of every token: 2^s with max |x| * 2^s < 2^15 (exact for bf16 inputs)
-#pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
-            if (t == tid) {
-                int xe;
-                frexpf(amx[t], &xe);
-                const int s = min(15 - xe, 100);
-                ms->xscale[t] = F16OP ? pow2i(s) : 1.f;
-                ms->xinv[t] = F16OP ? pow2i(-s) : 1.f;
-            }
+        if (tid < T) {
+            int xe;
+            frexpf(ms->tmax[tid], &xe);
+            const int s = min(15 - xe, 100);
+            ms->xscale[tid] = F16OP ? pow2i(s) : 1.f;
+            ms->xinv[tid] = F16OP ? pow2i(-s) : 1.f;
         }
-        csync();   // xb complete, operand scales known
+        csync();   // operand scales known
         mark(0, clock64() - tl0);
         // ---- 2. router: warp w computes the (row, token) pairs w, w + NW, ... ----------------------
         {
@@ -497,6 +518,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 aborted = true;
                 break;
             }
+            mark(15, clock64() - tl0);
             for (int pr = warp; pr < nrows * T; pr += NW) {
                 const int j = pr / T, t = pr - j * T;
                 const float *wr = rtr + (size_t)j * d;
@@ -512,7 +534,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
                 for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
                 const int e = cta + G * j;
-                if (lane == 0) p.x_logits[(size_t)t * E + e] = acc + __ldg(Lp.rb + e);
+                if (lane == 0) p.x_logits[(size_t)t * E + e] = acc + ms->rbias[j];
             }
         }
         csync();   // this CTA's logits are stored; the router rows and the bf16 rows are no longer read
@@ -542,6 +564,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const uint16_t *src = xb + (size_t)t * XS + 32 * b;
             xsum[t * nbd + b] = F16OP ? sum32_f16(src) : sum32_bf16(src);
         }
+        mark(16, clock64() - tl0);
         if (tid == 0) {
             ok = ctr_wait(p.cnt + C_LOGITS, (unsigned)(G * (l + 1)), err);
         }
@@ -577,6 +600,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 v[i] = x;                               // past E: NaN, never a candidate
                 if (e < E) lmax = fmaxf(lmax, x);
             }
+            mark(17, clock64() - tl0);
             int rk = 0;
             for (int j = 0; j < 32; ++j) {
                 const float mj = __shfl_sync(0xffffffffu, lmax, j);
@@ -601,14 +625,18 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
 #pragma unroll
                 for (int i = 0; i < EPL; ++i)
                     if ((32 * i < E) && v[i] >= tau) cand[pos++] = make_float2(v[i], __int_as_float(lane + 32 * i));
+                // padded to a multiple of 4 with entries ordered after every candidate
+                const int npad = (ncand + 3) & ~3;
+                if (lane < npad - ncand) cand[ncand + lane] = make_float2(-INFINITY, __int_as_float(0x7fffffff));
                 __syncwarp();
                 for (int ci = lane; ci < ncand; ci += 32) {
                     const float2 me = cand[ci];
                     const int id = __float_as_int(me.y);
                     int r = 0;
-                    for (int j = 0; j < ncand; ++j) {
-                        const float2 o = cand[j];
-                        r += better(o.x, __float_as_int(o.y), me.x, id);
+                    for (int j = 0; j < npad; j += 4) {
+                        const float2 o0 = cand[j], o1 = cand[j + 1], o2 = cand[j + 2], o3 = cand[j + 3];
+                        r += better(o0.x, __float_as_int(o0.y), me.x, id) + better(o1.x, __float_as_int(o1.y), me.x, id) +
+                             better(o2.x, __float_as_int(o2.y), me.x, id) + better(o3.x, __float_as_int(o3.y), me.x, id);
                     }
                     if (r < k) {
                         ms->ids[t][r] = id;
@@ -652,6 +680,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     }
                 }
             }
+            mark(18, clock64() - tl0);
             // softmax over the chosen logits, in rank order
             const float top = __shfl_sync(0xffffffffu, pv, 0);
             const float pe = lane < k ? expf(pv - top) : 0.f;
@@ -665,6 +694,12 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
         }
         csync();
+        mark(19, clock64() - tl0);
+        if (warp != 0) {
+            // the gate/up part sums share memory with the top-k candidates: zero them
+            float *pz = &ms->pacc[0][0][0];
+            for (int i = tid - 32; i < (NW - 1) * 32 * 4; i += NT - 32) pz[i] = 0.f;
+        }
         if (warp == 0) {
             // union in ascending expert order, then the shared experts
             const int nwords = (E + 31) / 32;
@@ -676,6 +711,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
             const int total = __shfl_sync(0xffffffffu, pre, 31);
             pre -= __popc(word);   // exclusive
+            ms->wpre[lane] = pre;
             unsigned wv = word;
             int pos = pre;
             while (wv) {
@@ -692,8 +728,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const int t = i / k, j = i - t * k;
                 const int e = ms->ids[t][j];
                 const int wi = e >> 5;
-                int slot = __popc(ms->bits[wi] & ((1u << (e & 31)) - 1u));
-                for (int q = 0; q < wi; ++q) slot += __popc(ms->bits[q]);
+                const int slot = ms->wpre[wi] + __popc(ms->bits[wi] & ((1u << (e & 31)) - 1u));
                 wtab[slot * TM + t] = ms->w[t][j];
             }
             for (int i = lane; i < p.nsh * T; i += 32) wtab[(total + i / T) * TM + i % T] = 1.f;
@@ -719,6 +754,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
             }
         }
+        mark(20, clock64() - tl0);
         csync();
         if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
         mark(3, clock64() - tl0);
@@ -731,10 +767,14 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             return a - fill * p.nslot;
         };
 
-        // ---- 4. gate/up: a warp takes whole units (both matrices' 8 rows over all of K) ----------------
-        // Units go round-robin to the warps; a unit's warp may reach its item while the slot still
-        // holds an older item consumed by another warp, so it first waits until every earlier item of
-        // the slot is consumed.  B operand: column g = token g (zero past T), from the token rows.
+        // ---- 4. gate/up: balanced ranges of (unit, k group) steps ----------------------------------
+        // The CTA's units times the d/64 k groups form one sequence of steps, cut into NW near-equal
+        // contiguous ranges, one per warp; a warp's range covers whole units plus at most a partial
+        // first and last unit.  A unit cut by warp boundaries is summed in shared memory (slot = its
+        // first warp) and its last part to finish applies SwiGLU and frees the slot.  Before waiting
+        // on a unit's fill, a warp waits until every earlier item of the slot is consumed (a later
+        // unit can reach a slot that still holds an older item).  B operand: column g = token g (zero
+        // past T), from the token rows.
         {
             const bool live = g < T;
             const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 2 * c;
@@ -743,7 +783,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const float *xs0 = xsum + (size_t)min(t0, TM - 1) * nbd;
             const float *xs1 = xsum + (size_t)min(t1, TM - 1) * nbd;
             const int nkg = d / 64;
-            for (int q = warp; q < sp.n_gu && ok; q += NW) {
+            const int S = sp.n_gu * nkg;
+            const int lo = warp * S / NW, hi = (warp + 1) * S / NW;
+            auto warp_of = [&](int x) { return ((x + 1) * NW + S - 1) / S - 1; };   // range holding step x
+            for (int q = lo / nkg; lo < hi && q <= (hi - 1) / nkg && ok; ++q) {
+                const int kb = max(lo - q * nkg, 0), ke = min(hi - q * nkg, nkg);
                 uint32_t par;
                 int fill;
                 const int s = slot_of(q, par, fill);
@@ -754,12 +798,9 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 if (!ok) break;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes;
                 const __half *sc = reinterpret_cast<const __half *>(tile + p.gu.code_bytes);
-                // two accumulator chains (even and odd k groups), summed at the end: the flushes of
-                // consecutive k groups do not wait on each other
-                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
-                for (int kg = 0; kg < nkg; ++kg) {
-                    float *acc = acc2[kg & 1];
+                for (int kg = kb; kg < ke; ++kg) {
                     uint32_t a[16];
                     frag16<FMT>(tile + (size_t)kg * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
                     uint32_t b0[4], b1[4];
@@ -781,23 +822,45 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     flush_block<FMT>(acc, Da, sg.x, s8.x, v00, v10, false);
                     flush_block<FMT>(acc, Db, sg.y, s8.y, v01, v11, true);
                 }
-                const float acc[4] = {acc2[0][0] + acc2[1][0], acc2[0][1] + acc2[1][1], acc2[0][2] + acc2[1][2],
-                                      acc2[0][3] + acc2[1][3]};
-                // rows g (gate) and g + 8 (up) of the unit for tokens 2c, 2c + 1: SwiGLU in place
-                const int n = cta + G * q;
-                const int u = n / ntile_gu, t8 = n - u * ntile_gu;
-                if (l0) {
-                    const float xi = ms->xinv[t0];
-                    p.x_h[((size_t)u * TM + t0) * I + 8 * t8 + g] = silu(acc[0] * xi) * (acc[2] * xi);
+                const int wa = warp_of(q * nkg), wb = warp_of(q * nkg + nkg - 1);
+                bool last = true;
+                if (wb > wa) {
+                    // a part of a cut unit: add into the unit's sums; the last part takes them
+                    float *pa = ms->pacc[wa][lane];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) atomicAdd(pa + j, acc[j]);
+                    __syncwarp();
+                    int before = 0;
+                    if (lane == 0) {
+                        __threadfence_block();
+                        before = atomicAdd(&ms->pcnt[wa], 1);
+                    }
+                    before = __shfl_sync(0xffffffffu, before, 0);
+                    last = before == wb - wa;
+                    if (last) {
+                        __threadfence_block();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[j] = *(volatile float *)(pa + j);
+                        if (lane == 0) ms->pcnt[wa] = 0;
+                    }
                 }
-                if (l1) {
-                    const float xi = ms->xinv[t1];
-                    p.x_h[((size_t)u * TM + t1) * I + 8 * t8 + g] = silu(acc[1] * xi) * (acc[3] * xi);
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    atomicAdd(&ms->ccnt[s], 1);
-                    mbar_arrive(&ms->empty[s]);      // the slot may be refilled
+                if (last) {
+                    // rows g (gate) and g + 8 (up) of the unit for tokens 2c, 2c + 1: SwiGLU in place
+                    const int n = cta + G * q;
+                    const int u = n / ntile_gu, t8 = n - u * ntile_gu;
+                    if (l0) {
+                        const float xi = ms->xinv[t0];
+                        p.x_h[((size_t)u * TM + t0) * I + 8 * t8 + g] = silu(acc[0] * xi) * (acc[2] * xi);
+                    }
+                    if (l1) {
+                        const float xi = ms->xinv[t1];
+                        p.x_h[((size_t)u * TM + t1) * I + 8 * t8 + g] = silu(acc[1] * xi) * (acc[3] * xi);
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        atomicAdd(&ms->ccnt[s], 1);
+                        mbar_arrive(&ms->empty[s]);      // the slot may be refilled
+                    }
                 }
             }
         }
@@ -819,9 +882,10 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 break;
             }
             mark(5, clock64() - tl0);
-            // h of the run's experts -> hi + lo B fragments (8 columns, zero past T) and, per
-            // (expert, token, 32-block), the sum of hi + lo and (fp16) the block's 2^-s
-            const int nq = n_span * TMAX * (I / 4);   // 4 values per thread and step; 8 lanes per block
+            // h of the run's experts -> hi + lo B fragments (columns of the T tokens; the rest is
+            // masked where it is read) and, per (expert, token, 32-block), the sum of hi + lo and
+            // (fp16) the block's 2^-s
+            const int nq = n_span * T * (I / 4);   // 4 values per thread and step; 8 lanes per block
             for (int i0 = 0; i0 < nq; i0 += HB_M * NT) {
               float4 hb[HB_M];   // a batch of loads in flight together, then the arithmetic
 #pragma unroll
@@ -829,20 +893,19 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const int i = i0 + bq * NT + tid;
                 hb[bq] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < nq) {
-                    const int su = i / (TMAX * (I / 4));
-                    const int rem = i - su * (TMAX * (I / 4));
+                    const int su = i / (T * (I / 4));
+                    const int rem = i - su * (T * (I / 4));
                     const int t = rem / (I / 4), k4 = rem - t * (I / 4);
-                    if (t < T) hb[bq] = __ldcg(reinterpret_cast<const float4 *>(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4));
+                    hb[bq] = __ldcg(reinterpret_cast<const float4 *>(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4));
                 }
               }
 #pragma unroll
               for (int bq = 0; bq < HB_M; ++bq) {
                 const int i = i0 + bq * NT + tid;
                 if (i >= nq) break;   // uniform across the warp (nq is a multiple of 32)
-                const int su = i / (TMAX * (I / 4));
-                const int rem = i - su * (TMAX * (I / 4));
+                const int su = i / (T * (I / 4));
+                const int rem = i - su * (T * (I / 4));
                 const int t = rem / (I / 4), k4 = rem - t * (I / 4);
-                const bool live = t < T;
                 const float4 hv = hb[bq];
                 const float h4[4] = {hv.x, hv.y, hv.z, hv.w};
                 float scale = 1.f;
@@ -855,7 +918,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     frexpf(mx, &he);
                     const int sh = min(15 - he, 100);
                     scale = pow2i(sh);
-                    if (live && (lane & 7) == 0) hinv[(su * TM + t) * nbi + (k4 >> 3)] = pow2i(-sh);
+                    if ((lane & 7) == 0) hinv[(su * TM + t) * nbi + (k4 >> 3)] = pow2i(-sh);
                 }
                 uint32_t hi2[2], lo2[2];
                 float part = 0.f;
@@ -882,7 +945,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 part += __shfl_xor_sync(0xffffffffu, part, 1);
                 part += __shfl_xor_sync(0xffffffffu, part, 2);
                 part += __shfl_xor_sync(0xffffffffu, part, 4);
-                if (live && (lane & 7) == 0) hsum[(su * TM + t) * nbi + (k4 >> 3)] = part;
+                if ((lane & 7) == 0) hsum[(su * TM + t) * nbi + (k4 >> 3)] = part;
                 // values k = 4 k4 .. 4 k4 + 3 of token t: slice sl, register b0 (kk < 8) or b1, the
                 // lanes (t, c0) and (t, c0 + 1)
                 const int kk = 4 * k4;
@@ -921,7 +984,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const int su = u - u_first;
                 const uint8_t *tile = ring + (size_t)s * p.slot_bytes + (size_t)ui * p.dn.tile_bytes;
                 const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
-                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const int t0 = 2 * c, t1 = 2 * c + 1;
                 const float *hs0 = hsum + (su * TM + min(t0, TM - 1)) * nbi;
                 const float *hs1 = hsum + (su * TM + min(t1, TM - 1)) * nbi;
@@ -930,13 +993,13 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const bool l0 = t0 < T, l1 = t1 < T;
 #pragma unroll 2
                 for (int kg = 0; kg < nkgi; ++kg) {
-                    float *acc = acc2[kg & 1];   // two accumulator chains (even and odd k groups)
                     uint32_t a[16];
                     frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
                     float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const uint4 bq = *reinterpret_cast<const uint4 *>(htab + hfrag_off(su, nkgi, kg, m, lane));
+                        const uint4 bq = g < T ? *reinterpret_cast<const uint4 *>(htab + hfrag_off(su, nkgi, kg, m, lane))
+                                               : make_uint4(0u, 0u, 0u, 0u);
                         float *D = (m < 2) ? Da : Db;
                         mma_fmt<FMT>(D, a + 4 * m, bq.x, bq.y);   // hi
                         mma_fmt<FMT>(D, a + 4 * m, bq.z, bq.w);   // lo
@@ -961,8 +1024,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                         }
                     }
                 }
-                const float acc[4] = {acc2[0][0] + acc2[1][0], acc2[0][1] + acc2[1][1], acc2[0][2] + acc2[1][2],
-                                      acc2[0][3] + acc2[1][3]};
                 // weighted by each token's routing weight for this expert, then 4 consecutive rows of
                 // one token per lane (a 4 x 4 transpose among the lanes g = 4m' .. 4m' + 3 of a column
                 // pair) for one vector atomic each
@@ -1002,6 +1063,16 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         }
         mark(7, clock64() - tl0);
         if (tid == 0) ctr_arrive(p.cnt + C_Y);
+        // the next layer's r_prev (this layer's r, complete since the logits exchange) into the
+        // idle ring: its load overlaps the wait for the other CTAs' outputs
+        if (p.stack && l + 1 < p.L) {
+            const float *rl = p.r_buf + (size_t)yb * TM * d;
+            for (int i = tid; i < T * d4; i += NT) {
+                const int t = i / d4, i4 = i - t * d4;
+                *reinterpret_cast<float4 *>(rsm + (size_t)t * d + 4 * i4) =
+                    __ldcg(reinterpret_cast<const float4 *>(rl + (size_t)t * d + 4 * i4));
+            }
+        }
         mark(8, clock64() - tl0);
         mark(9, tw_gu);
         mark(10, tw_dn);
@@ -1064,6 +1135,7 @@ bool decode_multi_supported(const moe_ctx *ctx) {
     if (c.flags & MOE_FLAG_NO_DECODE_KERNEL) return false;
     if (c.max_tokens < 2) return false;
     if (c.d_model > 2 * 4 * NT || c.d_model / 256 > NW || c.n_experts > 32 * EPL || c.n_experts % 4) return false;
+    if (c.d_ff % 128) return false;   // the h table's warps each take one token's whole 32-block groups
     if (c.top_k > KMAX) return false;
     return ctx->mdec.smem_bytes > 0;
 }

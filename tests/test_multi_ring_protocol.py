@@ -4,8 +4,10 @@ One CTA, one layer, random interleavings of the producer (fills items in
 order, refilling a slot once its previous item is consumed) and the compute
 warps:
 
-* gate/up items: one unit each; units go round-robin to all warps, and the
-  unit's warp frees the slot;
+* gate/up items: one unit each of nkg k-group steps; the units' steps form
+  one sequence cut into NW near-equal contiguous ranges, one per warp, so a
+  unit may be cut into parts taken by several warps; the last part of a unit
+  to finish frees its slot;
 * down items: batches of units; units go round-robin to all warps, the warp
   that finishes an item's last unit frees the slot;
 * before waiting on a slot, a unit's warp waits until every earlier item of
@@ -18,8 +20,9 @@ passes once the phase with parity P has completed, i.e. while the current
 phase parity differs from P).  The check: every run finishes, and every
 consumer reads the fill it expects.  Two planted mistakes show the check is
 not vacuous: without the wait on the slot's earlier items a unit reads an
-older fill (or the run stalls), and a slot freed by the first unit of an item
-instead of the last lets the producer overwrite units still being read.
+older fill (or the run stalls), a slot freed by the first unit of an item
+instead of the last lets the producer overwrite units still being read, and
+a gate/up slot freed by the first part of a cut unit does the same.
 """
 import random
 
@@ -45,7 +48,25 @@ class Stale(AssertionError):
     pass
 
 
-def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_last=True):
+def gu_parts(n_gu, nkg, NW):
+    """Per warp, its (unit, parts of that unit) list: balanced ranges of the n_gu * nkg steps."""
+    S = n_gu * nkg
+    rng = [(w * S // NW, (w + 1) * S // NW) for w in range(NW)]
+    owners = {}
+    for w, (lo, hi) in enumerate(rng):
+        for q in range(lo // nkg, (hi - 1) // nkg + 1) if lo < hi else []:
+            owners.setdefault(q, []).append(w)
+    # the kernel finds a unit's first and last warp from its first and last step
+    def warp_of(x):
+        return ((x + 1) * NW + S - 1) // S - 1
+    for q, ws in owners.items():
+        assert ws[0] == warp_of(q * nkg) and ws[-1] == warp_of(q * nkg + nkg - 1)
+        assert ws == list(range(ws[0], ws[-1] + 1))
+    return [[(q, len(owners[q])) for q in sorted(owners) if w in owners[q]] for w in range(NW)]
+
+
+def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_last=True, nkg=40,
+        gu_free_on_last=True):
     rnd = random.Random(seed)
     full = [MBar(1) for _ in range(nslot)]
     empty = [MBar(1) for _ in range(nslot)]
@@ -59,7 +80,9 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
     def slot(a):
         return a % nslot, (a // nslot) & 1, a // nslot
 
-    warps = [{"ph": "gu", "q": w, "u": w, "busy": None} for w in range(NW)]
+    plan = gu_parts(n_gu, nkg, NW)
+    pcnt = {}
+    warps = [{"ph": "gu", "j": 0, "u": w, "busy": None} for w in range(NW)]
     for _ in range(400000):
         actors = (["p"] if prod["q"] < n_items else []) + [w for w in range(NW) if warps[w]["ph"] != "done"]
         if not actors:
@@ -83,11 +106,23 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
                 break
             ws = warps[a]
             if ws["ph"] == "gu":
-                q = ws["q"]
-                if q >= n_gu:
+                if ws["busy"] is not None:            # finish the part being read
+                    s, q, nparts = ws["busy"]
+                    reading[s] -= 1
+                    pcnt[q] = pcnt.get(q, 0) + 1
+                    # planted mistake: the first part of a cut unit to finish frees the slot
+                    if pcnt[q] == (nparts if gu_free_on_last else 1):
+                        ccnt[s] += 1
+                        empty[s].arrive()
+                    ws["busy"] = None
+                    ws["j"] += 1
+                    moved = True
+                    break
+                if ws["j"] >= len(plan[a]):
                     ws["ph"] = "wait"
                     moved = True
                     break
+                q, nparts = plan[a][ws["j"]]
                 s, par, fill = slot(q)
                 if gate_on_earlier and ccnt[s] < fill:
                     continue
@@ -95,9 +130,8 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
                     continue
                 if content[s] != q:
                     raise Stale(f"gate/up unit {q} read slot {s} holding item {content[s]}")
-                ccnt[s] += 1
-                empty[s].arrive()
-                ws["q"] += NW
+                reading[s] += 1
+                ws["busy"] = (s, q, nparts)
                 moved = True
                 break
             if ws["ph"] == "wait":
@@ -146,7 +180,31 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
 
 
 CASES = [(5, 32, 81, 5), (5, 33, 81, 5), (7, 8, 20, 5), (5, 8, 4, 5), (8, 21, 52, 5),
-         (5, 10, 90, 5), (2, 4, 30, 5), (3, 1, 13, 4), (5, 8, 60, 1), (6, 3, 70, 2)]
+         (5, 10, 90, 5), (2, 4, 30, 5), (3, 1, 13, 4), (5, 8, 60, 1), (6, 3, 70, 2),
+         (8, 7, 19, 5), (5, 36, 88, 5), (4, 13, 40, 5), (2, 2, 5, 5)]
+
+
+@pytest.mark.parametrize("n_gu", [1, 2, 5, 7, 8, 11, 12, 13, 24, 35])
+def test_gate_up_ranges_cover_every_step_once(n_gu):
+    nkg, NW = 40, 12
+    plan = gu_parts(n_gu, nkg, NW)
+    S = n_gu * nkg
+    steps = []
+    for w in range(NW):
+        lo, hi = w * S // NW, (w + 1) * S // NW
+        steps += list(range(lo, hi))
+        # a cut unit is the first or the last of each warp that takes part of it
+        cut = [q for q, n in plan[w] if n > 1]
+        units = [q for q, _ in plan[w]]
+        assert all(q in (units[0], units[-1]) for q in cut)
+    assert steps == list(range(S))
+    # slots of cut units (their first warp) are distinct and below NW - 1
+    firsts = {}
+    for w in range(NW):
+        for q, n in plan[w]:
+            if n > 1:
+                firsts.setdefault(q, w)
+    assert len(set(firsts.values())) == len(firsts) and all(f < NW - 1 for f in firsts.values())
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -162,6 +220,17 @@ def test_planted_no_wait_on_earlier_items_is_caught():
             # one-unit items: a warp's next unit is twelve items on, past a whole turn of the ring
             ok = run(5, 8, 60, 1, seed=seed, gate_on_earlier=False)
         except Stale:
+            ok = False
+        caught += not ok
+    assert caught > 0
+
+
+def test_planted_gate_up_slot_freed_by_first_part_is_caught():
+    caught = 0
+    for seed in range(25):
+        try:
+            ok = run(5, 7, 20, 5, seed=seed, gu_free_on_last=False)
+        except (Stale, AssertionError):
             ok = False
         caught += not ok
     assert caught > 0
