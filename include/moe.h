@@ -94,10 +94,13 @@ typedef struct {
  * alternative single-token kernel (measured slower on this shape, kept for
  * comparison); MOE_FLAG_TRACE records the decode
  * kernel's phase clocks; MOE_FLAG_TEST_WITHHOLD is a test hook for the
- * bounded device waits: in the context's first single-token call the decode
- * kernel's CTA 0 withholds its router logits, every wait on them runs out
- * after about one second, and the call reports MOE_ERR_DEVICE_TIMEOUT through
- * moe_get_device_error; later calls run normally. */
+ * bounded device waits: in the context's first call of a decode kernel
+ * (single-token, few-token or split) that kernel's CTA 0 withholds its router
+ * logits, and in the context's first tensor-core gate/up GEMM CTA 0 never
+ * signals its first accumulator as complete; every wait on them runs out
+ * (about one second in the decode kernels, two in the GEMM), and the call
+ * reports MOE_ERR_DEVICE_TIMEOUT through moe_get_device_error; later calls
+ * run normally.  Both hooks are for tests only. */
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* small T runs the general path, not the single-token kernel */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
 #define MOE_FLAG_NO_MULTI_DECODE 8    /* 2..16 tokens run the single-token kernel per token, not the few-token kernel */

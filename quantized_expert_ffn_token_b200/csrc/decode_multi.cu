@@ -56,6 +56,7 @@ constexpr int CANDM = 64;       // top-k candidates per token held for ranking
 constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
 constexpr int IN_IT = 2;        // float4 columns of a token row per thread in the input phase (d <= 3072)
 constexpr int HB_M = 4;         // float4 loads of h in flight per thread
+constexpr int GU_CH = 4;        // chunks (k-group ranges) per gate/up unit
 
 struct MiscM {
     unsigned long long full[MAX_SLOTS];
@@ -69,14 +70,13 @@ struct MiscM {
     int ids[TMAX][KMAX];
     float w[TMAX][KMAX];
     unsigned bits[32];                     // union bitmap over E <= 1024
-    int wpre[32];                          // union slots below each bitmap word
     float xinv[TMAX];                      // 2^-s of a token's fp16 operand (1 for bf16 operands)
     float xscale[TMAX];                    // 2^s
     union {
         float2 cand[TMAX][CANDM];          // top-k: candidates of each token (logit, id bits)
-        float pacc[NW - 1][32][4];         // gate/up: sums of a unit cut by warp boundaries, by its first warp
+        float pacc[MAX_SLOTS][32][4];      // gate/up: chunk sums of the unit in each ring slot
     };
-    int pcnt[NW - 1];                      // gate/up: parts of that unit finished
+    int pcnt[MAX_SLOTS];                   // gate/up: chunks of that unit finished
     float ss[NW][TMAX];                    // per-warp sums of squares / maxima of the input phase
     float mx[NW][TMAX];
     float tinv[TMAX];                      // 1 / rms of each token's residual row
@@ -107,7 +107,7 @@ struct MultiParams {
     int withhold;
     unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
-    int off_ring, off_router, off_xb, off_xsum, off_hsum, off_uexp, off_wtab,
+    int off_ring, off_router, off_xb, off_hsum, off_uexp, off_wtab,
         off_misc, off_ltab;
 };
 
@@ -216,7 +216,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     float *rtr = reinterpret_cast<float *>(smem + p.off_router);
     uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_xb);     // [TM][d] bf16 input; then the h table
     uint8_t *htab = smem + p.off_xb;
-    float *xsum = reinterpret_cast<float *>(smem + p.off_xsum);       // [TM][d/32]
     float *hsum = reinterpret_cast<float *>(smem + p.off_hsum);       // [span][TM][I/32], then hinv
     int *uexp = reinterpret_cast<int *>(smem + p.off_uexp);           // [UM]
     float *wtab = reinterpret_cast<float *>(smem + p.off_wtab);       // [UM][TM]
@@ -249,7 +248,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         fence_mbar_init();
     }
     for (int i = tid; i < 32; i += NTT) ms->bits[i] = 0u;
-    for (int i = tid; i < NW - 1; i += NTT) ms->pcnt[i] = 0;
+    for (int i = tid; i < MAX_SLOTS; i += NTT) ms->pcnt[i] = 0;
     for (int l = tid; l < p.L; l += NTT) ltab[l] = p.layers[p.layer0 + l];
     __syncthreads();
 
@@ -262,8 +261,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         const int n_gu_all = nU * ntile_gu;
         sp.n_gu = (cta < n_gu_all) ? (n_gu_all - cta + G - 1) / G : 0;   // units cta, cta + G, ...
         const int n_dn_all = nU * ntile_dn;
-        sp.dn_lo = (int)((long long)cta * n_dn_all / G);
-        sp.dn_hi = (int)((long long)(cta + 1) * n_dn_all / G);
+        sp.dn_lo = cta * n_dn_all / G;   // < 2^31: n_dn_all <= UM * d / 16, checked at set-up
+        sp.dn_hi = (cta + 1) * n_dn_all / G;
         sp.n_dn = sp.dn_hi - sp.dn_lo;
         sp.n_dn_items = (sp.n_dn + dn_per_slot - 1) / dn_per_slot;
         sp.n_items = sp.n_gu + sp.n_dn_items;
@@ -296,12 +295,13 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             if (!mbar_wait(&ms->route, (uint32_t)(l & 1), err, true)) break;
             const Split sp = split(ms->nU);
             bool pok = true;
+            // the compute warps fenced their generic writes to the ring before the routing arrival
+            fence_proxy_async();
             for (int q = 0; q < sp.n_items && pok; ++q) {
                 const int s = s_next;
                 s_next = (s_next + 1 == p.nslot) ? 0 : s_next + 1;
                 if ((filled >> s) & 1u) pok = mbar_wait(&ms->empty[s], ((fpar >> s) & 1u) ^ 1u, err, true);
                 if (!pok) break;
-                fence_proxy_async();
                 uint8_t *dst = ring + (size_t)s * p.slot_bytes;
                 if (q < sp.n_gu) {
                     const int n = cta + G * q;
@@ -456,8 +456,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             csync();
             mark(13, clock64() - tl0);
             // pass 2: x = bf16(r * inv), r from shared memory
-            for (int i = tid; i < T * d4; i += NT) {
-                const int t = i / d4, i4 = i - t * d4;
+            for (int t = 0; t < T; ++t)
+            for (int i4 = tid; i4 < d4; i4 += NT) {
                 const float inv = ms->tinv[t];
                 const float4 r = *reinterpret_cast<const float4 *>(rsm + (size_t)t * d + 4 * i4);
                 const uint2 xv = make_uint2(
@@ -533,36 +533,41 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     acc = fmaf(wv.w, bf16f(xv.y >> 16), acc);
                 }
                 for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                const int e = cta + G * j;
-                if (lane == 0) p.x_logits[(size_t)t * E + e] = acc + ms->rbias[j];
+                if (lane == 0) p.x_logits[(size_t)t * E + cta + G * j] = acc + ms->rbias[j];
             }
         }
         csync();   // this CTA's logits are stored; the router rows and the bf16 rows are no longer read
         if (tid == 0 && !(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
         mark(1, clock64() - tl0);
-        // the gate/up B operand in place of the bf16 rows (fp16 of x * 2^s for fp16 code operands),
-        // and its 32-block sums (the offset removal in the gate/up flush)
-        if constexpr (F16OP) {
-            for (int i = tid; i < T * (d / 8); i += NT) {
-                const int t = i / (d / 8), i8 = i - t * (d / 8);
-                uint4 *pv = reinterpret_cast<uint4 *>(xb + (size_t)t * XS + 8 * i8);
-                const uint4 v = *pv;
-                const float sc = ms->xscale[t];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t o[4];
+        // the gate/up B operand in place of the bf16 rows: within each token's 64-wide k group the
+        // words are reordered so that lane c's eight B registers of the group (slices 0..3, both
+        // halves) are 32 contiguous bytes; fp16 code operands take fp16 of x * 2^s
+        for (int i = tid; i < T * (d / 64); i += NT) {
+            const int t = i / (d / 64), kg = i - t * (d / 64);
+            uint4 *pv = reinterpret_cast<uint4 *>(xb + (size_t)t * XS + 64 * kg);
+            uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const __half2 h2 = __floats2half2_rn(bf16f(w[j] & 0xFFFFu) * sc, bf16f(w[j] >> 16) * sc);
-                    o[j] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                *pv = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int j = 0; j < 8; ++j) {
+                const uint4 v = pv[j];
+                w[4 * j] = v.x;
+                w[4 * j + 1] = v.y;
+                w[4 * j + 2] = v.z;
+                w[4 * j + 3] = v.w;
             }
-            csync();
-        }
-        for (int i = tid; i < T * nbd; i += NT) {
-            const int t = i / nbd, b = i - t * nbd;
-            const uint16_t *src = xb + (size_t)t * XS + 32 * b;
-            xsum[t * nbd + b] = F16OP ? sum32_f16(src) : sum32_bf16(src);
+            if constexpr (F16OP) {
+                const float sc = ms->xscale[t];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const __half2 h2 = __floats2half2_rn(bf16f(w[j] & 0xFFFFu) * sc, bf16f(w[j] >> 16) * sc);
+                    w[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+            }
+            // word 8m + 4h + c (slice m, B register h, lane column c) goes to 8c + 2m + h
+            uint32_t o[32];
+#pragma unroll
+            for (int wo = 0; wo < 32; ++wo) o[8 * (wo & 3) + 2 * (wo >> 3) + ((wo >> 2) & 1)] = w[wo];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pv[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         }
         mark(16, clock64() - tl0);
         if (tid == 0) {
@@ -688,74 +693,75 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
             __syncwarp();
             if (lane < k) {
+                const float wt = pe / z;
                 ms->ids[t][lane] = pv_id;
-                ms->w[t][lane] = pe / z;
+                ms->w[t][lane] = wt;
                 atomicOr(&ms->bits[pv_id >> 5], 1u << (pv_id & 31));
-            }
-        }
-        csync();
-        mark(19, clock64() - tl0);
-        if (warp != 0) {
-            // the gate/up part sums share memory with the top-k candidates: zero them
-            float *pz = &ms->pacc[0][0][0];
-            for (int i = tid - 32; i < (NW - 1) * 32 * 4; i += NT - 32) pz[i] = 0.f;
-        }
-        if (warp == 0) {
-            // union in ascending expert order, then the shared experts
-            const int nwords = (E + 31) / 32;
-            const unsigned word = lane < nwords ? ms->bits[lane] : 0u;
-            int pre = __popc(word);
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, pre, o);
-                if (lane >= o) pre += n;
-            }
-            const int total = __shfl_sync(0xffffffffu, pre, 31);
-            pre -= __popc(word);   // exclusive
-            ms->wpre[lane] = pre;
-            unsigned wv = word;
-            int pos = pre;
-            while (wv) {
-                const int b = __ffs(wv) - 1;
-                wv &= wv - 1;
-                uexp[pos++] = 32 * lane + b;
-            }
-            if (lane < p.nsh) uexp[total + lane] = E + lane;
-            const int nU = total + p.nsh;
-            for (int i = lane; i < nU * TM; i += 32) wtab[i] = 0.f;
-            __syncwarp();
-            // weight table: token t's j-th expert sits at union slot (ones below it in the bitmap)
-            for (int i = lane; i < T * k; i += 32) {
-                const int t = i / k, j = i - t * k;
-                const int e = ms->ids[t][j];
-                const int wi = e >> 5;
-                const int slot = ms->wpre[wi] + __popc(ms->bits[wi] & ((1u << (e & 31)) - 1u));
-                wtab[slot * TM + t] = ms->w[t][j];
-            }
-            for (int i = lane; i < p.nsh * T; i += 32) wtab[(total + i / T) * TM + i % T] = 1.f;
-            __syncwarp();
-            if (lane < nwords) ms->bits[lane] = 0u;
-            if (lane == 0) {
-                ms->nU = nU;
-                ms->nR = total;
-            }
-            // routing outputs
-            if (cta == 0) {
-                for (int i = lane; i < T * k; i += 32) {
-                    const int t = i / k, j = i - t * k;
+                if (cta == 0) {   // routing outputs
                     if (p.stack && p.rec_on) {
-                        const size_t ro = ((size_t)l * p.rec_n + p.rec_r0 + t) * k + j;
-                        if (p.rec.ids) p.rec.ids[ro] = ms->ids[t][j];
-                        if (p.rec.w) p.rec.w[ro] = ms->w[t][j];
+                        const size_t ro = ((size_t)l * p.rec_n + p.rec_r0 + t) * k + lane;
+                        if (p.rec.ids) p.rec.ids[ro] = pv_id;
+                        if (p.rec.w) p.rec.w[ro] = wt;
                     }
                     if (!p.stack) {
-                        if (p.ids_out) p.ids_out[(size_t)t * k + j] = ms->ids[t][j];
-                        if (p.w_out) p.w_out[(size_t)t * k + j] = ms->w[t][j];
+                        if (p.ids_out) p.ids_out[(size_t)t * k + lane] = pv_id;
+                        if (p.w_out) p.w_out[(size_t)t * k + lane] = wt;
                     }
                 }
             }
         }
+        csync();   // the union bitmap is complete
+        mark(19, clock64() - tl0);
+        // Union in ascending expert order, then the shared experts: an expert's union slot is the
+        // number of bitmap ones below it.  Warp t < T writes column t of the weight table; the last
+        // warp lists the union; the others clear the gate/up chunk sums (they share memory with the
+        // top-k candidates).
+        {
+            const int nwords = (E + 31) / 32;
+            if (warp < T || warp == NW - 1) {
+                const unsigned word = lane < nwords ? ms->bits[lane] : 0u;
+                int pre = __popc(word);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int n = __shfl_up_sync(0xffffffffu, pre, o);
+                    if (lane >= o) pre += n;
+                }
+                const int total = __shfl_sync(0xffffffffu, pre, 31);
+                pre -= __popc(word);   // exclusive
+                const int nU = total + p.nsh;
+                if (warp < T) {
+                    const int t = warp;
+                    for (int u = lane; u < nU; u += 32) wtab[u * TM + t] = 0.f;
+                    int e = 0;
+                    if (lane < k) e = ms->ids[t][lane];
+                    const int wi = e >> 5;
+                    const int below = __shfl_sync(0xffffffffu, pre, wi);
+                    const unsigned wbits = __shfl_sync(0xffffffffu, word, wi);
+                    __syncwarp();
+                    if (lane < k) wtab[(below + __popc(wbits & ((1u << (e & 31)) - 1u))) * TM + t] = ms->w[t][lane];
+                    if (lane < p.nsh) wtab[(total + lane) * TM + t] = 1.f;
+                } else {
+                    unsigned wv = word;
+                    int pos = pre;
+                    while (wv) {
+                        const int b = __ffs(wv) - 1;
+                        wv &= wv - 1;
+                        uexp[pos++] = 32 * lane + b;
+                    }
+                    if (lane < p.nsh) uexp[total + lane] = E + lane;
+                    if (lane == 0) {
+                        ms->nU = nU;
+                        ms->nR = total;
+                    }
+                }
+            } else {
+                float *pz = &ms->pacc[0][0][0];
+                for (int i = tid - 32 * T; i < MAX_SLOTS * 32 * 4; i += 32 * (NW - 1 - T)) pz[i] = 0.f;
+            }
+        }
         mark(20, clock64() - tl0);
         csync();
+        // every warp has read the bitmap: clear it for the next layer
+        if (warp == NW - 1 && lane < (E + 31) / 32) ms->bits[lane] = 0u;
         if (tid == 0) mbar_arrive(&ms->route);   // the producer may issue this layer's copies
         mark(3, clock64() - tl0);
         const int nU = ms->nU;
@@ -767,27 +773,39 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             return a - fill * p.nslot;
         };
 
-        // ---- 4. gate/up: balanced ranges of (unit, k group) steps ----------------------------------
-        // The CTA's units times the d/64 k groups form one sequence of steps, cut into NW near-equal
-        // contiguous ranges, one per warp; a warp's range covers whole units plus at most a partial
-        // first and last unit.  A unit cut by warp boundaries is summed in shared memory (slot = its
-        // first warp) and its last part to finish applies SwiGLU and frees the slot.  Before waiting
-        // on a unit's fill, a warp waits until every earlier item of the slot is consumed (a later
-        // unit can reach a slot that still holds an older item).  B operand: column g = token g (zero
-        // past T), from the token rows.
+        // ---- 4. gate/up: units cut into GU_CH chunks of k groups, round-robin over the warps ------
+        // Chunk c of the CTA's chunk sequence goes to warp c % NW, so each unit is worked by several
+        // warps as soon as its tile lands.  A unit's chunk sums meet in shared memory (indexed by
+        // its ring slot) and its last chunk to finish applies SwiGLU, clears the sums and frees the
+        // slot.  Before waiting on a unit's fill, a warp waits until every earlier item of the slot
+        // is consumed (a later unit can reach a slot that still holds an older item).  B operand:
+        // column g = token g (zero past T), from the token rows.
         {
             const bool live = g < T;
-            const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 2 * c;
+            const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 16 * c;
             const int t0 = 2 * c, t1 = 2 * c + 1;
             const bool l0 = t0 < T, l1 = t1 < T;
-            const float *xs0 = xsum + (size_t)min(t0, TM - 1) * nbd;
-            const float *xs1 = xsum + (size_t)min(t1, TM - 1) * nbd;
+            // the code offset is removed inside the MMAs: a second MMA per k16 slice with A = minus
+            // the offset (rows g and g + 8 of each 32-block, exact in fp16/bf16) on the same B; the
+            // multipliers scale back the codes read as 1024 + F q
+            uint32_t cg0, c80, cg1, c81;
+            float mg0, m80, mg1, m81;
+            if constexpr (FMT == MOE_Q4B32) {
+                cg0 = cg1 = 0xE408E408u; c80 = c81 = 0xE480E480u;   // -1032, -1152 (fp16)
+                mg0 = mg1 = 1.f; m80 = m81 = 0.0625f;
+            } else if constexpr (FMT == MOE_Q2B32) {
+                cg0 = 0xE402E402u; c80 = 0xE408E408u;               // -1026, -1032
+                cg1 = 0xE420E420u; c81 = 0xE480E480u;               // -1056, -1152
+                mg0 = 1.f; m80 = 0.25f; mg1 = 0.0625f; m81 = 0.015625f;
+            } else {
+                cg0 = c80 = cg1 = c81 = 0xC304C304u;                // -132 (bf16)
+                mg0 = m80 = mg1 = m81 = 1.f;
+            }
+            const uint32_t off0[4] = {cg0, c80, cg0, c80}, off1[4] = {cg1, c81, cg1, c81};
             const int nkg = d / 64;
-            const int S = sp.n_gu * nkg;
-            const int lo = warp * S / NW, hi = (warp + 1) * S / NW;
-            auto warp_of = [&](int x) { return ((x + 1) * NW + S - 1) / S - 1; };   // range holding step x
-            for (int q = lo / nkg; lo < hi && q <= (hi - 1) / nkg && ok; ++q) {
-                const int kb = max(lo - q * nkg, 0), ke = min(hi - q * nkg, nkg);
+            for (int ch = warp; ch < sp.n_gu * GU_CH && ok; ch += NW) {
+                const int q = ch / GU_CH, j = ch - q * GU_CH;
+                const int kb = j * nkg / GU_CH, ke = (j + 1) * nkg / GU_CH;
                 uint32_t par;
                 int fill;
                 const int s = slot_of(q, par, fill);
@@ -803,48 +821,48 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 for (int kg = kb; kg < ke; ++kg) {
                     uint32_t a[16];
                     frag16<FMT>(tile + (size_t)kg * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
-                    uint32_t b0[4], b1[4];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        b0[m] = live ? *reinterpret_cast<const uint32_t *>(xr + 64 * kg + 16 * m) : 0u;
-                        b1[m] = live ? *reinterpret_cast<const uint32_t *>(xr + 64 * kg + 16 * m + 8) : 0u;
-                    }
+                    const uint4 q0 = live ? *reinterpret_cast<const uint4 *>(xr + 64 * kg) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 q1 = live ? *reinterpret_cast<const uint4 *>(xr + 64 * kg + 8) : make_uint4(0u, 0u, 0u, 0u);
                     float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_fmt<FMT>(Da, a + 0, b0[0], b1[0]);
-                    mma_fmt<FMT>(Da, a + 4, b0[1], b1[1]);
-                    mma_fmt<FMT>(Db, a + 8, b0[2], b1[2]);
-                    mma_fmt<FMT>(Db, a + 12, b0[3], b1[3]);
+                    mma_fmt<FMT>(Da, a + 0, q0.x, q0.y);
+                    mma_fmt<FMT>(Da, off0, q0.x, q0.y);
+                    mma_fmt<FMT>(Da, a + 4, q0.z, q0.w);
+                    mma_fmt<FMT>(Da, off0, q0.z, q0.w);
+                    mma_fmt<FMT>(Db, a + 8, q1.x, q1.y);
+                    mma_fmt<FMT>(Db, off1, q1.x, q1.y);
+                    mma_fmt<FMT>(Db, a + 12, q1.z, q1.w);
+                    mma_fmt<FMT>(Db, off1, q1.z, q1.w);
                     const int bl = 2 * kg;
                     const float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + bl));
                     const float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + bl));
-                    const float v00 = l0 ? xs0[bl] : 0.f, v10 = l1 ? xs1[bl] : 0.f;
-                    const float v01 = l0 ? xs0[bl + 1] : 0.f, v11 = l1 ? xs1[bl + 1] : 0.f;
-                    flush_block<FMT>(acc, Da, sg.x, s8.x, v00, v10, false);
-                    flush_block<FMT>(acc, Db, sg.y, s8.y, v01, v11, true);
+                    const float sga = sg.x * mg0, s8a = s8.x * m80, sgb = sg.y * mg1, s8b = s8.y * m81;
+                    acc[0] = fmaf(sga, Da[0], acc[0]);
+                    acc[1] = fmaf(sga, Da[1], acc[1]);
+                    acc[2] = fmaf(s8a, Da[2], acc[2]);
+                    acc[3] = fmaf(s8a, Da[3], acc[3]);
+                    acc[0] = fmaf(sgb, Db[0], acc[0]);
+                    acc[1] = fmaf(sgb, Db[1], acc[1]);
+                    acc[2] = fmaf(s8b, Db[2], acc[2]);
+                    acc[3] = fmaf(s8b, Db[3], acc[3]);
                 }
-                const int wa = warp_of(q * nkg), wb = warp_of(q * nkg + nkg - 1);
-                bool last = true;
-                if (wb > wa) {
-                    // a part of a cut unit: add into the unit's sums; the last part takes them
-                    float *pa = ms->pacc[wa][lane];
+                // this chunk's sums into the unit's; the last chunk takes them
+                float *pa = ms->pacc[s][lane];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) atomicAdd(pa + j, acc[j]);
-                    __syncwarp();
-                    int before = 0;
-                    if (lane == 0) {
-                        __threadfence_block();
-                        before = atomicAdd(&ms->pcnt[wa], 1);
-                    }
-                    before = __shfl_sync(0xffffffffu, before, 0);
-                    last = before == wb - wa;
-                    if (last) {
-                        __threadfence_block();
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[j] = *(volatile float *)(pa + j);
-                        if (lane == 0) ms->pcnt[wa] = 0;
-                    }
+                for (int jj = 0; jj < 4; ++jj) atomicAdd(pa + jj, acc[jj]);
+                __syncwarp();
+                int before = 0;
+                if (lane == 0) {
+                    __threadfence_block();
+                    before = atomicAdd(&ms->pcnt[s], 1);
                 }
-                if (last) {
+                before = __shfl_sync(0xffffffffu, before, 0);
+                if (before == GU_CH - 1) {
+                    __threadfence_block();
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        acc[jj] = *(volatile float *)(pa + jj);
+                        pa[jj] = 0.f;   // ready for the slot's next unit
+                    }
                     // rows g (gate) and g + 8 (up) of the unit for tokens 2c, 2c + 1: SwiGLU in place
                     const int n = cta + G * q;
                     const int u = n / ntile_gu, t8 = n - u * ntile_gu;
@@ -858,6 +876,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     }
                     __syncwarp();
                     if (lane == 0) {
+                        ms->pcnt[s] = 0;
+                        __threadfence_block();
                         atomicAdd(&ms->ccnt[s], 1);
                         mbar_arrive(&ms->empty[s]);      // the slot may be refilled
                     }
@@ -1168,7 +1188,6 @@ int decode_multi_setup(moe_ctx *ctx) {
     const size_t htab_bytes = (size_t)span * (c.d_ff / 64) * 4 * 32 * 16;
     ms.off_router = take((size_t)rpc * c.d_model * 4);
     ms.off_xb = take(xb_bytes > htab_bytes ? xb_bytes : htab_bytes);
-    ms.off_xsum = take((size_t)TM * (c.d_model / 32) * 4);
     ms.off_hsum = take((size_t)2 * span * TM * (c.d_ff / 32) * 4);
     ms.off_uexp = take((size_t)UM * 4);
     ms.off_wtab = take((size_t)UM * TM * 4);
@@ -1250,7 +1269,6 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.off_ring = ms.off_ring;
     p.off_router = ms.off_router;
     p.off_xb = ms.off_xb;
-    p.off_xsum = ms.off_xsum;
     p.off_hsum = ms.off_hsum;
     p.off_uexp = ms.off_uexp;
     p.off_wtab = ms.off_wtab;

@@ -83,6 +83,7 @@ struct TcParams {
     size_t cache_off;           // fp16 offset of this GEMM's stages within a slot
     size_t cache_stride;        // fp16 per slot (3 d I)
     int *err;
+    int withhold;               // test hook: CTA 0 never signals its first accumulator as full
 };
 
 enum TcMode { TC_GATEUP = 0, TC_DOWN = 1, TC_ROUTER = 2 };
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 }
                 __syncwarp();
             }
-            if (ok && lane == 0)
+            if (ok && lane == 0 && !(p.withhold && blockIdx.x == 0 && u == 0))
                 for (int a = 0; a < na; ++a) umma_commit(&ss->acc_full[(u + a) & 1]);
             __syncwarp();
             u += na;
@@ -941,10 +942,14 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.A = ws.x16;
     p.a_by_token = 1;
     p.h16 = ws.h16;
+    // test hook: the context's first gate/up GEMM leaves CTA 0's epilogue waiting until its bound
+    p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ctx->tc_withheld) ? 1 : 0;
+    if (p.withhold) ctx->tc_withheld = true;
     int grid = dev_sms;
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_GATEUP>(p, grid, st)));
     else if (c.fmt == MOE_Q2B32) QE_TRY((launch_tc<MOE_Q2B32, TC_GATEUP>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_GATEUP>(p, grid, st)));
+    p.withhold = 0;
 
     // down: A = h16 rows by grouped position, N = d, K = I
     QE_CHECK(cudaMemsetAsync(ws.y_acc, 0, Td * sizeof(float), st));

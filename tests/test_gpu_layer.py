@@ -296,6 +296,34 @@ def test_decode_wait_times_out_and_context_recovers():
     ref.close()
 
 
+def test_tensor_core_wait_times_out_and_context_recovers():
+    """The tensor-core path's bounded waits: with the test hook, CTA 0 of the
+    context's first gate/up GEMM never signals its first accumulator as full,
+    its epilogue's wait gives up after about two seconds, the call reports
+    MOE_ERR_DEVICE_TIMEOUT (the MMAs in flight are drained before the CTA frees
+    its tensor memory), and the next calls on the same context match a context
+    without the hook."""
+    capi, session = _cuda()
+    T = 64
+    s = session.Session(TINY, max_tokens=T, n_layers=1, flags=capi.MOE_FLAG_TEST_WITHHOLD)
+    ref = session.Session(TINY, max_tokens=T, n_layers=1)
+    W = synth.layer_weights(TINY, 0, device="cuda")
+    s.load(0, W)
+    ref.load(0, W)
+    del W
+    x = _tokens(TINY, T, stream=78)
+    _run(s, 0, x)
+    assert capi.moe_get_device_error(s.ctx) == capi.MOE_ERR_DEVICE_TIMEOUT
+    yb, yfb, idb, wb = _run(ref, 0, x)
+    for rep in range(3):
+        y, yf, ids, w = _run(s, 0, x)
+        assert capi.moe_get_device_error(s.ctx) == 0
+        assert np.array_equal(ids, idb)
+        assert rel_l2(yf, yfb) <= 1e-5
+    s.close()
+    ref.close()
+
+
 def _tiny_weights_with(mutate):
     W = synth.layer_weights(TINY, 0, device="cuda")
     mutate(W)

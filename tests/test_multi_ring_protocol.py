@@ -4,10 +4,9 @@ One CTA, one layer, random interleavings of the producer (fills items in
 order, refilling a slot once its previous item is consumed) and the compute
 warps:
 
-* gate/up items: one unit each of nkg k-group steps; the units' steps form
-  one sequence cut into NW near-equal contiguous ranges, one per warp, so a
-  unit may be cut into parts taken by several warps; the last part of a unit
-  to finish frees its slot;
+* gate/up items: one unit each, cut into four k-group chunks; the CTA's
+  chunks go round-robin to all warps, and the last chunk of a unit to finish
+  frees its slot;
 * down items: batches of units; units go round-robin to all warps, the warp
   that finishes an item's last unit frees the slot;
 * before waiting on a slot, a unit's warp waits until every earlier item of
@@ -22,7 +21,7 @@ consumer reads the fill it expects.  Two planted mistakes show the check is
 not vacuous: without the wait on the slot's earlier items a unit reads an
 older fill (or the run stalls), a slot freed by the first unit of an item
 instead of the last lets the producer overwrite units still being read, and
-a gate/up slot freed by the first part of a cut unit does the same.
+a gate/up slot freed by the first chunk of a unit does the same.
 """
 import random
 
@@ -48,21 +47,13 @@ class Stale(AssertionError):
     pass
 
 
-def gu_parts(n_gu, nkg, NW):
-    """Per warp, its (unit, parts of that unit) list: balanced ranges of the n_gu * nkg steps."""
-    S = n_gu * nkg
-    rng = [(w * S // NW, (w + 1) * S // NW) for w in range(NW)]
-    owners = {}
-    for w, (lo, hi) in enumerate(rng):
-        for q in range(lo // nkg, (hi - 1) // nkg + 1) if lo < hi else []:
-            owners.setdefault(q, []).append(w)
-    # the kernel finds a unit's first and last warp from its first and last step
-    def warp_of(x):
-        return ((x + 1) * NW + S - 1) // S - 1
-    for q, ws in owners.items():
-        assert ws[0] == warp_of(q * nkg) and ws[-1] == warp_of(q * nkg + nkg - 1)
-        assert ws == list(range(ws[0], ws[-1] + 1))
-    return [[(q, len(owners[q])) for q in sorted(owners) if w in owners[q]] for w in range(NW)]
+def gu_parts(n_gu, nkg, NW, nch=4):
+    """Per warp, its (unit, chunks of that unit) list in processing order: unit q is cut into nch
+    k-group chunks and the CTA's chunk c goes to warp c % NW."""
+    plan = [[] for _ in range(NW)]
+    for ch in range(n_gu * nch):
+        plan[ch % NW].append((ch // nch, nch))
+    return plan
 
 
 def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_last=True, nkg=40,
@@ -110,7 +101,7 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
                     s, q, nparts = ws["busy"]
                     reading[s] -= 1
                     pcnt[q] = pcnt.get(q, 0) + 1
-                    # planted mistake: the first part of a cut unit to finish frees the slot
+                    # planted mistake: the first chunk of a unit to finish frees the slot
                     if pcnt[q] == (nparts if gu_free_on_last else 1):
                         ccnt[s] += 1
                         empty[s].arrive()
@@ -185,26 +176,16 @@ CASES = [(5, 32, 81, 5), (5, 33, 81, 5), (7, 8, 20, 5), (5, 8, 4, 5), (8, 21, 52
 
 
 @pytest.mark.parametrize("n_gu", [1, 2, 5, 7, 8, 11, 12, 13, 24, 35])
-def test_gate_up_ranges_cover_every_step_once(n_gu):
-    nkg, NW = 40, 12
-    plan = gu_parts(n_gu, nkg, NW)
-    S = n_gu * nkg
-    steps = []
-    for w in range(NW):
-        lo, hi = w * S // NW, (w + 1) * S // NW
-        steps += list(range(lo, hi))
-        # a cut unit is the first or the last of each warp that takes part of it
-        cut = [q for q, n in plan[w] if n > 1]
-        units = [q for q, _ in plan[w]]
-        assert all(q in (units[0], units[-1]) for q in cut)
-    assert steps == list(range(S))
-    # slots of cut units (their first warp) are distinct and below NW - 1
-    firsts = {}
-    for w in range(NW):
-        for q, n in plan[w]:
-            if n > 1:
-                firsts.setdefault(q, w)
-    assert len(set(firsts.values())) == len(firsts) and all(f < NW - 1 for f in firsts.values())
+def test_gate_up_chunks_cover_every_step_once(n_gu):
+    """The kernel's chunk bounds kb = j nkg / 4, ke = (j + 1) nkg / 4 tile every unit's k groups."""
+    for nkg in (4, 5, 40, 48):
+        for q in range(n_gu):
+            steps = []
+            for j in range(4):
+                steps += list(range(j * nkg // 4, (j + 1) * nkg // 4))
+            assert steps == list(range(nkg))
+    plan = gu_parts(n_gu, 40, 12)
+    assert sorted(q for w in plan for q, _ in w) == sorted(q for q in range(n_gu) for _ in range(4))
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -225,7 +206,7 @@ def test_planted_no_wait_on_earlier_items_is_caught():
     assert caught > 0
 
 
-def test_planted_gate_up_slot_freed_by_first_part_is_caught():
+def test_planted_gate_up_slot_freed_by_first_chunk_is_caught():
     caught = 0
     for seed in range(25):
         try:
