@@ -370,6 +370,19 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
         step_roof = {"alg_bytes_per_step": step_bytes, "experts_streamed_per_layer": statistics.mean(unions),
                      "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
                      "frac": step_bytes / (ms_step / 1e3) / 1e9 / P["hbm_gbs"]}
+    l2_ab = None
+    if not tensor_bound:
+        # L2 residency: the same steps with every weight copy at the default eviction priority, against
+        # the default mode that keeps the shared experts (every layer's) in L2 across steps
+        capi.moe_set_l2_policy(sess.ctx, capi.MOE_L2_STREAM)
+        ms_stream, _ = timed_steps(capi, sess, cfg, xs, out, args.steps, args.warmup, stream, dist_on, flush)
+        capi.moe_set_l2_policy(sess.ctx, capi.MOE_L2_KEEP_SHARED)
+        ms_stream = max_over_ranks(ms_stream, dist_on, dev) / args.steps
+        kept = cfg.L * cfg.n_shared * expert_bytes(cfg)
+        l2_ab = {"mode": "shared experts evict_last, routed experts and router rows evict_first",
+                 "kept_bytes": kept, "kept_fraction_of_step_bytes": kept / step_bytes,
+                 "value_keep_shared": value, "value_stream": whole_job_rate(cfg.T, world, ms_stream / 1e3),
+                 "speedup": ms_stream / ms_step}
 
     # end to end through the public host-buffer entry point (copies inside the timed region)
     x_host = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).pin_memory()
@@ -403,6 +416,7 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
         "dtype": ("fp16 tensor-core MMA, fp32 accumulate, over " if tensor_bound else
                   "exact code operands, fp32 accumulate, over ") + fmt + " weights / bf16 activations",
         "roofline": roof, "step_roofline": step_roof, "e2e": e2e,
+        **({"l2_residency": l2_ab} if l2_ab else {}),
         "gpu_launches": tim["all_launches"], "clocks": clocks,
     }
     if with_cpu:
@@ -565,6 +579,8 @@ def main():
         }
         if "cpu_baseline" in head:
             out["cpu_baseline"] = head["cpu_baseline"]
+        if "l2_residency" in head:
+            out["l2_residency"] = head["l2_residency"]
         if world == 1 and not args.no_secondary and args.layers is None:
             out["secondary"] = {}
             for name in SECONDARY:

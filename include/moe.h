@@ -172,10 +172,11 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  *   weight) and w [T][k] their weights, either may be NULL.
  * Asynchronous on `stream`; no host synchronisation and no allocation.
  * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA.
- * Implementation (not part of the contract): up to 8 tokens run the
- * persistent single-token kernel once per token, 9 and more the tensor-core
- * grouped GEMMs; the CUDA-core grouped path runs where neither fits the shape
- * (or under MOE_FLAG_NO_DECODE_KERNEL / MOE_FLAG_NO_TENSOR_PREFILL); each path
+ * Implementation (not part of the contract): one token runs the persistent
+ * single-token kernel, 2 to 16 tokens the persistent few-token kernel (one
+ * launch per 8 tokens, reading the union of their experts once per layer),
+ * 17 and more the tensor-core grouped GEMMs; the CUDA-core grouped path runs
+ * where none fits the shape (or under the MOE_FLAG_NO_* flags); each path
  * meets the same accuracy bound. */
 MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
                 uint16_t *y_bf16, float *y_f32, int32_t *ids, float *w,
@@ -219,6 +220,22 @@ MOE_API int moe_destroy(moe_ctx *ctx);
  * up part-way leaves mid-count: after a nonzero code, call this before the
  * next forward on the context. */
 MOE_API int moe_get_device_error(moe_ctx *ctx, int *code);
+
+/* L2 residency of the decode kernels' weight stream, the counterpart on one
+ * GPU of the pages' expert cache, which keeps the experts in use in the
+ * faster memory ("Qwen3.8-Flash-Next on RTX 5090 + 64GB", section 2 "Expert
+ * Cache and CPU/GPU Split").  Here every expert already lives in HBM; the
+ * shared experts are read by every token of every call, so in mode
+ * MOE_L2_KEEP_SHARED (the default) their tiles are copied with the L2
+ * eviction priority evict_last and the routed experts' tiles and the router
+ * rows with evict_first, which keeps the shared experts of all layers in the
+ * 126 MB L2 across calls when they fit; MOE_L2_STREAM copies everything with
+ * the default priority.  Applies to the single-token and few-token kernels;
+ * results do not depend on it.  Errors: INVALID_ARG (NULL context, unknown
+ * mode). */
+#define MOE_L2_STREAM 0
+#define MOE_L2_KEEP_SHARED 1
+MOE_API int moe_set_l2_policy(moe_ctx *ctx, int mode);
 
 /* Measurement hook.  While enabled, each forward records a CUDA event pair on
  * the caller's stream around its dominant kernel (the kernel that streams the

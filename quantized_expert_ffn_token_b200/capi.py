@@ -32,6 +32,8 @@ MOE_FLAG_NO_MULTI_DECODE = 8
 MOE_FLAG_SPLIT_DECODE = 16
 MOE_FLAG_TEST_WITHHOLD = 256
 MOE_FLAG_TRACE = 4
+MOE_L2_STREAM = 0
+MOE_L2_KEEP_SHARED = 1
 MOE_ROUTE_STATIC_MAX_LOGITS = 65536
 FORMATS = {"q4": MOE_Q4B32, "q3": MOE_Q3B32, "q2": MOE_Q2B32}
 
@@ -39,7 +41,7 @@ EXPORTED = [
     "moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
     "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
     "moe_status_string", "moe_last_error", "moe_timing_enable", "moe_timing_read",
-    "moe_trace_read", "moe_route_static",
+    "moe_trace_read", "moe_route_static", "moe_set_l2_policy",
 ]
 
 
@@ -83,6 +85,7 @@ def _load() -> ctypes.CDLL:
     L.moe_destroy.argtypes = [vp]
     L.moe_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
     L.moe_timing_enable.argtypes = [vp, i]
+    L.moe_set_l2_policy.argtypes = [vp, i]
     L.moe_timing_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
                                   ctypes.POINTER(ctypes.c_longlong), ctypes.c_char_p, i]
     L.moe_trace_read.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong), i, ctypes.POINTER(i)]
@@ -93,7 +96,8 @@ def _load() -> ctypes.CDLL:
     L.moe_last_error.restype = ctypes.c_char_p
     for n in ("moe_create", "moe_load_layer", "moe_forward", "moe_forward_stack",
               "moe_forward_stack_host", "moe_destroy", "moe_get_device_error",
-              "moe_timing_enable", "moe_timing_read", "moe_trace_read", "moe_route_static"):
+              "moe_timing_enable", "moe_timing_read", "moe_trace_read", "moe_route_static",
+              "moe_set_l2_policy"):
         getattr(L, n).restype = i
     return L
 
@@ -163,6 +167,11 @@ def moe_forward_stack_host(ctx, layer0: int, n_layers: int, x_host, T: int, resi
 
 def moe_destroy(ctx) -> None:
     _check(lib.moe_destroy(ctx), "moe_destroy")
+
+
+def moe_set_l2_policy(ctx, mode: int) -> None:
+    """L2 eviction priorities of the decode kernels' weight copies (see include/moe.h)."""
+    _check(lib.moe_set_l2_policy(ctx, mode), "moe_set_l2_policy")
 
 
 def moe_get_device_error(ctx) -> int:

@@ -91,6 +91,7 @@ struct DecodeParams {
     float *x_y;                // [2][d]: the two parts of every output row
     int *err;
     int withhold;              // test hook: CTA 0 does not publish its logits
+    int l2_mode;               // 0: plain copies; 1: shared experts kept in L2, the rest streamed
     unsigned long long *trace; // [G][L][TRACE_WORDS] phase clocks, or NULL
     int nslot, slot_bytes, rpc;
     int off_ring, off_router, off_x16, off_xh, off_logits, off_htab, off_red, off_misc, off_resid, off_sums,
@@ -256,6 +257,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
     // ---- producer warp (lane 0): every bulk copy, paced by mbarriers only ----------------
     if (warp == NW) {
         if (lane != 0) return;
+        const uint64_t keep_pol = l2_policy(true), stream_pol = l2_policy(false);
         uint32_t gu_par = 0;     // bit s: parity of the gate/up items issued into slot s so far
         uint32_t fill_par = 0;   // bit s: parity of all fills of slot s so far
         uint32_t filled = 0;     // bit s: slot s was filled at least once
@@ -269,7 +271,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
             fence_proxy_async();
             mbar_expect_tx(&ms->rbar, (uint32_t)(nrows * d * 4));
             for (int j = 0; j < nrows; ++j)
-                bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
+                weight_copy(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar,
+                            p.l2_mode, false, keep_pol, stream_pol);
             ++router_fills;
         };
         issue_router(p.layer0);
@@ -283,20 +286,21 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
             if (!mbar_wait(&ms->route, (uint32_t)(l & 1), err, true)) break;
             const Split sp = split();
             bool pok = true;
+            fence_proxy_async();   // (the compute warps only read the ring)
             for (int q = 0; q < sp.n_items && pok; ++q) {
                 uint32_t par;
                 const int s = ring_slot(s0, p0, q, par);
                 // items past the ring reuse a slot whose gate/up unit of this layer is consumed
                 if (q >= p.nslot) pok = mbar_wait(&ms->empty[s], ((gu_par >> s) & 1u) ^ 1u, err, true);
                 if (!pok) break;
-                fence_proxy_async();
                 uint8_t *dst = ring + (size_t)s * p.slot_bytes;
                 if (q < sp.n_gu) {
                     const int u = cta + G * q;
                     const int us = u / ntile_gu, t = u % ntile_gu;
                     const uint8_t *src = Lp.gu + (size_t)ms->uexp[us] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
                     mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
-                    bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
+                    weight_copy(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s], p.l2_mode, ms->uexp[us] >= E,
+                                keep_pol, stream_pol);
                     gu_par ^= 1u << s;
                 } else {
                     const int q0 = (q - sp.n_gu) * dn_per_slot;
@@ -306,7 +310,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode(DecodeParams p) {
                         const int n = sp.dn_lo + q0 + i;
                         const int j = n / nU, us = n % nU;
                         const uint8_t *src = Lp.dn + (size_t)ms->uexp[us] * p.dn.expert_bytes + (size_t)j * p.dn.tile_bytes;
-                        bulk_g2s(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s]);
+                        weight_copy(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s],
+                                    p.l2_mode, ms->uexp[us] >= E, keep_pol, stream_pol);
                     }
                 }
                 fill_par ^= 1u << s;
@@ -1178,6 +1183,7 @@ int launch_decode(moe_ctx *ctx, int layer0, int L, const uint16_t *x, bool stack
     // test hook: the context's first single-token call withholds CTA 0's logits
     p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ds.withheld) ? 1 : 0;
     if (p.withhold) ds.withheld = true;
+    p.l2_mode = ctx->l2_mode;
     if (c.flags & MOE_FLAG_TRACE) QE_TRY(decode_trace_buffer(ctx, ds.grid, L, TRACE_WORDS, st, &p.trace));
     p.nslot = ds.nslot;
     p.slot_bytes = ds.slot_bytes;

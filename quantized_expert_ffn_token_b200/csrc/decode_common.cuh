@@ -48,6 +48,33 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// L2 residency of the streamed weights.  Every layer streams the union of its experts once per
+// call; the shared expert (and the router rows) recur in every call, the routed ones only when
+// chosen again.  A copy can carry an L2 eviction priority: evict_last for the bytes worth keeping
+// (the shared experts), evict_first for the rest, so that the stream does not push the kept
+// bytes out of the 126 MB L2.
+__device__ __forceinline__ uint64_t l2_policy(bool keep) {
+    uint64_t pol;
+    if (keep)
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    else
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes,
+                                              unsigned long long *bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// A weight copy under the context's L2 mode: 0 plain, 1 shared experts kept and the rest streamed.
+__device__ __forceinline__ void weight_copy(void *dst, const void *src, uint32_t bytes, unsigned long long *bar,
+                                            int l2_mode, bool shared, uint64_t keep_pol, uint64_t stream_pol) {
+    if (l2_mode == 0) bulk_g2s(dst, src, bytes, bar);
+    else bulk_g2s_hint(dst, src, bytes, bar, shared ? keep_pol : stream_pol);
+}
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

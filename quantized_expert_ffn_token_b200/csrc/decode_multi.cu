@@ -105,6 +105,7 @@ struct MultiParams {
     float *r_buf;                  // [2][TM][d] residual stream (stack)
     int *err;
     int withhold;
+    int l2_mode;                   // 0: plain copies; 1: shared experts kept in L2, the rest streamed
     unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
     int off_ring, off_router, off_xb, off_hsum, off_uexp, off_wtab,
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     // ---- producer warp (lane 0) -----------------------------------------------------------
     if (warp == NW) {
         if (lane != 0) return;
+        const uint64_t keep_pol = l2_policy(true), stream_pol = l2_policy(false);
         uint32_t fpar = 0;       // bit s: parity of the fills of slot s so far
         uint32_t filled = 0;     // bit s: slot s was filled at least once
         int router_fills = 0;
@@ -285,7 +287,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             fence_proxy_async();
             mbar_expect_tx(&ms->rbar, (uint32_t)(nrows * d * 4));
             for (int j = 0; j < nrows; ++j)
-                bulk_g2s(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar);
+                weight_copy(rtr + (size_t)j * d, rw + (size_t)(cta + G * j) * d, (uint32_t)(d * 4), &ms->rbar,
+                            p.l2_mode, false, keep_pol, stream_pol);
             ++router_fills;
         };
         issue_router(0);
@@ -308,7 +311,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     const int u = n / ntile_gu, t = n - u * ntile_gu;
                     const uint8_t *src = Lp.gu + (size_t)uexp[u] * p.gu.expert_bytes + (size_t)t * p.gu.tile_bytes;
                     mbar_expect_tx(&ms->full[s], (uint32_t)p.gu.tile_bytes);
-                    bulk_g2s(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s]);
+                    weight_copy(dst, src, (uint32_t)p.gu.tile_bytes, &ms->full[s], p.l2_mode, uexp[u] >= E, keep_pol,
+                                stream_pol);
                 } else {
                     const int q0 = (q - sp.n_gu) * dn_per_slot;
                     const int cnt = min(dn_per_slot, sp.n_dn - q0);
@@ -317,7 +321,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                         const int n = sp.dn_lo + q0 + i;
                         const int u = n / ntile_dn, j = n - u * ntile_dn;
                         const uint8_t *src = Lp.dn + (size_t)uexp[u] * p.dn.expert_bytes + (size_t)j * p.dn.tile_bytes;
-                        bulk_g2s(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s]);
+                        weight_copy(dst + (size_t)i * p.dn.tile_bytes, src, (uint32_t)p.dn.tile_bytes, &ms->full[s],
+                                    p.l2_mode, uexp[u] >= E, keep_pol, stream_pol);
                     }
                 }
                 fpar ^= 1u << s;
@@ -1260,6 +1265,7 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.err = ctx->ws.dev_error;
     p.withhold = ((c.flags & MOE_FLAG_TEST_WITHHOLD) && !ctx->dec.withheld) ? 1 : 0;
     if (p.withhold) ctx->dec.withheld = true;
+    p.l2_mode = ctx->l2_mode;
     if (c.flags & MOE_FLAG_TRACE) QE_TRY(decode_trace_buffer(ctx, ms.grid, L, TRACE_WORDS_M, st, &p.trace));
     p.nslot = ms.nslot;
     p.slot_bytes = ms.slot_bytes;

@@ -472,6 +472,12 @@ int moe_get_device_error(moe_ctx *ctx, int *code) {
     return MOE_OK;
 }
 
+int moe_set_l2_policy(moe_ctx *ctx, int mode) {
+    if (!ctx || (mode != MOE_L2_STREAM && mode != MOE_L2_KEEP_SHARED)) return MOE_ERR_INVALID_ARG;
+    ctx->l2_mode = mode;
+    return MOE_OK;
+}
+
 int moe_timing_enable(moe_ctx *ctx, int on) {
     if (!ctx) return MOE_ERR_INVALID_ARG;
     QE_CHECK(cudaSetDevice(ctx->device));

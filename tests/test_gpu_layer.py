@@ -324,6 +324,37 @@ def test_tensor_core_wait_times_out_and_context_recovers():
     ref.close()
 
 
+@pytest.mark.parametrize("T", [1, 4])
+def test_l2_policy_leaves_results_unchanged(T):
+    """The decode kernels' L2 eviction priorities change where the weights are
+    cached, never what is computed: a two-layer stack gives the same residual
+    stream under both modes (bit for bit for one token, whose kernel sums in a
+    fixed order; for several tokens the few-token kernel's fp32 atomics sum in
+    no fixed order, so two runs in the same mode differ too, and the bound is
+    the one its tests use against the single-token kernel)."""
+    capi, session = _cuda()
+    cfg = synth.CONFIGS["verify_48l_q3_t4_zipf"]
+    s = session.Session(cfg, max_tokens=max(T, 2), n_layers=2)
+    s.load_synthetic()
+    x = torch.from_numpy(_tokens(cfg, T, stream=91).view(np.int16)).cuda()
+    outs = []
+    for mode in (capi.MOE_L2_STREAM, capi.MOE_L2_KEEP_SHARED, capi.MOE_L2_KEEP_SHARED):
+        capi.moe_set_l2_policy(s.ctx, mode)
+        r = torch.empty((T, cfg.d), dtype=torch.float32, device="cuda")
+        capi.moe_forward_stack(s.ctx, 0, 2, x, T, r)
+        torch.cuda.synchronize()
+        assert capi.moe_get_device_error(s.ctx) == 0
+        outs.append(to_np(r))
+    for o in outs[1:]:
+        if T == 1:
+            assert np.array_equal(o, outs[0])
+        else:
+            assert rel_l2(o, outs[0]) <= 1e-4
+    with pytest.raises(capi.MoeError):
+        capi.moe_set_l2_policy(s.ctx, 7)
+    s.close()
+
+
 def _tiny_weights_with(mutate):
     W = synth.layer_weights(TINY, 0, device="cuda")
     mutate(W)
