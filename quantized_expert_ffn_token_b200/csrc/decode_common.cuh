@@ -230,6 +230,23 @@ __device__ __forceinline__ unsigned ctr_load(const unsigned *c) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
     return v;
 }
+// Tagged words: a 32-bit value and a 32-bit tag in one naturally aligned 64-bit store, so a reader
+// that sees the tag it expects also sees the value (single-copy atomicity of the 64-bit access) and
+// no release fence or arrival counter has to order the two.
+__device__ __forceinline__ void st_tagged(unsigned long long *p, float v, unsigned tag) {
+    const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long *p) {
+    unsigned long long w;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+    return w;
+}
+__device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long *p) {   // two tagged words
+    ulonglong2 w;
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
+    return w;
+}
 __device__ __forceinline__ float ld_gpu(const float *p) {
     float v;
     asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");

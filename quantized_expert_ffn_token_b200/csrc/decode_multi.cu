@@ -99,8 +99,9 @@ struct MultiParams {
     moe_stack_record rec;          // records: token t is record row rec_r0 + t of rec_n
     int rec_on, rec_n, rec_r0;
     unsigned *cnt;                 // [0] logits, [32] y and [64] h arrivals (one per CTA and layer each)
-    float *x_logits;               // [TM][E]
-    float *x_h;                    // [UM][TM][I]
+    unsigned long long *x_logits;  // [TM][E] tagged logits: (tag << 32) | float bits
+    unsigned tag0;                 // tag of this launch's first layer (tag0 + l for layer l)
+    unsigned long long *x_h;       // [UM][TM][I] tagged h (same tags as the logits)
     float *y_acc;                  // [2][TM][d] layer outputs, accumulated with atomics
     float *r_buf;                  // [2][TM][d] residual stream (stack)
     int *err;
@@ -112,7 +113,7 @@ struct MultiParams {
         off_misc, off_ltab;
 };
 
-constexpr int C_LOGITS = 0, C_Y = 32, C_H = 64;   // counters, 128 bytes apart
+constexpr int C_Y = 32;   // the layer-output arrival counter
 
 // Phase trace (MOE_FLAG_TRACE): per (CTA, layer) record of 24 words: CTA, layer, then SM clock
 // cycles since the layer started in this CTA:
@@ -538,11 +539,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     acc = fmaf(wv.w, bf16f(xv.y >> 16), acc);
                 }
                 for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (lane == 0) p.x_logits[(size_t)t * E + cta + G * j] = acc + ms->rbias[j];
+                if (lane == 0 && !(p.withhold && cta == 0))
+                    st_tagged(p.x_logits + (size_t)t * E + cta + G * j, acc + ms->rbias[j], p.tag0 + l);
             }
         }
         csync();   // this CTA's logits are stored; the router rows and the bf16 rows are no longer read
-        if (tid == 0 && !(p.withhold && cta == 0)) ctr_arrive(p.cnt + C_LOGITS);
         mark(1, clock64() - tl0);
         // the gate/up B operand in place of the bf16 rows: within each token's 64-wide k group the
         // words are reordered so that lane c's eight B registers of the group (slices 0..3, both
@@ -575,37 +576,50 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             for (int j = 0; j < 8; ++j) pv[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         }
         mark(16, clock64() - tl0);
-        if (tid == 0) {
-            ok = ctr_wait(p.cnt + C_LOGITS, (unsigned)(G * (l + 1)), err);
-        }
-        if (cta_failed(ok)) {
-            aborted = true;
-            break;
-        }
-        mark(2, clock64() - tl0);
-        // every CTA has read the previous layer's output: clear the owned columns of its buffer,
-        // which accumulates the next layer's output
-        if (l >= 1 && l + 1 < p.L) {
-            float *ynext = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
-            for (int i = tid; i < T * (own_hi - own_lo); i += NT) {
-                const int t = i / (own_hi - own_lo), i4 = own_lo + i - t * (own_hi - own_lo);
-                *reinterpret_cast<float4 *>(ynext + (size_t)t * d + 4 * i4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
 
         // ---- 3. top-k per token (warp t), union, weights --------------------------------------------
         // Threshold and rank: the k-th largest of the 32 lanes' maxima is a lower bound of the k-th
         // largest logit, so every expert of the top k is among the values at or above it; those
         // candidates are ranked by counting the candidates ordered before each (larger logit, equal
         // logits: lower id).  Too many candidates (flat or equal logits): k rounds of warp arg-max.
+        // The logits arrive tagged: a warp reads its token's row and re-reads (bounded) the words whose
+        // tag is not yet this layer's; a CTA's top-k warps have then seen every CTA's router output,
+        // i.e. every CTA is past its input phase.
         if (warp < T) {
             const int t = warp;
             float v[EPL];
             float lmax = -INFINITY;
+            unsigned long long wv[EPL];
+            const unsigned want = p.tag0 + l;
+            const unsigned long long *row = p.x_logits + (size_t)t * E;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) wv[i] = (lane + 32 * i < E) ? ld_tagged(row + lane + 32 * i) : 0ull;
+            bool got = true;
+            {
+                // words not yet tagged for this layer are read again together, round after round
+                const long long tw = clock64();
+                for (int it = 0;; ++it) {
+                    unsigned late = 0u;
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i)
+                        if (lane + 32 * i < E && (unsigned)(wv[i] >> 32) != want) late |= 1u << i;
+                    if (!late) break;
+                    if ((it & 15) == 15 && (*(volatile int *)err != 0 || clock64() - tw > SPIN_LIMIT)) {
+                        atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                        got = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i)
+                        if ((late >> i) & 1u) wv[i] = ld_tagged(row + lane + 32 * i);
+                }
+            }
+            if (!got) ok = false;
+            mark(2, clock64() - tl0);
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = lane + 32 * i;
-                float x = (e < E) ? __ldcg(p.x_logits + (size_t)t * E + e) : __int_as_float(0x7fc00000);
+                float x = (e < E) ? __uint_as_float((unsigned)wv[i]) : __int_as_float(0x7fc00000);
                 if (e < E && isnan(x)) x = -INFINITY;   // a NaN logit ranks as -inf (last, by id)
                 v[i] = x;                               // past E: NaN, never a candidate
                 if (e < E) lmax = fmaxf(lmax, x);
@@ -715,8 +729,20 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
             }
         }
-        csync();   // the union bitmap is complete
+        if (cta_failed(ok)) {   // the union bitmap is complete (or a token's logits never came)
+            aborted = true;
+            break;
+        }
         mark(19, clock64() - tl0);
+        // every CTA has read the previous layer's output: clear the owned columns of its buffer,
+        // which accumulates the next layer's output
+        if (l >= 1 && l + 1 < p.L) {
+            float *ynext = p.y_acc + (size_t)((l + 1) & 1) * TM * d;
+            for (int i = tid; i < T * (own_hi - own_lo); i += NT) {
+                const int t = i / (own_hi - own_lo), i4 = own_lo + i - t * (own_hi - own_lo);
+                *reinterpret_cast<float4 *>(ynext + (size_t)t * d + 4 * i4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
         // Union in ascending expert order, then the shared experts: an expert's union slot is the
         // number of bitmap ones below it.  Warp t < T writes column t of the weight table; the last
         // warp lists the union; the others clear the gate/up chunk sums (they share memory with the
@@ -873,11 +899,13 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     const int u = n / ntile_gu, t8 = n - u * ntile_gu;
                     if (l0) {
                         const float xi = ms->xinv[t0];
-                        p.x_h[((size_t)u * TM + t0) * I + 8 * t8 + g] = silu(acc[0] * xi) * (acc[2] * xi);
+                        st_tagged(p.x_h + ((size_t)u * TM + t0) * I + 8 * t8 + g, silu(acc[0] * xi) * (acc[2] * xi),
+                                  p.tag0 + l);
                     }
                     if (l1) {
                         const float xi = ms->xinv[t1];
-                        p.x_h[((size_t)u * TM + t1) * I + 8 * t8 + g] = silu(acc[1] * xi) * (acc[3] * xi);
+                        st_tagged(p.x_h + ((size_t)u * TM + t1) * I + 8 * t8 + g, silu(acc[1] * xi) * (acc[3] * xi),
+                                  p.tag0 + l);
                     }
                     __syncwarp();
                     if (lane == 0) {
@@ -893,37 +921,65 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             aborted = true;
             break;
         }
-        // this CTA's h values are stored: one release for all of them
-        if (tid == 0) ctr_arrive(p.cnt + C_H);
         mark(4, clock64() - tl0);
 
         // ---- 5. down ---------------------------------------------------------------------------------
         const int u_first = sp.n_dn > 0 ? sp.dn_lo / ntile_dn : 0;
         const int n_span = sp.n_dn > 0 ? (sp.dn_hi - 1) / ntile_dn - u_first + 1 : 0;
         if (n_span > 0) {
-            if (tid == 0) ok = ctr_wait(p.cnt + C_H, (unsigned)(G * (l + 1)), err);
-            if (cta_failed(ok)) {
-                aborted = true;
-                break;
-            }
             mark(5, clock64() - tl0);
             // h of the run's experts -> hi + lo B fragments (columns of the T tokens; the rest is
             // masked where it is read) and, per (expert, token, 32-block), the sum of hi + lo and
             // (fp16) the block's 2^-s
             const int nq = n_span * T * (I / 4);   // 4 values per thread and step; 8 lanes per block
-            for (int i0 = 0; i0 < nq; i0 += HB_M * NT) {
-              float4 hb[HB_M];   // a batch of loads in flight together, then the arithmetic
+            // h arrives tagged: the words of a batch are read together, and those not yet tagged for
+            // this layer are read again together, round after round (bounded)
+            const unsigned want = p.tag0 + l;
+            for (int i0 = 0; i0 < nq; i0 += HB_M * NT) {   // every lane runs every batch (shuffles below)
+              ulonglong2 hw[HB_M][2];
+              const unsigned long long *hp[HB_M];
 #pragma unroll
               for (int bq = 0; bq < HB_M; ++bq) {
                 const int i = i0 + bq * NT + tid;
-                hb[bq] = make_float4(0.f, 0.f, 0.f, 0.f);
+                hp[bq] = nullptr;
+                hw[bq][0] = hw[bq][1] = make_ulonglong2((unsigned long long)want << 32, (unsigned long long)want << 32);
                 if (i < nq) {
                     const int su = i / (T * (I / 4));
                     const int rem = i - su * (T * (I / 4));
                     const int t = rem / (I / 4), k4 = rem - t * (I / 4);
-                    hb[bq] = __ldcg(reinterpret_cast<const float4 *>(p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4));
+                    hp[bq] = p.x_h + ((size_t)(u_first + su) * TM + t) * I + 4 * k4;
+                    hw[bq][0] = ld_tagged2(hp[bq]);
+                    hw[bq][1] = ld_tagged2(hp[bq] + 2);
                 }
               }
+              {
+                const long long tw = clock64();
+                for (int it = 0;; ++it) {
+                  unsigned late = 0u;
+#pragma unroll
+                  for (int bq = 0; bq < HB_M; ++bq)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                      if ((unsigned)(hw[bq][hh].x >> 32) != want || (unsigned)(hw[bq][hh].y >> 32) != want)
+                        late |= 1u << (2 * bq + hh);
+                  if (!late) break;
+                  if ((it & 15) == 15 && (*(volatile int *)err != 0 || clock64() - tw > SPIN_LIMIT)) {
+                    atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+                    ok = false;
+                    break;
+                  }
+#pragma unroll
+                  for (int bq = 0; bq < HB_M; ++bq)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                      if ((late >> (2 * bq + hh)) & 1u) hw[bq][hh] = ld_tagged2(hp[bq] + 2 * hh);
+                }
+              }
+              float4 hb[HB_M];
+#pragma unroll
+              for (int bq = 0; bq < HB_M; ++bq)
+                hb[bq] = make_float4(__uint_as_float((unsigned)hw[bq][0].x), __uint_as_float((unsigned)hw[bq][0].y),
+                                     __uint_as_float((unsigned)hw[bq][1].x), __uint_as_float((unsigned)hw[bq][1].y));
 #pragma unroll
               for (int bq = 0; bq < HB_M; ++bq) {
                 const int i = i0 + bq * NT + tid;
@@ -984,7 +1040,10 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 }
               }
             }
-            csync();
+        }
+        if (cta_failed(ok)) {   // the h table is complete (or some h never came)
+            aborted = true;
+            break;
         }
         mark(6, clock64() - tl0);
         // units of this CTA's run, in batches of dn_per_slot (one ring item each); units go round-robin
@@ -1081,7 +1140,8 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             }
         }
         ring_base += sp.n_items;
-        __threadfence();
+        // (the output atomics are ordered before the arrival below by this barrier and the
+        // arriving thread's release, which is cumulative)
         if (cta_failed(ok)) {
             aborted = true;
             break;
@@ -1145,10 +1205,10 @@ static int multi_um(const moe_config &c) { return multi_tm(c) * c.top_k + c.n_sh
 size_t decode_multi_counter_bytes(const moe_config &) { return 512; }
 static size_t xm_logits_off(const moe_config &c) { return decode_multi_counter_bytes(c); }
 static size_t xm_h_off(const moe_config &c) {
-    return xm_logits_off(c) + (((size_t)multi_tm(c) * c.n_experts * 4 + 255) & ~(size_t)255);
+    return xm_logits_off(c) + (((size_t)multi_tm(c) * c.n_experts * 8 + 255) & ~(size_t)255);
 }
 static size_t xm_y_off(const moe_config &c) {
-    return xm_h_off(c) + (size_t)multi_um(c) * multi_tm(c) * c.d_ff * 4;
+    return xm_h_off(c) + (size_t)multi_um(c) * multi_tm(c) * c.d_ff * 8;
 }
 static size_t xm_r_off(const moe_config &c) { return xm_y_off(c) + (size_t)2 * multi_tm(c) * c.d_model * 4; }
 size_t decode_multi_xchg_bytes(const moe_config &c) {
@@ -1258,8 +1318,17 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     }
     uint8_t *xb = ms.xbuf;
     p.cnt = reinterpret_cast<unsigned *>(xb);
-    p.x_logits = reinterpret_cast<float *>(xb + xm_logits_off(c));
-    p.x_h = reinterpret_cast<float *>(xb + xm_h_off(c));
+    p.x_logits = reinterpret_cast<unsigned long long *>(xb + xm_logits_off(c));
+    // tags of this launch's layers; the area starts zeroed and tags start at 1, so no stale word
+    // (earlier launch, earlier layer) carries a tag a reader expects
+    p.tag0 = ms.tag;
+    ms.tag += (unsigned)L;
+    if (ms.tag < p.tag0) {   // wrapped: start the tags over on a cleared area
+        QE_CHECK(cudaMemsetAsync(xb + xm_logits_off(c), 0, xm_y_off(c) - xm_logits_off(c), st));
+        p.tag0 = 1;
+        ms.tag = 1 + (unsigned)L;
+    }
+    p.x_h = reinterpret_cast<unsigned long long *>(xb + xm_h_off(c));
     p.y_acc = reinterpret_cast<float *>(xb + xm_y_off(c));
     p.r_buf = reinterpret_cast<float *>(xb + xm_r_off(c));
     p.err = ctx->ws.dev_error;

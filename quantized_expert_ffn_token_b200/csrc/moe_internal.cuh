@@ -242,6 +242,7 @@ struct MultiState {
     int off_ring = 0, off_router = 0, off_xb = 0, off_hsum = 0, off_uexp = 0,
         off_wtab = 0, off_misc = 0, off_ltab = 0;
     uint8_t *xbuf = nullptr;   // counters, logits, h, output and residual buffers
+    unsigned tag = 1;          // tag of the next launch's first layer in the tagged logits area
 };
 
 // Launch plan of the single-token split kernel (decode_split.cu).
