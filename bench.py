@@ -426,33 +426,38 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
 
 # ---- token-count sweep (python bench.py --sweep): one layer, every path that accepts T ------------
 
-# The library's path selection by T (include/moe.h, moe_forward): the single-token kernel once per
-# token up to DISPATCH_DECODE_MAX tokens, the tensor-core path from DISPATCH_TC_MIN tokens, the
-# CUDA-core path in between.  The flags below pin a context to one path.
-DISPATCH_DECODE_MAX = 8
-DISPATCH_TC_MIN = 9
-SWEEP_T = (1, 2, 4, 6, 8, 9, 10, 12, 16, 24, 32, 48, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
-SWEEP_PATHS = ("single-token kernel", "cuda-core", "tensor-core")
+# The library's path selection by T (include/moe.h, moe_forward): the single-token kernel for one
+# token, the few-token kernel for 2 to DISPATCH_FEW_MAX tokens, the tensor-core path above; the
+# CUDA-core path only where none fits.  The flags below pin a context to one path.
+DISPATCH_FEW_MAX = 16
+DISPATCH_SINGLE_MAX = 8      # the single-token kernel, once per token, when pinned to it
+DISPATCH_TC_MIN = 9          # the tensor-core path's floor when the decode kernels are off
+SWEEP_T = (1, 2, 4, 6, 8, 9, 10, 12, 16, 17, 24, 32, 48, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
+SWEEP_PATHS = ("single-token kernel", "few-token kernel", "cuda-core", "tensor-core")
 
 
 def sweep_flags(path: str) -> int:
-    no_decode, no_tensor = 1, 2   # MOE_FLAG_NO_DECODE_KERNEL, MOE_FLAG_NO_TENSOR_PREFILL
-    return {"single-token kernel": 0, "cuda-core": no_decode | no_tensor, "tensor-core": no_decode}[path]
+    # MOE_FLAG_NO_DECODE_KERNEL, MOE_FLAG_NO_TENSOR_PREFILL, MOE_FLAG_NO_MULTI_DECODE
+    no_decode, no_tensor, no_multi = 1, 2, 8
+    return {"single-token kernel": no_multi, "few-token kernel": 0, "cuda-core": no_decode | no_tensor,
+            "tensor-core": no_decode}[path]
 
 
 def sweep_eligible(path: str, T: int) -> bool:
     """Whether a context pinned to `path` runs T tokens on that path."""
     if path == "single-token kernel":
-        return T <= DISPATCH_DECODE_MAX
+        return T <= DISPATCH_SINGLE_MAX
+    if path == "few-token kernel":
+        return 2 <= T <= DISPATCH_FEW_MAX
     if path == "tensor-core":
         return T >= DISPATCH_TC_MIN
     return True
 
 
 def default_path(T: int) -> str:
-    if T <= DISPATCH_DECODE_MAX:
+    if T == 1:
         return "single-token kernel"
-    return "tensor-core" if T >= DISPATCH_TC_MIN else "cuda-core"
+    return "few-token kernel" if T <= DISPATCH_FEW_MAX else "tensor-core"
 
 
 def sweep_summary(rows: list[dict]) -> list[dict]:

@@ -247,6 +247,33 @@ __device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long *p) { 
     asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p) : "memory");
     return w;
 }
+// Reads N tagged words (addr(i) == nullptr: not read, counted as arrived) and re-reads the late
+// ones together, round after round, until every word carries `want`.  Bounded: false on timeout
+// (the error word is set) or once another CTA has reported an error.
+template <int N, typename Addr>
+__device__ __forceinline__ bool read_tagged(unsigned long long (&w)[N], Addr addr, unsigned want, int *err) {
+    static_assert(N <= 32, "late-word mask");
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const unsigned long long *a = addr(i);
+        w[i] = a ? ld_tagged(a) : ((unsigned long long)want << 32);
+    }
+    const long long t0 = clock64();
+    for (int it = 0;; ++it) {
+        unsigned late = 0u;
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if ((unsigned)(w[i] >> 32) != want) late |= 1u << i;
+        if (!late) return true;
+        if ((it & 15) == 15 && (*(volatile int *)err != 0 || clock64() - t0 > SPIN_LIMIT)) {
+            atomicCAS(err, 0, MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if ((late >> i) & 1u) w[i] = ld_tagged(addr(i));
+    }
+}
 __device__ __forceinline__ float ld_gpu(const float *p) {
     float v;
     asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");

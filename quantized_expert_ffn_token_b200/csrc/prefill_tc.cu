@@ -43,6 +43,7 @@ constexpr int TC_ALD_MAXJ = (TC_BM * 8 + TC_ALD_NT - 1) / TC_ALD_NT;   // 16-byt
 constexpr int TC_BN = 256;                 // output columns per work item
 constexpr int TC_BK = 64;                  // k per pipeline stage (one 128-byte swizzle row)
 constexpr int TC_STAGES = 3;
+constexpr int TC_PF = 3;                    // k groups ahead that a weight producer prefetches into L2
 constexpr int A_STAGE_BYTES = TC_BM * TC_BK * 2;   // 32 KB
 constexpr int B_STAGE_BYTES = TC_BN * TC_BK * 2;   // 32 KB
 // Producers' weight staging: 2 slots x 3 fields (codes of tile 0, codes of
@@ -89,6 +90,7 @@ struct TcParams {
 enum TcMode { TC_GATEUP = 0, TC_DOWN = 1, TC_ROUTER = 2 };
 
 __device__ __forceinline__ uint32_t su32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 __device__ __forceinline__ void mbar_init(uint64_t *b, int count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
@@ -525,6 +527,12 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                         const uint8_t *sc = tile + p.L.code_bytes;
                         cp_async4(raw + 2 * RAW_FIELD + 8 * tt, sc + (size_t)(g * nb + 2 * kb) * 2);
                         cp_async4(raw + 2 * RAW_FIELD + 4 + 8 * tt, sc + (size_t)((g + 8) * nb + 2 * kb) * 2);
+                        // the stage's loads above wait on one round trip each: bring the codes of
+                        // the k group TC_PF ahead (and, at the item's start, the tile's scales) into
+                        // L2 now, so those loads find them there
+                        if (kb + TC_PF < nk && lane * 128 < p.L.kg_bytes)
+                            prefetch_l2(tile + (size_t)(kb + TC_PF) * p.L.kg_bytes + lane * 128);
+                        if (kb == 0 && lane * 128 < 16 * nb * 2) prefetch_l2(sc + lane * 128);
                     }
                 }
                 cp_async_commit();   // one group per stage: its weight bytes

@@ -436,7 +436,7 @@ def test_memory_limit_gives_oom():
     with pytest.raises(capi.MoeError) as e:
         session.Session(TINY, max_tokens=16, mem_limit=4096)
     assert e.value.status == capi.MOE_ERR_OOM
-    sess = session.Session(TINY, max_tokens=16, mem_limit=400_000)   # workspace fits, weights not
+    sess = session.Session(TINY, max_tokens=16, mem_limit=700_000)   # workspace fits, weights not
     with pytest.raises(capi.MoeError) as e:
         sess.load_synthetic(layers=[0])
     assert e.value.status == capi.MOE_ERR_OOM
