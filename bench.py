@@ -78,19 +78,31 @@ def router_flops(cfg, T: int) -> int:
     return 2 * T * cfg.E * cfg.d
 
 
-# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, per unit
-# of work, each with the SHA-256 of the kernel source it was measured on: a figure is reported only
-# while that source is unchanged (a changed kernel reports null until it is measured again).  The
-# commands that produced them are in the profiles/ summaries named beside each entry.
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, per layer,
+# each with the SHA-256 of the kernel sources it was measured on: a figure is reported only while
+# those sources are unchanged (a changed kernel reports null until it is measured again).  The decode
+# figures come from 4-layer captures (the 48-layer launch is reported as 48 x the per-layer mean:
+# the traffic grows with the layers, each streaming its own union of experts); the commands that
+# produced them are in the profiles/ summaries named beside each entry.
 MEASURED_TRAFFIC = [
-    # {"kernel": ..., "workload": ..., "src": "<file>", "sha256": "...", "bytes_per_layer": ...,
-    #  "profile": "profiles/<name>.md"}
+    {"kernel": "k_decode", "workload": "decode_48l_q4_t1", "src": ['decode.cu', 'decode_common.cuh', 'moe_internal.cuh'],
+     "sha256": "252498f9e2694898778653d245bc97b4547bb0ad183dd3463c0b4b77a0e53fde", "bytes_per_layer": 30_701_760,
+     "profile": "profiles/k_decode_decode_48l_q4_t1.md"},
+    {"kernel": "k_decode_multi", "workload": "verify_48l_q3_t4_zipf", "src": ['decode_multi.cu', 'decode_common.cuh', 'moe_internal.cuh'],
+     "sha256": "ebb5d3e364df8ed15b500000e5a9b4074dc3809096f71fc43fad5b7752a8fa27", "bytes_per_layer": 42_456_704,
+     "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
+    {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "69ff2c3cb756458483a3eef96664a711463ed17608454b13dffac78b50429dcc", "bytes_per_layer": 1_155_117_824,
+     "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 
 
-def _src_sha(rel: str) -> str:
-    with open(os.path.join(ROOT, "quantized_expert_ffn_token_b200", "csrc", rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+def _src_sha(rels) -> str:
+    h = hashlib.sha256()
+    for rel in ([rels] if isinstance(rels, str) else rels):
+        with open(os.path.join(ROOT, "quantized_expert_ffn_token_b200", "csrc", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def measured_traffic(kernel: str, workload: str, layers: int):
