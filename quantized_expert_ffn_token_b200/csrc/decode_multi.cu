@@ -225,6 +225,23 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     LayerPtrs *ltab = reinterpret_cast<LayerPtrs *>(smem + p.off_ltab);
 
     constexpr bool F16OP = (FMT != MOE_Q3B32);
+    // Gate/up, and down for up to four tokens, remove the code offset inside the MMAs: a second MMA
+    // per k16 slice with A = minus the offset (rows g and g + 8 of each 32-block, exact in
+    // fp16/bf16) on the same B; the multipliers scale back the codes read as 1024 + F q.
+    uint32_t cg0, c80, cg1, c81;
+    float mg0, m80, mg1, m81;
+    if constexpr (FMT == MOE_Q4B32) {
+        cg0 = cg1 = 0xE408E408u; c80 = c81 = 0xE480E480u;   // -1032, -1152 (fp16)
+        mg0 = mg1 = 1.f; m80 = m81 = 0.0625f;
+    } else if constexpr (FMT == MOE_Q2B32) {
+        cg0 = 0xE402E402u; c80 = 0xE408E408u;               // -1026, -1032
+        cg1 = 0xE420E420u; c81 = 0xE480E480u;               // -1056, -1152
+        mg0 = 1.f; m80 = 0.25f; mg1 = 0.0625f; m81 = 0.015625f;
+    } else {
+        cg0 = c80 = cg1 = c81 = 0xC304C304u;                // -132 (bf16)
+        mg0 = m80 = mg1 = m81 = 1.f;
+    }
+    const uint32_t off0[4] = {cg0, c80, cg0, c80}, off1[4] = {cg1, c81, cg1, c81};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const int G = gridDim.x, cta = blockIdx.x;
     const int d = p.d, E = p.E, I = p.I, k = p.k, T = p.T, TM = p.TM;
@@ -816,23 +833,6 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 16 * c;
             const int t0 = 2 * c, t1 = 2 * c + 1;
             const bool l0 = t0 < T, l1 = t1 < T;
-            // the code offset is removed inside the MMAs: a second MMA per k16 slice with A = minus
-            // the offset (rows g and g + 8 of each 32-block, exact in fp16/bf16) on the same B; the
-            // multipliers scale back the codes read as 1024 + F q
-            uint32_t cg0, c80, cg1, c81;
-            float mg0, m80, mg1, m81;
-            if constexpr (FMT == MOE_Q4B32) {
-                cg0 = cg1 = 0xE408E408u; c80 = c81 = 0xE480E480u;   // -1032, -1152 (fp16)
-                mg0 = mg1 = 1.f; m80 = m81 = 0.0625f;
-            } else if constexpr (FMT == MOE_Q2B32) {
-                cg0 = 0xE402E402u; c80 = 0xE408E408u;               // -1026, -1032
-                cg1 = 0xE420E420u; c81 = 0xE480E480u;               // -1056, -1152
-                mg0 = 1.f; m80 = 0.25f; mg1 = 0.0625f; m81 = 0.015625f;
-            } else {
-                cg0 = c80 = cg1 = c81 = 0xC304C304u;                // -132 (bf16)
-                mg0 = m80 = mg1 = m81 = 1.f;
-            }
-            const uint32_t off0[4] = {cg0, c80, cg0, c80}, off1[4] = {cg1, c81, cg1, c81};
             const int nkg = d / 64;
             for (int ch = warp; ch < sp.n_gu * GU_CH && ok; ch += NW) {
                 const int q = ch / GU_CH, j = ch - q * GU_CH;
@@ -1070,41 +1070,86 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                 const __half *sc = reinterpret_cast<const __half *>(tile + p.dn.code_bytes);
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const int t0 = 2 * c, t1 = 2 * c + 1;
-                const float *hs0 = hsum + (su * TM + min(t0, TM - 1)) * nbi;
-                const float *hs1 = hsum + (su * TM + min(t1, TM - 1)) * nbi;
-                const float *hi0 = hinv + (su * TM + min(t0, TM - 1)) * nbi;
-                const float *hi1 = hinv + (su * TM + min(t1, TM - 1)) * nbi;
                 const bool l0 = t0 < T, l1 = t1 < T;
+                if (T <= 4) {
+                    // Up to four tokens: hi and lo of h share one MMA, column g < 4 holding the hi part
+                    // of token g and column g >= 4 the lo part of token g - 4, and the code offset is
+                    // removed by a second MMA with the constant A (as in gate/up); the two parts of a
+                    // token meet at the end (lanes c and c ^ 2).
+                    const int srcl = lane & 15;                  // h table lane of this column's token
+                    const int poff = 8 * (g >> 2);               // bytes: hi (words 0-1) or lo (2-3)
+                    const bool colv = (g & 3) < T;
+                    const int tc0 = (2 * c) & 3, tc1 = (2 * c + 1) & 3;   // tokens of this lane's columns
+                    const float *ih0 = hinv + (su * TM + min(tc0, TM - 1)) * nbi;
+                    const float *ih1 = hinv + (su * TM + min(tc1, TM - 1)) * nbi;
 #pragma unroll 2
-                for (int kg = 0; kg < nkgi; ++kg) {
-                    uint32_t a[16];
-                    frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
-                    float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int kg = 0; kg < nkgi; ++kg) {
+                        uint32_t a[16];
+                        frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
+                        float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const uint4 bq = g < T ? *reinterpret_cast<const uint4 *>(htab + hfrag_off(su, nkgi, kg, m, lane))
-                                               : make_uint4(0u, 0u, 0u, 0u);
-                        float *D = (m < 2) ? Da : Db;
-                        mma_fmt<FMT>(D, a + 4 * m, bq.x, bq.y);   // hi
-                        mma_fmt<FMT>(D, a + 4 * m, bq.z, bq.w);   // lo
+                        for (int m = 0; m < 4; ++m) {
+                            const uint2 bq = colv ? *reinterpret_cast<const uint2 *>(htab + hfrag_off(su, nkgi, kg, m, srcl) + poff)
+                                                  : make_uint2(0u, 0u);
+                            float *D = (m < 2) ? Da : Db;
+                            mma_fmt<FMT>(D, a + 4 * m, bq.x, bq.y);
+                            mma_fmt<FMT>(D, m < 2 ? off0 : off1, bq.x, bq.y);
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int b = 2 * kg + h;
+                            float sg = __half2float(sc[g * nbi + b]) * (h ? mg1 : mg0);
+                            float s8 = __half2float(sc[(g + 8) * nbi + b]) * (h ? m81 : m80);
+                            float sg0 = sg, sg1 = sg, s80 = s8, s81 = s8;
+                            if constexpr (F16OP) {   // h entered as h * 2^s per (token, block)
+                                const float i0 = ih0[b], i1 = ih1[b];
+                                sg0 *= i0; s80 *= i0; sg1 *= i1; s81 *= i1;
+                            }
+                            const float *D = h ? Db : Da;
+                            acc[0] = fmaf(sg0, D[0], acc[0]);
+                            acc[1] = fmaf(sg1, D[1], acc[1]);
+                            acc[2] = fmaf(s80, D[2], acc[2]);
+                            acc[3] = fmaf(s81, D[3], acc[3]);
+                        }
                     }
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int b = 2 * kg + h;
-                        const float v0 = l0 ? hs0[b] : 0.f, v1 = l1 ? hs1[b] : 0.f;
-                        float sg = __half2float(sc[g * nbi + b]), s8 = __half2float(sc[(g + 8) * nbi + b]);
-                        float Dv[4] = {h ? Db[0] : Da[0], h ? Db[1] : Da[1], h ? Db[2] : Da[2], h ? Db[3] : Da[3]};
-                        if constexpr (F16OP) {
-                            // h entered as h * 2^s per (token, block): scale back per column
-                            const float i0 = l0 ? hi0[b] : 0.f, i1 = l1 ? hi1[b] : 0.f;
-                            float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-                            flush_block<FMT>(tmp, Dv, sg, s8, v0, v1, h == 1);
-                            acc[0] = fmaf(tmp[0], i0, acc[0]);
-                            acc[1] = fmaf(tmp[1], i1, acc[1]);
-                            acc[2] = fmaf(tmp[2], i0, acc[2]);
-                            acc[3] = fmaf(tmp[3], i1, acc[3]);
-                        } else {
-                            flush_block<FMT>(acc, Dv, sg, s8, v0, v1, h == 1);
+                    for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 2);
+                } else {
+                    const float *hs0 = hsum + (su * TM + min(t0, TM - 1)) * nbi;
+                    const float *hs1 = hsum + (su * TM + min(t1, TM - 1)) * nbi;
+                    const float *hi0 = hinv + (su * TM + min(t0, TM - 1)) * nbi;
+                    const float *hi1 = hinv + (su * TM + min(t1, TM - 1)) * nbi;
+    #pragma unroll 2
+                    for (int kg = 0; kg < nkgi; ++kg) {
+                        uint32_t a[16];
+                        frag16<FMT>(tile + (size_t)kg * p.dn.kg_bytes + lane * piece_bytes<FMT>(), a);
+                        float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const uint4 bq = g < T ? *reinterpret_cast<const uint4 *>(htab + hfrag_off(su, nkgi, kg, m, lane))
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+                            float *D = (m < 2) ? Da : Db;
+                            mma_fmt<FMT>(D, a + 4 * m, bq.x, bq.y);   // hi
+                            mma_fmt<FMT>(D, a + 4 * m, bq.z, bq.w);   // lo
+                        }
+    #pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int b = 2 * kg + h;
+                            const float v0 = l0 ? hs0[b] : 0.f, v1 = l1 ? hs1[b] : 0.f;
+                            float sg = __half2float(sc[g * nbi + b]), s8 = __half2float(sc[(g + 8) * nbi + b]);
+                            float Dv[4] = {h ? Db[0] : Da[0], h ? Db[1] : Da[1], h ? Db[2] : Da[2], h ? Db[3] : Da[3]};
+                            if constexpr (F16OP) {
+                                // h entered as h * 2^s per (token, block): scale back per column
+                                const float i0 = l0 ? hi0[b] : 0.f, i1 = l1 ? hi1[b] : 0.f;
+                                float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+                                flush_block<FMT>(tmp, Dv, sg, s8, v0, v1, h == 1);
+                                acc[0] = fmaf(tmp[0], i0, acc[0]);
+                                acc[1] = fmaf(tmp[1], i1, acc[1]);
+                                acc[2] = fmaf(tmp[2], i0, acc[2]);
+                                acc[3] = fmaf(tmp[3], i1, acc[3]);
+                            } else {
+                                flush_block<FMT>(acc, Dv, sg, s8, v0, v1, h == 1);
+                            }
                         }
                     }
                 }
