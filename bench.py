@@ -49,6 +49,9 @@ SECONDARY = ("verify_48l_q3_t4_zipf", "prefill_1l_q4_t4096_zipf", "prefill_48l_q
 FLUSH_BYTES = 256 << 20   # L2 flush between timed steps of workloads whose step streams less than ~1 GB
 
 
+L2_MODES = {"stream": 0, "keep": 1}   # MOE_L2_STREAM, MOE_L2_KEEP_SHARED
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -86,13 +89,13 @@ def router_flops(cfg, T: int) -> int:
 # produced them are in the profiles/ summaries named beside each entry.
 MEASURED_TRAFFIC = [
     {"kernel": "k_decode", "workload": "decode_48l_q4_t1", "src": ['decode.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "252498f9e2694898778653d245bc97b4547bb0ad183dd3463c0b4b77a0e53fde", "bytes_per_layer": 30_701_760,
+     "sha256": "bb83d8c4e6a9d1b31810d1a0ca4a6f065f5dce639259f11d18b212b6d4010aa1", "bytes_per_layer": 30_823_552,
      "profile": "profiles/k_decode_decode_48l_q4_t1.md"},
     {"kernel": "k_decode_multi", "workload": "verify_48l_q3_t4_zipf", "src": ['decode_multi.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "ebb5d3e364df8ed15b500000e5a9b4074dc3809096f71fc43fad5b7752a8fa27", "bytes_per_layer": 42_456_704,
+     "sha256": "b798a3d37b4443ab5bd7fe23f4c48ff67f0db01bc83e0710b1700aa62e769e02", "bytes_per_layer": 42_910_912,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "69ff2c3cb756458483a3eef96664a711463ed17608454b13dffac78b50429dcc", "bytes_per_layer": 1_155_117_824,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "a2c7311348aae65d7ec8831378c772ac392ad886710c34149419ff6a97afe889", "bytes_per_layer": 1_155_117_824,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 
@@ -330,6 +333,7 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
     stream = torch.cuda.Stream(dev)
     P = peaks()
     sess = session.Session(cfg, device=local_rank, max_tokens=cfg.T)
+    capi.moe_set_l2_policy(sess.ctx, L2_MODES[args.l2_policy])
     with torch.cuda.stream(stream):
         sess.load_synthetic(stream=stream)
     torch.cuda.synchronize()
@@ -384,17 +388,22 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
                      "frac": step_bytes / (ms_step / 1e3) / 1e9 / P["hbm_gbs"]}
     l2_ab = None
     if not tensor_bound:
-        # L2 residency: the same steps with every weight copy at the default eviction priority, against
-        # the default mode that keeps the shared experts (every layer's) in L2 across steps
-        capi.moe_set_l2_policy(sess.ctx, capi.MOE_L2_STREAM)
-        ms_stream, _ = timed_steps(capi, sess, cfg, xs, out, args.steps, args.warmup, stream, dist_on, flush)
-        capi.moe_set_l2_policy(sess.ctx, capi.MOE_L2_KEEP_SHARED)
-        ms_stream = max_over_ranks(ms_stream, dist_on, dev) / args.steps
+        # L2 residency: the same steps once more in the other L2 mode (keep the shared experts of every
+        # layer in L2 across steps: evict_last for them, evict_first for the rest; or plain copies)
+        other = capi.MOE_L2_KEEP_SHARED if L2_MODES[args.l2_policy] == capi.MOE_L2_STREAM else capi.MOE_L2_STREAM
+        capi.moe_set_l2_policy(sess.ctx, other)
+        ms_other, _ = timed_steps(capi, sess, cfg, xs, out, args.steps, args.warmup, stream, dist_on, flush)
+        capi.moe_set_l2_policy(sess.ctx, L2_MODES[args.l2_policy])
+        ms_other = max_over_ranks(ms_other, dist_on, dev) / args.steps
         kept = cfg.L * cfg.n_shared * expert_bytes(cfg)
-        l2_ab = {"mode": "shared experts evict_last, routed experts and router rows evict_first",
+        v_other = whole_job_rate(cfg.T, world, ms_other / 1e3)
+        keep_first = other == capi.MOE_L2_STREAM
+        l2_ab = {"mode_of_value": args.l2_policy,
+                 "keep_shared": "shared experts copied evict_last, routed experts and router rows evict_first",
                  "kept_bytes": kept, "kept_fraction_of_step_bytes": kept / step_bytes,
-                 "value_keep_shared": value, "value_stream": whole_job_rate(cfg.T, world, ms_stream / 1e3),
-                 "speedup": ms_stream / ms_step}
+                 "value_keep_shared": value if keep_first else v_other,
+                 "value_stream": v_other if keep_first else value,
+                 "keep_shared_speedup": (ms_other / ms_step) if keep_first else (ms_step / ms_other)}
 
     # end to end through the public host-buffer entry point (copies inside the timed region)
     x_host = [torch.from_numpy(synth.tokens_bf16(cfg, cfg.T, stream=rank * 100003 + s).view(np.int16)).pin_memory()
@@ -544,6 +553,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--no-secondary", action="store_true", help="time the headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="leave out the oracle's CPU baselines")
+    ap.add_argument("--l2-policy", default="stream", choices=sorted(L2_MODES),
+                    help="L2 mode of the decode kernels' weight copies for the timed steps (the other mode is "
+                         "timed too, for the l2_residency entry)")
     ap.add_argument("--layers", type=int, default=None,
                     help="stack depth override (small cases for profiler captures)")
     ap.add_argument("--sweep", action="store_true",

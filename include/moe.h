@@ -226,13 +226,15 @@ MOE_API int moe_get_device_error(moe_ctx *ctx, int *code);
  * faster memory ("Qwen3.8-Flash-Next on RTX 5090 + 64GB", section 2 "Expert
  * Cache and CPU/GPU Split").  Here every expert already lives in HBM; the
  * shared experts are read by every token of every call, so in mode
- * MOE_L2_KEEP_SHARED (the default) their tiles are copied with the L2
- * eviction priority evict_last and the routed experts' tiles and the router
- * rows with evict_first, which keeps the shared experts of all layers in the
- * 126 MB L2 across calls when they fit; MOE_L2_STREAM copies everything with
- * the default priority.  Applies to the single-token and few-token kernels;
- * results do not depend on it.  Errors: INVALID_ARG (NULL context, unknown
- * mode). */
+ * MOE_L2_KEEP_SHARED their tiles are copied with the L2 eviction priority
+ * evict_last and the routed experts' tiles and the router rows with
+ * evict_first, which keeps the shared experts of all layers in the 126 MB L2
+ * across calls when they fit; MOE_L2_STREAM (the default) copies everything
+ * with the default priority.  The decode kernels are bound by the latency of
+ * each layer's chain of steps, not by bandwidth, and keeping 83-106 MB of
+ * shared experts measured no faster (one token, Q4: 1.2 % slower), hence the
+ * default.  Applies to the single-token and few-token kernels; results do not
+ * depend on it.  Errors: INVALID_ARG (NULL context, unknown mode). */
 #define MOE_L2_STREAM 0
 #define MOE_L2_KEEP_SHARED 1
 MOE_API int moe_set_l2_policy(moe_ctx *ctx, int mode);

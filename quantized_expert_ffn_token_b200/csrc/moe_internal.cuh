@@ -286,7 +286,7 @@ struct moe_ctx {
     qeffn::ChunkLayout chunk;
     qeffn::SplitState sdec;
     bool tc_withheld = false;   // the MOE_FLAG_TEST_WITHHOLD gate/up GEMM has run
-    int l2_mode = MOE_L2_KEEP_SHARED;   // L2 eviction priorities of the decode kernels' weight copies
+    int l2_mode = MOE_L2_STREAM;   // L2 eviction priorities of the decode kernels' weight copies
 };
 
 namespace qeffn {
