@@ -109,7 +109,7 @@ struct MultiParams {
     int l2_mode;                   // 0: plain copies; 1: shared experts kept in L2, the rest streamed
     unsigned long long *trace;     // [G][L][24] phase clocks, or NULL
     int nslot, slot_bytes, rpc, span, UM;
-    int off_ring, off_router, off_xb, off_hsum, off_uexp, off_wtab,
+    int off_ring, off_router, off_xb, off_xoff, off_hsum, off_uexp, off_wtab,
         off_misc, off_ltab;
 };
 
@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
     uint16_t *xb = reinterpret_cast<uint16_t *>(smem + p.off_xb);     // [TM][d] bf16 input; then the h table
     uint8_t *htab = smem + p.off_xb;
     float *hsum = reinterpret_cast<float *>(smem + p.off_hsum);       // [span][TM][I/32], then hinv
+    float *xoff = reinterpret_cast<float *>(smem + p.off_xoff);       // [d/32][2][TM]: gate/up MMA start values
     int *uexp = reinterpret_cast<int *>(smem + p.off_uexp);           // [UM]
     float *wtab = reinterpret_cast<float *>(smem + p.off_wtab);       // [UM][TM]
     MiscM *ms = reinterpret_cast<MiscM *>(smem + p.off_misc);
@@ -242,6 +243,11 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
         mg0 = m80 = mg1 = m81 = 1.f;
     }
     const uint32_t off0[4] = {cg0, c80, cg0, c80}, off1[4] = {cg1, c81, cg1, c81};
+    // the same offsets as numbers (gate/up starts its MMAs from -offset x block sum)
+    constexpr float OFF_G0 = FMT == MOE_Q4B32 ? 1032.f : FMT == MOE_Q2B32 ? 1026.f : 132.f;
+    constexpr float OFF_80 = FMT == MOE_Q4B32 ? 1152.f : FMT == MOE_Q2B32 ? 1032.f : 132.f;
+    constexpr float OFF_G1 = FMT == MOE_Q4B32 ? 1032.f : FMT == MOE_Q2B32 ? 1056.f : 132.f;
+    constexpr float OFF_81 = FMT == MOE_Q4B32 ? 1152.f : FMT == MOE_Q2B32 ? 1152.f : 132.f;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const int G = gridDim.x, cta = blockIdx.x;
     const int d = p.d, E = p.E, I = p.I, k = p.k, T = p.T, TM = p.TM;
@@ -585,6 +591,31 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     w[j] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
             }
+            // the offset terms of the k group's two 32-blocks: -(offset) x (block sum of the operand as
+            // the MMA sees it), for the rows g and g + 8 of the A fragments; the gate/up MMAs of every
+            // tile start from them (k16 slices 0-1: block 2 kg, slices 2-3: block 2 kg + 1)
+            {
+                float bs[2] = {0.f, 0.f};
+#pragma unroll
+                for (int wo = 0; wo < 32; ++wo) {
+                    float v0, v1;
+                    if constexpr (F16OP) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[wo]));
+                        v0 = f.x;
+                        v1 = f.y;
+                    } else {
+                        v0 = bf16f(w[wo] & 0xFFFFu);
+                        v1 = bf16f(w[wo] >> 16);
+                    }
+                    bs[wo >> 4] += v0 + v1;   // words 0-15: slices 0-1 (block 2 kg)
+                }
+                const float og[2] = {OFF_G0, OFF_G1}, o8[2] = {OFF_80, OFF_81};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    xoff[((2 * kg + h) * 2 + 0) * TM + t] = -og[h] * bs[h];
+                    xoff[((2 * kg + h) * 2 + 1) * TM + t] = -o8[h] * bs[h];
+                }
+            }
             // word 8m + 4h + c (slice m, B register h, lane column c) goes to 8c + 2m + h
             uint32_t o[32];
 #pragma unroll
@@ -833,6 +864,7 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
             const uint16_t *xr = xb + (size_t)(live ? g : 0) * XS + 16 * c;
             const int t0 = 2 * c, t1 = 2 * c + 1;
             const bool l0 = t0 < T, l1 = t1 < T;
+            const int cx = 2 * c < TM ? 2 * c : 0;   // start values of columns 2c, 2c + 1 (past TM: dead)
             const int nkg = d / 64;
             for (int ch = warp; ch < sp.n_gu * GU_CH && ok; ch += NW) {
                 const int q = ch / GU_CH, j = ch - q * GU_CH;
@@ -854,16 +886,17 @@ __global__ void __launch_bounds__(NTT, 1) k_decode_multi(MultiParams p) {
                     frag16<FMT>(tile + (size_t)kg * p.gu.kg_bytes + lane * piece_bytes<FMT>(), a);
                     const uint4 q0 = live ? *reinterpret_cast<const uint4 *>(xr + 64 * kg) : make_uint4(0u, 0u, 0u, 0u);
                     const uint4 q1 = live ? *reinterpret_cast<const uint4 *>(xr + 64 * kg + 8) : make_uint4(0u, 0u, 0u, 0u);
-                    float Da[4] = {0.f, 0.f, 0.f, 0.f}, Db[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_fmt<FMT>(Da, a + 0, q0.x, q0.y);
-                    mma_fmt<FMT>(Da, off0, q0.x, q0.y);
-                    mma_fmt<FMT>(Da, a + 4, q0.z, q0.w);
-                    mma_fmt<FMT>(Da, off0, q0.z, q0.w);
-                    mma_fmt<FMT>(Db, a + 8, q1.x, q1.y);
-                    mma_fmt<FMT>(Db, off1, q1.x, q1.y);
-                    mma_fmt<FMT>(Db, a + 12, q1.z, q1.w);
-                    mma_fmt<FMT>(Db, off1, q1.z, q1.w);
                     const int bl = 2 * kg;
+                    // the MMAs start from the blocks' offset terms (columns 2c, 2c + 1; rows g, g + 8)
+                    const float2 oga = *reinterpret_cast<const float2 *>(xoff + (bl * 2 + 0) * TM + cx);
+                    const float2 o8a = *reinterpret_cast<const float2 *>(xoff + (bl * 2 + 1) * TM + cx);
+                    const float2 ogb = *reinterpret_cast<const float2 *>(xoff + (bl * 2 + 2) * TM + cx);
+                    const float2 o8b = *reinterpret_cast<const float2 *>(xoff + (bl * 2 + 3) * TM + cx);
+                    float Da[4] = {oga.x, oga.y, o8a.x, o8a.y}, Db[4] = {ogb.x, ogb.y, o8b.x, o8b.y};
+                    mma_fmt<FMT>(Da, a + 0, q0.x, q0.y);
+                    mma_fmt<FMT>(Da, a + 4, q0.z, q0.w);
+                    mma_fmt<FMT>(Db, a + 8, q1.x, q1.y);
+                    mma_fmt<FMT>(Db, a + 12, q1.z, q1.w);
                     const float2 sg = __half22float2(*reinterpret_cast<const __half2 *>(sc + g * nbd + bl));
                     const float2 s8 = __half22float2(*reinterpret_cast<const __half2 *>(sc + (g + 8) * nbd + bl));
                     const float sga = sg.x * mg0, s8a = s8.x * m80, sgb = sg.y * mg1, s8b = s8.y * m81;
@@ -1298,6 +1331,7 @@ int decode_multi_setup(moe_ctx *ctx) {
     const size_t htab_bytes = (size_t)span * (c.d_ff / 64) * 4 * 32 * 16;
     ms.off_router = take((size_t)rpc * c.d_model * 4);
     ms.off_xb = take(xb_bytes > htab_bytes ? xb_bytes : htab_bytes);
+    ms.off_xoff = take((size_t)(c.d_model / 32) * 2 * TM * 4);
     ms.off_hsum = take((size_t)2 * span * TM * (c.d_ff / 32) * 4);
     ms.off_uexp = take((size_t)UM * 4);
     ms.off_wtab = take((size_t)UM * TM * 4);
@@ -1389,6 +1423,7 @@ int launch_decode_multi(moe_ctx *ctx, int layer0, int L, const uint16_t *x, int 
     p.off_ring = ms.off_ring;
     p.off_router = ms.off_router;
     p.off_xb = ms.off_xb;
+    p.off_xoff = ms.off_xoff;
     p.off_hsum = ms.off_hsum;
     p.off_uexp = ms.off_uexp;
     p.off_wtab = ms.off_wtab;

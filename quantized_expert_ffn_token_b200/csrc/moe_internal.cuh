@@ -239,7 +239,7 @@ struct MultiState {
     int tm = 0;           // tokens per launch the carve holds (<= 8)
     int um = 0;           // union slots: tm * top_k + n_shared
     int nslot = 0, slot_bytes = 0, rpc = 0, span = 0;
-    int off_ring = 0, off_router = 0, off_xb = 0, off_hsum = 0, off_uexp = 0,
+    int off_ring = 0, off_router = 0, off_xb = 0, off_xoff = 0, off_hsum = 0, off_uexp = 0,
         off_wtab = 0, off_misc = 0, off_ltab = 0;
     uint8_t *xbuf = nullptr;   // counters, logits, h, output and residual buffers
     unsigned tag = 1;          // tag of the next launch's first layer in the tagged logits area
