@@ -56,7 +56,7 @@ constexpr int CANDM = 64;       // top-k candidates per token held for ranking
 constexpr int MAX_SPAN = 4;     // experts one CTA's down run may touch (checked at set-up)
 constexpr int IN_IT = 2;        // float4 columns of a token row per thread in the input phase (d <= 3072)
 constexpr int HB_M = 4;         // float4 loads of h in flight per thread
-constexpr int GU_CH = 4;        // chunks (k-group ranges) per gate/up unit
+constexpr int GU_CH = 2;        // chunks (k-group ranges) per gate/up unit (of 1, 2, 3, 4 and 8, 2 measured fastest)
 
 struct MiscM {
     unsigned long long full[MAX_SLOTS];

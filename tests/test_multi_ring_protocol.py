@@ -4,7 +4,7 @@ One CTA, one layer, random interleavings of the producer (fills items in
 order, refilling a slot once its previous item is consumed) and the compute
 warps:
 
-* gate/up items: one unit each, cut into four k-group chunks; the CTA's
+* gate/up items: one unit each, cut into k-group chunks (two in the kernel); the CTA's
   chunks go round-robin to all warps, and the last chunk of a unit to finish
   frees its slot;
 * down items: batches of units; units go round-robin to all warps, the warp
@@ -47,7 +47,7 @@ class Stale(AssertionError):
     pass
 
 
-def gu_parts(n_gu, nkg, NW, nch=4):
+def gu_parts(n_gu, nkg, NW, nch=2):
     """Per warp, its (unit, chunks of that unit) list in processing order: unit q is cut into nch
     k-group chunks and the CTA's chunk c goes to warp c % NW."""
     plan = [[] for _ in range(NW)]
@@ -57,7 +57,7 @@ def gu_parts(n_gu, nkg, NW, nch=4):
 
 
 def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_last=True, nkg=40,
-        gu_free_on_last=True):
+        gu_free_on_last=True, nch=2):
     rnd = random.Random(seed)
     full = [MBar(1) for _ in range(nslot)]
     empty = [MBar(1) for _ in range(nslot)]
@@ -71,7 +71,7 @@ def run(nslot, n_gu, n_dn, dps, NW=12, seed=0, gate_on_earlier=True, free_on_las
     def slot(a):
         return a % nslot, (a // nslot) & 1, a // nslot
 
-    plan = gu_parts(n_gu, nkg, NW)
+    plan = gu_parts(n_gu, nkg, NW, nch)
     pcnt = {}
     warps = [{"ph": "gu", "j": 0, "u": w, "busy": None} for w in range(NW)]
     for _ in range(400000):
@@ -177,21 +177,22 @@ CASES = [(5, 32, 81, 5), (5, 33, 81, 5), (7, 8, 20, 5), (5, 8, 4, 5), (8, 21, 52
 
 @pytest.mark.parametrize("n_gu", [1, 2, 5, 7, 8, 11, 12, 13, 24, 35])
 def test_gate_up_chunks_cover_every_step_once(n_gu):
-    """The kernel's chunk bounds kb = j nkg / 4, ke = (j + 1) nkg / 4 tile every unit's k groups."""
-    for nkg in (4, 5, 40, 48):
-        for q in range(n_gu):
+    """The kernel's chunk bounds kb = j nkg / GU_CH, ke = (j + 1) nkg / GU_CH tile every unit's k groups."""
+    for nch in (2, 4):
+        for nkg in (4, 5, 40, 48):
             steps = []
-            for j in range(4):
-                steps += list(range(j * nkg // 4, (j + 1) * nkg // 4))
+            for j in range(nch):
+                steps += list(range(j * nkg // nch, (j + 1) * nkg // nch))
             assert steps == list(range(nkg))
-    plan = gu_parts(n_gu, 40, 12)
-    assert sorted(q for w in plan for q, _ in w) == sorted(q for q in range(n_gu) for _ in range(4))
+        plan = gu_parts(n_gu, 40, 12, nch)
+        assert sorted(q for w in plan for q, _ in w) == sorted(q for q in range(n_gu) for _ in range(nch))
 
 
 @pytest.mark.parametrize("case", CASES)
-def test_ring_protocol_completes_and_reads_the_right_fill(case):
+@pytest.mark.parametrize("nch", [2, 4])
+def test_ring_protocol_completes_and_reads_the_right_fill(case, nch):
     for seed in range(25):
-        assert run(*case, seed=seed)
+        assert run(*case, seed=seed, nch=nch)
 
 
 def test_planted_no_wait_on_earlier_items_is_caught():
