@@ -174,7 +174,8 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA.
  * Implementation (not part of the contract): one token runs the persistent
  * single-token kernel, 2 to 16 tokens the persistent few-token kernel (one
- * launch per 8 tokens, reading the union of their experts once per layer),
+ * launch per 8 tokens, reading the union of their experts once per layer;
+ * shapes with n_experts <= 512, d_ff a multiple of 128 and d_model <= 3072),
  * 17 and more the tensor-core grouped GEMMs; the CUDA-core grouped path runs
  * where none fits the shape (or under the MOE_FLAG_NO_* flags); each path
  * meets the same accuracy bound. */
