@@ -496,8 +496,10 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
             }
             for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                 int s = it % TC_STAGES;
-                ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
-                if (!ok) break;
+                if constexpr (MODE == TC_ROUTER) {   // the loads below go straight into the B stage
+                    ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
+                    if (!ok) break;
+                }
                 uint8_t *b_dst = sB + s * B_STAGE_BYTES;
                 const int kx = MODE == TC_ROUTER ? kb % nkd : kb;   // k block of the activations
                 if constexpr (MODE == TC_ROUTER) {
@@ -545,6 +547,12 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                     mbar_arrive(&ss->full[pending]);
                 }
                 pending = s;
+                if constexpr (MODE != TC_ROUTER) {
+                    // the B stage this k group decodes into (next iteration) must be free; its raw
+                    // bytes were requested above without waiting for it, so the load latency overlaps
+                    // the wait for the MMA warp to release the stage
+                    ok = mbar_wait_b(&ss->empty[s], (uint32_t)(((it / TC_STAGES) & 1) ^ 1), p.err);
+                }
             }
             if (!ok) break;
             // flush: the last stage of the item

@@ -2,9 +2,13 @@
 
 Agents, as in the kernel:
   * B producers and A loaders each fill the stage ring (S stages) for every
-    k block of every item.  Before writing a stage they wait on its "empty"
-    barrier, and they publish a stage on its "full" barrier one k block late.
-    They flush the last stage at the end of each item.  For an item of a
+    k block of every item.  A loaders wait on a stage's "empty" barrier, then
+    write it; B producers request a k block's raw codes first (into their own
+    buffers, not the stage), then decode the previous k block into its stage
+    and publish it, and only then wait on "empty" for the stage of the k block
+    just requested (the stage it decodes into next).  Both publish a stage on
+    its "full" barrier one k block late and flush the last stage at the end of
+    each item.  For an item of a
     cached expert the B producers instead issue one bulk copy of the stage
     image, completing on the stage's "cbar" barrier, and arrive on "full" at
     once; the MMA issuer waits on both.
@@ -58,12 +62,21 @@ def run(items, nk, S, rng, mistake=None, cached=None):
                 continue
             for kb in range(nk):
                 s = it % S
-                yield ("wait", ("empty", s), ((it // S) & 1) ^ (0 if mistake == "producer_parity" else 1))
-                yield ("write", part, s, (i, kb))
-                if pending is not None:
-                    yield ("publish", part, pending)
+                par = ((it // S) & 1) ^ (0 if mistake == "producer_parity" else 1)
+                if part == "A":
+                    yield ("wait", ("empty", s), par)
+                    yield ("write", part, s, (i, kb))
+                    if pending is not None:
+                        yield ("publish", part, pending)
+                else:
+                    if pending is not None:   # decode the previous k block into its stage
+                        yield ("write", part, pending[0], pending[1])
+                        yield ("publish", part, pending)
+                    yield ("wait", ("empty", s), par)
                 pending = (s, (i, kb))
                 it += 1
+            if part == "B":
+                yield ("write", part, pending[0], pending[1])
             yield ("publish", part, pending)
             pending = None
 
