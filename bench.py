@@ -89,13 +89,13 @@ def router_flops(cfg, T: int) -> int:
 # produced them are in the profiles/ summaries named beside each entry.
 MEASURED_TRAFFIC = [
     {"kernel": "k_decode", "workload": "decode_48l_q4_t1", "src": ['decode.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "f93c9231e7c080080169413f5cc11e422c3d22454f7414563a7fedc1ae24f689", "bytes_per_layer": 30_823_552,
+     "sha256": "3244bb73841d42dc054ba8d39528026745358a73eb5c732be3bd87928ae198d7", "bytes_per_layer": 30_823_552,
      "profile": "profiles/k_decode_decode_48l_q4_t1.md"},
     {"kernel": "k_decode_multi", "workload": "verify_48l_q3_t4_zipf", "src": ['decode_multi.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "239990e64a9c150e69be6f20c0802811e01338ecd2b578a7dfa28a93e0f143f3", "bytes_per_layer": 42_253_376,
+     "sha256": "dc47924e40b899b93f15d88b224461a32a4ec7bccfaf09d8569cdf2b79c2f610", "bytes_per_layer": 42_253_376,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "e8bdad9e6c93ef488136794241c9793537a88a38fbf5773fab928d5c7b4e77e5", "bytes_per_layer": 1_155_117_824,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "f2866d32da870bda33e4d80a57dcea971865c816735740e7a88101eea77d9bac", "bytes_per_layer": 896_799_488,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 

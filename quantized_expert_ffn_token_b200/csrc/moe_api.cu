@@ -134,8 +134,9 @@ int alloc_workspace(moe_ctx *ctx) {
     QE_TRY(ctx_alloc(ctx, (void **)&ws.cache_slot, (size_t)ctx->nx * 4, "cache_slot"));
     QE_TRY(ctx_alloc(ctx, (void **)&ws.cache_n, 4, "cache_n"));
     {
-        // decoded-weight cache: at most one slot per 256 grouped rows beyond the first block of
-        // an expert; optional: left out when it does not fit the memory limit or the device
+        // decoded-weight cache: at most one slot per 256 grouped rows (a bound: only experts of
+        // more than three 256-row blocks take one); optional: left out when it does not fit the
+        // memory limit or the device
         size_t per = (size_t)6 * c.d_model * c.d_ff;   // bytes of one expert's fp16 B stages
         size_t cap = (size_t)c.max_tokens * (c.top_k + c.n_shared) / 256;
         if (cap > (size_t)ctx->nx) cap = ctx->nx;

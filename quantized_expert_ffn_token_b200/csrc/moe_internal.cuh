@@ -198,7 +198,7 @@ struct Workspace {
     int4 *tc_items = nullptr;    // work items of one grouped GEMM
     int32_t *tc_n_items = nullptr;
     size_t tc_items_max = 0;
-    // decoded-weight cache of the tensor-core path: experts with more than one 256-row block
+    // decoded-weight cache of the tensor-core path: experts with more than three 256-row blocks
     // get their fp16 B stages decoded once per forward (empty when it did not fit memory)
     uint16_t *wcache = nullptr;  // [cache_cap][3 d I] fp16, swizzled 256x64 stage images
     int32_t *cache_slot = nullptr;   // [experts] slot or -1

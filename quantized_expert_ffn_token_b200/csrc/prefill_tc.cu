@@ -51,6 +51,15 @@ constexpr int B_STAGE_BYTES = TC_BN * TC_BK * 2;   // 32 KB
 // so that a warp's accesses to one field are contiguous (no bank conflicts).
 constexpr int RAW_FIELD = TC_PROD_NW * 32 * 16;
 constexpr int RAW_BYTES = 2 * 3 * RAW_FIELD;
+constexpr int STG_WARP_FLOATS = 32 * 16;            // epilogue staging per warp: 32 rows x 16 fp32
+constexpr int STG_BYTES = 4 * STG_WARP_FLOATS * 4;  // four epilogue warps: 8 KB
+// Experts with at least this many rows in a call have their fp16 stage images decoded once
+// (k_cache_fill) and copied by every 256-row block; smaller ones are decoded by the GEMM's
+// producers per block.  An image costs 6 d I bytes written and read back against the few
+// bits per weight of codes that a block reads otherwise: measured on B200, with three
+// blocks per expert (uniform routing at 32,768 tokens) decoding in the GEMM was 10 %
+// faster, while Zipf-skewed experts of thousands of rows gain from the cache.
+constexpr int TC_CACHE_MIN_ROWS = 3 * 256 + 1;
 constexpr long long TC_SPIN = 4000000000LL;        // clock64 cycles, about two seconds
 
 struct TcParams {
@@ -78,7 +87,7 @@ struct TcParams {
     const float *rbias;         // [E]
     float *logits;              // [T][E]
     int n_items_direct;         // router: items computed from the index (no item list)
-    // decoded-weight cache: stage images of experts with more than one 256-row block
+    // decoded-weight cache: stage images of experts with more than three 256-row blocks
     const uint16_t *wcache;     // [slot][gate/up stages, down stages][256 x 64 fp16, swizzled]
     const int32_t *cache_slot;  // [expert] slot or -1 (NULL: no cache)
     size_t cache_off;           // fp16 offset of this GEMM's stages within a slot
@@ -370,7 +379,8 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
     uint8_t *sA = smem;                                  // [stage][256 rows][128 B]
     uint8_t *sB = smem + TC_STAGES * A_STAGE_BYTES;      // [stage][256 rows][128 B]
     uint8_t *sRaw = sB + TC_STAGES * B_STAGE_BYTES;      // producers' private weight staging
-    TcSmem *ss = reinterpret_cast<TcSmem *>(sRaw + RAW_BYTES);
+    float *sStg = reinterpret_cast<float *>(sRaw + RAW_BYTES);   // down epilogue: row-to-column staging
+    TcSmem *ss = reinterpret_cast<TcSmem *>(sRaw + RAW_BYTES + STG_BYTES);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
@@ -665,7 +675,10 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                                 for (int i = 0; i < 8; i += 2) {
                                     float g0 = v[16 * t2 + i], g1 = v[16 * t2 + i + 1];
                                     float u0 = v[16 * t2 + 8 + i], u1 = v[16 * t2 + 8 + i + 1];
-                                    float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+                                    // h is rounded to fp16 next: the fast exponential and division
+                                    // (a few fp32 ulp) are far inside that rounding
+                                    float h0 = __fdividef(g0, 1.f + __expf(-g0)) * u0;
+                                    float h1 = __fdividef(g1, 1.f + __expf(-g1)) * u1;
                                     __half2 hh = __floats2half2_rn(h0, h1);
                                     hw[4 * t2 + i / 2] = *reinterpret_cast<uint32_t *>(&hh);
                                 }
@@ -679,19 +692,47 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
                 } else {
                     int slot = p.perm[pos];
                     int tok = slot_token(slot, p.T, p.k);
-                    float wt = slot < p.T * p.k ? p.w_route[slot] : 1.f;
-                    float *yrow = p.y_acc + (size_t)tok * p.d + (size_t)nt * TC_BN;
+                    // The weighted rows are added into y with coalesced reductions: each lane holds one
+                    // row of 32 columns; 16 of them at a time pass through the warp's staging (row-major,
+                    // 16-byte slot c of row r at c ^ (r/2 % 4): conflict-free both ways), and are read
+                    // back so that four lanes cover 64 contiguous bytes of one row.  Row-per-lane
+                    // reductions (32 rows, 16 bytes each, per instruction) measured twice as slow: the
+                    // L2's reduction throughput bounds this epilogue.
+                    const float wt = slot < p.T * p.k ? p.w_route[slot] : 1.f;
+                    float *stg = sStg + q4 * STG_WARP_FLOATS;
+                    const int rr = lane >> 2, c4 = lane & 3;
+                    float *ydst[4];   // row 8 j + rr of this warp's 32 (null: past the item's rows)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = 8 * j + rr;
+                        const int tr = __shfl_sync(0xffffffffu, tok, r);
+                        const int lv = __shfl_sync(0xffffffffu, (int)live, r);
+                        ydst[j] = lv ? p.y_acc + (size_t)tr * p.d + (size_t)nt * TC_BN + 4 * c4 : nullptr;
+                    }
                     for (int cb = 0; cb < TC_BN / 32; ++cb) {
                         float v[32];
                         tmem_ld32(tbase + 32 * cb, v);
-                        if (live) {
 #pragma unroll
-                            for (int i = 0; i < 32; i += 4) {
-                                float *dst = yrow + 32 * cb + i;
-                                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst),
-                                             "f"(wt * v[i]), "f"(wt * v[i + 1]), "f"(wt * v[i + 2]), "f"(wt * v[i + 3])
-                                             : "memory");
+                        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int pc = c ^ ((lane >> 1) & 3);
+                                *reinterpret_cast<float4 *>(stg + lane * 16 + 4 * pc) =
+                                    make_float4(wt * v[16 * hh + 4 * c], wt * v[16 * hh + 4 * c + 1],
+                                                wt * v[16 * hh + 4 * c + 2], wt * v[16 * hh + 4 * c + 3]);
                             }
+                            __syncwarp();
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int r = 8 * j + rr;
+                                const float4 val =
+                                    *reinterpret_cast<const float4 *>(stg + r * 16 + 4 * (c4 ^ ((r >> 1) & 3)));
+                                if (ydst[j])
+                                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                                                 ::"l"(ydst[j] + 32 * cb + 16 * hh), "f"(val.x), "f"(val.y),
+                                                 "f"(val.z), "f"(val.w) : "memory");
+                            }
+                            __syncwarp();
                         }
                     }
                 }
@@ -707,13 +748,13 @@ __global__ void __launch_bounds__(TC_NT, 1) k_tc_gemm(TcParams p) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Cache slots for the experts with more than one 256-row block (slot order is
+// Cache slots for the experts with at least TC_CACHE_MIN_ROWS rows (slot order is
 // arbitrary; slots past the capacity fall back to decoding in the GEMM).
 __global__ void k_cache_assign(const int32_t *__restrict__ counts, int nx, int cap, int32_t *__restrict__ slot,
                                int32_t *__restrict__ expert, int32_t *__restrict__ n_used) {
     for (int e = threadIdx.x; e < nx; e += blockDim.x) {
         int sl = -1;
-        if (counts[e] > TC_BM) {
+        if (counts[e] >= TC_CACHE_MIN_ROWS) {
             sl = atomicAdd(n_used, 1);
             if (sl >= cap) sl = -1;
             else expert[sl] = e;
@@ -820,7 +861,7 @@ __global__ void k_finish(const float *__restrict__ yacc, size_t n, uint16_t *__r
 
 template <int FMT, int MODE>
 int launch_tc(const TcParams &p, int grid, cudaStream_t st) {
-    size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + RAW_BYTES + sizeof(TcSmem) + 1024;
+    size_t smem = (size_t)TC_STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + RAW_BYTES + STG_BYTES + sizeof(TcSmem) + 1024;
     QE_CHECK(cudaFuncSetAttribute(k_tc_gemm<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     k_tc_gemm<FMT, MODE><<<grid, TC_NT, smem, st>>>(p);
     QE_CHECK_LAUNCH(MODE == TC_GATEUP ? "k_tc_gemm<gate/up>" : MODE == TC_DOWN ? "k_tc_gemm<down>" : "k_tc_gemm<router>");
@@ -915,7 +956,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     p.d = c.d_model;
     p.err = ws.dev_error;
 
-    // decoded-weight cache for the experts with more than one 256-row block (part of the timed
+    // decoded-weight cache for the experts with more than three 256-row blocks (part of the timed
     // expert work: it takes over decoding from the GEMMs)
     QE_TRY(timing_begin(ctx, st, "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>"));
     if (ws.cache_cap > 0) {
