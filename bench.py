@@ -95,7 +95,7 @@ MEASURED_TRAFFIC = [
      "sha256": "dc47924e40b899b93f15d88b224461a32a4ec7bccfaf09d8569cdf2b79c2f610", "bytes_per_layer": 42_253_376,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "f2866d32da870bda33e4d80a57dcea971865c816735740e7a88101eea77d9bac", "bytes_per_layer": 896_799_488,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "58a9eed32a442f530873b43894b5bec6e4159c7502de16b3ea9774b23147a1e1", "bytes_per_layer": 968_600_576,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 
