@@ -89,13 +89,13 @@ def router_flops(cfg, T: int) -> int:
 # produced them are in the profiles/ summaries named beside each entry.
 MEASURED_TRAFFIC = [
     {"kernel": "k_decode", "workload": "decode_48l_q4_t1", "src": ['decode.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "3244bb73841d42dc054ba8d39528026745358a73eb5c732be3bd87928ae198d7", "bytes_per_layer": 30_823_552,
+     "sha256": "67b48eaa0b8a6bb4daaebc89b3fa2a4122f45fc73dd08d4f05fe71c6fb5a9bf7", "bytes_per_layer": 30_823_552,
      "profile": "profiles/k_decode_decode_48l_q4_t1.md"},
     {"kernel": "k_decode_multi", "workload": "verify_48l_q3_t4_zipf", "src": ['decode_multi.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "dc47924e40b899b93f15d88b224461a32a4ec7bccfaf09d8569cdf2b79c2f610", "bytes_per_layer": 42_253_376,
+     "sha256": "a07bf697d9c666014b7468df922dcfec793e4ce6ad60ac23df9f3f9d1658e16d", "bytes_per_layer": 42_253_376,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "58a9eed32a442f530873b43894b5bec6e4159c7502de16b3ea9774b23147a1e1", "bytes_per_layer": 968_600_576,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "2b6f5b2badb1f741e17e266b850e412bb3508336881af981c9de502798fb231c", "bytes_per_layer": 968_600_576,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 
@@ -450,10 +450,10 @@ def measure(args, cfg, rank, world, local_rank, dist_on, with_cpu: bool) -> dict
 # The library's path selection by T (include/moe.h, moe_forward): the single-token kernel for one
 # token, the few-token kernel for 2 to DISPATCH_FEW_MAX tokens, the tensor-core path above; the
 # CUDA-core path only where none fits.  The flags below pin a context to one path.
-DISPATCH_FEW_MAX = 16
+DISPATCH_FEW_MAX = 32
 DISPATCH_SINGLE_MAX = 8      # the single-token kernel, once per token, when pinned to it
 DISPATCH_TC_MIN = 9          # the tensor-core path's floor when the decode kernels are off
-SWEEP_T = (1, 2, 4, 6, 8, 9, 10, 12, 16, 17, 24, 32, 48, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
+SWEEP_T = (1, 2, 4, 6, 8, 9, 10, 12, 16, 17, 24, 32, 33, 40, 48, 64, 96, 128, 256, 512, 1024, 2048, 4096, 8192)
 SWEEP_PATHS = ("single-token kernel", "few-token kernel", "cuda-core", "tensor-core")
 
 

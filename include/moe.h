@@ -103,7 +103,7 @@ typedef struct {
  * run normally.  Both hooks are for tests only. */
 #define MOE_FLAG_NO_DECODE_KERNEL 1   /* small T runs the general path, not the single-token kernel */
 #define MOE_FLAG_NO_TENSOR_PREFILL 2  /* large T runs the CUDA-core expert path */
-#define MOE_FLAG_NO_MULTI_DECODE 8    /* 2..16 tokens run the single-token kernel per token, not the few-token kernel */
+#define MOE_FLAG_NO_MULTI_DECODE 8    /* 2..32 tokens run the single-token kernel per token (up to 8) or the tensor-core path, not the few-token kernel */
 #define MOE_FLAG_SPLIT_DECODE 16      /* with max_tokens == 1: the split single-token kernel (down projection by k chunk) */
 #define MOE_FLAG_TEST_WITHHOLD 256    /* test hook described above */
 #define MOE_FLAG_TRACE 4              /* record per-phase timestamps (moe_trace_read) */
@@ -173,10 +173,10 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  * Asynchronous on `stream`; no host synchronisation and no allocation.
  * T == 0 is a no-op.  Errors: INVALID_ARG, NOT_LOADED, TOO_MANY_TOKENS, CUDA.
  * Implementation (not part of the contract): one token runs the persistent
- * single-token kernel, 2 to 16 tokens the persistent few-token kernel (one
+ * single-token kernel, 2 to 32 tokens the persistent few-token kernel (one
  * launch per 8 tokens, reading the union of their experts once per layer;
  * shapes with n_experts <= 512, d_ff a multiple of 128 and d_model <= 3072),
- * 17 and more the tensor-core grouped GEMMs; the CUDA-core grouped path runs
+ * 33 and more the tensor-core grouped GEMMs; the CUDA-core grouped path runs
  * where none fits the shape (or under the MOE_FLAG_NO_* flags); each path
  * meets the same accuracy bound. */
 MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,

@@ -26,7 +26,9 @@ def test_flags_match_the_binding():
     (8, {"single-token kernel", "few-token kernel", "cuda-core"}, "few-token kernel"),
     (9, {"few-token kernel", "cuda-core", "tensor-core"}, "few-token kernel"),
     (16, {"few-token kernel", "cuda-core", "tensor-core"}, "few-token kernel"),
-    (17, {"cuda-core", "tensor-core"}, "tensor-core"),
+    (17, {"few-token kernel", "cuda-core", "tensor-core"}, "few-token kernel"),
+    (32, {"few-token kernel", "cuda-core", "tensor-core"}, "few-token kernel"),
+    (33, {"cuda-core", "tensor-core"}, "tensor-core"),
     (8192, {"cuda-core", "tensor-core"}, "tensor-core"),
 ])
 def test_eligible_paths_and_default(T, paths, default):
@@ -40,11 +42,11 @@ def test_summary_names_the_fastest_path_and_checks_the_default():
             {"T": 8, "path": "cuda-core", "ms": 0.15},
             {"T": 128, "path": "cuda-core", "ms": 1.0},
             {"T": 128, "path": "tensor-core", "ms": 0.4},
-            {"T": 32, "path": "tensor-core", "ms": 0.3}]
+            {"T": 64, "path": "tensor-core", "ms": 0.3}]
     s = {r["T"]: r for r in bench.sweep_summary(rows)}
-    assert [r["T"] for r in bench.sweep_summary(rows)] == [8, 32, 128]
+    assert [r["T"] for r in bench.sweep_summary(rows)] == [8, 64, 128]
     assert s[8]["fastest"] == "cuda-core" and not s[8]["default_is_fastest"] and s[8]["default_ms"] == 0.20
-    assert s[32]["fastest"] == "tensor-core" and s[32]["default_is_fastest"]
+    assert s[64]["fastest"] == "tensor-core" and s[64]["default_is_fastest"]
     assert s[128]["fastest"] == "tensor-core" and s[128]["default_is_fastest"] and s[128]["fastest_ms"] == 0.4
 
 
