@@ -29,6 +29,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -82,29 +83,38 @@ def router_flops(cfg, T: int) -> int:
 
 
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels, per layer,
-# each with the SHA-256 of the kernel sources it was measured on: a figure is reported only while
-# those sources are unchanged (a changed kernel reports null until it is measured again).  The decode
+# each with the SHA-256 of the kernel sources it was measured on (their code: comments and blank lines
+# are left out of the hash, so that a documentation edit does not void a measurement): a figure is
+# reported only while that code is unchanged (a changed kernel reports null until it is measured
+# again).  The decode
 # figures come from 4-layer captures (the 48-layer launch is reported as 48 x the per-layer mean:
 # the traffic grows with the layers, each streaming its own union of experts); the commands that
 # produced them are in the profiles/ summaries named beside each entry.
 MEASURED_TRAFFIC = [
     {"kernel": "k_decode", "workload": "decode_48l_q4_t1", "src": ['decode.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "67b48eaa0b8a6bb4daaebc89b3fa2a4122f45fc73dd08d4f05fe71c6fb5a9bf7", "bytes_per_layer": 30_823_552,
+     "sha256": "a2d18ae6d699d604e7ad84838a17d28788706e6860a2c0391a24a9ac304f0a62", "bytes_per_layer": 30_823_552,
      "profile": "profiles/k_decode_decode_48l_q4_t1.md"},
     {"kernel": "k_decode_multi", "workload": "verify_48l_q3_t4_zipf", "src": ['decode_multi.cu', 'decode_common.cuh', 'moe_internal.cuh'],
-     "sha256": "a07bf697d9c666014b7468df922dcfec793e4ce6ad60ac23df9f3f9d1658e16d", "bytes_per_layer": 42_253_376,
+     "sha256": "d4ad631ed59af87bb945793e0acc84987a5dd194c9dff1a3f562204901de8e06", "bytes_per_layer": 42_253_376,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "2b6f5b2badb1f741e17e266b850e412bb3508336881af981c9de502798fb231c", "bytes_per_layer": 968_600_576,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "1834a3d9cc871a7dd9b80db7ff9fe4c5ef1abfcd2bc1e6f96e972bc1e4eb191a", "bytes_per_layer": 968_600_576,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
+
+
+def _code_only(text: str) -> str:
+    """C/CUDA source without its comments, trailing blanks and empty lines."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.split("\n"))
+    return "\n".join(ln for ln in lines if ln)
 
 
 def _src_sha(rels) -> str:
     h = hashlib.sha256()
     for rel in ([rels] if isinstance(rels, str) else rels):
-        with open(os.path.join(ROOT, "quantized_expert_ffn_token_b200", "csrc", rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_expert_ffn_token_b200", "csrc", rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -14,10 +14,13 @@
 //                 describe;
 //   warps 9..11 : A-row loaders: A rows (tokens or h rows) are gathered with
 //                 16-byte cp.async into the same layout;
-//   warps 12..15: epilogue, tcgen05.ld from TMEM (lane quarter = warp % 4).
+//   warps 12..15: epilogue, tcgen05.ld from TMEM (lane quarter = warp % 4):
+//                 SwiGLU into fp16 h (gate/up), or w_slot * out reduced into
+//                 y through a small shared-memory transpose (down).
 // A work item is (expert, 256 slots, 256 output columns): two M=128
 // accumulators share every decoded weight stage (TMEM: 2 x 256 fp32 columns),
-// so the weight decode is paid once per 256 slots.
+// so the weight decode is paid once per 256 slots; experts of more than three
+// 256-slot blocks are decoded once per call into fp16 stage images instead.
 //
 // Expert network = SwiGLU; routing weights and block formats as in moe.h.
 // The weights are rounded to fp16 here (the tensor cores take one operand
