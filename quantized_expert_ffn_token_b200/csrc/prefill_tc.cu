@@ -256,16 +256,29 @@ constexpr uint32_t H_4TH = 0x34003400u;
 constexpr uint32_t H_M1026 = 0xE402E402u, H_M258 = 0xDC08DC08u, H_M66 = 0xD420D420u,   // Q2: -(1024+2),
                    H_M18 = 0xCC80CC80u;                                                 // -(256+2), -(64+2), -(16+2)
 
-// The 16 (q - zero) fp16 pairs of one lane's piece of a k group, register
-// q = 4*slice + reg (reg a0..a3 as in the row-tile layout).
+// Words of one lane's piece of a k group (Q4: 4, Q3: 3, Q2: 2 of the 4 loaded).
 template <int FMT>
-__device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16]) {
+__device__ __forceinline__ void load_piece(const uint8_t *src, uint32_t w[4]) {
+    if constexpr (FMT == MOE_Q2B32) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(src);
+        w[0] = a.x, w[1] = a.y, w[2] = w[3] = 0u;
+    } else if constexpr (FMT == MOE_Q4B32) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(src);
+        w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w;
+    } else {
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(src);
+        w[0] = wp[0], w[1] = wp[1], w[2] = wp[2], w[3] = 0u;
+    }
+}
+
+// The 16 (q - zero) fp16 pairs of one lane's piece of a k group, register
+// q = 4*slice + reg (reg a0..a3 as in the row-tile layout), from its words.
+template <int FMT>
+__device__ __forceinline__ void decode_words(const uint32_t wv[4], uint32_t r[16]) {
     if constexpr (FMT == MOE_Q2B32) {
         // word w: the 2-bit fields at bits 0, 2, 4, 6 of each half (of w, then of w >> 8) read
         // 1024 + {1, 4, 16, 64} q; fields 0,1,4,5 are registers a0..a3 of slice w, fields
         // 2,3,6,7 those of slice w + 2
-        uint2 a = *reinterpret_cast<const uint2 *>(src);
-        uint32_t wv[2] = {a.x, a.y};
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
             uint32_t x = wv[w], x8 = wv[w] >> 8;
@@ -279,8 +292,6 @@ __device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16])
             r[4 * w + 11] = hfma2((x8 & 0x00C000C0u) | H_MAGIC, H_64TH, H_M18);
         }
     } else if constexpr (FMT == MOE_Q4B32) {
-        uint4 a = *reinterpret_cast<const uint4 *>(src);
-        uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             uint32_t w = wv[m], w8 = w >> 8;
@@ -290,20 +301,25 @@ __device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16])
             r[4 * m + 3] = hfma2((w8 & 0x00F000F0u) | H_MAGIC, H_16TH, H_M72);
         }
     } else {
-        const uint32_t *wp = reinterpret_cast<const uint32_t *>(src);
-        uint32_t ws[3] = {wp[0], wp[1], wp[2]};
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-            uint32_t w = ws[j], w9 = ws[j] >> 9;
+            uint32_t w = wv[j], w9 = wv[j] >> 9;
             r[5 * j + 0] = hfma2((w & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
             r[5 * j + 1] = hfma2((w & 0x00380038u) | H_MAGIC, H_8TH, H_M132);
             r[5 * j + 2] = hfma2((w & 0x01C001C0u) | H_MAGIC, H_64TH, H_M20);
             r[5 * j + 3] = hfma2((w9 & 0x00070007u) | H_MAGIC, H_ONE, H_M1028);
             r[5 * j + 4] = hfma2((w9 & 0x00380038u) | H_MAGIC, H_8TH, H_M132);
         }
-        uint32_t s = ((ws[0] >> 15) & 0x00010001u) | ((ws[1] >> 14) & 0x00020002u) | ((ws[2] >> 13) & 0x00040004u);
+        uint32_t s = ((wv[0] >> 15) & 0x00010001u) | ((wv[1] >> 14) & 0x00020002u) | ((wv[2] >> 13) & 0x00040004u);
         r[15] = hfma2(s | H_MAGIC, H_ONE, H_M1028);
     }
+}
+
+template <int FMT>
+__device__ __forceinline__ void decode_piece(const uint8_t *src, uint32_t r[16]) {
+    uint32_t w[4];
+    load_piece<FMT>(src, w);
+    decode_words<FMT>(w, r);
 }
 
 // Four 8x8 fp16 matrices from mma-fragment registers to shared memory: lane i
@@ -825,20 +841,236 @@ __global__ void __launch_bounds__(256) k_cache_fill(const uint8_t *__restrict__ 
     }
 }
 
-// Work items of one GEMM: for every expert with slots, ceil(cnt/256) row
-// blocks x n_tiles column tiles.  Single block.  The items of two M = 128
+// ---- Small experts: a weight-streaming path ---------------------------------------------------
+// An expert with at most SMALL_MAX rows in a call costs the tensor-core GEMMs as many k-group steps
+// as one with 256 (at 4,096 Zipf-routed tokens, 124 of the 207 active experts have at most 16 rows).
+// Each such expert is instead one CTA's work: its rows of the fp16 layer input are staged in shared
+// memory once, every warp streams gate/up row tiles through its own ring of cp.async slots (SE_S k
+// groups in flight) and multiplies them with mma.sync m16n8k16 (the decoded tile, the same fp16
+// w = s (q - zero) as the GEMM's B stage, as A; the rows as one or two 8-column B groups; fp32
+// accumulation); SwiGLU h stays in shared memory for the down tiles, whose outputs are added into y.
+// Operand rows are stored permuted: within each 64-wide k group, fp16 pair 8m + 4h + c goes to
+// 8c + 2m + h, so the eight B registers a lane needs for the group's four k16 slices are 32
+// contiguous bytes; rows are padded by 16 bytes so the eight rows a load touches fall in distinct
+// banks.
+constexpr int SMALL_MAX = 16;
+constexpr int SE_W = 16;                 // warps per CTA
+constexpr int SE_S = 8;                  // k groups in flight per warp
+constexpr int SE_SLOT = 32 * 16 + 64;    // one k group of one row tile: 16 code bytes per lane, 4 scale bytes per row
+
+__device__ __forceinline__ int perm_word(int w) { return 8 * (w & 3) + 2 * (w >> 3) + ((w >> 2) & 1); }
+
+struct SmallParams {
+    const int4 *list;            // (expert, first grouped position, rows, -)
+    const int32_t *n_list;
+    const int32_t *perm;         // grouped position -> slot
+    const uint16_t *x16;         // [T][d] fp16 layer input (the GEMM's A operand)
+    const uint8_t *gu, *dn;
+    MatLayout Lg, Ld;
+    float *y_acc;                // [T][d]
+    const float *w_route;        // [T][k]
+    int T, k, d, I;
+};
+
+__host__ __device__ constexpr size_t small_smem_bytes(int d, int I) {
+    return (size_t)SMALL_MAX * (d + 8) * 2 + (size_t)SMALL_MAX * (I + 8) * 2 + (size_t)SE_W * SE_S * SE_SLOT +
+           (size_t)SMALL_MAX * 8;
+}
+
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One warp's share of one GEMM of a small expert: row tiles warp, warp + SE_W, ... over K, B rows
+// from `bs` (stride bstride halves).  Gate/up: SwiGLU of each tile's gate rows 0..7 and up rows
+// 8..15 into hs; down: w_slot x out added into y.
+template <int FMT, bool GU>
+__device__ __forceinline__ void small_gemm(const SmallParams &p, const int4 ent, const uint16_t *bs, int bstride,
+                                           uint16_t *hs, const int2 *tokw, uint8_t *wring, int warp, int lane) {
+    const MatLayout &L = GU ? p.Lg : p.Ld;
+    const int K = L.K, nkg = K / 64, nb = K / 32;
+    const int ntile = (GU ? 2 * p.I : p.d) / 16;
+    const int nmine = warp < ntile ? (ntile - 1 - warp) / SE_W + 1 : 0;
+    const int nq = nmine * nkg;   // this warp's steps: k group q % nkg of its tile q / nkg
+    const uint8_t *wexp = (GU ? p.gu : p.dn) + (size_t)ent.x * L.expert_bytes;
+    const int g = lane >> 2, c = lane & 3;
+    const bool two = ent.z > 8;
+    // step q's codes and scales into slot q % SE_S (one cp.async group per step, empty past the end);
+    // each lane copies and later reads only its own bytes of a slot
+    // request position (tile rt, k group rkg) and consume position (tile t, k group kg) advance by one
+    // k group per step; a slot holds the lane's code bytes and, from lanes 0..15, row lane's scales
+    const uint8_t *rtile = wexp + (size_t)warp * L.tile_bytes;
+    int rkg = 0, rq = 0;
+    const size_t tstep = (size_t)SE_W * L.tile_bytes;
+    const int code_off = lane * (FMT == MOE_Q4B32 ? 16 : FMT == MOE_Q2B32 ? 8 : 12);
+    const int sc_off = (lane & 15) * nb * 2;
+    auto request = [&]() {
+        if (rq < nq) {
+            uint8_t *slot = wring + (rq % SE_S) * SE_SLOT;
+            const uint8_t *cs = rtile + (size_t)rkg * L.kg_bytes + code_off;
+            if constexpr (FMT == MOE_Q4B32) {
+                cp_async16(slot + lane * 16, cs);
+            } else if constexpr (FMT == MOE_Q2B32) {
+                cp_async8(slot + lane * 16, cs);
+            } else {
+                cp_async4(slot + lane * 16, cs);
+                cp_async4(slot + lane * 16 + 4, cs + 4);
+                cp_async4(slot + lane * 16 + 8, cs + 8);
+            }
+            if (lane < 16) cp_async4(slot + 512 + lane * 4, rtile + L.code_bytes + sc_off + rkg * 4);
+            if (++rkg == nkg) {
+                rkg = 0;
+                rtile += tstep;
+            }
+            ++rq;
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int q = 0; q < SE_S - 1; ++q) request();
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    int t = warp, kg = 0;
+    const uint16_t *brow0 = bs + (size_t)g * bstride + 16 * c, *brow1 = brow0 + (size_t)8 * bstride;
+    for (int q = 0; q < nq; ++q) {
+        request();
+        cp_async_wait<SE_S - 1>();   // step q's bytes (this lane's) have landed
+        __syncwarp();                // ... and the scales, which lanes 0..15 copied
+        const uint8_t *slot = wring + (q % SE_S) * SE_SLOT;
+        uint32_t wv[4];
+        load_piece<FMT>(slot + lane * 16, wv);
+        const uint32_t sgp = *reinterpret_cast<const uint32_t *>(slot + 512 + g * 4);
+        const uint32_t s8p = *reinterpret_cast<const uint32_t *>(slot + 512 + (g + 8) * 4);
+        uint32_t qv[16];
+        decode_words<FMT>(wv, qv);
+        const uint32_t us0 = (sgp & 0xFFFFu) * 0x10001u, us1 = (sgp >> 16) * 0x10001u;
+        const uint32_t u80 = (s8p & 0xFFFFu) * 0x10001u, u81 = (s8p >> 16) * 0x10001u;
+        // B: rows g and 8 + g, this lane's 32 bytes of the k group
+        uint32_t b[2][8];
+        {
+            const uint4 *bp = reinterpret_cast<const uint4 *>(brow0 + 64 * kg);
+            const uint4 v0 = bp[0], v1 = bp[1];
+            b[0][0] = v0.x, b[0][1] = v0.y, b[0][2] = v0.z, b[0][3] = v0.w;
+            b[0][4] = v1.x, b[0][5] = v1.y, b[0][6] = v1.z, b[0][7] = v1.w;
+        }
+        if (two) {
+            const uint4 *bp = reinterpret_cast<const uint4 *>(brow1 + 64 * kg);
+            const uint4 v0 = bp[0], v1 = bp[1];
+            b[1][0] = v0.x, b[1][1] = v0.y, b[1][2] = v0.z, b[1][3] = v0.w;
+            b[1][4] = v1.x, b[1][5] = v1.y, b[1][6] = v1.z, b[1][7] = v1.w;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t sg = m < 2 ? us0 : us1, s8 = m < 2 ? u80 : u81;
+            const uint32_t a0 = hmul2(qv[4 * m + 0], sg), a1 = hmul2(qv[4 * m + 1], s8);
+            const uint32_t a2 = hmul2(qv[4 * m + 2], sg), a3 = hmul2(qv[4 * m + 3], s8);
+            mma16816_f16(acc[0], a0, a1, a2, a3, b[0][2 * m], b[0][2 * m + 1]);
+            if (two) mma16816_f16(acc[1], a0, a1, a2, a3, b[1][2 * m], b[1][2 * m + 1]);
+        }
+        if (kg == nkg - 1) {
+            // lane (g, c) holds rows g and g + 8 of the tile for columns 2c and 2c + 1 of each group
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = 8 * j + 2 * c + e;
+                    if (r < ent.z) {
+                        if constexpr (GU) {
+                            const int hk = 8 * t + g;   // h index of gate row g and up row g + 8
+                            const int hpos = 64 * (hk >> 6) + 2 * perm_word((hk & 63) >> 1) + (hk & 1);
+                            const float gt = acc[j][e], up = acc[j][2 + e];
+                            const __half h = __float2half_rn(__fdividef(gt, 1.f + __expf(-gt)) * up);
+                            hs[(size_t)r * (p.I + 8) + hpos] = *reinterpret_cast<const uint16_t *>(&h);
+                        } else {
+                            const int2 tw = tokw[r];
+                            float *y = p.y_acc + (size_t)tw.x * p.d + 16 * t + g;
+                            const float wt = __int_as_float(tw.y);
+                            atomicAdd(y, wt * acc[j][e]);
+                            atomicAdd(y + 8, wt * acc[j][2 + e]);
+                        }
+                    }
+                    acc[j][e] = acc[j][2 + e] = 0.f;
+                }
+            kg = 0;
+            t += SE_W;
+        } else {
+            ++kg;
+        }
+        __syncwarp();   // every lane has read the slot's scales before a lane re-requests into it
+    }
+    cp_async_wait<0>();
+}
+
+// Every small expert of the call: a CTA per expert (grid-stride), gate/up then down.
+template <int FMT>
+__global__ void __launch_bounds__(SE_W * 32, 1) k_small_expert(SmallParams p) {
+    extern __shared__ __align__(16) uint8_t sm_small[];
+    uint16_t *xs = reinterpret_cast<uint16_t *>(sm_small);                  // [SMALL_MAX][d + 8]
+    uint16_t *hs = xs + (size_t)SMALL_MAX * (p.d + 8);                       // [SMALL_MAX][I + 8]
+    uint8_t *ring = reinterpret_cast<uint8_t *>(hs + (size_t)SMALL_MAX * (p.I + 8));
+    int2 *tokw = reinterpret_cast<int2 *>(ring + (size_t)SE_W * SE_S * SE_SLOT);   // [SMALL_MAX] (token, weight)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t *wring = ring + (size_t)warp * SE_S * SE_SLOT;
+    const int n = *p.n_list;
+    const int ngd = p.d / 64;
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const int4 ent = p.list[i];
+        if (tid < ent.z) {
+            const int slot = p.perm[ent.y + tid];
+            tokw[tid] = make_int2(slot_token(slot, p.T, p.k),
+                                  __float_as_int(slot < p.T * p.k ? p.w_route[slot] : 1.f));
+        }
+        __syncthreads();
+        // the expert's rows of the layer input, permuted (rows past ent.z are never used)
+        for (int u = tid; u < ent.z * ngd; u += blockDim.x) {
+            const int r = u / ngd, kg = u - r * ngd;
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x16 + (size_t)tokw[r].x * p.d + 64 * kg);
+            uint32_t o[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 v = src[j];
+                o[perm_word(4 * j + 0)] = v.x;
+                o[perm_word(4 * j + 1)] = v.y;
+                o[perm_word(4 * j + 2)] = v.z;
+                o[perm_word(4 * j + 3)] = v.w;
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)r * (p.d + 8) + 64 * kg);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        }
+        __syncthreads();
+        small_gemm<FMT, true>(p, ent, xs, p.d + 8, hs, tokw, wring, warp, lane);
+        __syncthreads();   // every h value is in hs
+        small_gemm<FMT, false>(p, ent, hs, p.I + 8, hs, tokw, wring, warp, lane);
+        __syncthreads();   // xs, hs and tokw are free for the next expert
+    }
+}
+
+// Work items of one GEMM: for every expert with more than small_max slots,
+// ceil(cnt/256) row blocks x n_tiles column tiles; with `small` set, the list
+// of the others that have slots (expert, first position, rows, 0).  Single
+// block.  The items of two M = 128
 // accumulators (blocks of more than 128 rows) come first, then the single-
 // accumulator ones: the CTAs take items round-robin, so the costly ones are
 // spread first and the cheap ones even out the tail (an expert-ordered list
 // left the busiest CTA ~16 % above the mean on a Zipf-routed layer's gate/up
 // GEMM, by a count of k groups; this order ~6 %).
 __global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int nx,
-                           int n_tiles, int4 *__restrict__ items, int32_t *__restrict__ n_items, int max_items) {
-    __shared__ int n_big, n_small;
-    if (threadIdx.x == 0) n_big = n_small = 0;
+                           int n_tiles, int4 *__restrict__ items, int32_t *__restrict__ n_items, int max_items,
+                           int small_max, int4 *__restrict__ small, int32_t *__restrict__ n_small_out) {
+    __shared__ int n_big, n_small, n_sm;
+    if (threadIdx.x == 0) n_big = n_small = n_sm = 0;
     __syncthreads();
     for (int e = threadIdx.x; e < nx; e += blockDim.x) {
         const int cnt = counts[e];
+        if (cnt <= small_max) {
+            if (cnt > 0 && small) small[atomicAdd(&n_sm, 1)] = make_int4(e, offsets[e], cnt, 0);
+            continue;
+        }
         const int nb = cnt / TC_BM + (cnt % TC_BM > 128 ? 1 : 0);   // blocks of more than 128 rows
         if (nb == 0) continue;
         const int base = atomicAdd(&n_big, nb * n_tiles);
@@ -854,7 +1086,7 @@ __global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__
     for (int e = threadIdx.x; e < nx; e += blockDim.x) {
         const int cnt = counts[e];
         const int rem = cnt % TC_BM;   // the last, short block, when it has at most 128 rows
-        if (rem == 0 || rem > 128) continue;
+        if (cnt <= small_max || rem == 0 || rem > 128) continue;
         const int base = big + atomicAdd(&n_small, n_tiles);
         for (int t = 0; t < n_tiles; ++t) {
             const int idx = base + t;
@@ -862,7 +1094,10 @@ __global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0) *n_items = min(n_big + n_small, max_items);
+    if (threadIdx.x == 0) {
+        *n_items = min(n_big + n_small, max_items);
+        if (small) *n_small_out = n_sm;
+    }
 }
 
 __global__ void k_bf16_to_f16(const uint16_t *__restrict__ x, __half *__restrict__ y, size_t n) {
@@ -978,7 +1213,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
 
     // decoded-weight cache for the experts with more than three 256-row blocks (part of the timed
     // expert work: it takes over decoding from the GEMMs)
-    QE_TRY(timing_begin(ctx, st, "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>"));
+    QE_TRY(timing_begin(ctx, st, "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>+k_small_expert"));
     if (ws.cache_cap > 0) {
         QE_CHECK(cudaMemsetAsync(ws.cache_n, 0, 4, st));
         k_cache_assign<<<1, 1024, 0, st>>>(ws.counts, ctx->nx, ws.cache_cap, ws.cache_slot, ws.cache_expert,
@@ -1007,9 +1242,12 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
         p.cache_stride = (size_t)3 * c.d_model * c.d_ff;
     }
 
-    // gate/up: A = x16 rows gathered by token, N = 2I, K = d
+    // gate/up: A = x16 rows gathered by token, N = 2I, K = d; the experts of at most SMALL_MAX rows
+    // go to the streaming path (its list in the CUDA-core path's chunk list, unused by this path)
+    const size_t small_smem = small_smem_bytes(c.d_model, c.d_ff);
+    const int small_max = small_smem <= (size_t)227 * 1024 ? SMALL_MAX : 0;   // the per-CTA opt-in limit
     k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, (2 * c.d_ff) / TC_BN, ws.tc_items,
-                                   ws.tc_n_items, max_items);
+                                   ws.tc_n_items, max_items, small_max, ws.chunks, ws.n_chunks);
     QE_CHECK_LAUNCH("k_tc_items");
     p.cache_off = 0;
     p.K = c.d_model;
@@ -1031,7 +1269,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     // down: A = h16 rows by grouped position, N = d, K = I
     QE_CHECK(cudaMemsetAsync(ws.y_acc, 0, Td * sizeof(float), st));
     k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, c.d_model / TC_BN, ws.tc_items,
-                                   ws.tc_n_items, max_items);
+                                   ws.tc_n_items, max_items, small_max, nullptr, nullptr);
     QE_CHECK_LAUNCH("k_tc_items");
     p.K = c.d_ff;
     p.N = c.d_model;
@@ -1045,6 +1283,34 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     if (c.fmt == MOE_Q4B32) QE_TRY((launch_tc<MOE_Q4B32, TC_DOWN>(p, grid, st)));
     else if (c.fmt == MOE_Q2B32) QE_TRY((launch_tc<MOE_Q2B32, TC_DOWN>(p, grid, st)));
     else QE_TRY((launch_tc<MOE_Q3B32, TC_DOWN>(p, grid, st)));
+    if (small_max > 0) {
+        SmallParams sp;
+        sp.list = ws.chunks;
+        sp.n_list = ws.n_chunks;
+        sp.perm = ws.perm;
+        sp.x16 = reinterpret_cast<const uint16_t *>(ws.x16);
+        sp.gu = Ly.gu;
+        sp.dn = Ly.dn;
+        sp.Lg = ctx->gu;
+        sp.Ld = ctx->dn;
+        sp.y_acc = ws.y_acc;
+        sp.w_route = w_route;
+        sp.T = T;
+        sp.k = c.top_k;
+        sp.d = c.d_model;
+        sp.I = c.d_ff;
+        if (c.fmt == MOE_Q4B32) {
+            QE_CHECK(cudaFuncSetAttribute(k_small_expert<MOE_Q4B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem));
+            k_small_expert<MOE_Q4B32><<<dev_sms, SE_W * 32, small_smem, st>>>(sp);
+        } else if (c.fmt == MOE_Q2B32) {
+            QE_CHECK(cudaFuncSetAttribute(k_small_expert<MOE_Q2B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem));
+            k_small_expert<MOE_Q2B32><<<dev_sms, SE_W * 32, small_smem, st>>>(sp);
+        } else {
+            QE_CHECK(cudaFuncSetAttribute(k_small_expert<MOE_Q3B32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem));
+            k_small_expert<MOE_Q3B32><<<dev_sms, SE_W * 32, small_smem, st>>>(sp);
+        }
+        QE_CHECK_LAUNCH("k_small_expert");
+    }
     QE_TRY(timing_end(ctx, st));
     k_finish<<<592, 256, 0, st>>>(ws.y_acc, Td, y, yf);
     QE_CHECK_LAUNCH("k_finish");
