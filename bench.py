@@ -98,7 +98,7 @@ MEASURED_TRAFFIC = [
      "sha256": "d4ad631ed59af87bb945793e0acc84987a5dd194c9dff1a3f562204901de8e06", "bytes_per_layer": 42_253_376,
      "profile": "profiles/k_decode_multi_verify_48l_q3_t4_zipf.md"},
     {"kernel": "k_cache_fill+k_tc_gemm<gate/up>+k_tc_gemm<down>+k_small_expert", "workload": "prefill_1l_q4_t4096_zipf",
-     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "ab7248d9958c2f96940ee9d09631d5d3a0be87d1a914f0e60f4fe04dcd731258", "bytes_per_layer": 897_861_120,
+     "src": ['prefill_tc.cu', 'moe_internal.cuh'], "sha256": "63b61a15554d6c56edb185a70e7e87ad6f2c547418375d632bde9c5b0c49a7ee", "bytes_per_layer": 897_861_120,
      "profile": "profiles/k_tc_gemm_prefill_1l_q4_t4096_zipf.md"},
 ]
 

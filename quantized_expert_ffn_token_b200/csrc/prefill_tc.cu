@@ -854,6 +854,12 @@ __global__ void __launch_bounds__(256) k_cache_fill(const uint8_t *__restrict__ 
 // contiguous bytes; rows are padded by 16 bytes so the eight rows a load touches fall in distinct
 // banks.
 constexpr int SMALL_MAX = 16;
+// Calls of fewer tokens keep their small experts in the GEMMs: there the GEMMs are short and nearly
+// every expert is small, and the streaming kernel added its own time to theirs (sweep, one layer of
+// the 4,096-token shape: 420-430 us against 365 at 17-128 tokens, even at 256-512) while from 1,024
+// tokens on it took 2-8 % off (597 / 733 / 997 / 1,509 us against 609 / 779 / 1,055 / 1,588 at
+// 1,024 / 2,048 / 4,096 / 8,192).
+constexpr int SMALL_MIN_TOKENS = 1024;
 constexpr int SE_W = 16;                 // warps per CTA
 constexpr int SE_S = 8;                  // k groups in flight per warp
 constexpr int SE_SLOT = 32 * 16 + 64;    // one k group of one row tile: 16 code bytes per lane, 4 scale bytes per row
@@ -1052,8 +1058,11 @@ __global__ void __launch_bounds__(SE_W * 32, 1) k_small_expert(SmallParams p) {
 
 // Work items of one GEMM: for every expert with more than small_max slots,
 // ceil(cnt/256) row blocks x n_tiles column tiles; with `small` set, the list
-// of the others that have slots (expert, first position, rows, 0).  Single
-// block.  The items of two M = 128
+// of the others that have slots (expert, first position, rows, 0).  The small
+// experts go to the streaming kernel only when they fit one wave of its CTAs
+// (at most small_ctas of them: at 64 tokens ~250 one-row experts took two waves
+// and 15 % longer than the GEMMs); the decision depends on the counts alone, so
+// both GEMMs' calls make it alike.  Single block.  The items of two M = 128
 // accumulators (blocks of more than 128 rows) come first, then the single-
 // accumulator ones: the CTAs take items round-robin, so the costly ones are
 // spread first and the cheap ones even out the tail (an expert-ordered list
@@ -1061,10 +1070,15 @@ __global__ void __launch_bounds__(SE_W * 32, 1) k_small_expert(SmallParams p) {
 // GEMM, by a count of k groups; this order ~6 %).
 __global__ void k_tc_items(const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int nx,
                            int n_tiles, int4 *__restrict__ items, int32_t *__restrict__ n_items, int max_items,
-                           int small_max, int4 *__restrict__ small, int32_t *__restrict__ n_small_out) {
-    __shared__ int n_big, n_small, n_sm;
-    if (threadIdx.x == 0) n_big = n_small = n_sm = 0;
+                           int small_max, int small_ctas, int4 *__restrict__ small,
+                           int32_t *__restrict__ n_small_out) {
+    __shared__ int n_big, n_small, n_sm, n_cand;
+    if (threadIdx.x == 0) n_big = n_small = n_sm = n_cand = 0;
     __syncthreads();
+    for (int e = threadIdx.x; e < nx; e += blockDim.x)
+        if (counts[e] > 0 && counts[e] <= small_max) atomicAdd(&n_cand, 1);
+    __syncthreads();
+    if (n_cand > small_ctas) small_max = 0;
     for (int e = threadIdx.x; e < nx; e += blockDim.x) {
         const int cnt = counts[e];
         if (cnt <= small_max) {
@@ -1245,9 +1259,10 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     // gate/up: A = x16 rows gathered by token, N = 2I, K = d; the experts of at most SMALL_MAX rows
     // go to the streaming path (its list in the CUDA-core path's chunk list, unused by this path)
     const size_t small_smem = small_smem_bytes(c.d_model, c.d_ff);
-    const int small_max = small_smem <= (size_t)227 * 1024 ? SMALL_MAX : 0;   // the per-CTA opt-in limit
+    const int small_max =
+        (T >= SMALL_MIN_TOKENS && small_smem <= (size_t)227 * 1024) ? SMALL_MAX : 0;   // per-CTA opt-in limit
     k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, (2 * c.d_ff) / TC_BN, ws.tc_items,
-                                   ws.tc_n_items, max_items, small_max, ws.chunks, ws.n_chunks);
+                                   ws.tc_n_items, max_items, small_max, dev_sms, ws.chunks, ws.n_chunks);
     QE_CHECK_LAUNCH("k_tc_items");
     p.cache_off = 0;
     p.K = c.d_model;
@@ -1269,7 +1284,7 @@ int launch_tc_experts(moe_ctx *ctx, const Layer &Ly, const uint16_t *x, int T, c
     // down: A = h16 rows by grouped position, N = d, K = I
     QE_CHECK(cudaMemsetAsync(ws.y_acc, 0, Td * sizeof(float), st));
     k_tc_items<<<1, 1024, 0, st>>>(ws.counts, ws.offsets, ctx->nx, c.d_model / TC_BN, ws.tc_items,
-                                   ws.tc_n_items, max_items, small_max, nullptr, nullptr);
+                                   ws.tc_n_items, max_items, small_max, dev_sms, nullptr, nullptr);
     QE_CHECK_LAUNCH("k_tc_items");
     p.K = c.d_ff;
     p.N = c.d_model;
