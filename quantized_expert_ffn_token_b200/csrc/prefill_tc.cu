@@ -856,7 +856,7 @@ __global__ void __launch_bounds__(256) k_cache_fill(const uint8_t *__restrict__ 
 constexpr int SMALL_MAX = 16;
 // Calls of fewer tokens keep their small experts in the GEMMs: there the GEMMs are short and nearly
 // every expert is small, and the streaming kernel added its own time to theirs (sweep, one layer of
-// the 4,096-token shape: 420-430 us against 365 at 17-128 tokens, even at 256-512) while from 1,024
+// the 4,096-token shape: 420-430 us against 365 at 17-128 tokens, no gain at 256-512) while from 1,024
 // tokens on it took 2-8 % off (597 / 733 / 997 / 1,509 us against 609 / 779 / 1,055 / 1,588 at
 // 1,024 / 2,048 / 4,096 / 8,192).
 constexpr int SMALL_MIN_TOKENS = 1024;
