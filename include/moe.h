@@ -176,7 +176,8 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int layer, const moe_layer_weights *w, 
  * single-token kernel, 2 to 32 tokens the persistent few-token kernel (one
  * launch per 8 tokens, reading the union of their experts once per layer;
  * shapes with n_experts <= 512, d_ff a multiple of 128 and d_model <= 3072),
- * 33 and more the tensor-core grouped GEMMs; the CUDA-core grouped path runs
+ * 33 and more the tensor-core grouped GEMMs (from 1,024 tokens, experts
+ * with at most 16 of them on a weight-streaming kernel); the CUDA-core grouped path runs
  * where none fits the shape (or under the MOE_FLAG_NO_* flags); each path
  * meets the same accuracy bound. */
 MOE_API int moe_forward(moe_ctx *ctx, int layer, const uint16_t *x_bf16, int T,
